@@ -1,0 +1,459 @@
+#!/usr/bin/env python
+"""Benchmark of the action-expert denoise loop (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+                    [--impl ours|reference] [--no-secondary] [--no-cpu-baseline]
+
+A "step" is one pae_denoise call: the whole hot path (input projection, 18
+expert layers, output projection and Euler update, for all Euler steps) over
+one batch of synthetic action chunks whose prefix K/V is already cached.
+Throughput follows the pages' definition: batch size over synchronised batch
+time (PhyAI report, Sec. 5.2 / Eq. 9), here chunks/s.  Timing: W untimed
+warm-up calls, then K calls between CUDA events on the launching stream,
+bracketed by a barrier and a device synchronise; the max over ranks is taken.
+Each rank runs an independent replica (pi0.5 requests are data-parallel with no
+exchange in the loop), so scaling is weak and there is no collective on the
+data path.  The weights (623 MB of projections) are larger than L2, so every
+Euler step streams them from HBM; no L2 flush is needed.
+
+--impl reference times the float64 CPU oracle instead (the only reference this
+build has), on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "denoise-loop action chunks/s at bs1 and bs32; achieved HBM GB/s / TC util vs peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.index = index
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+
+    def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return self
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                    r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    for bit, name in self.REASONS.items():
+                        if r & bit and name != "gpu_idle":
+                            self.reasons.add(name)
+                except Exception:
+                    pass
+                time.sleep(self.period)
+
+        self._t = threading.Thread(target=run, daemon=True)
+        self._t.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+        if not self.ok or not self.samples:
+            return None
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
+
+
+def algorithmic(cfg: wl.ExpertConfig, batch: int, lens=None):
+    """Algorithmic bytes and FLOPs per launch of each kernel class and per
+    Euler step (weights and prefix/action K/V once, activations once; table
+    build excluded)."""
+    D, F, A, H, L = cfg.width, cfg.mlp_dim, cfg.action_dim, cfg.chunk, cfg.layers
+    qkv, att = cfg.qkv_dim, cfg.attn_dim
+    M = batch * H
+    if lens is None:
+        lens = [cfg.prefix] * batch
+    if cfg.dtype == wl.W4A16:
+        wb = lambda n, k: n * k / 2 + n * (k // cfg.group_size) * 2  # noqa: E731
+    else:
+        es = 4 if cfg.dtype == wl.FP32 else 2
+        wb = lambda n, k: n * k * es  # noqa: E731
+    ae = 4 if cfg.dtype == wl.FP32 else 2
+    kv_tokens = sum(p + H for p in lens)
+    out = {
+        "qkv": {"bytes": wb(qkv, D) + M * D * ae + M * qkv * ae, "flops": 2 * M * qkv * D},
+        "attention": {"bytes": 2 * kv_tokens * cfg.n_kv_heads * cfg.head_dim * ae + 2 * M * att * ae,
+                      "flops": 4 * cfg.n_q_heads * H * cfg.head_dim * sum(p + H for p in lens)},
+        "o_proj": {"bytes": wb(D, att) + M * att * ae + 2 * M * D * 4, "flops": 2 * M * D * att},
+        "gate_up": {"bytes": wb(2 * F, D) + M * D * ae + M * F * ae, "flops": 2 * M * 2 * F * D},
+        "down": {"bytes": wb(D, F) + M * F * ae + 2 * M * D * 4, "flops": 2 * M * D * F},
+    }
+    step_w = L * (wb(qkv, D) + wb(D, att) + wb(2 * F, D) + wb(D, F)) + wb(D, A) * 2
+    step_kv = L * 2 * sum(lens) * cfg.n_kv_heads * cfg.head_dim * ae
+    step_flops = L * (out["qkv"]["flops"] + out["o_proj"]["flops"] + out["gate_up"]["flops"] +
+                      out["down"]["flops"] + out["attention"]["flops"]) + 2 * 2 * M * A * D
+    return out, {"bytes": step_w + step_kv, "flops": step_flops}
+
+
+def src_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "flow_matching_action_pi0_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(f"{workload}:{kernel}")
+    if not e or e.get("src_sha") != src_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# --------------------------------------------------------------- oracle timing
+def oracle_sample_time(cfg, W, ks, vs, noise, euler_steps: int):
+    """Seconds the float64 oracle takes for one request over `euler_steps`
+    Euler steps of the workload's grid (tables excluded, as on the GPU)."""
+    import oracle
+    p = oracle.params_from_weights(cfg, W)
+    grid = wl.uniform_grid(cfg.steps)
+    tabs = oracle.modulation_tables(grid, p)[:euler_steps]
+    kp = [np.asarray(a, np.float64) for a in ks[0]]
+    vp = [np.asarray(a, np.float64) for a in vs[0]]
+    t0 = time.perf_counter()
+    oracle.denoise_row(noise[0].astype(np.float64), tabs, p, kp, vp)
+    return time.perf_counter() - t0
+
+
+def run_reference(args, cfg):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    W = wl.make_weights(cfg)
+    lens = wl.prefix_lengths(cfg)[:1]
+    ks, vs = wl.make_prefix(cfg, lengths=lens)
+    noise = wl.make_noise(cfg, batch=1)
+    per = []
+    for i in range(args.warmup + args.steps):
+        t = oracle_sample_time(cfg, W, ks, vs, noise, 1)
+        if i >= args.warmup:
+            per.append(t)
+    t_euler = float(np.mean(per))
+    chunk_s = t_euler * cfg.steps            # one request, all Euler steps
+    value = 1.0 / chunk_s                    # rows are independent: chunks/s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "chunks/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": chunk_s * 1e3 * cfg.batch,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(cfg),
+        "cpu_baseline": {"value": value, "unit": "chunks/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"one request, one Euler step per timed step (x{cfg.steps} for a chunk)"},
+        "e2e": {"value": value, "unit": "chunks/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(cfg, batch=None):
+    return {"workload": cfg.name, "batch": cfg.batch if batch is None else batch, "chunk": cfg.chunk,
+            "action_dim": cfg.action_dim, "prefix": cfg.prefix, "euler_steps": cfg.steps,
+            "layers": cfg.layers, "width": cfg.width, "heads": f"{cfg.n_q_heads}q/{cfg.n_kv_heads}kv",
+            "head_dim": cfg.head_dim, "mlp_dim": cfg.mlp_dim, "weights": cfg.dtype,
+            "l2": "no flush: inputs larger than L2 (projection weights stream from HBM every Euler step)",
+            "parallelism": "replicas (one independent context per GPU)"}
+
+
+# ------------------------------------------------------------------ GPU timing
+def setup_context(cfg, W, batch: int, lens=None):
+    import flow_matching_action_pi0_b200 as fm
+    from workloads import device as wd
+    dev_w = wd.upload_weights(cfg, W)
+    ex = fm.ActionExpert(fm.make_config(**wd.abi_config(cfg, max_batch=batch)), dev_w)
+    del dev_w
+    if lens is None:
+        lens = [cfg.prefix] * batch
+    ks, vs = wl.make_prefix(cfg, lengths=lens)
+    kd, vd = wd.upload_prefix(cfg, ks, vs)
+    for b in range(batch):
+        ex.set_prefix(b, kd[b], vd[b], lens[b])
+    t0 = time.perf_counter()
+    ex.precompute_tables(wl.uniform_grid(cfg.steps))
+    ex.sync()
+    table_ms = (time.perf_counter() - t0) * 1e3
+    return ex, ks, vs, kd, vd, lens, table_ms
+
+
+def timed(fn, steps, warmup, stream, barrier):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    return e0.elapsed_time(e1) / steps
+
+
+def measure(cfg, W, batch, args, stream, barrier, maxr, lens=None, with_e2e=True, gpu_index=0):
+    import torch
+    import flow_matching_action_pi0_b200 as fm
+    ex, ks, vs, kd, vd, lens, table_ms = setup_context(cfg, W, batch, lens)
+    noise = wl.make_noise(cfg, batch=batch)
+    nd = torch.from_numpy(noise).cuda()
+    od = torch.empty_like(nd)
+    res = {"lens": lens}
+    with torch.cuda.stream(stream):
+        clk = ClockSampler(gpu_index).start()
+        ms = timed(lambda: ex.denoise(nd, od, stream), args.steps, args.warmup, stream, barrier)
+        res["clocks"] = clk.stop()
+        res["ms_per_step"] = maxr(ms)
+        res["graph_kernels"] = ex.query(fm.PAE_Q_GRAPH_KERNELS, batch)
+        res["splits"] = ex.query(fm.PAE_Q_SPLITS, batch)
+        res["token_tile"] = ex.query(fm.PAE_Q_TOKEN_TILE, batch)
+        res["table_ms"] = table_ms
+        if with_e2e:
+            nh = torch.from_numpy(noise).pin_memory()
+            oh = torch.empty_like(nh).pin_memory()
+            for _ in range(args.warmup):
+                ex.denoise_host(nh, oh, stream)
+            torch.cuda.synchronize()
+            barrier()
+            t0 = time.perf_counter()
+            for _ in range(args.steps):
+                ex.denoise_host(nh, oh, stream)
+                stream.synchronize()      # result read back on the host every step
+            wall = (time.perf_counter() - t0) / args.steps
+            res["e2e_ms"] = maxr(wall * 1e3)
+            res["io_bytes"] = int(nh.numel() * 4)
+        # live per-kernel timing: the same graph with CUDA events around every launch
+        ex.set_option(fm.PAE_OPT_PROFILE, (1 << 7) - 1)
+        n_prof = max(3, min(args.steps, 10))
+        for _ in range(2):
+            ex.denoise(nd, od, stream)
+        torch.cuda.synchronize()
+        tot = {c: 0.0 for c in fm.KERNEL_CLASSES}
+        cnt = {c: 0 for c in fm.KERNEL_CLASSES}
+        for _ in range(n_prof):
+            ex.denoise(nd, od, stream)
+            stream.synchronize()
+            for i, c in enumerate(fm.KERNEL_CLASSES):
+                t, n = ex.profile_read(i)
+                tot[c] += t
+                cnt[c] += n
+        ex.set_option(fm.PAE_OPT_PROFILE, 0)
+        res["kernels"] = {c: {"ms_per_launch": (tot[c] / cnt[c]) if cnt[c] else 0.0,
+                              "launches_per_step": cnt[c] // n_prof,
+                              "ms_per_step": tot[c] / n_prof} for c in fm.KERNEL_CLASSES}
+    res["ex"] = ex
+    res["ks"], res["vs"] = ks, vs
+    res["noise"] = noise
+    return res
+
+
+def roofline_for(cfg, batch, res, peaks, peak_kind, lens):
+    per, step = algorithmic(cfg, batch, lens)
+    ks = res["kernels"]
+    total = sum(v["ms_per_step"] for v in ks.values()) or 1.0
+    dom = max((c for c in per), key=lambda c: ks[c]["ms_per_step"])
+    dur_s = ks[dom]["ms_per_launch"] * 1e-3
+    hbm_bound = per[dom]["flops"] / max(per[dom]["bytes"], 1) < (peaks["bf16_tflops_sustained"] * 1e12) / (
+        peaks["hbm_gbs"] * 1e9)
+    if hbm_bound:
+        ach = per[dom]["bytes"] / dur_s / 1e9
+        peak = peaks["hbm_gbs"]
+        rl = {"bound": "hbm", "unit": "GB/s", "algorithmic_bytes_per_launch": per[dom]["bytes"]}
+    else:
+        ach = per[dom]["flops"] / dur_s / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        rl = {"bound": "tensor", "unit": "TFLOP/s", "algorithmic_flops_per_launch": per[dom]["flops"]}
+    rl.update({"kernel": dom, "achieved": ach, "peak": peak, "frac": ach / peak,
+               "peak_source": f"{peak_kind} ({'hbm_gbs' if hbm_bound else 'bf16_tflops_sustained'})",
+               "ms_per_launch": ks[dom]["ms_per_launch"], "share_of_step": ks[dom]["ms_per_step"] / total,
+               "traffic": ncu_traffic(cfg.name if batch == cfg.batch else f"{cfg.name}@{batch}", dom)})
+    # whole loop against the HBM and tensor rooflines
+    t_step = res["ms_per_step"] * 1e-3 / cfg.steps
+    hbm_t = step["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    tc_t = step["flops"] / (peaks["bf16_tflops_sustained"] * 1e12)
+    loop = {"euler_step_us": t_step * 1e6, "bytes_per_euler_step": step["bytes"],
+            "flops_per_euler_step": step["flops"], "hbm_roofline_us": hbm_t * 1e6,
+            "tensor_roofline_us": tc_t * 1e6, "frac_of_roofline": max(hbm_t, tc_t) / t_step,
+            "achieved_gbs": step["bytes"] / t_step / 1e9, "achieved_tflops": step["flops"] / t_step / 1e12}
+    shares = {c: ks[c]["ms_per_step"] / total for c in ks}
+    return rl, loop, shares
+
+
+def run_ours(args, cfg):
+    import torch
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local))
+
+        def barrier():
+            dist.barrier()
+
+        def maxr(v):
+            t = torch.tensor([float(v)], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            return float(t.item())
+    else:
+        def barrier():
+            pass
+
+        def maxr(v):
+            return float(v)
+    import flow_matching_action_pi0_b200 as fm
+    fm.lib()
+    peaks, peak_kind = load_peaks()
+    stream = torch.cuda.Stream()
+    W = wl.make_weights(cfg)
+    lens = wl.prefix_lengths(cfg)
+    gpu_index = local
+    res = measure(cfg, W, cfg.batch, args, stream, barrier, maxr, lens=lens, gpu_index=gpu_index)
+    ms = res["ms_per_step"]
+    value = ws * cfg.batch / (ms * 1e-3)
+    rl, loop, shares = roofline_for(cfg, cfg.batch, res, peaks, peak_kind, lens)
+    line = {
+        "metric": METRIC, "value": value, "unit": "chunks/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if cfg.dtype == wl.BF16 else cfg.dtype,
+        "data": "synthetic: seeded N(0,0.02) weights, N(0,1) prefix K/V and noise",
+        "config": workload_config(cfg), "per_euler_step_us": ms * 1e3 / cfg.steps,
+        "roofline": rl, "loop_roofline": loop, "kernel_shares": shares,
+        "kernels_ms_per_launch": {c: v["ms_per_launch"] for c, v in res["kernels"].items()},
+        "gpu_launches": int(res["graph_kernels"]) * args.steps,
+        "graph_kernels_per_step": int(res["graph_kernels"]),
+        "splitk": {"qkv": res["splits"] & 255, "o": (res["splits"] >> 8) & 255,
+                   "gate_up": (res["splits"] >> 16) & 255, "down": (res["splits"] >> 24) & 255},
+        "token_tile": res["token_tile"], "table_build_ms": res["table_ms"],
+        "clocks": res["clocks"],
+        "e2e": {"value": ws * cfg.batch / (res["e2e_ms"] * 1e-3), "unit": "chunks/s",
+                "h2d_bytes_per_step": res["io_bytes"], "d2h_bytes_per_step": res["io_bytes"],
+                "ms_per_step": res["e2e_ms"], "api": "pae_denoise_host (pinned host buffers)"},
+    }
+    ex = res.pop("ex")
+    ex.close()
+    del res
+    torch.cuda.empty_cache()
+    if args.secondary and cfg.name == wl.PI05_BF16_BS1.name:
+        c32 = wl.PI05_BF16_BS32
+        r32 = measure(c32, W, c32.batch, args, stream, barrier, maxr, with_e2e=False, gpu_index=gpu_index)
+        rl32, loop32, sh32 = roofline_for(c32, c32.batch, r32, peaks, peak_kind, r32["lens"])
+        line["secondary"] = {c32.name: {
+            "value": ws * c32.batch / (r32["ms_per_step"] * 1e-3), "unit": "chunks/s",
+            "ms_per_step": r32["ms_per_step"], "roofline": rl32, "loop_roofline": loop32,
+            "kernel_shares": sh32, "clocks": r32["clocks"],
+            "kernels_ms_per_launch": {c: v["ms_per_launch"] for c, v in r32["kernels"].items()},
+            "splitk": r32["splits"], "token_tile": r32["token_tile"],
+            "note": "same weights as the batch-1 line; 32 independent 968-token prefixes"}}
+        r32.pop("ex").close()
+        del r32
+    if args.cpu_baseline and ws == 1 and rank == 0:
+        t = oracle_sample_time(cfg, W, *wl.make_prefix(cfg, lengths=lens[:1]), wl.make_noise(cfg, batch=1),
+                               cfg.steps)
+        line["cpu_baseline"] = {"value": 1.0 / t, "unit": "chunks/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"one request of the workload, all {cfg.steps} Euler steps "
+                                          f"({t:.1f} s); requests are independent"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default=wl.PI05_BF16_BS1.name, choices=sorted(wl.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-secondary", dest="secondary", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    cfg = wl.CONFIGS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,57 @@
+// GEMM epilogues shared by the CUDA-core and tcgen05 projection kernels.
+// One call handles one (token m, output feature f) with the accumulated
+// dot products acc0 (and acc1 for the GeGLU up projection).
+#pragma once
+
+#include "internal.h"
+
+namespace pae {
+
+// [q | k | v] = y W_qkv^T: q goes to the per-request head-major buffer
+// q[b][hq][i][:], k and v into this layer's KV slot of request b right after its
+// prefix (position lens[b] + i), so attention reads one contiguous key range.
+template <typename TA>
+__device__ __forceinline__ void epi_qkv(const Shape& s, const EpiArgs& e, int m, int f, float acc) {
+  const int b = m / s.H, i = m - b * s.H;
+  const int qd = s.Hq * s.d;
+  if (f < qd) {
+    const int hq = f / s.d, j = f - hq * s.d;
+    st_act<TA>(static_cast<TA*>(e.q) + ((size_t)(b * s.Hq + hq) * s.H + i) * s.d + j, acc);
+  } else {
+    const int kvd = s.Hkv * s.d;
+    const bool is_v = f >= qd + kvd;
+    const int fk = f - qd - (is_v ? kvd : 0);
+    const int g = fk / s.d, j = fk - g * s.d;
+    const int pos = e.lens[b] + i;
+    const size_t off = (((size_t)(e.layer * s.Bmax + b) * s.Hkv + g) * s.Ptot + pos) * s.d + j;
+    st_act<TA>(static_cast<TA*>(is_v ? e.vc : e.kc) + off, acc);
+  }
+}
+
+// h += gate * acc  (gated residual; gate from this step's modulation table)
+__device__ __forceinline__ void epi_resid(const Shape& s, const EpiArgs& e, int m, int f, float acc) {
+  float* hp = e.h + (size_t)m * s.D + f;
+  *hp = fmaf(e.gate[f], acc, *hp);
+}
+
+// u = gelu_tanh(y W_gate^T) * (y W_up^T)
+template <typename TA>
+__device__ __forceinline__ void epi_geglu(const Shape& s, const EpiArgs& e, int m, int f, float g, float up) {
+  st_act<TA>(static_cast<TA*>(e.u) + (size_t)m * s.F + f, gelu_tanh(g) * up);
+}
+
+template <typename TA>
+__device__ __forceinline__ void epi_apply(const Shape& s, const EpiArgs& e, int m, int f, float a0, float a1) {
+  if (e.epi == EPI_QKV)
+    epi_qkv<TA>(s, e, m, f, a0);
+  else if (e.epi == EPI_RESID)
+    epi_resid(s, e, m, f, a0);
+  else
+    epi_geglu<TA>(s, e, m, f, a0, a1);
+}
+
+// Row of the weight matrix holding output feature f (GeGLU: gate/up
+// interleaved in 128-row tiles: tile t = [gate rows 128t.., up rows 128t..]).
+__host__ __device__ __forceinline__ int gate_row(int f) { return (f >> 7) * 256 + (f & 127); }
+
+}  // namespace pae

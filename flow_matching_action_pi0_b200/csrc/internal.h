@@ -1,0 +1,113 @@
+// Internal launch interface between the context (pae_api.cu) and the kernel
+// files.  Host-side declarations only.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace pae {
+
+// Shapes the kernels need, fixed at pae_create.
+struct Shape {
+  int L, D, Hq, Hkv, d, F, A, H;
+  int Bmax, Pmax, Ptot;  // Ptot = Pmax + H: slot length (prefix + action keys)
+  int G;                 // Hq / Hkv
+  int qkv_rows;          // (Hq + 2 Hkv) d
+  int attn_dim;          // Hq d
+  int group;             // W4A16 group size
+  float eps;
+  int table_rows;        // (2L*3 + 2) D floats per step
+};
+
+// Where the modulation of one norm sits inside a step's table row.
+__host__ __device__ inline int mod_offset(const Shape& s, int layer, int norm, int chunk) {
+  return ((layer * 2 + norm) * 3 + chunk) * s.D;
+}
+__host__ __device__ inline int final_offset(const Shape& s, int chunk) {
+  return s.L * 2 * 3 * s.D + chunk * s.D;
+}
+
+// ------------------------------------------------------------ table builders
+// t (device, K+1 doubles) -> e/c in `tc` [K][D] fp32 and dt [K].
+void launch_time_mlp(const Shape& s, int act_bf16, const double* t, int K, const void* w_t1,
+                     const void* b_t1, const void* w_t2, const void* b_t2, float* emb, float* zbuf,
+                     float* cbuf, float* dt, cudaStream_t st);
+// tables[k][r] = W_all[r] . c_k + b_all[r] for all table rows.
+void launch_mod_tables(const Shape& s, int act_bf16, const float* cbuf, int K, const void* w_all,
+                       const void* b_all, float* tables, cudaStream_t st);
+
+// ------------------------------------------------------------ token kernels
+// Per token: optionally (final adaRMSNorm, out_proj, Euler update of x with
+// step k_out), then optionally (in_proj of x and the first attention norm of
+// step k_in).  Writes h (fp32) and y (act dtype).
+struct TransitionArgs {
+  float* x;               // [M][A]
+  const float* x_src;     // read x from here in the first launch of a call (may equal x)
+  float* h;               // [M][D]
+  void* y;                // [M][D] act dtype
+  const void* w_in; const void* b_in; const void* w_out; const void* b_out;
+  const float* tab_out;   // table row of the step being finished (null: no out step)
+  const float* dt;        // dt array (device)
+  int k_out;
+  const float* tab_in;    // table row of the step being started (null: no in step)
+  float* x_dst;           // write x here after the out step (may equal x)
+  int M;
+};
+void launch_transition(const Shape& s, int act_bf16, const TransitionArgs& a, cudaStream_t st);
+
+// y = adaRMSNorm(h; scale, shift) per token.
+void launch_norm(const Shape& s, int act_bf16, const float* h, void* y, const float* scale,
+                 const float* shift, int M, cudaStream_t st);
+
+// --------------------------------------------------------- CUDA-core (fp32)
+enum Epi : int { EPI_QKV = 0, EPI_RESID = 1, EPI_GEGLU = 2 };
+
+struct EpiArgs {
+  int epi;
+  int M;
+  // EPI_QKV
+  void* q;            // [B][Hq][H][d] act dtype
+  void* kc; void* vc; // [L][Bmax][Hkv][Ptot][d] act dtype
+  const int* lens;    // [Bmax] prefix length per row
+  int layer;
+  // EPI_RESID
+  float* h;           // [M][D]
+  const float* gate;  // [D]
+  // EPI_GEGLU
+  void* u;            // [M][F]
+};
+
+// out-features N (for GEGLU: F, weight rows interleaved in 128-row tiles).
+void launch_gemm_simple(const Shape& s, const float* X, const float* W, int N, int K,
+                        const EpiArgs& e, cudaStream_t st);
+
+// o = attention(q, [prefix | action] keys) per request; CUDA cores.
+void launch_attention_simple(const Shape& s, int act_bf16, const void* q, const void* kc,
+                             const void* vc, const int* lens, int layer, void* o, int B,
+                             cudaStream_t st);
+
+// ----------------------------------------------------------- tcgen05 GEMM
+struct TcPlan {
+  int tn;          // token tile (MMA N), multiple of 16, <= 256
+  int tok_tiles;
+  int splits;
+  int stages;
+};
+struct TcGemmArgs {
+  EpiArgs e;
+  int N;           // output features (GEGLU: F)
+  int K;
+  int w_row0;      // first row of this layer's matrix inside the stacked weight map
+  float* partials; // split-K workspace
+  int* counters;   // split-K arrival counters (zeroed; the last CTA re-zeroes)
+  DevErr err;
+};
+void launch_tc_gemm(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* tmX, int na,
+                    const TcPlan& p, const TcGemmArgs& a, cudaStream_t st);
+size_t tc_gemm_smem_bytes(int na, const TcPlan& p);
+cudaError_t tc_gemm_init();  // once per process: opt in to large dynamic shared memory
+
+}  // namespace pae

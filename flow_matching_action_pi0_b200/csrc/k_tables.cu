@@ -1,0 +1,117 @@
+// Timestep conditioning, built once per timestep grid (PhyAI report, Sec. 5.1:
+// "precomputing timestep and modulation tables also avoids repeated setup").
+//
+//   e_k  = sinusoidal embedding of t_k (half = D/2 geometric periods from
+//          4e-3 to 4.0; sines then cosines)
+//   c_k  = swish(W_t2 swish(W_t1 e_k + b_t1) + b_t2)
+//   tab_k[r] = W_all[r] . c_k + b_all[r]   for every modulation row r
+//   dt_k = t_{k+1} - t_k
+//
+// The modulation rows are stacked [layer][norm][scale|shift|gate][D] followed by
+// the final norm's [scale|shift][D].  All weights for all steps are read once
+// (a batched GEMV with K columns); results are fp32.
+#include "internal.h"
+
+namespace pae {
+
+namespace {
+
+constexpr int KC = 16;  // timesteps per pass of the batched GEMV
+
+__global__ void k_time_embed(const double* __restrict__ t, int K, int D, float* __restrict__ emb,
+                             float* __restrict__ dt) {
+  const int k = blockIdx.x;
+  const int half = D / 2;
+  const double tk = t[k];
+  const double ratio = 4.0 / 4e-3;
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    const double frac = half > 1 ? (double)i / (double)(half - 1) : 0.0;
+    const double period = 4e-3 * pow(ratio, frac);
+    const double ang = 2.0 * 3.141592653589793238 * tk / period;
+    emb[(size_t)k * D + i] = (float)sin(ang);
+    emb[(size_t)k * D + half + i] = (float)cos(ang);
+  }
+  if (threadIdx.x == 0) dt[k] = (float)(t[k + 1] - t[k]);
+}
+
+template <typename TW>
+__device__ __forceinline__ float ldw(const TW* p);
+template <>
+__device__ __forceinline__ float ldw<float>(const float* p) { return __ldg(p); }
+template <>
+__device__ __forceinline__ float ldw<bf16>(const bf16* p) { return bf2f(*p); }
+
+// out[k][r] = act(W[r] . in[k] + b[r]) for k < K, r < R.  One warp per row;
+// the input columns of up to KC timesteps are staged in shared memory.
+template <typename TW>
+__global__ void k_batched_gemv(const TW* __restrict__ W, const TW* __restrict__ b,
+                               const float* __restrict__ in, int K, int R, int D, int swish_out,
+                               float* __restrict__ out) {
+  extern __shared__ float xs[];  // [KC][D]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int k0 = 0; k0 < K; k0 += KC) {
+    const int kc = min(KC, K - k0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kc * D; i += blockDim.x) xs[i] = in[(size_t)k0 * D + i];
+    __syncthreads();
+    for (int r = blockIdx.x * nw + warp; r < R; r += gridDim.x * nw) {
+      float acc[KC];
+#pragma unroll
+      for (int j = 0; j < KC; ++j) acc[j] = 0.f;
+      const TW* wr = W + (size_t)r * D;
+      for (int i = lane; i < D; i += 32) {
+        const float w = ldw(wr + i);
+#pragma unroll
+        for (int j = 0; j < KC; ++j)
+          if (j < kc) acc[j] = fmaf(w, xs[j * D + i], acc[j]);
+      }
+      const float bias = ldw(b + r);
+#pragma unroll
+      for (int j = 0; j < KC; ++j) {
+        if (j < kc) {
+          float v = warp_sum(acc[j]) + bias;
+          if (swish_out) v = swishf(v);
+          if (lane == 0) out[(size_t)(k0 + j) * R + r] = v;
+        }
+      }
+    }
+  }
+}
+
+template <typename TW>
+void gemv(const void* W, const void* b, const float* in, int K, int R, int D, int swish_out, float* out,
+          cudaStream_t st) {
+  const int threads = 256, wpb = threads / 32;
+  int blocks = (R + wpb - 1) / wpb;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  const size_t smem = (size_t)KC * D * sizeof(float);
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(k_batched_gemv<TW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  k_batched_gemv<TW><<<blocks, threads, smem, st>>>(static_cast<const TW*>(W), static_cast<const TW*>(b), in,
+                                                     K, R, D, swish_out, out);
+}
+
+}  // namespace
+
+void launch_time_mlp(const Shape& s, int act_bf16, const double* t, int K, const void* w_t1, const void* b_t1,
+                     const void* w_t2, const void* b_t2, float* emb, float* zbuf, float* cbuf, float* dt,
+                     cudaStream_t st) {
+  k_time_embed<<<K, 256, 0, st>>>(t, K, s.D, emb, dt);
+  if (act_bf16) {
+    gemv<bf16>(w_t1, b_t1, emb, K, s.D, s.D, 1, zbuf, st);
+    gemv<bf16>(w_t2, b_t2, zbuf, K, s.D, s.D, 1, cbuf, st);
+  } else {
+    gemv<float>(w_t1, b_t1, emb, K, s.D, s.D, 1, zbuf, st);
+    gemv<float>(w_t2, b_t2, zbuf, K, s.D, s.D, 1, cbuf, st);
+  }
+}
+
+void launch_mod_tables(const Shape& s, int act_bf16, const float* cbuf, int K, const void* w_all,
+                       const void* b_all, float* tables, cudaStream_t st) {
+  if (act_bf16)
+    gemv<bf16>(w_all, b_all, cbuf, K, s.table_rows, s.D, 0, tables, st);
+  else
+    gemv<float>(w_all, b_all, cbuf, K, s.table_rows, s.D, 0, tables, st);
+}
+
+}  // namespace pae

@@ -1,0 +1,909 @@
+// The C ABI of include/pae.h: context lifetime, weight repacking, prefix slots,
+// timestep tables, and the K-step loop (enqueued directly or replayed from a
+// captured CUDA graph).
+//
+// The loop structure is the pi0.5 path of "PhyAI: Real-Time Physical AI at
+// the Edge" (Sec. 5.1 and Sec. 5.5): the prefix K/V stays fixed across the
+// Euler steps and is replaced only by a new observation (pae_set_prefix), the
+// timestep/modulation tables are built once (pae_precompute_tables), and the
+// stable loop is replayed as a CUDA graph (pae_denoise).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <vector>
+
+#include "../../include/pae.h"
+#include "internal.h"
+
+using namespace pae;
+
+namespace {
+
+thread_local std::string g_create_error;
+
+constexpr int kMaxSteps = 64;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct ProfRec {
+  int kind;
+  int ev0, ev1;  // indices into the context's event pool
+};
+
+struct Plan {
+  int B = 0, M = 0;
+  TcPlan qkv{}, o{}, gu{}, down{};
+  CUtensorMap tmY{}, tmO{}, tmU{};
+  cudaGraphExec_t graph = nullptr;
+  int graph_K = 0;
+  long long graph_kernels = 0;
+  std::vector<ProfRec> recs;  // profiled launches of the last enqueue / capture
+};
+
+__global__ void k_set_len(int* lens, int row, int len) { lens[row] = len; }
+
+template <typename T>
+__global__ void k_transpose(const T* __restrict__ src, T* __restrict__ dst, int rows, int cols) {
+  // dst[c][r] = src[r][c]
+  const size_t n = (size_t)rows * cols;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t r = i / cols, c = i - r * cols;
+    dst[c * rows + r] = src[i];
+  }
+}
+
+}  // namespace
+
+struct pae_ctx {
+  pae_config cfg{};
+  Shape s{};
+  int device = 0;
+  int act_bf16 = 0;  // bf16 activations (BF16 and W4A16 modes)
+  size_t esize = 4;  // bytes per weight element (non-quantised)
+  std::vector<void*> allocs;
+  // weights (device, repacked)
+  void *w_inT = nullptr, *b_in = nullptr, *w_out = nullptr, *b_out = nullptr;
+  void *w_t1 = nullptr, *b_t1 = nullptr, *w_t2 = nullptr, *b_t2 = nullptr;
+  void *w_modall = nullptr, *b_modall = nullptr;
+  void *w_qkv = nullptr, *w_o = nullptr, *w_gu = nullptr, *w_down = nullptr;  // stacked over layers
+  CUtensorMap tmWqkv{}, tmWo{}, tmWgu{}, tmWdown{};
+  // tables
+  double* t_dev = nullptr;
+  float *emb = nullptr, *zbuf = nullptr, *cbuf = nullptr, *tables = nullptr, *dt = nullptr;
+  int K = 0;
+  bool tables_ready = false;
+  // prefix slots
+  void *kc = nullptr, *vc = nullptr;
+  int* lens_dev = nullptr;
+  std::vector<int> lens_host;
+  // activations and workspaces
+  float *x = nullptr, *h = nullptr;
+  void *y = nullptr, *q = nullptr, *o = nullptr, *u = nullptr;
+  float* partials = nullptr;
+  size_t partials_floats = 0;
+  int* counters = nullptr;
+  int counters_n = 0;
+  // error word (host-mapped)
+  int* err_host = nullptr;
+  int* err_dev = nullptr;
+  long long wait_ns = 2000000000LL;
+  bool use_graph = true;
+  std::map<int, Plan> plans;
+  Plan* last_plan = nullptr;
+  unsigned profile_mask = 0;
+  std::vector<cudaEvent_t> ev_pool;
+  int ev_next = 0;
+  std::vector<ProfRec>* rec_sink = nullptr;
+  cudaStream_t cap_stream = nullptr;
+  EncodeTiledFn encode = nullptr;
+  std::string last_error;
+};
+
+namespace {
+
+pae_status fail(pae_ctx* c, pae_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  if (c)
+    c->last_error = buf;
+  else
+    g_create_error = buf;
+  return st;
+}
+
+#define CK(call)                                                                              \
+  do {                                                                                        \
+    cudaError_t e_ = (call);                                                                  \
+    if (e_ != cudaSuccess) return fail(ctx, PAE_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+pae_status dev_alloc(pae_ctx* ctx, void** p, size_t bytes) {
+  *p = nullptr;
+  if (bytes == 0) bytes = 16;
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(ctx, PAE_ERR_OOM, "cudaMalloc(%zu bytes): %s", bytes, cudaGetErrorString(e));
+  }
+  ctx->allocs.push_back(*p);
+  return PAE_OK;
+}
+
+pae_status check_err_word(pae_ctx* ctx) {
+  if (ctx->err_host && *(volatile int*)ctx->err_host != 0) {
+    const int code = *(volatile int*)ctx->err_host;
+    return fail(ctx, PAE_ERR_TIMEOUT, "device error word set (%d): a bounded device wait ran out", code);
+  }
+  return PAE_OK;
+}
+
+pae_status make_map(pae_ctx* ctx, CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                    uint32_t box_inner, uint32_t box_outer) {
+  // bf16 matrix [outer][inner], 128-byte swizzled boxes of box_inner x box_outer.
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = ctx->encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(ctx, PAE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for [%llu][%llu] box %ux%u", (int)r,
+                (unsigned long long)outer, (unsigned long long)inner, box_outer, box_inner);
+  return PAE_OK;
+}
+
+// Token tile and split-K choice for one projection of `nfeat` outputs and K
+// inputs: the token tile covers the tokens with as little padding as possible
+// (<= 256 per MMA), and split-K fills the 148 SMs when the tile count is small.
+TcPlan plan_gemm(int M, int nfeat, int K, int na) {
+  TcPlan p{};
+  p.tok_tiles = (M + 255) / 256;
+  int per = (M + p.tok_tiles - 1) / p.tok_tiles;
+  p.tn = std::max(16, ((per + 15) / 16) * 16);
+  const int base = ((nfeat + 127) / 128) * p.tok_tiles;
+  const int nkb = K / 64;
+  const int target = 2 * 148;
+  p.splits = 1;
+  for (int sp = 1; sp <= nkb; ++sp)
+    if (nkb % sp == 0 && base * sp <= target) p.splits = sp;
+  const uint32_t stage = (uint32_t)na * 16384u + (uint32_t)p.tn * 128u;
+  int st = (int)((200u * 1024u) / stage);  // leaves room for barriers and alignment slack
+  st = std::max(2, std::min(st, 6));
+  p.stages = st;
+  return p;
+}
+
+pae_status build_plan(pae_ctx* ctx, int B, Plan* P) {
+  const Shape& s = ctx->s;
+  P->B = B;
+  P->M = B * s.H;
+  if (!ctx->act_bf16) return PAE_OK;
+  P->qkv = plan_gemm(P->M, s.qkv_rows, s.D, 1);
+  P->o = plan_gemm(P->M, s.D, s.attn_dim, 1);
+  P->gu = plan_gemm(P->M, s.F, s.D, 2);
+  P->down = plan_gemm(P->M, s.D, s.F, 1);
+  const uint64_t Mmax = (uint64_t)s.Bmax * s.H;
+  pae_status st;
+  if ((st = make_map(ctx, &P->tmY, ctx->y, s.D, Mmax, 64, P->qkv.tn)) != PAE_OK) return st;
+  if ((st = make_map(ctx, &P->tmO, ctx->o, s.attn_dim, Mmax, 64, P->o.tn)) != PAE_OK) return st;
+  if ((st = make_map(ctx, &P->tmU, ctx->u, s.F, Mmax, 64, P->down.tn)) != PAE_OK) return st;
+  return PAE_OK;
+}
+
+size_t plan_partials(const Plan& P, const Shape& s) {
+  auto one = [&](const TcPlan& p, int n, int na) -> size_t {
+    if (p.splits <= 1) return 0;
+    return (size_t)p.splits * na * p.tok_tiles * p.tn * n;
+  };
+  return std::max(std::max(one(P.qkv, s.qkv_rows, 1), one(P.o, s.D, 1)),
+                  std::max(one(P.gu, s.F, 2), one(P.down, s.D, 1)));
+}
+int plan_counters(const Plan& P, const Shape& s) {
+  auto one = [&](const TcPlan& p, int n) { return ((n + 127) / 128) * p.tok_tiles; };
+  return std::max(std::max(one(P.qkv, s.qkv_rows), one(P.o, s.D)), std::max(one(P.gu, s.F), one(P.down, s.D)));
+}
+
+// Launch bracketing for PAE_OPT_PROFILE: events come from a pool sized before
+// capture starts (ensure_events), so nothing is created during capture.
+struct ProfScope {
+  pae_ctx* ctx;
+  cudaStream_t st;
+  int kind, ev0 = -1;
+  ProfScope(pae_ctx* c, int k, cudaStream_t s) : ctx(c), st(s), kind(k) {
+    if ((ctx->profile_mask >> kind) & 1u) {
+      if (ctx->ev_next + 2 <= (int)ctx->ev_pool.size() && ctx->rec_sink) {
+        ev0 = ctx->ev_next;
+        ctx->ev_next += 2;
+        cudaEventRecord(ctx->ev_pool[ev0], st);
+      }
+    }
+  }
+  ~ProfScope() {
+    if (ev0 >= 0) {
+      cudaEventRecord(ctx->ev_pool[ev0 + 1], st);
+      ctx->rec_sink->push_back(ProfRec{kind, ev0, ev0 + 1});
+    }
+  }
+};
+
+pae_status ensure_events(pae_ctx* ctx, int k_steps) {
+  if (!ctx->profile_mask) return PAE_OK;
+  const size_t need = (size_t)2 * ((size_t)k_steps * (7 * ctx->s.L + 1) + 2);
+  while (ctx->ev_pool.size() < need) {
+    cudaEvent_t e;
+    CK(cudaEventCreate(&e));
+    ctx->ev_pool.push_back(e);
+  }
+  return PAE_OK;
+}
+
+const float* tab(const pae_ctx* ctx, int k) { return ctx->tables + (size_t)k * ctx->s.table_rows; }
+
+void run_gemm(pae_ctx* ctx, const Plan& P, int which, int layer, const EpiArgs& e, cudaStream_t st) {
+  const Shape& s = ctx->s;
+  const size_t es = ctx->esize;
+  if (!ctx->act_bf16) {
+    const float* X;
+    const float* W;
+    int N, K;
+    switch (which) {
+      case 0: X = (const float*)ctx->y; W = (const float*)((char*)ctx->w_qkv + (size_t)layer * s.qkv_rows * s.D * es); N = s.qkv_rows; K = s.D; break;
+      case 1: X = (const float*)ctx->o; W = (const float*)((char*)ctx->w_o + (size_t)layer * s.D * s.attn_dim * es); N = s.D; K = s.attn_dim; break;
+      case 2: X = (const float*)ctx->y; W = (const float*)((char*)ctx->w_gu + (size_t)layer * 2 * s.F * s.D * es); N = s.F; K = s.D; break;
+      default: X = (const float*)ctx->u; W = (const float*)((char*)ctx->w_down + (size_t)layer * s.D * s.F * es); N = s.D; K = s.F; break;
+    }
+    launch_gemm_simple(s, X, W, N, K, e, st);
+    return;
+  }
+  TcGemmArgs a{};
+  a.e = e;
+  a.partials = ctx->partials;
+  a.counters = ctx->counters;
+  a.err = DevErr{ctx->err_dev, ctx->wait_ns};
+  const CUtensorMap *tw, *tx;
+  const TcPlan* p;
+  int na = 1;
+  switch (which) {
+    case 0: tw = &ctx->tmWqkv; tx = &P.tmY; p = &P.qkv; a.N = s.qkv_rows; a.K = s.D; a.w_row0 = layer * s.qkv_rows; break;
+    case 1: tw = &ctx->tmWo; tx = &P.tmO; p = &P.o; a.N = s.D; a.K = s.attn_dim; a.w_row0 = layer * s.D; break;
+    case 2: tw = &ctx->tmWgu; tx = &P.tmY; p = &P.gu; a.N = s.F; a.K = s.D; a.w_row0 = layer * 2 * s.F; na = 2; break;
+    default: tw = &ctx->tmWdown; tx = &P.tmU; p = &P.down; a.N = s.D; a.K = s.F; a.w_row0 = layer * s.D; break;
+  }
+  launch_tc_gemm(s, tw, tx, na, *p, a, st);
+}
+
+// Enqueue Euler steps k_begin..k_end-1 for the plan's batch on `st`, with the
+// state in ctx->x.
+void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStream_t st) {
+  const Shape& s = ctx->s;
+  const int M = P.M;
+  TransitionArgs ta{};
+  ta.x = ctx->x;
+  ta.x_src = ctx->x;
+  ta.x_dst = ctx->x;
+  ta.h = ctx->h;
+  ta.y = ctx->y;
+  ta.w_in = ctx->w_inT;
+  ta.b_in = ctx->b_in;
+  ta.w_out = ctx->w_out;
+  ta.b_out = ctx->b_out;
+  ta.dt = ctx->dt;
+  ta.M = M;
+  ctx->ev_next = 0;
+  for (int k = k_begin; k < k_end; ++k) {
+    const float* tk = tab(ctx, k);
+    ta.tab_out = (k == k_begin) ? nullptr : tab(ctx, k - 1);
+    ta.k_out = k - 1;
+    ta.tab_in = tk;
+    {
+      ProfScope ps(ctx, PAE_K_TRANSITION, st);
+      launch_transition(s, ctx->act_bf16, ta, st);
+    }
+    for (int l = 0; l < s.L; ++l) {
+      EpiArgs e{};
+      e.M = M;
+      e.layer = l;
+      e.epi = EPI_QKV;
+      e.q = ctx->q;
+      e.kc = ctx->kc;
+      e.vc = ctx->vc;
+      e.lens = ctx->lens_dev;
+      {
+        ProfScope ps(ctx, PAE_K_QKV, st);
+        run_gemm(ctx, P, 0, l, e, st);
+      }
+      {
+        ProfScope ps(ctx, PAE_K_ATTENTION, st);
+        launch_attention_simple(s, ctx->act_bf16, ctx->q, ctx->kc, ctx->vc, ctx->lens_dev, l, ctx->o, P.B, st);
+      }
+      e = EpiArgs{};
+      e.M = M;
+      e.epi = EPI_RESID;
+      e.h = ctx->h;
+      e.gate = tk + mod_offset(s, l, 0, 2);
+      {
+        ProfScope ps(ctx, PAE_K_OPROJ, st);
+        run_gemm(ctx, P, 1, l, e, st);
+      }
+      {
+        ProfScope ps(ctx, PAE_K_NORM, st);
+        launch_norm(s, ctx->act_bf16, ctx->h, ctx->y, tk + mod_offset(s, l, 1, 0), tk + mod_offset(s, l, 1, 1), M,
+                    st);
+      }
+      e = EpiArgs{};
+      e.M = M;
+      e.epi = EPI_GEGLU;
+      e.u = ctx->u;
+      {
+        ProfScope ps(ctx, PAE_K_GATEUP, st);
+        run_gemm(ctx, P, 2, l, e, st);
+      }
+      e = EpiArgs{};
+      e.M = M;
+      e.epi = EPI_RESID;
+      e.h = ctx->h;
+      e.gate = tk + mod_offset(s, l, 1, 2);
+      {
+        ProfScope ps(ctx, PAE_K_DOWN, st);
+        run_gemm(ctx, P, 3, l, e, st);
+      }
+      if (l + 1 < s.L) {
+        ProfScope ps(ctx, PAE_K_NORM, st);
+        launch_norm(s, ctx->act_bf16, ctx->h, ctx->y, tk + mod_offset(s, l + 1, 0, 0), tk + mod_offset(s, l + 1, 0, 1),
+                    M, st);
+      }
+    }
+  }
+  ta.tab_out = tab(ctx, k_end - 1);
+  ta.k_out = k_end - 1;
+  ta.tab_in = nullptr;
+  {
+    ProfScope ps(ctx, PAE_K_TRANSITION, st);
+    launch_transition(s, ctx->act_bf16, ta, st);
+  }
+}
+
+pae_status get_plan(pae_ctx* ctx, int B, Plan** out) {
+  auto it = ctx->plans.find(B);
+  if (it == ctx->plans.end()) {
+    Plan P;
+    pae_status st = build_plan(ctx, B, &P);
+    if (st != PAE_OK) return st;
+    it = ctx->plans.emplace(B, P).first;
+  }
+  *out = &it->second;
+  return PAE_OK;
+}
+
+void drop_graphs(pae_ctx* ctx) {
+  for (auto& kv : ctx->plans) {
+    if (kv.second.graph) cudaGraphExecDestroy(kv.second.graph);
+    kv.second.graph = nullptr;
+    kv.second.graph_K = 0;
+  }
+}
+
+pae_status check_rows(pae_ctx* ctx, int batch) {
+  for (int b = 0; b < batch; ++b)
+    if (ctx->lens_host[b] < 0) return fail(ctx, PAE_ERR_STATE, "prefix row %d was never set", b);
+  return PAE_OK;
+}
+
+pae_status run_loop(pae_ctx* ctx, Plan* P, cudaStream_t stream) {
+  pae_status pst = ensure_events(ctx, ctx->K);
+  if (pst != PAE_OK) return pst;
+  ctx->last_plan = P;
+  if (!ctx->use_graph) {
+    P->recs.clear();
+    ctx->rec_sink = &P->recs;
+    enqueue_steps(ctx, *P, 0, ctx->K, stream);
+    ctx->rec_sink = nullptr;
+    CK(cudaGetLastError());
+    return PAE_OK;
+  }
+  if (!P->graph || P->graph_K != ctx->K) {
+    if (P->graph) cudaGraphExecDestroy(P->graph);
+    P->graph = nullptr;
+    cudaGraph_t g = nullptr;
+    P->recs.clear();
+    ctx->rec_sink = &P->recs;
+    CK(cudaStreamBeginCapture(ctx->cap_stream, cudaStreamCaptureModeThreadLocal));
+    enqueue_steps(ctx, *P, 0, ctx->K, ctx->cap_stream);
+    ctx->rec_sink = nullptr;
+    cudaError_t e1 = cudaGetLastError();
+    cudaError_t e2 = cudaStreamEndCapture(ctx->cap_stream, &g);
+    if (e1 != cudaSuccess || e2 != cudaSuccess) {
+      if (g) cudaGraphDestroy(g);
+      return fail(ctx, PAE_ERR_CUDA, "graph capture failed: %s / %s", cudaGetErrorString(e1), cudaGetErrorString(e2));
+    }
+    size_t nn = 0;
+    P->graph_kernels = 0;
+    if (cudaGraphGetNodes(g, nullptr, &nn) == cudaSuccess && nn > 0) {
+      std::vector<cudaGraphNode_t> nodes(nn);
+      if (cudaGraphGetNodes(g, nodes.data(), &nn) == cudaSuccess)
+        for (size_t i = 0; i < nn; ++i) {
+          cudaGraphNodeType t;
+          if (cudaGraphNodeGetType(nodes[i], &t) == cudaSuccess && t == cudaGraphNodeTypeKernel) ++P->graph_kernels;
+        }
+    }
+    cudaError_t e3 = cudaGraphInstantiate(&P->graph, g, 0);
+    cudaGraphDestroy(g);
+    if (e3 != cudaSuccess) {
+      P->graph = nullptr;
+      return fail(ctx, PAE_ERR_CUDA, "cudaGraphInstantiate: %s", cudaGetErrorString(e3));
+    }
+    P->graph_K = ctx->K;
+  }
+  CK(cudaGraphLaunch(P->graph, stream));
+  return PAE_OK;
+}
+
+void free_all(pae_ctx* ctx) {
+  if (!ctx) return;
+  drop_graphs(ctx);
+  for (cudaEvent_t e : ctx->ev_pool) cudaEventDestroy(e);
+  ctx->ev_pool.clear();
+  for (void* p : ctx->allocs) cudaFree(p);
+  ctx->allocs.clear();
+  if (ctx->err_host) cudaFreeHost(ctx->err_host);
+  ctx->err_host = nullptr;
+  if (ctx->cap_stream) cudaStreamDestroy(ctx->cap_stream);
+  ctx->cap_stream = nullptr;
+}
+
+bool is_pos(int v) { return v > 0; }
+
+pae_status validate_config(const pae_config* c) {
+  if (!is_pos(c->layers) || !is_pos(c->width) || !is_pos(c->n_q_heads) || !is_pos(c->n_kv_heads) ||
+      !is_pos(c->head_dim) || !is_pos(c->mlp_dim) || !is_pos(c->action_dim) || !is_pos(c->chunk) ||
+      !is_pos(c->max_batch) || c->max_prefix < 0 || !(c->rms_eps > 0.f))
+    return fail(nullptr, PAE_ERR_ARG, "config: sizes must be positive (max_prefix >= 0, rms_eps > 0)");
+  if (c->dtype != PAE_FP32 && c->dtype != PAE_BF16 && c->dtype != PAE_W4A16)
+    return fail(nullptr, PAE_ERR_ARG, "config: unknown dtype %d", c->dtype);
+  if (c->n_q_heads % c->n_kv_heads != 0)
+    return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: n_q_heads must be a multiple of n_kv_heads");
+  if (c->n_q_heads / c->n_kv_heads > 16)
+    return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: at most 16 query heads per KV head");
+  if (c->width % 32 != 0 || c->width % 2 != 0)
+    return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: width must be a multiple of 32");
+  if (c->dtype == PAE_W4A16)
+    return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: W4A16 kernels are not built yet");
+  if (c->dtype != PAE_FP32) {
+    const int qd = c->n_q_heads * c->head_dim;
+    if (c->width % 128 || qd % 128 || c->mlp_dim % 128 || (c->n_kv_heads * c->head_dim) % 64)
+      return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: bf16 kernels need width, n_q_heads*head_dim, mlp_dim "
+                                                "multiples of 128");
+    if (c->chunk > 256 || (long long)c->max_batch * c->chunk > 4096)
+      return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: chunk <= 256 and max_batch*chunk <= 4096");
+  }
+  return PAE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out) {
+  if (!out) return fail(nullptr, PAE_ERR_ARG, "out is NULL");
+  *out = nullptr;
+  if (!cfg || !w) return fail(nullptr, PAE_ERR_ARG, "cfg or weights is NULL");
+  pae_status st = validate_config(cfg);
+  if (st != PAE_OK) return st;
+  const void* req[] = {w->w_in, w->b_in, w->w_out, w->b_out, w->w_t1, w->b_t1, w->w_t2, w->b_t2,
+                       w->w_mod, w->b_mod, w->w_modf, w->b_modf, w->w_qkv, w->w_o, w->w_gate, w->w_up, w->w_down};
+  for (const void* p : req)
+    if (!p) return fail(nullptr, PAE_ERR_ARG, "a required weight pointer is NULL");
+  for (int l = 0; l < cfg->layers; ++l)
+    if (!w->w_qkv[l] || !w->w_o[l] || !w->w_gate[l] || !w->w_up[l] || !w->w_down[l])
+      return fail(nullptr, PAE_ERR_ARG, "layer %d weight pointer is NULL", l);
+
+  pae_ctx* ctx = new pae_ctx();
+  ctx->cfg = *cfg;
+  Shape& s = ctx->s;
+  s.L = cfg->layers;
+  s.D = cfg->width;
+  s.Hq = cfg->n_q_heads;
+  s.Hkv = cfg->n_kv_heads;
+  s.d = cfg->head_dim;
+  s.F = cfg->mlp_dim;
+  s.A = cfg->action_dim;
+  s.H = cfg->chunk;
+  s.Bmax = cfg->max_batch;
+  s.Pmax = cfg->max_prefix;
+  s.Ptot = cfg->max_prefix + cfg->chunk;
+  s.G = s.Hq / s.Hkv;
+  s.qkv_rows = (s.Hq + 2 * s.Hkv) * s.d;
+  s.attn_dim = s.Hq * s.d;
+  s.group = cfg->group_size;
+  s.eps = cfg->rms_eps;
+  s.table_rows = (s.L * 2 * 3 + 2) * s.D;
+  ctx->act_bf16 = cfg->dtype != PAE_FP32;
+  ctx->esize = ctx->act_bf16 ? 2 : 4;
+  const size_t es = ctx->esize;
+  ctx->lens_host.assign(s.Bmax, -1);
+
+  auto bail = [&](pae_status code) {
+    g_create_error = ctx->last_error;
+    free_all(ctx);
+    delete ctx;
+    return code;
+  };
+#define CKC(call)                                                                                   \
+  do {                                                                                              \
+    cudaError_t e_ = (call);                                                                        \
+    if (e_ != cudaSuccess) {                                                                        \
+      fail(ctx, PAE_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_));                             \
+      return bail(PAE_ERR_CUDA);                                                                    \
+    }                                                                                               \
+  } while (0)
+#define ALLOC(ptr, bytes)                                                     \
+  do {                                                                        \
+    void* p_ = nullptr;                                                       \
+    if ((st = dev_alloc(ctx, &p_, (bytes))) != PAE_OK) return bail(st);       \
+    ptr = reinterpret_cast<decltype(ptr)>(p_);                                \
+  } while (0)
+
+  CKC(cudaGetDevice(&ctx->device));
+  if (ctx->act_bf16) {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    CKC(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+    if (!fn || q != cudaDriverEntryPointSuccess) {
+      fail(ctx, PAE_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
+      return bail(PAE_ERR_CUDA);
+    }
+    ctx->encode = reinterpret_cast<EncodeTiledFn>(fn);
+    CKC(tc_gemm_init());
+  }
+  CKC(cudaStreamCreateWithFlags(&ctx->cap_stream, cudaStreamNonBlocking));
+  CKC(cudaHostAlloc(reinterpret_cast<void**>(&ctx->err_host), sizeof(int), cudaHostAllocMapped));
+  *ctx->err_host = 0;
+  CKC(cudaHostGetDevicePointer(reinterpret_cast<void**>(&ctx->err_dev), ctx->err_host, 0));
+
+  const int L = s.L, D = s.D, A = s.A, F = s.F;
+  // ---- weights
+  ALLOC(ctx->w_inT, (size_t)D * A * es);
+  ALLOC(ctx->b_in, (size_t)D * es);
+  ALLOC(ctx->w_out, (size_t)A * D * es);
+  ALLOC(ctx->b_out, (size_t)A * es);
+  ALLOC(ctx->w_t1, (size_t)D * D * es);
+  ALLOC(ctx->b_t1, (size_t)D * es);
+  ALLOC(ctx->w_t2, (size_t)D * D * es);
+  ALLOC(ctx->b_t2, (size_t)D * es);
+  ALLOC(ctx->w_modall, (size_t)s.table_rows * D * es);
+  ALLOC(ctx->b_modall, (size_t)s.table_rows * es);
+  ALLOC(ctx->w_qkv, (size_t)L * s.qkv_rows * D * es);
+  ALLOC(ctx->w_o, (size_t)L * D * s.attn_dim * es);
+  ALLOC(ctx->w_gu, (size_t)L * 2 * F * D * es);
+  ALLOC(ctx->w_down, (size_t)L * D * F * es);
+  cudaStream_t cs = ctx->cap_stream;
+  if (ctx->act_bf16)
+    k_transpose<uint16_t><<<64, 256, 0, cs>>>((const uint16_t*)w->w_in, (uint16_t*)ctx->w_inT, D, A);
+  else
+    k_transpose<float><<<64, 256, 0, cs>>>((const float*)w->w_in, (float*)ctx->w_inT, D, A);
+  CKC(cudaGetLastError());
+  CKC(cudaMemcpyAsync(ctx->b_in, w->b_in, (size_t)D * es, cudaMemcpyDeviceToDevice, cs));
+  CKC(cudaMemcpyAsync(ctx->w_out, w->w_out, (size_t)A * D * es, cudaMemcpyDeviceToDevice, cs));
+  CKC(cudaMemcpyAsync(ctx->b_out, w->b_out, (size_t)A * es, cudaMemcpyDeviceToDevice, cs));
+  CKC(cudaMemcpyAsync(ctx->w_t1, w->w_t1, (size_t)D * D * es, cudaMemcpyDeviceToDevice, cs));
+  CKC(cudaMemcpyAsync(ctx->b_t1, w->b_t1, (size_t)D * es, cudaMemcpyDeviceToDevice, cs));
+  CKC(cudaMemcpyAsync(ctx->w_t2, w->w_t2, (size_t)D * D * es, cudaMemcpyDeviceToDevice, cs));
+  CKC(cudaMemcpyAsync(ctx->b_t2, w->b_t2, (size_t)D * es, cudaMemcpyDeviceToDevice, cs));
+  const size_t mod_rows = (size_t)L * 2 * 3 * D;
+  CKC(cudaMemcpyAsync(ctx->w_modall, w->w_mod, mod_rows * D * es, cudaMemcpyDeviceToDevice, cs));
+  CKC(cudaMemcpyAsync((char*)ctx->w_modall + mod_rows * D * es, w->w_modf, (size_t)2 * D * D * es,
+                      cudaMemcpyDeviceToDevice, cs));
+  CKC(cudaMemcpyAsync(ctx->b_modall, w->b_mod, mod_rows * es, cudaMemcpyDeviceToDevice, cs));
+  CKC(cudaMemcpyAsync((char*)ctx->b_modall + mod_rows * es, w->b_modf, (size_t)2 * D * es,
+                      cudaMemcpyDeviceToDevice, cs));
+  for (int l = 0; l < L; ++l) {
+    CKC(cudaMemcpyAsync((char*)ctx->w_qkv + (size_t)l * s.qkv_rows * D * es, w->w_qkv[l],
+                        (size_t)s.qkv_rows * D * es, cudaMemcpyDeviceToDevice, cs));
+    CKC(cudaMemcpyAsync((char*)ctx->w_o + (size_t)l * D * s.attn_dim * es, w->w_o[l], (size_t)D * s.attn_dim * es,
+                        cudaMemcpyDeviceToDevice, cs));
+    CKC(cudaMemcpyAsync((char*)ctx->w_down + (size_t)l * D * F * es, w->w_down[l], (size_t)D * F * es,
+                        cudaMemcpyDeviceToDevice, cs));
+    // gate/up interleaved in 128-row tiles: [gate 128 rows | up 128 rows] per tile
+    char* gu = (char*)ctx->w_gu + (size_t)l * 2 * F * D * es;
+    const size_t tile_bytes = (size_t)128 * D * es;
+    const int full_tiles = F / 128;
+    if (full_tiles > 0) {
+      CKC(cudaMemcpy2DAsync(gu, 2 * tile_bytes, w->w_gate[l], tile_bytes, tile_bytes, full_tiles,
+                            cudaMemcpyDeviceToDevice, cs));
+      CKC(cudaMemcpy2DAsync(gu + tile_bytes, 2 * tile_bytes, w->w_up[l], tile_bytes, tile_bytes, full_tiles,
+                            cudaMemcpyDeviceToDevice, cs));
+    }
+    const int rem = F - full_tiles * 128;  // fp32 mode only (bf16 needs F % 128 == 0)
+    if (rem > 0) {
+      const size_t rb = (size_t)rem * D * es;
+      CKC(cudaMemcpyAsync(gu + full_tiles * 2 * tile_bytes, (const char*)w->w_gate[l] + full_tiles * tile_bytes, rb,
+                          cudaMemcpyDeviceToDevice, cs));
+      CKC(cudaMemcpyAsync(gu + full_tiles * 2 * tile_bytes + tile_bytes,
+                          (const char*)w->w_up[l] + full_tiles * tile_bytes, rb, cudaMemcpyDeviceToDevice, cs));
+    }
+  }
+  // ---- tables, prefix slots, activations
+  ALLOC(ctx->t_dev, sizeof(double) * (kMaxSteps + 1));
+  ALLOC(ctx->emb, sizeof(float) * kMaxSteps * D);
+  ALLOC(ctx->zbuf, sizeof(float) * kMaxSteps * D);
+  ALLOC(ctx->cbuf, sizeof(float) * kMaxSteps * D);
+  ALLOC(ctx->tables, sizeof(float) * kMaxSteps * (size_t)s.table_rows);
+  ALLOC(ctx->dt, sizeof(float) * kMaxSteps);
+  const size_t slot_elems = (size_t)L * s.Bmax * s.Hkv * s.Ptot * s.d;
+  ALLOC(ctx->kc, slot_elems * es);
+  ALLOC(ctx->vc, slot_elems * es);
+  CKC(cudaMemsetAsync(ctx->kc, 0, slot_elems * es, cs));
+  CKC(cudaMemsetAsync(ctx->vc, 0, slot_elems * es, cs));
+  ALLOC(ctx->lens_dev, sizeof(int) * s.Bmax);
+  CKC(cudaMemsetAsync(ctx->lens_dev, 0, sizeof(int) * s.Bmax, cs));
+  const size_t Mmax = (size_t)s.Bmax * s.H;
+  const size_t Mpad = ((Mmax + 255) / 256 + 1) * 256;  // token tiles may pad past Mmax
+  ALLOC(ctx->x, sizeof(float) * Mmax * A);
+  ALLOC(ctx->h, sizeof(float) * Mmax * D);
+  ALLOC(ctx->y, Mpad * D * es);
+  ALLOC(ctx->q, Mmax * s.attn_dim * es);
+  ALLOC(ctx->o, Mpad * s.attn_dim * es);
+  ALLOC(ctx->u, Mpad * F * es);
+  CKC(cudaMemsetAsync(ctx->y, 0, Mpad * D * es, cs));
+  CKC(cudaMemsetAsync(ctx->o, 0, Mpad * s.attn_dim * es, cs));
+  CKC(cudaMemsetAsync(ctx->u, 0, Mpad * F * es, cs));
+  if (ctx->act_bf16) {
+    if ((st = make_map(ctx, &ctx->tmWqkv, ctx->w_qkv, D, (uint64_t)L * s.qkv_rows, 64, 128)) != PAE_OK) return bail(st);
+    if ((st = make_map(ctx, &ctx->tmWo, ctx->w_o, s.attn_dim, (uint64_t)L * D, 64, 128)) != PAE_OK) return bail(st);
+    if ((st = make_map(ctx, &ctx->tmWgu, ctx->w_gu, D, (uint64_t)L * 2 * F, 64, 256)) != PAE_OK) return bail(st);
+    if ((st = make_map(ctx, &ctx->tmWdown, ctx->w_down, F, (uint64_t)L * D, 64, 128)) != PAE_OK) return bail(st);
+    // split-K workspace: the largest any batch size needs
+    size_t pf = 0;
+    int cn = 0;
+    for (int B = 1; B <= s.Bmax; ++B) {
+      Plan P;
+      const int M = B * s.H;
+      P.qkv = plan_gemm(M, s.qkv_rows, D, 1);
+      P.o = plan_gemm(M, D, s.attn_dim, 1);
+      P.gu = plan_gemm(M, F, D, 2);
+      P.down = plan_gemm(M, D, F, 1);
+      pf = std::max(pf, plan_partials(P, s));
+      cn = std::max(cn, plan_counters(P, s));
+    }
+    ctx->partials_floats = pf;
+    ctx->counters_n = cn;
+    ALLOC(ctx->partials, sizeof(float) * std::max<size_t>(pf, 4));
+    ALLOC(ctx->counters, sizeof(int) * std::max(cn, 1));
+    CKC(cudaMemsetAsync(ctx->counters, 0, sizeof(int) * std::max(cn, 1), cs));
+  }
+  CKC(cudaStreamSynchronize(cs));
+  CKC(cudaGetLastError());
+  *out = ctx;
+  return PAE_OK;
+#undef CKC
+#undef ALLOC
+}
+
+pae_status pae_set_prefix(pae_ctx* ctx, int row, const void* const* k_per_layer, const void* const* v_per_layer,
+                          int len, pae_stream stream) {
+  if (!ctx) return fail(nullptr, PAE_ERR_ARG, "ctx is NULL");
+  pae_status st = check_err_word(ctx);
+  if (st != PAE_OK) return st;
+  const Shape& s = ctx->s;
+  if (row < 0 || row >= s.Bmax) return fail(ctx, PAE_ERR_ARG, "row %d out of range [0, %d)", row, s.Bmax);
+  if (len < 0 || len > s.Pmax) return fail(ctx, PAE_ERR_ARG, "len %d out of range [0, %d]", len, s.Pmax);
+  if (len > 0) {
+    if (!k_per_layer || !v_per_layer) return fail(ctx, PAE_ERR_ARG, "k/v pointer arrays are NULL");
+    for (int l = 0; l < s.L; ++l)
+      if (!k_per_layer[l] || !v_per_layer[l]) return fail(ctx, PAE_ERR_ARG, "layer %d k/v pointer is NULL", l);
+  }
+  cudaStream_t stm = reinterpret_cast<cudaStream_t>(stream);
+  const size_t es = ctx->esize;
+  const size_t rowb = (size_t)s.d * es;
+  for (int l = 0; l < s.L && len > 0; ++l) {
+    for (int g = 0; g < s.Hkv; ++g) {
+      const size_t slot = (((size_t)l * s.Bmax + row) * s.Hkv + g) * s.Ptot * s.d * es;
+      const char* ks = static_cast<const char*>(k_per_layer[l]) + g * rowb;
+      const char* vs = static_cast<const char*>(v_per_layer[l]) + g * rowb;
+      CK(cudaMemcpy2DAsync((char*)ctx->kc + slot, rowb, ks, s.Hkv * rowb, rowb, len, cudaMemcpyDeviceToDevice, stm));
+      CK(cudaMemcpy2DAsync((char*)ctx->vc + slot, rowb, vs, s.Hkv * rowb, rowb, len, cudaMemcpyDeviceToDevice, stm));
+    }
+  }
+  k_set_len<<<1, 1, 0, stm>>>(ctx->lens_dev, row, len);
+  CK(cudaGetLastError());
+  ctx->lens_host[row] = len;
+  return PAE_OK;
+}
+
+pae_status pae_precompute_tables(pae_ctx* ctx, const double* t, int K, pae_stream stream) {
+  if (!ctx) return fail(nullptr, PAE_ERR_ARG, "ctx is NULL");
+  pae_status st = check_err_word(ctx);
+  if (st != PAE_OK) return st;
+  if (!t) return fail(ctx, PAE_ERR_ARG, "t is NULL");
+  if (K < 1 || K > kMaxSteps) return fail(ctx, PAE_ERR_ARG, "K = %d out of range [1, %d]", K, kMaxSteps);
+  const double dir = t[1] - t[0];
+  for (int k = 0; k < K; ++k) {
+    const double dk = t[k + 1] - t[k];
+    if (!(dk * dir > 0.0)) return fail(ctx, PAE_ERR_ARG, "t must be strictly monotone (at index %d)", k);
+  }
+  cudaStream_t stm = reinterpret_cast<cudaStream_t>(stream);
+  CK(cudaMemcpyAsync(ctx->t_dev, t, sizeof(double) * (K + 1), cudaMemcpyHostToDevice, stm));
+  launch_time_mlp(ctx->s, ctx->act_bf16, ctx->t_dev, K, ctx->w_t1, ctx->b_t1, ctx->w_t2, ctx->b_t2, ctx->emb,
+                  ctx->zbuf, ctx->cbuf, ctx->dt, stm);
+  launch_mod_tables(ctx->s, ctx->act_bf16, ctx->cbuf, K, ctx->w_modall, ctx->b_modall, ctx->tables, stm);
+  CK(cudaGetLastError());
+  if (K != ctx->K) drop_graphs(ctx);
+  ctx->K = K;
+  ctx->tables_ready = true;
+  return PAE_OK;
+}
+
+static pae_status denoise_common(pae_ctx* ctx, const float* noise, float* out, int batch, pae_stream stream,
+                                 cudaMemcpyKind in_kind, cudaMemcpyKind out_kind) {
+  if (!ctx) return fail(nullptr, PAE_ERR_ARG, "ctx is NULL");
+  pae_status st = check_err_word(ctx);
+  if (st != PAE_OK) return st;
+  if (batch < 0 || batch > ctx->s.Bmax) return fail(ctx, PAE_ERR_ARG, "batch %d out of range [0, %d]", batch, ctx->s.Bmax);
+  if (batch == 0) return PAE_OK;
+  if (!noise || !out) return fail(ctx, PAE_ERR_ARG, "noise or out is NULL");
+  if (!ctx->tables_ready) return fail(ctx, PAE_ERR_STATE, "pae_precompute_tables has not been called");
+  if ((st = check_rows(ctx, batch)) != PAE_OK) return st;
+  Plan* P = nullptr;
+  if ((st = get_plan(ctx, batch, &P)) != PAE_OK) return st;
+  cudaStream_t stm = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bytes = sizeof(float) * (size_t)batch * ctx->s.H * ctx->s.A;
+  CK(cudaMemcpyAsync(ctx->x, noise, bytes, in_kind, stm));
+  if ((st = run_loop(ctx, P, stm)) != PAE_OK) return st;
+  CK(cudaMemcpyAsync(out, ctx->x, bytes, out_kind, stm));
+  return PAE_OK;
+}
+
+pae_status pae_denoise(pae_ctx* ctx, const float* noise, float* out, int batch, pae_stream stream) {
+  return denoise_common(ctx, noise, out, batch, stream, cudaMemcpyDeviceToDevice, cudaMemcpyDeviceToDevice);
+}
+
+pae_status pae_denoise_host(pae_ctx* ctx, const float* noise_host, float* out_host, int batch, pae_stream stream) {
+  return denoise_common(ctx, noise_host, out_host, batch, stream, cudaMemcpyHostToDevice, cudaMemcpyDeviceToHost);
+}
+
+pae_status pae_denoise_steps(pae_ctx* ctx, const float* x_in, float* x_out, int batch, int k_begin, int k_end,
+                             pae_stream stream) {
+  if (!ctx) return fail(nullptr, PAE_ERR_ARG, "ctx is NULL");
+  pae_status st = check_err_word(ctx);
+  if (st != PAE_OK) return st;
+  if (batch < 0 || batch > ctx->s.Bmax) return fail(ctx, PAE_ERR_ARG, "batch %d out of range [0, %d]", batch, ctx->s.Bmax);
+  if (!ctx->tables_ready) return fail(ctx, PAE_ERR_STATE, "pae_precompute_tables has not been called");
+  if (k_begin < 0 || k_end > ctx->K || k_begin >= k_end)
+    return fail(ctx, PAE_ERR_ARG, "step range [%d, %d) invalid for K = %d", k_begin, k_end, ctx->K);
+  if (batch == 0) return PAE_OK;
+  if (!x_in || !x_out) return fail(ctx, PAE_ERR_ARG, "x_in or x_out is NULL");
+  if ((st = check_rows(ctx, batch)) != PAE_OK) return st;
+  Plan* P = nullptr;
+  if ((st = get_plan(ctx, batch, &P)) != PAE_OK) return st;
+  cudaStream_t stm = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bytes = sizeof(float) * (size_t)batch * ctx->s.H * ctx->s.A;
+  if ((st = ensure_events(ctx, k_end - k_begin)) != PAE_OK) return st;
+  CK(cudaMemcpyAsync(ctx->x, x_in, bytes, cudaMemcpyDeviceToDevice, stm));
+  P->recs.clear();
+  ctx->rec_sink = &P->recs;
+  ctx->last_plan = P;
+  enqueue_steps(ctx, *P, k_begin, k_end, stm);
+  ctx->rec_sink = nullptr;
+  CK(cudaGetLastError());
+  CK(cudaMemcpyAsync(x_out, ctx->x, bytes, cudaMemcpyDeviceToDevice, stm));
+  return PAE_OK;
+}
+
+pae_status pae_set_option(pae_ctx* ctx, int option, long long value) {
+  if (!ctx) return fail(nullptr, PAE_ERR_ARG, "ctx is NULL");
+  switch (option) {
+    case PAE_OPT_USE_GRAPH: ctx->use_graph = value != 0; return PAE_OK;
+    case PAE_OPT_WAIT_LIMIT_US:
+      if (value <= 0) return fail(ctx, PAE_ERR_ARG, "wait limit must be positive");
+      ctx->wait_ns = value * 1000LL;
+      drop_graphs(ctx);  // captured launches hold the old limit
+      return PAE_OK;
+    case PAE_OPT_PROFILE:
+      if (value < 0 || value >= (1LL << PAE_K_COUNT)) return fail(ctx, PAE_ERR_ARG, "bad profile mask");
+      if ((unsigned)value != ctx->profile_mask) drop_graphs(ctx);
+      ctx->profile_mask = (unsigned)value;
+      return PAE_OK;
+    default: return fail(ctx, PAE_ERR_ARG, "unknown option %d", option);
+  }
+}
+
+pae_status pae_profile_read(pae_ctx* ctx, int kernel_class, double* total_ms, int* launches) {
+  if (!ctx || !total_ms || !launches) return fail(ctx, PAE_ERR_ARG, "null argument");
+  if (kernel_class < 0 || kernel_class >= PAE_K_COUNT) return fail(ctx, PAE_ERR_ARG, "bad kernel class");
+  *total_ms = 0.0;
+  *launches = 0;
+  if (!ctx->last_plan) return PAE_OK;
+  for (const ProfRec& r : ctx->last_plan->recs) {
+    if (r.kind != kernel_class) continue;
+    float ms = 0.f;
+    CK(cudaEventElapsedTime(&ms, ctx->ev_pool[r.ev0], ctx->ev_pool[r.ev1]));
+    *total_ms += ms;
+    ++*launches;
+  }
+  return PAE_OK;
+}
+
+pae_status pae_query(pae_ctx* ctx, int what, int batch, long long* value) {
+  if (!ctx || !value) return fail(ctx, PAE_ERR_ARG, "null argument");
+  if (batch < 1 || batch > ctx->s.Bmax) return fail(ctx, PAE_ERR_ARG, "batch %d out of range", batch);
+  Plan* P = nullptr;
+  pae_status st = get_plan(ctx, batch, &P);
+  if (st != PAE_OK) return st;
+  switch (what) {
+    case PAE_Q_GRAPH_KERNELS: *value = P->graph ? P->graph_kernels : 0; return PAE_OK;
+    case PAE_Q_SPLITS:
+      *value = (long long)P->qkv.splits | ((long long)P->o.splits << 8) | ((long long)P->gu.splits << 16) |
+               ((long long)P->down.splits << 24);
+      return PAE_OK;
+    case PAE_Q_TOKEN_TILE: *value = P->qkv.tn; return PAE_OK;
+    default: return fail(ctx, PAE_ERR_ARG, "unknown query %d", what);
+  }
+}
+
+pae_status pae_sync(pae_ctx* ctx, pae_stream stream) {
+  if (!ctx) return fail(nullptr, PAE_ERR_ARG, "ctx is NULL");
+  CK(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  CK(cudaGetLastError());
+  return check_err_word(ctx);
+}
+
+void pae_clear_error(pae_ctx* ctx) {
+  if (!ctx) return;
+  cudaDeviceSynchronize();
+  if (ctx->err_host) *(volatile int*)ctx->err_host = 0;
+  if (ctx->counters) cudaMemset(ctx->counters, 0, sizeof(int) * std::max(ctx->counters_n, 1));
+  ctx->last_error.clear();
+}
+
+const char* pae_last_error(const pae_ctx* ctx) {
+  return ctx ? ctx->last_error.c_str() : g_create_error.c_str();
+}
+
+pae_status pae_debug_copy(pae_ctx* ctx, const char* name, void* dst_host, size_t* bytes) {
+  if (!ctx || !name || !bytes) return fail(ctx, PAE_ERR_ARG, "null argument");
+  const Shape& s = ctx->s;
+  const size_t es = ctx->esize;
+  const size_t Mmax = (size_t)s.Bmax * s.H;
+  const void* src = nullptr;
+  size_t n = 0;
+  const std::string nm(name);
+  if (nm == "x") { src = ctx->x; n = sizeof(float) * Mmax * s.A; }
+  else if (nm == "h") { src = ctx->h; n = sizeof(float) * Mmax * s.D; }
+  else if (nm == "y") { src = ctx->y; n = Mmax * s.D * es; }
+  else if (nm == "q") { src = ctx->q; n = Mmax * s.attn_dim * es; }
+  else if (nm == "o") { src = ctx->o; n = Mmax * s.attn_dim * es; }
+  else if (nm == "u") { src = ctx->u; n = Mmax * s.F * es; }
+  else if (nm == "kcache") { src = ctx->kc; n = (size_t)s.L * s.Bmax * s.Hkv * s.Ptot * s.d * es; }
+  else if (nm == "vcache") { src = ctx->vc; n = (size_t)s.L * s.Bmax * s.Hkv * s.Ptot * s.d * es; }
+  else if (nm == "tables") { src = ctx->tables; n = sizeof(float) * (size_t)std::max(ctx->K, 1) * s.table_rows; }
+  else if (nm == "dt") { src = ctx->dt; n = sizeof(float) * std::max(ctx->K, 1); }
+  else if (nm == "lens") { src = ctx->lens_dev; n = sizeof(int) * s.Bmax; }
+  else return fail(ctx, PAE_ERR_ARG, "unknown buffer '%s'", name);
+  if (!dst_host) { *bytes = n; return PAE_OK; }
+  if (*bytes < n) return fail(ctx, PAE_ERR_ARG, "buffer '%s' needs %zu bytes", name, n);
+  CK(cudaDeviceSynchronize());
+  CK(cudaMemcpy(dst_host, src, n, cudaMemcpyDeviceToHost));
+  *bytes = n;
+  return PAE_OK;
+}
+
+void pae_destroy(pae_ctx* ctx) {
+  if (!ctx) return;
+  cudaDeviceSynchronize();
+  free_all(ctx);
+  delete ctx;
+}
+
+}  // extern "C"

@@ -1,0 +1,200 @@
+"""Semantics of the C ABI on the GPU: graph replay, step splitting, prefix
+invalidation, host buffers, determinism, argument and state errors.
+
+These follow the reproduction check the PhyAI reading proposes (Sec. 8.2,
+Check 1): cached-prefix execution and graph replay must give the reference
+result; unchanged-condition repeats must reproduce it; a changed observation
+must change it (no stale-condition output).
+"""
+import numpy as np
+import pytest
+import torch
+
+import flow_matching_action_pi0_b200 as fm
+import workloads as wl
+from tests.helpers import assert_parity, build_expert, oracle_rows, run_gpu, set_prefixes
+
+pytestmark = pytest.mark.gpu
+
+CFG_BF16 = wl.TINY_FP32.replace(name="tiny_bf16_b3", dtype=wl.BF16, batch=3)
+CFG_FP32 = wl.TINY_FP32.replace(name="tiny_fp32_b3", batch=3)
+
+
+@pytest.fixture(params=[CFG_BF16, CFG_FP32], ids=["bf16", "fp32"])
+def setup(request):
+    cfg = request.param
+    ex, W = build_expert(cfg)
+    ks, vs = wl.make_prefix(cfg, lengths=[64, 30, 9])
+    set_prefixes(ex, cfg, ks, vs)
+    grid = wl.uniform_grid(cfg.steps)
+    ex.precompute_tables(grid)
+    noise = wl.make_noise(cfg)
+    yield cfg, ex, W, ks, vs, grid, noise
+    ex.close()
+
+
+def test_graph_replay_equals_direct_launch(setup):
+    cfg, ex, W, ks, vs, grid, noise = setup
+    a = run_gpu(ex, noise)
+    b = run_gpu(ex, noise)           # replay of the captured graph
+    ex.set_option(fm.PAE_OPT_USE_GRAPH, 0)
+    c = run_gpu(ex, noise)
+    ex.set_option(fm.PAE_OPT_USE_GRAPH, 1)
+    np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(a, c)
+
+
+def test_step_split_bitwise(setup):
+    cfg, ex, W, ks, vs, grid, noise = setup
+    full = run_gpu(ex, noise)
+    x = torch.from_numpy(noise).cuda()
+    mid = torch.empty_like(x)
+    end = torch.empty_like(x)
+    ex.denoise_steps(x, mid, 0, 1)
+    ex.denoise_steps(mid, mid, 1, 3)
+    ex.denoise_steps(mid, end, 3, cfg.steps)
+    ex.sync()
+    np.testing.assert_array_equal(end.cpu().numpy(), full)
+
+
+def test_host_buffers_equal_device_buffers(setup):
+    cfg, ex, W, ks, vs, grid, noise = setup
+    dev = run_gpu(ex, noise)
+    nh = torch.from_numpy(noise).pin_memory()
+    oh = torch.empty_like(nh).pin_memory()
+    ex.denoise_host(nh, oh)
+    ex.sync()
+    np.testing.assert_array_equal(oh.numpy(), dev)
+
+
+def test_alias_out_equals_noise(setup):
+    cfg, ex, W, ks, vs, grid, noise = setup
+    ref = run_gpu(ex, noise)
+    x = torch.from_numpy(noise).cuda()
+    ex.denoise(x, out=x)
+    ex.sync()
+    np.testing.assert_array_equal(x.cpu().numpy(), ref)
+
+
+def test_invalidation_changes_only_that_row(setup):
+    cfg, ex, W, ks, vs, grid, noise = setup
+    before = run_gpu(ex, noise)
+    again = run_gpu(ex, noise)                   # cache hit: bitwise repeat
+    np.testing.assert_array_equal(before, again)
+    ks2, vs2 = wl.make_prefix(cfg, lengths=[30], seed=123)
+    set_prefixes(ex, cfg, ks2, vs2, rows=[1])   # new observation for row 1
+    after = run_gpu(ex, noise)
+    np.testing.assert_array_equal(after[0], before[0])
+    np.testing.assert_array_equal(after[2], before[2])
+    assert np.max(np.abs(after[1] - before[1])) > 1e-3
+    ks_new = [ks[0], ks2[0], ks[2]]
+    vs_new = [vs[0], vs2[0], vs[2]]
+    ref = oracle_rows(cfg, W, ks_new, vs_new, noise, grid)
+    assert_parity(after, ref, cfg.dtype, "after invalidation")
+
+
+def test_masked_slot_garbage_has_no_effect(setup):
+    cfg, ex, W, ks, vs, grid, noise = setup
+    ref = run_gpu(ex, noise)
+    # fill row 2's slot far past its length with NaN, then set the real prefix again
+    nan_k = [np.full((cfg.prefix, 1, cfg.head_dim), np.nan, np.float32) for _ in range(cfg.layers)]
+    set_prefixes(ex, cfg, [nan_k], [nan_k], rows=[2])
+    set_prefixes(ex, cfg, [ks[2]], [vs[2]], rows=[2])
+    out = run_gpu(ex, noise)
+    np.testing.assert_array_equal(out, ref)
+
+
+def test_rows_independent_of_batch(setup):
+    cfg, ex, W, ks, vs, grid, noise = setup
+    full = run_gpu(ex, noise)
+    one = run_gpu(ex, noise[:1].copy())          # batch 1 uses rows < 1 only
+    assert_parity(one[0], full[0], cfg.dtype, "row 0 alone vs in batch")
+
+
+def test_tables_rebuild_same_k_keeps_graph_and_new_grid_changes_result(setup):
+    cfg, ex, W, ks, vs, grid, noise = setup
+    a = run_gpu(ex, noise)
+    ex.precompute_tables([1.0, 0.6, 0.3, 0.1, 0.0])
+    b = run_gpu(ex, noise)
+    ref = oracle_rows(cfg, W, ks, vs, noise, [1.0, 0.6, 0.3, 0.1, 0.0])
+    assert_parity(b, ref, cfg.dtype, "non-uniform grid")
+    assert np.max(np.abs(a - b)) > 1e-4
+    ex.precompute_tables(wl.uniform_grid(2))        # different K: graph re-captured
+    c = run_gpu(ex, noise)
+    ref2 = oracle_rows(cfg, W, ks, vs, noise, wl.uniform_grid(2))
+    assert_parity(c, ref2, cfg.dtype, "K=2")
+
+
+def test_state_and_argument_errors():
+    cfg = CFG_BF16
+    ex, W = build_expert(cfg)
+    try:
+        x = torch.from_numpy(wl.make_noise(cfg)).cuda()
+        with pytest.raises(fm.PaeError) as e:
+            ex.denoise(x)                          # no tables yet
+        assert e.value.status == fm.PAE_ERR_STATE
+        ex.precompute_tables(wl.uniform_grid(cfg.steps))
+        with pytest.raises(fm.PaeError) as e:
+            ex.denoise(x)                          # rows never set
+        assert e.value.status == fm.PAE_ERR_STATE
+        with pytest.raises(fm.PaeError) as e:
+            fm.pae_denoise(ex.ctx, x.data_ptr(), x.data_ptr(), cfg.batch + 1)
+        assert e.value.status == fm.PAE_ERR_ARG
+        ks, vs = wl.make_prefix(cfg, lengths=[3])
+        with pytest.raises(fm.PaeError) as e:
+            fm.pae_set_prefix(ex.ctx, 0, [0] * cfg.layers, [0] * cfg.layers, cfg.prefix + 1)
+        assert e.value.status == fm.PAE_ERR_ARG
+        with pytest.raises(fm.PaeError) as e:
+            fm.pae_set_prefix(ex.ctx, cfg.batch, [0] * cfg.layers, [0] * cfg.layers, 0)
+        assert e.value.status == fm.PAE_ERR_ARG
+        with pytest.raises(fm.PaeError) as e:
+            ex.precompute_tables([1.0, 0.5, 0.7])  # not monotone
+        assert e.value.status == fm.PAE_ERR_ARG
+        with pytest.raises(fm.PaeError) as e:
+            ex.precompute_tables([1.0])            # K = 0
+        assert e.value.status == fm.PAE_ERR_ARG
+        # batch 0 is a no-op
+        fm.pae_denoise(ex.ctx, x.data_ptr(), x.data_ptr(), 0)
+        # empty prefixes are valid
+        for b in range(cfg.batch):
+            fm.pae_set_prefix(ex.ctx, b, [], [], 0)
+        out = run_gpu(ex, wl.make_noise(cfg))
+        assert np.all(np.isfinite(out))
+    finally:
+        ex.close()
+
+
+def test_device_wait_timeout_reports_status():
+    """A device-side bounded wait that runs out returns PAE_ERR_TIMEOUT and
+    leaves the context usable after pae_clear_error.  The limit is set to
+    1 microsecond so the tensor-core kernels' first mbarrier waits expire; every
+    wait ends, and the kernels drain their copies and free TMEM before
+    returning."""
+    cfg = wl.TINY_FP32.replace(name="tiny_bf16_to", dtype=wl.BF16)
+    ex, W = build_expert(cfg)
+    try:
+        ks, vs = wl.make_prefix(cfg)
+        set_prefixes(ex, cfg, ks, vs)
+        grid = wl.uniform_grid(cfg.steps)
+        ex.precompute_tables(grid)
+        noise = wl.make_noise(cfg)
+        good = run_gpu(ex, noise)
+        ex.set_option(fm.PAE_OPT_WAIT_LIMIT_US, 1)
+        hit = False
+        for _ in range(20):
+            x = torch.from_numpy(noise).cuda()
+            try:
+                ex.denoise(x)
+                ex.sync()
+            except fm.PaeError as e:
+                assert e.status == fm.PAE_ERR_TIMEOUT
+                hit = True
+                break
+        fm.pae_clear_error(ex.ctx)
+        ex.set_option(fm.PAE_OPT_WAIT_LIMIT_US, 2_000_000)
+        again = run_gpu(ex, noise)
+        np.testing.assert_array_equal(again, good)
+        if not hit:
+            pytest.skip("no wait ran out at a 1 us limit on this run")
+    finally:
+        ex.close()

@@ -1,0 +1,73 @@
+"""GPU-vs-oracle parity on the same seeded inputs, through the C ABI.
+
+Small configs are compared element by element on every output; the full-size
+pi0.5-shaped configs on every output (batch 1) or on sampled rows that the
+oracle computes one by one (batch 32, ragged batch 16), in the same launch
+configuration the benchmark times (captured graph, same batch size).
+"""
+import numpy as np
+import pytest
+
+import workloads as wl
+from tests.helpers import assert_parity, build_expert, oracle_rows, run_gpu, set_prefixes
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_case(cfg, rows=None, lengths=None, max_batch=None):
+    ex, W = build_expert(cfg, max_batch=max_batch)
+    try:
+        ks, vs = wl.make_prefix(cfg, lengths=lengths)
+        set_prefixes(ex, cfg, ks, vs)
+        grid = wl.uniform_grid(cfg.steps)
+        ex.precompute_tables(grid)
+        noise = wl.make_noise(cfg)
+        out = run_gpu(ex, noise)
+        ref = oracle_rows(cfg, W, ks, vs, noise, grid, rows=rows)
+        got = out if rows is None else out[rows]
+        return assert_parity(got, ref, cfg.dtype, cfg.name)
+    finally:
+        ex.close()
+
+
+def test_tiny_fp32():
+    _run_case(wl.TINY_FP32)
+
+
+def test_tiny_bf16():
+    _run_case(wl.TINY_FP32.replace(name="tiny_bf16", dtype=wl.BF16))
+
+
+def test_tiny_bf16_ragged_batch():
+    # several tiles' worth of rows, ragged lengths including an empty prefix
+    cfg = wl.TINY_FP32.replace(name="tiny_bf16_b5", dtype=wl.BF16, batch=5)
+    _run_case(cfg, lengths=[64, 0, 17, 63, 1])
+
+
+def test_tiny_fp32_ragged_batch():
+    cfg = wl.TINY_FP32.replace(name="tiny_fp32_b3", batch=3)
+    _run_case(cfg, lengths=[5, 64, 0])
+
+
+def test_tiny_bf16_gqa2_many_tokens():
+    # Hkv = 2, 300 tokens (two token tiles with a ragged tail)
+    cfg = wl.TINY_FP32.replace(name="tiny_bf16_gqa2", dtype=wl.BF16, n_kv_heads=2, batch=20, chunk=15)
+    _run_case(cfg, lengths=[(7 * b) % 65 for b in range(20)])
+
+
+@pytest.mark.slow
+def test_pi05_bf16_bs1():
+    _run_case(wl.PI05_BF16_BS1)
+
+
+@pytest.mark.slow
+def test_pi05_bf16_bs32_sampled_rows():
+    _run_case(wl.PI05_BF16_BS32, rows=[0, 13, 31])
+
+
+@pytest.mark.slow
+def test_ragged_bf16_bs16_sampled_rows():
+    cfg = wl.RAGGED_BF16_BS16
+    lens = wl.prefix_lengths(cfg)
+    rows = [int(np.argmin(lens)), int(np.argmax(lens)), 7]
+    _run_case(cfg, rows=rows)

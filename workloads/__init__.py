@@ -87,11 +87,13 @@ def rng(seed: int) -> np.random.Generator:
 
 def round_bf16(a: np.ndarray) -> np.ndarray:
     """Round float values to the nearest bf16 (ties to even); returns float32."""
-    a32 = np.ascontiguousarray(a, dtype=np.float32)
-    u = a32.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    u = ((u + 0x7FFF + lsb) >> 16) << 16
-    return u.astype(np.uint32).view(np.float32)
+    a32 = np.array(a, dtype=np.float32, copy=True, order="C")
+    u = a32.view(np.uint32)          # finite inputs: the add cannot wrap
+    lsb = (u >> 16) & np.uint32(1)
+    u += np.uint32(0x7FFF)
+    u += lsb
+    u &= np.uint32(0xFFFF0000)
+    return a32
 
 
 def bf16_bits(a: np.ndarray) -> np.ndarray:
