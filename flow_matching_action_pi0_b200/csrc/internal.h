@@ -110,4 +110,25 @@ void launch_tc_gemm(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* t
 size_t tc_gemm_smem_bytes(int na, const TcPlan& p);
 cudaError_t tc_gemm_init();  // once per process: opt in to large dynamic shared memory
 
+// ------------------------------------------------------ tcgen05 attention
+struct AttnPlan {
+  int qtiles;          // ceil(G*H / 128) query tiles per (request, KV head)
+  int splits;          // key splits (split-KV)
+  int keys_per_split;  // multiple of 64
+};
+struct AttnArgs {
+  const int* lens;
+  int layer;
+  int keys_per_split;
+  void* o;             // [M][Hq d] bf16, token-major
+  float* part_o;       // [units][splits][128][d] partial outputs (splits > 1)
+  float* part_ml;      // [units][splits][128][2] row max (log2 domain), row sum
+  int* counters;       // [units]
+  DevErr err;
+};
+size_t attn_tc_smem_bytes(int d);
+cudaError_t attn_tc_init();
+void launch_attn_tc(const Shape& s, const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                    const AttnPlan& p, const AttnArgs& a, int B, cudaStream_t st);
+
 }  // namespace pae

@@ -1,0 +1,413 @@
+// GQA attention over [cached prefix | action keys] on the tcgen05 tensor cores.
+//
+// For request b and KV head g, the G query heads x H action tokens that read
+// that KV head form G*H query rows (row r = head-in-group * H + token); they
+// share every K and V tile, so they are one M dimension of 128-row tiles.
+// Keys are the row's slot: prefix positions [0, lens[b]) then this step's H
+// action keys at [lens[b], lens[b] + H) (written by the QKV epilogue).  The mask
+// reading: every action token sees all valid prefix keys and all H action
+// keys; keys past lens[b] + H are masked.
+//
+// One CTA = (b, g, 128-row query tile, key split).  Per 64-key chunk c:
+//   MMA warp   S_c = Q K_c^T  (M=128, N=64, K=head_dim; TMEM, double buffered)
+//   4 warps    online softmax on S_c (thread = query row, log2 domain),
+//              rescale O in TMEM when the row max grows, write P_c (bf16,
+//              128-byte swizzled K-major) to shared memory
+//   MMA warp   O += P_c V_c   (M=128, N=head_dim, K=64; V read MN-major)
+// Warps 0-3 run the softmax and the output (thread = query row = TMEM lane);
+// warp 4 is the TMA producer (Q once, K/V chunks through a 2-stage ring);
+// warp 5 issues the MMAs.
+// Key splits (split-KV, for small batches) write unnormalised partial O with
+// the row max and sum; the last CTA of a (b, g, tile) to finish merges them in
+// split order, so the result does not depend on arrival order.
+#include "internal.h"
+
+namespace pae {
+
+namespace {
+
+constexpr int CK = 64;          // keys per chunk
+constexpr int QROWS = 128;      // query rows per CTA
+constexpr long long kDrainNs = 4000000000LL;
+
+struct AttnSmem {
+  uint32_t q_off, k_off[2], v_off[2], p_off, bar_off, total;
+};
+
+__host__ __device__ inline AttnSmem attn_layout(int d) {
+  AttnSmem L;
+  const uint32_t qbytes = QROWS * d * 2;   // d/64 boxes of [128][64]
+  const uint32_t kvbytes = CK * d * 2;     // d/64 boxes of [64][64]
+  L.q_off = 0;
+  L.k_off[0] = qbytes;
+  L.v_off[0] = L.k_off[0] + kvbytes;
+  L.k_off[1] = L.v_off[0] + kvbytes;
+  L.v_off[1] = L.k_off[1] + kvbytes;
+  L.p_off = L.v_off[1] + kvbytes;          // [128][64] bf16
+  L.bar_off = L.p_off + QROWS * CK * 2;
+  L.total = L.bar_off + 256 + 1024;
+  return L;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  const uint32_t lo = __bfloat16_as_ushort(f2bf(a));
+  const uint32_t hi = __bfloat16_as_ushort(f2bf(b));
+  return lo | (hi << 16);
+}
+
+// AND-reduction over the first `n` threads (named barrier `id`).
+__device__ __forceinline__ bool named_and(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__host__ __device__ inline uint32_t attn_tmem_cols(int d) {
+  uint32_t c = 32;
+  while ((int)c < 2 * CK + d) c <<= 1;
+  return c;
+}
+
+__global__ void __launch_bounds__(192, 1)
+    k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const Shape s, const AttnArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int d = s.d;
+  const int nbox = d / 64;
+  const AttnSmem L = attn_layout(d);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;   // [2]
+  uint64_t* v_full = bars + 3;   // [2]
+  uint64_t* kv_empty = bars + 5; // [2]
+  uint64_t* s_full = bars + 7;   // [2]
+  uint64_t* p_full = bars + 9;
+  uint64_t* o_done = bars + 10;
+  uint64_t* drain = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);  // [0] abort [1] last
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = blockIdx.x, split = blockIdx.y, bg = blockIdx.z;
+  const int b = bg / s.Hkv, g = bg - b * s.Hkv;
+  const int GH = s.G * s.H;
+  const int n_valid = a.lens[b] + s.H;
+  const int kps = a.keys_per_split;
+  const int start = split * kps;
+  const int end = min(n_valid, start + kps);
+  const int nch = end > start ? (end - start + CK - 1) / CK : 0;
+  const int slot_row0 = ((a.layer * s.Bmax + b) * s.Hkv + g) * s.Ptot;
+  const float scale_log2 = rsqrtf((float)d) * 1.4426950408889634f;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 12; ++i) mbar_init(&bars[i], i == 9 ? 128 : 1);
+    s_flag[0] = 0;
+    s_flag[1] = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  const uint32_t ncols = attn_tmem_cols(d);
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, ncols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_s[2] = {tmem, tmem + CK};
+  const uint32_t t_o = tmem + 2 * CK;
+
+  // ------------------------------------------------------------ producer (warp 4)
+  if (warp == 4 && lane == 0 && nch > 0) {
+    const uint32_t kvbytes = CK * d * 2;
+    mbar_arrive_expect_tx(q_full, QROWS * d * 2);
+    const int qrow0 = bg * GH + qt * QROWS;
+    for (int x = 0; x < nbox; ++x) tma_load_2d(smem + L.q_off + x * QROWS * 128, &tmQ, x * 64, qrow0, q_full);
+    int issued = 0;
+    for (int c = 0; c < nch; ++c) {
+      const int st = c & 1;
+      if (c >= 2 && !mbar_wait(&kv_empty[st], ((c >> 1) & 1) ^ 1, a.err.wait_ns)) {
+        s_flag[0] = 1;
+        set_error(a.err, DEV_TIMEOUT);
+        break;
+      }
+      const int krow = slot_row0 + start + c * CK;
+      mbar_arrive_expect_tx(&k_full[st], kvbytes);
+      for (int x = 0; x < nbox; ++x) tma_load_2d(smem + L.k_off[st] + x * CK * 128, &tmK, x * 64, krow, &k_full[st]);
+      mbar_arrive_expect_tx(&v_full[st], kvbytes);
+      for (int x = 0; x < nbox; ++x) tma_load_2d(smem + L.v_off[st] + x * CK * 128, &tmV, x * 64, krow, &v_full[st]);
+      issued = c + 1;
+    }
+    if (!mbar_wait(q_full, 0, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
+    for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c) {
+      if (!mbar_wait(&k_full[c & 1], (c >> 1) & 1, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
+      if (!mbar_wait(&v_full[c & 1], (c >> 1) & 1, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
+    }
+  }
+
+  // ------------------------------------------------------------ MMA (warp 5)
+  if (warp == 5 && lane == 0 && nch > 0) {
+    const uint32_t idesc_s = idesc_bf16(QROWS, CK);
+    const uint32_t idesc_o = idesc_bf16(QROWS, d, 0, 1);
+    const uint32_t q_base = smem_u32(smem + L.q_off);
+    const uint32_t p_base = smem_u32(smem + L.p_off);
+    bool good = mbar_wait(q_full, 0, a.err.wait_ns);
+    auto issue_s = [&](int c) -> bool {
+      const int st = c & 1;
+      if (!mbar_wait(&k_full[st], (c >> 1) & 1, a.err.wait_ns)) return false;
+      tc_fence_after();
+      const uint32_t kb = smem_u32(smem + L.k_off[st]);
+      for (int k16 = 0; k16 < d / 16; ++k16) {
+        const int x = k16 >> 2, w = (k16 & 3) * 32;
+        const uint64_t ad = sw128_desc(q_base + x * QROWS * 128 + w, 16, 1024);
+        const uint64_t bd = sw128_desc(kb + x * CK * 128 + w, 16, 1024);
+        umma_bf16(t_s[st], ad, bd, idesc_s, k16 > 0 ? 1u : 0u);
+      }
+      umma_commit(&s_full[st]);
+      return true;
+    };
+    if (good) good = issue_s(0);
+    if (good && nch > 1) good = issue_s(1);
+    for (int c = 0; good && c < nch; ++c) {
+      const int st = c & 1;
+      if (!mbar_wait(p_full, c & 1, a.err.wait_ns) || !mbar_wait(&v_full[st], (c >> 1) & 1, a.err.wait_ns)) {
+        good = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t vb = smem_u32(smem + L.v_off[st]);
+      for (int k16 = 0; k16 < CK / 16; ++k16) {
+        const uint64_t ad = sw128_desc(p_base + k16 * 32, 16, 1024);
+        const uint64_t bd = sw128_desc(vb + k16 * 16 * 128, CK * 128, 1024);
+        umma_bf16(t_o, ad, bd, idesc_o, (c > 0 || k16 > 0) ? 1u : 0u);
+      }
+      umma_commit(o_done);
+      umma_commit(&kv_empty[st]);
+      if (c + 2 < nch) good = issue_s(c + 2);
+    }
+    if (!good) {
+      s_flag[0] = 1;
+      set_error(a.err, DEV_TIMEOUT);
+    }
+    // every MMA this thread issued must finish before TMEM is freed
+    umma_commit(drain);
+    if (!mbar_wait(drain, 0, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
+  }
+  __syncwarp();
+
+  // ------------------------------------------------------------ softmax (warps 0-3)
+  if (warp < 4) {
+  const int r = warp * 32 + lane;  // query row within the tile (TMEM lane)
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  float m_run = -INFINITY, l_run = 0.f;
+  bool ok = true;
+  const uint32_t p_row = smem_u32(smem + L.p_off) + r * 128;
+  for (int c = 0; c < nch; ++c) {
+    const int st = c & 1;
+    const bool w1 = mbar_wait(&s_full[st], (c >> 1) & 1, a.err.wait_ns);
+    if (!__all_sync(0xffffffffu, w1) || s_flag[0]) {  // warp-uniform: the TMEM loads are collective
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    float sv[CK];
+#pragma unroll
+    for (int j = 0; j < CK; j += 16) tmem_ld16(t_s[st] + lane_off + j, sv + j);
+    tmem_ld_wait();
+    const int vc = min(CK, end - (start + c * CK));
+    float mx = m_run;
+#pragma unroll
+    for (int j = 0; j < CK; ++j) {
+      sv[j] = j < vc ? sv[j] * scale_log2 : -INFINITY;
+      mx = fmaxf(mx, sv[j]);
+    }
+    const float alpha = exp2f(m_run - mx);  // m_run = -inf on the first chunk -> 0
+    float psum = 0.f;
+#pragma unroll
+    for (int j = 0; j < CK; ++j) {
+      sv[j] = exp2f(sv[j] - mx);
+      psum += sv[j];
+    }
+    l_run = l_run * alpha + psum;
+    m_run = mx;
+    if (c > 0) {
+      // PV of the previous chunk must be done before O is rescaled and P reused.
+      const bool w2 = mbar_wait(o_done, (c - 1) & 1, a.err.wait_ns);
+      if (!__all_sync(0xffffffffu, w2)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, alpha < 1.f)) {
+        for (int j = 0; j < 256 && j < d; j += 16) {
+          float ov[16];
+          tmem_ld16(t_o + lane_off + j, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int t = 0; t < 16; ++t) ov[t] *= alpha;
+          tmem_st16(t_o + lane_off + j, ov);
+        }
+        tmem_st_wait();
+      }
+    }
+    // P row: 64 bf16 = 8 chunks of 16 bytes, chunk index XOR (row % 8)
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+      const uint32_t addr = p_row + (((uint32_t)ch ^ (uint32_t)(r & 7)) << 4);
+      st_shared_v4(addr, pack_bf16x2(sv[ch * 8 + 0], sv[ch * 8 + 1]), pack_bf16x2(sv[ch * 8 + 2], sv[ch * 8 + 3]),
+                   pack_bf16x2(sv[ch * 8 + 4], sv[ch * 8 + 5]), pack_bf16x2(sv[ch * 8 + 6], sv[ch * 8 + 7]));
+    }
+    if (vc < CK) {
+      // Masked keys have P = 0, but 0 * (NaN or Inf) in V would still poison O:
+      // zero the V rows past the valid keys once their load has landed.
+      const bool w3 = mbar_wait(&v_full[st], (c >> 1) & 1, kDrainNs);
+      if (w3) {
+        uint8_t* vbase = smem + L.v_off[st];
+        const int rows = CK - vc;
+        for (int i = r; i < rows * nbox * 8; i += 128) {
+          const int rr = vc + i / (nbox * 8), rem = i % (nbox * 8), x = rem / 8, ch = rem % 8;
+          *reinterpret_cast<uint4*>(vbase + x * CK * 128 + rr * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+        }
+      } else {
+        set_error(a.err, DEV_TIMEOUT);
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    mbar_arrive(p_full);
+  }
+  if (!ok) set_error(a.err, DEV_TIMEOUT);
+  if (nch > 0 && ok) ok = mbar_wait(o_done, (nch - 1) & 1, kDrainNs);
+  ok = named_and(1, 128, ok) && s_flag[0] == 0;  // CTA-uniform among the 128 softmax threads
+  tc_fence_after();
+
+  // ------------------------------------------------------------ output
+  const int nsplit = gridDim.y;
+  const bool row_valid = qt * QROWS + r < GH;
+  const int rq = qt * QROWS + r;
+  const int hl = rq / s.H, ti = rq - hl * s.H;
+  bf16* orow = reinterpret_cast<bf16*>(a.o) + (size_t)(b * s.H + ti) * s.attn_dim + (g * s.G + hl) * d;
+  if (ok && nsplit == 1) {
+    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+    for (int j = 0; j < d; j += 16) {
+      float ov[16];
+      tmem_ld16(t_o + lane_off + j, ov);
+      tmem_ld_wait();
+      if (row_valid && nch > 0) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) pk[t] = pack_bf16x2(ov[2 * t] * inv, ov[2 * t + 1] * inv);
+        uint4* dst = reinterpret_cast<uint4*>(orow + j);
+        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      }
+    }
+  } else if (ok) {
+    // partial: O (unnormalised), row max (log2 domain) and row sum
+    const size_t unit = (size_t)bg * gridDim.x + qt;
+    float* po = a.part_o + ((unit * nsplit + split) * QROWS + r) * (size_t)d;
+    float* pml = a.part_ml + ((unit * nsplit + split) * QROWS + r) * 2;
+    for (int j = 0; j < d; j += 16) {
+      float ov[16];
+      if (nch > 0) {
+        tmem_ld16(t_o + lane_off + j, ov);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int t = 0; t < 16; ++t) ov[t] = 0.f;
+      }
+#pragma unroll
+      for (int t = 0; t < 16; t += 4)
+        *reinterpret_cast<float4*>(po + j + t) = make_float4(ov[t], ov[t + 1], ov[t + 2], ov[t + 3]);
+    }
+    pml[0] = nch > 0 ? m_run : -INFINITY;
+    pml[1] = nch > 0 ? l_run : 0.f;
+    __threadfence();
+    named_sync(2, 128);
+    if (threadIdx.x == 0) {
+      int* ctr = a.counters + unit;
+      const int prev = atomicAdd(ctr, 1);
+      const int last = prev == nsplit - 1;
+      s_flag[1] = last;
+      if (last) *ctr = 0;
+    }
+    named_sync(2, 128);
+    if (s_flag[1] && row_valid) {
+      __threadfence();
+      const float* pm0 = a.part_ml + ((unit * nsplit) * QROWS + r) * 2;
+      float M = -INFINITY;
+      for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, __ldcg(pm0 + (size_t)sp * QROWS * 2));
+      float wsum = 0.f;
+      for (int sp = 0; sp < nsplit; ++sp) {
+        const float m_s = __ldcg(pm0 + (size_t)sp * QROWS * 2);
+        const float l_s = __ldcg(pm0 + (size_t)sp * QROWS * 2 + 1);
+        wsum += (l_s > 0.f) ? l_s * exp2f(m_s - M) : 0.f;
+      }
+      const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+      const float* po0 = a.part_o + ((unit * nsplit) * QROWS + r) * (size_t)d;
+      for (int j = 0; j < d; j += 8) {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int sp = 0; sp < nsplit; ++sp) {
+          const float m_s = __ldcg(pm0 + (size_t)sp * QROWS * 2);
+          const float l_s = __ldcg(pm0 + (size_t)sp * QROWS * 2 + 1);
+          if (!(l_s > 0.f)) continue;
+          const float wgt = exp2f(m_s - M);
+          const float* src = po0 + (size_t)sp * QROWS * d + j;
+          const float4 x0 = __ldcg(reinterpret_cast<const float4*>(src));
+          const float4 x1 = __ldcg(reinterpret_cast<const float4*>(src + 4));
+          acc[0] = fmaf(wgt, x0.x, acc[0]);
+          acc[1] = fmaf(wgt, x0.y, acc[1]);
+          acc[2] = fmaf(wgt, x0.z, acc[2]);
+          acc[3] = fmaf(wgt, x0.w, acc[3]);
+          acc[4] = fmaf(wgt, x1.x, acc[4]);
+          acc[5] = fmaf(wgt, x1.y, acc[5]);
+          acc[6] = fmaf(wgt, x1.z, acc[6]);
+          acc[7] = fmaf(wgt, x1.w, acc[7]);
+        }
+        *reinterpret_cast<uint4*>(orow + j) =
+            make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
+                       pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
+      }
+    }
+  }
+
+  }  // warps 0-3
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, ncols);
+}
+
+}  // namespace
+
+size_t attn_tc_smem_bytes(int d) { return attn_layout(d).total; }
+
+cudaError_t attn_tc_init() {
+  return cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+}
+
+void launch_attn_tc(const Shape& s, const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                    const AttnPlan& p, const AttnArgs& a, int B, cudaStream_t st) {
+  dim3 grid(p.qtiles, p.splits, B * s.Hkv);
+  k_attn_tc<<<grid, 192, attn_tc_smem_bytes(s.d), st>>>(*tmQ, *tmK, *tmV, s, a);
+}
+
+}  // namespace pae

@@ -41,6 +41,7 @@ struct ProfRec {
 struct Plan {
   int B = 0, M = 0;
   TcPlan qkv{}, o{}, gu{}, down{};
+  AttnPlan attn{};
   CUtensorMap tmY{}, tmO{}, tmU{};
   cudaGraphExec_t graph = nullptr;
   int graph_K = 0;
@@ -75,6 +76,7 @@ struct pae_ctx {
   void *w_modall = nullptr, *b_modall = nullptr;
   void *w_qkv = nullptr, *w_o = nullptr, *w_gu = nullptr, *w_down = nullptr;  // stacked over layers
   CUtensorMap tmWqkv{}, tmWo{}, tmWgu{}, tmWdown{};
+  CUtensorMap tmQ{}, tmK{}, tmV{};  // attention operands (bf16 modes)
   // tables
   double* t_dev = nullptr;
   float *emb = nullptr, *zbuf = nullptr, *cbuf = nullptr, *tables = nullptr, *dt = nullptr;
@@ -91,6 +93,9 @@ struct pae_ctx {
   size_t partials_floats = 0;
   int* counters = nullptr;
   int counters_n = 0;
+  float *attn_part_o = nullptr, *attn_part_ml = nullptr;
+  int* attn_counters = nullptr;
+  int attn_counters_n = 0;
   // error word (host-mapped)
   int* err_host = nullptr;
   int* err_dev = nullptr;
@@ -185,6 +190,19 @@ TcPlan plan_gemm(int M, int nfeat, int K, int na) {
   return p;
 }
 
+// Query tiles of 128 rows per (request, KV head); key splits only when the
+// batch gives too few tiles to fill the 148 SMs (split-KV at small batch).
+AttnPlan plan_attn(const Shape& s, int B) {
+  AttnPlan p{};
+  p.qtiles = (s.G * s.H + 127) / 128;
+  const int base = B * s.Hkv * p.qtiles;
+  const int max_splits = (s.Ptot + 63) / 64;
+  int splits = base * 4 >= 3 * 148 ? 1 : std::max(1, std::min(max_splits, 148 / base));
+  p.keys_per_split = ((s.Ptot + splits - 1) / splits + 63) / 64 * 64;
+  p.splits = (s.Ptot + p.keys_per_split - 1) / p.keys_per_split;
+  return p;
+}
+
 pae_status build_plan(pae_ctx* ctx, int B, Plan* P) {
   const Shape& s = ctx->s;
   P->B = B;
@@ -194,6 +212,7 @@ pae_status build_plan(pae_ctx* ctx, int B, Plan* P) {
   P->o = plan_gemm(P->M, s.D, s.attn_dim, 1);
   P->gu = plan_gemm(P->M, s.F, s.D, 2);
   P->down = plan_gemm(P->M, s.D, s.F, 1);
+  P->attn = plan_attn(s, B);
   const uint64_t Mmax = (uint64_t)s.Bmax * s.H;
   pae_status st;
   if ((st = make_map(ctx, &P->tmY, ctx->y, s.D, Mmax, 64, P->qkv.tn)) != PAE_OK) return st;
@@ -226,13 +245,23 @@ struct ProfScope {
       if (ctx->ev_next + 2 <= (int)ctx->ev_pool.size() && ctx->rec_sink) {
         ev0 = ctx->ev_next;
         ctx->ev_next += 2;
-        cudaEventRecord(ctx->ev_pool[ev0], st);
+        record(ctx->ev_pool[ev0]);
       }
     }
   }
+  // Inside stream capture an event becomes a graph node only when recorded
+  // as an external event.
+  void record(cudaEvent_t e) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(st, &cs);
+    if (cs == cudaStreamCaptureStatusActive)
+      cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+    else
+      cudaEventRecord(e, st);
+  }
   ~ProfScope() {
     if (ev0 >= 0) {
-      cudaEventRecord(ctx->ev_pool[ev0 + 1], st);
+      record(ctx->ev_pool[ev0 + 1]);
       ctx->rec_sink->push_back(ProfRec{kind, ev0, ev0 + 1});
     }
   }
@@ -326,7 +355,20 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
       }
       {
         ProfScope ps(ctx, PAE_K_ATTENTION, st);
-        launch_attention_simple(s, ctx->act_bf16, ctx->q, ctx->kc, ctx->vc, ctx->lens_dev, l, ctx->o, P.B, st);
+        if (ctx->act_bf16) {
+          AttnArgs aa{};
+          aa.lens = ctx->lens_dev;
+          aa.layer = l;
+          aa.keys_per_split = P.attn.keys_per_split;
+          aa.o = ctx->o;
+          aa.part_o = ctx->attn_part_o;
+          aa.part_ml = ctx->attn_part_ml;
+          aa.counters = ctx->attn_counters;
+          aa.err = DevErr{ctx->err_dev, ctx->wait_ns};
+          launch_attn_tc(s, &ctx->tmQ, &ctx->tmK, &ctx->tmV, P.attn, aa, P.B, st);
+        } else {
+          launch_attention_simple(s, ctx->act_bf16, ctx->q, ctx->kc, ctx->vc, ctx->lens_dev, l, ctx->o, P.B, st);
+        }
       }
       e = EpiArgs{};
       e.M = M;
@@ -485,6 +527,8 @@ pae_status validate_config(const pae_config* c) {
     if (c->width % 128 || qd % 128 || c->mlp_dim % 128 || (c->n_kv_heads * c->head_dim) % 64)
       return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: bf16 kernels need width, n_q_heads*head_dim, mlp_dim "
                                                 "multiples of 128");
+    if (c->head_dim != 64 && c->head_dim != 128 && c->head_dim != 256)
+      return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: bf16 attention needs head_dim 64, 128 or 256");
     if (c->chunk > 256 || (long long)c->max_batch * c->chunk > 4096)
       return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: chunk <= 256 and max_batch*chunk <= 4096");
   }
@@ -664,6 +708,24 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
     if ((st = make_map(ctx, &ctx->tmWo, ctx->w_o, s.attn_dim, (uint64_t)L * D, 64, 128)) != PAE_OK) return bail(st);
     if ((st = make_map(ctx, &ctx->tmWgu, ctx->w_gu, D, (uint64_t)L * 2 * F, 64, 256)) != PAE_OK) return bail(st);
     if ((st = make_map(ctx, &ctx->tmWdown, ctx->w_down, F, (uint64_t)L * D, 64, 128)) != PAE_OK) return bail(st);
+    CKC(attn_tc_init());
+    const uint64_t kv_rows = (uint64_t)L * s.Bmax * s.Hkv * s.Ptot;
+    if ((st = make_map(ctx, &ctx->tmQ, ctx->q, s.d, (uint64_t)s.Bmax * s.Hq * s.H, 64, 128)) != PAE_OK) return bail(st);
+    if ((st = make_map(ctx, &ctx->tmK, ctx->kc, s.d, kv_rows, 64, 64)) != PAE_OK) return bail(st);
+    if ((st = make_map(ctx, &ctx->tmV, ctx->vc, s.d, kv_rows, 64, 64)) != PAE_OK) return bail(st);
+    size_t ao = 0;
+    int an = 0;
+    for (int B = 1; B <= s.Bmax; ++B) {
+      const AttnPlan ap = plan_attn(s, B);
+      const size_t units = (size_t)B * s.Hkv * ap.qtiles;
+      if (ap.splits > 1) ao = std::max(ao, units * ap.splits * 128);
+      an = std::max(an, (int)units);
+    }
+    ALLOC(ctx->attn_part_o, sizeof(float) * std::max<size_t>(ao * s.d, 4));
+    ALLOC(ctx->attn_part_ml, sizeof(float) * std::max<size_t>(ao * 2, 4));
+    ALLOC(ctx->attn_counters, sizeof(int) * std::max(an, 1));
+    ctx->attn_counters_n = an;
+    CKC(cudaMemsetAsync(ctx->attn_counters, 0, sizeof(int) * std::max(an, 1), cs));
     // split-K workspace: the largest any batch size needs
     size_t pf = 0;
     int cn = 0;
@@ -848,6 +910,7 @@ pae_status pae_query(pae_ctx* ctx, int what, int batch, long long* value) {
                ((long long)P->down.splits << 24);
       return PAE_OK;
     case PAE_Q_TOKEN_TILE: *value = P->qkv.tn; return PAE_OK;
+    case PAE_Q_ATTN_SPLITS: *value = P->attn.splits; return PAE_OK;
     default: return fail(ctx, PAE_ERR_ARG, "unknown query %d", what);
   }
 }
@@ -864,6 +927,7 @@ void pae_clear_error(pae_ctx* ctx) {
   cudaDeviceSynchronize();
   if (ctx->err_host) *(volatile int*)ctx->err_host = 0;
   if (ctx->counters) cudaMemset(ctx->counters, 0, sizeof(int) * std::max(ctx->counters_n, 1));
+  if (ctx->attn_counters) cudaMemset(ctx->attn_counters, 0, sizeof(int) * std::max(ctx->attn_counters_n, 1));
   ctx->last_error.clear();
 }
 

@@ -177,8 +177,9 @@ pae_status pae_profile_read(pae_ctx* ctx, int kernel_class, double* total_ms, in
 /* Queries.  PAE_Q_GRAPH_KERNELS: kernel nodes in the captured graph of
  * `batch` (0 if none captured yet).  PAE_Q_SPLITS: split-K factors of the four
  * projections for `batch`, packed as qkv | o<<8 | gateup<<16 | down<<24.
- * PAE_Q_TOKEN_TILE: MMA token tile for `batch`. */
-enum { PAE_Q_GRAPH_KERNELS = 1, PAE_Q_SPLITS = 2, PAE_Q_TOKEN_TILE = 3 };
+ * PAE_Q_TOKEN_TILE: MMA token tile for `batch`.  PAE_Q_ATTN_SPLITS: key splits
+ * of the attention for `batch`. */
+enum { PAE_Q_GRAPH_KERNELS = 1, PAE_Q_SPLITS = 2, PAE_Q_TOKEN_TILE = 3, PAE_Q_ATTN_SPLITS = 4 };
 pae_status pae_query(pae_ctx* ctx, int what, int batch, long long* value);
 
 /* Synchronise `stream` and report the device error word (PAE_ERR_TIMEOUT if a
