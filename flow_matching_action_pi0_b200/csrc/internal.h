@@ -56,11 +56,11 @@ struct TransitionArgs {
   float* x_dst;           // write x here after the out step (may equal x)
   int M;
 };
-void launch_transition(const Shape& s, int act_bf16, const TransitionArgs& a, cudaStream_t st);
+cudaError_t launch_transition(const Shape& s, int act_bf16, const TransitionArgs& a, bool pdl, cudaStream_t st);
 
 // y = adaRMSNorm(h; scale, shift) per token.
-void launch_norm(const Shape& s, int act_bf16, const float* h, void* y, const float* scale,
-                 const float* shift, int M, cudaStream_t st);
+cudaError_t launch_norm(const Shape& s, int act_bf16, const float* h, void* y, const float* scale,
+                        const float* shift, int M, bool pdl, cudaStream_t st);
 
 // --------------------------------------------------------- CUDA-core (fp32)
 enum Epi : int { EPI_QKV = 0, EPI_RESID = 1, EPI_GEGLU = 2 };
@@ -101,12 +101,10 @@ struct TcGemmArgs {
   int N;           // output features (GEGLU: F)
   int K;
   int w_row0;      // first row of this layer's matrix inside the stacked weight map
-  float* partials; // split-K workspace
-  int* counters;   // split-K arrival counters (zeroed; the last CTA re-zeroes)
   DevErr err;
 };
-void launch_tc_gemm(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* tmX, int na,
-                    const TcPlan& p, const TcGemmArgs& a, cudaStream_t st);
+cudaError_t launch_tc_gemm(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* tmX, int na,
+                           const TcPlan& p, const TcGemmArgs& a, bool pdl, cudaStream_t st);
 size_t tc_gemm_smem_bytes(int na, const TcPlan& p);
 cudaError_t tc_gemm_init();  // once per process: opt in to large dynamic shared memory
 
@@ -121,14 +119,11 @@ struct AttnArgs {
   int layer;
   int keys_per_split;
   void* o;             // [M][Hq d] bf16, token-major
-  float* part_o;       // [units][splits][128][d] partial outputs (splits > 1)
-  float* part_ml;      // [units][splits][128][2] row max (log2 domain), row sum
-  int* counters;       // [units]
   DevErr err;
 };
 size_t attn_tc_smem_bytes(int d);
 cudaError_t attn_tc_init();
-void launch_attn_tc(const Shape& s, const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
-                    const AttnPlan& p, const AttnArgs& a, int B, cudaStream_t st);
+cudaError_t launch_attn_tc(const Shape& s, const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                           const AttnPlan& p, const AttnArgs& a, int B, bool pdl, cudaStream_t st);
 
 }  // namespace pae

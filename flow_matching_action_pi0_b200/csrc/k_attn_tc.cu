@@ -17,10 +17,12 @@
 // Warps 0-3 run the softmax and the output (thread = query row = TMEM lane);
 // warp 4 is the TMA producer (Q once, K/V chunks through a 2-stage ring);
 // warp 5 issues the MMAs.
-// Key splits (split-KV, for small batches) write unnormalised partial O with
-// the row max and sum; the last CTA of a (b, g, tile) to finish merges them in
-// split order, so the result does not depend on arrival order.
+// Key splits (split-KV, for small batches) form a thread-block cluster; their
+// unnormalised partial O rows, row maxima and sums are merged through
+// distributed shared memory in rank order, so the result is bitwise
+// reproducible and no partial touches global memory.
 #include "internal.h"
+#include "launch.cuh"
 
 namespace pae {
 
@@ -31,7 +33,7 @@ constexpr int QROWS = 128;      // query rows per CTA
 constexpr long long kDrainNs = 4000000000LL;
 
 struct AttnSmem {
-  uint32_t q_off, k_off[2], v_off[2], p_off, bar_off, total;
+  uint32_t q_off, k_off[2], v_off[2], p_off, bar_off, ml_off, total;
 };
 
 __host__ __device__ inline AttnSmem attn_layout(int d) {
@@ -45,7 +47,8 @@ __host__ __device__ inline AttnSmem attn_layout(int d) {
   L.v_off[1] = L.k_off[1] + kvbytes;
   L.p_off = L.v_off[1] + kvbytes;          // [128][64] bf16
   L.bar_off = L.p_off + QROWS * CK * 2;
-  L.total = L.bar_off + 256 + 1024;
+  L.ml_off = L.bar_off + 256;
+  L.total = L.ml_off + QROWS * 12 + 1024;
   return L;
 }
 
@@ -100,13 +103,15 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* o_done = bars + 10;
   uint64_t* drain = bars + 11;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
-  volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);  // [0] abort [1] last
+  volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);  // [0] abort
+  float* s_ml = reinterpret_cast<float*>(smem + L.ml_off);                // [128][2] row max, row sum
+  int* s_ok = reinterpret_cast<int*>(smem + L.ml_off + QROWS * 8);        // [128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x, split = blockIdx.y, bg = blockIdx.z;
   const int b = bg / s.Hkv, g = bg - b * s.Hkv;
   const int GH = s.G * s.H;
-  const int n_valid = a.lens[b] + s.H;
+  const int n_valid = a.lens[b] + s.H;  // written only by pae_set_prefix, before the loop
   const int kps = a.keys_per_split;
   const int start = split * kps;
   const int end = min(n_valid, start + kps);
@@ -117,7 +122,6 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < 12; ++i) mbar_init(&bars[i], i == 9 ? 128 : 1);
     s_flag[0] = 0;
-    s_flag[1] = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
@@ -132,6 +136,8 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_launch_dependents();  // after the TMEM is held (see the projection kernel)
+  pdl_wait();               // q, k, v come from the previous kernel
   const uint32_t t_s[2] = {tmem, tmem + CK};
   const uint32_t t_o = tmem + 2 * CK;
 
@@ -299,97 +305,100 @@ __global__ void __launch_bounds__(192, 1)
   ok = named_and(1, 128, ok) && s_flag[0] == 0;  // CTA-uniform among the 128 softmax threads
   tc_fence_after();
 
-  // ------------------------------------------------------------ output
+  // ------------------------------------------------------------ output (single split)
   const int nsplit = gridDim.y;
-  const bool row_valid = qt * QROWS + r < GH;
-  const int rq = qt * QROWS + r;
-  const int hl = rq / s.H, ti = rq - hl * s.H;
-  bf16* orow = reinterpret_cast<bf16*>(a.o) + (size_t)(b * s.H + ti) * s.attn_dim + (g * s.G + hl) * d;
-  if (ok && nsplit == 1) {
+  if (nsplit == 1) {
+    const int rq = qt * QROWS + r;
+    const bool row_valid = rq < GH;
+    const int hl = rq / s.H, ti = rq - hl * s.H;
+    bf16* orow = reinterpret_cast<bf16*>(a.o) + (size_t)(b * s.H + ti) * s.attn_dim + (g * s.G + hl) * d;
     const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-    for (int j = 0; j < d; j += 16) {
-      float ov[16];
-      tmem_ld16(t_o + lane_off + j, ov);
-      tmem_ld_wait();
-      if (row_valid && nch > 0) {
-        uint32_t pk[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) pk[t] = pack_bf16x2(ov[2 * t] * inv, ov[2 * t + 1] * inv);
-        uint4* dst = reinterpret_cast<uint4*>(orow + j);
-        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-      }
-    }
-  } else if (ok) {
-    // partial: O (unnormalised), row max (log2 domain) and row sum
-    const size_t unit = (size_t)bg * gridDim.x + qt;
-    float* po = a.part_o + ((unit * nsplit + split) * QROWS + r) * (size_t)d;
-    float* pml = a.part_ml + ((unit * nsplit + split) * QROWS + r) * 2;
-    for (int j = 0; j < d; j += 16) {
-      float ov[16];
-      if (nch > 0) {
+    if (ok) {
+      for (int j = 0; j < d; j += 16) {
+        float ov[16];
         tmem_ld16(t_o + lane_off + j, ov);
         tmem_ld_wait();
-      } else {
+        if (row_valid && nch > 0) {
+          uint32_t pk[8];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) ov[t] = 0.f;
+          for (int t = 0; t < 8; ++t) pk[t] = pack_bf16x2(ov[2 * t] * inv, ov[2 * t + 1] * inv);
+          uint4* dst = reinterpret_cast<uint4*>(orow + j);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
       }
+    }
+  } else {
+    s_ok[r] = ok ? 1 : 0;
+    s_ml[2 * r] = m_run;
+    s_ml[2 * r + 1] = l_run;
+  }
+  }  // warps 0-3
+
+  if (gridDim.y > 1) {
+    // Split-KV merge inside the cluster of key splits.  Every CTA parks its
+    // unnormalised O rows (stride d+4 floats, bank-conflict free) and its row
+    // max / sum in shared memory (the Q and K/V buffers are idle now); CTA
+    // rank r then merges rows [r*R, r*R+R) over all ranks in rank order.
+    __syncthreads();  // all MMAs and TMEM reads of this CTA are done
+    const int ld = d + 4;
+    float* red = reinterpret_cast<float*>(smem);
+    if (warp < 4) {
+      const int r = warp * 32 + lane;
+      const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+      const bool has = s_ok[r] && nch > 0;
+      for (int j = 0; j < d; j += 16) {
+        float ov[16];
+        if (__all_sync(0xffffffffu, s_ok[warp * 32] != 0) && nch > 0) {
+          tmem_ld16(t_o + lane_off + j, ov);
+          tmem_ld_wait();
+        }
 #pragma unroll
-      for (int t = 0; t < 16; t += 4)
-        *reinterpret_cast<float4*>(po + j + t) = make_float4(ov[t], ov[t + 1], ov[t + 2], ov[t + 3]);
+        for (int t = 0; t < 16; t += 4)
+          *reinterpret_cast<float4*>(red + r * ld + j + t) =
+              has ? make_float4(ov[t], ov[t + 1], ov[t + 2], ov[t + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      if (!has) {
+        s_ml[2 * r] = -INFINITY;
+        s_ml[2 * r + 1] = 0.f;
+      }
     }
-    pml[0] = nch > 0 ? m_run : -INFINITY;
-    pml[1] = nch > 0 ? l_run : 0.f;
-    __threadfence();
-    named_sync(2, 128);
-    if (threadIdx.x == 0) {
-      int* ctr = a.counters + unit;
-      const int prev = atomicAdd(ctr, 1);
-      const int last = prev == nsplit - 1;
-      s_flag[1] = last;
-      if (last) *ctr = 0;
-    }
-    named_sync(2, 128);
-    if (s_flag[1] && row_valid) {
-      __threadfence();
-      const float* pm0 = a.part_ml + ((unit * nsplit) * QROWS + r) * 2;
+    cluster_sync();
+    const int S = gridDim.y;
+    const uint32_t rank = cluster_rank();
+    const int R = QROWS / S;
+    const uint32_t red_base = smem_u32(red), ml_base = smem_u32(s_ml);
+    const int per_row = d / 4;  // float4 columns
+    for (int el = threadIdx.x; el < R * per_row; el += blockDim.x) {
+      const int rr = el / per_row, c4 = el - rr * per_row;
+      const int row = (int)rank * R + rr;
+      const int rq = qt * QROWS + row;
+      if (rq >= GH) continue;
       float M = -INFINITY;
-      for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, __ldcg(pm0 + (size_t)sp * QROWS * 2));
+      for (int q = 0; q < S; ++q) M = fmaxf(M, ld_cluster_f32(map_cluster(ml_base + row * 8, (uint32_t)q)));
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
       float wsum = 0.f;
-      for (int sp = 0; sp < nsplit; ++sp) {
-        const float m_s = __ldcg(pm0 + (size_t)sp * QROWS * 2);
-        const float l_s = __ldcg(pm0 + (size_t)sp * QROWS * 2 + 1);
-        wsum += (l_s > 0.f) ? l_s * exp2f(m_s - M) : 0.f;
+      for (int q = 0; q < S; ++q) {
+        const float m_s = ld_cluster_f32(map_cluster(ml_base + row * 8, (uint32_t)q));
+        const float l_s = ld_cluster_f32(map_cluster(ml_base + row * 8 + 4, (uint32_t)q));
+        if (!(l_s > 0.f)) continue;
+        const float w = exp2f(m_s - M);
+        wsum = fmaf(w, l_s, wsum);
+        const uint32_t src = map_cluster(red_base + (uint32_t)((row * ld + c4 * 4) * 4), (uint32_t)q);
+        const float4 v = ld_cluster_f32x4(src);
+        acc[0] = fmaf(w, v.x, acc[0]);
+        acc[1] = fmaf(w, v.y, acc[1]);
+        acc[2] = fmaf(w, v.z, acc[2]);
+        acc[3] = fmaf(w, v.w, acc[3]);
       }
       const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-      const float* po0 = a.part_o + ((unit * nsplit) * QROWS + r) * (size_t)d;
-      for (int j = 0; j < d; j += 8) {
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int sp = 0; sp < nsplit; ++sp) {
-          const float m_s = __ldcg(pm0 + (size_t)sp * QROWS * 2);
-          const float l_s = __ldcg(pm0 + (size_t)sp * QROWS * 2 + 1);
-          if (!(l_s > 0.f)) continue;
-          const float wgt = exp2f(m_s - M);
-          const float* src = po0 + (size_t)sp * QROWS * d + j;
-          const float4 x0 = __ldcg(reinterpret_cast<const float4*>(src));
-          const float4 x1 = __ldcg(reinterpret_cast<const float4*>(src + 4));
-          acc[0] = fmaf(wgt, x0.x, acc[0]);
-          acc[1] = fmaf(wgt, x0.y, acc[1]);
-          acc[2] = fmaf(wgt, x0.z, acc[2]);
-          acc[3] = fmaf(wgt, x0.w, acc[3]);
-          acc[4] = fmaf(wgt, x1.x, acc[4]);
-          acc[5] = fmaf(wgt, x1.y, acc[5]);
-          acc[6] = fmaf(wgt, x1.z, acc[6]);
-          acc[7] = fmaf(wgt, x1.w, acc[7]);
-        }
-        *reinterpret_cast<uint4*>(orow + j) =
-            make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
-                       pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
-      }
+      const int hl = rq / s.H, ti = rq - hl * s.H;
+      bf16* orow = reinterpret_cast<bf16*>(a.o) + (size_t)(b * s.H + ti) * s.attn_dim + (g * s.G + hl) * d;
+      *reinterpret_cast<uint2*>(orow + c4 * 4) =
+          make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
     }
+    cluster_sync();  // peers may still be reading this CTA's partial
   }
-
-  }  // warps 0-3
 
   tc_fence_before();
   __syncthreads();
@@ -404,10 +413,11 @@ cudaError_t attn_tc_init() {
   return cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
 }
 
-void launch_attn_tc(const Shape& s, const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
-                    const AttnPlan& p, const AttnArgs& a, int B, cudaStream_t st) {
+cudaError_t launch_attn_tc(const Shape& s, const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                           const AttnPlan& p, const AttnArgs& a, int B, bool pdl, cudaStream_t st) {
   dim3 grid(p.qtiles, p.splits, B * s.Hkv);
-  k_attn_tc<<<grid, 192, attn_tc_smem_bytes(s.d), st>>>(*tmQ, *tmK, *tmV, s, a);
+  return launch_ex(k_attn_tc, grid, dim3(192), attn_tc_smem_bytes(s.d), st, p.splits, pdl, *tmQ, *tmK, *tmV, s,
+                   a);
 }
 
 }  // namespace pae

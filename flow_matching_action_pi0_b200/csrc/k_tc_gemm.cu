@@ -12,11 +12,14 @@
 //   warp 1 / lane 0  MMA issuer: tcgen05.mma kind::f16 (bf16 in, fp32 in TMEM)
 //   warps 0-3        epilogue: tcgen05.ld of the accumulator (thread = weight
 //                    row = output feature, 16 token columns per load)
-// Split-K: grid.y CTAs share one output tile; each writes its fp32 partial to a
-// workspace, and the last CTA to arrive (atomic counter) sums the partials in
-// split order and runs the epilogue.  No CTA waits for another, and the sum
-// order is fixed, so results are bitwise reproducible.
+// Split-K: the grid.y CTAs of one output tile form a thread-block cluster;
+// their fp32 partials are reduced on chip through distributed shared memory,
+// each CTA summing a 1/S slice of the rows over all ranks in rank order, so
+// results are bitwise reproducible and no partial touches global memory.
+// The weight loads of the first ring are issued before griddepcontrol.wait, so
+// under programmatic dependent launch they overlap the previous kernel.
 #include "epilogue.cuh"
+#include "launch.cuh"
 
 namespace pae {
 
@@ -57,7 +60,7 @@ __global__ void __launch_bounds__(128, 1)
   uint64_t* empty = full + p.stages;
   uint64_t* accf = empty + p.stages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
-  volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);  // [0] abort, [1] last
+  volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);  // [0] abort
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntile = blockIdx.x, split = blockIdx.y, ttile = blockIdx.z;
@@ -73,7 +76,6 @@ __global__ void __launch_bounds__(128, 1)
     }
     mbar_init(accf, 1);
     s_flag[0] = 0;
-    s_flag[1] = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmX);
@@ -86,23 +88,35 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Only now, with its TMEM held, may this CTA let the next kernel's CTAs in:
+  // a successor that took the TMEM first would wait on us forever.
+  pdl_launch_dependents();
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- producer
+    // Weight tiles do not depend on the previous kernel: the first ring's worth
+    // is requested before waiting for it (programmatic dependent launch).
     const uint64_t pol_w = policy_evict_first();  // weights: streamed once
-    int issued = 0;
-    for (int kb = 0; kb < nkb; ++kb) {
+    const int npre = nkb < p.stages ? nkb : p.stages;
+    const int wrow = a.w_row0 + ntile * 128 * NA;
+    for (int kb = 0; kb < npre; ++kb) {
+      mbar_arrive_expect_tx(&full[kb], L.stage_bytes);
+      tma_load_2d_hint(smem + (size_t)kb * L.stage_bytes, &tmW, k0 + kb * 64, wrow, &full[kb], pol_w);
+    }
+    pdl_wait();
+    for (int kb = 0; kb < npre; ++kb)
+      tma_load_2d(smem + (size_t)kb * L.stage_bytes + L.a_bytes, &tmX, k0 + kb * 64, ttile * p.tn, &full[kb]);
+    int issued = npre;
+    for (int kb = npre; kb < nkb; ++kb) {
       const int st = kb % p.stages;
-      if (kb >= p.stages) {
-        if (!mbar_wait(&empty[st], ((kb / p.stages) & 1) ^ 1, a.err.wait_ns)) {
-          s_flag[0] = 1;
-          set_error(a.err, DEV_TIMEOUT);
-          break;
-        }
+      if (!mbar_wait(&empty[st], ((kb / p.stages) & 1) ^ 1, a.err.wait_ns)) {
+        s_flag[0] = 1;
+        set_error(a.err, DEV_TIMEOUT);
+        break;
       }
       uint8_t* sa = smem + (size_t)st * L.stage_bytes;
       mbar_arrive_expect_tx(&full[st], L.stage_bytes);
-      tma_load_2d_hint(sa, &tmW, k0 + kb * 64, a.w_row0 + ntile * 128 * NA, &full[st], pol_w);
+      tma_load_2d_hint(sa, &tmW, k0 + kb * 64, wrow, &full[st], pol_w);
       tma_load_2d(sa + L.a_bytes, &tmX, k0 + kb * 64, ttile * p.tn, &full[st]);
       issued = kb + 1;
     }
@@ -136,6 +150,7 @@ __global__ void __launch_bounds__(128, 1)
     umma_commit(accf);  // always issued, so the epilogue wait ends
   }
   __syncwarp();
+  pdl_wait();  // the epilogue reads the residual stream / slot lengths
 
   // ------------------------------------------------------------------ epilogue
   const bool acc_ok = mbar_wait(accf, 0, kDrainNs);
@@ -145,64 +160,67 @@ __global__ void __launch_bounds__(128, 1)
   const bool ok = __syncthreads_and(acc_ok ? 1 : 0) != 0 && s_flag[0] == 0;
 
   const int row = warp * 32 + lane;
-  const int f = ntile * 128 + row;
   const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
   const int mbase = ttile * p.tn;
   const EpiArgs& e = a.e;
 
-  if (ok && p.splits == 1) {
-    for (int c0 = 0; c0 < p.tn; c0 += 16) {
-      float v0[16], v1[16];
-      tmem_ld16(trow + c0, v0);
-      if (NA == 2) tmem_ld16(trow + p.tn + c0, v1);
-      tmem_ld_wait();
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int m = mbase + c0 + j;
-        if (m < e.M && f < a.N) epi_apply<bf16>(s, e, m, f, v0[j], NA == 2 ? v1[j] : 0.f);
-      }
-    }
-  } else if (ok) {
-    const size_t Mpad = (size_t)p.tok_tiles * p.tn;
-    for (int c0 = 0; c0 < p.tn; c0 += 16) {
-      float v0[16], v1[16];
-      tmem_ld16(trow + c0, v0);
-      if (NA == 2) tmem_ld16(trow + p.tn + c0, v1);
-      tmem_ld_wait();
-      if (f < a.N) {
+  if (p.splits == 1) {
+    const int f = ntile * 128 + row;
+    if (ok) {
+      for (int c0 = 0; c0 < p.tn; c0 += 16) {
+        float v0[16], v1[16];
+        tmem_ld16(trow + c0, v0);
+        if (NA == 2) tmem_ld16(trow + p.tn + c0, v1);
+        tmem_ld_wait();
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const size_t m = mbase + c0 + j;
-          a.partials[((size_t)(split * NA) * Mpad + m) * a.N + f] = v0[j];
-          if (NA == 2) a.partials[((size_t)(split * NA + 1) * Mpad + m) * a.N + f] = v1[j];
+          const int m = mbase + c0 + j;
+          if (m < e.M && f < a.N) epi_apply<bf16>(s, e, m, f, v0[j], NA == 2 ? v1[j] : 0.f);
         }
       }
     }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int* ctr = a.counters + ttile * gridDim.x + ntile;
-      const int prev = atomicAdd(ctr, 1);
-      const int last = (prev == p.splits - 1);
-      s_flag[1] = last;
-      if (last) *ctr = 0;  // every split has arrived: reset for the next launch
-    }
-    __syncthreads();
-    if (s_flag[1]) {
-      __threadfence();
-      if (f < a.N) {
-        for (int c = 0; c < p.tn; ++c) {
-          const int m = mbase + c;
-          if (m >= e.M) break;
-          float s0 = 0.f, s1 = 0.f;
-          for (int sp = 0; sp < p.splits; ++sp) {
-            s0 += __ldcg(&a.partials[((size_t)(sp * NA) * Mpad + m) * a.N + f]);
-            if (NA == 2) s1 += __ldcg(&a.partials[((size_t)(sp * NA + 1) * Mpad + m) * a.N + f]);
-          }
-          epi_apply<bf16>(s, e, m, f, s0, s1);
+  } else {
+    // Split-K inside a cluster of p.splits CTAs: each parks its fp32 partial
+    // in its own shared memory, token-major ([na][token][128 rows]), then CTA
+    // rank r sums rows [r*R, r*R+R) over all ranks in rank order through
+    // distributed shared memory and runs the epilogue on them.
+    float* red = reinterpret_cast<float*>(smem);
+    if (ok) {
+      for (int c0 = 0; c0 < p.tn; c0 += 16) {
+        float v0[16], v1[16];
+        tmem_ld16(trow + c0, v0);
+        if (NA == 2) tmem_ld16(trow + p.tn + c0, v1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          red[(c0 + j) * 128 + row] = v0[j];
+          if (NA == 2) red[(p.tn + c0 + j) * 128 + row] = v1[j];
         }
       }
     }
+    cluster_sync();
+    const int S = p.splits;
+    const uint32_t rank = cluster_rank();
+    const int R = 128 / S;
+    const uint32_t red_base = smem_u32(red);
+    const int any_ok = ok ? 1 : 0;
+    if (any_ok) {
+      for (int el = threadIdx.x; el < R * p.tn; el += 128) {
+        const int rr = el % R, col = el / R;
+        const int rw = (int)rank * R + rr;
+        const int m = mbase + col, f = ntile * 128 + rw;
+        const uint32_t off0 = (uint32_t)((col * 128 + rw) * 4);
+        const uint32_t off1 = (uint32_t)(((p.tn + col) * 128 + rw) * 4);
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll 4
+        for (int q = 0; q < S; ++q) {
+          s0 += ld_cluster_f32(map_cluster(red_base + off0, (uint32_t)q));
+          if (NA == 2) s1 += ld_cluster_f32(map_cluster(red_base + off1, (uint32_t)q));
+        }
+        if (m < e.M && f < a.N) epi_apply<bf16>(s, e, m, f, s0, s1);
+      }
+    }
+    cluster_sync();  // peers may still be reading this CTA's partial
   }
 
   tc_fence_before();
@@ -217,19 +235,19 @@ size_t tc_gemm_smem_bytes(int na, const TcPlan& p) { return tc_layout(na, p.tn, 
 cudaError_t tc_gemm_init() {
   const int max_smem = 227 * 1024;
   cudaError_t e = cudaFuncSetAttribute(k_tc_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(k_tc_gemm<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_tc_gemm<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_tc_gemm<1>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_tc_gemm<2>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
 }
 
-void launch_tc_gemm(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* tmX, int na, const TcPlan& p,
-                    const TcGemmArgs& a, cudaStream_t st) {
+cudaError_t launch_tc_gemm(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* tmX, int na, const TcPlan& p,
+                           const TcGemmArgs& a, bool pdl, cudaStream_t st) {
   const int ntiles = (a.N + 127) / 128;
   dim3 grid(ntiles, p.splits, p.tok_tiles);
   const size_t smem = tc_gemm_smem_bytes(na, p);
-  if (na == 2)
-    k_tc_gemm<2><<<grid, 128, smem, st>>>(*tmW, *tmX, s, p, a);
-  else
-    k_tc_gemm<1><<<grid, 128, smem, st>>>(*tmW, *tmX, s, p, a);
+  if (na == 2) return launch_ex(k_tc_gemm<2>, grid, dim3(128), smem, st, p.splits, pdl, *tmW, *tmX, s, p, a);
+  return launch_ex(k_tc_gemm<1>, grid, dim3(128), smem, st, p.splits, pdl, *tmW, *tmX, s, p, a);
 }
 
 }  // namespace pae

@@ -9,6 +9,7 @@
 // adaRMSNorm(h) = h / sqrt(mean(h^2) + eps) * (1 + scale) + shift (no learned gain).
 // Reductions use a fixed tree, so results are bitwise reproducible.
 #include "internal.h"
+#include "launch.cuh"
 
 namespace pae {
 
@@ -34,6 +35,8 @@ __global__ void __launch_bounds__(256) k_transition(const Shape s, const Transit
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
   const float* xsrc = a.x_src + (size_t)m * A;
   float* xdst = a.x_dst + (size_t)m * A;
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (a.tab_out) {
     const float* hrow = a.h + (size_t)m * D;
@@ -99,6 +102,8 @@ __global__ void __launch_bounds__(256) k_norm(const Shape s, const float* __rest
                                               int M) {
   const int lane = threadIdx.x & 31;
   const int m = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_launch_dependents();
   if (m >= M) return;
   const int D = s.D;
   const float* hr = h + (size_t)m * D;
@@ -112,21 +117,20 @@ __global__ void __launch_bounds__(256) k_norm(const Shape s, const float* __rest
 
 }  // namespace
 
-void launch_transition(const Shape& s, int act_bf16, const TransitionArgs& a, cudaStream_t st) {
+cudaError_t launch_transition(const Shape& s, int act_bf16, const TransitionArgs& a, bool pdl, cudaStream_t st) {
   const size_t smem = (size_t)(s.D + s.A + 32) * sizeof(float);
-  if (act_bf16)
-    k_transition<bf16, bf16><<<a.M, 256, smem, st>>>(s, a);
-  else
-    k_transition<float, float><<<a.M, 256, smem, st>>>(s, a);
+  if (act_bf16) return launch_ex(k_transition<bf16, bf16>, dim3(a.M), dim3(256), smem, st, 1, pdl, s, a);
+  return launch_ex(k_transition<float, float>, dim3(a.M), dim3(256), smem, st, 1, pdl, s, a);
 }
 
-void launch_norm(const Shape& s, int act_bf16, const float* h, void* y, const float* scale, const float* shift,
-                 int M, cudaStream_t st) {
+cudaError_t launch_norm(const Shape& s, int act_bf16, const float* h, void* y, const float* scale, const float* shift,
+                        int M, bool pdl, cudaStream_t st) {
   const int blocks = (M + 7) / 8;
   if (act_bf16)
-    k_norm<bf16><<<blocks, 256, 0, st>>>(s, h, static_cast<bf16*>(y), scale, shift, M);
-  else
-    k_norm<float><<<blocks, 256, 0, st>>>(s, h, static_cast<float*>(y), scale, shift, M);
+    return launch_ex(k_norm<bf16>, dim3(blocks), dim3(256), 0, st, 1, pdl, s, h, static_cast<bf16*>(y), scale, shift,
+                     M);
+  return launch_ex(k_norm<float>, dim3(blocks), dim3(256), 0, st, 1, pdl, s, h, static_cast<float*>(y), scale, shift,
+                   M);
 }
 
 }  // namespace pae

@@ -89,18 +89,12 @@ struct pae_ctx {
   // activations and workspaces
   float *x = nullptr, *h = nullptr;
   void *y = nullptr, *q = nullptr, *o = nullptr, *u = nullptr;
-  float* partials = nullptr;
-  size_t partials_floats = 0;
-  int* counters = nullptr;
-  int counters_n = 0;
-  float *attn_part_o = nullptr, *attn_part_ml = nullptr;
-  int* attn_counters = nullptr;
-  int attn_counters_n = 0;
   // error word (host-mapped)
   int* err_host = nullptr;
   int* err_dev = nullptr;
   long long wait_ns = 2000000000LL;
   bool use_graph = true;
+  bool use_pdl = true;
   std::map<int, Plan> plans;
   Plan* last_plan = nullptr;
   unsigned profile_mask = 0;
@@ -170,8 +164,11 @@ pae_status make_map(pae_ctx* ctx, CUtensorMap* m, const void* base, uint64_t inn
 }
 
 // Token tile and split-K choice for one projection of `nfeat` outputs and K
-// inputs: the token tile covers the tokens with as little padding as possible
-// (<= 256 per MMA), and split-K fills the 148 SMs when the tile count is small.
+// inputs.  The token tile covers the tokens with as little padding as possible
+// (<= 256 per MMA).  Split-K (a cluster of S CTAs, S a power of two <= 16 that
+// divides the 64-wide K blocks) fills the 148 SMs when the tile count is small;
+// small token tiles keep shared memory under half an SM so that two CTAs (or a
+// CTA and its successor under PDL) fit per SM.
 TcPlan plan_gemm(int M, int nfeat, int K, int na) {
   TcPlan p{};
   p.tok_tiles = (M + 255) / 256;
@@ -179,27 +176,34 @@ TcPlan plan_gemm(int M, int nfeat, int K, int na) {
   p.tn = std::max(16, ((per + 15) / 16) * 16);
   const int base = ((nfeat + 127) / 128) * p.tok_tiles;
   const int nkb = K / 64;
-  const int target = 2 * 148;
-  p.splits = 1;
-  for (int sp = 1; sp <= nkb; ++sp)
-    if (nkb % sp == 0 && base * sp <= target) p.splits = sp;
   const uint32_t stage = (uint32_t)na * 16384u + (uint32_t)p.tn * 128u;
-  int st = (int)((200u * 1024u) / stage);  // leaves room for barriers and alignment slack
+  const uint32_t red = (uint32_t)na * p.tn * 128u * 4u;  // parked fp32 partial
+  const bool small = p.tn <= 64;
+  const uint32_t budget = small ? 100u * 1024u : 200u * 1024u;
+  const int target = small ? 2 * 148 : 148;
+  p.splits = 1;
+  for (int sp = 2; sp <= 16; sp *= 2)
+    if (nkb % sp == 0 && base * sp <= target && red <= budget) p.splits = sp;
+  int st = (int)(budget / stage);
   st = std::max(2, std::min(st, 6));
+  st = std::min(st, std::max(2, nkb / p.splits));
+  if (p.splits > 1) st = std::max(st, (int)((red + stage - 1) / stage));
   p.stages = st;
   return p;
 }
 
-// Query tiles of 128 rows per (request, KV head); key splits only when the
-// batch gives too few tiles to fill the 148 SMs (split-KV at small batch).
+// Query tiles of 128 rows per (request, KV head); key splits (a cluster of
+// S <= 8 CTAs, S a power of two) only when the batch gives too few tiles to
+// fill the 148 SMs (split-KV at small batch).
 AttnPlan plan_attn(const Shape& s, int B) {
   AttnPlan p{};
   p.qtiles = (s.G * s.H + 127) / 128;
   const int base = B * s.Hkv * p.qtiles;
   const int max_splits = (s.Ptot + 63) / 64;
-  int splits = base * 4 >= 3 * 148 ? 1 : std::max(1, std::min(max_splits, 148 / base));
+  int splits = 1;
+  while (splits < 8 && base * splits * 2 <= 148 && splits * 2 <= max_splits) splits *= 2;
   p.keys_per_split = ((s.Ptot + splits - 1) / splits + 63) / 64 * 64;
-  p.splits = (s.Ptot + p.keys_per_split - 1) / p.keys_per_split;
+  p.splits = splits;
   return p;
 }
 
@@ -219,19 +223,6 @@ pae_status build_plan(pae_ctx* ctx, int B, Plan* P) {
   if ((st = make_map(ctx, &P->tmO, ctx->o, s.attn_dim, Mmax, 64, P->o.tn)) != PAE_OK) return st;
   if ((st = make_map(ctx, &P->tmU, ctx->u, s.F, Mmax, 64, P->down.tn)) != PAE_OK) return st;
   return PAE_OK;
-}
-
-size_t plan_partials(const Plan& P, const Shape& s) {
-  auto one = [&](const TcPlan& p, int n, int na) -> size_t {
-    if (p.splits <= 1) return 0;
-    return (size_t)p.splits * na * p.tok_tiles * p.tn * n;
-  };
-  return std::max(std::max(one(P.qkv, s.qkv_rows, 1), one(P.o, s.D, 1)),
-                  std::max(one(P.gu, s.F, 2), one(P.down, s.D, 1)));
-}
-int plan_counters(const Plan& P, const Shape& s) {
-  auto one = [&](const TcPlan& p, int n) { return ((n + 127) / 128) * p.tok_tiles; };
-  return std::max(std::max(one(P.qkv, s.qkv_rows), one(P.o, s.D)), std::max(one(P.gu, s.F), one(P.down, s.D)));
 }
 
 // Launch bracketing for PAE_OPT_PROFILE: events come from a pool sized before
@@ -278,6 +269,10 @@ pae_status ensure_events(pae_ctx* ctx, int k_steps) {
   return PAE_OK;
 }
 
+// PDL is used in the bf16 modes, and not while launches are bracketed by
+// profiling events (an event between two kernels is not a kernel edge).
+bool pdl_on(const pae_ctx* ctx) { return ctx->use_pdl && ctx->act_bf16 && ctx->profile_mask == 0; }
+
 const float* tab(const pae_ctx* ctx, int k) { return ctx->tables + (size_t)k * ctx->s.table_rows; }
 
 void run_gemm(pae_ctx* ctx, const Plan& P, int which, int layer, const EpiArgs& e, cudaStream_t st) {
@@ -298,8 +293,6 @@ void run_gemm(pae_ctx* ctx, const Plan& P, int which, int layer, const EpiArgs& 
   }
   TcGemmArgs a{};
   a.e = e;
-  a.partials = ctx->partials;
-  a.counters = ctx->counters;
   a.err = DevErr{ctx->err_dev, ctx->wait_ns};
   const CUtensorMap *tw, *tx;
   const TcPlan* p;
@@ -310,7 +303,7 @@ void run_gemm(pae_ctx* ctx, const Plan& P, int which, int layer, const EpiArgs& 
     case 2: tw = &ctx->tmWgu; tx = &P.tmY; p = &P.gu; a.N = s.F; a.K = s.D; a.w_row0 = layer * 2 * s.F; na = 2; break;
     default: tw = &ctx->tmWdown; tx = &P.tmU; p = &P.down; a.N = s.D; a.K = s.F; a.w_row0 = layer * s.D; break;
   }
-  launch_tc_gemm(s, tw, tx, na, *p, a, st);
+  launch_tc_gemm(s, tw, tx, na, *p, a, pdl_on(ctx), st);
 }
 
 // Enqueue Euler steps k_begin..k_end-1 for the plan's batch on `st`, with the
@@ -338,7 +331,7 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
     ta.tab_in = tk;
     {
       ProfScope ps(ctx, PAE_K_TRANSITION, st);
-      launch_transition(s, ctx->act_bf16, ta, st);
+      launch_transition(s, ctx->act_bf16, ta, pdl_on(ctx), st);
     }
     for (int l = 0; l < s.L; ++l) {
       EpiArgs e{};
@@ -361,11 +354,8 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
           aa.layer = l;
           aa.keys_per_split = P.attn.keys_per_split;
           aa.o = ctx->o;
-          aa.part_o = ctx->attn_part_o;
-          aa.part_ml = ctx->attn_part_ml;
-          aa.counters = ctx->attn_counters;
           aa.err = DevErr{ctx->err_dev, ctx->wait_ns};
-          launch_attn_tc(s, &ctx->tmQ, &ctx->tmK, &ctx->tmV, P.attn, aa, P.B, st);
+          launch_attn_tc(s, &ctx->tmQ, &ctx->tmK, &ctx->tmV, P.attn, aa, P.B, pdl_on(ctx), st);
         } else {
           launch_attention_simple(s, ctx->act_bf16, ctx->q, ctx->kc, ctx->vc, ctx->lens_dev, l, ctx->o, P.B, st);
         }
@@ -381,8 +371,7 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
       }
       {
         ProfScope ps(ctx, PAE_K_NORM, st);
-        launch_norm(s, ctx->act_bf16, ctx->h, ctx->y, tk + mod_offset(s, l, 1, 0), tk + mod_offset(s, l, 1, 1), M,
-                    st);
+        launch_norm(s, ctx->act_bf16, ctx->h, ctx->y, tk + mod_offset(s, l, 1, 0), tk + mod_offset(s, l, 1, 1), M, pdl_on(ctx), st);
       }
       e = EpiArgs{};
       e.M = M;
@@ -404,7 +393,7 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
       if (l + 1 < s.L) {
         ProfScope ps(ctx, PAE_K_NORM, st);
         launch_norm(s, ctx->act_bf16, ctx->h, ctx->y, tk + mod_offset(s, l + 1, 0, 0), tk + mod_offset(s, l + 1, 0, 1),
-                    M, st);
+                    M, pdl_on(ctx), st);
       }
     }
   }
@@ -413,7 +402,7 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
   ta.tab_in = nullptr;
   {
     ProfScope ps(ctx, PAE_K_TRANSITION, st);
-    launch_transition(s, ctx->act_bf16, ta, st);
+    launch_transition(s, ctx->act_bf16, ta, pdl_on(ctx), st);
   }
 }
 
@@ -713,37 +702,6 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
     if ((st = make_map(ctx, &ctx->tmQ, ctx->q, s.d, (uint64_t)s.Bmax * s.Hq * s.H, 64, 128)) != PAE_OK) return bail(st);
     if ((st = make_map(ctx, &ctx->tmK, ctx->kc, s.d, kv_rows, 64, 64)) != PAE_OK) return bail(st);
     if ((st = make_map(ctx, &ctx->tmV, ctx->vc, s.d, kv_rows, 64, 64)) != PAE_OK) return bail(st);
-    size_t ao = 0;
-    int an = 0;
-    for (int B = 1; B <= s.Bmax; ++B) {
-      const AttnPlan ap = plan_attn(s, B);
-      const size_t units = (size_t)B * s.Hkv * ap.qtiles;
-      if (ap.splits > 1) ao = std::max(ao, units * ap.splits * 128);
-      an = std::max(an, (int)units);
-    }
-    ALLOC(ctx->attn_part_o, sizeof(float) * std::max<size_t>(ao * s.d, 4));
-    ALLOC(ctx->attn_part_ml, sizeof(float) * std::max<size_t>(ao * 2, 4));
-    ALLOC(ctx->attn_counters, sizeof(int) * std::max(an, 1));
-    ctx->attn_counters_n = an;
-    CKC(cudaMemsetAsync(ctx->attn_counters, 0, sizeof(int) * std::max(an, 1), cs));
-    // split-K workspace: the largest any batch size needs
-    size_t pf = 0;
-    int cn = 0;
-    for (int B = 1; B <= s.Bmax; ++B) {
-      Plan P;
-      const int M = B * s.H;
-      P.qkv = plan_gemm(M, s.qkv_rows, D, 1);
-      P.o = plan_gemm(M, D, s.attn_dim, 1);
-      P.gu = plan_gemm(M, F, D, 2);
-      P.down = plan_gemm(M, D, F, 1);
-      pf = std::max(pf, plan_partials(P, s));
-      cn = std::max(cn, plan_counters(P, s));
-    }
-    ctx->partials_floats = pf;
-    ctx->counters_n = cn;
-    ALLOC(ctx->partials, sizeof(float) * std::max<size_t>(pf, 4));
-    ALLOC(ctx->counters, sizeof(int) * std::max(cn, 1));
-    CKC(cudaMemsetAsync(ctx->counters, 0, sizeof(int) * std::max(cn, 1), cs));
   }
   CKC(cudaStreamSynchronize(cs));
   CKC(cudaGetLastError());
@@ -872,6 +830,10 @@ pae_status pae_set_option(pae_ctx* ctx, int option, long long value) {
       ctx->wait_ns = value * 1000LL;
       drop_graphs(ctx);  // captured launches hold the old limit
       return PAE_OK;
+    case PAE_OPT_PDL:
+      if ((value != 0) != ctx->use_pdl) drop_graphs(ctx);
+      ctx->use_pdl = value != 0;
+      return PAE_OK;
     case PAE_OPT_PROFILE:
       if (value < 0 || value >= (1LL << PAE_K_COUNT)) return fail(ctx, PAE_ERR_ARG, "bad profile mask");
       if ((unsigned)value != ctx->profile_mask) drop_graphs(ctx);
@@ -926,8 +888,6 @@ void pae_clear_error(pae_ctx* ctx) {
   if (!ctx) return;
   cudaDeviceSynchronize();
   if (ctx->err_host) *(volatile int*)ctx->err_host = 0;
-  if (ctx->counters) cudaMemset(ctx->counters, 0, sizeof(int) * std::max(ctx->counters_n, 1));
-  if (ctx->attn_counters) cudaMemset(ctx->attn_counters, 0, sizeof(int) * std::max(ctx->attn_counters_n, 1));
   ctx->last_error.clear();
 }
 

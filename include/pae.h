@@ -151,8 +151,10 @@ pae_status pae_denoise_steps(pae_ctx* ctx, const float* x_in, float* x_out, int 
 
 /* Options.  PAE_OPT_USE_GRAPH (default 1): 0 makes pae_denoise launch the
  * kernels directly.  PAE_OPT_WAIT_LIMIT_US (default 2000000): bound of every
- * device-side wait, in microseconds. */
-enum { PAE_OPT_USE_GRAPH = 1, PAE_OPT_WAIT_LIMIT_US = 2 };
+ * device-side wait, in microseconds.  PAE_OPT_PDL (default 1, bf16 modes):
+ * programmatic dependent launch between the loop's kernels, so a kernel's
+ * weight loads overlap its predecessor's tail; 0 serialises the kernels. */
+enum { PAE_OPT_USE_GRAPH = 1, PAE_OPT_WAIT_LIMIT_US = 2, PAE_OPT_PDL = 4 };
 pae_status pae_set_option(pae_ctx* ctx, int option, long long value);
 
 /* Kernel classes for profiling, as bit positions of PAE_OPT_PROFILE. */

@@ -44,6 +44,17 @@ def test_graph_replay_equals_direct_launch(setup):
     np.testing.assert_array_equal(a, c)
 
 
+def test_pdl_does_not_change_results(setup):
+    cfg, ex, W, ks, vs, grid, noise = setup
+    a = run_gpu(ex, noise)
+    ex.set_option(fm.PAE_OPT_PDL, 0)
+    b = run_gpu(ex, noise)
+    ex.set_option(fm.PAE_OPT_PDL, 1)
+    c = run_gpu(ex, noise)
+    np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(a, c)
+
+
 def test_step_split_bitwise(setup):
     cfg, ex, W, ks, vs, grid, noise = setup
     full = run_gpu(ex, noise)
