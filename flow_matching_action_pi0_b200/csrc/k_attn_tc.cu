@@ -374,22 +374,31 @@ __global__ void __launch_bounds__(192, 1)
       const int row = (int)rank * R + rr;
       const int rq = qt * QROWS + row;
       if (rq >= GH) continue;
+      // issue every rank's loads first (they pipeline), then merge in rank order
+      float ms[8], ls[8];
+      float4 vs[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (q < S) {
+          ms[q] = ld_cluster_f32(map_cluster(ml_base + row * 8, (uint32_t)q));
+          ls[q] = ld_cluster_f32(map_cluster(ml_base + row * 8 + 4, (uint32_t)q));
+          vs[q] = ld_cluster_f32x4(map_cluster(red_base + (uint32_t)((row * ld + c4 * 4) * 4), (uint32_t)q));
+        }
       float M = -INFINITY;
-      for (int q = 0; q < S; ++q) M = fmaxf(M, ld_cluster_f32(map_cluster(ml_base + row * 8, (uint32_t)q)));
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (q < S) M = fmaxf(M, ms[q]);
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
       float wsum = 0.f;
-      for (int q = 0; q < S; ++q) {
-        const float m_s = ld_cluster_f32(map_cluster(ml_base + row * 8, (uint32_t)q));
-        const float l_s = ld_cluster_f32(map_cluster(ml_base + row * 8 + 4, (uint32_t)q));
-        if (!(l_s > 0.f)) continue;
-        const float w = exp2f(m_s - M);
-        wsum = fmaf(w, l_s, wsum);
-        const uint32_t src = map_cluster(red_base + (uint32_t)((row * ld + c4 * 4) * 4), (uint32_t)q);
-        const float4 v = ld_cluster_f32x4(src);
-        acc[0] = fmaf(w, v.x, acc[0]);
-        acc[1] = fmaf(w, v.y, acc[1]);
-        acc[2] = fmaf(w, v.z, acc[2]);
-        acc[3] = fmaf(w, v.w, acc[3]);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (q >= S || !(ls[q] > 0.f)) continue;
+        const float w = exp2f(ms[q] - M);
+        wsum = fmaf(w, ls[q], wsum);
+        acc[0] = fmaf(w, vs[q].x, acc[0]);
+        acc[1] = fmaf(w, vs[q].y, acc[1]);
+        acc[2] = fmaf(w, vs[q].z, acc[2]);
+        acc[3] = fmaf(w, vs[q].w, acc[3]);
       }
       const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
       const int hl = rq / s.H, ti = rq - hl * s.H;

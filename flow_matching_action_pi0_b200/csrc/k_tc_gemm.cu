@@ -96,7 +96,9 @@ __global__ void __launch_bounds__(128, 1)
     // ---------------------------------------------------------------- producer
     // Weight tiles do not depend on the previous kernel: the first ring's worth
     // is requested before waiting for it (programmatic dependent launch).
-    const uint64_t pol_w = policy_evict_first();  // weights: streamed once
+    // weights are streamed once per step when one token tile covers the batch;
+    // otherwise the other token tiles re-read them from L2
+    const uint64_t pol_w = p.tok_tiles == 1 ? policy_evict_first() : policy_evict_last();
     const int npre = nkb < p.stages ? nkb : p.stages;
     const int wrow = a.w_row0 + ntile * 128 * NA;
     for (int kb = 0; kb < npre; ++kb) {
@@ -211,12 +213,21 @@ __global__ void __launch_bounds__(128, 1)
         const int m = mbase + col, f = ntile * 128 + rw;
         const uint32_t off0 = (uint32_t)((col * 128 + rw) * 4);
         const uint32_t off1 = (uint32_t)(((p.tn + col) * 128 + rw) * 4);
+        // issue every rank's load first (they pipeline), then sum in rank order
+        float v0[16], v1[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          if (q < S) {
+            v0[q] = ld_cluster_f32(map_cluster(red_base + off0, (uint32_t)q));
+            if (NA == 2) v1[q] = ld_cluster_f32(map_cluster(red_base + off1, (uint32_t)q));
+          }
         float s0 = 0.f, s1 = 0.f;
-#pragma unroll 4
-        for (int q = 0; q < S; ++q) {
-          s0 += ld_cluster_f32(map_cluster(red_base + off0, (uint32_t)q));
-          if (NA == 2) s1 += ld_cluster_f32(map_cluster(red_base + off1, (uint32_t)q));
-        }
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          if (q < S) {
+            s0 += v0[q];
+            if (NA == 2) s1 += v1[q];
+          }
         if (m < e.M && f < a.N) epi_apply<bf16>(s, e, m, f, s0, s1);
       }
     }

@@ -7,7 +7,9 @@
 //   (start of k+1)    h = x W_in^T + b_in,
 //                     y = adaRMSNorm(h; layer-0 attention scale/shift)
 // adaRMSNorm(h) = h / sqrt(mean(h^2) + eps) * (1 + scale) + shift (no learned gain).
-// Reductions use a fixed tree, so results are bitwise reproducible.
+// These kernels are latency-bound (tens of KB per token), so every thread
+// issues all of its 16-byte loads before it uses any of them.  Reductions use
+// a fixed tree, so results are bitwise reproducible.
 #include "internal.h"
 #include "launch.cuh"
 
@@ -15,15 +17,45 @@ namespace pae {
 
 namespace {
 
-template <typename TW>
-__device__ __forceinline__ float ldw(const TW* p);
-template <>
-__device__ __forceinline__ float ldw<float>(const float* p) { return __ldg(p); }
-template <>
-__device__ __forceinline__ float ldw<bf16>(const bf16* p) { return bf2f(*p); }
+// 8 consecutive weights as floats (16-byte loads for bf16, 2 x 16 for fp32).
+__device__ __forceinline__ void load8(const bf16* p, float* w) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    w[2 * i] = __uint_as_float(q[i] << 16);
+    w[2 * i + 1] = __uint_as_float(q[i] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void load8(const float* p, float* w) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+  w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+}
+// 4 consecutive values as floats.
+__device__ __forceinline__ void load4(const bf16* p, float* w) {
+  const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+  w[0] = __uint_as_float(u.x << 16);
+  w[1] = __uint_as_float(u.x & 0xFFFF0000u);
+  w[2] = __uint_as_float(u.y << 16);
+  w[3] = __uint_as_float(u.y & 0xFFFF0000u);
+}
+__device__ __forceinline__ void load4(const float* p, float* w) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+}
+__device__ __forceinline__ void store4(bf16* p, const float* v) {
+  const uint32_t a = (uint32_t)__bfloat16_as_ushort(f2bf(v[0])) | ((uint32_t)__bfloat16_as_ushort(f2bf(v[1])) << 16);
+  const uint32_t b = (uint32_t)__bfloat16_as_ushort(f2bf(v[2])) | ((uint32_t)__bfloat16_as_ushort(f2bf(v[3])) << 16);
+  *reinterpret_cast<uint2*>(p) = make_uint2(a, b);
+}
+__device__ __forceinline__ void store4(float* p, const float* v) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
 
-// One CTA per token.  w_in is stored transposed ([A][D]) so that the D outputs
-// read it coalesced.
+// One CTA (256 threads) per token.  w_in is stored transposed ([A][D]).
+// Requires D % 8 == 0 (16-byte weight loads).
 template <typename TW, typename TA>
 __global__ void __launch_bounds__(256) k_transition(const Shape s, const TransitionArgs a) {
   extern __shared__ float sm[];
@@ -40,32 +72,61 @@ __global__ void __launch_bounds__(256) k_transition(const Shape s, const Transit
 
   if (a.tab_out) {
     const float* hrow = a.h + (size_t)m * D;
+    const float* sc = a.tab_out + final_offset(s, 0);
+    const float* sh = a.tab_out + final_offset(s, 1);
     float ss = 0.f;
-    for (int j = tid; j < D; j += blockDim.x) {
-      const float v = hrow[j];
-      hs[j] = v;
-      ss = fmaf(v, v, ss);
+    for (int j = 4 * tid; j < D; j += 4 * blockDim.x) {
+      const float4 v = *reinterpret_cast<const float4*>(hrow + j);
+      *reinterpret_cast<float4*>(hs + j) = v;
+      ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
     }
     ss = block_sum(ss, red);
     const float r = rsqrtf(ss / (float)D + s.eps);
-    const float* sc = a.tab_out + final_offset(s, 0);
-    const float* sh = a.tab_out + final_offset(s, 1);
+    for (int j = 4 * tid; j < D; j += 4 * blockDim.x) {
+      float4 v = *reinterpret_cast<const float4*>(hs + j);
+      const float4 c = *reinterpret_cast<const float4*>(sc + j);
+      const float4 d = *reinterpret_cast<const float4*>(sh + j);
+      v.x = v.x * r * (1.f + c.x) + d.x;
+      v.y = v.y * r * (1.f + c.y) + d.y;
+      v.z = v.z * r * (1.f + c.z) + d.z;
+      v.w = v.w * r * (1.f + c.w) + d.w;
+      *reinterpret_cast<float4*>(hs + j) = v;
+    }
     __syncthreads();
-    for (int j = tid; j < D; j += blockDim.x) hs[j] = hs[j] * r * (1.f + sc[j]) + sh[j];
-    __syncthreads();
+    // v = y W_out^T + b_out: warp w takes outputs w, w+8, ...; each lane 8
+    // consecutive inputs per 256-wide chunk, all loads issued up front.
     const TW* wout = static_cast<const TW*>(a.w_out);
     const TW* bout = static_cast<const TW*>(a.b_out);
     const float dtk = a.dt[a.k_out];
-    for (int o = warp; o < A; o += nw) {
-      float acc = 0.f;
-      const TW* wr = wout + (size_t)o * D;
-      for (int j = lane; j < D; j += 32) acc = fmaf(hs[j], ldw(wr + j), acc);
-      acc = warp_sum(acc);
-      if (lane == 0) {
-        const float v = acc + ldw(bout + o);
-        const float xn = xsrc[o] + dtk * v;
-        xdst[o] = xn;
-        xs[o] = xn;
+    for (int o0 = warp; o0 < A; o0 += 4 * nw) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int j0 = 8 * lane; j0 < D; j0 += 256) {
+        float w[4][8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int o = o0 + u * nw;
+          if (o < A) load8(wout + (size_t)o * D + j0, w[u]);
+        }
+        const float4 y0 = *reinterpret_cast<const float4*>(hs + j0);
+        const float4 y1 = *reinterpret_cast<const float4*>(hs + j0 + 4);
+        const float yv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (o0 + u * nw < A)
+#pragma unroll
+            for (int t = 0; t < 8; ++t) acc[u] = fmaf(yv[t], w[u][t], acc[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int o = o0 + u * nw;
+        const float v = warp_sum(acc[u]);
+        if (lane == 0 && o < A) {
+          float bo;
+          if constexpr (sizeof(TW) == 2) bo = bf2f(bout[o]); else bo = bout[o];
+          const float xn = xsrc[o] + dtk * (v + bo);
+          xdst[o] = xn;
+          xs[o] = xn;
+        }
       }
     }
     __syncthreads();
@@ -75,28 +136,49 @@ __global__ void __launch_bounds__(256) k_transition(const Shape s, const Transit
   }
 
   if (a.tab_in) {
+    // h = x W_in^T + b_in: thread owns 4 consecutive features per 1024-wide chunk.
     const TW* winT = static_cast<const TW*>(a.w_in);  // [A][D]
     const TW* bin = static_cast<const TW*>(a.b_in);
     float* hrow = a.h + (size_t)m * D;
     float ss = 0.f;
-    for (int j = tid; j < D; j += blockDim.x) {
-      float acc = ldw(bin + j);
-      for (int o = 0; o < A; ++o) acc = fmaf(xs[o], ldw(winT + (size_t)o * D + j), acc);
-      hs[j] = acc;
-      hrow[j] = acc;
-      ss = fmaf(acc, acc, ss);
+    for (int j = 4 * tid; j < D; j += 4 * blockDim.x) {
+      float acc[4];
+      load4(bin + j, acc);
+      for (int o0 = 0; o0 < A; o0 += 16) {
+        float w[16][4];
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          if (o0 + u < A) load4(winT + (size_t)(o0 + u) * D + j, w[u]);
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          if (o0 + u < A) {
+            const float xv = xs[o0 + u];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) acc[t] = fmaf(xv, w[u][t], acc[t]);
+          }
+      }
+      *reinterpret_cast<float4*>(hs + j) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      *reinterpret_cast<float4*>(hrow + j) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      ss = fmaf(acc[0], acc[0], fmaf(acc[1], acc[1], fmaf(acc[2], acc[2], fmaf(acc[3], acc[3], ss))));
     }
     ss = block_sum(ss, red);
     const float r = rsqrtf(ss / (float)D + s.eps);
     const float* sc = a.tab_in + mod_offset(s, 0, 0, 0);
     const float* sh = a.tab_in + mod_offset(s, 0, 0, 1);
     TA* yrow = static_cast<TA*>(a.y) + (size_t)m * D;
-    for (int j = tid; j < D; j += blockDim.x) st_act<TA>(yrow + j, hs[j] * r * (1.f + sc[j]) + sh[j]);
+    for (int j = 4 * tid; j < D; j += 4 * blockDim.x) {
+      const float4 v = *reinterpret_cast<const float4*>(hs + j);
+      const float4 c = *reinterpret_cast<const float4*>(sc + j);
+      const float4 d = *reinterpret_cast<const float4*>(sh + j);
+      const float o[4] = {v.x * r * (1.f + c.x) + d.x, v.y * r * (1.f + c.y) + d.y, v.z * r * (1.f + c.z) + d.z,
+                          v.w * r * (1.f + c.w) + d.w};
+      store4(yrow + j, o);
+    }
   }
 }
 
-// One warp per token.
-template <typename TA>
+// One warp per token; the row stays in registers (NV float4 per lane).
+template <typename TA, int NV>
 __global__ void __launch_bounds__(256) k_norm(const Shape s, const float* __restrict__ h, TA* __restrict__ y,
                                               const float* __restrict__ scale, const float* __restrict__ shift,
                                               int M) {
@@ -107,12 +189,40 @@ __global__ void __launch_bounds__(256) k_norm(const Shape s, const float* __rest
   if (m >= M) return;
   const int D = s.D;
   const float* hr = h + (size_t)m * D;
+  float4 v[NV];
   float ss = 0.f;
-  for (int j = lane; j < D; j += 32) ss = fmaf(hr[j], hr[j], ss);
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int j = 4 * (lane + 32 * i);
+    v[i] = j < D ? *reinterpret_cast<const float4*>(hr + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int i = 0; i < NV; ++i) ss = fmaf(v[i].x, v[i].x, fmaf(v[i].y, v[i].y, fmaf(v[i].z, v[i].z, fmaf(v[i].w, v[i].w, ss))));
   ss = warp_sum(ss);
   const float r = rsqrtf(ss / (float)D + s.eps);
   TA* yr = y + (size_t)m * D;
-  for (int j = lane; j < D; j += 32) st_act<TA>(yr + j, hr[j] * r * (1.f + scale[j]) + shift[j]);
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int j = 4 * (lane + 32 * i);
+    if (j < D) {
+      const float4 c = *reinterpret_cast<const float4*>(scale + j);
+      const float4 d = *reinterpret_cast<const float4*>(shift + j);
+      const float o[4] = {v[i].x * r * (1.f + c.x) + d.x, v[i].y * r * (1.f + c.y) + d.y,
+                          v[i].z * r * (1.f + c.z) + d.z, v[i].w * r * (1.f + c.w) + d.w};
+      store4(yr + j, o);
+    }
+  }
+}
+
+template <typename TA>
+cudaError_t norm_dispatch(const Shape& s, const float* h, TA* y, const float* scale, const float* shift, int M,
+                          bool pdl, cudaStream_t st) {
+  const dim3 grid((M + 7) / 8), block(256);
+  const int nv = (s.D + 127) / 128;
+  if (nv <= 2) return launch_ex(k_norm<TA, 2>, grid, block, 0, st, 1, pdl, s, h, y, scale, shift, M);
+  if (nv <= 4) return launch_ex(k_norm<TA, 4>, grid, block, 0, st, 1, pdl, s, h, y, scale, shift, M);
+  if (nv <= 8) return launch_ex(k_norm<TA, 8>, grid, block, 0, st, 1, pdl, s, h, y, scale, shift, M);
+  return launch_ex(k_norm<TA, 16>, grid, block, 0, st, 1, pdl, s, h, y, scale, shift, M);
 }
 
 }  // namespace
@@ -125,12 +235,8 @@ cudaError_t launch_transition(const Shape& s, int act_bf16, const TransitionArgs
 
 cudaError_t launch_norm(const Shape& s, int act_bf16, const float* h, void* y, const float* scale, const float* shift,
                         int M, bool pdl, cudaStream_t st) {
-  const int blocks = (M + 7) / 8;
-  if (act_bf16)
-    return launch_ex(k_norm<bf16>, dim3(blocks), dim3(256), 0, st, 1, pdl, s, h, static_cast<bf16*>(y), scale, shift,
-                     M);
-  return launch_ex(k_norm<float>, dim3(blocks), dim3(256), 0, st, 1, pdl, s, h, static_cast<float*>(y), scale, shift,
-                   M);
+  if (act_bf16) return norm_dispatch<bf16>(s, h, static_cast<bf16*>(y), scale, shift, M, pdl, st);
+  return norm_dispatch<float>(s, h, static_cast<float*>(y), scale, shift, M, pdl, st);
 }
 
 }  // namespace pae

@@ -507,8 +507,8 @@ pae_status validate_config(const pae_config* c) {
     return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: n_q_heads must be a multiple of n_kv_heads");
   if (c->n_q_heads / c->n_kv_heads > 16)
     return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: at most 16 query heads per KV head");
-  if (c->width % 32 != 0 || c->width % 2 != 0)
-    return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: width must be a multiple of 32");
+  if (c->width % 32 != 0 || c->width > 2048)
+    return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: width must be a multiple of 32 and at most 2048");
   if (c->dtype == PAE_W4A16)
     return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: W4A16 kernels are not built yet");
   if (c->dtype != PAE_FP32) {

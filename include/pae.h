@@ -64,7 +64,8 @@ typedef enum {
  * quantisation group along K (must be 128; ignored otherwise).  rms_eps is the
  * epsilon of every adaptive RMSNorm.
  *
- * Supported (else PAE_ERR_UNSUPPORTED): Hq % Hkv == 0; FP32 mode: D % 32 == 0;
+ * Supported (else PAE_ERR_UNSUPPORTED): Hq % Hkv == 0, Hq/Hkv <= 16, D % 32 == 0,
+ * D <= 2048;
  * BF16/W4A16: D, Hq*d, F multiples of 128, d in {64, 128, 256}, H <= 256,
  * max_batch*H <= 4096.
  */
