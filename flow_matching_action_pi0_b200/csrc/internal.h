@@ -93,8 +93,9 @@ void launch_attention_simple(const Shape& s, int act_bf16, const void* q, const 
 struct TcPlan {
   int tn;          // token tile (MMA N), multiple of 16, <= 256
   int tok_tiles;
-  int splits;
+  int splits;      // split-K cluster size (power of two <= 16)
   int stages;
+  int recv_alias;  // split-K receive buffer overlays the stage ring
 };
 struct TcGemmArgs {
   EpiArgs e;

@@ -10,11 +10,13 @@
 //   warp 0 / lane 0  TMA producer: weight tile [128*NA][64] and token tile
 //                    [tn][64] per stage, both 128-byte swizzled, into a ring
 //   warp 1 / lane 0  MMA issuer: tcgen05.mma kind::f16 (bf16 in, fp32 in TMEM)
-//   warps 0-3        epilogue: tcgen05.ld of the accumulator (thread = weight
-//                    row = output feature, 16 token columns per load)
+//   warps 0-7        epilogue: tcgen05.ld of the accumulator (thread = weight
+//                    row = output feature, 16 token columns per load; the two
+//                    warpgroups take alternate 16-token chunks)
 // Split-K: the grid.y CTAs of one output tile form a thread-block cluster;
-// their fp32 partials are reduced on chip through distributed shared memory,
-// each CTA summing a 1/S slice of the rows over all ranks in rank order, so
+// each CTA pushes its fp32 partial rows into the owning rank's shared memory
+// (distributed shared memory stores), and after one cluster barrier every
+// rank sums its 1/S slice of the rows over all sources in rank order, so
 // results are bitwise reproducible and no partial touches global memory.
 // The weight loads of the first ring are issued before griddepcontrol.wait, so
 // under programmatic dependent launch they overlap the previous kernel.
@@ -36,26 +38,90 @@ __host__ __device__ inline uint32_t tmem_cols_for(int n) {
 }
 
 struct TcSmemLayout {
-  uint32_t a_bytes, b_bytes, stage_bytes, bar_off, total;
+  uint32_t a_bytes, b_bytes, stage_bytes, recv_off, recv_bytes, bar_off, total;
 };
 
-__host__ __device__ inline TcSmemLayout tc_layout(int na, int tn, int stages) {
+// Stages ring at offset 0; the split-K receive buffer ([na][src][token][R]
+// fp32, na*tn*128 floats) either after the ring or, when p.recv_alias, over it
+// (then an extra cluster barrier makes sure every peer's MMAs are done with
+// its ring before anyone pushes).
+__host__ __device__ inline TcSmemLayout tc_layout(int na, const TcPlan& p) {
   TcSmemLayout L;
   L.a_bytes = (uint32_t)na * 128u * 128u;
-  L.b_bytes = (uint32_t)tn * 128u;
+  L.b_bytes = (uint32_t)p.tn * 128u;
   L.stage_bytes = L.a_bytes + L.b_bytes;
-  L.bar_off = L.stage_bytes * (uint32_t)stages;
+  const uint32_t ring = L.stage_bytes * (uint32_t)p.stages;
+  L.recv_bytes = p.splits > 1 ? (uint32_t)na * (uint32_t)p.tn * 128u * 4u : 0u;
+  L.recv_off = p.recv_alias ? 0u : ring;
+  const uint32_t used = p.recv_alias ? (ring > L.recv_bytes ? ring : L.recv_bytes) : ring + L.recv_bytes;
+  L.bar_off = (used + 15u) & ~15u;
   L.total = L.bar_off + 256 + 1024;  // barriers + slack for 1024-byte alignment
   return L;
 }
 
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+// Epilogue of one output feature f over n <= 16 tokens ms[] (accumulators a0,
+// and a1 for the GeGLU up projection).  Loads that the results need (residual
+// stream, slot lengths) are issued for the whole batch before any is used.
 template <int NA>
-__global__ void __launch_bounds__(128, 1)
+__device__ __forceinline__ void epi_batch(const Shape& s, const EpiArgs& e, int f, const int* ms, const float* a0,
+                                          const float* a1, int n) {
+  if (e.epi == EPI_RESID) {
+    float hv[16];
+    const float g = e.gate[f];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < n) hv[i] = e.h[(size_t)ms[i] * s.D + f];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < n) e.h[(size_t)ms[i] * s.D + f] = fmaf(g, a0[i], hv[i]);
+  } else if (e.epi == EPI_GEGLU) {
+    bf16* u = static_cast<bf16*>(e.u);
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < n) u[(size_t)ms[i] * s.F + f] = f2bf(gelu_tanh(a0[i]) * a1[i]);
+  } else {
+    const int qd = s.Hq * s.d;
+    if (f < qd) {
+      const int hq = f / s.d, j = f - hq * s.d;
+      bf16* q = static_cast<bf16*>(e.q) + (size_t)hq * s.H * s.d + j;
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (i < n) {
+          const int b = ms[i] / s.H, t = ms[i] - b * s.H;
+          q[((size_t)b * s.Hq * s.H + t) * s.d] = f2bf(a0[i]);
+        }
+    } else {
+      const int kvd = s.Hkv * s.d;
+      const bool is_v = f >= qd + kvd;
+      const int fk = f - qd - (is_v ? kvd : 0);
+      const int g = fk / s.d, j = fk - g * s.d;
+      bf16* base = static_cast<bf16*>(is_v ? e.vc : e.kc) +
+                   ((size_t)e.layer * s.Bmax * s.Hkv + g) * s.Ptot * s.d + j;
+      int lens[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (i < n) lens[i] = e.lens[ms[i] / s.H];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (i < n) {
+          const int b = ms[i] / s.H, t = ms[i] - b * s.H;
+          base[((size_t)b * s.Hkv * s.Ptot + lens[i] + t) * s.d] = f2bf(a0[i]);
+        }
+    }
+  }
+}
+
+template <int NA>
+__global__ void __launch_bounds__(256, 2)
     k_tc_gemm(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, const Shape s,
               const TcPlan p, const TcGemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const TcSmemLayout L = tc_layout(NA, p.tn, p.stages);
+  const TcSmemLayout L = tc_layout(NA, p);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* empty = full + p.stages;
   uint64_t* accf = empty + p.stages;
@@ -96,8 +162,8 @@ __global__ void __launch_bounds__(128, 1)
     // ---------------------------------------------------------------- producer
     // Weight tiles do not depend on the previous kernel: the first ring's worth
     // is requested before waiting for it (programmatic dependent launch).
-    // weights are streamed once per step when one token tile covers the batch;
-    // otherwise the other token tiles re-read them from L2
+    // Weights are streamed once per step when one token tile covers the batch;
+    // otherwise the other token tiles re-read them from L2.
     const uint64_t pol_w = p.tok_tiles == 1 ? policy_evict_first() : policy_evict_last();
     const int npre = nkb < p.stages ? nkb : p.stages;
     const int wrow = a.w_row0 + ntile * 128 * NA;
@@ -161,77 +227,87 @@ __global__ void __launch_bounds__(128, 1)
   // CTA-uniform decision: the TMEM loads below are warp-collective.
   const bool ok = __syncthreads_and(acc_ok ? 1 : 0) != 0 && s_flag[0] == 0;
 
-  const int row = warp * 32 + lane;
-  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+  // Eight epilogue warps: warp w reads TMEM lanes 32*(w%4).. (its rows) and
+  // the 16-token chunks c with c % 2 == w / 4.
+  const int quarter = warp & 3, half = warp >> 2;
+  const int row = quarter * 32 + lane;
+  const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
   const int mbase = ttile * p.tn;
   const EpiArgs& e = a.e;
+  const int nchunks = p.tn / 16;
 
   if (p.splits == 1) {
     const int f = ntile * 128 + row;
     if (ok) {
-      for (int c0 = 0; c0 < p.tn; c0 += 16) {
+      for (int c = half; c < nchunks; c += 2) {
         float v0[16], v1[16];
-        tmem_ld16(trow + c0, v0);
-        if (NA == 2) tmem_ld16(trow + p.tn + c0, v1);
+        tmem_ld16(trow + c * 16, v0);
+        if (NA == 2) tmem_ld16(trow + p.tn + c * 16, v1);
         tmem_ld_wait();
+        const int m0 = mbase + c * 16;
+        int ms[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int m = mbase + c0 + j;
-          if (m < e.M && f < a.N) epi_apply<bf16>(s, e, m, f, v0[j], NA == 2 ? v1[j] : 0.f);
-        }
+        for (int j = 0; j < 16; ++j) ms[j] = m0 + j;
+        const int n = min(16, e.M - m0);
+        if (n > 0 && f < a.N) epi_batch<NA>(s, e, f, ms, v0, v1, n);
       }
     }
   } else {
-    // Split-K inside a cluster of p.splits CTAs: each parks its fp32 partial
-    // in its own shared memory, token-major ([na][token][128 rows]), then CTA
-    // rank r sums rows [r*R, r*R+R) over all ranks in rank order through
-    // distributed shared memory and runs the epilogue on them.
-    float* red = reinterpret_cast<float*>(smem);
+    // Split-K inside a cluster of S CTAs: rank r owns rows [r*R, r*R+R).  Every
+    // CTA pushes each row's partial into the owner's receive buffer through
+    // distributed shared memory; after one cluster barrier each owner sums its
+    // rows over the S sources in rank order, reading only local memory.
+    const int S = p.splits, R = 128 / S;
+    const uint32_t rank = cluster_rank();
+    float* recv = reinterpret_cast<float*>(smem + L.recv_off);
+    if (p.recv_alias) cluster_sync();  // every peer's MMAs are done with the ring
     if (ok) {
-      for (int c0 = 0; c0 < p.tn; c0 += 16) {
+      const int owner = row / R, rr = row - owner * R;
+      const uint32_t dst = map_cluster(smem_u32(recv), (uint32_t)owner);
+      for (int c = half; c < nchunks; c += 2) {
         float v0[16], v1[16];
-        tmem_ld16(trow + c0, v0);
-        if (NA == 2) tmem_ld16(trow + p.tn + c0, v1);
+        tmem_ld16(trow + c * 16, v0);
+        if (NA == 2) tmem_ld16(trow + p.tn + c * 16, v1);
         tmem_ld_wait();
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          red[(c0 + j) * 128 + row] = v0[j];
-          if (NA == 2) red[(p.tn + c0 + j) * 128 + row] = v1[j];
+          const uint32_t col = (uint32_t)(c * 16 + j);
+          st_cluster_f32(dst + ((((uint32_t)0 * S + rank) * p.tn + col) * R + rr) * 4u, v0[j]);
+          if (NA == 2) st_cluster_f32(dst + ((((uint32_t)1 * S + rank) * p.tn + col) * R + rr) * 4u, v1[j]);
         }
       }
     }
     cluster_sync();
-    const int S = p.splits;
-    const uint32_t rank = cluster_rank();
-    const int R = 128 / S;
-    const uint32_t red_base = smem_u32(red);
-    const int any_ok = ok ? 1 : 0;
-    if (any_ok) {
-      for (int el = threadIdx.x; el < R * p.tn; el += 128) {
-        const int rr = el % R, col = el / R;
-        const int rw = (int)rank * R + rr;
-        const int m = mbase + col, f = ntile * 128 + rw;
-        const uint32_t off0 = (uint32_t)((col * 128 + rw) * 4);
-        const uint32_t off1 = (uint32_t)(((p.tn + col) * 128 + rw) * 4);
-        // issue every rank's load first (they pipeline), then sum in rank order
-        float v0[16], v1[16];
+    if (ok) {
+      // Thread t keeps one row (t % R) and walks the tokens t / R, t / R + 256 / R, ...
+      const int rr = threadIdx.x % R;
+      const int f = ntile * 128 + (int)rank * R + rr;
+      const int cstep = 256 / R;
+      for (int c0 = threadIdx.x / R; c0 < p.tn; c0 += 16 * cstep) {
+        float s0[16], s1[16];
+        int ms[16];
+        int n = 0;
 #pragma unroll
-        for (int q = 0; q < 16; ++q)
-          if (q < S) {
-            v0[q] = ld_cluster_f32(map_cluster(red_base + off0, (uint32_t)q));
-            if (NA == 2) v1[q] = ld_cluster_f32(map_cluster(red_base + off1, (uint32_t)q));
-          }
-        float s0 = 0.f, s1 = 0.f;
+        for (int i = 0; i < 16; ++i) {
+          const int col = c0 + i * cstep;
+          s0[i] = 0.f;
+          s1[i] = 0.f;
+          ms[i] = mbase + col;
+          if (col < p.tn && mbase + col < e.M) n = i + 1;
+        }
+        for (int src = 0; src < S; ++src) {
 #pragma unroll
-        for (int q = 0; q < 16; ++q)
-          if (q < S) {
-            s0 += v0[q];
-            if (NA == 2) s1 += v1[q];
+          for (int i = 0; i < 16; ++i) {
+            const int col = c0 + i * cstep;
+            if (i < n) {
+              s0[i] += recv[((0 * S + src) * p.tn + col) * R + rr];
+              if (NA == 2) s1[i] += recv[((1 * S + src) * p.tn + col) * R + rr];
+            }
           }
-        if (m < e.M && f < a.N) epi_apply<bf16>(s, e, m, f, s0, s1);
+        }
+        if (n > 0 && f < a.N) epi_batch<NA>(s, e, f, ms, s0, s1, n);
       }
     }
-    cluster_sync();  // peers may still be reading this CTA's partial
   }
 
   tc_fence_before();
@@ -241,7 +317,7 @@ __global__ void __launch_bounds__(128, 1)
 
 }  // namespace
 
-size_t tc_gemm_smem_bytes(int na, const TcPlan& p) { return tc_layout(na, p.tn, p.stages).total; }
+size_t tc_gemm_smem_bytes(int na, const TcPlan& p) { return tc_layout(na, p).total; }
 
 cudaError_t tc_gemm_init() {
   const int max_smem = 227 * 1024;
@@ -257,8 +333,8 @@ cudaError_t launch_tc_gemm(const Shape& s, const CUtensorMap* tmW, const CUtenso
   const int ntiles = (a.N + 127) / 128;
   dim3 grid(ntiles, p.splits, p.tok_tiles);
   const size_t smem = tc_gemm_smem_bytes(na, p);
-  if (na == 2) return launch_ex(k_tc_gemm<2>, grid, dim3(128), smem, st, p.splits, pdl, *tmW, *tmX, s, p, a);
-  return launch_ex(k_tc_gemm<1>, grid, dim3(128), smem, st, p.splits, pdl, *tmW, *tmX, s, p, a);
+  if (na == 2) return launch_ex(k_tc_gemm<2>, grid, dim3(256), smem, st, p.splits, pdl, *tmW, *tmX, s, p, a);
+  return launch_ex(k_tc_gemm<1>, grid, dim3(256), smem, st, p.splits, pdl, *tmW, *tmX, s, p, a);
 }
 
 }  // namespace pae

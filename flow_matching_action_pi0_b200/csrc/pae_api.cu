@@ -18,7 +18,7 @@
 #include <string>
 #include <vector>
 
-#include "../../include/pae.h"
+#include "pae.h"
 #include "internal.h"
 
 using namespace pae;
@@ -177,17 +177,27 @@ TcPlan plan_gemm(int M, int nfeat, int K, int na) {
   const int base = ((nfeat + 127) / 128) * p.tok_tiles;
   const int nkb = K / 64;
   const uint32_t stage = (uint32_t)na * 16384u + (uint32_t)p.tn * 128u;
-  const uint32_t red = (uint32_t)na * p.tn * 128u * 4u;  // parked fp32 partial
-  const bool small = p.tn <= 64;
-  const uint32_t budget = small ? 100u * 1024u : 200u * 1024u;
+  const uint32_t recv = (uint32_t)na * p.tn * 128u * 4u;  // split-K receive buffer
+  const bool small = p.tn <= 64;  // two CTAs per SM (shared memory and the 128-register cap allow it)
+  const uint32_t budget = small ? 110u * 1024u : 200u * 1024u;
   const int target = small ? 2 * 148 : 148;
   p.splits = 1;
   for (int sp = 2; sp <= 16; sp *= 2)
-    if (nkb % sp == 0 && base * sp <= target && red <= budget) p.splits = sp;
-  int st = (int)(budget / stage);
-  st = std::max(2, std::min(st, 6));
+    if (nkb % sp == 0 && base * sp <= target && recv <= budget) p.splits = sp;
+  int st = std::max(2, std::min((int)(budget / stage), 6));
   st = std::min(st, std::max(2, nkb / p.splits));
-  if (p.splits > 1) st = std::max(st, (int)((red + stage - 1) / stage));
+  p.recv_alias = 0;
+  if (p.splits > 1) {
+    // a separate receive buffer saves a cluster barrier; overlay it on the
+    // ring when both do not fit
+    int st_sep = std::min(st, (int)((budget - std::min(budget, recv)) / stage));
+    if (st_sep >= 2) {
+      st = st_sep;
+    } else {
+      p.recv_alias = 1;
+      st = std::max(st, (int)((recv + stage - 1) / stage));
+    }
+  }
   p.stages = st;
   return p;
 }
