@@ -66,10 +66,10 @@ __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
 // Epilogue of one output feature f over n <= 16 tokens ms[] (accumulators a0,
 // and a1 for the GeGLU up projection).  Loads that the results need (residual
 // stream, slot lengths) are issued for the whole batch before any is used.
-template <int NA>
+template <int EPI>
 __device__ __forceinline__ void epi_batch(const Shape& s, const EpiArgs& e, int f, const int* ms, const float* a0,
                                           const float* a1, int n) {
-  if (e.epi == EPI_RESID) {
+  if constexpr (EPI == EPI_RESID) {
     float hv[16];
     const float g = e.gate[f];
 #pragma unroll
@@ -78,7 +78,7 @@ __device__ __forceinline__ void epi_batch(const Shape& s, const EpiArgs& e, int 
 #pragma unroll
     for (int i = 0; i < 16; ++i)
       if (i < n) e.h[(size_t)ms[i] * s.D + f] = fmaf(g, a0[i], hv[i]);
-  } else if (e.epi == EPI_GEGLU) {
+  } else if constexpr (EPI == EPI_GEGLU) {
     bf16* u = static_cast<bf16*>(e.u);
 #pragma unroll
     for (int i = 0; i < 16; ++i)
@@ -115,7 +115,7 @@ __device__ __forceinline__ void epi_batch(const Shape& s, const EpiArgs& e, int 
   }
 }
 
-template <int NA>
+template <int NA, int EPI, bool SPLIT>
 __global__ void __launch_bounds__(256, 2)
     k_tc_gemm(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, const Shape s,
               const TcPlan p, const TcGemmArgs a) {
@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(256, 2)
   const EpiArgs& e = a.e;
   const int nchunks = p.tn / 16;
 
-  if (p.splits == 1) {
+  if constexpr (!SPLIT) {
     const int f = ntile * 128 + row;
     if (ok) {
       for (int c = half; c < nchunks; c += 2) {
@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
         for (int j = 0; j < 16; ++j) ms[j] = m0 + j;
         const int n = min(16, e.M - m0);
-        if (n > 0 && f < a.N) epi_batch<NA>(s, e, f, ms, v0, v1, n);
+        if (n > 0 && f < a.N) epi_batch<EPI>(s, e, f, ms, v0, v1, n);
       }
     }
   } else {
@@ -305,7 +305,7 @@ __global__ void __launch_bounds__(256, 2)
             }
           }
         }
-        if (n > 0 && f < a.N) epi_batch<NA>(s, e, f, ms, s0, s1, n);
+        if (n > 0 && f < a.N) epi_batch<EPI>(s, e, f, ms, s0, s1, n);
       }
     }
   }
@@ -315,26 +315,46 @@ __global__ void __launch_bounds__(256, 2)
   if (warp == 0) tmem_dealloc(tmem, ncols);
 }
 
+size_t smem_bytes_impl(int na, const TcPlan& p) { return tc_layout(na, p).total; }
+
+template <int NA, int EPI, bool SPLIT>
+cudaError_t init_one() {
+  cudaError_t e = cudaFuncSetAttribute(k_tc_gemm<NA, EPI, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       227 * 1024);
+  if (e == cudaSuccess && SPLIT)
+    e = cudaFuncSetAttribute(k_tc_gemm<NA, EPI, SPLIT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
+}
+
+template <int NA, int EPI>
+cudaError_t launch_one(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* tmX, const TcPlan& p,
+                       const TcGemmArgs& a, bool pdl, cudaStream_t st) {
+  dim3 grid((a.N + 127) / 128, p.splits, p.tok_tiles);
+  const size_t smem = smem_bytes_impl(NA, p);
+  if (p.splits > 1)
+    return launch_ex(k_tc_gemm<NA, EPI, true>, grid, dim3(256), smem, st, p.splits, pdl, *tmW, *tmX, s, p, a);
+  return launch_ex(k_tc_gemm<NA, EPI, false>, grid, dim3(256), smem, st, 1, pdl, *tmW, *tmX, s, p, a);
+}
+
 }  // namespace
 
-size_t tc_gemm_smem_bytes(int na, const TcPlan& p) { return tc_layout(na, p).total; }
+size_t tc_gemm_smem_bytes(int na, const TcPlan& p) { return smem_bytes_impl(na, p); }
 
 cudaError_t tc_gemm_init() {
-  const int max_smem = 227 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(k_tc_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_tc_gemm<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_tc_gemm<1>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_tc_gemm<2>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaError_t e = init_one<1, EPI_QKV, false>();
+  if (e == cudaSuccess) e = init_one<1, EPI_QKV, true>();
+  if (e == cudaSuccess) e = init_one<1, EPI_RESID, false>();
+  if (e == cudaSuccess) e = init_one<1, EPI_RESID, true>();
+  if (e == cudaSuccess) e = init_one<2, EPI_GEGLU, false>();
+  if (e == cudaSuccess) e = init_one<2, EPI_GEGLU, true>();
   return e;
 }
 
 cudaError_t launch_tc_gemm(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* tmX, int na, const TcPlan& p,
                            const TcGemmArgs& a, bool pdl, cudaStream_t st) {
-  const int ntiles = (a.N + 127) / 128;
-  dim3 grid(ntiles, p.splits, p.tok_tiles);
-  const size_t smem = tc_gemm_smem_bytes(na, p);
-  if (na == 2) return launch_ex(k_tc_gemm<2>, grid, dim3(256), smem, st, p.splits, pdl, *tmW, *tmX, s, p, a);
-  return launch_ex(k_tc_gemm<1>, grid, dim3(256), smem, st, p.splits, pdl, *tmW, *tmX, s, p, a);
+  if (na == 2) return launch_one<2, EPI_GEGLU>(s, tmW, tmX, p, a, pdl, st);
+  if (a.e.epi == EPI_QKV) return launch_one<1, EPI_QKV>(s, tmW, tmX, p, a, pdl, st);
+  return launch_one<1, EPI_RESID>(s, tmW, tmX, p, a, pdl, st);
 }
 
 }  // namespace pae
