@@ -363,13 +363,16 @@ def run_minimal(args, cfg):
     W = wl.make_weights(cfg)
     ex, *_ = setup_context(cfg, W, cfg.batch, wl.prefix_lengths(cfg))
     ex.set_option(fm.PAE_OPT_PDL, args.pdl)
+    if args.max_splitk:
+        ex.set_option(fm.PAE_OPT_MAX_SPLITK, args.max_splitk)
     nd = torch.from_numpy(wl.make_noise(cfg)).cuda()
     od = torch.empty_like(nd)
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
         ms = timed(lambda: ex.denoise(nd, od, stream), args.steps, args.warmup, stream, lambda: None)
     k = ex.query(fm.PAE_Q_GRAPH_KERNELS, cfg.batch)
-    print(json.dumps({"workload": cfg.name, "pdl": args.pdl, "ms_per_step": ms, "graph_kernels": k,
+    print(json.dumps({"workload": cfg.name, "pdl": args.pdl, "max_splitk": args.max_splitk, "ms_per_step": ms,
+                      "splits": ex.query(fm.PAE_Q_SPLITS, cfg.batch), "graph_kernels": k,
                       "launches_before_timed": 1 + cfg.batch + 4 + args.warmup * k}), flush=True)
     ex.close()
     return 0
@@ -470,6 +473,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--minimal", action="store_true", help="only warm-up and timed calls (for profilers)")
     ap.add_argument("--pdl", type=int, default=1, help="programmatic dependent launch inside the loop (1/0)")
+    ap.add_argument("--max-splitk", type=int, default=0, help="cap on the projection split-K (0: library default)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

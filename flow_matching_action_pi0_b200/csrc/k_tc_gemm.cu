@@ -59,6 +59,25 @@ __host__ __device__ inline TcSmemLayout tc_layout(int na, const TcPlan& p) {
   return L;
 }
 
+__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// Epilogue of one output (token m, feature f); compact on purpose.
+template <int EPI>
+__device__ __forceinline__ void epi_one(const Shape& s, const EpiArgs& e, int f, int m, float a0, float a1) {
+  if constexpr (EPI == EPI_RESID) {
+    float* hp = e.h + (size_t)m * s.D + f;
+    *hp = fmaf(e.gate[f], a0, *hp);
+  } else if constexpr (EPI == EPI_GEGLU) {
+    static_cast<bf16*>(e.u)[(size_t)m * s.F + f] = f2bf(gelu_tanh(a0) * a1);
+  } else {
+    epi_qkv<bf16>(s, e, m, f, a0);
+  }
+}
+
 __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
@@ -283,29 +302,21 @@ __global__ void __launch_bounds__(256, 2)
       const int rr = threadIdx.x % R;
       const int f = ntile * 128 + (int)rank * R + rr;
       const int cstep = 256 / R;
-      for (int c0 = threadIdx.x / R; c0 < p.tn; c0 += 16 * cstep) {
-        float s0[16], s1[16];
-        int ms[16];
-        int n = 0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int col = c0 + i * cstep;
-          s0[i] = 0.f;
-          s1[i] = 0.f;
-          ms[i] = mbase + col;
-          if (col < p.tn && mbase + col < e.M) n = i + 1;
-        }
+      const uint32_t rbase = smem_u32(recv) + (uint32_t)rr * 4u;
+      const uint32_t src_stride = (uint32_t)p.tn * R * 4u;
+      const uint32_t na_stride = (uint32_t)S * src_stride;
+#pragma unroll 1
+      for (int col = threadIdx.x / R; col < p.tn; col += cstep) {
+        const int m = mbase + col;
+        if (m >= e.M || f >= a.N) break;
+        const uint32_t addr = rbase + (uint32_t)col * R * 4u;
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll 1
         for (int src = 0; src < S; ++src) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int col = c0 + i * cstep;
-            if (i < n) {
-              s0[i] += recv[((0 * S + src) * p.tn + col) * R + rr];
-              if (NA == 2) s1[i] += recv[((1 * S + src) * p.tn + col) * R + rr];
-            }
-          }
+          s0 += ld_shared_f32(addr + src * src_stride);
+          if (NA == 2) s1 += ld_shared_f32(addr + na_stride + src * src_stride);
         }
-        if (n > 0 && f < a.N) epi_batch<EPI>(s, e, f, ms, s0, s1, n);
+        epi_one<EPI>(s, e, f, m, s0, s1);
       }
     }
   }

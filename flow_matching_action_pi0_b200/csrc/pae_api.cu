@@ -95,6 +95,7 @@ struct pae_ctx {
   long long wait_ns = 2000000000LL;
   bool use_graph = true;
   bool use_pdl = true;
+  int max_splitk = 8;
   std::map<int, Plan> plans;
   Plan* last_plan = nullptr;
   unsigned profile_mask = 0;
@@ -169,7 +170,7 @@ pae_status make_map(pae_ctx* ctx, CUtensorMap* m, const void* base, uint64_t inn
 // divides the 64-wide K blocks) fills the 148 SMs when the tile count is small;
 // small token tiles keep shared memory under half an SM so that two CTAs (or a
 // CTA and its successor under PDL) fit per SM.
-TcPlan plan_gemm(int M, int nfeat, int K, int na) {
+TcPlan plan_gemm(int M, int nfeat, int K, int na, int max_splits = 16) {
   TcPlan p{};
   p.tok_tiles = (M + 255) / 256;
   int per = (M + p.tok_tiles - 1) / p.tok_tiles;
@@ -182,9 +183,11 @@ TcPlan plan_gemm(int M, int nfeat, int K, int na) {
   const uint32_t budget = small ? 110u * 1024u : 200u * 1024u;
   const int target = small ? 2 * 148 : 148;
   p.splits = 1;
-  for (int sp = 2; sp <= 16; sp *= 2)
+  for (int sp = 2; sp <= std::min(16, max_splits); sp *= 2)
     if (nkb % sp == 0 && base * sp <= target && recv <= budget) p.splits = sp;
-  int st = std::max(2, std::min((int)(budget / stage), 6));
+  // without split-K a CTA streams a long K range: give it a deep ring
+  const uint32_t ring_budget = p.splits == 1 ? 200u * 1024u : budget;
+  int st = std::max(2, std::min((int)(ring_budget / stage), 8));
   st = std::min(st, std::max(2, nkb / p.splits));
   p.recv_alias = 0;
   if (p.splits > 1) {
@@ -222,10 +225,10 @@ pae_status build_plan(pae_ctx* ctx, int B, Plan* P) {
   P->B = B;
   P->M = B * s.H;
   if (!ctx->act_bf16) return PAE_OK;
-  P->qkv = plan_gemm(P->M, s.qkv_rows, s.D, 1);
-  P->o = plan_gemm(P->M, s.D, s.attn_dim, 1);
-  P->gu = plan_gemm(P->M, s.F, s.D, 2);
-  P->down = plan_gemm(P->M, s.D, s.F, 1);
+  P->qkv = plan_gemm(P->M, s.qkv_rows, s.D, 1, ctx->max_splitk);
+  P->o = plan_gemm(P->M, s.D, s.attn_dim, 1, ctx->max_splitk);
+  P->gu = plan_gemm(P->M, s.F, s.D, 2, ctx->max_splitk);
+  P->down = plan_gemm(P->M, s.D, s.F, 1, ctx->max_splitk);
   P->attn = plan_attn(s, B);
   const uint64_t Mmax = (uint64_t)s.Bmax * s.H;
   pae_status st;
@@ -839,6 +842,15 @@ pae_status pae_set_option(pae_ctx* ctx, int option, long long value) {
       if (value <= 0) return fail(ctx, PAE_ERR_ARG, "wait limit must be positive");
       ctx->wait_ns = value * 1000LL;
       drop_graphs(ctx);  // captured launches hold the old limit
+      return PAE_OK;
+    case PAE_OPT_MAX_SPLITK:
+      if (value < 1 || value > 16) return fail(ctx, PAE_ERR_ARG, "max split-K must be in [1, 16]");
+      if ((int)value != ctx->max_splitk) {
+        drop_graphs(ctx);
+        ctx->plans.clear();
+        ctx->last_plan = nullptr;
+      }
+      ctx->max_splitk = (int)value;
       return PAE_OK;
     case PAE_OPT_PDL:
       if ((value != 0) != ctx->use_pdl) drop_graphs(ctx);

@@ -154,8 +154,11 @@ pae_status pae_denoise_steps(pae_ctx* ctx, const float* x_in, float* x_out, int 
  * kernels directly.  PAE_OPT_WAIT_LIMIT_US (default 2000000): bound of every
  * device-side wait, in microseconds.  PAE_OPT_PDL (default 1, bf16 modes):
  * programmatic dependent launch between the loop's kernels, so a kernel's
- * weight loads overlap its predecessor's tail; 0 serialises the kernels. */
-enum { PAE_OPT_USE_GRAPH = 1, PAE_OPT_WAIT_LIMIT_US = 2, PAE_OPT_PDL = 4 };
+ * weight loads overlap its predecessor's tail; 0 serialises the kernels.
+ * PAE_OPT_MAX_SPLITK (default 8, range 1..16): largest split-K cluster the
+ * projection planner may choose (a tuning knob; results stay within the
+ * parity tolerance, bitwise identical only for the same setting). */
+enum { PAE_OPT_USE_GRAPH = 1, PAE_OPT_WAIT_LIMIT_US = 2, PAE_OPT_PDL = 4, PAE_OPT_MAX_SPLITK = 5 };
 pae_status pae_set_option(pae_ctx* ctx, int option, long long value);
 
 /* Kernel classes for profiling, as bit positions of PAE_OPT_PROFILE. */
