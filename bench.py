@@ -447,6 +447,19 @@ def run_ours(args, cfg):
             "note": "same weights as the batch-1 line; 32 independent 968-token prefixes"}}
         r32.pop("ex").close()
         del r32
+    if args.secondary and cfg.name == wl.PI05_BF16_BS1.name:
+        c4 = wl.PI05_W4A16_BS1
+        W4 = wl.make_weights(c4)
+        r4 = measure(c4, W4, c4.batch, args, stream, barrier, maxr, with_e2e=False, gpu_index=gpu_index)
+        rl4, loop4, sh4 = roofline_for(c4, c4.batch, r4, peaks, peak_kind, r4["lens"])
+        line.setdefault("secondary", {})[c4.name] = {
+            "value": ws * c4.batch / (r4["ms_per_step"] * 1e-3), "unit": "chunks/s",
+            "ms_per_step": r4["ms_per_step"], "roofline": rl4, "loop_roofline": loop4, "kernel_shares": sh4,
+            "clocks": r4["clocks"],
+            "kernels_ms_per_launch": {c: v["ms_per_launch"] for c, v in r4["kernels"].items()},
+            "note": "int4 weights (group 128, bf16 scales), bf16 activations"}
+        r4.pop("ex").close()
+        del r4, W4
     if args.cpu_baseline and ws == 1 and rank == 0:
         t = oracle_sample_time(cfg, W, *wl.make_prefix(cfg, lengths=lens[:1]), wl.make_noise(cfg, batch=1),
                                cfg.steps)

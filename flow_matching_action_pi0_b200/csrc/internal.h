@@ -99,6 +99,7 @@ struct TcPlan {
 };
 struct TcGemmArgs {
   EpiArgs e;
+  const bf16* scales;  // int4 weights: [rows][K/128] group scales (null: bf16 weights)
   int N;           // output features (GEGLU: F)
   int K;
   int w_row0;      // first row of this layer's matrix inside the stacked weight map
@@ -106,7 +107,7 @@ struct TcGemmArgs {
 };
 cudaError_t launch_tc_gemm(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* tmX, int na,
                            const TcPlan& p, const TcGemmArgs& a, bool pdl, cudaStream_t st);
-size_t tc_gemm_smem_bytes(int na, const TcPlan& p);
+size_t tc_gemm_smem_bytes(int na, const TcPlan& p, bool w4);
 cudaError_t tc_gemm_init();  // once per process: opt in to large dynamic shared memory
 
 // ------------------------------------------------------ tcgen05 attention

@@ -20,6 +20,10 @@
 // results are bitwise reproducible and no partial touches global memory.
 // The weight loads of the first ring are issued before griddepcontrol.wait, so
 // under programmatic dependent launch they overlap the previous kernel.
+// int4 weights (W4A16): TMA brings the packed [rows][32 bytes] tile per K
+// block; warps 4-7 dequantise it into the bf16 A tile (code * group scale,
+// rounded once) and arrive on a barrier the MMA thread waits for; the rest of
+// the pipeline and the epilogues are shared with the bf16 path.
 #include "epilogue.cuh"
 #include "launch.cuh"
 
@@ -38,18 +42,21 @@ __host__ __device__ inline uint32_t tmem_cols_for(int n) {
 }
 
 struct TcSmemLayout {
-  uint32_t a_bytes, b_bytes, stage_bytes, recv_off, recv_bytes, bar_off, total;
+  uint32_t a_bytes, b_bytes, raw_bytes, stage_bytes, recv_off, recv_bytes, bar_off, total;
 };
 
-// Stages ring at offset 0; the split-K receive buffer ([na][src][token][R]
-// fp32, na*tn*128 floats) either after the ring or, when p.recv_alias, over it
-// (then an extra cluster barrier makes sure every peer's MMAs are done with
-// its ring before anyone pushes).
-__host__ __device__ inline TcSmemLayout tc_layout(int na, const TcPlan& p) {
+// Per stage: the bf16 weight tile A ([128*na][64], 128-byte swizzled), the
+// token tile B ([tn][64], swizzled) and, for int4 weights, the raw packed tile
+// ([128*na][32 bytes]) that the dequantising warps turn into A.  The split-K
+// receive buffer ([na][src][token][R] fp32, na*tn*128 floats) follows the ring
+// or, when p.recv_alias, overlays it (then an extra cluster barrier makes sure
+// every peer's MMAs are done with its ring before anyone pushes).
+__host__ __device__ inline TcSmemLayout tc_layout(int na, const TcPlan& p, bool w4) {
   TcSmemLayout L;
   L.a_bytes = (uint32_t)na * 128u * 128u;
   L.b_bytes = (uint32_t)p.tn * 128u;
-  L.stage_bytes = L.a_bytes + L.b_bytes;
+  L.raw_bytes = w4 ? (uint32_t)na * 128u * 32u : 0u;
+  L.stage_bytes = L.a_bytes + L.b_bytes + L.raw_bytes;
   const uint32_t ring = L.stage_bytes * (uint32_t)p.stages;
   L.recv_bytes = p.splits > 1 ? (uint32_t)na * (uint32_t)p.tn * 128u * 4u : 0u;
   L.recv_off = p.recv_alias ? 0u : ring;
@@ -134,16 +141,28 @@ __device__ __forceinline__ void epi_batch(const Shape& s, const EpiArgs& e, int 
   }
 }
 
-template <int NA, int EPI, bool SPLIT>
+// Two packed int4 codes (nibbles at bits 4i and 16+4i, two's complement)
+// -> bf16x2 of code * scale, rounded once (to nearest even).  (n ^ 8) | 0x4300
+// is the bf16 of 128 + (code + 8); subtracting 136 is exact.
+__device__ __forceinline__ uint32_t dequant_pair(uint32_t w, int i, __nv_bfloat162 sc) {
+  const uint32_t t = (((w >> (4 * i)) & 0x000F000Fu) ^ 0x00080008u) | 0x43004300u;
+  __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&t);
+  const __nv_bfloat162 off = __floats2bfloat162_rn(136.f, 136.f);
+  v = __hmul2(__hsub2(v, off), sc);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <int NA, int EPI, bool SPLIT, bool W4>
 __global__ void __launch_bounds__(256, 2)
     k_tc_gemm(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, const Shape s,
               const TcPlan p, const TcGemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const TcSmemLayout L = tc_layout(NA, p);
+  const TcSmemLayout L = tc_layout(NA, p, W4);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* empty = full + p.stages;
-  uint64_t* accf = empty + p.stages;
+  uint64_t* a_ready = empty + p.stages;  // int4 weights: dequantised A tile written
+  uint64_t* accf = a_ready + p.stages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
   volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);  // [0] abort
 
@@ -158,6 +177,7 @@ __global__ void __launch_bounds__(256, 2)
     for (int i = 0; i < p.stages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
+      mbar_init(&a_ready[i], 128);
     }
     mbar_init(accf, 1);
     s_flag[0] = 0;
@@ -186,9 +206,13 @@ __global__ void __launch_bounds__(256, 2)
     const uint64_t pol_w = p.tok_tiles == 1 ? policy_evict_first() : policy_evict_last();
     const int npre = nkb < p.stages ? nkb : p.stages;
     const int wrow = a.w_row0 + ntile * 128 * NA;
+    const uint32_t wdst = W4 ? L.a_bytes + L.b_bytes : 0u;         // raw tile or A tile
+    const int wx = W4 ? (k0 + 0) / 2 : k0;                            // packed: two codes per byte
+    const int wstep = W4 ? 32 : 64;
+    const uint32_t tx = W4 ? L.raw_bytes + L.b_bytes : L.a_bytes + L.b_bytes;
     for (int kb = 0; kb < npre; ++kb) {
-      mbar_arrive_expect_tx(&full[kb], L.stage_bytes);
-      tma_load_2d_hint(smem + (size_t)kb * L.stage_bytes, &tmW, k0 + kb * 64, wrow, &full[kb], pol_w);
+      mbar_arrive_expect_tx(&full[kb], tx);
+      tma_load_2d_hint(smem + (size_t)kb * L.stage_bytes + wdst, &tmW, wx + kb * wstep, wrow, &full[kb], pol_w);
     }
     pdl_wait();
     for (int kb = 0; kb < npre; ++kb)
@@ -202,8 +226,8 @@ __global__ void __launch_bounds__(256, 2)
         break;
       }
       uint8_t* sa = smem + (size_t)st * L.stage_bytes;
-      mbar_arrive_expect_tx(&full[st], L.stage_bytes);
-      tma_load_2d_hint(sa, &tmW, k0 + kb * 64, wrow, &full[st], pol_w);
+      mbar_arrive_expect_tx(&full[st], tx);
+      tma_load_2d_hint(sa + wdst, &tmW, wx + kb * wstep, wrow, &full[st], pol_w);
       tma_load_2d(sa + L.a_bytes, &tmX, k0 + kb * 64, ttile * p.tn, &full[st]);
       issued = kb + 1;
     }
@@ -215,7 +239,8 @@ __global__ void __launch_bounds__(256, 2)
     const uint32_t idesc = idesc_bf16(128, p.tn);
     for (int kb = 0; kb < nkb; ++kb) {
       const int st = kb % p.stages;
-      if (!mbar_wait(&full[st], (kb / p.stages) & 1, a.err.wait_ns)) {
+      if (!mbar_wait(&full[st], (kb / p.stages) & 1, a.err.wait_ns) ||
+          (W4 && !mbar_wait(&a_ready[st], (kb / p.stages) & 1, a.err.wait_ns))) {
         s_flag[0] = 1;
         set_error(a.err, DEV_TIMEOUT);
         break;
@@ -235,6 +260,44 @@ __global__ void __launch_bounds__(256, 2)
       umma_commit(&empty[st]);  // stage reusable once these MMAs have read it
     }
     umma_commit(accf);  // always issued, so the epilogue wait ends
+  } else if (W4 && warp >= 4) {
+    // ---------------------------------------------------------------- dequant
+    // Thread t owns weight row t (and t + 128 for the gate/up pair): its 64
+    // packed codes per K block become 64 bf16 code * scale values, written as
+    // eight 16-byte chunks in the 128-byte swizzled layout the MMA reads.
+    const int dr = threadIdx.x - 128;
+    const int gpr = a.K / 128;  // scale groups per weight row
+    const bf16* srow0 = a.scales + (size_t)(a.w_row0 + ntile * 128 * NA + dr) * gpr;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int st = kb % p.stages;
+      if (!mbar_wait(&full[st], (kb / p.stages) & 1, a.err.wait_ns)) {
+        s_flag[0] = 1;
+        set_error(a.err, DEV_TIMEOUT);
+        break;
+      }
+      uint8_t* stage = smem + (size_t)st * L.stage_bytes;
+      const int g = (k0 + kb * 64) / 128;
+#pragma unroll
+      for (int na = 0; na < NA; ++na) {
+        const int r = dr + na * 128;
+        const bf16 sv = srow0[(size_t)na * 128 * gpr + g];
+        const __nv_bfloat162 sc = __halves2bfloat162(sv, sv);
+        const uint4* raw = reinterpret_cast<const uint4*>(stage + L.a_bytes + L.b_bytes + r * 32);
+        const uint4 w0 = raw[0], w1 = raw[1];
+        const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        const uint32_t arow = smem_u32(stage) + (uint32_t)r * 128u;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t addr = arow + (((uint32_t)c ^ (uint32_t)(r & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                       "r"(dequant_pair(words[c], 0, sc)), "r"(dequant_pair(words[c], 1, sc)),
+                       "r"(dequant_pair(words[c], 2, sc)), "r"(dequant_pair(words[c], 3, sc))
+                       : "memory");
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&a_ready[st]);
+    }
   }
   __syncwarp();
   pdl_wait();  // the epilogue reads the residual stream / slot lengths
@@ -326,46 +389,60 @@ __global__ void __launch_bounds__(256, 2)
   if (warp == 0) tmem_dealloc(tmem, ncols);
 }
 
-size_t smem_bytes_impl(int na, const TcPlan& p) { return tc_layout(na, p).total; }
+size_t smem_bytes_impl(int na, const TcPlan& p, bool w4) { return tc_layout(na, p, w4).total; }
 
-template <int NA, int EPI, bool SPLIT>
+template <int NA, int EPI, bool SPLIT, bool W4>
 cudaError_t init_one() {
-  cudaError_t e = cudaFuncSetAttribute(k_tc_gemm<NA, EPI, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(k_tc_gemm<NA, EPI, SPLIT, W4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        227 * 1024);
   if (e == cudaSuccess && SPLIT)
-    e = cudaFuncSetAttribute(k_tc_gemm<NA, EPI, SPLIT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    e = cudaFuncSetAttribute(k_tc_gemm<NA, EPI, SPLIT, W4>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   return e;
 }
 
-template <int NA, int EPI>
+template <int NA, int EPI, bool W4>
 cudaError_t launch_one(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* tmX, const TcPlan& p,
                        const TcGemmArgs& a, bool pdl, cudaStream_t st) {
   dim3 grid((a.N + 127) / 128, p.splits, p.tok_tiles);
-  const size_t smem = smem_bytes_impl(NA, p);
+  const size_t smem = smem_bytes_impl(NA, p, W4);
   if (p.splits > 1)
-    return launch_ex(k_tc_gemm<NA, EPI, true>, grid, dim3(256), smem, st, p.splits, pdl, *tmW, *tmX, s, p, a);
-  return launch_ex(k_tc_gemm<NA, EPI, false>, grid, dim3(256), smem, st, 1, pdl, *tmW, *tmX, s, p, a);
+    return launch_ex(k_tc_gemm<NA, EPI, true, W4>, grid, dim3(256), smem, st, p.splits, pdl, *tmW, *tmX, s, p, a);
+  return launch_ex(k_tc_gemm<NA, EPI, false, W4>, grid, dim3(256), smem, st, 1, pdl, *tmW, *tmX, s, p, a);
+}
+
+template <bool W4>
+cudaError_t init_all() {
+  cudaError_t e = init_one<1, EPI_QKV, false, W4>();
+  if (e == cudaSuccess) e = init_one<1, EPI_QKV, true, W4>();
+  if (e == cudaSuccess) e = init_one<1, EPI_RESID, false, W4>();
+  if (e == cudaSuccess) e = init_one<1, EPI_RESID, true, W4>();
+  if (e == cudaSuccess) e = init_one<2, EPI_GEGLU, false, W4>();
+  if (e == cudaSuccess) e = init_one<2, EPI_GEGLU, true, W4>();
+  return e;
+}
+
+template <bool W4>
+cudaError_t launch_sel(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* tmX, int na, const TcPlan& p,
+                       const TcGemmArgs& a, bool pdl, cudaStream_t st) {
+  if (na == 2) return launch_one<2, EPI_GEGLU, W4>(s, tmW, tmX, p, a, pdl, st);
+  if (a.e.epi == EPI_QKV) return launch_one<1, EPI_QKV, W4>(s, tmW, tmX, p, a, pdl, st);
+  return launch_one<1, EPI_RESID, W4>(s, tmW, tmX, p, a, pdl, st);
 }
 
 }  // namespace
 
-size_t tc_gemm_smem_bytes(int na, const TcPlan& p) { return smem_bytes_impl(na, p); }
+size_t tc_gemm_smem_bytes(int na, const TcPlan& p, bool w4) { return smem_bytes_impl(na, p, w4); }
 
 cudaError_t tc_gemm_init() {
-  cudaError_t e = init_one<1, EPI_QKV, false>();
-  if (e == cudaSuccess) e = init_one<1, EPI_QKV, true>();
-  if (e == cudaSuccess) e = init_one<1, EPI_RESID, false>();
-  if (e == cudaSuccess) e = init_one<1, EPI_RESID, true>();
-  if (e == cudaSuccess) e = init_one<2, EPI_GEGLU, false>();
-  if (e == cudaSuccess) e = init_one<2, EPI_GEGLU, true>();
+  cudaError_t e = init_all<false>();
+  if (e == cudaSuccess) e = init_all<true>();
   return e;
 }
 
 cudaError_t launch_tc_gemm(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* tmX, int na, const TcPlan& p,
                            const TcGemmArgs& a, bool pdl, cudaStream_t st) {
-  if (na == 2) return launch_one<2, EPI_GEGLU>(s, tmW, tmX, p, a, pdl, st);
-  if (a.e.epi == EPI_QKV) return launch_one<1, EPI_QKV>(s, tmW, tmX, p, a, pdl, st);
-  return launch_one<1, EPI_RESID>(s, tmW, tmX, p, a, pdl, st);
+  if (a.scales) return launch_sel<true>(s, tmW, tmX, na, p, a, pdl, st);
+  return launch_sel<false>(s, tmW, tmX, na, p, a, pdl, st);
 }
 
 }  // namespace pae

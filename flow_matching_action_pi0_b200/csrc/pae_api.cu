@@ -61,6 +61,30 @@ __global__ void k_transpose(const T* __restrict__ src, T* __restrict__ dst, int 
   }
 }
 
+// Packed int4 rows [rows][kbytes] -> the kernels' layout: within every
+// 32-bit word the nibbles of k = 0..7 move to bit positions
+// 0, 16, 4, 20, 8, 24, 12, 28, so that (w >> 4i) & 0x000F000F holds the
+// pair (k = 2i, 2i + 1).  Row r goes to destination row dst_row(r):
+// mode 0 identity, 1 gate rows and 2 up rows of the 128-row interleave.
+__global__ void k_repack_int4(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, int rows, int kbytes,
+                              int mode) {
+  const int words = kbytes / 4;
+  const size_t n = (size_t)rows * words;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const int r = (int)(i / words), c = (int)(i - (size_t)r * words);
+    const uint32_t w = reinterpret_cast<const uint32_t*>(src + (size_t)r * kbytes)[c];
+    uint32_t o = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t nib = (w >> (4 * k)) & 0xFu;
+      const int pos = (k & 1) ? 16 + 4 * (k >> 1) : 4 * (k >> 1);
+      o |= nib << pos;
+    }
+    const int dr = mode == 0 ? r : ((r >> 7) * 256 + (r & 127) + (mode == 2 ? 128 : 0));
+    reinterpret_cast<uint32_t*>(dst + (size_t)dr * kbytes)[c] = o;
+  }
+}
+
 }  // namespace
 
 struct pae_ctx {
@@ -77,6 +101,11 @@ struct pae_ctx {
   void *w_qkv = nullptr, *w_o = nullptr, *w_gu = nullptr, *w_down = nullptr;  // stacked over layers
   CUtensorMap tmWqkv{}, tmWo{}, tmWgu{}, tmWdown{};
   CUtensorMap tmQ{}, tmK{}, tmV{};  // attention operands (bf16 modes)
+  // int4 weights (W4A16): packed codes [L*rows][K/2] and group scales [L*rows][K/128]
+  int w4 = 0;
+  void *q_qkv = nullptr, *q_o = nullptr, *q_gu = nullptr, *q_down = nullptr;
+  void *sc_qkv = nullptr, *sc_o = nullptr, *sc_gu = nullptr, *sc_down = nullptr;
+  CUtensorMap tmQqkv{}, tmQo{}, tmQgu{}, tmQdown{};
   // tables
   double* t_dev = nullptr;
   float *emb = nullptr, *zbuf = nullptr, *cbuf = nullptr, *tables = nullptr, *dt = nullptr;
@@ -164,20 +193,35 @@ pae_status make_map(pae_ctx* ctx, CUtensorMap* m, const void* base, uint64_t inn
   return PAE_OK;
 }
 
+pae_status make_map_u8(pae_ctx* ctx, CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                       uint32_t box_inner, uint32_t box_outer) {
+  // uint8 matrix [outer][inner], unswizzled boxes (the packed int4 tiles).
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = ctx->encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(ctx, PAE_ERR_CUDA, "cuTensorMapEncodeTiled (uint8) failed (%d)", (int)r);
+  return PAE_OK;
+}
+
 // Token tile and split-K choice for one projection of `nfeat` outputs and K
 // inputs.  The token tile covers the tokens with as little padding as possible
 // (<= 256 per MMA).  Split-K (a cluster of S CTAs, S a power of two <= 16 that
 // divides the 64-wide K blocks) fills the 148 SMs when the tile count is small;
 // small token tiles keep shared memory under half an SM so that two CTAs (or a
 // CTA and its successor under PDL) fit per SM.
-TcPlan plan_gemm(int M, int nfeat, int K, int na, int max_splits = 16) {
+TcPlan plan_gemm(int M, int nfeat, int K, int na, int max_splits = 16, bool w4 = false) {
   TcPlan p{};
   p.tok_tiles = (M + 255) / 256;
   int per = (M + p.tok_tiles - 1) / p.tok_tiles;
   p.tn = std::max(16, ((per + 15) / 16) * 16);
   const int base = ((nfeat + 127) / 128) * p.tok_tiles;
   const int nkb = K / 64;
-  const uint32_t stage = (uint32_t)na * 16384u + (uint32_t)p.tn * 128u;
+  const uint32_t stage = (uint32_t)na * 16384u + (uint32_t)p.tn * 128u + (w4 ? (uint32_t)na * 4096u : 0u);
   const uint32_t recv = (uint32_t)na * p.tn * 128u * 4u;  // split-K receive buffer
   const bool small = p.tn <= 64;  // two CTAs per SM (shared memory and the 128-register cap allow it)
   const uint32_t budget = small ? 110u * 1024u : 200u * 1024u;
@@ -225,10 +269,11 @@ pae_status build_plan(pae_ctx* ctx, int B, Plan* P) {
   P->B = B;
   P->M = B * s.H;
   if (!ctx->act_bf16) return PAE_OK;
-  P->qkv = plan_gemm(P->M, s.qkv_rows, s.D, 1, ctx->max_splitk);
-  P->o = plan_gemm(P->M, s.D, s.attn_dim, 1, ctx->max_splitk);
-  P->gu = plan_gemm(P->M, s.F, s.D, 2, ctx->max_splitk);
-  P->down = plan_gemm(P->M, s.D, s.F, 1, ctx->max_splitk);
+  const bool w4 = ctx->w4 != 0;
+  P->qkv = plan_gemm(P->M, s.qkv_rows, s.D, 1, ctx->max_splitk, w4);
+  P->o = plan_gemm(P->M, s.D, s.attn_dim, 1, ctx->max_splitk, w4);
+  P->gu = plan_gemm(P->M, s.F, s.D, 2, ctx->max_splitk, w4);
+  P->down = plan_gemm(P->M, s.D, s.F, 1, ctx->max_splitk, w4);
   P->attn = plan_attn(s, B);
   const uint64_t Mmax = (uint64_t)s.Bmax * s.H;
   pae_status st;
@@ -310,12 +355,18 @@ void run_gemm(pae_ctx* ctx, const Plan& P, int which, int layer, const EpiArgs& 
   const CUtensorMap *tw, *tx;
   const TcPlan* p;
   int na = 1;
+  const bool w4 = ctx->w4 != 0;
   switch (which) {
-    case 0: tw = &ctx->tmWqkv; tx = &P.tmY; p = &P.qkv; a.N = s.qkv_rows; a.K = s.D; a.w_row0 = layer * s.qkv_rows; break;
-    case 1: tw = &ctx->tmWo; tx = &P.tmO; p = &P.o; a.N = s.D; a.K = s.attn_dim; a.w_row0 = layer * s.D; break;
-    case 2: tw = &ctx->tmWgu; tx = &P.tmY; p = &P.gu; a.N = s.F; a.K = s.D; a.w_row0 = layer * 2 * s.F; na = 2; break;
-    default: tw = &ctx->tmWdown; tx = &P.tmU; p = &P.down; a.N = s.D; a.K = s.F; a.w_row0 = layer * s.D; break;
+    case 0: tw = w4 ? &ctx->tmQqkv : &ctx->tmWqkv; tx = &P.tmY; p = &P.qkv; a.N = s.qkv_rows; a.K = s.D;
+            a.w_row0 = layer * s.qkv_rows; a.scales = (const bf16*)ctx->sc_qkv; break;
+    case 1: tw = w4 ? &ctx->tmQo : &ctx->tmWo; tx = &P.tmO; p = &P.o; a.N = s.D; a.K = s.attn_dim;
+            a.w_row0 = layer * s.D; a.scales = (const bf16*)ctx->sc_o; break;
+    case 2: tw = w4 ? &ctx->tmQgu : &ctx->tmWgu; tx = &P.tmY; p = &P.gu; a.N = s.F; a.K = s.D;
+            a.w_row0 = layer * 2 * s.F; na = 2; a.scales = (const bf16*)ctx->sc_gu; break;
+    default: tw = w4 ? &ctx->tmQdown : &ctx->tmWdown; tx = &P.tmU; p = &P.down; a.N = s.D; a.K = s.F;
+             a.w_row0 = layer * s.D; a.scales = (const bf16*)ctx->sc_down; break;
   }
+  if (!w4) a.scales = nullptr;
   launch_tc_gemm(s, tw, tx, na, *p, a, pdl_on(ctx), st);
 }
 
@@ -522,8 +573,8 @@ pae_status validate_config(const pae_config* c) {
     return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: at most 16 query heads per KV head");
   if (c->width % 32 != 0 || c->width > 2048)
     return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: width must be a multiple of 32 and at most 2048");
-  if (c->dtype == PAE_W4A16)
-    return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: W4A16 kernels are not built yet");
+  if (c->dtype == PAE_W4A16 && c->group_size != 128)
+    return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: W4A16 needs group_size 128");
   if (c->dtype != PAE_FP32) {
     const int qd = c->n_q_heads * c->head_dim;
     if (c->width % 128 || qd % 128 || c->mlp_dim % 128 || (c->n_kv_heads * c->head_dim) % 64)
@@ -554,6 +605,13 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
   for (int l = 0; l < cfg->layers; ++l)
     if (!w->w_qkv[l] || !w->w_o[l] || !w->w_gate[l] || !w->w_up[l] || !w->w_down[l])
       return fail(nullptr, PAE_ERR_ARG, "layer %d weight pointer is NULL", l);
+  if (cfg->dtype == PAE_W4A16) {
+    if (!w->s_qkv || !w->s_o || !w->s_gate || !w->s_up || !w->s_down)
+      return fail(nullptr, PAE_ERR_ARG, "W4A16 needs the s_* scale arrays");
+    for (int l = 0; l < cfg->layers; ++l)
+      if (!w->s_qkv[l] || !w->s_o[l] || !w->s_gate[l] || !w->s_up[l] || !w->s_down[l])
+        return fail(nullptr, PAE_ERR_ARG, "layer %d scale pointer is NULL", l);
+  }
 
   pae_ctx* ctx = new pae_ctx();
   ctx->cfg = *cfg;
@@ -576,6 +634,7 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
   s.eps = cfg->rms_eps;
   s.table_rows = (s.L * 2 * 3 + 2) * s.D;
   ctx->act_bf16 = cfg->dtype != PAE_FP32;
+  ctx->w4 = cfg->dtype == PAE_W4A16;
   ctx->esize = ctx->act_bf16 ? 2 : 4;
   const size_t es = ctx->esize;
   ctx->lens_host.assign(s.Bmax, -1);
@@ -630,10 +689,21 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
   ALLOC(ctx->b_t2, (size_t)D * es);
   ALLOC(ctx->w_modall, (size_t)s.table_rows * D * es);
   ALLOC(ctx->b_modall, (size_t)s.table_rows * es);
-  ALLOC(ctx->w_qkv, (size_t)L * s.qkv_rows * D * es);
-  ALLOC(ctx->w_o, (size_t)L * D * s.attn_dim * es);
-  ALLOC(ctx->w_gu, (size_t)L * 2 * F * D * es);
-  ALLOC(ctx->w_down, (size_t)L * D * F * es);
+  if (!ctx->w4) {
+    ALLOC(ctx->w_qkv, (size_t)L * s.qkv_rows * D * es);
+    ALLOC(ctx->w_o, (size_t)L * D * s.attn_dim * es);
+    ALLOC(ctx->w_gu, (size_t)L * 2 * F * D * es);
+    ALLOC(ctx->w_down, (size_t)L * D * F * es);
+  } else {
+    ALLOC(ctx->q_qkv, (size_t)L * s.qkv_rows * D / 2);
+    ALLOC(ctx->q_o, (size_t)L * D * s.attn_dim / 2);
+    ALLOC(ctx->q_gu, (size_t)L * 2 * F * D / 2);
+    ALLOC(ctx->q_down, (size_t)L * D * F / 2);
+    ALLOC(ctx->sc_qkv, (size_t)L * s.qkv_rows * (D / 128) * 2);
+    ALLOC(ctx->sc_o, (size_t)L * D * (s.attn_dim / 128) * 2);
+    ALLOC(ctx->sc_gu, (size_t)L * 2 * F * (D / 128) * 2);
+    ALLOC(ctx->sc_down, (size_t)L * D * (F / 128) * 2);
+  }
   cudaStream_t cs = ctx->cap_stream;
   if (ctx->act_bf16)
     k_transpose<uint16_t><<<64, 256, 0, cs>>>((const uint16_t*)w->w_in, (uint16_t*)ctx->w_inT, D, A);
@@ -654,7 +724,29 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
   CKC(cudaMemcpyAsync(ctx->b_modall, w->b_mod, mod_rows * es, cudaMemcpyDeviceToDevice, cs));
   CKC(cudaMemcpyAsync((char*)ctx->b_modall + mod_rows * es, w->b_modf, (size_t)2 * D * es,
                       cudaMemcpyDeviceToDevice, cs));
-  for (int l = 0; l < L; ++l) {
+  for (int l = 0; l < L && ctx->w4; ++l) {
+    auto rep = [&](const void* src, void* dst, int rows, int K, int mode) {
+      k_repack_int4<<<256, 256, 0, cs>>>((const uint8_t*)src, (uint8_t*)dst, rows, K / 2, mode);
+    };
+    rep(w->w_qkv[l], (char*)ctx->q_qkv + (size_t)l * s.qkv_rows * D / 2, s.qkv_rows, D, 0);
+    rep(w->w_o[l], (char*)ctx->q_o + (size_t)l * D * s.attn_dim / 2, D, s.attn_dim, 0);
+    rep(w->w_down[l], (char*)ctx->q_down + (size_t)l * D * F / 2, D, F, 0);
+    rep(w->w_gate[l], (char*)ctx->q_gu + (size_t)l * 2 * F * D / 2, F, D, 1);
+    rep(w->w_up[l], (char*)ctx->q_gu + (size_t)l * 2 * F * D / 2, F, D, 2);
+    CKC(cudaGetLastError());
+    const size_t g1 = D / 128, g2 = s.attn_dim / 128, g3 = F / 128;
+    CKC(cudaMemcpyAsync((char*)ctx->sc_qkv + (size_t)l * s.qkv_rows * g1 * 2, w->s_qkv[l], (size_t)s.qkv_rows * g1 * 2,
+                        cudaMemcpyDeviceToDevice, cs));
+    CKC(cudaMemcpyAsync((char*)ctx->sc_o + (size_t)l * D * g2 * 2, w->s_o[l], (size_t)D * g2 * 2,
+                        cudaMemcpyDeviceToDevice, cs));
+    CKC(cudaMemcpyAsync((char*)ctx->sc_down + (size_t)l * D * g3 * 2, w->s_down[l], (size_t)D * g3 * 2,
+                        cudaMemcpyDeviceToDevice, cs));
+    char* gu = (char*)ctx->sc_gu + (size_t)l * 2 * F * g1 * 2;
+    const size_t tile = (size_t)128 * g1 * 2;
+    CKC(cudaMemcpy2DAsync(gu, 2 * tile, w->s_gate[l], tile, tile, F / 128, cudaMemcpyDeviceToDevice, cs));
+    CKC(cudaMemcpy2DAsync(gu + tile, 2 * tile, w->s_up[l], tile, tile, F / 128, cudaMemcpyDeviceToDevice, cs));
+  }
+  for (int l = 0; l < L && !ctx->w4; ++l) {
     CKC(cudaMemcpyAsync((char*)ctx->w_qkv + (size_t)l * s.qkv_rows * D * es, w->w_qkv[l],
                         (size_t)s.qkv_rows * D * es, cudaMemcpyDeviceToDevice, cs));
     CKC(cudaMemcpyAsync((char*)ctx->w_o + (size_t)l * D * s.attn_dim * es, w->w_o[l], (size_t)D * s.attn_dim * es,
@@ -705,11 +797,23 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
   CKC(cudaMemsetAsync(ctx->y, 0, Mpad * D * es, cs));
   CKC(cudaMemsetAsync(ctx->o, 0, Mpad * s.attn_dim * es, cs));
   CKC(cudaMemsetAsync(ctx->u, 0, Mpad * F * es, cs));
-  if (ctx->act_bf16) {
+  if (ctx->act_bf16 && !ctx->w4) {
     if ((st = make_map(ctx, &ctx->tmWqkv, ctx->w_qkv, D, (uint64_t)L * s.qkv_rows, 64, 128)) != PAE_OK) return bail(st);
     if ((st = make_map(ctx, &ctx->tmWo, ctx->w_o, s.attn_dim, (uint64_t)L * D, 64, 128)) != PAE_OK) return bail(st);
     if ((st = make_map(ctx, &ctx->tmWgu, ctx->w_gu, D, (uint64_t)L * 2 * F, 64, 256)) != PAE_OK) return bail(st);
     if ((st = make_map(ctx, &ctx->tmWdown, ctx->w_down, F, (uint64_t)L * D, 64, 128)) != PAE_OK) return bail(st);
+  }
+  if (ctx->w4) {
+    if ((st = make_map_u8(ctx, &ctx->tmQqkv, ctx->q_qkv, D / 2, (uint64_t)L * s.qkv_rows, 32, 128)) != PAE_OK)
+      return bail(st);
+    if ((st = make_map_u8(ctx, &ctx->tmQo, ctx->q_o, s.attn_dim / 2, (uint64_t)L * D, 32, 128)) != PAE_OK)
+      return bail(st);
+    if ((st = make_map_u8(ctx, &ctx->tmQgu, ctx->q_gu, D / 2, (uint64_t)L * 2 * F, 32, 256)) != PAE_OK)
+      return bail(st);
+    if ((st = make_map_u8(ctx, &ctx->tmQdown, ctx->q_down, F / 2, (uint64_t)L * D, 32, 128)) != PAE_OK)
+      return bail(st);
+  }
+  if (ctx->act_bf16) {
     CKC(attn_tc_init());
     const uint64_t kv_rows = (uint64_t)L * s.Bmax * s.Hkv * s.Ptot;
     if ((st = make_map(ctx, &ctx->tmQ, ctx->q, s.d, (uint64_t)s.Bmax * s.Hq * s.H, 64, 128)) != PAE_OK) return bail(st);

@@ -55,6 +55,20 @@ def test_tiny_bf16_gqa2_many_tokens():
     _run_case(cfg, lengths=[(7 * b) % 65 for b in range(20)])
 
 
+def test_tiny_w4a16():
+    _run_case(wl.TINY_FP32.replace(name="tiny_w4a16", dtype=wl.W4A16))
+
+
+def test_tiny_w4a16_batch3_gqa2():
+    cfg = wl.TINY_FP32.replace(name="tiny_w4a16_b3", dtype=wl.W4A16, batch=3, n_kv_heads=2)
+    _run_case(cfg, lengths=[64, 7, 0])
+
+
+@pytest.mark.slow
+def test_pi05_w4a16_bs1():
+    _run_case(wl.PI05_W4A16_BS1)
+
+
 @pytest.mark.slow
 def test_pi05_bf16_bs1():
     _run_case(wl.PI05_BF16_BS1)
