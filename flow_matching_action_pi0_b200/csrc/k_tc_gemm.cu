@@ -92,22 +92,22 @@ __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
 // Epilogue of one output feature f over n <= 16 tokens ms[] (accumulators a0,
 // and a1 for the GeGLU up projection).  Loads that the results need (residual
 // stream, slot lengths) are issued for the whole batch before any is used.
-template <int EPI>
+template <int EPI, int NB = 16>
 __device__ __forceinline__ void epi_batch(const Shape& s, const EpiArgs& e, int f, const int* ms, const float* a0,
                                           const float* a1, int n) {
   if constexpr (EPI == EPI_RESID) {
-    float hv[16];
+    float hv[NB];
     const float g = e.gate[f];
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
+    for (int i = 0; i < NB; ++i)
       if (i < n) hv[i] = e.h[(size_t)ms[i] * s.D + f];
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
+    for (int i = 0; i < NB; ++i)
       if (i < n) e.h[(size_t)ms[i] * s.D + f] = fmaf(g, a0[i], hv[i]);
   } else if constexpr (EPI == EPI_GEGLU) {
     bf16* u = static_cast<bf16*>(e.u);
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
+    for (int i = 0; i < NB; ++i)
       if (i < n) u[(size_t)ms[i] * s.F + f] = f2bf(gelu_tanh(a0[i]) * a1[i]);
   } else {
     const int qd = s.Hq * s.d;
@@ -115,7 +115,7 @@ __device__ __forceinline__ void epi_batch(const Shape& s, const EpiArgs& e, int 
       const int hq = f / s.d, j = f - hq * s.d;
       bf16* q = static_cast<bf16*>(e.q) + (size_t)hq * s.H * s.d + j;
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
+      for (int i = 0; i < NB; ++i)
         if (i < n) {
           const int b = ms[i] / s.H, t = ms[i] - b * s.H;
           q[((size_t)b * s.Hq * s.H + t) * s.d] = f2bf(a0[i]);
@@ -127,12 +127,12 @@ __device__ __forceinline__ void epi_batch(const Shape& s, const EpiArgs& e, int 
       const int g = fk / s.d, j = fk - g * s.d;
       bf16* base = static_cast<bf16*>(is_v ? e.vc : e.kc) +
                    ((size_t)e.layer * s.Bmax * s.Hkv + g) * s.Ptot * s.d + j;
-      int lens[16];
+      int lens[NB];
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
+      for (int i = 0; i < NB; ++i)
         if (i < n) lens[i] = e.lens[ms[i] / s.H];
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
+      for (int i = 0; i < NB; ++i)
         if (i < n) {
           const int b = ms[i] / s.H, t = ms[i] - b * s.H;
           base[((size_t)b * s.Hkv * s.Ptot + lens[i] + t) * s.d] = f2bf(a0[i]);
@@ -368,18 +368,33 @@ __global__ void __launch_bounds__(256, 2)
       const uint32_t rbase = smem_u32(recv) + (uint32_t)rr * 4u;
       const uint32_t src_stride = (uint32_t)p.tn * R * 4u;
       const uint32_t na_stride = (uint32_t)S * src_stride;
+      // eight tokens per batch: their loads (partials, residual) overlap
 #pragma unroll 1
-      for (int col = threadIdx.x / R; col < p.tn; col += cstep) {
-        const int m = mbase + col;
-        if (m >= e.M || f >= a.N) break;
-        const uint32_t addr = rbase + (uint32_t)col * R * 4u;
-        float s0 = 0.f, s1 = 0.f;
+      for (int c0 = threadIdx.x / R; c0 < p.tn; c0 += 8 * cstep) {
+        float s0[8], s1[8];
+        int ms[16];
+        int n = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int col = c0 + i * cstep;
+          s0[i] = 0.f;
+          s1[i] = 0.f;
+          ms[i] = mbase + col;
+          if (col < p.tn && mbase + col < e.M) n = i + 1;
+        }
+        if (n == 0 || f >= a.N) break;
 #pragma unroll 1
         for (int src = 0; src < S; ++src) {
-          s0 += ld_shared_f32(addr + src * src_stride);
-          if (NA == 2) s1 += ld_shared_f32(addr + na_stride + src * src_stride);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t addr = rbase + (uint32_t)(c0 + i * cstep) * R * 4u + src * src_stride;
+            if (i < n) {
+              s0[i] += ld_shared_f32(addr);
+              if (NA == 2) s1[i] += ld_shared_f32(addr + na_stride);
+            }
+          }
         }
-        epi_one<EPI>(s, e, f, m, s0, s1);
+        epi_batch<EPI, 8>(s, e, f, ms, s0, s1, n);
       }
     }
   }
