@@ -31,7 +31,8 @@ STATUS_NAMES = {0: "PAE_OK", 1: "PAE_ERR_ARG", 2: "PAE_ERR_STATE", 3: "PAE_ERR_C
 # Every symbol include/pae.h declares.
 EXPORTS = ("pae_create", "pae_set_prefix", "pae_precompute_tables", "pae_denoise", "pae_denoise_host",
            "pae_denoise_steps", "pae_set_option", "pae_profile_read", "pae_query", "pae_sync",
-           "pae_clear_error", "pae_last_error", "pae_debug_copy", "pae_destroy")
+           "pae_clear_error", "pae_last_error", "pae_debug_copy", "pae_precompute_tables_static",
+           "pae_destroy")
 
 
 class PaeError(RuntimeError):
@@ -84,6 +85,8 @@ def lib() -> ctypes.CDLL:
         "pae_last_error": (ctypes.c_char_p, [v]),
         "pae_debug_copy": (i, [v, ctypes.c_char_p, v, ctypes.POINTER(ctypes.c_size_t)]),
         "pae_destroy": (None, [v]),
+        "pae_precompute_tables_static": (i, [i, i, i, ctypes.POINTER(pae_weights), ctypes.POINTER(ctypes.c_double),
+                                             i, v, v, st]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -174,6 +177,15 @@ def pae_debug_copy(ctx: int, name: str):
     buf = np.empty(n.value, dtype=np.uint8)
     _check(lib().pae_debug_copy(ctx, name.encode(), buf.ctypes.data, ctypes.byref(n)), ctx)
     return buf
+
+
+def pae_precompute_tables_static(layers: int, width: int, dtype: int, weights: pae_weights, t: Sequence[float],
+                                 tables_ptr: int, dt_ptr: int, stream=None):
+    """Context-free, allocation-free table build into caller-owned buffers."""
+    K = len(t) - 1
+    arr = (ctypes.c_double * (K + 1))(*[float(x) for x in t])
+    _check(lib().pae_precompute_tables_static(layers, width, dtype, ctypes.byref(weights), arr, K, tables_ptr,
+                                              dt_ptr, _stream(stream)))
 
 
 def pae_destroy(ctx: int):

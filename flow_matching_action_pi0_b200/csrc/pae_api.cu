@@ -27,6 +27,15 @@ namespace {
 
 thread_local std::string g_create_error;
 
+}  // namespace
+
+namespace pae {
+// Message that pae_last_error(NULL) reports (context-free entry points).
+void set_create_error(const char* msg) { g_create_error = msg ? msg : ""; }
+}  // namespace pae
+
+namespace {
+
 constexpr int kMaxSteps = 64;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,

@@ -203,6 +203,30 @@ const char* pae_last_error(const pae_ctx* ctx);
  * NULL to query the size). */
 pae_status pae_debug_copy(pae_ctx* ctx, const char* name, void* dst_host, size_t* bytes);
 
+/* Timestep/modulation tables without a context and without allocating.
+ * The pages have no counterpart: this entry point exists for callers that may
+ * not allocate device memory while they run (a real-time control process past
+ * its set-up, a host framework that owns all device memory in its own arena,
+ * code that is capturing a stream into a CUDA graph).  They cannot call
+ * pae_create, which allocates, but can build the same tables as
+ * pae_precompute_tables into buffers they own.
+ *   w: only w_t1, b_t1, w_t2, b_t2, w_mod, b_mod, w_modf, b_modf are read
+ *      (device, layouts as in pae_create; fp32 if dtype is PAE_FP32, else bf16).
+ *   t: host float64 grid t[0..K], strictly monotone.
+ *   tables: device fp32 [K][(6*layers + 2)*width], the layout of the context's
+ *      tables: per layer l and norm j (0 attention, 1 MLP) the rows
+ *      (scale, shift, gate), then the final norm's (scale, shift).
+ *   dt: device fp32 [K], dt_k = t[k+1] - t[k].
+ * Limits: 1 <= K <= 64 and width <= 2048 (else PAE_ERR_ARG, message in
+ * pae_last_error(NULL)).  Intermediates live in one fixed 1.5 MB device array
+ * per device that every call shares: calls whose GPU work overlaps (streams
+ * with no ordering between them) race and must be serialised by the caller.
+ * The first call on a device looks the array up and sets kernel attributes;
+ * make that first call before any stream capture.  Asynchronous on `stream`. */
+pae_status pae_precompute_tables_static(int layers, int width, int dtype, const pae_weights* w,
+                                        const double* t, int K, float* tables, float* dt,
+                                        pae_stream stream);
+
 /* Free everything the context owns.  NULL is a no-op. */
 void pae_destroy(pae_ctx* ctx);
 
