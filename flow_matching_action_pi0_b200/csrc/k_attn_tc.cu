@@ -11,7 +11,8 @@
 // One CTA = (b, g, 128-row query tile, key split).  Per 64-key chunk c:
 //   MMA warp   S_c = Q K_c^T  (M=128, N=64, K=head_dim; TMEM, double buffered)
 //   4 warps    online softmax on S_c (thread = query row, log2 domain),
-//              rescale O in TMEM when the row max grows, write P_c (bf16,
+//              rescale O in TMEM when the row max grows by more than 2^8
+//              (otherwise keep the old reference), write P_c (bf16,
 //              128-byte swizzled K-major) to shared memory
 //   MMA warp   O += P_c V_c   (M=128, N=head_dim, K=64; V read MN-major)
 // Warps 0-3 run the softmax and the output (thread = query row = TMEM lane);
@@ -239,13 +240,17 @@ __global__ void __launch_bounds__(192, 1)
     for (int j = 0; j < CK; j += 16) tmem_ld16(t_s[st] + lane_off + j, sv + j);
     tmem_ld_wait();
     const int vc = min(CK, end - (start + c * CK));
-    float mx = m_run;
+    float cmax = -INFINITY;
 #pragma unroll
     for (int j = 0; j < CK; ++j) {
       sv[j] = j < vc ? sv[j] * scale_log2 : -INFINITY;
-      mx = fmaxf(mx, sv[j]);
+      cmax = fmaxf(cmax, sv[j]);
     }
-    const float alpha = exp2f(m_run - mx);  // m_run = -inf on the first chunk -> 0
+    // Lazy rescaling: the reference maximum moves only when the row maximum
+    // grows by more than 8 (a factor 256), so O is rescaled in TMEM rarely.
+    // Probabilities then lie in [0, 256]; the final O / l is the same.
+    const float mx = cmax > m_run + 8.f ? cmax : m_run;
+    const float alpha = exp2f(m_run - mx);  // 1 when unchanged; 0 on the first chunk
     float psum = 0.f;
 #pragma unroll
     for (int j = 0; j < CK; ++j) {

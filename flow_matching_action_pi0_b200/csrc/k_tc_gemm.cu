@@ -66,6 +66,56 @@ __host__ __device__ inline TcSmemLayout tc_layout(int na, const TcPlan& p, bool 
   return L;
 }
 
+__device__ __forceinline__ void named_bar(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ void store16_bf16(bf16* p, const float* v) {
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    w[i] = (uint32_t)__bfloat16_as_ushort(f2bf(v[2 * i])) | ((uint32_t)__bfloat16_as_ushort(f2bf(v[2 * i + 1])) << 16);
+  uint4* d = reinterpret_cast<uint4*>(p);
+  d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+// Epilogue of 16 consecutive output features f..f+15 of token m (v holds the
+// accumulators; for GeGLU already gelu(gate) * up).  16 divides head_dim and
+// 128, so the run never crosses a q/k/v head.
+template <int EPI>
+__device__ __forceinline__ void epi_vec16(const Shape& s, const EpiArgs& e, int m, int f, const float* v) {
+  if constexpr (EPI == EPI_RESID) {
+    float* hp = e.h + (size_t)m * s.D + f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float4 h4 = reinterpret_cast<float4*>(hp)[q];
+      const float4 g4 = reinterpret_cast<const float4*>(e.gate + f)[q];
+      h4.x = fmaf(g4.x, v[4 * q], h4.x);
+      h4.y = fmaf(g4.y, v[4 * q + 1], h4.y);
+      h4.z = fmaf(g4.z, v[4 * q + 2], h4.z);
+      h4.w = fmaf(g4.w, v[4 * q + 3], h4.w);
+      reinterpret_cast<float4*>(hp)[q] = h4;
+    }
+  } else if constexpr (EPI == EPI_GEGLU) {
+    store16_bf16(static_cast<bf16*>(e.u) + (size_t)m * s.F + f, v);
+  } else {
+    const int b = m / s.H, t = m - b * s.H;
+    const int qd = s.Hq * s.d;
+    if (f < qd) {
+      const int hq = f / s.d, j = f - hq * s.d;
+      store16_bf16(static_cast<bf16*>(e.q) + ((size_t)(b * s.Hq + hq) * s.H + t) * s.d + j, v);
+    } else {
+      const int kvd = s.Hkv * s.d;
+      const bool is_v = f >= qd + kvd;
+      const int fk = f - qd - (is_v ? kvd : 0);
+      const int g = fk / s.d, j = fk - g * s.d;
+      const size_t off = (((size_t)(e.layer * s.Bmax + b) * s.Hkv + g) * s.Ptot + e.lens[b] + t) * s.d + j;
+      store16_bf16(static_cast<bf16*>(is_v ? e.vc : e.kc) + off, v);
+    }
+  }
+}
+
 __device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
@@ -319,20 +369,34 @@ __global__ void __launch_bounds__(256, 2)
   const int nchunks = p.tn / 16;
 
   if constexpr (!SPLIT) {
-    const int f = ntile * 128 + row;
-    if (ok) {
-      for (int c = half; c < nchunks; c += 2) {
+    // Staged through shared memory (the ring is idle now): thread = weight row
+    // parks 16 tokens of its row, then thread = (token, 16 consecutive
+    // features) writes them as vectors.  Each warpgroup has its own 8 KB tile.
+    float* stg = reinterpret_cast<float*>(smem) + half * (16 * 128);
+    const int th = row;  // thread index within the warpgroup
+    const int tj = th >> 3, fg = (th & 7) * 16;
+    const int f = ntile * 128 + fg;
+    for (int c = half; c < nchunks; c += 2) {
+      if (ok) {
         float v0[16], v1[16];
         tmem_ld16(trow + c * 16, v0);
         if (NA == 2) tmem_ld16(trow + p.tn + c * 16, v1);
         tmem_ld_wait();
-        const int m0 = mbase + c * 16;
-        int ms[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) ms[j] = m0 + j;
-        const int n = min(16, e.M - m0);
-        if (n > 0 && f < a.N) epi_batch<EPI>(s, e, f, ms, v0, v1, n);
+        for (int j = 0; j < 16; ++j) stg[j * 128 + row] = NA == 2 ? gelu_tanh(v0[j]) * v1[j] : v0[j];
       }
+      named_bar(1 + half, 128);
+      const int m = mbase + c * 16 + tj;
+      if (ok && m < e.M && f < a.N) {
+        float v[16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 t4 = *reinterpret_cast<const float4*>(stg + tj * 128 + fg + 4 * q);
+          v[4 * q] = t4.x; v[4 * q + 1] = t4.y; v[4 * q + 2] = t4.z; v[4 * q + 3] = t4.w;
+        }
+        epi_vec16<EPI>(s, e, m, f, v);
+      }
+      named_bar(1 + half, 128);
     }
   } else {
     // Split-K inside a cluster of S CTAs: rank r owns rows [r*R, r*R+R).  Every
