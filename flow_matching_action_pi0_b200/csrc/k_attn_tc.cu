@@ -16,8 +16,8 @@
 //              128-byte swizzled K-major) to shared memory
 //   MMA warp   O += P_c V_c   (M=128, N=head_dim, K=64; V read MN-major)
 // Warps 0-3 run the softmax and the output (thread = query row = TMEM lane);
-// warp 4 is the TMA producer (Q once, K/V chunks through a 2-stage ring);
-// warp 5 issues the MMAs.
+// warp 4 streams Q and the K chunks, warp 6 the V chunks (2-slot rings each,
+// a K slot refilled as soon as S of its chunk is done); warp 5 issues the MMAs.
 // Key splits (split-KV, for small batches) form a thread-block cluster; their
 // unnormalised partial O rows, row maxima and sums are merged through
 // distributed shared memory in rank order, so the result is bitwise
@@ -86,7 +86,7 @@ __host__ __device__ inline uint32_t attn_tmem_cols(int d) {
   return c;
 }
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(224, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const Shape s, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -98,12 +98,13 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;   // [2]
   uint64_t* v_full = bars + 3;   // [2]
-  uint64_t* kv_empty = bars + 5; // [2]
+  uint64_t* k_empty = bars + 5;  // [2] K slot free once S of its chunk is done
   uint64_t* s_full = bars + 7;   // [2]
   uint64_t* p_full = bars + 9;
   uint64_t* o_done = bars + 10;
   uint64_t* drain = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* v_empty = bars + 12;  // [2] V slot free once PV of its chunk is done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
   volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);  // [0] abort
   float* s_ml = reinterpret_cast<float*>(smem + L.ml_off);                // [128][2] row max, row sum
   int* s_ok = reinterpret_cast<int*>(smem + L.ml_off + QROWS * 8);        // [128]
@@ -121,7 +122,7 @@ __global__ void __launch_bounds__(192, 1)
   const float scale_log2 = rsqrtf((float)d) * 1.4426950408889634f;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 12; ++i) mbar_init(&bars[i], i == 9 ? 128 : 1);
+    for (int i = 0; i < 14; ++i) mbar_init(&bars[i], i == 9 ? 128 : 1);
     s_flag[0] = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -142,7 +143,9 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t t_s[2] = {tmem, tmem + CK};
   const uint32_t t_o = tmem + 2 * CK;
 
-  // ------------------------------------------------------------ producer (warp 4)
+  // ------------------------------------------------------------ producers
+  // Warp 4 streams Q once and the K chunks, warp 6 the V chunks: a K slot is
+  // refilled as soon as S of its chunk is done, ahead of the PV that frees V.
   if (warp == 4 && lane == 0 && nch > 0) {
     const uint32_t kvbytes = CK * d * 2;
     mbar_arrive_expect_tx(q_full, QROWS * d * 2);
@@ -151,7 +154,7 @@ __global__ void __launch_bounds__(192, 1)
     int issued = 0;
     for (int c = 0; c < nch; ++c) {
       const int st = c & 1;
-      if (c >= 2 && !mbar_wait(&kv_empty[st], ((c >> 1) & 1) ^ 1, a.err.wait_ns)) {
+      if (c >= 2 && !mbar_wait(&k_empty[st], ((c >> 1) & 1) ^ 1, a.err.wait_ns)) {
         s_flag[0] = 1;
         set_error(a.err, DEV_TIMEOUT);
         break;
@@ -159,15 +162,29 @@ __global__ void __launch_bounds__(192, 1)
       const int krow = slot_row0 + start + c * CK;
       mbar_arrive_expect_tx(&k_full[st], kvbytes);
       for (int x = 0; x < nbox; ++x) tma_load_2d(smem + L.k_off[st] + x * CK * 128, &tmK, x * 64, krow, &k_full[st]);
+      issued = c + 1;
+    }
+    if (!mbar_wait(q_full, 0, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
+    for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c)
+      if (!mbar_wait(&k_full[c & 1], (c >> 1) & 1, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
+  }
+  if (warp == 6 && lane == 0 && nch > 0) {
+    const uint32_t kvbytes = CK * d * 2;
+    int issued = 0;
+    for (int c = 0; c < nch; ++c) {
+      const int st = c & 1;
+      if (c >= 2 && !mbar_wait(&v_empty[st], ((c >> 1) & 1) ^ 1, a.err.wait_ns)) {
+        s_flag[0] = 1;
+        set_error(a.err, DEV_TIMEOUT);
+        break;
+      }
+      const int krow = slot_row0 + start + c * CK;
       mbar_arrive_expect_tx(&v_full[st], kvbytes);
       for (int x = 0; x < nbox; ++x) tma_load_2d(smem + L.v_off[st] + x * CK * 128, &tmV, x * 64, krow, &v_full[st]);
       issued = c + 1;
     }
-    if (!mbar_wait(q_full, 0, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
-    for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c) {
-      if (!mbar_wait(&k_full[c & 1], (c >> 1) & 1, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
+    for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c)
       if (!mbar_wait(&v_full[c & 1], (c >> 1) & 1, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
-    }
   }
 
   // ------------------------------------------------------------ MMA (warp 5)
@@ -189,6 +206,7 @@ __global__ void __launch_bounds__(192, 1)
         umma_bf16(t_s[st], ad, bd, idesc_s, k16 > 0 ? 1u : 0u);
       }
       umma_commit(&s_full[st]);
+      umma_commit(&k_empty[st]);
       return true;
     };
     if (good) good = issue_s(0);
@@ -207,7 +225,7 @@ __global__ void __launch_bounds__(192, 1)
         umma_bf16(t_o, ad, bd, idesc_o, (c > 0 || k16 > 0) ? 1u : 0u);
       }
       umma_commit(o_done);
-      umma_commit(&kv_empty[st]);
+      umma_commit(&v_empty[st]);
       if (c + 2 < nch) good = issue_s(c + 2);
     }
     if (!good) {
@@ -341,69 +359,69 @@ __global__ void __launch_bounds__(192, 1)
   }  // warps 0-3
 
   if (gridDim.y > 1) {
-    // Split-KV merge inside the cluster of key splits.  Every CTA parks its
-    // unnormalised O rows (stride d+4 floats, bank-conflict free) and its row
-    // max / sum in shared memory (the Q and K/V buffers are idle now); CTA
-    // rank r then merges rows [r*R, r*R+R) over all ranks in rank order.
-    __syncthreads();  // all MMAs and TMEM reads of this CTA are done
-    const int ld = d + 4;
-    float* red = reinterpret_cast<float*>(smem);
+    // Split-KV merge inside the cluster of key splits.  After a cluster
+    // barrier (every peer is done with its Q/K/V/P buffers) each CTA pushes its
+    // unnormalised O rows, row maxima and sums into the owning rank's shared
+    // memory; after a second barrier rank r merges rows [r*R, r*R+R) over all
+    // sources in rank order from local memory.
+    const int S = gridDim.y;
+    const int R = QROWS / S;
+    const int ld = d + 4;  // padded row stride (floats)
+    float my_m = -INFINITY, my_l = 0.f;
+    if (warp < 4) {
+      const int r = warp * 32 + lane;
+      if (s_ok[r] && nch > 0) {
+        my_m = s_ml[2 * r];
+        my_l = s_ml[2 * r + 1];
+      }
+    }
+    __syncthreads();  // own row statistics read before peers can overwrite them
+    cluster_sync();
+    const uint32_t rank = cluster_rank();
+    float* recv = reinterpret_cast<float*>(smem);  // [S][R][ld]
+    float* rml = s_ml;                              // [S][R][2]
     if (warp < 4) {
       const int r = warp * 32 + lane;
       const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-      const bool has = s_ok[r] && nch > 0;
+      const int owner = r / R, rr = r - owner * R;
+      const uint32_t dst = map_cluster(smem_u32(recv) + (uint32_t)((rank * R + rr) * ld) * 4u, (uint32_t)owner);
+      const uint32_t dml = map_cluster(smem_u32(rml) + (uint32_t)((rank * R + rr) * 2) * 4u, (uint32_t)owner);
+      const bool has = s_ok[r] && nch > 0;  // uniform over the CTA
       for (int j = 0; j < d; j += 16) {
         float ov[16];
-        if (__all_sync(0xffffffffu, s_ok[warp * 32] != 0) && nch > 0) {
+        if (has) {
           tmem_ld16(t_o + lane_off + j, ov);
           tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int t = 0; t < 16; ++t) ov[t] = 0.f;
         }
 #pragma unroll
-        for (int t = 0; t < 16; t += 4)
-          *reinterpret_cast<float4*>(red + r * ld + j + t) =
-              has ? make_float4(ov[t], ov[t + 1], ov[t + 2], ov[t + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int t = 0; t < 16; t += 4) st_cluster_f32x4(dst + (uint32_t)(j + t) * 4u, ov[t], ov[t + 1], ov[t + 2], ov[t + 3]);
       }
-      if (!has) {
-        s_ml[2 * r] = -INFINITY;
-        s_ml[2 * r + 1] = 0.f;
-      }
+      st_cluster_f32x2(dml, has ? my_m : -INFINITY, has ? my_l : 0.f);
     }
     cluster_sync();
-    const int S = gridDim.y;
-    const uint32_t rank = cluster_rank();
-    const int R = QROWS / S;
-    const uint32_t red_base = smem_u32(red), ml_base = smem_u32(s_ml);
     const int per_row = d / 4;  // float4 columns
     for (int el = threadIdx.x; el < R * per_row; el += blockDim.x) {
       const int rr = el / per_row, c4 = el - rr * per_row;
       const int row = (int)rank * R + rr;
       const int rq = qt * QROWS + row;
       if (rq >= GH) continue;
-      // issue every rank's loads first (they pipeline), then merge in rank order
-      float ms[8], ls[8];
-      float4 vs[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        if (q < S) {
-          ms[q] = ld_cluster_f32(map_cluster(ml_base + row * 8, (uint32_t)q));
-          ls[q] = ld_cluster_f32(map_cluster(ml_base + row * 8 + 4, (uint32_t)q));
-          vs[q] = ld_cluster_f32x4(map_cluster(red_base + (uint32_t)((row * ld + c4 * 4) * 4), (uint32_t)q));
-        }
       float M = -INFINITY;
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        if (q < S) M = fmaxf(M, ms[q]);
+      for (int q = 0; q < S; ++q) M = fmaxf(M, rml[(q * R + rr) * 2]);
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
       float wsum = 0.f;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        if (q >= S || !(ls[q] > 0.f)) continue;
-        const float w = exp2f(ms[q] - M);
-        wsum = fmaf(w, ls[q], wsum);
-        acc[0] = fmaf(w, vs[q].x, acc[0]);
-        acc[1] = fmaf(w, vs[q].y, acc[1]);
-        acc[2] = fmaf(w, vs[q].z, acc[2]);
-        acc[3] = fmaf(w, vs[q].w, acc[3]);
+      for (int q = 0; q < S; ++q) {
+        const float l_s = rml[(q * R + rr) * 2 + 1];
+        if (!(l_s > 0.f)) continue;
+        const float w = exp2f(rml[(q * R + rr) * 2] - M);
+        wsum = fmaf(w, l_s, wsum);
+        const float4 v = *reinterpret_cast<const float4*>(recv + (q * R + rr) * ld + c4 * 4);
+        acc[0] = fmaf(w, v.x, acc[0]);
+        acc[1] = fmaf(w, v.y, acc[1]);
+        acc[2] = fmaf(w, v.z, acc[2]);
+        acc[3] = fmaf(w, v.w, acc[3]);
       }
       const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
       const int hl = rq / s.H, ti = rq - hl * s.H;
@@ -411,7 +429,6 @@ __global__ void __launch_bounds__(192, 1)
       *reinterpret_cast<uint2*>(orow + c4 * 4) =
           make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
     }
-    cluster_sync();  // peers may still be reading this CTA's partial
   }
 
   tc_fence_before();
@@ -430,7 +447,7 @@ cudaError_t attn_tc_init() {
 cudaError_t launch_attn_tc(const Shape& s, const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                            const AttnPlan& p, const AttnArgs& a, int B, bool pdl, cudaStream_t st) {
   dim3 grid(p.qtiles, p.splits, B * s.Hkv);
-  return launch_ex(k_attn_tc, grid, dim3(192), attn_tc_smem_bytes(s.d), st, p.splits, pdl, *tmQ, *tmK, *tmV, s,
+  return launch_ex(k_attn_tc, grid, dim3(224), attn_tc_smem_bytes(s.d), st, p.splits, pdl, *tmQ, *tmK, *tmV, s,
                    a);
 }
 
