@@ -17,7 +17,8 @@
 //   MMA warp   O += P_c V_c   (M=128, N=head_dim, K=64; V read MN-major)
 // Warps 0-3 run the softmax and the output (thread = query row = TMEM lane);
 // warp 4 streams Q and the K chunks, warp 6 the V chunks (2-slot rings each,
-// a K slot refilled as soon as S of its chunk is done); warp 5 issues the MMAs.
+// a K slot refilled as soon as S of its chunk is done); warp 5 issues the MMAs;
+// all eight warps take part in the split-KV merge.
 // Key splits (split-KV, for small batches) form a thread-block cluster; their
 // unnormalised partial O rows, row maxima and sums are merged through
 // distributed shared memory in rank order, so the result is bitwise
@@ -86,7 +87,7 @@ __host__ __device__ inline uint32_t attn_tmem_cols(int d) {
   return c;
 }
 
-__global__ void __launch_bounds__(224, 1)
+__global__ void __launch_bounds__(256, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const Shape s, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -359,76 +360,92 @@ __global__ void __launch_bounds__(224, 1)
   }  // warps 0-3
 
   if (gridDim.y > 1) {
-    // Split-KV merge inside the cluster of key splits.  After a cluster
-    // barrier (every peer is done with its Q/K/V/P buffers) each CTA pushes its
-    // unnormalised O rows, row maxima and sums into the owning rank's shared
-    // memory; after a second barrier rank r merges rows [r*R, r*R+R) over all
-    // sources in rank order from local memory.
-    const int S = gridDim.y;
-    const int R = QROWS / S;
-    const int ld = d + 4;  // padded row stride (floats)
-    float my_m = -INFINITY, my_l = 0.f;
-    if (warp < 4) {
-      const int r = warp * 32 + lane;
-      if (s_ok[r] && nch > 0) {
-        my_m = s_ml[2 * r];
-        my_l = s_ml[2 * r + 1];
-      }
-    }
-    __syncthreads();  // own row statistics read before peers can overwrite them
-    cluster_sync();
-    const uint32_t rank = cluster_rank();
-    float* recv = reinterpret_cast<float*>(smem);  // [S][R][ld]
-    float* rml = s_ml;                              // [S][R][2]
+    // Split-KV merge inside the cluster of key splits.  Every CTA parks its
+    // unnormalised O rows (stride d+4 floats) and its row max / sum in shared
+    // memory (Q, K and V are idle now); after a cluster barrier rank r merges
+    // rows [r*R, r*R+R): 16 threads per row, each pulling 16 columns from all
+    // S ranks with every load issued before any is used, then summing in rank
+    // order.  A second barrier keeps the buffers alive until all peers read.
+    __syncthreads();  // all MMAs and TMEM reads of this CTA are done
+    const int ld = d + 4;
+    float* red = reinterpret_cast<float*>(smem);
     if (warp < 4) {
       const int r = warp * 32 + lane;
       const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-      const int owner = r / R, rr = r - owner * R;
-      const uint32_t dst = map_cluster(smem_u32(recv) + (uint32_t)((rank * R + rr) * ld) * 4u, (uint32_t)owner);
-      const uint32_t dml = map_cluster(smem_u32(rml) + (uint32_t)((rank * R + rr) * 2) * 4u, (uint32_t)owner);
       const bool has = s_ok[r] && nch > 0;  // uniform over the CTA
-      for (int j = 0; j < d; j += 16) {
-        float ov[16];
+      for (int j = 0; j < d; j += 64) {
+        float ov[64];
         if (has) {
-          tmem_ld16(t_o + lane_off + j, ov);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) tmem_ld16(t_o + lane_off + j + 16 * u, ov + 16 * u);
           tmem_ld_wait();
         } else {
 #pragma unroll
-          for (int t = 0; t < 16; ++t) ov[t] = 0.f;
+          for (int t = 0; t < 64; ++t) ov[t] = 0.f;
         }
 #pragma unroll
-        for (int t = 0; t < 16; t += 4) st_cluster_f32x4(dst + (uint32_t)(j + t) * 4u, ov[t], ov[t + 1], ov[t + 2], ov[t + 3]);
+        for (int t = 0; t < 64; t += 4)
+          *reinterpret_cast<float4*>(red + r * ld + j + t) = make_float4(ov[t], ov[t + 1], ov[t + 2], ov[t + 3]);
       }
-      st_cluster_f32x2(dml, has ? my_m : -INFINITY, has ? my_l : 0.f);
+      if (!has) {
+        s_ml[2 * r] = -INFINITY;
+        s_ml[2 * r + 1] = 0.f;
+      }
     }
     cluster_sync();
-    const int per_row = d / 4;  // float4 columns
-    for (int el = threadIdx.x; el < R * per_row; el += blockDim.x) {
-      const int rr = el / per_row, c4 = el - rr * per_row;
+    const int S = gridDim.y;
+    const uint32_t rank = cluster_rank();
+    const int R = QROWS / S;
+    const uint32_t red_base = smem_u32(red), ml_base = smem_u32(s_ml);
+    // 16 threads per row, 16 columns each; rows (rank*R + rr) for rr < R
+    for (int task = threadIdx.x; task < R * (d / 16); task += blockDim.x) {
+      const int rr = task / (d / 16), cb = (task - rr * (d / 16)) * 16;
       const int row = (int)rank * R + rr;
       const int rq = qt * QROWS + row;
       if (rq >= GH) continue;
+      float ms[8], ls[8];
+      float4 vs[8][4];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (q < S) {
+          ms[q] = ld_cluster_f32(map_cluster(ml_base + row * 8, (uint32_t)q));
+          ls[q] = ld_cluster_f32(map_cluster(ml_base + row * 8 + 4, (uint32_t)q));
+          const uint32_t src = map_cluster(red_base + (uint32_t)((row * ld + cb) * 4), (uint32_t)q);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) vs[q][u] = ld_cluster_f32x4(src + 16u * u);
+        }
       float M = -INFINITY;
-      for (int q = 0; q < S; ++q) M = fmaxf(M, rml[(q * R + rr) * 2]);
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (q < S) M = fmaxf(M, ms[q]);
+      float acc[16];
+#pragma unroll
+      for (int t = 0; t < 16; ++t) acc[t] = 0.f;
       float wsum = 0.f;
-      for (int q = 0; q < S; ++q) {
-        const float l_s = rml[(q * R + rr) * 2 + 1];
-        if (!(l_s > 0.f)) continue;
-        const float w = exp2f(rml[(q * R + rr) * 2] - M);
-        wsum = fmaf(w, l_s, wsum);
-        const float4 v = *reinterpret_cast<const float4*>(recv + (q * R + rr) * ld + c4 * 4);
-        acc[0] = fmaf(w, v.x, acc[0]);
-        acc[1] = fmaf(w, v.y, acc[1]);
-        acc[2] = fmaf(w, v.z, acc[2]);
-        acc[3] = fmaf(w, v.w, acc[3]);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (q >= S || !(ls[q] > 0.f)) continue;
+        const float w = exp2f(ms[q] - M);
+        wsum = fmaf(w, ls[q], wsum);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          acc[4 * u] = fmaf(w, vs[q][u].x, acc[4 * u]);
+          acc[4 * u + 1] = fmaf(w, vs[q][u].y, acc[4 * u + 1]);
+          acc[4 * u + 2] = fmaf(w, vs[q][u].z, acc[4 * u + 2]);
+          acc[4 * u + 3] = fmaf(w, vs[q][u].w, acc[4 * u + 3]);
+        }
       }
       const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
       const int hl = rq / s.H, ti = rq - hl * s.H;
-      bf16* orow = reinterpret_cast<bf16*>(a.o) + (size_t)(b * s.H + ti) * s.attn_dim + (g * s.G + hl) * d;
-      *reinterpret_cast<uint2*>(orow + c4 * 4) =
-          make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+      bf16* orow = reinterpret_cast<bf16*>(a.o) + (size_t)(b * s.H + ti) * s.attn_dim + (g * s.G + hl) * d + cb;
+      uint32_t pk[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) pk[t] = pack_bf16x2(acc[2 * t] * inv, acc[2 * t + 1] * inv);
+      uint4* dst = reinterpret_cast<uint4*>(orow);
+      dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
     }
+    cluster_sync();  // peers may still be reading this CTA's partial
   }
 
   tc_fence_before();
@@ -447,7 +464,7 @@ cudaError_t attn_tc_init() {
 cudaError_t launch_attn_tc(const Shape& s, const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                            const AttnPlan& p, const AttnArgs& a, int B, bool pdl, cudaStream_t st) {
   dim3 grid(p.qtiles, p.splits, B * s.Hkv);
-  return launch_ex(k_attn_tc, grid, dim3(224), attn_tc_smem_bytes(s.d), st, p.splits, pdl, *tmQ, *tmK, *tmV, s,
+  return launch_ex(k_attn_tc, grid, dim3(256), attn_tc_smem_bytes(s.d), st, p.splits, pdl, *tmQ, *tmK, *tmV, s,
                    a);
 }
 
