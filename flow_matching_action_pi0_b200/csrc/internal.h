@@ -78,12 +78,6 @@ struct EpiArgs {
   const float* gate;  // [D]
   // EPI_GEGLU
   void* u;            // [M][F]
-  // EPI_RESID, small batches: the last CTA to finish also writes
-  // y = adaRMSNorm(h; norm_scale, norm_shift) for all M tokens (null: off)
-  const float* norm_scale;
-  const float* norm_shift;
-  void* norm_y;       // [M][D] bf16
-  int* norm_ctr;      // arrival counter, zero between launches
 };
 
 // out-features N (for GEGLU: F, weight rows interleaved in 128-row tiles).

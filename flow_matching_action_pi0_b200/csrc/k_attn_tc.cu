@@ -361,31 +361,26 @@ __global__ void __launch_bounds__(256, 1)
 
   if (gridDim.y > 1) {
     // Split-KV merge inside the cluster of key splits.  Every CTA parks its
-    // unnormalised O rows (stride d+4 floats) and its row max / sum in shared
-    // memory (Q, K and V are idle now); after a cluster barrier rank r merges
-    // rows [r*R, r*R+R): 16 threads per row, each pulling 16 columns from all
-    // S ranks with every load issued before any is used, then summing in rank
-    // order.  A second barrier keeps the buffers alive until all peers read.
+    // unnormalised O rows (stride d+4 floats, bank-conflict free) and its row
+    // max / sum in shared memory (the Q and K/V buffers are idle now); CTA
+    // rank r then merges rows [r*R, r*R+R) over all ranks in rank order.
     __syncthreads();  // all MMAs and TMEM reads of this CTA are done
     const int ld = d + 4;
     float* red = reinterpret_cast<float*>(smem);
     if (warp < 4) {
       const int r = warp * 32 + lane;
       const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-      const bool has = s_ok[r] && nch > 0;  // uniform over the CTA
-      for (int j = 0; j < d; j += 64) {
-        float ov[64];
-        if (has) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) tmem_ld16(t_o + lane_off + j + 16 * u, ov + 16 * u);
+      const bool has = s_ok[r] && nch > 0;
+      for (int j = 0; j < d; j += 16) {
+        float ov[16];
+        if (__all_sync(0xffffffffu, s_ok[warp * 32] != 0) && nch > 0) {
+          tmem_ld16(t_o + lane_off + j, ov);
           tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int t = 0; t < 64; ++t) ov[t] = 0.f;
         }
 #pragma unroll
-        for (int t = 0; t < 64; t += 4)
-          *reinterpret_cast<float4*>(red + r * ld + j + t) = make_float4(ov[t], ov[t + 1], ov[t + 2], ov[t + 3]);
+        for (int t = 0; t < 16; t += 4)
+          *reinterpret_cast<float4*>(red + r * ld + j + t) =
+              has ? make_float4(ov[t], ov[t + 1], ov[t + 2], ov[t + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
       if (!has) {
         s_ml[2 * r] = -INFINITY;
@@ -397,53 +392,43 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t rank = cluster_rank();
     const int R = QROWS / S;
     const uint32_t red_base = smem_u32(red), ml_base = smem_u32(s_ml);
-    // 16 threads per row, 16 columns each; rows (rank*R + rr) for rr < R
-    for (int task = threadIdx.x; task < R * (d / 16); task += blockDim.x) {
-      const int rr = task / (d / 16), cb = (task - rr * (d / 16)) * 16;
+    const int per_row = d / 4;  // float4 columns
+    for (int el = threadIdx.x; el < R * per_row; el += blockDim.x) {
+      const int rr = el / per_row, c4 = el - rr * per_row;
       const int row = (int)rank * R + rr;
       const int rq = qt * QROWS + row;
       if (rq >= GH) continue;
+      // issue every rank's loads first (they pipeline), then merge in rank order
       float ms[8], ls[8];
-      float4 vs[8][4];
+      float4 vs[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q)
         if (q < S) {
           ms[q] = ld_cluster_f32(map_cluster(ml_base + row * 8, (uint32_t)q));
           ls[q] = ld_cluster_f32(map_cluster(ml_base + row * 8 + 4, (uint32_t)q));
-          const uint32_t src = map_cluster(red_base + (uint32_t)((row * ld + cb) * 4), (uint32_t)q);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) vs[q][u] = ld_cluster_f32x4(src + 16u * u);
+          vs[q] = ld_cluster_f32x4(map_cluster(red_base + (uint32_t)((row * ld + c4 * 4) * 4), (uint32_t)q));
         }
       float M = -INFINITY;
 #pragma unroll
       for (int q = 0; q < 8; ++q)
         if (q < S) M = fmaxf(M, ms[q]);
-      float acc[16];
-#pragma unroll
-      for (int t = 0; t < 16; ++t) acc[t] = 0.f;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
       float wsum = 0.f;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         if (q >= S || !(ls[q] > 0.f)) continue;
         const float w = exp2f(ms[q] - M);
         wsum = fmaf(w, ls[q], wsum);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          acc[4 * u] = fmaf(w, vs[q][u].x, acc[4 * u]);
-          acc[4 * u + 1] = fmaf(w, vs[q][u].y, acc[4 * u + 1]);
-          acc[4 * u + 2] = fmaf(w, vs[q][u].z, acc[4 * u + 2]);
-          acc[4 * u + 3] = fmaf(w, vs[q][u].w, acc[4 * u + 3]);
-        }
+        acc[0] = fmaf(w, vs[q].x, acc[0]);
+        acc[1] = fmaf(w, vs[q].y, acc[1]);
+        acc[2] = fmaf(w, vs[q].z, acc[2]);
+        acc[3] = fmaf(w, vs[q].w, acc[3]);
       }
       const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
       const int hl = rq / s.H, ti = rq - hl * s.H;
-      bf16* orow = reinterpret_cast<bf16*>(a.o) + (size_t)(b * s.H + ti) * s.attn_dim + (g * s.G + hl) * d + cb;
-      uint32_t pk[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) pk[t] = pack_bf16x2(acc[2 * t] * inv, acc[2 * t + 1] * inv);
-      uint4* dst = reinterpret_cast<uint4*>(orow);
-      dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      bf16* orow = reinterpret_cast<bf16*>(a.o) + (size_t)(b * s.H + ti) * s.attn_dim + (g * s.G + hl) * d;
+      *reinterpret_cast<uint2*>(orow + c4 * 4) =
+          make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
     }
     cluster_sync();  // peers may still be reading this CTA's partial
   }

@@ -463,53 +463,6 @@ __global__ void __launch_bounds__(256, 2)
     }
   }
 
-  if constexpr (EPI == EPI_RESID) {
-    if (e.norm_scale) {
-      // The last CTA to finish its residual update normalises every row
-      // (fixed order, no waiting): y = h / sqrt(mean h^2 + eps) * (1 + scale) + shift.
-      __threadfence();
-      __syncthreads();
-      volatile int* s_last = s_flag + 1;
-      if (threadIdx.x == 0) {
-        const int total = (int)(gridDim.x * gridDim.y * gridDim.z);
-        const int prev = atomicAdd(e.norm_ctr, 1);
-        *s_last = (prev == total - 1) ? 1 : 0;
-        if (prev == total - 1) *e.norm_ctr = 0;
-      }
-      __syncthreads();
-      if (*s_last) {
-        __threadfence();
-        bf16* y = static_cast<bf16*>(e.norm_y);
-        for (int m = warp; m < e.M; m += 8) {
-          const float* hr = e.h + (size_t)m * s.D;
-          float4 v[16];
-          float ss = 0.f;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int j = 4 * (lane + 32 * i);
-            v[i] = j < s.D ? __ldcg(reinterpret_cast<const float4*>(hr + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
-            ss = fmaf(v[i].x, v[i].x, fmaf(v[i].y, v[i].y, fmaf(v[i].z, v[i].z, fmaf(v[i].w, v[i].w, ss))));
-          }
-          ss = warp_sum(ss);
-          const float r = rsqrtf(ss / (float)s.D + s.eps);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int j = 4 * (lane + 32 * i);
-            if (j < s.D) {
-              const float4 c = *reinterpret_cast<const float4*>(e.norm_scale + j);
-              const float4 d = *reinterpret_cast<const float4*>(e.norm_shift + j);
-              const uint32_t lo = (uint32_t)__bfloat16_as_ushort(f2bf(v[i].x * r * (1.f + c.x) + d.x)) |
-                                  ((uint32_t)__bfloat16_as_ushort(f2bf(v[i].y * r * (1.f + c.y) + d.y)) << 16);
-              const uint32_t hi = (uint32_t)__bfloat16_as_ushort(f2bf(v[i].z * r * (1.f + c.z) + d.z)) |
-                                  ((uint32_t)__bfloat16_as_ushort(f2bf(v[i].w * r * (1.f + c.w) + d.w)) << 16);
-              *reinterpret_cast<uint2*>(y + (size_t)m * s.D + j) = make_uint2(lo, hi);
-            }
-          }
-        }
-      }
-    }
-  }
-
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, ncols);

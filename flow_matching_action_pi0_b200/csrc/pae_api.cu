@@ -126,7 +126,6 @@ struct pae_ctx {
   std::vector<int> lens_host;
   // activations and workspaces
   float *x = nullptr, *h = nullptr;
-  int* norm_ctr = nullptr;  // arrival counter of the fused small-batch norm
   void *y = nullptr, *q = nullptr, *o = nullptr, *u = nullptr;
   // error word (host-mapped)
   int* err_host = nullptr;
@@ -434,25 +433,16 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
           launch_attention_simple(s, ctx->act_bf16, ctx->q, ctx->kc, ctx->vc, ctx->lens_dev, l, ctx->o, P.B, st);
         }
       }
-      // Small batches: the residual GEMM's last CTA also writes the next
-      // adaRMSNorm (saves a dependent launch); large batches use k_norm.
-      const bool fuse_norm = ctx->act_bf16 && M <= 128;
       e = EpiArgs{};
       e.M = M;
       e.epi = EPI_RESID;
       e.h = ctx->h;
       e.gate = tk + mod_offset(s, l, 0, 2);
-      if (fuse_norm) {
-        e.norm_scale = tk + mod_offset(s, l, 1, 0);
-        e.norm_shift = tk + mod_offset(s, l, 1, 1);
-        e.norm_y = ctx->y;
-        e.norm_ctr = ctx->norm_ctr;
-      }
       {
         ProfScope ps(ctx, PAE_K_OPROJ, st);
         run_gemm(ctx, P, 1, l, e, st);
       }
-      if (!fuse_norm) {
+      {
         ProfScope ps(ctx, PAE_K_NORM, st);
         launch_norm(s, ctx->act_bf16, ctx->h, ctx->y, tk + mod_offset(s, l, 1, 0), tk + mod_offset(s, l, 1, 1), M,
                     pdl_on(ctx), st);
@@ -470,17 +460,11 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
       e.epi = EPI_RESID;
       e.h = ctx->h;
       e.gate = tk + mod_offset(s, l, 1, 2);
-      if (fuse_norm && l + 1 < s.L) {
-        e.norm_scale = tk + mod_offset(s, l + 1, 0, 0);
-        e.norm_shift = tk + mod_offset(s, l + 1, 0, 1);
-        e.norm_y = ctx->y;
-        e.norm_ctr = ctx->norm_ctr;
-      }
       {
         ProfScope ps(ctx, PAE_K_DOWN, st);
         run_gemm(ctx, P, 3, l, e, st);
       }
-      if (l + 1 < s.L && !fuse_norm) {
+      if (l + 1 < s.L) {
         ProfScope ps(ctx, PAE_K_NORM, st);
         launch_norm(s, ctx->act_bf16, ctx->h, ctx->y, tk + mod_offset(s, l + 1, 0, 0), tk + mod_offset(s, l + 1, 0, 1),
                     M, pdl_on(ctx), st);
@@ -814,8 +798,6 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
   CKC(cudaMemsetAsync(ctx->lens_dev, 0, sizeof(int) * s.Bmax, cs));
   const size_t Mmax = (size_t)s.Bmax * s.H;
   const size_t Mpad = ((Mmax + 255) / 256 + 1) * 256;  // token tiles may pad past Mmax
-  ALLOC(ctx->norm_ctr, sizeof(int) * 4);
-  CKC(cudaMemsetAsync(ctx->norm_ctr, 0, sizeof(int) * 4, cs));
   ALLOC(ctx->x, sizeof(float) * Mmax * A);
   ALLOC(ctx->h, sizeof(float) * Mmax * D);
   ALLOC(ctx->y, Mpad * D * es);
@@ -1042,7 +1024,6 @@ void pae_clear_error(pae_ctx* ctx) {
   if (!ctx) return;
   cudaDeviceSynchronize();
   if (ctx->err_host) *(volatile int*)ctx->err_host = 0;
-  if (ctx->norm_ctr) cudaMemset(ctx->norm_ctr, 0, sizeof(int) * 4);
   ctx->last_error.clear();
 }
 
