@@ -378,6 +378,62 @@ def run_minimal(args, cfg):
     return 0
 
 
+def rank_helpers(world_size: int, device: str = "cuda"):
+    """Barrier and max-over-ranks for the timing protocol (the process group
+    must already exist when world_size > 1).  Replicas share nothing else."""
+    if world_size <= 1:
+        return (lambda: None), (lambda v: float(v))
+    import torch
+    import torch.distributed as dist
+
+    def barrier():
+        dist.barrier()
+
+    def maxr(v):
+        t = torch.tensor([float(v)], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    return barrier, maxr
+
+
+def measure_ragged(args, stream, barrier, maxr, ws, gpu_index):
+    """Ragged batch 16: per-request prefix lengths drawn on [512, 1024]; every
+    timed step re-sets 8 rows with fresh prefixes (a new observation each) and
+    keeps 8 (cache hits), then runs the denoise loop."""
+    import torch
+    import flow_matching_action_pi0_b200 as fm
+    from workloads import device as wd
+    cfg = wl.RAGGED_BF16_BS16
+    W = wl.make_weights(cfg)
+    lens = wl.prefix_lengths(cfg)
+    ex, ks, vs, kd, vd, lens, _ = setup_context(cfg, W, cfg.batch, lens)
+    # a second set of prefixes for the fresh rows, swapped in alternately
+    ks2, vs2 = wl.make_prefix(cfg, lengths=lens[:8], seed=1000 + cfg.index)
+    kd2, vd2 = wd.upload_prefix(cfg, ks2, vs2)
+    noise = wl.make_noise(cfg)
+    nd = torch.from_numpy(noise).cuda()
+    od = torch.empty_like(nd)
+    flip = [0]
+
+    def step():
+        src_k, src_v = (kd2, vd2) if flip[0] % 2 == 0 else (kd[:8], vd[:8])
+        for r in range(8):
+            ex.set_prefix(r, src_k[r], src_v[r], lens[r], stream)
+        flip[0] += 1
+        ex.denoise(nd, od, stream)
+
+    with torch.cuda.stream(stream):
+        ms = maxr(timed(step, args.steps, args.warmup, stream, barrier))
+        ms_loop = maxr(timed(lambda: ex.denoise(nd, od, stream), args.steps, args.warmup, stream, barrier))
+    per, st = algorithmic(cfg, cfg.batch, lens)
+    ex.close()
+    return {"value": ws * cfg.batch / (ms * 1e-3), "unit": "chunks/s", "ms_per_step": ms,
+            "ms_per_step_cached_only": ms_loop, "prefix_lengths": lens,
+            "loop_roofline": {"bytes_per_euler_step": st["bytes"], "flops_per_euler_step": st["flops"]},
+            "note": "each step: 8 fresh set_prefix calls (new observations) + 8 cached rows + pae_denoise"}
+
+
 def run_ours(args, cfg):
     import torch
     ws, rank, local = dist_env()
@@ -387,20 +443,7 @@ def run_ours(args, cfg):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
                                 device_id=torch.device("cuda", local))
-
-        def barrier():
-            dist.barrier()
-
-        def maxr(v):
-            t = torch.tensor([float(v)], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            return float(t.item())
-    else:
-        def barrier():
-            pass
-
-        def maxr(v):
-            return float(v)
+    barrier, maxr = rank_helpers(ws)
     import flow_matching_action_pi0_b200 as fm
     fm.lib()
     peaks, peak_kind = load_peaks()
@@ -447,6 +490,9 @@ def run_ours(args, cfg):
             "note": "same weights as the batch-1 line; 32 independent 968-token prefixes"}}
         r32.pop("ex").close()
         del r32
+    if args.secondary and cfg.name == wl.PI05_BF16_BS1.name:
+        line.setdefault("secondary", {})[wl.RAGGED_BF16_BS16.name] = measure_ragged(args, stream, barrier, maxr,
+                                                                                   ws, gpu_index)
     if args.secondary and cfg.name == wl.PI05_BF16_BS1.name:
         c4 = wl.PI05_W4A16_BS1
         W4 = wl.make_weights(c4)
