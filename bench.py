@@ -138,6 +138,8 @@ def algorithmic(cfg: wl.ExpertConfig, batch: int, lens=None):
     step_kv = L * 2 * sum(lens) * cfg.n_kv_heads * cfg.head_dim * ae
     step_flops = L * (out["qkv"]["flops"] + out["o_proj"]["flops"] + out["gate_up"]["flops"] +
                       out["down"]["flops"] + out["attention"]["flops"]) + 2 * 2 * M * A * D
+    # the persistent kernel runs a whole call (all Euler steps) in one launch
+    out["persistent"] = {"bytes": cfg.steps * (step_w + step_kv), "flops": cfg.steps * step_flops}
     return out, {"bytes": step_w + step_kv, "flops": step_flops}
 
 
@@ -278,7 +280,9 @@ def measure(cfg, W, batch, args, stream, barrier, maxr, lens=None, with_e2e=True
         ms = timed(lambda: ex.denoise(nd, od, stream), args.steps, args.warmup, stream, barrier)
         res["clocks"] = clk.stop()
         res["ms_per_step"] = maxr(ms)
-        res["graph_kernels"] = ex.query(fm.PAE_Q_GRAPH_KERNELS, batch)
+        res["persistent"] = ex.query(fm.PAE_Q_PERSISTENT, batch)
+        # kernels per pae_denoise call: one persistent launch, or the captured graph's kernel nodes
+        res["graph_kernels"] = 1 if res["persistent"] else ex.query(fm.PAE_Q_GRAPH_KERNELS, batch)
         res["splits"] = ex.query(fm.PAE_Q_SPLITS, batch)
         res["token_tile"] = ex.query(fm.PAE_Q_TOKEN_TILE, batch)
         res["table_ms"] = table_ms
@@ -297,7 +301,7 @@ def measure(cfg, W, batch, args, stream, barrier, maxr, lens=None, with_e2e=True
             res["e2e_ms"] = maxr(wall * 1e3)
             res["io_bytes"] = int(nh.numel() * 4)
         # live per-kernel timing: the same graph with CUDA events around every launch
-        ex.set_option(fm.PAE_OPT_PROFILE, (1 << 7) - 1)
+        ex.set_option(fm.PAE_OPT_PROFILE, (1 << len(fm.KERNEL_CLASSES)) - 1)
         n_prof = max(3, min(args.steps, 10))
         for _ in range(2):
             ex.denoise(nd, od, stream)
@@ -363,6 +367,7 @@ def run_minimal(args, cfg):
     W = wl.make_weights(cfg)
     ex, *_ = setup_context(cfg, W, cfg.batch, wl.prefix_lengths(cfg))
     ex.set_option(fm.PAE_OPT_PDL, args.pdl)
+    ex.set_option(fm.PAE_OPT_PERSISTENT, args.persistent)
     if args.max_splitk:
         ex.set_option(fm.PAE_OPT_MAX_SPLITK, args.max_splitk)
     nd = torch.from_numpy(wl.make_noise(cfg)).cuda()
@@ -370,8 +375,10 @@ def run_minimal(args, cfg):
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
         ms = timed(lambda: ex.denoise(nd, od, stream), args.steps, args.warmup, stream, lambda: None)
-    k = ex.query(fm.PAE_Q_GRAPH_KERNELS, cfg.batch)
-    print(json.dumps({"workload": cfg.name, "pdl": args.pdl, "max_splitk": args.max_splitk, "ms_per_step": ms,
+    persist = ex.query(fm.PAE_Q_PERSISTENT, cfg.batch)
+    k = 1 if persist else ex.query(fm.PAE_Q_GRAPH_KERNELS, cfg.batch)
+    print(json.dumps({"workload": cfg.name, "pdl": args.pdl, "persistent": persist,
+                      "max_splitk": args.max_splitk, "ms_per_step": ms,
                       "splits": ex.query(fm.PAE_Q_SPLITS, cfg.batch), "graph_kernels": k,
                       "launches_before_timed": 1 + cfg.batch + 4 + args.warmup * k}), flush=True)
     ex.close()
@@ -464,7 +471,8 @@ def run_ours(args, cfg):
         "roofline": rl, "loop_roofline": loop, "kernel_shares": shares,
         "kernels_ms_per_launch": {c: v["ms_per_launch"] for c, v in res["kernels"].items()},
         "gpu_launches": int(res["graph_kernels"]) * args.steps,
-        "graph_kernels_per_step": int(res["graph_kernels"]),
+        "kernels_per_call": int(res["graph_kernels"]),
+        "loop": "persistent kernel" if res["persistent"] else "captured graph",
         "splitk": {"qkv": res["splits"] & 255, "o": (res["splits"] >> 8) & 255,
                    "gate_up": (res["splits"] >> 16) & 255, "down": (res["splits"] >> 24) & 255},
         "token_tile": res["token_tile"], "table_build_ms": res["table_ms"],
@@ -533,6 +541,8 @@ def main():
     ap.add_argument("--minimal", action="store_true", help="only warm-up and timed calls (for profilers)")
     ap.add_argument("--pdl", type=int, default=1, help="programmatic dependent launch inside the loop (1/0)")
     ap.add_argument("--max-splitk", type=int, default=0, help="cap on the projection split-K (0: library default)")
+    ap.add_argument("--persistent", type=int, default=1,
+                    help="persistent kernel for batches of <= 64 tokens (1/0; 0 runs the captured graph)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -128,4 +128,45 @@ cudaError_t attn_tc_init();
 cudaError_t launch_attn_tc(const Shape& s, const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                            const AttnPlan& p, const AttnArgs& a, int B, bool pdl, cudaStream_t st);
 
+// ------------------------------------------- persistent loop (B*H <= 64)
+// One projection of the persistent loop: nt tiles of 128 weight rows, each
+// K range split over s CTAs (CTA i owns tile i / s, split i % s); na tiles
+// form one reduction group (2: the gate and up tiles of the same features);
+// reducer r of a group owns rows [r*rp, r*rp + rp).
+struct PersistPhase {
+  int nt, na, s, nkb, rp;
+  int wrows;  // weight rows per layer in the stacked matrix
+};
+constexpr int kPersistGroups = 256;                     // counters per phase kind
+constexpr int kPersistAbortIdx = 1 + 5 * kPersistGroups;  // launch-wide abort flag
+constexpr int kPersistCtrWords = kPersistAbortIdx + 1;
+struct PersistArgs {
+  int M, ncta, k_begin, k_end;
+  PersistPhase ph[4];  // QKV, O, gate/up, down
+  int a_qtiles, a_splits, a_kps, a_items;
+  float* x;
+  float* h;
+  bf16* q;
+  bf16* o;
+  bf16* u;
+  bf16* kc;
+  bf16* vc;
+  const int* lens;
+  const float* tables;
+  const float* dt;
+  const bf16* w_inT;
+  const bf16* b_in;
+  const bf16* w_out;
+  const bf16* b_out;
+  float* part;    // split-K / split-KV partials
+  float* ss;      // [slot][64] per-token sums of squares of the residual stream
+  unsigned* ctr;  // [kPersistCtrWords], zero at launch
+  DevErr err;
+};
+size_t persist_smem_bytes();
+cudaError_t persist_init();
+// Cooperative launch of a.ncta CTAs (one per SM).
+cudaError_t launch_persistent(const Shape& s, const CUtensorMap* maps /* Wqkv, Wo, Wgu (128-row box), Wdown, Q, K, V */,
+                              const PersistArgs& a, cudaStream_t st);
+
 }  // namespace pae

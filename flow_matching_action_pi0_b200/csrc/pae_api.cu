@@ -51,6 +51,8 @@ struct Plan {
   int B = 0, M = 0;
   TcPlan qkv{}, o{}, gu{}, down{};
   AttnPlan attn{};
+  bool persist = false;  // eligible for the persistent kernel
+  PersistArgs pa{};
   CUtensorMap tmY{}, tmO{}, tmU{};
   cudaGraphExec_t graph = nullptr;
   int graph_K = 0;
@@ -110,6 +112,13 @@ struct pae_ctx {
   void *w_qkv = nullptr, *w_o = nullptr, *w_gu = nullptr, *w_down = nullptr;  // stacked over layers
   CUtensorMap tmWqkv{}, tmWo{}, tmWgu{}, tmWdown{};
   CUtensorMap tmQ{}, tmK{}, tmV{};  // attention operands (bf16 modes)
+  CUtensorMap tmWgu1{};             // gate/up weights with 128-row boxes (persistent kernel)
+  // persistent kernel: one CTA per SM, split-K / split-KV workspace, counters
+  int ncta = 0;
+  bool use_persistent = true;
+  float* pw_part = nullptr;
+  float* pw_ss = nullptr;
+  unsigned* pw_ctr = nullptr;
   // int4 weights (W4A16): packed codes [L*rows][K/2] and group scales [L*rows][K/128]
   int w4 = 0;
   void *q_qkv = nullptr, *q_o = nullptr, *q_gu = nullptr, *q_down = nullptr;
@@ -273,11 +282,74 @@ AttnPlan plan_attn(const Shape& s, int B) {
   return p;
 }
 
+// Persistent-kernel plan for M = B*H <= 64 tokens (bf16 weights): every
+// projection's K range is split so that its tiles x splits fill the SMs; the
+// attention keys are split into 64-key chunks over the (request, KV head,
+// query tile) groups.  Returns false when the batch or shape is not eligible.
+bool plan_persistent(const pae_ctx* ctx, int B, PersistArgs* pa) {
+  const Shape& s = ctx->s;
+  const int M = B * s.H, n = ctx->ncta;
+  if (!ctx->act_bf16 || ctx->w4 || n < 1 || M > 64 || M > n) return false;
+  if (s.d != 64 && s.d != 128 && s.d != 256) return false;
+  if ((size_t)(s.D + s.A) * 4 > 128 * 1024) return false;
+  *pa = PersistArgs{};
+  pa->M = M;
+  pa->ncta = n;
+  auto mk = [&](PersistPhase& p, int rows, int K, int na, bool resid) -> bool {
+    p.nt = rows / 128;
+    p.na = na;
+    p.nkb = K / 64;
+    p.wrows = rows;
+    if (p.nt < 1 || p.nt > n || p.nt / na > kPersistGroups) return false;
+    p.s = std::max(1, std::min(n / p.nt, p.nkb));
+    if ((p.nkb + p.s - 1) / p.s > 16) return false;  // token operand must fit the 128 KB work area
+    int q4 = ((128 + na * p.s - 1) / (na * p.s) + 3) / 4;
+    if (resid) {
+      int pw = 1;
+      while (pw < q4) pw <<= 1;
+      q4 = pw;
+    }
+    p.rp = 4 * q4;
+    return true;
+  };
+  if (!mk(pa->ph[0], s.qkv_rows, s.D, 1, false) || !mk(pa->ph[1], s.D, s.attn_dim, 1, true) ||
+      !mk(pa->ph[2], 2 * s.F, s.D, 2, false) || !mk(pa->ph[3], s.D, s.F, 1, true))
+    return false;
+  pa->a_qtiles = (s.G * s.H + 127) / 128;
+  const int base = B * s.Hkv * pa->a_qtiles;
+  if (base > n || base > kPersistGroups) return false;
+  const int chunks = (s.Ptot + 63) / 64;
+  int sa = std::max(1, std::min(chunks, n / base));
+  pa->a_kps = 64 * ((chunks + sa - 1) / sa);
+  sa = (s.Ptot + pa->a_kps - 1) / pa->a_kps;
+  pa->a_splits = sa;
+  pa->a_items = base * sa;
+  pa->x = ctx->x;
+  pa->h = ctx->h;
+  pa->q = static_cast<bf16*>(ctx->q);
+  pa->o = static_cast<bf16*>(ctx->o);
+  pa->u = static_cast<bf16*>(ctx->u);
+  pa->kc = static_cast<bf16*>(ctx->kc);
+  pa->vc = static_cast<bf16*>(ctx->vc);
+  pa->lens = ctx->lens_dev;
+  pa->tables = ctx->tables;
+  pa->dt = ctx->dt;
+  pa->w_inT = static_cast<const bf16*>(ctx->w_inT);
+  pa->b_in = static_cast<const bf16*>(ctx->b_in);
+  pa->w_out = static_cast<const bf16*>(ctx->w_out);
+  pa->b_out = static_cast<const bf16*>(ctx->b_out);
+  pa->part = ctx->pw_part;
+  pa->ss = ctx->pw_ss;
+  pa->ctr = ctx->pw_ctr;
+  return true;
+}
+
 pae_status build_plan(pae_ctx* ctx, int B, Plan* P) {
   const Shape& s = ctx->s;
   P->B = B;
   P->M = B * s.H;
   if (!ctx->act_bf16) return PAE_OK;
+  P->persist = plan_persistent(ctx, B, &P->pa);
   const bool w4 = ctx->w4 != 0;
   P->qkv = plan_gemm(P->M, s.qkv_rows, s.D, 1, ctx->max_splitk, w4);
   P->o = plan_gemm(P->M, s.D, s.attn_dim, 1, ctx->max_splitk, w4);
@@ -327,7 +399,7 @@ struct ProfScope {
 
 pae_status ensure_events(pae_ctx* ctx, int k_steps) {
   if (!ctx->profile_mask) return PAE_OK;
-  const size_t need = (size_t)2 * ((size_t)k_steps * (7 * ctx->s.L + 1) + 2);
+  const size_t need = (size_t)2 * ((size_t)k_steps * (7 * ctx->s.L + 1) + 3);
   while (ctx->ev_pool.size() < need) {
     cudaEvent_t e;
     CK(cudaEventCreate(&e));
@@ -506,10 +578,34 @@ pae_status check_rows(pae_ctx* ctx, int batch) {
   return PAE_OK;
 }
 
+bool use_persist(const pae_ctx* ctx, const Plan* P) { return ctx->use_persistent && P->persist; }
+
+// Steps k_begin..k_end-1 (and the final Euler update) as one persistent launch.
+pae_status enqueue_persistent(pae_ctx* ctx, Plan* P, int k_begin, int k_end, cudaStream_t st) {
+  PersistArgs pa = P->pa;
+  pa.k_begin = k_begin;
+  pa.k_end = k_end;
+  pa.err = DevErr{ctx->err_dev, ctx->wait_ns};
+  const CUtensorMap maps[7] = {ctx->tmWqkv, ctx->tmWo, ctx->tmWgu1, ctx->tmWdown, ctx->tmQ, ctx->tmK, ctx->tmV};
+  P->recs.clear();
+  ctx->rec_sink = &P->recs;
+  ctx->ev_next = 0;
+  CK(cudaMemsetAsync(ctx->pw_ctr, 0, sizeof(unsigned) * kPersistCtrWords, st));
+  cudaError_t e;
+  {
+    ProfScope ps(ctx, PAE_K_PERSISTENT, st);
+    e = launch_persistent(ctx->s, maps, pa, st);
+  }
+  ctx->rec_sink = nullptr;
+  if (e != cudaSuccess) return fail(ctx, PAE_ERR_CUDA, "persistent launch: %s", cudaGetErrorString(e));
+  return PAE_OK;
+}
+
 pae_status run_loop(pae_ctx* ctx, Plan* P, cudaStream_t stream) {
   pae_status pst = ensure_events(ctx, ctx->K);
   if (pst != PAE_OK) return pst;
   ctx->last_plan = P;
+  if (use_persist(ctx, P)) return enqueue_persistent(ctx, P, 0, ctx->K, stream);
   if (!ctx->use_graph) {
     P->recs.clear();
     ctx->rec_sink = &P->recs;
@@ -823,6 +919,20 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
     if ((st = make_map_u8(ctx, &ctx->tmQdown, ctx->q_down, F / 2, (uint64_t)L * D, 32, 128)) != PAE_OK)
       return bail(st);
   }
+  if (ctx->act_bf16 && !ctx->w4) {
+    // persistent kernel: 128-row gate/up boxes, workspace, one CTA per SM
+    if ((st = make_map(ctx, &ctx->tmWgu1, ctx->w_gu, D, (uint64_t)L * 2 * F, 64, 128)) != PAE_OK) return bail(st);
+    CKC(persist_init());
+    int nsm = 0;
+    CKC(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, ctx->device));
+    int coop = 0;
+    CKC(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, ctx->device));
+    ctx->ncta = coop ? nsm : 0;
+    const size_t part = (size_t)nsm * std::max<size_t>(128 * 64, (size_t)128 * s.d + 256);
+    ALLOC(ctx->pw_part, sizeof(float) * part);
+    ALLOC(ctx->pw_ss, sizeof(float) * kPersistGroups * 64);
+    ALLOC(ctx->pw_ctr, sizeof(unsigned) * kPersistCtrWords);
+  }
   if (ctx->act_bf16) {
     CKC(attn_tc_init());
     const uint64_t kv_rows = (uint64_t)L * s.Bmax * s.Hkv * s.Ptot;
@@ -938,11 +1048,15 @@ pae_status pae_denoise_steps(pae_ctx* ctx, const float* x_in, float* x_out, int 
   const size_t bytes = sizeof(float) * (size_t)batch * ctx->s.H * ctx->s.A;
   if ((st = ensure_events(ctx, k_end - k_begin)) != PAE_OK) return st;
   CK(cudaMemcpyAsync(ctx->x, x_in, bytes, cudaMemcpyDeviceToDevice, stm));
-  P->recs.clear();
-  ctx->rec_sink = &P->recs;
   ctx->last_plan = P;
-  enqueue_steps(ctx, *P, k_begin, k_end, stm);
-  ctx->rec_sink = nullptr;
+  if (use_persist(ctx, P)) {
+    if ((st = enqueue_persistent(ctx, P, k_begin, k_end, stm)) != PAE_OK) return st;
+  } else {
+    P->recs.clear();
+    ctx->rec_sink = &P->recs;
+    enqueue_steps(ctx, *P, k_begin, k_end, stm);
+    ctx->rec_sink = nullptr;
+  }
   CK(cudaGetLastError());
   CK(cudaMemcpyAsync(x_out, ctx->x, bytes, cudaMemcpyDeviceToDevice, stm));
   return PAE_OK;
@@ -970,6 +1084,7 @@ pae_status pae_set_option(pae_ctx* ctx, int option, long long value) {
       if ((value != 0) != ctx->use_pdl) drop_graphs(ctx);
       ctx->use_pdl = value != 0;
       return PAE_OK;
+    case PAE_OPT_PERSISTENT: ctx->use_persistent = value != 0; return PAE_OK;
     case PAE_OPT_PROFILE:
       if (value < 0 || value >= (1LL << PAE_K_COUNT)) return fail(ctx, PAE_ERR_ARG, "bad profile mask");
       if ((unsigned)value != ctx->profile_mask) drop_graphs(ctx);
@@ -1009,6 +1124,7 @@ pae_status pae_query(pae_ctx* ctx, int what, int batch, long long* value) {
       return PAE_OK;
     case PAE_Q_TOKEN_TILE: *value = P->qkv.tn; return PAE_OK;
     case PAE_Q_ATTN_SPLITS: *value = P->attn.splits; return PAE_OK;
+    case PAE_Q_PERSISTENT: *value = use_persist(ctx, P) ? 1 : 0; return PAE_OK;
     default: return fail(ctx, PAE_ERR_ARG, "unknown query %d", what);
   }
 }

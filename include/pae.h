@@ -157,8 +157,20 @@ pae_status pae_denoise_steps(pae_ctx* ctx, const float* x_in, float* x_out, int 
  * weight loads overlap its predecessor's tail; 0 serialises the kernels.
  * PAE_OPT_MAX_SPLITK (default 8, range 1..16): largest split-K cluster the
  * projection planner may choose (a tuning knob; results stay within the
- * parity tolerance, bitwise identical only for the same setting). */
-enum { PAE_OPT_USE_GRAPH = 1, PAE_OPT_WAIT_LIMIT_US = 2, PAE_OPT_PDL = 4, PAE_OPT_MAX_SPLITK = 5 };
+ * parity tolerance, bitwise identical only for the same setting).
+ * PAE_OPT_PERSISTENT (default 1, bf16 mode): when batch * chunk <= 64, run all
+ * K steps of a call as one persistent kernel (one CTA per SM, grid barriers
+ * between the phases of each layer) instead of the graph of per-phase
+ * kernels; 0 forces the graph.  The two paths round differently (both stay
+ * within the parity tolerance); each is bitwise reproducible on its own, and
+ * pae_denoise and pae_denoise_steps take the same path for the same batch. */
+enum {
+  PAE_OPT_USE_GRAPH = 1,
+  PAE_OPT_WAIT_LIMIT_US = 2,
+  PAE_OPT_PDL = 4,
+  PAE_OPT_MAX_SPLITK = 5,
+  PAE_OPT_PERSISTENT = 6
+};
 pae_status pae_set_option(pae_ctx* ctx, int option, long long value);
 
 /* Kernel classes for profiling, as bit positions of PAE_OPT_PROFILE. */
@@ -170,7 +182,8 @@ enum {
   PAE_K_NORM = 4,       /* adaRMSNorm of the residual stream                          */
   PAE_K_GATEUP = 5,     /* GeGLU gate/up projection                                   */
   PAE_K_DOWN = 6,       /* down projection, gated residual                            */
-  PAE_K_COUNT = 7
+  PAE_K_PERSISTENT = 7, /* the whole loop as one persistent kernel (small batches)    */
+  PAE_K_COUNT = 8
 };
 /* PAE_OPT_PROFILE (default 0): bit mask of PAE_K_* classes.  Launches of those
  * classes are bracketed by CUDA events on their stream (inside the captured
@@ -184,8 +197,15 @@ pae_status pae_profile_read(pae_ctx* ctx, int kernel_class, double* total_ms, in
  * `batch` (0 if none captured yet).  PAE_Q_SPLITS: split-K factors of the four
  * projections for `batch`, packed as qkv | o<<8 | gateup<<16 | down<<24.
  * PAE_Q_TOKEN_TILE: MMA token tile for `batch`.  PAE_Q_ATTN_SPLITS: key splits
- * of the attention for `batch`. */
-enum { PAE_Q_GRAPH_KERNELS = 1, PAE_Q_SPLITS = 2, PAE_Q_TOKEN_TILE = 3, PAE_Q_ATTN_SPLITS = 4 };
+ * of the attention for `batch`.  PAE_Q_PERSISTENT: 1 if pae_denoise runs the
+ * persistent kernel for `batch` (option on and the batch eligible), else 0. */
+enum {
+  PAE_Q_GRAPH_KERNELS = 1,
+  PAE_Q_SPLITS = 2,
+  PAE_Q_TOKEN_TILE = 3,
+  PAE_Q_ATTN_SPLITS = 4,
+  PAE_Q_PERSISTENT = 5
+};
 pae_status pae_query(pae_ctx* ctx, int what, int batch, long long* value);
 
 /* Synchronise `stream` and report the device error word (PAE_ERR_TIMEOUT if a
