@@ -441,6 +441,24 @@ def measure_ragged(args, stream, barrier, maxr, ws, gpu_index):
             "note": "each step: 8 fresh set_prefix calls (new observations) + 8 cached rows + pae_denoise"}
 
 
+def measure_persistent(cfg, W, args, stream, barrier, maxr, ws):
+    """The same batch-1 workload through the persistent kernel (one launch per
+    call, grid barriers between phases) instead of the captured graph."""
+    import torch
+    import flow_matching_action_pi0_b200 as fm
+    lens = wl.prefix_lengths(cfg)
+    ex, *_ = setup_context(cfg, W, cfg.batch, lens)
+    ex.set_option(fm.PAE_OPT_PERSISTENT, 1)
+    nd = torch.from_numpy(wl.make_noise(cfg)).cuda()
+    od = torch.empty_like(nd)
+    with torch.cuda.stream(stream):
+        ms = maxr(timed(lambda: ex.denoise(nd, od, stream), args.steps, args.warmup, stream, barrier))
+    used = ex.query(fm.PAE_Q_PERSISTENT, cfg.batch)
+    ex.close()
+    return {"value": ws * cfg.batch / (ms * 1e-3), "unit": "chunks/s", "ms_per_step": ms, "persistent": used,
+            "note": "one cooperative launch per call; slower than the captured graph on this workload"}
+
+
 def run_ours(args, cfg):
     import torch
     ws, rank, local = dist_env()
@@ -502,6 +520,9 @@ def run_ours(args, cfg):
         line.setdefault("secondary", {})[wl.RAGGED_BF16_BS16.name] = measure_ragged(args, stream, barrier, maxr,
                                                                                    ws, gpu_index)
     if args.secondary and cfg.name == wl.PI05_BF16_BS1.name:
+        line.setdefault("secondary", {})["pi05_bf16_bs1_persistent_kernel"] = measure_persistent(
+            cfg, W, args, stream, barrier, maxr, ws)
+    if args.secondary and cfg.name == wl.PI05_BF16_BS1.name:
         c4 = wl.PI05_W4A16_BS1
         W4 = wl.make_weights(c4)
         r4 = measure(c4, W4, c4.batch, args, stream, barrier, maxr, with_e2e=False, gpu_index=gpu_index)
@@ -541,7 +562,7 @@ def main():
     ap.add_argument("--minimal", action="store_true", help="only warm-up and timed calls (for profilers)")
     ap.add_argument("--pdl", type=int, default=1, help="programmatic dependent launch inside the loop (1/0)")
     ap.add_argument("--max-splitk", type=int, default=0, help="cap on the projection split-K (0: library default)")
-    ap.add_argument("--persistent", type=int, default=1,
+    ap.add_argument("--persistent", type=int, default=0,
                     help="persistent kernel for batches of <= 64 tokens (1/0; 0 runs the captured graph)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -115,7 +115,7 @@ struct pae_ctx {
   CUtensorMap tmWgu1{};             // gate/up weights with 128-row boxes (persistent kernel)
   // persistent kernel: one CTA per SM, split-K / split-KV workspace, counters
   int ncta = 0;
-  bool use_persistent = true;
+  bool use_persistent = false;  // opt-in: measured slower than the graph at batch 1
   float* pw_part = nullptr;
   float* pw_ss = nullptr;
   unsigned* pw_ctr = nullptr;

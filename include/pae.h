@@ -158,11 +158,11 @@ pae_status pae_denoise_steps(pae_ctx* ctx, const float* x_in, float* x_out, int 
  * PAE_OPT_MAX_SPLITK (default 8, range 1..16): largest split-K cluster the
  * projection planner may choose (a tuning knob; results stay within the
  * parity tolerance, bitwise identical only for the same setting).
- * PAE_OPT_PERSISTENT (default 1, bf16 mode): when batch * chunk <= 64, run all
- * K steps of a call as one persistent kernel (one CTA per SM, grid barriers
- * between the phases of each layer) instead of the graph of per-phase
- * kernels; 0 forces the graph.  The two paths round differently (both stay
- * within the parity tolerance); each is bitwise reproducible on its own, and
+ * PAE_OPT_PERSISTENT (default 0, bf16 mode): 1 runs all K steps of a call as
+ * one persistent kernel (one CTA per SM, grid barriers between the phases of
+ * each layer) instead of the graph of per-phase kernels, for batches with
+ * batch * chunk <= 64.  The two paths round differently (both stay within
+ * the parity tolerance); each is bitwise reproducible on its own, and
  * pae_denoise and pae_denoise_steps take the same path for the same batch. */
 enum {
   PAE_OPT_USE_GRAPH = 1,

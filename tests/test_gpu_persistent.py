@@ -19,6 +19,7 @@ def _both_paths(cfg, lengths=None, max_prefix=None):
     """(persistent output, graph output, oracle) on the same context and inputs."""
     ex, W = build_expert(cfg, max_prefix=max_prefix)
     try:
+        ex.set_option(fm.PAE_OPT_PERSISTENT, 1)
         ks, vs = wl.make_prefix(cfg, lengths=lengths)
         set_prefixes(ex, cfg, ks, vs)
         grid = wl.uniform_grid(cfg.steps)
@@ -49,6 +50,8 @@ def test_eligibility():
     cfg = TINY_BF16.replace(batch=5)
     ex, _ = build_expert(cfg)
     try:
+        assert ex.query(fm.PAE_Q_PERSISTENT, 1) == 0   # off by default
+        ex.set_option(fm.PAE_OPT_PERSISTENT, 1)
         assert ex.query(fm.PAE_Q_PERSISTENT, 1) == 1   # 16 tokens
         assert ex.query(fm.PAE_Q_PERSISTENT, 4) == 1   # 64 tokens
         assert ex.query(fm.PAE_Q_PERSISTENT, 5) == 0   # 80 tokens: graph of kernels
@@ -59,6 +62,7 @@ def test_eligibility():
     for c in (wl.TINY_FP32, wl.TINY_FP32.replace(name="tiny_w4_p", dtype=wl.W4A16)):
         ex, _ = build_expert(c)
         try:
+            ex.set_option(fm.PAE_OPT_PERSISTENT, 1)
             assert ex.query(fm.PAE_Q_PERSISTENT, 1) == 0
         finally:
             ex.close()
@@ -93,18 +97,55 @@ def test_gqa2_long_prefix_two_chunks_per_cta():
 
 
 @pytest.mark.slow
-def test_pi05_bf16_bs1_graph_path():
-    """The captured-graph path at batch 1 (the persistent kernel is the default there)."""
+def test_pi05_bf16_bs1_persistent():
+    """The persistent kernel at the full pi0.5 batch-1 size (the graph is the default there)."""
     cfg = wl.PI05_BF16_BS1
     ex, W = build_expert(cfg)
     try:
-        ex.set_option(fm.PAE_OPT_PERSISTENT, 0)
+        ex.set_option(fm.PAE_OPT_PERSISTENT, 1)
         ks, vs = wl.make_prefix(cfg)
         set_prefixes(ex, cfg, ks, vs)
         grid = wl.uniform_grid(cfg.steps)
         ex.precompute_tables(grid)
         noise = wl.make_noise(cfg)
         out = run_gpu(ex, noise)
-        assert_parity(out, oracle_rows(cfg, W, ks, vs, noise, grid), cfg.dtype, "pi05 bs1 graph path")
+        assert_parity(out, oracle_rows(cfg, W, ks, vs, noise, grid), cfg.dtype, "pi05 bs1 persistent")
+    finally:
+        ex.close()
+
+
+def test_persistent_wait_timeout_reports_status():
+    """With a 1 microsecond wait limit the persistent kernel's first grid barrier
+    runs out: the CTA that times out raises the launch-wide abort flag, every
+    other CTA's bounded wait sees it, each CTA drains its copies and MMAs and
+    frees TMEM, and the call reports PAE_ERR_TIMEOUT.  After pae_clear_error the
+    context gives the same result as before, bitwise."""
+    import torch
+    cfg = TINY_BF16.replace(name="tiny_bf16_pto")
+    ex, W = build_expert(cfg)
+    try:
+        ex.set_option(fm.PAE_OPT_PERSISTENT, 1)
+        ks, vs = wl.make_prefix(cfg)
+        set_prefixes(ex, cfg, ks, vs)
+        ex.precompute_tables(wl.uniform_grid(cfg.steps))
+        noise = wl.make_noise(cfg)
+        good = run_gpu(ex, noise)
+        ex.set_option(fm.PAE_OPT_WAIT_LIMIT_US, 1)
+        hit = False
+        for _ in range(20):
+            x = torch.from_numpy(noise).cuda()
+            try:
+                ex.denoise(x)
+                ex.sync()
+            except fm.PaeError as e:
+                assert e.status == fm.PAE_ERR_TIMEOUT
+                hit = True
+                break
+        fm.pae_clear_error(ex.ctx)
+        ex.set_option(fm.PAE_OPT_WAIT_LIMIT_US, 2_000_000)
+        again = run_gpu(ex, noise)
+        np.testing.assert_array_equal(again, good)
+        if not hit:
+            pytest.skip("no wait ran out at a 1 us limit on this run")
     finally:
         ex.close()
