@@ -55,6 +55,7 @@ struct TransitionArgs {
   const float* tab_in;    // table row of the step being started (null: no in step)
   float* x_dst;           // write x here after the out step (may equal x)
   int M;
+  float* ss_out;          // non-null: the first norm's sum of squares per token -> ss_out[m] (slot 0)
 };
 cudaError_t launch_transition(const Shape& s, int act_bf16, const TransitionArgs& a, bool pdl, cudaStream_t st);
 
@@ -76,6 +77,8 @@ struct EpiArgs {
   // EPI_RESID
   float* h;           // [M][D]
   const float* gate;  // [D]
+  float* ss_out;      // non-null: per-token sums of squares of the updated h, slot (tile * S + rank)
+  int ss_ld;          // token stride of the sum-of-squares slots
   // EPI_GEGLU
   void* u;            // [M][F]
 };
@@ -100,6 +103,12 @@ struct TcPlan {
 struct TcGemmArgs {
   EpiArgs e;
   const bf16* scales;  // int4 weights: [rows][K/128] group scales (null: bf16 weights)
+  // adaRMSNorm of the token operand inside the kernel (tmX is then the fp32
+  // residual stream): rstd from nslots sum-of-squares slots, scale / shift rows
+  const float* ss_in;
+  int nslots, ss_ld;
+  const float* nscale;
+  const float* nshift;
   int N;           // output features (GEGLU: F)
   int K;
   int w_row0;      // first row of this layer's matrix inside the stacked weight map
@@ -107,7 +116,7 @@ struct TcGemmArgs {
 };
 cudaError_t launch_tc_gemm(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* tmX, int na,
                            const TcPlan& p, const TcGemmArgs& a, bool pdl, cudaStream_t st);
-size_t tc_gemm_smem_bytes(int na, const TcPlan& p, bool w4);
+size_t tc_gemm_smem_bytes(int na, const TcPlan& p, bool w4, bool norm = false);
 cudaError_t tc_gemm_init();  // once per process: opt in to large dynamic shared memory
 
 // ------------------------------------------------------ tcgen05 attention

@@ -24,6 +24,11 @@
 // block; warps 4-7 dequantise it into the bf16 A tile (code * group scale,
 // rounded once) and arrive on a barrier the MMA thread waits for; the rest of
 // the pipeline and the epilogues are shared with the bf16 path.
+// In-kernel adaRMSNorm (small batches): the token operand comes from the fp32
+// residual stream h, TMA'd per K block into a staging tile; warps 4-7 turn it
+// into y = h * rstd * (1 + scale) + shift (bf16, swizzled) and arrive on the
+// same barrier.  rstd comes from per-token sum-of-squares slots that the
+// residual projections' split-K epilogue writes (one per tile and rank).
 #include "epilogue.cuh"
 #include "launch.cuh"
 
@@ -42,7 +47,7 @@ __host__ __device__ inline uint32_t tmem_cols_for(int n) {
 }
 
 struct TcSmemLayout {
-  uint32_t a_bytes, b_bytes, raw_bytes, stage_bytes, recv_off, recv_bytes, bar_off, total;
+  uint32_t a_bytes, b_bytes, raw_bytes, h_bytes, stage_bytes, recv_off, recv_bytes, bar_off, norm_off, total;
 };
 
 // Per stage: the bf16 weight tile A ([128*na][64], 128-byte swizzled), the
@@ -51,18 +56,20 @@ struct TcSmemLayout {
 // receive buffer ([na][src][token][R] fp32, na*tn*128 floats) follows the ring
 // or, when p.recv_alias, overlays it (then an extra cluster barrier makes sure
 // every peer's MMAs are done with its ring before anyone pushes).
-__host__ __device__ inline TcSmemLayout tc_layout(int na, const TcPlan& p, bool w4) {
+__host__ __device__ inline TcSmemLayout tc_layout(int na, const TcPlan& p, bool w4, bool norm = false) {
   TcSmemLayout L;
   L.a_bytes = (uint32_t)na * 128u * 128u;
   L.b_bytes = (uint32_t)p.tn * 128u;
   L.raw_bytes = w4 ? (uint32_t)na * 128u * 32u : 0u;
-  L.stage_bytes = L.a_bytes + L.b_bytes + L.raw_bytes;
+  L.h_bytes = norm ? (uint32_t)p.tn * 256u : 0u;  // fp32 [tn][64] residual staging
+  L.stage_bytes = L.a_bytes + L.b_bytes + L.raw_bytes + L.h_bytes;
   const uint32_t ring = L.stage_bytes * (uint32_t)p.stages;
   L.recv_bytes = p.splits > 1 ? (uint32_t)na * (uint32_t)p.tn * 128u * 4u : 0u;
   L.recv_off = p.recv_alias ? 0u : ring;
   const uint32_t used = p.recv_alias ? (ring > L.recv_bytes ? ring : L.recv_bytes) : ring + L.recv_bytes;
   L.bar_off = (used + 15u) & ~15u;
-  L.total = L.bar_off + 256 + 1024;  // barriers + slack for 1024-byte alignment
+  L.norm_off = L.bar_off + 256;  // rstd [64] + partial sums [2][64]
+  L.total = L.norm_off + (norm ? 768u : 0u) + 1024;  // + slack for 1024-byte alignment
   return L;
 }
 
@@ -202,16 +209,16 @@ __device__ __forceinline__ uint32_t dequant_pair(uint32_t w, int i, __nv_bfloat1
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-template <int NA, int EPI, bool SPLIT, bool W4>
+template <int NA, int EPI, bool SPLIT, bool W4, bool NORM>
 __global__ void __launch_bounds__(256, 2)
     k_tc_gemm(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, const Shape s,
               const TcPlan p, const TcGemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const TcSmemLayout L = tc_layout(NA, p, W4);
+  const TcSmemLayout L = tc_layout(NA, p, W4, NORM);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* empty = full + p.stages;
-  uint64_t* a_ready = empty + p.stages;  // int4 weights: dequantised A tile written
+  uint64_t* a_ready = empty + p.stages;  // int4 weights: A tile dequantised / norm: B tile built
   uint64_t* accf = a_ready + p.stages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
   volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);  // [0] abort
@@ -259,14 +266,15 @@ __global__ void __launch_bounds__(256, 2)
     const uint32_t wdst = W4 ? L.a_bytes + L.b_bytes : 0u;         // raw tile or A tile
     const int wx = W4 ? (k0 + 0) / 2 : k0;                            // packed: two codes per byte
     const int wstep = W4 ? 32 : 64;
-    const uint32_t tx = W4 ? L.raw_bytes + L.b_bytes : L.a_bytes + L.b_bytes;
+    const uint32_t tx = W4 ? L.raw_bytes + L.b_bytes : NORM ? L.a_bytes + L.h_bytes : L.a_bytes + L.b_bytes;
+    const uint32_t xdst = NORM ? L.a_bytes + L.b_bytes : L.a_bytes;  // fp32 staging or the B tile
     for (int kb = 0; kb < npre; ++kb) {
       mbar_arrive_expect_tx(&full[kb], tx);
       tma_load_2d_hint(smem + (size_t)kb * L.stage_bytes + wdst, &tmW, wx + kb * wstep, wrow, &full[kb], pol_w);
     }
     pdl_wait();
     for (int kb = 0; kb < npre; ++kb)
-      tma_load_2d(smem + (size_t)kb * L.stage_bytes + L.a_bytes, &tmX, k0 + kb * 64, ttile * p.tn, &full[kb]);
+      tma_load_2d(smem + (size_t)kb * L.stage_bytes + xdst, &tmX, k0 + kb * 64, ttile * p.tn, &full[kb]);
     int issued = npre;
     for (int kb = npre; kb < nkb; ++kb) {
       const int st = kb % p.stages;
@@ -278,7 +286,7 @@ __global__ void __launch_bounds__(256, 2)
       uint8_t* sa = smem + (size_t)st * L.stage_bytes;
       mbar_arrive_expect_tx(&full[st], tx);
       tma_load_2d_hint(sa + wdst, &tmW, wx + kb * wstep, wrow, &full[st], pol_w);
-      tma_load_2d(sa + L.a_bytes, &tmX, k0 + kb * 64, ttile * p.tn, &full[st]);
+      tma_load_2d(sa + xdst, &tmX, k0 + kb * 64, ttile * p.tn, &full[st]);
       issued = kb + 1;
     }
     // Loads still in flight must land before this CTA may exit.
@@ -290,7 +298,7 @@ __global__ void __launch_bounds__(256, 2)
     for (int kb = 0; kb < nkb; ++kb) {
       const int st = kb % p.stages;
       if (!mbar_wait(&full[st], (kb / p.stages) & 1, a.err.wait_ns) ||
-          (W4 && !mbar_wait(&a_ready[st], (kb / p.stages) & 1, a.err.wait_ns))) {
+          ((W4 || NORM) && !mbar_wait(&a_ready[st], (kb / p.stages) & 1, a.err.wait_ns))) {
         s_flag[0] = 1;
         set_error(a.err, DEV_TIMEOUT);
         break;
@@ -310,6 +318,68 @@ __global__ void __launch_bounds__(256, 2)
       umma_commit(&empty[st]);  // stage reusable once these MMAs have read it
     }
     umma_commit(accf);  // always issued, so the epilogue wait ends
+  } else if (NORM && warp >= 4) {
+    // ---------------------------------------------------------------- norm
+    // The sum-of-squares slots and the residual stream come from the previous
+    // kernel.  rstd for the tile's tokens first (thread = token, two halves of
+    // the slots, added in a fixed order), then per K block: thread = (token,
+    // 8 features) chunks of the fp32 staging tile -> bf16 y in the swizzled B
+    // tile.
+    pdl_wait();
+    const int ct = threadIdx.x - 128;
+    float* s_rstd = reinterpret_cast<float*>(smem + L.norm_off);
+    float* s_part = s_rstd + 64;
+    const int mbase = ttile * p.tn;
+    {
+      const int j = ct & 63, half = ct >> 6;
+      float acc = 0.f;
+      if (j < p.tn) {
+        const float* sp = a.ss_in + mbase + j;
+#pragma unroll 8
+        for (int sl = half; sl < a.nslots; sl += 2) acc += __ldcg(sp + (size_t)sl * a.ss_ld);
+      }
+      s_part[half * 64 + j] = acc;
+      named_bar(3, 128);
+      if (ct < 64) s_rstd[ct] = rsqrtf((s_part[ct] + s_part[64 + ct]) / (float)s.D + s.eps);
+      named_bar(3, 128);
+    }
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int st = kb % p.stages;
+      if (!mbar_wait(&full[st], (kb / p.stages) & 1, a.err.wait_ns)) {
+        s_flag[0] = 1;
+        set_error(a.err, DEV_TIMEOUT);
+        break;
+      }
+      uint8_t* stage = smem + (size_t)st * L.stage_bytes;
+      const float* hs = reinterpret_cast<const float*>(stage + L.a_bytes + L.b_bytes);
+      const uint32_t bbase = smem_u32(stage + L.a_bytes);
+      const int kf = k0 + kb * 64;
+      for (int i = ct; i < p.tn * 8; i += 128) {
+        const int r = i >> 3, q = i & 7;
+        const float4 h0 = *reinterpret_cast<const float4*>(hs + r * 64 + q * 8);
+        const float4 h1 = *reinterpret_cast<const float4*>(hs + r * 64 + q * 8 + 4);
+        const float4 c0 = __ldg(reinterpret_cast<const float4*>(a.nscale + kf + q * 8));
+        const float4 c1 = __ldg(reinterpret_cast<const float4*>(a.nscale + kf + q * 8 + 4));
+        const float4 d0 = __ldg(reinterpret_cast<const float4*>(a.nshift + kf + q * 8));
+        const float4 d1 = __ldg(reinterpret_cast<const float4*>(a.nshift + kf + q * 8 + 4));
+        const float rs = s_rstd[r];
+        const float y[8] = {h0.x * rs * (1.f + c0.x) + d0.x, h0.y * rs * (1.f + c0.y) + d0.y,
+                            h0.z * rs * (1.f + c0.z) + d0.z, h0.w * rs * (1.f + c0.w) + d0.w,
+                            h1.x * rs * (1.f + c1.x) + d1.x, h1.y * rs * (1.f + c1.y) + d1.y,
+                            h1.z * rs * (1.f + c1.z) + d1.z, h1.w * rs * (1.f + c1.w) + d1.w};
+        uint32_t w[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          w[t] = (uint32_t)__bfloat16_as_ushort(f2bf(y[2 * t])) |
+                 ((uint32_t)__bfloat16_as_ushort(f2bf(y[2 * t + 1])) << 16);
+        const uint32_t addr = bbase + (uint32_t)r * 128u + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                     "r"(w[3])
+                     : "memory");
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&a_ready[st]);
+    }
   } else if (W4 && warp >= 4) {
     // ---------------------------------------------------------------- dequant
     // Thread t owns weight row t (and t + 128 for the gate/up pair): its 64
@@ -458,7 +528,32 @@ __global__ void __launch_bounds__(256, 2)
             }
           }
         }
-        epi_batch<EPI, 8>(s, e, f, ms, s0, s1, n);
+        if (EPI == EPI_RESID && e.ss_out) {
+          // Gated residual, then the sum of squares of the updated h over this
+          // rank's R rows per token: the R threads of a token group are
+          // adjacent lanes (R is a power of two <= 32), reduced by a fixed
+          // shuffle tree into slot (tile * S + rank).
+          const float g = e.gate[f];
+          float hv[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (i < n) hv[i] = e.h[(size_t)ms[i] * s.D + f];
+          const int lane_g = (threadIdx.x & 31) & ~(R - 1);
+          const unsigned gmask = R >= 32 ? 0xffffffffu : (((1u << R) - 1u) << lane_g);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float v = 0.f;
+            if (i < n) {
+              hv[i] = fmaf(g, s0[i], hv[i]);
+              e.h[(size_t)ms[i] * s.D + f] = hv[i];
+              v = hv[i] * hv[i];
+            }
+            for (int o = R >> 1; o >= 1; o >>= 1) v += __shfl_xor_sync(gmask, v, o);
+            if (i < n && rr == 0) e.ss_out[(size_t)(ntile * S + (int)rank) * e.ss_ld + ms[i]] = v;
+          }
+        } else {
+          epi_batch<EPI, 8>(s, e, f, ms, s0, s1, n);
+        }
       }
     }
   }
@@ -468,58 +563,73 @@ __global__ void __launch_bounds__(256, 2)
   if (warp == 0) tmem_dealloc(tmem, ncols);
 }
 
-size_t smem_bytes_impl(int na, const TcPlan& p, bool w4) { return tc_layout(na, p, w4).total; }
+size_t smem_bytes_impl(int na, const TcPlan& p, bool w4, bool norm) { return tc_layout(na, p, w4, norm).total; }
 
-template <int NA, int EPI, bool SPLIT, bool W4>
+template <int NA, int EPI, bool SPLIT, bool W4, bool NORM>
 cudaError_t init_one() {
-  cudaError_t e = cudaFuncSetAttribute(k_tc_gemm<NA, EPI, SPLIT, W4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       227 * 1024);
-  if (e == cudaSuccess && SPLIT)
-    e = cudaFuncSetAttribute(k_tc_gemm<NA, EPI, SPLIT, W4>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  auto kern = k_tc_gemm<NA, EPI, SPLIT, W4, NORM>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e == cudaSuccess && SPLIT) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   return e;
 }
 
-template <int NA, int EPI, bool W4>
+template <int NA, int EPI, bool W4, bool NORM>
 cudaError_t launch_one(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* tmX, const TcPlan& p,
                        const TcGemmArgs& a, bool pdl, cudaStream_t st) {
   dim3 grid((a.N + 127) / 128, p.splits, p.tok_tiles);
-  const size_t smem = smem_bytes_impl(NA, p, W4);
+  const size_t smem = smem_bytes_impl(NA, p, W4, NORM);
   if (p.splits > 1)
-    return launch_ex(k_tc_gemm<NA, EPI, true, W4>, grid, dim3(256), smem, st, p.splits, pdl, *tmW, *tmX, s, p, a);
-  return launch_ex(k_tc_gemm<NA, EPI, false, W4>, grid, dim3(256), smem, st, 1, pdl, *tmW, *tmX, s, p, a);
+    return launch_ex(k_tc_gemm<NA, EPI, true, W4, NORM>, grid, dim3(256), smem, st, p.splits, pdl, *tmW, *tmX, s, p,
+                     a);
+  return launch_ex(k_tc_gemm<NA, EPI, false, W4, NORM>, grid, dim3(256), smem, st, 1, pdl, *tmW, *tmX, s, p, a);
 }
 
 template <bool W4>
 cudaError_t init_all() {
-  cudaError_t e = init_one<1, EPI_QKV, false, W4>();
-  if (e == cudaSuccess) e = init_one<1, EPI_QKV, true, W4>();
-  if (e == cudaSuccess) e = init_one<1, EPI_RESID, false, W4>();
-  if (e == cudaSuccess) e = init_one<1, EPI_RESID, true, W4>();
-  if (e == cudaSuccess) e = init_one<2, EPI_GEGLU, false, W4>();
-  if (e == cudaSuccess) e = init_one<2, EPI_GEGLU, true, W4>();
+  cudaError_t e = init_one<1, EPI_QKV, false, W4, false>();
+  if (e == cudaSuccess) e = init_one<1, EPI_QKV, true, W4, false>();
+  if (e == cudaSuccess) e = init_one<1, EPI_RESID, false, W4, false>();
+  if (e == cudaSuccess) e = init_one<1, EPI_RESID, true, W4, false>();
+  if (e == cudaSuccess) e = init_one<2, EPI_GEGLU, false, W4, false>();
+  if (e == cudaSuccess) e = init_one<2, EPI_GEGLU, true, W4, false>();
+  return e;
+}
+
+cudaError_t init_norm() {
+  cudaError_t e = init_one<1, EPI_QKV, false, false, true>();
+  if (e == cudaSuccess) e = init_one<1, EPI_QKV, true, false, true>();
+  if (e == cudaSuccess) e = init_one<2, EPI_GEGLU, false, false, true>();
+  if (e == cudaSuccess) e = init_one<2, EPI_GEGLU, true, false, true>();
   return e;
 }
 
 template <bool W4>
 cudaError_t launch_sel(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* tmX, int na, const TcPlan& p,
                        const TcGemmArgs& a, bool pdl, cudaStream_t st) {
-  if (na == 2) return launch_one<2, EPI_GEGLU, W4>(s, tmW, tmX, p, a, pdl, st);
-  if (a.e.epi == EPI_QKV) return launch_one<1, EPI_QKV, W4>(s, tmW, tmX, p, a, pdl, st);
-  return launch_one<1, EPI_RESID, W4>(s, tmW, tmX, p, a, pdl, st);
+  if (na == 2) return launch_one<2, EPI_GEGLU, W4, false>(s, tmW, tmX, p, a, pdl, st);
+  if (a.e.epi == EPI_QKV) return launch_one<1, EPI_QKV, W4, false>(s, tmW, tmX, p, a, pdl, st);
+  return launch_one<1, EPI_RESID, W4, false>(s, tmW, tmX, p, a, pdl, st);
 }
 
 }  // namespace
 
-size_t tc_gemm_smem_bytes(int na, const TcPlan& p, bool w4) { return smem_bytes_impl(na, p, w4); }
+size_t tc_gemm_smem_bytes(int na, const TcPlan& p, bool w4, bool norm) { return smem_bytes_impl(na, p, w4, norm); }
 
 cudaError_t tc_gemm_init() {
   cudaError_t e = init_all<false>();
   if (e == cudaSuccess) e = init_all<true>();
+  if (e == cudaSuccess) e = init_norm();
   return e;
 }
 
 cudaError_t launch_tc_gemm(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* tmX, int na, const TcPlan& p,
                            const TcGemmArgs& a, bool pdl, cudaStream_t st) {
+  if (a.ss_in) {  // adaRMSNorm in the kernel: bf16 weights only, QKV or gate/up
+    if (a.scales) return cudaErrorInvalidValue;
+    if (na == 2) return launch_one<2, EPI_GEGLU, false, true>(s, tmW, tmX, p, a, pdl, st);
+    if (a.e.epi != EPI_QKV) return cudaErrorInvalidValue;
+    return launch_one<1, EPI_QKV, false, true>(s, tmW, tmX, p, a, pdl, st);
+  }
   if (a.scales) return launch_sel<true>(s, tmW, tmX, na, p, a, pdl, st);
   return launch_sel<false>(s, tmW, tmX, na, p, a, pdl, st);
 }

@@ -162,6 +162,7 @@ __global__ void __launch_bounds__(256) k_transition(const Shape s, const Transit
       ss = fmaf(acc[0], acc[0], fmaf(acc[1], acc[1], fmaf(acc[2], acc[2], fmaf(acc[3], acc[3], ss))));
     }
     ss = block_sum(ss, red);
+    if (a.ss_out && tid == 0) a.ss_out[m] = ss;  // slot 0 for a projection that normalises in-kernel
     const float r = rsqrtf(ss / (float)D + s.eps);
     const float* sc = a.tab_in + mod_offset(s, 0, 0, 0);
     const float* sh = a.tab_in + mod_offset(s, 0, 0, 1);

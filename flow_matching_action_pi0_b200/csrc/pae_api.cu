@@ -37,6 +37,7 @@ void set_create_error(const char* msg) { g_create_error = msg ? msg : ""; }
 namespace {
 
 constexpr int kMaxSteps = 64;
+constexpr int kSsSlots = 256;  // sum-of-squares slots: (D / 128) tiles x split-K ranks
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -53,7 +54,8 @@ struct Plan {
   AttnPlan attn{};
   bool persist = false;  // eligible for the persistent kernel
   PersistArgs pa{};
-  CUtensorMap tmY{}, tmO{}, tmU{};
+  bool fuse_norm = false;  // QKV / gate-up normalise their fp32 operand in-kernel
+  CUtensorMap tmY{}, tmO{}, tmU{}, tmH{};
   cudaGraphExec_t graph = nullptr;
   int graph_K = 0;
   long long graph_kernels = 0;
@@ -119,6 +121,10 @@ struct pae_ctx {
   float* pw_part = nullptr;
   float* pw_ss = nullptr;
   unsigned* pw_ctr = nullptr;
+  // in-kernel adaRMSNorm: per-token sum-of-squares slots [kSsSlots][ss_ld]
+  bool use_fused_norm = true;
+  float* ss_buf = nullptr;
+  int ss_ld = 0;
   // int4 weights (W4A16): packed codes [L*rows][K/2] and group scales [L*rows][K/128]
   int w4 = 0;
   void *q_qkv = nullptr, *q_o = nullptr, *q_gu = nullptr, *q_down = nullptr;
@@ -211,6 +217,21 @@ pae_status make_map(pae_ctx* ctx, CUtensorMap* m, const void* base, uint64_t inn
   return PAE_OK;
 }
 
+pae_status make_map_f32(pae_ctx* ctx, CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                        uint32_t box_inner, uint32_t box_outer) {
+  // fp32 matrix [outer][inner], unswizzled boxes (the residual stream tiles).
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 4};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = ctx->encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, es,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(ctx, PAE_ERR_CUDA, "cuTensorMapEncodeTiled (fp32) failed (%d)", (int)r);
+  return PAE_OK;
+}
+
 pae_status make_map_u8(pae_ctx* ctx, CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                        uint32_t box_inner, uint32_t box_outer) {
   // uint8 matrix [outer][inner], unswizzled boxes (the packed int4 tiles).
@@ -232,14 +253,15 @@ pae_status make_map_u8(pae_ctx* ctx, CUtensorMap* m, const void* base, uint64_t 
 // divides the 64-wide K blocks) fills the 148 SMs when the tile count is small;
 // small token tiles keep shared memory under half an SM so that two CTAs (or a
 // CTA and its successor under PDL) fit per SM.
-TcPlan plan_gemm(int M, int nfeat, int K, int na, int max_splits = 16, bool w4 = false) {
+TcPlan plan_gemm(int M, int nfeat, int K, int na, int max_splits = 16, bool w4 = false, bool norm = false) {
   TcPlan p{};
   p.tok_tiles = (M + 255) / 256;
   int per = (M + p.tok_tiles - 1) / p.tok_tiles;
   p.tn = std::max(16, ((per + 15) / 16) * 16);
   const int base = ((nfeat + 127) / 128) * p.tok_tiles;
   const int nkb = K / 64;
-  const uint32_t stage = (uint32_t)na * 16384u + (uint32_t)p.tn * 128u + (w4 ? (uint32_t)na * 4096u : 0u);
+  const uint32_t stage = (uint32_t)na * 16384u + (uint32_t)p.tn * 128u + (w4 ? (uint32_t)na * 4096u : 0u) +
+                         (norm ? (uint32_t)p.tn * 256u : 0u);
   const uint32_t recv = (uint32_t)na * p.tn * 128u * 4u;  // split-K receive buffer
   const bool small = p.tn <= 64;  // two CTAs per SM (shared memory and the 128-register cap allow it)
   const uint32_t budget = small ? 110u * 1024u : 200u * 1024u;
@@ -351,16 +373,24 @@ pae_status build_plan(pae_ctx* ctx, int B, Plan* P) {
   if (!ctx->act_bf16) return PAE_OK;
   P->persist = plan_persistent(ctx, B, &P->pa);
   const bool w4 = ctx->w4 != 0;
-  P->qkv = plan_gemm(P->M, s.qkv_rows, s.D, 1, ctx->max_splitk, w4);
   P->o = plan_gemm(P->M, s.D, s.attn_dim, 1, ctx->max_splitk, w4);
-  P->gu = plan_gemm(P->M, s.F, s.D, 2, ctx->max_splitk, w4);
   P->down = plan_gemm(P->M, s.D, s.F, 1, ctx->max_splitk, w4);
+  // In-kernel adaRMSNorm for small batches (one token tile of <= 64): the
+  // residual projections' split-K ranks (R = 128 / S <= 32 rows each) write
+  // the sum-of-squares slots, so the separate norm kernels disappear.
+  const int tn_small = std::max(16, ((P->M + 15) / 16) * 16);
+  P->fuse_norm = ctx->use_fused_norm && !w4 && P->M <= 64 && tn_small <= 64 && P->o.splits >= 4 &&
+                 P->down.splits >= 4 && P->o.tok_tiles == 1 && P->down.tok_tiles == 1 &&
+                 (s.D / 128) * std::max(P->o.splits, P->down.splits) <= kSsSlots;
+  P->qkv = plan_gemm(P->M, s.qkv_rows, s.D, 1, ctx->max_splitk, w4, P->fuse_norm);
+  P->gu = plan_gemm(P->M, s.F, s.D, 2, ctx->max_splitk, w4, P->fuse_norm);
   P->attn = plan_attn(s, B);
   const uint64_t Mmax = (uint64_t)s.Bmax * s.H;
   pae_status st;
   if ((st = make_map(ctx, &P->tmY, ctx->y, s.D, Mmax, 64, P->qkv.tn)) != PAE_OK) return st;
   if ((st = make_map(ctx, &P->tmO, ctx->o, s.attn_dim, Mmax, 64, P->o.tn)) != PAE_OK) return st;
   if ((st = make_map(ctx, &P->tmU, ctx->u, s.F, Mmax, 64, P->down.tn)) != PAE_OK) return st;
+  if (P->fuse_norm && (st = make_map_f32(ctx, &P->tmH, ctx->h, s.D, Mmax, 64, P->qkv.tn)) != PAE_OK) return st;
   return PAE_OK;
 }
 
@@ -414,7 +444,16 @@ bool pdl_on(const pae_ctx* ctx) { return ctx->use_pdl && ctx->act_bf16 && ctx->p
 
 const float* tab(const pae_ctx* ctx, int k) { return ctx->tables + (size_t)k * ctx->s.table_rows; }
 
-void run_gemm(pae_ctx* ctx, const Plan& P, int which, int layer, const EpiArgs& e, cudaStream_t st) {
+// `norm` (QKV and gate/up with P.fuse_norm): the step's scale / shift rows of
+// that adaRMSNorm and how many sum-of-squares slots hold its statistics.
+struct NormIn {
+  const float* scale = nullptr;
+  const float* shift = nullptr;
+  int nslots = 0;
+};
+
+void run_gemm(pae_ctx* ctx, const Plan& P, int which, int layer, const EpiArgs& e, cudaStream_t st,
+              const NormIn& norm = NormIn{}) {
   const Shape& s = ctx->s;
   const size_t es = ctx->esize;
   if (!ctx->act_bf16) {
@@ -448,6 +487,14 @@ void run_gemm(pae_ctx* ctx, const Plan& P, int which, int layer, const EpiArgs& 
              a.w_row0 = layer * s.D; a.scales = (const bf16*)ctx->sc_down; break;
   }
   if (!w4) a.scales = nullptr;
+  if (norm.scale) {
+    tx = &P.tmH;
+    a.ss_in = ctx->ss_buf;
+    a.ss_ld = ctx->ss_ld;
+    a.nslots = norm.nslots;
+    a.nscale = norm.scale;
+    a.nshift = norm.shift;
+  }
   launch_tc_gemm(s, tw, tx, na, *p, a, pdl_on(ctx), st);
 }
 
@@ -468,7 +515,9 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
   ta.b_out = ctx->b_out;
   ta.dt = ctx->dt;
   ta.M = M;
+  ta.ss_out = P.fuse_norm ? ctx->ss_buf : nullptr;
   ctx->ev_next = 0;
+  const int slots_o = (s.D / 128) * P.o.splits, slots_down = (s.D / 128) * P.down.splits;
   for (int k = k_begin; k < k_end; ++k) {
     const float* tk = tab(ctx, k);
     ta.tab_out = (k == k_begin) ? nullptr : tab(ctx, k - 1);
@@ -489,7 +538,9 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
       e.lens = ctx->lens_dev;
       {
         ProfScope ps(ctx, PAE_K_QKV, st);
-        run_gemm(ctx, P, 0, l, e, st);
+        NormIn nq;
+        if (P.fuse_norm) nq = NormIn{tk + mod_offset(s, l, 0, 0), tk + mod_offset(s, l, 0, 1), l == 0 ? 1 : slots_down};
+        run_gemm(ctx, P, 0, l, e, st, nq);
       }
       {
         ProfScope ps(ctx, PAE_K_ATTENTION, st);
@@ -510,11 +561,15 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
       e.epi = EPI_RESID;
       e.h = ctx->h;
       e.gate = tk + mod_offset(s, l, 0, 2);
+      if (P.fuse_norm) {
+        e.ss_out = ctx->ss_buf;
+        e.ss_ld = ctx->ss_ld;
+      }
       {
         ProfScope ps(ctx, PAE_K_OPROJ, st);
         run_gemm(ctx, P, 1, l, e, st);
       }
-      {
+      if (!P.fuse_norm) {
         ProfScope ps(ctx, PAE_K_NORM, st);
         launch_norm(s, ctx->act_bf16, ctx->h, ctx->y, tk + mod_offset(s, l, 1, 0), tk + mod_offset(s, l, 1, 1), M,
                     pdl_on(ctx), st);
@@ -525,18 +580,24 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
       e.u = ctx->u;
       {
         ProfScope ps(ctx, PAE_K_GATEUP, st);
-        run_gemm(ctx, P, 2, l, e, st);
+        NormIn ng;
+        if (P.fuse_norm) ng = NormIn{tk + mod_offset(s, l, 1, 0), tk + mod_offset(s, l, 1, 1), slots_o};
+        run_gemm(ctx, P, 2, l, e, st, ng);
       }
       e = EpiArgs{};
       e.M = M;
       e.epi = EPI_RESID;
       e.h = ctx->h;
       e.gate = tk + mod_offset(s, l, 1, 2);
+      if (P.fuse_norm) {
+        e.ss_out = ctx->ss_buf;
+        e.ss_ld = ctx->ss_ld;
+      }
       {
         ProfScope ps(ctx, PAE_K_DOWN, st);
         run_gemm(ctx, P, 3, l, e, st);
       }
-      if (l + 1 < s.L) {
+      if (l + 1 < s.L && !P.fuse_norm) {
         ProfScope ps(ctx, PAE_K_NORM, st);
         launch_norm(s, ctx->act_bf16, ctx->h, ctx->y, tk + mod_offset(s, l + 1, 0, 0), tk + mod_offset(s, l + 1, 0, 1),
                     M, pdl_on(ctx), st);
@@ -903,6 +964,9 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
   CKC(cudaMemsetAsync(ctx->y, 0, Mpad * D * es, cs));
   CKC(cudaMemsetAsync(ctx->o, 0, Mpad * s.attn_dim * es, cs));
   CKC(cudaMemsetAsync(ctx->u, 0, Mpad * F * es, cs));
+  ctx->ss_ld = (int)Mpad;
+  ALLOC(ctx->ss_buf, sizeof(float) * kSsSlots * Mpad);
+  CKC(cudaMemsetAsync(ctx->ss_buf, 0, sizeof(float) * kSsSlots * Mpad, cs));
   if (ctx->act_bf16 && !ctx->w4) {
     if ((st = make_map(ctx, &ctx->tmWqkv, ctx->w_qkv, D, (uint64_t)L * s.qkv_rows, 64, 128)) != PAE_OK) return bail(st);
     if ((st = make_map(ctx, &ctx->tmWo, ctx->w_o, s.attn_dim, (uint64_t)L * D, 64, 128)) != PAE_OK) return bail(st);
@@ -1085,6 +1149,14 @@ pae_status pae_set_option(pae_ctx* ctx, int option, long long value) {
       ctx->use_pdl = value != 0;
       return PAE_OK;
     case PAE_OPT_PERSISTENT: ctx->use_persistent = value != 0; return PAE_OK;
+    case PAE_OPT_FUSED_NORM:
+      if ((value != 0) != ctx->use_fused_norm) {
+        drop_graphs(ctx);
+        ctx->plans.clear();
+        ctx->last_plan = nullptr;
+      }
+      ctx->use_fused_norm = value != 0;
+      return PAE_OK;
     case PAE_OPT_PROFILE:
       if (value < 0 || value >= (1LL << PAE_K_COUNT)) return fail(ctx, PAE_ERR_ARG, "bad profile mask");
       if ((unsigned)value != ctx->profile_mask) drop_graphs(ctx);
@@ -1125,6 +1197,7 @@ pae_status pae_query(pae_ctx* ctx, int what, int batch, long long* value) {
     case PAE_Q_TOKEN_TILE: *value = P->qkv.tn; return PAE_OK;
     case PAE_Q_ATTN_SPLITS: *value = P->attn.splits; return PAE_OK;
     case PAE_Q_PERSISTENT: *value = use_persist(ctx, P) ? 1 : 0; return PAE_OK;
+    case PAE_Q_FUSED_NORM: *value = P->fuse_norm ? 1 : 0; return PAE_OK;
     default: return fail(ctx, PAE_ERR_ARG, "unknown query %d", what);
   }
 }

@@ -163,13 +163,19 @@ pae_status pae_denoise_steps(pae_ctx* ctx, const float* x_in, float* x_out, int 
  * each layer) instead of the graph of per-phase kernels, for batches with
  * batch * chunk <= 64.  The two paths round differently (both stay within
  * the parity tolerance); each is bitwise reproducible on its own, and
- * pae_denoise and pae_denoise_steps take the same path for the same batch. */
+ * pae_denoise and pae_denoise_steps take the same path for the same batch.
+ * PAE_OPT_FUSED_NORM (default 1, bf16 weights): for batches of at most one
+ * 64-token tile, the QKV and gate/up projections apply the adaRMSNorm to their
+ * fp32 input inside the kernel (statistics from the residual projections'
+ * epilogues) instead of separate norm kernels; 0 keeps the norm kernels.
+ * Both round within the parity tolerance; each is bitwise reproducible. */
 enum {
   PAE_OPT_USE_GRAPH = 1,
   PAE_OPT_WAIT_LIMIT_US = 2,
   PAE_OPT_PDL = 4,
   PAE_OPT_MAX_SPLITK = 5,
-  PAE_OPT_PERSISTENT = 6
+  PAE_OPT_PERSISTENT = 6,
+  PAE_OPT_FUSED_NORM = 7
 };
 pae_status pae_set_option(pae_ctx* ctx, int option, long long value);
 
@@ -198,13 +204,16 @@ pae_status pae_profile_read(pae_ctx* ctx, int kernel_class, double* total_ms, in
  * projections for `batch`, packed as qkv | o<<8 | gateup<<16 | down<<24.
  * PAE_Q_TOKEN_TILE: MMA token tile for `batch`.  PAE_Q_ATTN_SPLITS: key splits
  * of the attention for `batch`.  PAE_Q_PERSISTENT: 1 if pae_denoise runs the
- * persistent kernel for `batch` (option on and the batch eligible), else 0. */
+ * persistent kernel for `batch` (option on and the batch eligible), else 0.
+ * PAE_Q_FUSED_NORM: 1 if the graph for `batch` normalises inside the
+ * projections (no separate norm kernels), else 0. */
 enum {
   PAE_Q_GRAPH_KERNELS = 1,
   PAE_Q_SPLITS = 2,
   PAE_Q_TOKEN_TILE = 3,
   PAE_Q_ATTN_SPLITS = 4,
-  PAE_Q_PERSISTENT = 5
+  PAE_Q_PERSISTENT = 5,
+  PAE_Q_FUSED_NORM = 6
 };
 pae_status pae_query(pae_ctx* ctx, int what, int batch, long long* value);
 

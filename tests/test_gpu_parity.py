@@ -8,6 +8,7 @@ configuration the benchmark times (captured graph, same batch size).
 import numpy as np
 import pytest
 
+import flow_matching_action_pi0_b200 as fm
 import workloads as wl
 from tests.helpers import assert_parity, build_expert, oracle_rows, run_gpu, set_prefixes
 
@@ -85,3 +86,34 @@ def test_ragged_bf16_bs16_sampled_rows():
     lens = wl.prefix_lengths(cfg)
     rows = [int(np.argmin(lens)), int(np.argmax(lens)), 7]
     _run_case(cfg, rows=rows)
+
+
+def _fused_vs_separate(cfg, lengths=None):
+    ex, W = build_expert(cfg)
+    try:
+        ks, vs = wl.make_prefix(cfg, lengths=lengths)
+        set_prefixes(ex, cfg, ks, vs)
+        grid = wl.uniform_grid(cfg.steps)
+        ex.precompute_tables(grid)
+        noise = wl.make_noise(cfg)
+        assert ex.query(fm.PAE_Q_FUSED_NORM, cfg.batch) == 1
+        fused = run_gpu(ex, noise)
+        np.testing.assert_array_equal(run_gpu(ex, noise), fused)  # bitwise reproducible
+        ex.set_option(fm.PAE_OPT_FUSED_NORM, 0)
+        assert ex.query(fm.PAE_Q_FUSED_NORM, cfg.batch) == 0
+        sep = run_gpu(ex, noise)
+        ref = oracle_rows(cfg, W, ks, vs, noise, grid)
+        assert_parity(fused, ref, cfg.dtype, cfg.name + " in-kernel norm")
+        assert_parity(sep, ref, cfg.dtype, cfg.name + " norm kernels")
+    finally:
+        ex.close()
+
+
+def test_fused_norm_tiny_batch3_ragged():
+    # adaRMSNorm inside the QKV / gate-up projections vs the separate norm kernels
+    _fused_vs_separate(wl.TINY_FP32.replace(name="tiny_bf16_fn", dtype=wl.BF16, batch=3), lengths=[64, 5, 0])
+
+
+@pytest.mark.slow
+def test_fused_norm_pi05_bs1():
+    _fused_vs_separate(wl.PI05_BF16_BS1)
