@@ -110,6 +110,9 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
 
 
+FUSED_NORM = [0]  # PAE_OPT_FUSED_NORM for every context the benchmark creates
+
+
 def algorithmic(cfg: wl.ExpertConfig, batch: int, lens=None):
     """Algorithmic bytes and FLOPs per launch of each kernel class and per
     Euler step (weights and prefix/action K/V once, activations once; table
@@ -236,6 +239,7 @@ def setup_context(cfg, W, batch: int, lens=None):
     dev_w = wd.upload_weights(cfg, W)
     ex = fm.ActionExpert(fm.make_config(**wd.abi_config(cfg, max_batch=batch)), dev_w)
     del dev_w
+    ex.set_option(fm.PAE_OPT_FUSED_NORM, FUSED_NORM[0])
     if lens is None:
         lens = [cfg.prefix] * batch
     ks, vs = wl.make_prefix(cfg, lengths=lens)
@@ -562,12 +566,15 @@ def main():
     ap.add_argument("--minimal", action="store_true", help="only warm-up and timed calls (for profilers)")
     ap.add_argument("--pdl", type=int, default=1, help="programmatic dependent launch inside the loop (1/0)")
     ap.add_argument("--max-splitk", type=int, default=0, help="cap on the projection split-K (0: library default)")
+    ap.add_argument("--fused-norm", type=int, default=0,
+                    help="adaRMSNorm inside the projections for batches of <= 64 tokens (1/0; 0 keeps norm kernels)")
     ap.add_argument("--persistent", type=int, default=0,
                     help="persistent kernel for batches of <= 64 tokens (1/0; 0 runs the captured graph)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     cfg = wl.CONFIGS[args.config]
+    FUSED_NORM[0] = args.fused_norm
     if args.impl == "reference":
         return run_reference(args, cfg)
     if args.minimal:

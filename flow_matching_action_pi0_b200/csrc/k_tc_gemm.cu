@@ -61,7 +61,9 @@ __host__ __device__ inline TcSmemLayout tc_layout(int na, const TcPlan& p, bool 
   L.a_bytes = (uint32_t)na * 128u * 128u;
   L.b_bytes = (uint32_t)p.tn * 128u;
   L.raw_bytes = w4 ? (uint32_t)na * 128u * 32u : 0u;
-  L.h_bytes = norm ? (uint32_t)p.tn * 256u : 0u;  // fp32 [tn][64] residual staging
+  // norm: fp32 [tn][64] residual staging at the B position; the bf16 B tile is
+  // written over its front half once every thread has read its chunks
+  L.h_bytes = norm ? (uint32_t)p.tn * 128u : 0u;
   L.stage_bytes = L.a_bytes + L.b_bytes + L.raw_bytes + L.h_bytes;
   const uint32_t ring = L.stage_bytes * (uint32_t)p.stages;
   L.recv_bytes = p.splits > 1 ? (uint32_t)na * (uint32_t)p.tn * 128u * 4u : 0u;
@@ -266,8 +268,8 @@ __global__ void __launch_bounds__(256, 2)
     const uint32_t wdst = W4 ? L.a_bytes + L.b_bytes : 0u;         // raw tile or A tile
     const int wx = W4 ? (k0 + 0) / 2 : k0;                            // packed: two codes per byte
     const int wstep = W4 ? 32 : 64;
-    const uint32_t tx = W4 ? L.raw_bytes + L.b_bytes : NORM ? L.a_bytes + L.h_bytes : L.a_bytes + L.b_bytes;
-    const uint32_t xdst = NORM ? L.a_bytes + L.b_bytes : L.a_bytes;  // fp32 staging or the B tile
+    const uint32_t tx = W4 ? L.raw_bytes + L.b_bytes : NORM ? L.a_bytes + L.b_bytes + L.h_bytes : L.a_bytes + L.b_bytes;
+    const uint32_t xdst = L.a_bytes;  // the B tile, or (norm) the fp32 staging that the B tile overlays
     for (int kb = 0; kb < npre; ++kb) {
       mbar_arrive_expect_tx(&full[kb], tx);
       tma_load_2d_hint(smem + (size_t)kb * L.stage_bytes + wdst, &tmW, wx + kb * wstep, wrow, &full[kb], pol_w);
@@ -325,18 +327,41 @@ __global__ void __launch_bounds__(256, 2)
     // the slots, added in a fixed order), then per K block: thread = (token,
     // 8 features) chunks of the fp32 staging tile -> bf16 y in the swizzled B
     // tile.
-    pdl_wait();
+    // The scale / shift rows (tables built before the loop) are read before
+    // waiting for the previous kernel; a thread's 8 features are the same in
+    // every K block (chunk index q = thread % 8), at most two blocks here.
     const int ct = threadIdx.x - 128;
+    const int qf = (ct & 7) * 8;
+    float4 tc[2][4];
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb)
+      if (kb < nkb) {
+        const int kf = k0 + kb * 64 + qf;
+        tc[kb][0] = __ldg(reinterpret_cast<const float4*>(a.nscale + kf));
+        tc[kb][1] = __ldg(reinterpret_cast<const float4*>(a.nscale + kf + 4));
+        tc[kb][2] = __ldg(reinterpret_cast<const float4*>(a.nshift + kf));
+        tc[kb][3] = __ldg(reinterpret_cast<const float4*>(a.nshift + kf + 4));
+      }
+    pdl_wait();
     float* s_rstd = reinterpret_cast<float*>(smem + L.norm_off);
     float* s_part = s_rstd + 64;
     const int mbase = ttile * p.tn;
     {
+      // thread = (token j, half): slots half, half + 2, ... with all loads in flight
       const int j = ct & 63, half = ct >> 6;
       float acc = 0.f;
       if (j < p.tn) {
         const float* sp = a.ss_in + mbase + j;
-#pragma unroll 8
-        for (int sl = half; sl < a.nslots; sl += 2) acc += __ldcg(sp + (size_t)sl * a.ss_ld);
+        constexpr int NB = 32;
+        for (int s0 = half; s0 < a.nslots; s0 += 2 * NB) {
+          float v[NB];
+#pragma unroll
+          for (int i = 0; i < NB; ++i)
+            if (s0 + 2 * i < a.nslots) v[i] = __ldcg(sp + (size_t)(s0 + 2 * i) * a.ss_ld);
+#pragma unroll
+          for (int i = 0; i < NB; ++i)
+            if (s0 + 2 * i < a.nslots) acc += v[i];
+        }
       }
       s_part[half * 64 + j] = acc;
       named_bar(3, 128);
@@ -351,31 +376,57 @@ __global__ void __launch_bounds__(256, 2)
         break;
       }
       uint8_t* stage = smem + (size_t)st * L.stage_bytes;
-      const float* hs = reinterpret_cast<const float*>(stage + L.a_bytes + L.b_bytes);
+      const float* hs = reinterpret_cast<const float*>(stage + L.a_bytes);
       const uint32_t bbase = smem_u32(stage + L.a_bytes);
-      const int kf = k0 + kb * 64;
-      for (int i = ct; i < p.tn * 8; i += 128) {
-        const int r = i >> 3, q = i & 7;
-        const float4 h0 = *reinterpret_cast<const float4*>(hs + r * 64 + q * 8);
-        const float4 h1 = *reinterpret_cast<const float4*>(hs + r * 64 + q * 8 + 4);
-        const float4 c0 = __ldg(reinterpret_cast<const float4*>(a.nscale + kf + q * 8));
-        const float4 c1 = __ldg(reinterpret_cast<const float4*>(a.nscale + kf + q * 8 + 4));
-        const float4 d0 = __ldg(reinterpret_cast<const float4*>(a.nshift + kf + q * 8));
-        const float4 d1 = __ldg(reinterpret_cast<const float4*>(a.nshift + kf + q * 8 + 4));
-        const float rs = s_rstd[r];
-        const float y[8] = {h0.x * rs * (1.f + c0.x) + d0.x, h0.y * rs * (1.f + c0.y) + d0.y,
-                            h0.z * rs * (1.f + c0.z) + d0.z, h0.w * rs * (1.f + c0.w) + d0.w,
-                            h1.x * rs * (1.f + c1.x) + d1.x, h1.y * rs * (1.f + c1.y) + d1.y,
-                            h1.z * rs * (1.f + c1.z) + d1.z, h1.w * rs * (1.f + c1.w) + d1.w};
-        uint32_t w[4];
+      float4 c0, c1, d0, d1;
+      if (kb == 0) {
+        c0 = tc[0][0];
+        c1 = tc[0][1];
+        d0 = tc[0][2];
+        d1 = tc[0][3];
+      } else if (kb == 1) {
+        c0 = tc[1][0];
+        c1 = tc[1][1];
+        d0 = tc[1][2];
+        d1 = tc[1][3];
+      } else {
+        const int kf = k0 + kb * 64 + qf;
+        c0 = __ldg(reinterpret_cast<const float4*>(a.nscale + kf));
+        c1 = __ldg(reinterpret_cast<const float4*>(a.nscale + kf + 4));
+        d0 = __ldg(reinterpret_cast<const float4*>(a.nshift + kf));
+        d1 = __ldg(reinterpret_cast<const float4*>(a.nshift + kf + 4));
+      }
+      // thread = (token, 8 features): at most four chunks per thread (tn <= 64)
+      uint32_t w[4][4];
 #pragma unroll
-        for (int t = 0; t < 4; ++t)
-          w[t] = (uint32_t)__bfloat16_as_ushort(f2bf(y[2 * t])) |
-                 ((uint32_t)__bfloat16_as_ushort(f2bf(y[2 * t + 1])) << 16);
-        const uint32_t addr = bbase + (uint32_t)r * 128u + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]),
-                     "r"(w[3])
-                     : "memory");
+      for (int c = 0; c < 4; ++c) {
+        const int i = ct + c * 128;
+        if (i < p.tn * 8) {
+          const int r = i >> 3;
+          const float4 h0 = *reinterpret_cast<const float4*>(hs + r * 64 + qf);
+          const float4 h1 = *reinterpret_cast<const float4*>(hs + r * 64 + qf + 4);
+          const float rs = s_rstd[r];
+          const float y[8] = {h0.x * rs * (1.f + c0.x) + d0.x, h0.y * rs * (1.f + c0.y) + d0.y,
+                              h0.z * rs * (1.f + c0.z) + d0.z, h0.w * rs * (1.f + c0.w) + d0.w,
+                              h1.x * rs * (1.f + c1.x) + d1.x, h1.y * rs * (1.f + c1.y) + d1.y,
+                              h1.z * rs * (1.f + c1.z) + d1.z, h1.w * rs * (1.f + c1.w) + d1.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t)
+            w[c][t] = (uint32_t)__bfloat16_as_ushort(f2bf(y[2 * t])) |
+                      ((uint32_t)__bfloat16_as_ushort(f2bf(y[2 * t + 1])) << 16);
+        }
+      }
+      named_bar(3, 128);  // every chunk of the staging is read before B overwrites it
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int i = ct + c * 128;
+        if (i < p.tn * 8) {
+          const int r = i >> 3, q = i & 7;
+          const uint32_t addr = bbase + (uint32_t)r * 128u + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[c][0]), "r"(w[c][1]),
+                       "r"(w[c][2]), "r"(w[c][3])
+                       : "memory");
+        }
       }
       fence_proxy_async_smem();
       mbar_arrive(&a_ready[st]);
@@ -540,16 +591,28 @@ __global__ void __launch_bounds__(256, 2)
             if (i < n) hv[i] = e.h[(size_t)ms[i] * s.D + f];
           const int lane_g = (threadIdx.x & 31) & ~(R - 1);
           const unsigned gmask = R >= 32 ? 0xffffffffu : (((1u << R) - 1u) << lane_g);
+          float v[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            float v = 0.f;
+            v[i] = 0.f;
             if (i < n) {
               hv[i] = fmaf(g, s0[i], hv[i]);
               e.h[(size_t)ms[i] * s.D + f] = hv[i];
-              v = hv[i] * hv[i];
+              v[i] = hv[i] * hv[i];
             }
-            for (int o = R >> 1; o >= 1; o >>= 1) v += __shfl_xor_sync(gmask, v, o);
-            if (i < n && rr == 0) e.ss_out[(size_t)(ntile * S + (int)rank) * e.ss_ld + ms[i]] = v;
+          }
+#pragma unroll
+          for (int lv = 4; lv >= 0; --lv) {  // offsets R/2 .. 1, all eight tokens per level
+            const int o = 1 << lv;
+            if (o < R) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[i] += __shfl_xor_sync(gmask, v[i], o);
+            }
+          }
+          if (rr == 0) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              if (i < n) e.ss_out[(size_t)(ntile * S + (int)rank) * e.ss_ld + ms[i]] = v[i];
           }
         } else {
           epi_batch<EPI, 8>(s, e, f, ms, s0, s1, n);

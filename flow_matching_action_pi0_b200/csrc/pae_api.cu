@@ -122,7 +122,7 @@ struct pae_ctx {
   float* pw_ss = nullptr;
   unsigned* pw_ctr = nullptr;
   // in-kernel adaRMSNorm: per-token sum-of-squares slots [kSsSlots][ss_ld]
-  bool use_fused_norm = true;
+  bool use_fused_norm = false;  // opt-in: measured slower than the norm kernels under PDL
   float* ss_buf = nullptr;
   int ss_ld = 0;
   // int4 weights (W4A16): packed codes [L*rows][K/2] and group scales [L*rows][K/128]
@@ -261,7 +261,7 @@ TcPlan plan_gemm(int M, int nfeat, int K, int na, int max_splits = 16, bool w4 =
   const int base = ((nfeat + 127) / 128) * p.tok_tiles;
   const int nkb = K / 64;
   const uint32_t stage = (uint32_t)na * 16384u + (uint32_t)p.tn * 128u + (w4 ? (uint32_t)na * 4096u : 0u) +
-                         (norm ? (uint32_t)p.tn * 256u : 0u);
+                         (norm ? (uint32_t)p.tn * 128u : 0u);
   const uint32_t recv = (uint32_t)na * p.tn * 128u * 4u;  // split-K receive buffer
   const bool small = p.tn <= 64;  // two CTAs per SM (shared memory and the 128-register cap allow it)
   const uint32_t budget = small ? 110u * 1024u : 200u * 1024u;

@@ -164,11 +164,11 @@ pae_status pae_denoise_steps(pae_ctx* ctx, const float* x_in, float* x_out, int 
  * batch * chunk <= 64.  The two paths round differently (both stay within
  * the parity tolerance); each is bitwise reproducible on its own, and
  * pae_denoise and pae_denoise_steps take the same path for the same batch.
- * PAE_OPT_FUSED_NORM (default 1, bf16 weights): for batches of at most one
- * 64-token tile, the QKV and gate/up projections apply the adaRMSNorm to their
- * fp32 input inside the kernel (statistics from the residual projections'
- * epilogues) instead of separate norm kernels; 0 keeps the norm kernels.
- * Both round within the parity tolerance; each is bitwise reproducible. */
+ * PAE_OPT_FUSED_NORM (default 0, bf16 weights): 1 makes the QKV and gate/up
+ * projections apply the adaRMSNorm to their fp32 input inside the kernel
+ * (statistics from the residual projections' epilogues) instead of separate
+ * norm kernels, for batches of at most one 64-token tile.  Both round within
+ * the parity tolerance; each is bitwise reproducible. */
 enum {
   PAE_OPT_USE_GRAPH = 1,
   PAE_OPT_WAIT_LIMIT_US = 2,

@@ -96,6 +96,8 @@ def _fused_vs_separate(cfg, lengths=None):
         grid = wl.uniform_grid(cfg.steps)
         ex.precompute_tables(grid)
         noise = wl.make_noise(cfg)
+        assert ex.query(fm.PAE_Q_FUSED_NORM, cfg.batch) == 0  # off by default
+        ex.set_option(fm.PAE_OPT_FUSED_NORM, 1)
         assert ex.query(fm.PAE_Q_FUSED_NORM, cfg.batch) == 1
         fused = run_gpu(ex, noise)
         np.testing.assert_array_equal(run_gpu(ex, noise), fused)  # bitwise reproducible
