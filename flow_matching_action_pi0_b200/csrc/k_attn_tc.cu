@@ -35,7 +35,10 @@ constexpr int QROWS = 128;      // query rows per CTA
 constexpr long long kDrainNs = 4000000000LL;
 
 struct AttnSmem {
-  uint32_t q_off, k_off[2], v_off[2], p_off, bar_off, ml_off, total;
+  uint32_t q_off, k0_off, v0_off, slot, p_off, bar_off, ml_off, total;
+  // ring slot st of K / V (arithmetic, so no local-memory array is indexed)
+  __host__ __device__ uint32_t k_off(int st) const { return k0_off + (uint32_t)st * slot; }
+  __host__ __device__ uint32_t v_off(int st) const { return v0_off + (uint32_t)st * slot; }
 };
 
 __host__ __device__ inline AttnSmem attn_layout(int d) {
@@ -43,11 +46,10 @@ __host__ __device__ inline AttnSmem attn_layout(int d) {
   const uint32_t qbytes = QROWS * d * 2;   // d/64 boxes of [128][64]
   const uint32_t kvbytes = CK * d * 2;     // d/64 boxes of [64][64]
   L.q_off = 0;
-  L.k_off[0] = qbytes;
-  L.v_off[0] = L.k_off[0] + kvbytes;
-  L.k_off[1] = L.v_off[0] + kvbytes;
-  L.v_off[1] = L.k_off[1] + kvbytes;
-  L.p_off = L.v_off[1] + kvbytes;          // [128][64] bf16
+  L.k0_off = qbytes;
+  L.v0_off = qbytes + kvbytes;
+  L.slot = 2 * kvbytes;                    // [K0 | V0 | K1 | V1]
+  L.p_off = qbytes + 4 * kvbytes;          // [128][64] bf16
   L.bar_off = L.p_off + QROWS * CK * 2;
   L.ml_off = L.bar_off + 256;
   L.total = L.ml_off + QROWS * 12 + 1024;
@@ -140,20 +142,47 @@ __global__ void __launch_bounds__(256, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_launch_dependents();  // after the TMEM is held (see the projection kernel)
-  pdl_wait();               // q, k, v come from the previous kernel
+  // q and the action keys come from the previous kernel; the prefix keys were
+  // written by pae_set_prefix before the loop, so the producers fetch the
+  // chunks that lie wholly inside the prefix before waiting (below).
+  if (warp != 4 && warp != 6) pdl_wait();
+  const int n_prefix = a.lens[b];
   const uint32_t t_s[2] = {tmem, tmem + CK};
   const uint32_t t_o = tmem + 2 * CK;
 
   // ------------------------------------------------------------ producers
   // Warp 4 streams Q once and the K chunks, warp 6 the V chunks: a K slot is
   // refilled as soon as S of its chunk is done, ahead of the PV that frees V.
+  // chunks 0 and 1 (the two ring slots) if they end inside the prefix
+  const int npre = nch < 2 ? (start + CK <= n_prefix ? nch : 0)
+                            : (start + 2 * CK <= n_prefix ? 2 : (start + CK <= n_prefix ? 1 : 0));
+  if (warp == 4) {
+    if (lane == 0)
+      for (int c = 0; c < npre; ++c) {
+        mbar_arrive_expect_tx(&k_full[c], CK * d * 2);
+        for (int x = 0; x < nbox; ++x)
+          tma_load_2d(smem + L.k_off(c) + x * CK * 128, &tmK, x * 64, slot_row0 + start + c * CK, &k_full[c]);
+      }
+    __syncwarp();
+    pdl_wait();
+  }
+  if (warp == 6) {
+    if (lane == 0)
+      for (int c = 0; c < npre; ++c) {
+        mbar_arrive_expect_tx(&v_full[c], CK * d * 2);
+        for (int x = 0; x < nbox; ++x)
+          tma_load_2d(smem + L.v_off(c) + x * CK * 128, &tmV, x * 64, slot_row0 + start + c * CK, &v_full[c]);
+      }
+    __syncwarp();
+    pdl_wait();
+  }
   if (warp == 4 && lane == 0 && nch > 0) {
     const uint32_t kvbytes = CK * d * 2;
     mbar_arrive_expect_tx(q_full, QROWS * d * 2);
     const int qrow0 = bg * GH + qt * QROWS;
     for (int x = 0; x < nbox; ++x) tma_load_2d(smem + L.q_off + x * QROWS * 128, &tmQ, x * 64, qrow0, q_full);
-    int issued = 0;
-    for (int c = 0; c < nch; ++c) {
+    int issued = npre;
+    for (int c = npre; c < nch; ++c) {
       const int st = c & 1;
       if (c >= 2 && !mbar_wait(&k_empty[st], ((c >> 1) & 1) ^ 1, a.err.wait_ns)) {
         s_flag[0] = 1;
@@ -162,7 +191,7 @@ __global__ void __launch_bounds__(256, 1)
       }
       const int krow = slot_row0 + start + c * CK;
       mbar_arrive_expect_tx(&k_full[st], kvbytes);
-      for (int x = 0; x < nbox; ++x) tma_load_2d(smem + L.k_off[st] + x * CK * 128, &tmK, x * 64, krow, &k_full[st]);
+      for (int x = 0; x < nbox; ++x) tma_load_2d(smem + L.k_off(st) + x * CK * 128, &tmK, x * 64, krow, &k_full[st]);
       issued = c + 1;
     }
     if (!mbar_wait(q_full, 0, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
@@ -171,8 +200,8 @@ __global__ void __launch_bounds__(256, 1)
   }
   if (warp == 6 && lane == 0 && nch > 0) {
     const uint32_t kvbytes = CK * d * 2;
-    int issued = 0;
-    for (int c = 0; c < nch; ++c) {
+    int issued = npre;
+    for (int c = npre; c < nch; ++c) {
       const int st = c & 1;
       if (c >= 2 && !mbar_wait(&v_empty[st], ((c >> 1) & 1) ^ 1, a.err.wait_ns)) {
         s_flag[0] = 1;
@@ -181,7 +210,7 @@ __global__ void __launch_bounds__(256, 1)
       }
       const int krow = slot_row0 + start + c * CK;
       mbar_arrive_expect_tx(&v_full[st], kvbytes);
-      for (int x = 0; x < nbox; ++x) tma_load_2d(smem + L.v_off[st] + x * CK * 128, &tmV, x * 64, krow, &v_full[st]);
+      for (int x = 0; x < nbox; ++x) tma_load_2d(smem + L.v_off(st) + x * CK * 128, &tmV, x * 64, krow, &v_full[st]);
       issued = c + 1;
     }
     for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c)
@@ -199,7 +228,7 @@ __global__ void __launch_bounds__(256, 1)
       const int st = c & 1;
       if (!mbar_wait(&k_full[st], (c >> 1) & 1, a.err.wait_ns)) return false;
       tc_fence_after();
-      const uint32_t kb = smem_u32(smem + L.k_off[st]);
+      const uint32_t kb = smem_u32(smem + L.k_off(st));
       for (int k16 = 0; k16 < d / 16; ++k16) {
         const int x = k16 >> 2, w = (k16 & 3) * 32;
         const uint64_t ad = sw128_desc(q_base + x * QROWS * 128 + w, 16, 1024);
@@ -219,7 +248,7 @@ __global__ void __launch_bounds__(256, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t vb = smem_u32(smem + L.v_off[st]);
+      const uint32_t vb = smem_u32(smem + L.v_off(st));
       for (int k16 = 0; k16 < CK / 16; ++k16) {
         const uint64_t ad = sw128_desc(p_base + k16 * 32, 16, 1024);
         const uint64_t bd = sw128_desc(vb + k16 * 16 * 128, CK * 128, 1024);
@@ -310,7 +339,7 @@ __global__ void __launch_bounds__(256, 1)
       // zero the V rows past the valid keys once their load has landed.
       const bool w3 = mbar_wait(&v_full[st], (c >> 1) & 1, kDrainNs);
       if (w3) {
-        uint8_t* vbase = smem + L.v_off[st];
+        uint8_t* vbase = smem + L.v_off(st);
         const int rows = CK - vc;
         for (int i = r; i < rows * nbox * 8; i += 128) {
           const int rr = vc + i / (nbox * 8), rem = i % (nbox * 8), x = rem / 8, ch = rem % 8;
