@@ -35,7 +35,8 @@ constexpr int QROWS = 128;      // query rows per CTA
 constexpr long long kDrainNs = 4000000000LL;
 
 struct AttnSmem {
-  uint32_t q_off, k0_off, v0_off, slot, p_off, bar_off, ml_off, total;
+  uint32_t q_off, k0_off, v0_off, slot, p0_off, bar_off, ml_off, total;
+  __host__ __device__ uint32_t p_off(int j) const { return p0_off + (uint32_t)j * (QROWS * CK * 2); }
   // ring slot st of K / V (arithmetic, so no local-memory array is indexed)
   __host__ __device__ uint32_t k_off(int st) const { return k0_off + (uint32_t)st * slot; }
   __host__ __device__ uint32_t v_off(int st) const { return v0_off + (uint32_t)st * slot; }
@@ -49,8 +50,8 @@ __host__ __device__ inline AttnSmem attn_layout(int d) {
   L.k0_off = qbytes;
   L.v0_off = qbytes + kvbytes;
   L.slot = 2 * kvbytes;                    // [K0 | V0 | K1 | V1]
-  L.p_off = qbytes + 4 * kvbytes;          // [128][64] bf16
-  L.bar_off = L.p_off + QROWS * CK * 2;
+  L.p0_off = qbytes + 4 * kvbytes;         // two [128][64] bf16 P buffers
+  L.bar_off = L.p0_off + 2 * QROWS * CK * 2;
   L.ml_off = L.bar_off + 256;
   L.total = L.ml_off + QROWS * 12 + 1024;
   return L;
@@ -103,11 +104,11 @@ __global__ void __launch_bounds__(256, 1)
   uint64_t* v_full = bars + 3;   // [2]
   uint64_t* k_empty = bars + 5;  // [2] K slot free once S of its chunk is done
   uint64_t* s_full = bars + 7;   // [2]
-  uint64_t* p_full = bars + 9;
-  uint64_t* o_done = bars + 10;
-  uint64_t* drain = bars + 11;
-  uint64_t* v_empty = bars + 12;  // [2] V slot free once PV of its chunk is done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* p_full = bars + 9;    // [2] P buffer j written (chunks j, j + 2, ...)
+  uint64_t* o_done = bars + 11;   // [2] PV of the chunks in P buffer j done
+  uint64_t* drain = bars + 13;
+  uint64_t* v_empty = bars + 14;  // [2] V slot free once PV of its chunk is done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);  // [0] abort
   float* s_ml = reinterpret_cast<float*>(smem + L.ml_off);                // [128][2] row max, row sum
   int* s_ok = reinterpret_cast<int*>(smem + L.ml_off + QROWS * 8);        // [128]
@@ -125,7 +126,7 @@ __global__ void __launch_bounds__(256, 1)
   const float scale_log2 = rsqrtf((float)d) * 1.4426950408889634f;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 14; ++i) mbar_init(&bars[i], i == 9 ? 128 : 1);
+    for (int i = 0; i < 16; ++i) mbar_init(&bars[i], (i == 9 || i == 10) ? 128 : 1);
     s_flag[0] = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -222,7 +223,7 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t idesc_s = idesc_bf16(QROWS, CK);
     const uint32_t idesc_o = idesc_bf16(QROWS, d, 0, 1);
     const uint32_t q_base = smem_u32(smem + L.q_off);
-    const uint32_t p_base = smem_u32(smem + L.p_off);
+    const uint32_t p_base = smem_u32(smem + L.p0_off);
     bool good = mbar_wait(q_full, 0, a.err.wait_ns);
     auto issue_s = [&](int c) -> bool {
       const int st = c & 1;
@@ -243,18 +244,19 @@ __global__ void __launch_bounds__(256, 1)
     if (good && nch > 1) good = issue_s(1);
     for (int c = 0; good && c < nch; ++c) {
       const int st = c & 1;
-      if (!mbar_wait(p_full, c & 1, a.err.wait_ns) || !mbar_wait(&v_full[st], (c >> 1) & 1, a.err.wait_ns)) {
+      if (!mbar_wait(&p_full[st], (c >> 1) & 1, a.err.wait_ns) ||
+          !mbar_wait(&v_full[st], (c >> 1) & 1, a.err.wait_ns)) {
         good = false;
         break;
       }
       tc_fence_after();
       const uint32_t vb = smem_u32(smem + L.v_off(st));
       for (int k16 = 0; k16 < CK / 16; ++k16) {
-        const uint64_t ad = sw128_desc(p_base + k16 * 32, 16, 1024);
+        const uint64_t ad = sw128_desc(p_base + st * (QROWS * CK * 2) + k16 * 32, 16, 1024);
         const uint64_t bd = sw128_desc(vb + k16 * 16 * 128, CK * 128, 1024);
         umma_bf16(t_o, ad, bd, idesc_o, (c > 0 || k16 > 0) ? 1u : 0u);
       }
-      umma_commit(o_done);
+      umma_commit(&o_done[st]);
       umma_commit(&v_empty[st]);
       if (c + 2 < nch) good = issue_s(c + 2);
     }
@@ -274,7 +276,6 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
   float m_run = -INFINITY, l_run = 0.f;
   bool ok = true;
-  const uint32_t p_row = smem_u32(smem + L.p_off) + r * 128;
   for (int c = 0; c < nch; ++c) {
     const int st = c & 1;
     const bool w1 = mbar_wait(&s_full[st], (c >> 1) & 1, a.err.wait_ns);
@@ -307,15 +308,23 @@ __global__ void __launch_bounds__(256, 1)
     }
     l_run = l_run * alpha + psum;
     m_run = mx;
-    if (c > 0) {
-      // PV of the previous chunk must be done before O is rescaled and P reused.
-      const bool w2 = mbar_wait(o_done, (c - 1) & 1, a.err.wait_ns);
+    // P is double-buffered: buffer st is free once PV of chunk c - 2 is done.
+    if (c >= 2) {
+      const bool w2 = mbar_wait(&o_done[st], ((c - 2) >> 1) & 1, a.err.wait_ns);
+      if (!__all_sync(0xffffffffu, w2)) {
+        ok = false;
+        break;
+      }
+    }
+    if (c > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
+      // O may be rescaled only once PV of the previous chunk has landed in it.
+      const bool w2 = mbar_wait(&o_done[st ^ 1], ((c - 1) >> 1) & 1, a.err.wait_ns);
       if (!__all_sync(0xffffffffu, w2)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      if (__any_sync(0xffffffffu, alpha < 1.f)) {
+      {
         for (int j = 0; j < 256 && j < d; j += 16) {
           float ov[16];
           tmem_ld16(t_o + lane_off + j, ov);
@@ -328,6 +337,7 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
     // P row: 64 bf16 = 8 chunks of 16 bytes, chunk index XOR (row % 8)
+    const uint32_t p_row = smem_u32(smem + L.p_off(st)) + r * 128;
 #pragma unroll
     for (int ch = 0; ch < 8; ++ch) {
       const uint32_t addr = p_row + (((uint32_t)ch ^ (uint32_t)(r & 7)) << 4);
@@ -351,10 +361,11 @@ __global__ void __launch_bounds__(256, 1)
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    mbar_arrive(p_full);
+    mbar_arrive(&p_full[st]);
   }
   if (!ok) set_error(a.err, DEV_TIMEOUT);
-  if (nch > 0 && ok) ok = mbar_wait(o_done, (nch - 1) & 1, kDrainNs);
+  // PVs complete in issue order: the last chunk's commit covers them all
+  if (nch > 0 && ok) ok = mbar_wait(&o_done[(nch - 1) & 1], ((nch - 1) >> 1) & 1, kDrainNs);
   ok = named_and(1, 128, ok) && s_flag[0] == 0;  // CTA-uniform among the 128 softmax threads
   tc_fence_after();
 
