@@ -55,7 +55,9 @@ struct Plan {
   bool persist = false;  // eligible for the persistent kernel
   PersistArgs pa{};
   bool fuse_norm = false;  // QKV / gate-up normalise their fp32 operand in-kernel
-  CUtensorMap tmY{}, tmO{}, tmU{}, tmH{};
+  // token-operand maps; a map's box height is the token tile of the projection
+  // that reads it (QKV and gate/up may tile the same y differently)
+  CUtensorMap tmY{}, tmYg{}, tmO{}, tmU{}, tmH{}, tmHg{};
   cudaGraphExec_t graph = nullptr;
   int graph_K = 0;
   long long graph_kernels = 0;
@@ -455,9 +457,11 @@ pae_status build_plan(pae_ctx* ctx, int B, Plan* P) {
   const uint64_t Mmax = (uint64_t)s.Bmax * s.H;
   pae_status st;
   if ((st = make_map(ctx, &P->tmY, ctx->y, s.D, Mmax, 64, P->qkv.tn)) != PAE_OK) return st;
+  if ((st = make_map(ctx, &P->tmYg, ctx->y, s.D, Mmax, 64, P->gu.tn)) != PAE_OK) return st;
   if ((st = make_map(ctx, &P->tmO, ctx->o, s.attn_dim, Mmax, 64, P->o.tn)) != PAE_OK) return st;
   if ((st = make_map(ctx, &P->tmU, ctx->u, s.F, Mmax, 64, P->down.tn)) != PAE_OK) return st;
   if (P->fuse_norm && (st = make_map_f32(ctx, &P->tmH, ctx->h, s.D, Mmax, 64, P->qkv.tn)) != PAE_OK) return st;
+  if (P->fuse_norm && (st = make_map_f32(ctx, &P->tmHg, ctx->h, s.D, Mmax, 64, P->gu.tn)) != PAE_OK) return st;
   return PAE_OK;
 }
 
@@ -548,14 +552,14 @@ void run_gemm(pae_ctx* ctx, const Plan& P, int which, int layer, const EpiArgs& 
             a.w_row0 = layer * s.qkv_rows; a.scales = (const bf16*)ctx->sc_qkv; break;
     case 1: tw = w4 ? &ctx->tmQo : &ctx->tmWo; tx = &P.tmO; p = &P.o; a.N = s.D; a.K = s.attn_dim;
             a.w_row0 = layer * s.D; a.scales = (const bf16*)ctx->sc_o; break;
-    case 2: tw = w4 ? &ctx->tmQgu : &ctx->tmWgu; tx = &P.tmY; p = &P.gu; a.N = s.F; a.K = s.D;
+    case 2: tw = w4 ? &ctx->tmQgu : &ctx->tmWgu; tx = &P.tmYg; p = &P.gu; a.N = s.F; a.K = s.D;
             a.w_row0 = layer * 2 * s.F; na = 2; a.scales = (const bf16*)ctx->sc_gu; break;
     default: tw = w4 ? &ctx->tmQdown : &ctx->tmWdown; tx = &P.tmU; p = &P.down; a.N = s.D; a.K = s.F;
              a.w_row0 = layer * s.D; a.scales = (const bf16*)ctx->sc_down; break;
   }
   if (!w4) a.scales = nullptr;
   if (norm.scale) {
-    tx = &P.tmH;
+    tx = which == 2 ? &P.tmHg : &P.tmH;
     a.ss_in = ctx->ss_buf;
     a.ss_ld = ctx->ss_ld;
     a.nslots = norm.nslots;
