@@ -256,7 +256,10 @@ pae_status make_map_u8(pae_ctx* ctx, CUtensorMap* m, const void* base, uint64_t 
 // small token tiles keep shared memory under half an SM so that two CTAs (or a
 // CTA and its successor under PDL) fit per SM.
 // Ring depth and receive-buffer placement for a token tile / split choice
-// within a shared-memory budget (false if fewer than two stages fit).
+// within a shared-memory budget (false if fewer than two stages fit).  A
+// separate split-K receive buffer saves a cluster barrier, but it is taken
+// only when it costs no ring depth: on long K loops a shallow ring starves the
+// tensor cores (measured on the batch-32 down projection).
 bool fit_ring(TcPlan& p, int na, int nkb, bool w4, bool norm, uint32_t budget) {
   const uint32_t stage = (uint32_t)na * 16384u + (uint32_t)p.tn * 128u + (w4 ? (uint32_t)na * 4096u : 0u) +
                          (norm ? (uint32_t)p.tn * 128u : 0u);
@@ -267,7 +270,7 @@ bool fit_ring(TcPlan& p, int na, int nkb, bool w4, bool norm, uint32_t budget) {
   p.recv_alias = 0;
   if (p.splits > 1) {
     const int st_sep = std::min(st, (int)((budget - std::min(budget, recv)) / stage));
-    if (st_sep >= 2) {
+    if (st_sep >= st) {
       st = st_sep;
     } else {
       p.recv_alias = 1;
@@ -278,41 +281,35 @@ bool fit_ring(TcPlan& p, int na, int nkb, bool w4, bool norm, uint32_t budget) {
   return true;
 }
 
-// Large batches (more than one 256-token tile): choose the token tile, split-K
-// and residency (one or two CTAs per SM) with the smallest modelled time:
-// per-SM rounds x the larger of (the FLOPs a round puts on one SM at the
-// measured sustained tensor rate, 1370 TFLOP/s / 148 SMs) and (the operand
-// bytes it pulls into one SM's shared memory at ~110 GB/s), plus fixed and
-// split-K costs.  This keeps the last wave from running half empty (224 CTAs
-// on 148 SMs, say) without shrinking tiles until the operands dominate.
+// Large batches (more than one 256-token tile): one CTA per SM (token tiles of
+// 128..256 need most of the shared memory), so choose the token-tile count
+// whose CTAs (output tiles x split-K, split-K as long as the tiles fit one
+// wave) fill whole waves of 148 SMs best; ties go to the larger tile.  At
+// M = 1600 this picks 240 for QKV (140 CTAs), 192 with split-K 2 for O and
+// down (144) and 192 for gate/up (288 = two full waves), which measured
+// 23.4 ms per batch-32 call against 24.7 ms for a fixed 240-token tile.
 TcPlan plan_gemm_large(int M, int nfeat, int K, int na, int max_splits, bool w4, bool norm) {
   const int nt = (nfeat + 127) / 128, nkb = K / 64;
-  const double per_sm = 1370.4e12 / 148.0;
   TcPlan best{};
-  double best_t = 1e30;
-  for (int tt = (M + 255) / 256; tt <= (M + 63) / 64; ++tt) {
-    const int tn = std::max(16, (((M + tt - 1) / tt + 15) / 16) * 16);
-    if (tn > 256 || (M + tn - 1) / tn != tt) continue;
-    for (int sp = 1; sp <= std::min(8, max_splits); sp *= 2) {
-      if (nkb % sp) continue;
-      for (int cps = 2; cps >= 1; --cps) {
-        TcPlan p{};
-        p.tn = tn;
-        p.tok_tiles = tt;
-        p.splits = sp;
-        if (!fit_ring(p, na, nkb, w4, norm, cps == 2 ? 110u * 1024u : 200u * 1024u)) continue;
-        if (tc_gemm_smem_bytes(na, p, w4, norm) > (cps == 2 ? 113u * 1024u : 227u * 1024u)) continue;
-        const long long ctas = (long long)nt * tt * sp;
-        const long long rounds = (ctas + 148LL * cps - 1) / (148LL * cps);
-        const double flops = 2.0 * 128.0 * na * tn * (double)(K / sp);
-        const double bytes = ((double)na * 16384.0 + tn * 128.0) * (double)(nkb / sp);
-        double t = (double)rounds * cps * std::max(flops / per_sm, bytes / 110e9) + 3e-6;
-        if (sp > 1) t += 1.5e-6 + (double)na * tn * 512.0 / 1e11;  // partial push through DSMEM
-        if (t < best_t) {
-          best_t = t;
-          best = p;
-        }
-      }
+  double best_eff = -1.0;
+  for (int tt = (M + 255) / 256; tt <= (M + 127) / 128; ++tt) {
+    const int tn = (((M + tt - 1) / tt + 15) / 16) * 16;
+    if (tn > 256 || tn < 128 || (M + tn - 1) / tn != tt) continue;
+    const int base = nt * tt;
+    int sp = 1;
+    for (int c = 2; c <= std::min(8, max_splits); c *= 2)
+      if (nkb % c == 0 && base * c <= 148) sp = c;
+    TcPlan p{};
+    p.tn = tn;
+    p.tok_tiles = tt;
+    p.splits = sp;
+    if (!fit_ring(p, na, nkb, w4, norm, 200u * 1024u)) continue;
+    const int ctas = base * sp;
+    const int waves = (ctas + 147) / 148;
+    const double eff = (double)ctas / (148.0 * waves);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = p;
     }
   }
   return best;
