@@ -63,8 +63,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return lo | (hi << 16);
 }
 
-// AND-reduction over the first `n` threads (named barrier `id`).
+// AND-reduction over the threads of named barrier `id` (`n` of them).  Lanes
+// may leave a bounded wait at different times: the warp reconverges before the
+// warp-aligned barrier instruction.
 __device__ __forceinline__ bool named_and(int id, int n, bool v) {
+  __syncwarp();
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
@@ -77,6 +80,7 @@ __device__ __forceinline__ bool named_and(int id, int n, bool v) {
   return r != 0;
 }
 __device__ __forceinline__ void named_sync(int id, int n) {
+  __syncwarp();
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
@@ -90,7 +94,7 @@ __host__ __device__ inline uint32_t attn_tmem_cols(int d) {
   return c;
 }
 
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const Shape s, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -126,7 +130,7 @@ __global__ void __launch_bounds__(256, 1)
   const float scale_log2 = rsqrtf((float)d) * 1.4426950408889634f;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 16; ++i) mbar_init(&bars[i], (i == 9 || i == 10) ? 128 : 1);
+    for (int i = 0; i < 16; ++i) mbar_init(&bars[i], (i == 9 || i == 10) ? 256 : 1);
     s_flag[0] = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -270,31 +274,45 @@ __global__ void __launch_bounds__(256, 1)
   }
   __syncwarp();
 
-  // ------------------------------------------------------------ softmax (warps 0-3)
-  if (warp < 4) {
-  const int r = warp * 32 + lane;  // query row within the tile (TMEM lane)
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  // ------------------------------------------------------------ softmax
+  // Warps 0-3 and 8-11: thread = (query row r = TMEM lane, column half h);
+  // half h owns key columns [32h, 32h + 32) of each chunk and output columns
+  // [h d/2, (h+1) d/2).  The two halves of a row agree on the running
+  // reference maximum through shared memory (s_ml as [2][128] exchange
+  // slots, two barriers per chunk); each keeps its own partial row sum, added
+  // in a fixed order at the end.  Decisions that guard a named barrier are
+  // taken CTA-uniformly over the 256 softmax threads (bar.red.and).
+  const bool smx = warp < 4 || warp >= 8;
+  if (smx) {
+  const int h = warp >= 8 ? 1 : 0;
+  const int r = (warp & 3) * 32 + lane;  // query row within the tile (TMEM lane)
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  const int oc0 = h * (d / 2), oc1 = oc0 + d / 2;  // this half's output columns
   float m_run = -INFINITY, l_run = 0.f;
   bool ok = true;
   for (int c = 0; c < nch; ++c) {
     const int st = c & 1;
     const bool w1 = mbar_wait(&s_full[st], (c >> 1) & 1, a.err.wait_ns);
-    if (!__all_sync(0xffffffffu, w1) || s_flag[0]) {  // warp-uniform: the TMEM loads are collective
+    if (!named_and(1, 256, w1 && s_flag[0] == 0)) {  // uniform: named barriers follow
       ok = false;
       break;
     }
     tc_fence_after();
-    float sv[CK];
-#pragma unroll
-    for (int j = 0; j < CK; j += 16) tmem_ld16(t_s[st] + lane_off + j, sv + j);
+    float sv[CK / 2];
+    tmem_ld16(t_s[st] + lane_off + h * 32, sv);
+    tmem_ld16(t_s[st] + lane_off + h * 32 + 16, sv + 16);
     tmem_ld_wait();
     const int vc = min(CK, end - (start + c * CK));
     float cmax = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < CK; ++j) {
-      sv[j] = j < vc ? sv[j] * scale_log2 : -INFINITY;
+    for (int j = 0; j < CK / 2; ++j) {
+      sv[j] = j + h * 32 < vc ? sv[j] * scale_log2 : -INFINITY;
       cmax = fmaxf(cmax, sv[j]);
     }
+    s_ml[h * QROWS + r] = cmax;
+    named_sync(1, 256);
+    cmax = fmaxf(s_ml[r], s_ml[QROWS + r]);  // same operands, same order, in both halves
+    named_sync(1, 256);                      // both read before the next chunk writes
     // Lazy rescaling: the reference maximum moves only when the row maximum
     // grows by more than 8 (a factor 256), so O is rescaled in TMEM rarely.
     // Probabilities then lie in [0, 256]; the final O / l is the same.
@@ -302,47 +320,40 @@ __global__ void __launch_bounds__(256, 1)
     const float alpha = exp2f(m_run - mx);  // 1 when unchanged; 0 on the first chunk
     float psum = 0.f;
 #pragma unroll
-    for (int j = 0; j < CK; ++j) {
+    for (int j = 0; j < CK / 2; ++j) {
       sv[j] = exp2f(sv[j] - mx);
       psum += sv[j];
     }
     l_run = l_run * alpha + psum;
     m_run = mx;
     // P is double-buffered: buffer st is free once PV of chunk c - 2 is done.
-    if (c >= 2) {
-      const bool w2 = mbar_wait(&o_done[st], ((c - 2) >> 1) & 1, a.err.wait_ns);
-      if (!__all_sync(0xffffffffu, w2)) {
-        ok = false;
-        break;
-      }
-    }
-    if (c > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
+    bool good = true;
+    if (c >= 2) good = mbar_wait(&o_done[st], ((c - 2) >> 1) & 1, a.err.wait_ns);
+    if (good && c > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
       // O may be rescaled only once PV of the previous chunk has landed in it.
-      const bool w2 = mbar_wait(&o_done[st ^ 1], ((c - 1) >> 1) & 1, a.err.wait_ns);
-      if (!__all_sync(0xffffffffu, w2)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      {
-        for (int j = 0; j < 256 && j < d; j += 16) {
+      good = __all_sync(0xffffffffu, mbar_wait(&o_done[st ^ 1], ((c - 1) >> 1) & 1, a.err.wait_ns));
+      if (good) {
+        tc_fence_after();
+        for (int jj = oc0; jj < oc1; jj += 16) {
           float ov[16];
-          tmem_ld16(t_o + lane_off + j, ov);
+          tmem_ld16(t_o + lane_off + jj, ov);
           tmem_ld_wait();
 #pragma unroll
           for (int t = 0; t < 16; ++t) ov[t] *= alpha;
-          tmem_st16(t_o + lane_off + j, ov);
+          tmem_st16(t_o + lane_off + jj, ov);
         }
         tmem_st_wait();
       }
     }
-    // P row: 64 bf16 = 8 chunks of 16 bytes, chunk index XOR (row % 8)
+    if (!good) s_flag[0] = 1;  // every thread stops at the next uniform check
+    // P row: 64 bf16 = 8 chunks of 16 bytes, chunk index XOR (row % 8); half h
+    // writes chunks 4h .. 4h + 3
     const uint32_t p_row = smem_u32(smem + L.p_off(st)) + r * 128;
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-      const uint32_t addr = p_row + (((uint32_t)ch ^ (uint32_t)(r & 7)) << 4);
-      st_shared_v4(addr, pack_bf16x2(sv[ch * 8 + 0], sv[ch * 8 + 1]), pack_bf16x2(sv[ch * 8 + 2], sv[ch * 8 + 3]),
-                   pack_bf16x2(sv[ch * 8 + 4], sv[ch * 8 + 5]), pack_bf16x2(sv[ch * 8 + 6], sv[ch * 8 + 7]));
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t addr = p_row + (((uint32_t)(h * 4 + q) ^ (uint32_t)(r & 7)) << 4);
+      st_shared_v4(addr, pack_bf16x2(sv[q * 8 + 0], sv[q * 8 + 1]), pack_bf16x2(sv[q * 8 + 2], sv[q * 8 + 3]),
+                   pack_bf16x2(sv[q * 8 + 4], sv[q * 8 + 5]), pack_bf16x2(sv[q * 8 + 6], sv[q * 8 + 7]));
     }
     if (vc < CK) {
       // Masked keys have P = 0, but 0 * (NaN or Inf) in V would still poison O:
@@ -351,23 +362,28 @@ __global__ void __launch_bounds__(256, 1)
       if (w3) {
         uint8_t* vbase = smem + L.v_off(st);
         const int rows = CK - vc;
-        for (int i = r; i < rows * nbox * 8; i += 128) {
+        for (int i = h * QROWS + r; i < rows * nbox * 8; i += 2 * QROWS) {
           const int rr = vc + i / (nbox * 8), rem = i % (nbox * 8), x = rem / 8, ch = rem % 8;
           *reinterpret_cast<uint4*>(vbase + x * CK * 128 + rr * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
         }
       } else {
-        set_error(a.err, DEV_TIMEOUT);
+        s_flag[0] = 1;
       }
     }
     fence_proxy_async_smem();
     tc_fence_before();
     mbar_arrive(&p_full[st]);
   }
-  if (!ok) set_error(a.err, DEV_TIMEOUT);
+  if (!ok || s_flag[0]) set_error(a.err, DEV_TIMEOUT);
   // PVs complete in issue order: the last chunk's commit covers them all
   if (nch > 0 && ok) ok = mbar_wait(&o_done[(nch - 1) & 1], ((nch - 1) >> 1) & 1, kDrainNs);
-  ok = named_and(1, 128, ok) && s_flag[0] == 0;  // CTA-uniform among the 128 softmax threads
+  ok = named_and(1, 256, ok) && s_flag[0] == 0;  // CTA-uniform among the 256 softmax threads
   tc_fence_after();
+  // row sum = half 0 + half 1 (the exchange slots are free: both passed the barrier)
+  s_ml[h * QROWS + r] = l_run;
+  named_sync(1, 256);
+  const float l_tot = s_ml[r] + s_ml[QROWS + r];
+  named_sync(1, 256);
 
   // ------------------------------------------------------------ output (single split)
   const int nsplit = gridDim.y;
@@ -376,28 +392,28 @@ __global__ void __launch_bounds__(256, 1)
     const bool row_valid = rq < GH;
     const int hl = rq / s.H, ti = rq - hl * s.H;
     bf16* orow = reinterpret_cast<bf16*>(a.o) + (size_t)(b * s.H + ti) * s.attn_dim + (g * s.G + hl) * d;
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+    const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
     if (ok) {
-      for (int j = 0; j < d; j += 16) {
+      for (int jj = oc0; jj < oc1; jj += 16) {
         float ov[16];
-        tmem_ld16(t_o + lane_off + j, ov);
+        tmem_ld16(t_o + lane_off + jj, ov);
         tmem_ld_wait();
         if (row_valid && nch > 0) {
           uint32_t pk[8];
 #pragma unroll
           for (int t = 0; t < 8; ++t) pk[t] = pack_bf16x2(ov[2 * t] * inv, ov[2 * t + 1] * inv);
-          uint4* dst = reinterpret_cast<uint4*>(orow + j);
+          uint4* dst = reinterpret_cast<uint4*>(orow + jj);
           dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       }
     }
-  } else {
+  } else if (h == 0) {
     s_ok[r] = ok ? 1 : 0;
     s_ml[2 * r] = m_run;
-    s_ml[2 * r + 1] = l_run;
+    s_ml[2 * r + 1] = l_tot;
   }
-  }  // warps 0-3
+  }  // softmax warps
 
   if (gridDim.y > 1) {
     // Split-KV merge inside the cluster of key splits.  Every CTA parks its
@@ -407,13 +423,14 @@ __global__ void __launch_bounds__(256, 1)
     __syncthreads();  // all MMAs and TMEM reads of this CTA are done
     const int ld = d + 4;
     float* red = reinterpret_cast<float*>(smem);
-    if (warp < 4) {
-      const int r = warp * 32 + lane;
-      const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    if (smx) {
+      const int h = warp >= 8 ? 1 : 0;
+      const int r = (warp & 3) * 32 + lane;
+      const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
       const bool has = s_ok[r] && nch > 0;
-      for (int j = 0; j < d; j += 16) {
+      for (int j = h * (d / 2); j < (h + 1) * (d / 2); j += 16) {
         float ov[16];
-        if (__all_sync(0xffffffffu, s_ok[warp * 32] != 0) && nch > 0) {
+        if (__all_sync(0xffffffffu, s_ok[(warp & 3) * 32] != 0) && nch > 0) {
           tmem_ld16(t_o + lane_off + j, ov);
           tmem_ld_wait();
         }
@@ -422,7 +439,7 @@ __global__ void __launch_bounds__(256, 1)
           *reinterpret_cast<float4*>(red + r * ld + j + t) =
               has ? make_float4(ov[t], ov[t + 1], ov[t + 2], ov[t + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      if (!has) {
+      if (!has && h == 0) {
         s_ml[2 * r] = -INFINITY;
         s_ml[2 * r + 1] = 0.f;
       }
@@ -489,7 +506,7 @@ cudaError_t attn_tc_init() {
 cudaError_t launch_attn_tc(const Shape& s, const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                            const AttnPlan& p, const AttnArgs& a, int B, bool pdl, cudaStream_t st) {
   dim3 grid(p.qtiles, p.splits, B * s.Hkv);
-  return launch_ex(k_attn_tc, grid, dim3(256), attn_tc_smem_bytes(s.d), st, p.splits, pdl, *tmQ, *tmK, *tmV, s,
+  return launch_ex(k_attn_tc, grid, dim3(384), attn_tc_smem_bytes(s.d), st, p.splits, pdl, *tmQ, *tmK, *tmV, s,
                    a);
 }
 
