@@ -168,11 +168,6 @@ __global__ void __launch_bounds__(384, 1)
         for (int x = 0; x < nbox; ++x)
           tma_load_2d(smem + L.k_off(c) + x * CK * 128, &tmK, x * 64, slot_row0 + start + c * CK, &k_full[c]);
       }
-    // V of the chunks after the prefetched ones: into L2 now, so that the V
-    // loads (gated by the PV of two chunks earlier) do not wait for HBM
-    if (lane == 0)
-      for (int c = npre; c < nch && c < npre + 2; ++c)
-        for (int x = 0; x < nbox; ++x) tma_prefetch_l2_2d(&tmV, x * 64, slot_row0 + start + c * CK);
     __syncwarp();
     pdl_wait();
   }
@@ -202,8 +197,6 @@ __global__ void __launch_bounds__(384, 1)
       const int krow = slot_row0 + start + c * CK;
       mbar_arrive_expect_tx(&k_full[st], kvbytes);
       for (int x = 0; x < nbox; ++x) tma_load_2d(smem + L.k_off(st) + x * CK * 128, &tmK, x * 64, krow, &k_full[st]);
-      if (c + 2 < nch)  // V two chunks ahead into L2
-        for (int x = 0; x < nbox; ++x) tma_prefetch_l2_2d(&tmV, x * 64, krow + 2 * CK);
       issued = c + 1;
     }
     if (!mbar_wait(q_full, 0, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
