@@ -235,6 +235,11 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_byte
   return d;
 }
 
+// The same descriptor moved `bytes` (a multiple of 16) further into shared
+// memory: the start address sits in the low 14 bits in 16-byte units, and
+// shared addresses stay below 256 KB, so the add never carries out of it.
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) { return desc + (uint64_t)(bytes >> 4); }
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
 // Bits: D format [4,6) = 1 (f32); A format [7,10) = 1 (bf16); B format
 // [10,13) = 1 (bf16); A major bit 15, B major bit 16 (0 = K-major,

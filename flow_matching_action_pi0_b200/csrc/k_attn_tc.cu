@@ -229,16 +229,18 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t q_base = smem_u32(smem + L.q_off);
     const uint32_t p_base = smem_u32(smem + L.p0_off);
     bool good = mbar_wait(q_full, 0, a.err.wait_ns);
+    // descriptors are built once per operand and stepped in 16-byte units
+    const uint64_t q_desc = sw128_desc(q_base, 16, 1024);
     auto issue_s = [&](int c) -> bool {
       const int st = c & 1;
       if (!mbar_wait(&k_full[st], (c >> 1) & 1, a.err.wait_ns)) return false;
       tc_fence_after();
-      const uint32_t kb = smem_u32(smem + L.k_off(st));
+      const uint64_t k_desc = sw128_desc(smem_u32(smem + L.k_off(st)), 16, 1024);
+#pragma unroll 4
       for (int k16 = 0; k16 < d / 16; ++k16) {
-        const int x = k16 >> 2, w = (k16 & 3) * 32;
-        const uint64_t ad = sw128_desc(q_base + x * QROWS * 128 + w, 16, 1024);
-        const uint64_t bd = sw128_desc(kb + x * CK * 128 + w, 16, 1024);
-        umma_bf16(t_s[st], ad, bd, idesc_s, k16 > 0 ? 1u : 0u);
+        const uint32_t x = (uint32_t)k16 >> 2, w = ((uint32_t)k16 & 3u) * 32u;
+        umma_bf16(t_s[st], desc_add(q_desc, x * QROWS * 128u + w), desc_add(k_desc, x * CK * 128u + w), idesc_s,
+                  k16 > 0 ? 1u : 0u);
       }
       umma_commit(&s_full[st]);
       umma_commit(&k_empty[st]);
@@ -254,12 +256,12 @@ __global__ void __launch_bounds__(384, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t vb = smem_u32(smem + L.v_off(st));
-      for (int k16 = 0; k16 < CK / 16; ++k16) {
-        const uint64_t ad = sw128_desc(p_base + st * (QROWS * CK * 2) + k16 * 32, 16, 1024);
-        const uint64_t bd = sw128_desc(vb + k16 * 16 * 128, CK * 128, 1024);
-        umma_bf16(t_o, ad, bd, idesc_o, (c > 0 || k16 > 0) ? 1u : 0u);
-      }
+      const uint64_t p_desc = sw128_desc(p_base + st * (QROWS * CK * 2), 16, 1024);
+      const uint64_t v_desc = sw128_desc(smem_u32(smem + L.v_off(st)), CK * 128, 1024);
+#pragma unroll
+      for (int k16 = 0; k16 < CK / 16; ++k16)
+        umma_bf16(t_o, desc_add(p_desc, k16 * 32u), desc_add(v_desc, k16 * 16u * 128u), idesc_o,
+                  (c > 0 || k16 > 0) ? 1u : 0u);
       umma_commit(&o_done[st]);
       umma_commit(&v_empty[st]);
       if (c + 2 < nch) good = issue_s(c + 2);

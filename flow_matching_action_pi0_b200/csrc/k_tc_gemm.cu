@@ -307,15 +307,14 @@ __global__ void __launch_bounds__(256, 2)
       }
       tc_fence_after();
       const uint32_t sa = smem_u32(smem + (size_t)st * L.stage_bytes);
-      const uint32_t sb = sa + L.a_bytes;
+      const uint64_t a_desc = sw128_desc(sa, 16, 1024);
+      const uint64_t b_desc = sw128_desc(sa + L.a_bytes, 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t bdesc = sw128_desc(sb + kk * 32, 16, 1024);
 #pragma unroll
-        for (int na = 0; na < NA; ++na) {
-          const uint64_t adesc = sw128_desc(sa + na * 16384 + kk * 32, 16, 1024);
-          umma_bf16(tmem + na * p.tn, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
-        }
+        for (int na = 0; na < NA; ++na)
+          umma_bf16(tmem + na * p.tn, desc_add(a_desc, na * 16384u + kk * 32u), desc_add(b_desc, kk * 32u), idesc,
+                    (kb | kk) != 0 ? 1u : 0u);
       }
       umma_commit(&empty[st]);  // stage reusable once these MMAs have read it
     }
