@@ -79,20 +79,6 @@ __device__ __forceinline__ bool named_and(int id, int n, bool v) {
       : "memory");
   return r != 0;
 }
-// OR-reduction over the threads of named barrier `id`.
-__device__ __forceinline__ bool named_or(int id, int n, bool v) {
-  __syncwarp();
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)v), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
-}
 __device__ __forceinline__ void named_sync(int id, int n) {
   __syncwarp();
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -102,11 +88,9 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-// TMEM: per S buffer two accumulation chains of CK columns (even and odd K
-// steps, so consecutive MMAs do not wait on each other), then O (d columns).
 __host__ __device__ inline uint32_t attn_tmem_cols(int d) {
   uint32_t c = 32;
-  while ((int)c < 4 * CK + d) c <<= 1;
+  while ((int)c < 2 * CK + d) c <<= 1;
   return c;
 }
 
@@ -168,8 +152,8 @@ __global__ void __launch_bounds__(384, 1)
   // chunks that lie wholly inside the prefix before waiting (below).
   if (warp != 4 && warp != 6) pdl_wait();
   const int n_prefix = a.lens[b];
-  const uint32_t t_s[2] = {tmem, tmem + 2 * CK};  // chain a at +0, chain b at +CK
-  const uint32_t t_o = tmem + 4 * CK;
+  const uint32_t t_s[2] = {tmem, tmem + CK};
+  const uint32_t t_o = tmem + 2 * CK;
 
   // ------------------------------------------------------------ producers
   // Warp 4 streams Q once and the K chunks, warp 6 the V chunks: a K slot is
@@ -255,8 +239,8 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll 4
       for (int k16 = 0; k16 < d / 16; ++k16) {
         const uint32_t x = (uint32_t)k16 >> 2, w = ((uint32_t)k16 & 3u) * 32u;
-        umma_bf16(t_s[st] + (k16 & 1) * CK, desc_add(q_desc, x * QROWS * 128u + w),
-                  desc_add(k_desc, x * CK * 128u + w), idesc_s, k16 >= 2 ? 1u : 0u);
+        umma_bf16(t_s[st], desc_add(q_desc, x * QROWS * 128u + w), desc_add(k_desc, x * CK * 128u + w), idesc_s,
+                  k16 > 0 ? 1u : 0u);
       }
       umma_commit(&s_full[st]);
       umma_commit(&k_empty[st]);
@@ -295,14 +279,11 @@ __global__ void __launch_bounds__(384, 1)
   // ------------------------------------------------------------ softmax
   // Warps 0-3 and 8-11: thread = (query row r = TMEM lane, column half h);
   // half h owns key columns [32h, 32h + 32) of each chunk and output columns
-  // [h d/2, (h+1) d/2).  S arrives as two partial accumulators (even / odd K
-  // steps), added here.  The two halves of a row keep the same running
-  // reference maximum: one OR-barrier per chunk asks whether any row's
-  // maximum grew past the reference by more than 8; only then do the halves
-  // exchange their maxima through shared memory (s_ml as [2][128]).  Each
-  // half keeps its own partial row sum, added in a fixed order at the end.
-  // A failed wait raises s_flag instead of leaving the loop, so every thread
-  // reaches every barrier; the remaining waits then return at once.
+  // [h d/2, (h+1) d/2).  The two halves of a row agree on the running
+  // reference maximum through shared memory (s_ml as [2][128] exchange
+  // slots, two barriers per chunk); each keeps its own partial row sum, added
+  // in a fixed order at the end.  Decisions that guard a named barrier are
+  // taken CTA-uniformly over the 256 softmax threads (bar.red.and).
   const bool smx = warp < 4 || warp >= 8;
   if (smx) {
   const int h = warp >= 8 ? 1 : 0;
@@ -311,41 +292,33 @@ __global__ void __launch_bounds__(384, 1)
   const int oc0 = h * (d / 2), oc1 = oc0 + d / 2;  // this half's output columns
   float m_run = -INFINITY, l_run = 0.f;
   bool ok = true;
-  auto wait_live = [&](uint64_t* bar, uint32_t parity, long long limit) -> bool {
-    if (s_flag[0]) return false;
-    if (mbar_wait(bar, parity, limit)) return true;
-    s_flag[0] = 1;
-    return false;
-  };
   for (int c = 0; c < nch; ++c) {
     const int st = c & 1;
-    wait_live(&s_full[st], (c >> 1) & 1, a.err.wait_ns);
-    __syncwarp();
+    const bool w1 = mbar_wait(&s_full[st], (c >> 1) & 1, a.err.wait_ns);
+    if (!named_and(1, 256, w1 && s_flag[0] == 0)) {  // uniform: named barriers follow
+      ok = false;
+      break;
+    }
     tc_fence_after();
-    float sv[CK / 2], sb[CK / 2];
+    float sv[CK / 2];
     tmem_ld16(t_s[st] + lane_off + h * 32, sv);
     tmem_ld16(t_s[st] + lane_off + h * 32 + 16, sv + 16);
-    tmem_ld16(t_s[st] + CK + lane_off + h * 32, sb);
-    tmem_ld16(t_s[st] + CK + lane_off + h * 32 + 16, sb + 16);
     tmem_ld_wait();
     const int vc = min(CK, end - (start + c * CK));
     float cmax = -INFINITY;
 #pragma unroll
     for (int j = 0; j < CK / 2; ++j) {
-      sv[j] = j + h * 32 < vc ? (sv[j] + sb[j]) * scale_log2 : -INFINITY;
+      sv[j] = j + h * 32 < vc ? sv[j] * scale_log2 : -INFINITY;
       cmax = fmaxf(cmax, sv[j]);
     }
+    s_ml[h * QROWS + r] = cmax;
+    named_sync(1, 256);
+    cmax = fmaxf(s_ml[r], s_ml[QROWS + r]);  // same operands, same order, in both halves
+    named_sync(1, 256);                      // both read before the next chunk writes
     // Lazy rescaling: the reference maximum moves only when the row maximum
     // grows by more than 8 (a factor 256), so O is rescaled in TMEM rarely.
     // Probabilities then lie in [0, 256]; the final O / l is the same.
-    float mx = m_run;
-    if (named_or(1, 256, cmax > m_run + 8.f)) {
-      s_ml[h * QROWS + r] = cmax;
-      named_sync(1, 256);
-      cmax = fmaxf(s_ml[r], s_ml[QROWS + r]);  // same operands, same order, in both halves
-      named_sync(1, 256);                      // both read before the exchange is reused
-      mx = cmax > m_run + 8.f ? cmax : m_run;
-    }
+    const float mx = cmax > m_run + 8.f ? cmax : m_run;
     const float alpha = exp2f(m_run - mx);  // 1 when unchanged; 0 on the first chunk
     float psum = 0.f;
 #pragma unroll
@@ -357,10 +330,10 @@ __global__ void __launch_bounds__(384, 1)
     m_run = mx;
     // P is double-buffered: buffer st is free once PV of chunk c - 2 is done.
     bool good = true;
-    if (c >= 2) good = wait_live(&o_done[st], ((c - 2) >> 1) & 1, a.err.wait_ns);
+    if (c >= 2) good = mbar_wait(&o_done[st], ((c - 2) >> 1) & 1, a.err.wait_ns);
     if (good && c > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
       // O may be rescaled only once PV of the previous chunk has landed in it.
-      good = __all_sync(0xffffffffu, wait_live(&o_done[st ^ 1], ((c - 1) >> 1) & 1, a.err.wait_ns));
+      good = __all_sync(0xffffffffu, mbar_wait(&o_done[st ^ 1], ((c - 1) >> 1) & 1, a.err.wait_ns));
       if (good) {
         tc_fence_after();
         for (int jj = oc0; jj < oc1; jj += 16) {
@@ -374,7 +347,7 @@ __global__ void __launch_bounds__(384, 1)
         tmem_st_wait();
       }
     }
-    if (!good) s_flag[0] = 1;
+    if (!good) s_flag[0] = 1;  // every thread stops at the next uniform check
     // P row: 64 bf16 = 8 chunks of 16 bytes, chunk index XOR (row % 8); half h
     // writes chunks 4h .. 4h + 3
     const uint32_t p_row = smem_u32(smem + L.p_off(st)) + r * 128;
@@ -387,7 +360,7 @@ __global__ void __launch_bounds__(384, 1)
     if (vc < CK) {
       // Masked keys have P = 0, but 0 * (NaN or Inf) in V would still poison O:
       // zero the V rows past the valid keys once their load has landed.
-      const bool w3 = wait_live(&v_full[st], (c >> 1) & 1, kDrainNs);
+      const bool w3 = mbar_wait(&v_full[st], (c >> 1) & 1, kDrainNs);
       if (w3) {
         uint8_t* vbase = smem + L.v_off(st);
         const int rows = CK - vc;
@@ -403,11 +376,10 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_before();
     mbar_arrive(&p_full[st]);
   }
-  if (s_flag[0]) ok = false;
-  if (!ok) set_error(a.err, DEV_TIMEOUT);
+  if (!ok || s_flag[0]) set_error(a.err, DEV_TIMEOUT);
   // PVs complete in issue order: the last chunk's commit covers them all
   if (nch > 0 && ok) ok = mbar_wait(&o_done[(nch - 1) & 1], ((nch - 1) >> 1) & 1, kDrainNs);
-  ok = named_and(1, 256, ok && s_flag[0] == 0);  // CTA-uniform among the 256 softmax threads
+  ok = named_and(1, 256, ok) && s_flag[0] == 0;  // CTA-uniform among the 256 softmax threads
   tc_fence_after();
   // row sum = half 0 + half 1 (the exchange slots are free: both passed the barrier)
   s_ml[h * QROWS + r] = l_run;
