@@ -37,7 +37,10 @@ __device__ __forceinline__ void epi_resid(const Shape& s, const EpiArgs& e, int 
 // u = gelu_tanh(y W_gate^T) * (y W_up^T)
 template <typename TA>
 __device__ __forceinline__ void epi_geglu(const Shape& s, const EpiArgs& e, int m, int f, float g, float up) {
-  st_act<TA>(static_cast<TA*>(e.u) + (size_t)m * s.F + f, gelu_tanh(g) * up);
+  if constexpr (sizeof(TA) == 2)
+    st_act<TA>(static_cast<TA*>(e.u) + (size_t)m * s.F + f, gelu_tanh_bf16out(g) * up);
+  else
+    st_act<TA>(static_cast<TA*>(e.u) + (size_t)m * s.F + f, gelu_tanh(g) * up);
 }
 
 template <typename TA>

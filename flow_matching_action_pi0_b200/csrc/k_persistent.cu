@@ -599,8 +599,8 @@ __device__ bool gemm_phase(const Ctx& c, int ph, int k, int l, int use, int& gi,
         ua.w += x.w;
       }
       const int f = g * 128 + row;
-      store4_bf16(a.u + (size_t)m * s.F + f, gelu_tanh(ga.x) * ua.x, gelu_tanh(ga.y) * ua.y,
-                  gelu_tanh(ga.z) * ua.z, gelu_tanh(ga.w) * ua.w);
+      store4_bf16(a.u + (size_t)m * s.F + f, gelu_tanh_bf16out(ga.x) * ua.x, gelu_tanh_bf16out(ga.y) * ua.y,
+                  gelu_tanh_bf16out(ga.z) * ua.z, gelu_tanh_bf16out(ga.w) * ua.w);
     }
   }
   return true;

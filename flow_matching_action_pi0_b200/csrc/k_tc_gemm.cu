@@ -138,7 +138,7 @@ __device__ __forceinline__ void epi_one(const Shape& s, const EpiArgs& e, int f,
     float* hp = e.h + (size_t)m * s.D + f;
     *hp = fmaf(e.gate[f], a0, *hp);
   } else if constexpr (EPI == EPI_GEGLU) {
-    static_cast<bf16*>(e.u)[(size_t)m * s.F + f] = f2bf(gelu_tanh(a0) * a1);
+    static_cast<bf16*>(e.u)[(size_t)m * s.F + f] = f2bf(gelu_tanh_bf16out(a0) * a1);
   } else {
     epi_qkv<bf16>(s, e, m, f, a0);
   }
@@ -167,7 +167,7 @@ __device__ __forceinline__ void epi_batch(const Shape& s, const EpiArgs& e, int 
     bf16* u = static_cast<bf16*>(e.u);
 #pragma unroll
     for (int i = 0; i < NB; ++i)
-      if (i < n) u[(size_t)ms[i] * s.F + f] = f2bf(gelu_tanh(a0[i]) * a1[i]);
+      if (i < n) u[(size_t)ms[i] * s.F + f] = f2bf(gelu_tanh_bf16out(a0[i]) * a1[i]);
   } else {
     const int qd = s.Hq * s.d;
     if (f < qd) {
@@ -503,7 +503,7 @@ __global__ void __launch_bounds__(256, 2)
         if (NA == 2) tmem_ld16(trow + p.tn + c * 16, v1);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) stg[j * 128 + row] = NA == 2 ? gelu_tanh(v0[j]) * v1[j] : v0[j];
+        for (int j = 0; j < 16; ++j) stg[j * 128 + row] = NA == 2 ? gelu_tanh_bf16out(v0[j]) * v1[j] : v0[j];
       }
       named_bar(1 + half, 128);
       const int m = mbase + c * 16 + tj;
