@@ -50,8 +50,8 @@ __host__ __device__ inline AttnSmem attn_layout(int d) {
   L.k0_off = qbytes;
   L.v0_off = qbytes + kvbytes;
   L.slot = 2 * kvbytes;                    // [K0 | V0 | K1 | V1]
-  L.p0_off = qbytes + 4 * kvbytes;         // two [128][64] bf16 P buffers
-  L.bar_off = L.p0_off + 2 * QROWS * CK * 2;
+  L.p0_off = qbytes + 4 * kvbytes;         // (P lives in TMEM, over its S columns)
+  L.bar_off = L.p0_off;
   L.ml_off = L.bar_off + 256;
   L.total = L.ml_off + QROWS * 12 + 1024;
   return L;
@@ -227,7 +227,6 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t idesc_s = idesc_bf16(QROWS, CK);
     const uint32_t idesc_o = idesc_bf16(QROWS, d, 0, 1);
     const uint32_t q_base = smem_u32(smem + L.q_off);
-    const uint32_t p_base = smem_u32(smem + L.p0_off);
     bool good = mbar_wait(q_full, 0, a.err.wait_ns);
     // descriptors are built once per operand and stepped in 16-byte units
     const uint64_t q_desc = sw128_desc(q_base, 16, 1024);
@@ -256,12 +255,12 @@ __global__ void __launch_bounds__(384, 1)
         break;
       }
       tc_fence_after();
-      const uint64_t p_desc = sw128_desc(p_base + st * (QROWS * CK * 2), 16, 1024);
       const uint64_t v_desc = sw128_desc(smem_u32(smem + L.v_off(st)), CK * 128, 1024);
+      // A = P in TMEM: 16 keys per MMA = 8 columns of bf16 pairs
 #pragma unroll
       for (int k16 = 0; k16 < CK / 16; ++k16)
-        umma_bf16(t_o, desc_add(p_desc, k16 * 32u), desc_add(v_desc, k16 * 16u * 128u), idesc_o,
-                  (c > 0 || k16 > 0) ? 1u : 0u);
+        umma_bf16_tmem_a(t_o, t_s[st] + k16 * 8u, desc_add(v_desc, k16 * 16u * 128u), idesc_o,
+                         (c > 0 || k16 > 0) ? 1u : 0u);
       umma_commit(&o_done[st]);
       umma_commit(&v_empty[st]);
       if (c + 2 < nch) good = issue_s(c + 2);
@@ -328,9 +327,10 @@ __global__ void __launch_bounds__(384, 1)
     }
     l_run = l_run * alpha + psum;
     m_run = mx;
-    // P is double-buffered: buffer st is free once PV of chunk c - 2 is done.
+    // P goes into the S columns of this buffer (both halves read them before
+    // the exchange barriers); PV of chunk c - 2, which read the previous P
+    // there, finished before S of chunk c did (commits complete in issue order).
     bool good = true;
-    if (c >= 2) good = mbar_wait(&o_done[st], ((c - 2) >> 1) & 1, a.err.wait_ns);
     if (good && c > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
       // O may be rescaled only once PV of the previous chunk has landed in it.
       good = __all_sync(0xffffffffu, mbar_wait(&o_done[st ^ 1], ((c - 1) >> 1) & 1, a.err.wait_ns));
@@ -348,14 +348,13 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
     if (!good) s_flag[0] = 1;  // every thread stops at the next uniform check
-    // P row: 64 bf16 = 8 chunks of 16 bytes, chunk index XOR (row % 8); half h
-    // writes chunks 4h .. 4h + 3
-    const uint32_t p_row = smem_u32(smem + L.p_off(st)) + r * 128;
+    // P row in TMEM: keys 32h .. 32h + 31 as bf16 pairs in columns 16h .. 16h + 15
+    {
+      float pk[16];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint32_t addr = p_row + (((uint32_t)(h * 4 + q) ^ (uint32_t)(r & 7)) << 4);
-      st_shared_v4(addr, pack_bf16x2(sv[q * 8 + 0], sv[q * 8 + 1]), pack_bf16x2(sv[q * 8 + 2], sv[q * 8 + 3]),
-                   pack_bf16x2(sv[q * 8 + 4], sv[q * 8 + 5]), pack_bf16x2(sv[q * 8 + 6], sv[q * 8 + 7]));
+      for (int q = 0; q < 16; ++q) pk[q] = __uint_as_float(pack_bf16x2(sv[2 * q], sv[2 * q + 1]));
+      tmem_st16(t_s[st] + lane_off + h * 16, pk);
+      tmem_st_wait();
     }
     if (vc < CK) {
       // Masked keys have P = 0, but 0 * (NaN or Inf) in V would still poison O:
@@ -371,8 +370,8 @@ __global__ void __launch_bounds__(384, 1)
       } else {
         s_flag[0] = 1;
       }
+      fence_proxy_async_smem();  // the zeroed V rows are read by the tensor cores
     }
-    fence_proxy_async_smem();
     tc_fence_before();
     mbar_arrive(&p_full[st]);
   }
