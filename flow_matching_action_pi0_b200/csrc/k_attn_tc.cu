@@ -10,15 +10,17 @@
 //
 // One CTA = (b, g, 128-row query tile, key split).  Per 64-key chunk c:
 //   MMA warp   S_c = Q K_c^T  (M=128, N=64, K=head_dim; TMEM, double buffered)
-//   4 warps    online softmax on S_c (thread = query row, log2 domain),
+//   8 warps    online softmax on S_c (two threads per row, log2 domain),
 //              rescale O in TMEM when the row max grows by more than 2^8
-//              (otherwise keep the old reference), write P_c (bf16,
-//              128-byte swizzled K-major) to shared memory
-//   MMA warp   O += P_c V_c   (M=128, N=head_dim, K=64; V read MN-major)
-// Warps 0-3 run the softmax and the output (thread = query row = TMEM lane);
+//              (otherwise keep the old reference), write P_c as bf16
+//              pairs back into TMEM over the first 32 columns of S_c
+//   MMA warp   O += P_c V_c   (M=128, N=head_dim, K=64; A = P_c read from
+//              TMEM, V read MN-major from shared memory)
+// Warps 0-3 and 8-11 run the softmax and the output (two threads per query
+// row: one per 32-key half of the chunk; row = TMEM lane);
 // warp 4 streams Q and the K chunks, warp 6 the V chunks (2-slot rings each,
 // a K slot refilled as soon as S of its chunk is done); warp 5 issues the MMAs;
-// all eight warps take part in the split-KV merge.
+// all twelve warps take part in the split-KV merge.
 // Key splits (split-KV, for small batches) form a thread-block cluster; their
 // unnormalised partial O rows, row maxima and sums are merged through
 // distributed shared memory in rank order, so the result is bitwise
@@ -35,8 +37,7 @@ constexpr int QROWS = 128;      // query rows per CTA
 constexpr long long kDrainNs = 4000000000LL;
 
 struct AttnSmem {
-  uint32_t q_off, k0_off, v0_off, slot, p0_off, bar_off, ml_off, total;
-  __host__ __device__ uint32_t p_off(int j) const { return p0_off + (uint32_t)j * (QROWS * CK * 2); }
+  uint32_t q_off, k0_off, v0_off, slot, bar_off, ml_off, total;
   // ring slot st of K / V (arithmetic, so no local-memory array is indexed)
   __host__ __device__ uint32_t k_off(int st) const { return k0_off + (uint32_t)st * slot; }
   __host__ __device__ uint32_t v_off(int st) const { return v0_off + (uint32_t)st * slot; }
@@ -50,8 +51,7 @@ __host__ __device__ inline AttnSmem attn_layout(int d) {
   L.k0_off = qbytes;
   L.v0_off = qbytes + kvbytes;
   L.slot = 2 * kvbytes;                    // [K0 | V0 | K1 | V1]
-  L.p0_off = qbytes + 4 * kvbytes;         // (P lives in TMEM, over its S columns)
-  L.bar_off = L.p0_off;
+  L.bar_off = qbytes + 4 * kvbytes;        // (P lives in TMEM, over its S columns)
   L.ml_off = L.bar_off + 256;
   L.total = L.ml_off + QROWS * 12 + 1024;
   return L;
@@ -82,10 +82,6 @@ __device__ __forceinline__ bool named_and(int id, int n, bool v) {
 __device__ __forceinline__ void named_sync(int id, int n) {
   __syncwarp();
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
 __host__ __device__ inline uint32_t attn_tmem_cols(int d) {

@@ -131,72 +131,63 @@ __device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
   return v;
 }
 
-// Epilogue of one output (token m, feature f); compact on purpose.
-template <int EPI>
-__device__ __forceinline__ void epi_one(const Shape& s, const EpiArgs& e, int f, int m, float a0, float a1) {
-  if constexpr (EPI == EPI_RESID) {
-    float* hp = e.h + (size_t)m * s.D + f;
-    *hp = fmaf(e.gate[f], a0, *hp);
-  } else if constexpr (EPI == EPI_GEGLU) {
-    static_cast<bf16*>(e.u)[(size_t)m * s.F + f] = f2bf(gelu_tanh_bf16out(a0) * a1);
-  } else {
-    epi_qkv<bf16>(s, e, m, f, a0);
-  }
-}
-
 __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
-// Epilogue of one output feature f over n <= 16 tokens ms[] (accumulators a0,
-// and a1 for the GeGLU up projection).  Loads that the results need (residual
-// stream, slot lengths) are issued for the whole batch before any is used.
-template <int EPI, int NB = 16>
-__device__ __forceinline__ void epi_batch(const Shape& s, const EpiArgs& e, int f, const int* ms, const float* a0,
-                                          const float* a1, int n) {
+__device__ __forceinline__ float4 ld_shared_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void add4(float4& a, const float4 b) {
+  a.x += b.x;
+  a.y += b.y;
+  a.z += b.z;
+  a.w += b.w;
+}
+
+__device__ __forceinline__ void store4_bf16(bf16* p, float x, float y, float z, float w) {
+  const uint32_t lo = (uint32_t)__bfloat16_as_ushort(f2bf(x)) | ((uint32_t)__bfloat16_as_ushort(f2bf(y)) << 16);
+  const uint32_t hi = (uint32_t)__bfloat16_as_ushort(f2bf(z)) | ((uint32_t)__bfloat16_as_ushort(f2bf(w)) << 16);
+  *reinterpret_cast<uint2*>(p) = make_uint2(lo, hi);
+}
+
+// Epilogue of 4 consecutive output features f..f+3 of token m from the
+// reduced accumulators a0 (and a1, the up projection, for GeGLU); h4 is the
+// residual stream there and g4 the gate (gated residual), len the slot length
+// of the token's request (k / v rows).  4 divides head_dim, so the run never
+// crosses a head.
+template <int EPI>
+__device__ __forceinline__ void epi_vec4(const Shape& s, const EpiArgs& e, int m, int f, float4 a0, float4 a1,
+                                         float4 h4, float4 g4, int len) {
   if constexpr (EPI == EPI_RESID) {
-    float hv[NB];
-    const float g = e.gate[f];
-#pragma unroll
-    for (int i = 0; i < NB; ++i)
-      if (i < n) hv[i] = e.h[(size_t)ms[i] * s.D + f];
-#pragma unroll
-    for (int i = 0; i < NB; ++i)
-      if (i < n) e.h[(size_t)ms[i] * s.D + f] = fmaf(g, a0[i], hv[i]);
+    h4.x = fmaf(g4.x, a0.x, h4.x);
+    h4.y = fmaf(g4.y, a0.y, h4.y);
+    h4.z = fmaf(g4.z, a0.z, h4.z);
+    h4.w = fmaf(g4.w, a0.w, h4.w);
+    *reinterpret_cast<float4*>(e.h + (size_t)m * s.D + f) = h4;
   } else if constexpr (EPI == EPI_GEGLU) {
-    bf16* u = static_cast<bf16*>(e.u);
-#pragma unroll
-    for (int i = 0; i < NB; ++i)
-      if (i < n) u[(size_t)ms[i] * s.F + f] = f2bf(gelu_tanh_bf16out(a0[i]) * a1[i]);
+    store4_bf16(static_cast<bf16*>(e.u) + (size_t)m * s.F + f, gelu_tanh_bf16out(a0.x) * a1.x,
+                gelu_tanh_bf16out(a0.y) * a1.y, gelu_tanh_bf16out(a0.z) * a1.z, gelu_tanh_bf16out(a0.w) * a1.w);
   } else {
+    const int b = m / s.H, t = m - b * s.H;
     const int qd = s.Hq * s.d;
+    bf16* dst;
     if (f < qd) {
       const int hq = f / s.d, j = f - hq * s.d;
-      bf16* q = static_cast<bf16*>(e.q) + (size_t)hq * s.H * s.d + j;
-#pragma unroll
-      for (int i = 0; i < NB; ++i)
-        if (i < n) {
-          const int b = ms[i] / s.H, t = ms[i] - b * s.H;
-          q[((size_t)b * s.Hq * s.H + t) * s.d] = f2bf(a0[i]);
-        }
+      dst = static_cast<bf16*>(e.q) + ((size_t)(b * s.Hq + hq) * s.H + t) * s.d + j;
     } else {
       const int kvd = s.Hkv * s.d;
       const bool is_v = f >= qd + kvd;
       const int fk = f - qd - (is_v ? kvd : 0);
       const int g = fk / s.d, j = fk - g * s.d;
-      bf16* base = static_cast<bf16*>(is_v ? e.vc : e.kc) +
-                   ((size_t)e.layer * s.Bmax * s.Hkv + g) * s.Ptot * s.d + j;
-      int lens[NB];
-#pragma unroll
-      for (int i = 0; i < NB; ++i)
-        if (i < n) lens[i] = e.lens[ms[i] / s.H];
-#pragma unroll
-      for (int i = 0; i < NB; ++i)
-        if (i < n) {
-          const int b = ms[i] / s.H, t = ms[i] - b * s.H;
-          base[((size_t)b * s.Hkv * s.Ptot + lens[i] + t) * s.d] = f2bf(a0[i]);
-        }
+      dst = static_cast<bf16*>(is_v ? e.vc : e.kc) +
+            (((size_t)(e.layer * s.Bmax + b) * s.Hkv + g) * s.Ptot + len + t) * s.d + j;
     }
+    store4_bf16(dst, a0.x, a0.y, a0.z, a0.w);
   }
 }
 
@@ -489,40 +480,63 @@ __global__ void __launch_bounds__(256, 2)
   const int nchunks = p.tn / 16;
 
   if constexpr (!SPLIT) {
-    // Staged through shared memory (the ring is idle now): thread = weight row
-    // parks 16 tokens of its row, then thread = (token, 16 consecutive
-    // features) writes them as vectors.  Each warpgroup has its own 8 KB tile.
-    float* stg = reinterpret_cast<float*>(smem) + half * (16 * 128);
-    const int th = row;  // thread index within the warpgroup
-    const int tj = th >> 3, fg = (th & 7) * 16;
-    const int f = ntile * 128 + fg;
-    for (int c = half; c < nchunks; c += 2) {
-      if (ok) {
-        float v0[16], v1[16];
-        tmem_ld16(trow + c * 16, v0);
-        if (NA == 2) tmem_ld16(trow + p.tn + c * 16, v1);
-        tmem_ld_wait();
+    // Per warp, with no barrier across warps: the warp's 32 rows (output
+    // features) x 16 tokens of a chunk pass through its own [16][36] fp32 tile
+    // (the ring is idle now), thread = row on the way in and thread = (token,
+    // 16 consecutive features) on the way out, so each token's 32 features are
+    // written as 64 contiguous bytes.  The TMEM load of the warp's next chunk
+    // is in flight while the current one is written out.
+    constexpr int TLD = 36;  // row stride in floats: 16-byte rows, conflict-free both ways
+    float* tb = reinterpret_cast<float*>(smem) + warp * (16 * TLD);
+    const int jt = lane >> 1, fh = (lane & 1) * 16;
+    const int f = ntile * 128 + quarter * 32 + fh;
+    float a0[16], a1[16], b0[16], b1[16];
+    auto load = [&](int c, float* x0, float* x1) {
+      tmem_ld16(trow + c * 16, x0);
+      if (NA == 2) tmem_ld16(trow + p.tn + c * 16, x1);
+    };
+    auto settle = [&](float* x0, float* x1) {
+      tmem_ld_wait();
+      reg_fence16(x0);
+      if (NA == 2) reg_fence16(x1);
+    };
+    auto emit = [&](int c, const float* x0, const float* x1) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) stg[j * 128 + row] = NA == 2 ? gelu_tanh_bf16out(v0[j]) * v1[j] : v0[j];
-      }
-      named_bar(1 + half, 128);
-      const int m = mbase + c * 16 + tj;
-      if (ok && m < e.M && f < a.N) {
+      for (int j = 0; j < 16; ++j) tb[j * TLD + lane] = NA == 2 ? gelu_tanh_bf16out(x0[j]) * x1[j] : x0[j];
+      __syncwarp();
+      const int m = mbase + c * 16 + jt;
+      if (m < e.M && f < a.N) {
         float v[16];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const float4 t4 = *reinterpret_cast<const float4*>(stg + tj * 128 + fg + 4 * q);
+          const float4 t4 = *reinterpret_cast<const float4*>(tb + jt * TLD + fh + 4 * q);
           v[4 * q] = t4.x; v[4 * q + 1] = t4.y; v[4 * q + 2] = t4.z; v[4 * q + 3] = t4.w;
         }
         epi_vec16<EPI>(s, e, m, f, v);
       }
-      named_bar(1 + half, 128);
+      __syncwarp();
+    };
+    if (ok) {
+      int c = half;
+      if (c < nchunks) load(c, a0, a1);
+      for (; c < nchunks; c += 4) {
+        settle(a0, a1);
+        if (c + 2 < nchunks) load(c + 2, b0, b1);
+        emit(c, a0, a1);
+        if (c + 2 < nchunks) {
+          settle(b0, b1);
+          if (c + 4 < nchunks) load(c + 4, a0, a1);
+          emit(c + 2, b0, b1);
+        }
+      }
     }
   } else {
     // Split-K inside a cluster of S CTAs: rank r owns rows [r*R, r*R+R).  Every
     // CTA pushes each row's partial into the owner's receive buffer through
-    // distributed shared memory; after one cluster barrier each owner sums its
-    // rows over the S sources in rank order, reading only local memory.
+    // distributed shared memory (layout [na][src][token][row]); after one
+    // cluster barrier each owner sums its rows over the S sources in rank
+    // order, reading only local memory, so results are bitwise reproducible
+    // and no partial touches global memory.
     const int S = p.splits, R = 128 / S;
     const uint32_t rank = cluster_rank();
     float* recv = reinterpret_cast<float*>(smem + L.recv_off);
@@ -530,39 +544,117 @@ __global__ void __launch_bounds__(256, 2)
     if (ok) {
       const int owner = row / R, rr = row - owner * R;
       const uint32_t dst = map_cluster(smem_u32(recv), (uint32_t)owner);
-      for (int c = half; c < nchunks; c += 2) {
-        float v0[16], v1[16];
-        tmem_ld16(trow + c * 16, v0);
-        if (NA == 2) tmem_ld16(trow + p.tn + c * 16, v1);
+      float a0[16], a1[16], b0[16], b1[16];
+      auto load = [&](int c, float* x0, float* x1) {
+        tmem_ld16(trow + c * 16, x0);
+        if (NA == 2) tmem_ld16(trow + p.tn + c * 16, x1);
+      };
+      auto settle = [&](float* x0, float* x1) {
         tmem_ld_wait();
+        reg_fence16(x0);
+        if (NA == 2) reg_fence16(x1);
+      };
+      auto push = [&](int c, const float* x0, const float* x1) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const uint32_t col = (uint32_t)(c * 16 + j);
-          st_cluster_f32(dst + ((((uint32_t)0 * S + rank) * p.tn + col) * R + rr) * 4u, v0[j]);
-          if (NA == 2) st_cluster_f32(dst + ((((uint32_t)1 * S + rank) * p.tn + col) * R + rr) * 4u, v1[j]);
+          st_cluster_f32(dst + ((((uint32_t)0 * S + rank) * p.tn + col) * R + rr) * 4u, x0[j]);
+          if (NA == 2) st_cluster_f32(dst + ((((uint32_t)1 * S + rank) * p.tn + col) * R + rr) * 4u, x1[j]);
+        }
+      };
+      int c = half;
+      if (c < nchunks) load(c, a0, a1);
+      for (; c < nchunks; c += 4) {
+        settle(a0, a1);
+        if (c + 2 < nchunks) load(c + 2, b0, b1);
+        push(c, a0, a1);
+        if (c + 2 < nchunks) {
+          settle(b0, b1);
+          if (c + 4 < nchunks) load(c + 4, a0, a1);
+          push(c + 2, b0, b1);
         }
       }
     }
+
+    // Reduction by thread = (4 consecutive rows of this rank, token): rows
+    // 4*(t % (R/4)).. and tokens t / (R/4) + k * 256 / (R/4), one float4 per
+    // source in rank order.  The loads the epilogue needs (residual stream,
+    // gate, slot lengths) are issued before the cluster barrier, so they
+    // overlap the wait for the slowest rank.  (The residual epilogue that
+    // also writes the per-token sums of squares keeps one row per thread: its
+    // shuffle tree runs over the R threads of a token.)
+    constexpr int UB = 8;  // tokens per batch
+    const bool vec = !(EPI == EPI_RESID && e.ss_out);
+    const int G4 = R / 4, lg4 = __ffs(G4) - 1;
+    const int g4 = threadIdx.x & (G4 - 1);
+    const int cstep4 = 256 >> lg4;
+    const int col0 = threadIdx.x >> lg4;
+    const int fv = ntile * 128 + (int)rank * R + 4 * g4;
+    const bool fv_ok = fv < a.N;
+    const bool need_len = EPI == EPI_QKV && fv >= s.Hq * s.d;
+    float4 hv[UB];
+    int lv[UB];
+    float4 gv = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (EPI == EPI_RESID && ok && vec && fv_ok) gv = *reinterpret_cast<const float4*>(e.gate + fv);
+    auto prefetch = [&](int cb) {
+#pragma unroll
+      for (int k = 0; k < UB; ++k) {
+        const int col = cb + k * cstep4, m = mbase + col;
+        if (col < p.tn && m < e.M && fv_ok) {
+          if constexpr (EPI == EPI_RESID) hv[k] = __ldcg(reinterpret_cast<const float4*>(e.h + (size_t)m * s.D + fv));
+          if constexpr (EPI == EPI_QKV) lv[k] = need_len ? e.lens[m / s.H] : 0;
+        }
+      }
+    };
+    if (ok && vec) prefetch(col0);
     cluster_sync();
-    if (ok) {
+    if (ok && vec) {
+      const uint32_t rb = smem_u32(recv) + (uint32_t)(16 * g4);
+      const uint32_t src_stride = (uint32_t)p.tn * R * 4u;
+      const uint32_t na_stride = (uint32_t)S * src_stride;
+#pragma unroll 1
+      for (int cb = col0; cb < p.tn; cb += UB * cstep4) {
+        if (cb != col0) prefetch(cb);
+        float4 s0[UB], s1[UB];
+#pragma unroll
+        for (int k = 0; k < UB; ++k) {
+          s0[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+          s1[k] = s0[k];
+        }
+#pragma unroll 1
+        for (int src = 0; src < S; ++src) {
+#pragma unroll
+          for (int k = 0; k < UB; ++k) {
+            const int col = cb + k * cstep4;
+            if (col < p.tn) {
+              const uint32_t addr = rb + (uint32_t)col * R * 4u + (uint32_t)src * src_stride;
+              add4(s0[k], ld_shared_f32x4(addr));
+              if (NA == 2) add4(s1[k], ld_shared_f32x4(addr + na_stride));
+            }
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < UB; ++k) {
+          const int col = cb + k * cstep4, m = mbase + col;
+          if (col < p.tn && m < e.M && fv_ok) epi_vec4<EPI>(s, e, m, fv, s0[k], s1[k], hv[k], gv, lv[k]);
+        }
+      }
+    } else if (ok) {
       // Thread t keeps one row (t % R) and walks the tokens t / R, t / R + 256 / R, ...
       const int rr = threadIdx.x % R;
       const int f = ntile * 128 + (int)rank * R + rr;
       const int cstep = 256 / R;
       const uint32_t rbase = smem_u32(recv) + (uint32_t)rr * 4u;
       const uint32_t src_stride = (uint32_t)p.tn * R * 4u;
-      const uint32_t na_stride = (uint32_t)S * src_stride;
-      // eight tokens per batch: their loads (partials, residual) overlap
 #pragma unroll 1
       for (int c0 = threadIdx.x / R; c0 < p.tn; c0 += 8 * cstep) {
-        float s0[8], s1[8];
-        int ms[16];
+        float s0[8];
+        int ms[8];
         int n = 0;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int col = c0 + i * cstep;
           s0[i] = 0.f;
-          s1[i] = 0.f;
           ms[i] = mbase + col;
           if (col < p.tn && mbase + col < e.M) n = i + 1;
         }
@@ -572,49 +664,42 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const uint32_t addr = rbase + (uint32_t)(c0 + i * cstep) * R * 4u + src * src_stride;
-            if (i < n) {
-              s0[i] += ld_shared_f32(addr);
-              if (NA == 2) s1[i] += ld_shared_f32(addr + na_stride);
-            }
+            if (i < n) s0[i] += ld_shared_f32(addr);
           }
         }
-        if (EPI == EPI_RESID && e.ss_out) {
-          // Gated residual, then the sum of squares of the updated h over this
-          // rank's R rows per token: the R threads of a token group are
-          // adjacent lanes (R is a power of two <= 32), reduced by a fixed
-          // shuffle tree into slot (tile * S + rank).
-          const float g = e.gate[f];
-          float hv[8];
+        // Gated residual, then the sum of squares of the updated h over this
+        // rank's R rows per token: the R threads of a token group are
+        // adjacent lanes (R is a power of two <= 32), reduced by a fixed
+        // shuffle tree into slot (tile * S + rank).
+        const float g = e.gate[f];
+        float hv1[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (i < n) hv1[i] = e.h[(size_t)ms[i] * s.D + f];
+        const int lane_g = (threadIdx.x & 31) & ~(R - 1);
+        const unsigned gmask = R >= 32 ? 0xffffffffu : (((1u << R) - 1u) << lane_g);
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          v[i] = 0.f;
+          if (i < n) {
+            hv1[i] = fmaf(g, s0[i], hv1[i]);
+            e.h[(size_t)ms[i] * s.D + f] = hv1[i];
+            v[i] = hv1[i] * hv1[i];
+          }
+        }
+#pragma unroll
+        for (int lvl = 4; lvl >= 0; --lvl) {  // offsets R/2 .. 1, all eight tokens per level
+          const int o = 1 << lvl;
+          if (o < R) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] += __shfl_xor_sync(gmask, v[i], o);
+          }
+        }
+        if (rr == 0) {
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            if (i < n) hv[i] = e.h[(size_t)ms[i] * s.D + f];
-          const int lane_g = (threadIdx.x & 31) & ~(R - 1);
-          const unsigned gmask = R >= 32 ? 0xffffffffu : (((1u << R) - 1u) << lane_g);
-          float v[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            v[i] = 0.f;
-            if (i < n) {
-              hv[i] = fmaf(g, s0[i], hv[i]);
-              e.h[(size_t)ms[i] * s.D + f] = hv[i];
-              v[i] = hv[i] * hv[i];
-            }
-          }
-#pragma unroll
-          for (int lv = 4; lv >= 0; --lv) {  // offsets R/2 .. 1, all eight tokens per level
-            const int o = 1 << lv;
-            if (o < R) {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) v[i] += __shfl_xor_sync(gmask, v[i], o);
-            }
-          }
-          if (rr == 0) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              if (i < n) e.ss_out[(size_t)(ntile * S + (int)rank) * e.ss_ld + ms[i]] = v[i];
-          }
-        } else {
-          epi_batch<EPI, 8>(s, e, f, ms, s0, s1, n);
+            if (i < n) e.ss_out[(size_t)(ntile * S + (int)rank) * e.ss_ld + ms[i]] = v[i];
         }
       }
     }
