@@ -185,10 +185,21 @@ __global__ void __launch_bounds__(256) k_norm(const Shape s, const float* __rest
                                               int M) {
   const int lane = threadIdx.x & 31;
   const int m = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int D = s.D;
+  // The modulation rows are built before the loop, not by the previous
+  // kernel: read them before waiting for it.
+  float4 cs[NV], ds[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int j = 4 * (lane + 32 * i);
+    if (j < D && m < M) {
+      cs[i] = __ldg(reinterpret_cast<const float4*>(scale + j));
+      ds[i] = __ldg(reinterpret_cast<const float4*>(shift + j));
+    }
+  }
   pdl_wait();
   pdl_launch_dependents();
   if (m >= M) return;
-  const int D = s.D;
   const float* hr = h + (size_t)m * D;
   float4 v[NV];
   float ss = 0.f;
@@ -206,8 +217,8 @@ __global__ void __launch_bounds__(256) k_norm(const Shape s, const float* __rest
   for (int i = 0; i < NV; ++i) {
     const int j = 4 * (lane + 32 * i);
     if (j < D) {
-      const float4 c = *reinterpret_cast<const float4*>(scale + j);
-      const float4 d = *reinterpret_cast<const float4*>(shift + j);
+      const float4 c = cs[i];
+      const float4 d = ds[i];
       const float o[4] = {v[i].x * r * (1.f + c.x) + d.x, v[i].y * r * (1.f + c.y) + d.y,
                           v[i].z * r * (1.f + c.z) + d.z, v[i].w * r * (1.f + c.w) + d.w};
       store4(yr + j, o);
