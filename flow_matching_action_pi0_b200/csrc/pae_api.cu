@@ -315,7 +315,16 @@ TcPlan plan_gemm_large(int M, int nfeat, int K, int na, int max_splits, bool w4,
   return best;
 }
 
-TcPlan plan_gemm(int M, int nfeat, int K, int na, int max_splits = 16, bool w4 = false, bool norm = false) {
+// whole_sm (small batches): the projection follows the norm kernel, which
+// holds no shared memory, so its CTAs can take a whole SM and still start
+// early under programmatic dependent launch: split-K only as far as one CTA
+// per SM (tiles x splits <= 148) with a deep ring.  Measured at batch 1
+// (QKV 20 tiles -> split 4, gate/up 32 tiles -> split 4): 9.0 ms per call
+// against 9.6 ms with split 8 and two CTAs per SM.  O and down follow the
+// attention and gate/up kernels, which fill most of an SM's shared memory, and
+// keep the two-CTA footprint (splitting them 4 or 16 ways measured slower).
+TcPlan plan_gemm(int M, int nfeat, int K, int na, int max_splits = 16, bool w4 = false, bool norm = false,
+                 bool whole_sm = false) {
   if (M > 256) {
     const TcPlan p = plan_gemm_large(M, nfeat, K, na, max_splits, w4, norm);
     if (p.tn > 0) return p;
@@ -329,12 +338,14 @@ TcPlan plan_gemm(int M, int nfeat, int K, int na, int max_splits = 16, bool w4 =
   const uint32_t stage = (uint32_t)na * 16384u + (uint32_t)p.tn * 128u + (w4 ? (uint32_t)na * 4096u : 0u) +
                          (norm ? (uint32_t)p.tn * 128u : 0u);
   const uint32_t recv = (uint32_t)na * p.tn * 128u * 4u;  // split-K receive buffer
-  const bool small = p.tn <= 64;  // two CTAs per SM (shared memory and the 128-register cap allow it)
+  // two CTAs per SM (shared memory and the 128-register cap allow it)
+  const bool small = p.tn <= 64 && !whole_sm;
   const uint32_t budget = small ? 110u * 1024u : 200u * 1024u;
   const int target = small ? 2 * 148 : 148;
   p.splits = 1;
   for (int sp = 2; sp <= std::min(16, max_splits); sp *= 2)
     if (nkb % sp == 0 && base * sp <= target && recv <= budget) p.splits = sp;
+  if (whole_sm && p.tn <= 64 && fit_ring(p, na, nkb, w4, norm, budget)) return p;
   // without split-K a CTA streams a long K range: give it a deep ring
   const uint32_t ring_budget = p.splits == 1 ? 200u * 1024u : budget;
   int st = std::max(2, std::min((int)(ring_budget / stage), 8));
@@ -448,8 +459,9 @@ pae_status build_plan(pae_ctx* ctx, int B, Plan* P) {
   P->fuse_norm = ctx->use_fused_norm && !w4 && P->M <= 64 && tn_small <= 64 && P->o.splits >= 4 &&
                  P->down.splits >= 4 && P->o.tok_tiles == 1 && P->down.tok_tiles == 1 &&
                  (s.D / 128) * std::max(P->o.splits, P->down.splits) <= kSsSlots;
-  P->qkv = plan_gemm(P->M, s.qkv_rows, s.D, 1, ctx->max_splitk, w4, P->fuse_norm);
-  P->gu = plan_gemm(P->M, s.F, s.D, 2, ctx->max_splitk, w4, P->fuse_norm);
+  const bool whole_sm = !w4 && !P->fuse_norm;  // they follow the norm kernel
+  P->qkv = plan_gemm(P->M, s.qkv_rows, s.D, 1, ctx->max_splitk, w4, P->fuse_norm, whole_sm);
+  P->gu = plan_gemm(P->M, s.F, s.D, 2, ctx->max_splitk, w4, P->fuse_norm, whole_sm);
   P->attn = plan_attn(s, B);
   const uint64_t Mmax = (uint64_t)s.Bmax * s.H;
   pae_status st;
