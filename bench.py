@@ -146,13 +146,22 @@ def algorithmic(cfg: wl.ExpertConfig, batch: int, lens=None):
     return out, {"bytes": step_w + step_kv, "flops": step_flops}
 
 
-def src_hash():
+# The files each kernel class is compiled from (its own file and the headers
+# it includes); a traffic figure stays valid while these are unchanged.
+KERNEL_SOURCES = {
+    "attention": ["k_attn_tc.cu", "internal.h", "common.cuh", "launch.cuh"],
+    "gemm": ["k_tc_gemm.cu", "epilogue.cuh", "internal.h", "common.cuh", "launch.cuh"],
+}
+
+
+def src_hash(kernel=None):
+    """Hash of the kernel sources: all of csrc, or the files of one kernel class."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "flow_matching_action_pi0_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    names = KERNEL_SOURCES.get(kernel) or [n for n in os.listdir(csrc) if n.endswith((".cu", ".cuh", ".h"))]
+    for name in sorted(names):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
@@ -165,7 +174,7 @@ def ncu_traffic(workload: str, kernel: str):
     with open(p) as f:
         d = json.load(f)
     e = d.get(f"{workload}:{kernel}")
-    if not e or e.get("src_sha") != src_hash():
+    if not e or e.get("src_sha") != src_hash(kernel if kernel in KERNEL_SOURCES else None):
         return None
     return e.get("dram_bytes_per_launch")
 
