@@ -320,7 +320,8 @@ TcPlan plan_gemm_large(int M, int nfeat, int K, int na, int max_splits, bool w4,
 // early under programmatic dependent launch: split-K only as far as one CTA
 // per SM (tiles x splits <= 148) with a deep ring.  Measured at batch 1
 // (QKV 20 tiles -> split 4, gate/up 32 tiles -> split 4): 9.0 ms per call
-// against 9.6 ms with split 8 and two CTAs per SM.  O and down follow the
+// against 9.6 ms with split 8 and two CTAs per SM (int4 weights: 9.5 against
+// 10.5 ms).  O and down follow the
 // attention and gate/up kernels, which fill most of an SM's shared memory, and
 // keep the two-CTA footprint (splitting them 4 or 16 ways measured slower).
 TcPlan plan_gemm(int M, int nfeat, int K, int na, int max_splits = 16, bool w4 = false, bool norm = false,
@@ -459,7 +460,7 @@ pae_status build_plan(pae_ctx* ctx, int B, Plan* P) {
   P->fuse_norm = ctx->use_fused_norm && !w4 && P->M <= 64 && tn_small <= 64 && P->o.splits >= 4 &&
                  P->down.splits >= 4 && P->o.tok_tiles == 1 && P->down.tok_tiles == 1 &&
                  (s.D / 128) * std::max(P->o.splits, P->down.splits) <= kSsSlots;
-  const bool whole_sm = !w4 && !P->fuse_norm;  // they follow the norm kernel
+  const bool whole_sm = !P->fuse_norm;  // they follow the norm kernel
   P->qkv = plan_gemm(P->M, s.qkv_rows, s.D, 1, ctx->max_splitk, w4, P->fuse_norm, whole_sm);
   P->gu = plan_gemm(P->M, s.F, s.D, 2, ctx->max_splitk, w4, P->fuse_norm, whole_sm);
   P->attn = plan_attn(s, B);
