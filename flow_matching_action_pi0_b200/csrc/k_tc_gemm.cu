@@ -12,12 +12,14 @@
 //   warp 1 / lane 0  MMA issuer: tcgen05.mma kind::f16 (bf16 in, fp32 in TMEM)
 //   warps 0-7        epilogue: tcgen05.ld of the accumulator (thread = weight
 //                    row = output feature, 16 token columns per load; the two
-//                    warpgroups take alternate 16-token chunks)
+//                    warpgroups take alternate 16-token chunks, each warp on
+//                    its own with the next chunk's load in flight)
 // Split-K: the grid.y CTAs of one output tile form a thread-block cluster;
 // each CTA pushes its fp32 partial rows into the owning rank's shared memory
 // (distributed shared memory stores), and after one cluster barrier every
-// rank sums its 1/S slice of the rows over all sources in rank order, so
-// results are bitwise reproducible and no partial touches global memory.
+// rank sums its 1/S slice of the rows over all sources in rank order (thread =
+// 4 rows x 1 token, float4 per source), so results are bitwise reproducible
+// and no partial touches global memory.
 // The weight loads of the first ring are issued before griddepcontrol.wait, so
 // under programmatic dependent launch they overlap the previous kernel.
 // int4 weights (W4A16): TMA brings the packed [rows][32 bytes] tile per K
