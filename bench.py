@@ -137,7 +137,8 @@ def algorithmic(cfg: wl.ExpertConfig, batch: int, lens=None):
         "gate_up": {"bytes": wb(2 * F, D) + M * D * ae + M * F * ae, "flops": 2 * M * 2 * F * D},
         "down": {"bytes": wb(D, F) + M * F * ae + 2 * M * D * 4, "flops": 2 * M * D * F},
     }
-    step_w = L * (wb(qkv, D) + wb(D, att) + wb(2 * F, D) + wb(D, F)) + wb(D, A) * 2
+    # in/out projections stay in the activation dtype (bf16 in int4 mode)
+    step_w = L * (wb(qkv, D) + wb(D, att) + wb(2 * F, D) + wb(D, F)) + 2 * D * A * (4 if cfg.dtype == wl.FP32 else 2)
     step_kv = L * 2 * sum(lens) * cfg.n_kv_heads * cfg.head_dim * ae
     step_flops = L * (out["qkv"]["flops"] + out["o_proj"]["flops"] + out["gate_up"]["flops"] +
                       out["down"]["flops"] + out["attention"]["flops"]) + 2 * 2 * M * A * D
