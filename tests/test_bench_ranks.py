@@ -42,3 +42,25 @@ def test_single_rank_helpers_are_identity():
     barrier, maxr = bench.rank_helpers(1)
     barrier()
     assert maxr(3.25) == 3.25
+
+
+def test_reference_arm_prints_contract_line():
+    """`bench.py --impl reference` (the oracle on the host cores) prints one JSON
+    line with the contract's keys, on the workload it is asked for."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--config", "tiny_fp32",
+                        "--steps", "1", "--warmup", "3"], capture_output=True, text=True, cwd=root, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["config"]["workload"] == "tiny_fp32"
+    assert d["value"] > 0 and d["unit"] == "chunks/s" and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
