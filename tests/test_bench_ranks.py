@@ -64,3 +64,20 @@ def test_reference_arm_prints_contract_line():
     assert d["value"] > 0 and d["unit"] == "chunks/s" and d["higher_is_better"] is True
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_oracle_sample_is_bounded():
+    """The CPU-baseline sample repeats one request's oracle run until enough
+    work is timed, and never more than the cap."""
+    import bench
+    import workloads as wl
+    cfg = wl.TINY_FP32
+    W = wl.make_weights(cfg)
+    ks, vs = wl.make_prefix(cfg, lengths=wl.prefix_lengths(cfg)[:1])
+    noise = wl.make_noise(cfg, batch=1)
+    one = bench.oracle_sample_times(cfg, W, ks, vs, noise, cfg.steps)
+    assert len(one) == 1 and one[0] > 0
+    capped = bench.oracle_sample_times(cfg, W, ks, vs, noise, cfg.steps, min_seconds=1e9, max_reps=3)
+    assert len(capped) == 3 and all(t > 0 for t in capped)
+    enough = bench.oracle_sample_times(cfg, W, ks, vs, noise, cfg.steps, min_seconds=1e-9, max_reps=5)
+    assert len(enough) == 1
