@@ -32,7 +32,7 @@ STATUS_NAMES = {0: "PAE_OK", 1: "PAE_ERR_ARG", 2: "PAE_ERR_STATE", 3: "PAE_ERR_C
 
 # Every symbol include/pae.h declares.
 EXPORTS = ("pae_create", "pae_set_prefix", "pae_precompute_tables", "pae_denoise", "pae_denoise_host",
-           "pae_denoise_steps", "pae_set_option", "pae_profile_read", "pae_query", "pae_sync",
+           "pae_denoise_steps", "pae_set_option", "pae_profile_read", "pae_query", "pae_plan_query", "pae_sync",
            "pae_clear_error", "pae_last_error", "pae_debug_copy", "pae_precompute_tables_static",
            "pae_destroy")
 
@@ -82,6 +82,7 @@ def lib() -> ctypes.CDLL:
         "pae_set_option": (i, [v, i, ctypes.c_longlong]),
         "pae_profile_read": (i, [v, i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
         "pae_query": (i, [v, i, i, ctypes.POINTER(ctypes.c_longlong)]),
+        "pae_plan_query": (i, [ctypes.POINTER(pae_config), i, i, ctypes.POINTER(ctypes.c_longlong)]),
         "pae_sync": (i, [v, st]),
         "pae_clear_error": (None, [v]),
         "pae_last_error": (ctypes.c_char_p, [v]),
@@ -161,6 +162,12 @@ def pae_profile_read(ctx: int, kernel_class: int):
 def pae_query(ctx: int, what: int, batch: int) -> int:
     v = ctypes.c_longlong(0)
     _check(lib().pae_query(ctx, what, batch, ctypes.byref(v)), ctx)
+    return v.value
+
+
+def pae_plan_query(cfg: pae_config, what: int, batch: int) -> int:
+    v = ctypes.c_longlong(0)
+    _check(lib().pae_plan_query(ctypes.byref(cfg), what, batch, ctypes.byref(v)))
     return v.value
 
 

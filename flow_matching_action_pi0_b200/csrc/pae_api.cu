@@ -38,6 +38,7 @@ namespace {
 
 constexpr int kMaxSteps = 64;
 constexpr int kSsSlots = 256;  // sum-of-squares slots: (D / 128) tiles x split-K ranks
+constexpr int kDefaultMaxSplitK = 8;  // PAE_OPT_MAX_SPLITK until set
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -150,7 +151,7 @@ struct pae_ctx {
   long long wait_ns = 2000000000LL;
   bool use_graph = true;
   bool use_pdl = true;
-  int max_splitk = 8;
+  int max_splitk = kDefaultMaxSplitK;
   std::map<int, Plan> plans;
   Plan* last_plan = nullptr;
   unsigned profile_mask = 0;
@@ -444,26 +445,45 @@ bool plan_persistent(const pae_ctx* ctx, int B, PersistArgs* pa) {
   return true;
 }
 
+// The launch shapes of one batch size (tensor-core modes): host arithmetic
+// only, shared by the context and pae_plan_query.
+struct LaunchPlans {
+  TcPlan qkv, o, gu, down;
+  AttnPlan attn;
+  bool fuse_norm;
+};
+LaunchPlans plan_launches(const Shape& s, int B, bool w4, int max_splitk, bool use_fused_norm) {
+  LaunchPlans L{};
+  const int M = B * s.H;
+  L.o = plan_gemm(M, s.D, s.attn_dim, 1, max_splitk, w4);
+  L.down = plan_gemm(M, s.D, s.F, 1, max_splitk, w4);
+  // In-kernel adaRMSNorm for small batches (one token tile of <= 64): the
+  // residual projections' split-K ranks (R = 128 / S <= 32 rows each) write
+  // the sum-of-squares slots, so the separate norm kernels disappear.
+  const int tn_small = std::max(16, ((M + 15) / 16) * 16);
+  L.fuse_norm = use_fused_norm && !w4 && M <= 64 && tn_small <= 64 && L.o.splits >= 4 && L.down.splits >= 4 &&
+                L.o.tok_tiles == 1 && L.down.tok_tiles == 1 &&
+                (s.D / 128) * std::max(L.o.splits, L.down.splits) <= kSsSlots;
+  const bool whole_sm = !L.fuse_norm;  // they follow the norm kernel
+  L.qkv = plan_gemm(M, s.qkv_rows, s.D, 1, max_splitk, w4, L.fuse_norm, whole_sm);
+  L.gu = plan_gemm(M, s.F, s.D, 2, max_splitk, w4, L.fuse_norm, whole_sm);
+  L.attn = plan_attn(s, B);
+  return L;
+}
+
 pae_status build_plan(pae_ctx* ctx, int B, Plan* P) {
   const Shape& s = ctx->s;
   P->B = B;
   P->M = B * s.H;
   if (!ctx->act_bf16) return PAE_OK;
   P->persist = plan_persistent(ctx, B, &P->pa);
-  const bool w4 = ctx->w4 != 0;
-  P->o = plan_gemm(P->M, s.D, s.attn_dim, 1, ctx->max_splitk, w4);
-  P->down = plan_gemm(P->M, s.D, s.F, 1, ctx->max_splitk, w4);
-  // In-kernel adaRMSNorm for small batches (one token tile of <= 64): the
-  // residual projections' split-K ranks (R = 128 / S <= 32 rows each) write
-  // the sum-of-squares slots, so the separate norm kernels disappear.
-  const int tn_small = std::max(16, ((P->M + 15) / 16) * 16);
-  P->fuse_norm = ctx->use_fused_norm && !w4 && P->M <= 64 && tn_small <= 64 && P->o.splits >= 4 &&
-                 P->down.splits >= 4 && P->o.tok_tiles == 1 && P->down.tok_tiles == 1 &&
-                 (s.D / 128) * std::max(P->o.splits, P->down.splits) <= kSsSlots;
-  const bool whole_sm = !P->fuse_norm;  // they follow the norm kernel
-  P->qkv = plan_gemm(P->M, s.qkv_rows, s.D, 1, ctx->max_splitk, w4, P->fuse_norm, whole_sm);
-  P->gu = plan_gemm(P->M, s.F, s.D, 2, ctx->max_splitk, w4, P->fuse_norm, whole_sm);
-  P->attn = plan_attn(s, B);
+  const LaunchPlans LP = plan_launches(s, B, ctx->w4 != 0, ctx->max_splitk, ctx->use_fused_norm);
+  P->qkv = LP.qkv;
+  P->o = LP.o;
+  P->gu = LP.gu;
+  P->down = LP.down;
+  P->attn = LP.attn;
+  P->fuse_norm = LP.fuse_norm;
   const uint64_t Mmax = (uint64_t)s.Bmax * s.H;
   pae_status st;
   if ((st = make_map(ctx, &P->tmY, ctx->y, s.D, Mmax, 64, P->qkv.tn)) != PAE_OK) return st;
@@ -808,6 +828,28 @@ void free_all(pae_ctx* ctx) {
 
 bool is_pos(int v) { return v > 0; }
 
+Shape shape_from_config(const pae_config* cfg) {
+  Shape s{};
+  s.L = cfg->layers;
+  s.D = cfg->width;
+  s.Hq = cfg->n_q_heads;
+  s.Hkv = cfg->n_kv_heads;
+  s.d = cfg->head_dim;
+  s.F = cfg->mlp_dim;
+  s.A = cfg->action_dim;
+  s.H = cfg->chunk;
+  s.Bmax = cfg->max_batch;
+  s.Pmax = cfg->max_prefix;
+  s.Ptot = cfg->max_prefix + cfg->chunk;
+  s.G = s.Hq / s.Hkv;
+  s.qkv_rows = (s.Hq + 2 * s.Hkv) * s.d;
+  s.attn_dim = s.Hq * s.d;
+  s.group = cfg->group_size;
+  s.eps = cfg->rms_eps;
+  s.table_rows = (s.L * 2 * 3 + 2) * s.D;
+  return s;
+}
+
 pae_status validate_config(const pae_config* c) {
   if (!is_pos(c->layers) || !is_pos(c->width) || !is_pos(c->n_q_heads) || !is_pos(c->n_kv_heads) ||
       !is_pos(c->head_dim) || !is_pos(c->mlp_dim) || !is_pos(c->action_dim) || !is_pos(c->chunk) ||
@@ -863,24 +905,8 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
 
   pae_ctx* ctx = new pae_ctx();
   ctx->cfg = *cfg;
+  ctx->s = shape_from_config(cfg);
   Shape& s = ctx->s;
-  s.L = cfg->layers;
-  s.D = cfg->width;
-  s.Hq = cfg->n_q_heads;
-  s.Hkv = cfg->n_kv_heads;
-  s.d = cfg->head_dim;
-  s.F = cfg->mlp_dim;
-  s.A = cfg->action_dim;
-  s.H = cfg->chunk;
-  s.Bmax = cfg->max_batch;
-  s.Pmax = cfg->max_prefix;
-  s.Ptot = cfg->max_prefix + cfg->chunk;
-  s.G = s.Hq / s.Hkv;
-  s.qkv_rows = (s.Hq + 2 * s.Hkv) * s.d;
-  s.attn_dim = s.Hq * s.d;
-  s.group = cfg->group_size;
-  s.eps = cfg->rms_eps;
-  s.table_rows = (s.L * 2 * 3 + 2) * s.D;
   ctx->act_bf16 = cfg->dtype != PAE_FP32;
   ctx->w4 = cfg->dtype == PAE_W4A16;
   ctx->esize = ctx->act_bf16 ? 2 : 4;
@@ -1281,6 +1307,29 @@ pae_status pae_query(pae_ctx* ctx, int what, int batch, long long* value) {
     case PAE_Q_FUSED_NORM: *value = P->fuse_norm ? 1 : 0; return PAE_OK;
     default: return fail(ctx, PAE_ERR_ARG, "unknown query %d", what);
   }
+}
+
+pae_status pae_plan_query(const pae_config* cfg, int what, int batch, long long* value) {
+  if (!cfg || !value) return fail(nullptr, PAE_ERR_ARG, "null argument");
+  pae_status st = validate_config(cfg);
+  if (st != PAE_OK) return st;
+  if (batch < 1 || batch > cfg->max_batch) return fail(nullptr, PAE_ERR_ARG, "batch %d out of range", batch);
+  if (what != PAE_Q_SPLITS && what != PAE_Q_TOKEN_TILE && what != PAE_Q_ATTN_SPLITS && what != PAE_Q_FUSED_NORM)
+    return fail(nullptr, PAE_ERR_ARG, "query %d needs a context", what);
+  *value = 0;
+  if (cfg->dtype == PAE_FP32) return PAE_OK;  // CUDA-core kernels: no tensor-core launch plan
+  const Shape s = shape_from_config(cfg);
+  const LaunchPlans L = plan_launches(s, batch, cfg->dtype == PAE_W4A16, kDefaultMaxSplitK, false);
+  switch (what) {
+    case PAE_Q_SPLITS:
+      *value = (long long)L.qkv.splits | ((long long)L.o.splits << 8) | ((long long)L.gu.splits << 16) |
+               ((long long)L.down.splits << 24);
+      break;
+    case PAE_Q_TOKEN_TILE: *value = L.qkv.tn; break;
+    case PAE_Q_ATTN_SPLITS: *value = L.attn.splits; break;
+    default: *value = L.fuse_norm ? 1 : 0; break;
+  }
+  return PAE_OK;
 }
 
 pae_status pae_sync(pae_ctx* ctx, pae_stream stream) {

@@ -217,6 +217,15 @@ enum {
 };
 pae_status pae_query(pae_ctx* ctx, int what, int batch, long long* value);
 
+/* The same launch-plan queries without a context or a device: what a context
+ * created from `cfg`, with its options at their defaults, would use for
+ * `batch` (PAE_Q_SPLITS, PAE_Q_TOKEN_TILE, PAE_Q_ATTN_SPLITS or
+ * PAE_Q_FUSED_NORM; 0 in PAE_FP32 mode, which has no tensor-core plan).
+ * Host arithmetic only.  Errors: PAE_ERR_ARG for a NULL argument, a batch
+ * outside [1, max_batch] or another query; the config is checked as by
+ * pae_create (PAE_ERR_ARG / PAE_ERR_UNSUPPORTED). */
+pae_status pae_plan_query(const pae_config* cfg, int what, int batch, long long* value);
+
 /* Synchronise `stream` and report the device error word (PAE_ERR_TIMEOUT if a
  * bounded wait ran out since the last pae_clear_error). */
 pae_status pae_sync(pae_ctx* ctx, pae_stream stream);
