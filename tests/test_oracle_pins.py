@@ -91,6 +91,91 @@ def test_time_conditioning_zero_weight_closed_form():
     np.testing.assert_allclose(c, want, rtol=1e-14)
 
 
+def _swish(x: float) -> float:
+    return x / (1.0 + math.exp(-x))
+
+
+def test_time_conditioning_one_hot_closed_form():
+    # W_t1 with one 1 at [j][i] routes embedding channel i into hidden unit j;
+    # W_t2 = identity, b_t2 = 0.  Then c_j = swish(swish(e_i(t) + b1_j)) and
+    # every other c_m = swish(swish(b1_m)).  Channel i = half - 1 is sin(2 pi t / 4),
+    # which is 1 at t = 1 and 0 at t = 0, so a grid read backwards (1 - t) fails,
+    # a dropped inner swish fails, and j != i makes a transposed W_t1 fail.
+    cfg = _tiny()
+    p = _params(cfg)
+    D = cfg.width
+    half = D // 2
+    i, j = half - 1, 3
+    p.w_t1[:] = 0
+    p.w_t1[j, i] = 1.0
+    p.b_t1[:] = np.linspace(-0.5, 0.7, D)
+    p.w_t2[:] = np.eye(D)
+    p.b_t2[:] = 0
+    for t, e_i in ((1.0, 1.0), (0.0, 0.0), (0.5, math.sin(math.pi / 4))):
+        c = oracle.time_conditioning(t, p)
+        assert c[j] == pytest.approx(_swish(_swish(e_i + p.b_t1[j])), abs=1e-14)
+        others = [m for m in range(D) if m != j]
+        want = np.array([_swish(_swish(p.b_t1[m])) for m in others])
+        np.testing.assert_allclose(c[others], want, rtol=0, atol=1e-14)
+
+
+def test_time_conditioning_second_layer_closed_form():
+    # W_t1 = 0 makes the hidden layer z = swish(b_t1), a known vector; a W_t2
+    # with one 1 at [a][b] (a != b) gives c_a = swish(z_b + b2_a) and
+    # c_m = swish(b2_m) elsewhere, so a transposed W_t2 or a dropped outer
+    # swish fails.
+    cfg = _tiny()
+    p = _params(cfg)
+    D = cfg.width
+    a, b = 10, 200
+    p.w_t1[:] = 0
+    p.b_t1[:] = np.linspace(-2.0, 3.0, D)
+    p.w_t2[:] = 0
+    p.w_t2[a, b] = 1.0
+    p.b_t2[:] = np.linspace(0.4, -0.3, D)
+    c = oracle.time_conditioning(0.25, p)
+    z_b = _swish(p.b_t1[b])
+    assert c[a] == pytest.approx(_swish(z_b + p.b_t2[a]), abs=1e-14)
+    others = [m for m in range(D) if m != a]
+    np.testing.assert_allclose(c[others], [_swish(p.b_t2[m]) for m in others], rtol=0, atol=1e-14)
+
+
+def test_time_conditioning_and_tables_against_library():
+    # Random non-zero weights (large enough that both swishes are non-linear),
+    # several timesteps: PyTorch float64 linear / silu over an embedding built
+    # from the closed form, then the modulation rows through linear again.
+    cfg = _tiny()
+    p = _params(cfg)
+    g = np.random.default_rng(11)
+    D, L = cfg.width, cfg.layers
+    p.w_t1[:] = g.standard_normal((D, D)) * 0.2
+    p.w_t2[:] = g.standard_normal((D, D)) * 0.2
+    p.b_t1[:] = g.standard_normal(D) * 0.5
+    p.b_t2[:] = g.standard_normal(D) * 0.5
+    half = D // 2
+    period = 4e-3 * (4.0 / 4e-3) ** (torch.arange(half, dtype=torch.float64) / (half - 1))
+    grid = [1.0, 0.7, 0.3, 0.05, 0.0]
+    tabs = oracle.modulation_tables(grid, p)
+    T = lambda a: torch.tensor(a, dtype=torch.float64)  # noqa: E731
+    for k, t in enumerate(grid):
+        ang = 2 * math.pi * t / period
+        e = torch.cat([torch.sin(ang), torch.cos(ang)])
+        c = Fn.silu(Fn.linear(Fn.silu(Fn.linear(e, T(p.w_t1), T(p.b_t1))), T(p.w_t2), T(p.b_t2)))
+        # the fast embedding channels reach angles of ~1.6e3 rad: allow round-off there
+        np.testing.assert_allclose(oracle.time_conditioning(t, p), c.numpy(), rtol=1e-10, atol=1e-12)
+        if k == len(grid) - 1:
+            break
+        m = Fn.linear(c, T(p.w_mod.reshape(-1, D)), T(p.b_mod.reshape(-1))).reshape(L, 2, 3, D).numpy()
+        f = Fn.linear(c, T(p.w_modf), T(p.b_modf)).numpy()
+        tab = tabs[k]
+        np.testing.assert_allclose(tab.scale, m[:, :, 0], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(tab.shift, m[:, :, 1], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(tab.gate, m[:, :, 2], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(tab.scale_f, f[:D], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(tab.shift_f, f[D:], rtol=1e-10, atol=1e-12)
+        assert tab.dt == pytest.approx(grid[k + 1] - t, abs=1e-15)
+
+
 def test_tables_chunk_order_and_dt():
     cfg = _tiny()
     p = _params(cfg)
