@@ -12,6 +12,7 @@ the tests under ``tests/test_oracle_*.py``.
 from .expert import (  # noqa: F401
     sinusoidal_embedding, swish, time_conditioning, modulation_tables,
     ada_rms_norm, gelu_tanh, attention, expert_layer, velocity, denoise,
-    denoise_row, brute_force_denoise_row, prefix_stack_kv, OracleParams,
+    denoise_row, brute_force_denoise_row, prefix_stack_kv, prefix_stack_hidden,
+    prefix_kv_from_hidden, rope, OracleParams,
     params_from_weights,
 )

@@ -125,6 +125,28 @@ def gelu_tanh(x: np.ndarray) -> np.ndarray:
     return 0.5 * x * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)))
 
 
+def rope(x: np.ndarray, positions: np.ndarray, base: float) -> np.ndarray:
+    """Rotary position embedding of per-head vectors x [T][H][d] at integer
+    positions [T].
+
+    Reading (the pages do not print it; the vla.cpp abstract on page 1 only
+    warns that positional-index precision matters): the rotate-half form, in
+    which channel i < d/2 pairs with channel i + d/2 and the pair turns by
+    angle pos * base^(-2i/d):
+      out_i       = x_i cos(a_i) - x_{i+d/2} sin(a_i)
+      out_{i+d/2} = x_{i+d/2} cos(a_i) + x_i sin(a_i).
+    Angles are formed in float64 from the integer positions.
+    """
+    d = x.shape[-1]
+    half = d // 2
+    inv_freq = base ** (-2.0 * np.arange(half, dtype=F64) / d)          # [half]
+    ang = np.asarray(positions, dtype=F64)[:, None] * inv_freq[None, :]  # [T][half]
+    c = np.cos(ang)[:, None, :]
+    sn = np.sin(ang)[:, None, :]
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * sn, x2 * c + x1 * sn], axis=-1)
+
+
 def attention(q: np.ndarray, keys: np.ndarray, values: np.ndarray,
               mask: Optional[np.ndarray] = None, return_probs: bool = False):
     """Grouped-query attention, one request.
@@ -181,6 +203,7 @@ class OracleParams:
     w_gate: List[np.ndarray]
     w_up: List[np.ndarray]
     w_down: List[np.ndarray]
+    rope_base: float = 0.0  # 0: no rotary embedding; else its base (positions P_b + i)
 
 
 def params_from_weights(cfg, W) -> OracleParams:
@@ -205,7 +228,8 @@ def params_from_weights(cfg, W) -> OracleParams:
         b_modf=f(W["b_modf"]),
         w_qkv=[mat("w_qkv", l) for l in range(L)], w_o=[mat("w_o", l) for l in range(L)],
         w_gate=[mat("w_gate", l) for l in range(L)], w_up=[mat("w_up", l) for l in range(L)],
-        w_down=[mat("w_down", l) for l in range(L)])
+        w_down=[mat("w_down", l) for l in range(L)],
+        rope_base=float(getattr(cfg, "rope_base", 0.0)))
 
 
 def expert_layer(h: np.ndarray, l: int, tab: StepTables, p: OracleParams,
@@ -218,7 +242,9 @@ def expert_layer(h: np.ndarray, l: int, tab: StepTables, p: OracleParams,
     to all H action keys (no mask inside the action block; reading),
     h += gate_a * (o W_o^T).  MLP block: y = adaRMSNorm(h; MLP modulation),
     h += gate_m * ((gelu_tanh(y W_gate^T) * (y W_up^T)) W_down^T).
-    Attention and MLP carry no biases (reading).
+    Attention and MLP carry no biases (reading).  With p.rope_base set, q and
+    the action keys are rotated at positions P + i (the cached prefix keys
+    already carry their own positions 0..P-1).
     """
     H = h.shape[0]
     Hq, Hkv, d = p.Hq, p.Hkv, p.d
@@ -227,6 +253,11 @@ def expert_layer(h: np.ndarray, l: int, tab: StepTables, p: OracleParams,
     q = qkv[:, :Hq * d].reshape(H, Hq, d)
     k = qkv[:, Hq * d:(Hq + Hkv) * d].reshape(H, Hkv, d)
     v = qkv[:, (Hq + Hkv) * d:].reshape(H, Hkv, d)
+    if p.rope_base:
+        # action token i of a request with a P-token prefix sits at position P + i
+        pos = k_pre.shape[0] + np.arange(H)
+        q = rope(q, pos, p.rope_base)
+        k = rope(k, pos, p.rope_base)
     keys = np.concatenate([k_pre, k], axis=0)
     vals = np.concatenate([v_pre, v], axis=0)
     if trace is not None:
@@ -300,24 +331,69 @@ def _rms(h, eps):
 
 
 def prefix_stack_kv(z: np.ndarray, ps: PrefixStack, p: OracleParams):
-    """Run the prefix stack alone on prefix hidden states z [P][D] and return
-    its per-layer K/V (lists of [P][Hkv][d]): the cache a runner keeps."""
+    """Run the prefix stack alone on prefix hidden states z [P][Dp] and return
+    its per-layer K/V (lists of [P][Hkv][d]): the cache a runner keeps.  The
+    stack's width Dp is z's; with p.rope_base its queries and keys sit at
+    positions 0..P-1."""
+    ks, vs, _ = _prefix_stack_run(z, ps, p)
+    return ks, vs
+
+
+def prefix_stack_hidden(z: np.ndarray, ps: PrefixStack, p: OracleParams) -> List[np.ndarray]:
+    """The input hidden state of every layer of the prefix stack ([P][Dp] per
+    layer; layer 0's is z): what a runner holds when it produces the cache
+    layer by layer."""
+    return _prefix_stack_run(z, ps, p)[2]
+
+
+def _prefix_stack_run(z, ps, p):
     P = z.shape[0]
     Hq, Hkv, d = p.Hq, p.Hkv, p.d
-    ks, vs = [], []
-    h = z.copy()
+    ks, vs, hs = [], [], []
+    h = np.asarray(z, dtype=F64).copy()
+    pos = np.arange(P)
     for l in range(p.L):
+        hs.append(h.copy())
         y = _rms(h, p.eps)
         qkv = y @ ps.w_qkv[l].T
         q = qkv[:, :Hq * d].reshape(P, Hq, d)
         k = qkv[:, Hq * d:(Hq + Hkv) * d].reshape(P, Hkv, d)
         v = qkv[:, (Hq + Hkv) * d:].reshape(P, Hkv, d)
+        if p.rope_base:
+            q = rope(q, pos, p.rope_base)
+            k = rope(k, pos, p.rope_base)
         ks.append(k)
         vs.append(v)
         o = attention(q, k, v)
         h = h + o.reshape(P, Hq * d) @ ps.w_o[l].T
         y = _rms(h, p.eps)
         h = h + (gelu_tanh(y @ ps.w_gate[l].T) * (y @ ps.w_up[l].T)) @ ps.w_down[l].T
+    return ks, vs, hs
+
+
+def prefix_kv_from_hidden(hs: Sequence[np.ndarray], w_kv: Sequence[np.ndarray], p: OracleParams):
+    """The prefix production step: per layer l, the cached keys and values of
+    a P-token prefix from that layer's input hidden state hs[l] [P][Dp].
+
+    y = h / sqrt(mean(h^2) + eps) (a plain RMSNorm, no gain); [k | v] = y W_kv[l]^T
+    where W_kv[l] [2 Hkv d][Dp] holds the layer's key rows then its value rows;
+    with p.rope_base the keys are rotated at positions 0..P-1 (the prefix comes
+    first in the joint sequence).  Returns lists of [P][Hkv][d].  PhyAI report
+    Sec. 5.1: the prefix is computed once per observation and its per-layer K/V
+    is cached."""
+    Hkv, d = p.Hkv, p.d
+    ks, vs = [], []
+    for l, h in enumerate(hs):
+        h = np.asarray(h, dtype=F64)
+        P = h.shape[0]
+        y = h / np.sqrt(np.mean(h * h, axis=-1, keepdims=True) + p.eps)
+        kv = y @ np.asarray(w_kv[l], dtype=F64).T
+        k = kv[:, :Hkv * d].reshape(P, Hkv, d)
+        v = kv[:, Hkv * d:].reshape(P, Hkv, d)
+        if p.rope_base:
+            k = rope(k, np.arange(P), p.rope_base)
+        ks.append(k)
+        vs.append(v)
     return ks, vs
 
 
@@ -325,8 +401,10 @@ def brute_force_denoise_row(x0: np.ndarray, t_grid: Sequence[float], p: OraclePa
                             z: np.ndarray, ps: PrefixStack) -> np.ndarray:
     """Every Euler step recomputes the joint [prefix | action] sequence under a
     block-causal mask: prefix tokens see only prefix tokens, action tokens see
-    everything.  Prefix tokens use the prefix stack's weights, action tokens
-    the expert's.  No cache is kept between steps."""
+    everything.  Prefix tokens use the prefix stack's weights (width Dp, z's),
+    action tokens the expert's.  With p.rope_base every query and key is
+    rotated at its position in the joint sequence.  No cache is kept between
+    steps."""
     tables = modulation_tables(t_grid, p)
     Hq, Hkv, d = p.Hq, p.Hkv, p.d
     P = z.shape[0]
@@ -346,6 +424,9 @@ def brute_force_denoise_row(x0: np.ndarray, t_grid: Sequence[float], p: OraclePa
             q = qkv[:, :Hq * d].reshape(S, Hq, d)
             k = qkv[:, Hq * d:(Hq + Hkv) * d].reshape(S, Hkv, d)
             v = qkv[:, (Hq + Hkv) * d:].reshape(S, Hkv, d)
+            if p.rope_base:
+                q = rope(q, np.arange(S), p.rope_base)
+                k = rope(k, np.arange(S), p.rope_base)
             o = attention(q, k, v, mask=mask).reshape(S, Hq * d)
             hp = hp + o[:P] @ ps.w_o[l].T
             ha = ha + tab.gate[l, 0] * (o[P:] @ p.w_o[l].T)

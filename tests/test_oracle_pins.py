@@ -478,3 +478,121 @@ def test_attention_rows_sum_to_one_in_trace():
     for pr in tr["probs"]:
         assert pr.shape == (cfg.n_q_heads, cfg.chunk, cfg.prefix + cfg.chunk)
         np.testing.assert_allclose(pr.sum(-1), 1.0, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# Rotary position embedding (vla.cpp abstract, page 1: positional-index
+# precision matters) and the prefix production step
+# --------------------------------------------------------------------------
+
+def test_rope_closed_forms():
+    base = 10000.0
+    g = np.random.default_rng(21)
+    x = g.standard_normal((5, 3, 64))
+    # position 0 is the identity
+    np.testing.assert_array_equal(oracle.rope(x, np.zeros(5, int), base), x)
+    # d = 2: one pair turned by the plain angle pos (base^0 = 1)
+    v = np.array([[[0.3, -1.2]]])
+    for pos in (1, 7, 1000):
+        got = oracle.rope(v, np.array([pos]), base)[0, 0]
+        c, s_ = math.cos(pos), math.sin(pos)
+        np.testing.assert_allclose(got, [0.3 * c + 1.2 * s_, -1.2 * c + 0.3 * s_], rtol=0, atol=1e-13)
+    # a one-hot channel i at position p lands on (cos, sin) of p * base^(-2i/d) in channels i, i + d/2
+    d = 64
+    for i in (0, 5, 31):
+        e = np.zeros((1, 1, d))
+        e[0, 0, i] = 1.0
+        ang = 37 * math.pow(base, -2.0 * i / d)
+        out = oracle.rope(e, np.array([37]), base)[0, 0]
+        want = np.zeros(d)
+        want[i] = math.cos(ang)
+        want[i + d // 2] = math.sin(ang)
+        np.testing.assert_allclose(out, want, rtol=0, atol=1e-13)
+
+
+def test_rope_complex_rotation_norm_and_relative_positions():
+    base = 10000.0
+    g = np.random.default_rng(22)
+    d = 256
+    x = g.standard_normal((7, 2, d))
+    pos = np.array([0, 1, 5, 50, 968, 1017, 3])
+    # pairs (i, i + d/2) as complex numbers, multiplied by e^{j a}
+    z = x[..., :d // 2] + 1j * x[..., d // 2:]
+    a = pos[:, None, None] * base ** (-np.arange(d // 2) * 2.0 / d)[None, None, :]
+    zr = z * np.exp(1j * a)
+    out = oracle.rope(x, pos, base)
+    np.testing.assert_allclose(out, np.concatenate([zr.real, zr.imag], axis=-1), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(np.linalg.norm(out, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-13)
+    # q . k depends only on the position difference
+    q, k = g.standard_normal((1, 1, d)), g.standard_normal((1, 1, d))
+    def dot(m, n):
+        return float(np.sum(oracle.rope(q, np.array([m]), base) * oracle.rope(k, np.array([n]), base)))
+    for m, n, sh in ((3, 10, 100), (968, 0, 37), (50, 50, 900)):
+        assert dot(m, n) == pytest.approx(dot(m + sh, n + sh), abs=1e-10)
+    assert abs(dot(3, 10) - dot(3, 11)) > 1e-6
+
+
+def _prefix_stack_w(cfg, seed, Dp=None):
+    g = np.random.default_rng(seed)
+    D = cfg.width if Dp is None else Dp
+    L, F = cfg.layers, cfg.mlp_dim
+    n = lambda *s: g.standard_normal(s) * 0.05  # noqa: E731
+    return PrefixStack(w_qkv=[n(cfg.qkv_dim, D) for _ in range(L)], w_o=[n(D, cfg.attn_dim) for _ in range(L)],
+                       w_gate=[n(F, D) for _ in range(L)], w_up=[n(F, D) for _ in range(L)],
+                       w_down=[n(D, F) for _ in range(L)])
+
+
+@pytest.mark.parametrize("P,Hkv,Dp", [(64, 1, None), (13, 2, None), (0, 1, None), (40, 1, 384)])
+def test_cached_prefix_equals_brute_force_with_rope(P, Hkv, Dp):
+    # every query and key rotated at its place in the joint [prefix | action]
+    # sequence: the cached path must rotate action tokens at P_b + i
+    cfg = _tiny(n_kv_heads=Hkv)
+    p = _params(cfg)
+    p.rope_base = 10000.0
+    p.b_mod *= 5.0
+    ps = _prefix_stack_w(cfg, 99, Dp)
+    z = np.random.default_rng(7).standard_normal((P, cfg.width if Dp is None else Dp))
+    x0 = wl.make_noise(cfg).astype(F64)[0]
+    grid = wl.uniform_grid(cfg.steps)
+    if P > 0:
+        ks, vs = oracle.prefix_stack_kv(z, ps, p)
+    else:
+        ks = [np.zeros((0, Hkv, cfg.head_dim))] * cfg.layers
+        vs = ks
+    cached = oracle.denoise_row(x0, oracle.modulation_tables(grid, p), p, ks, vs)
+    brute = oracle.brute_force_denoise_row(x0, grid, p, z, ps)
+    np.testing.assert_allclose(cached, brute, rtol=0, atol=1e-11)
+    # the rotation matters for the result
+    p0 = oracle.params_from_weights(cfg, wl.make_weights(cfg))
+    p0.b_mod *= 5.0
+    if P > 0:
+        ks0, vs0 = oracle.prefix_stack_kv(z, ps, p0)
+        plain = oracle.denoise_row(x0, oracle.modulation_tables(grid, p0), p0, ks0, vs0)
+        assert np.max(np.abs(plain - cached)) > 1e-6
+
+
+@pytest.mark.parametrize("rope_base,Dp", [(0.0, None), (10000.0, None), (10000.0, 384)])
+def test_prefix_kv_from_hidden_matches_prefix_stack(rope_base, Dp):
+    # the production step (norm + key/value rows + rotation of the keys) gives
+    # the cache the whole stack gives, layer by layer
+    cfg = _tiny(n_kv_heads=2)
+    p = _params(cfg)
+    p.rope_base = rope_base
+    ps = _prefix_stack_w(cfg, 5, Dp)
+    P = 30
+    z = np.random.default_rng(8).standard_normal((P, cfg.width if Dp is None else Dp)) * 2.0
+    ks, vs = oracle.prefix_stack_kv(z, ps, p)
+    hs = oracle.prefix_stack_hidden(z, ps, p)
+    assert len(hs) == cfg.layers and np.array_equal(hs[0], z)
+    qd = cfg.n_q_heads * cfg.head_dim
+    w_kv = [w[qd:] for w in ps.w_qkv]
+    k2, v2 = oracle.prefix_kv_from_hidden(hs, w_kv, p)
+    for l in range(cfg.layers):
+        np.testing.assert_allclose(k2[l], ks[l], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(v2[l], vs[l], rtol=0, atol=1e-12)
+    # against a library restatement for one layer: torch rms_norm, then linear
+    y = Fn.rms_norm(torch.tensor(hs[1]), (hs[1].shape[1],), eps=p.eps)
+    kv = Fn.linear(y, torch.tensor(w_kv[1])).numpy()
+    np.testing.assert_allclose(v2[1].reshape(P, -1), kv[:, 2 * cfg.head_dim:], rtol=1e-12, atol=1e-13)
+    if not rope_base:
+        np.testing.assert_allclose(k2[1].reshape(P, -1), kv[:, :2 * cfg.head_dim], rtol=1e-12, atol=1e-13)
