@@ -232,7 +232,12 @@ def run_reference(args, cfg):
     value = 1.0 / chunk_s                    # rows are independent: chunks/s
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "chunks/s", "n_gpus": ws,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": chunk_s * 1e3 * cfg.batch,
+        "steps": args.steps, "warmup": args.warmup,
+        # what one timed step is: one Euler step of one request
+        "ms_per_step": t_euler * 1e3,
+        "step": "one Euler step of one request (the oracle's unit of work)",
+        "chunk_ms_extrapolated": chunk_s * 1e3,
+        "batch_ms_extrapolated": chunk_s * 1e3 * cfg.batch,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(cfg),
         "cpu_baseline": {"value": value, "unit": "chunks/s", "cores": blas_threads(), "kind": "oracle",
@@ -291,6 +296,30 @@ def timed(fn, steps, warmup, stream, barrier):
     return e0.elapsed_time(e1) / steps
 
 
+def profile_classes(ex, nd, od, stream, args):
+    """Live per-kernel timing: the same loop with CUDA events around every
+    launch (PAE_OPT_PROFILE), a few calls, per class the mean device time per
+    launch, the launches per call and the time per call."""
+    import flow_matching_action_pi0_b200 as fm
+    ex.set_option(fm.PAE_OPT_PROFILE, (1 << len(fm.KERNEL_CLASSES)) - 1)
+    n_prof = max(3, min(args.steps, 10))
+    for _ in range(2):
+        ex.denoise(nd, od, stream)
+    stream.synchronize()
+    tot = {c: 0.0 for c in fm.KERNEL_CLASSES}
+    cnt = {c: 0 for c in fm.KERNEL_CLASSES}
+    for _ in range(n_prof):
+        ex.denoise(nd, od, stream)
+        stream.synchronize()
+        for i, c in enumerate(fm.KERNEL_CLASSES):
+            t, n = ex.profile_read(i)
+            tot[c] += t
+            cnt[c] += n
+    ex.set_option(fm.PAE_OPT_PROFILE, 0)
+    return {c: {"ms_per_launch": (tot[c] / cnt[c]) if cnt[c] else 0.0, "launches_per_step": cnt[c] // n_prof,
+                "ms_per_step": tot[c] / n_prof} for c in fm.KERNEL_CLASSES}
+
+
 def measure(cfg, W, batch, args, stream, barrier, maxr, lens=None, with_e2e=True, gpu_index=0):
     import torch
     import flow_matching_action_pi0_b200 as fm
@@ -324,58 +353,72 @@ def measure(cfg, W, batch, args, stream, barrier, maxr, lens=None, with_e2e=True
             wall = (time.perf_counter() - t0) / args.steps
             res["e2e_ms"] = maxr(wall * 1e3)
             res["io_bytes"] = int(nh.numel() * 4)
-        # live per-kernel timing: the same graph with CUDA events around every launch
-        ex.set_option(fm.PAE_OPT_PROFILE, (1 << len(fm.KERNEL_CLASSES)) - 1)
-        n_prof = max(3, min(args.steps, 10))
-        for _ in range(2):
-            ex.denoise(nd, od, stream)
-        torch.cuda.synchronize()
-        tot = {c: 0.0 for c in fm.KERNEL_CLASSES}
-        cnt = {c: 0 for c in fm.KERNEL_CLASSES}
-        for _ in range(n_prof):
-            ex.denoise(nd, od, stream)
-            stream.synchronize()
-            for i, c in enumerate(fm.KERNEL_CLASSES):
-                t, n = ex.profile_read(i)
-                tot[c] += t
-                cnt[c] += n
-        ex.set_option(fm.PAE_OPT_PROFILE, 0)
-        res["kernels"] = {c: {"ms_per_launch": (tot[c] / cnt[c]) if cnt[c] else 0.0,
-                              "launches_per_step": cnt[c] // n_prof,
-                              "ms_per_step": tot[c] / n_prof} for c in fm.KERNEL_CLASSES}
+        res["kernels"] = profile_classes(ex, nd, od, stream, args)
     res["ex"] = ex
     res["ks"], res["vs"] = ks, vs
     res["noise"] = noise
     return res
 
 
+def class_fractions(per_c, dur_ms, peaks):
+    """Both roofline fractions of one kernel class from its algorithmic bytes and
+    FLOPs per launch and its measured duration per launch."""
+    if dur_ms <= 0:
+        return None
+    dur = dur_ms * 1e-3
+    gbs = per_c["bytes"] / dur / 1e9
+    tfs = per_c["flops"] / dur / 1e12
+    ridge = (peaks["bf16_tflops_sustained"] * 1e12) / (peaks["hbm_gbs"] * 1e9)
+    return {"bound": "hbm" if per_c["flops"] / max(per_c["bytes"], 1) < ridge else "tensor",
+            "ms_per_launch": dur_ms, "algorithmic_bytes_per_launch": per_c["bytes"],
+            "algorithmic_flops_per_launch": per_c["flops"], "achieved_gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+            "achieved_tflops": tfs, "frac_tensor": tfs / peaks["bf16_tflops_sustained"]}
+
+
 def roofline_for(cfg, batch, res, peaks, peak_kind, lens):
+    """Roofline block for the kernel class that sets the bound of the loop.
+
+    The loop is HBM-bound when its algorithmic bytes take longer at the HBM
+    peak than its FLOPs at the tensor peak (batch 1); the class reported is
+    then the one that moves the most bytes per Euler step (the gate/up
+    projection).  Otherwise (batch 32, ragged 16) it is the class with the
+    largest share of the measured step time.  Per-class durations come from
+    CUDA events around every launch of the same loop; those events serialise
+    the launches (no programmatic overlap), so each duration is an upper bound
+    and each achieved figure a lower bound."""
     per, step = algorithmic(cfg, batch, lens)
     ks = res["kernels"]
     total = sum(v["ms_per_step"] for v in ks.values()) or 1.0
-    dom = max((c for c in per), key=lambda c: ks[c]["ms_per_step"])
-    dur_s = ks[dom]["ms_per_launch"] * 1e-3
-    hbm_bound = per[dom]["flops"] / max(per[dom]["bytes"], 1) < (peaks["bf16_tflops_sustained"] * 1e12) / (
-        peaks["hbm_gbs"] * 1e9)
-    if hbm_bound:
-        ach = per[dom]["bytes"] / dur_s / 1e9
-        peak = peaks["hbm_gbs"]
-        rl = {"bound": "hbm", "unit": "GB/s", "algorithmic_bytes_per_launch": per[dom]["bytes"]}
-    else:
-        ach = per[dom]["flops"] / dur_s / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        rl = {"bound": "tensor", "unit": "TFLOP/s", "algorithmic_flops_per_launch": per[dom]["flops"]}
-    rl.update({"kernel": dom, "achieved": ach, "peak": peak, "frac": ach / peak,
-               "peak_source": f"{peak_kind} ({'hbm_gbs' if hbm_bound else 'bf16_tflops_sustained'})",
-               "ms_per_launch": ks[dom]["ms_per_launch"], "share_of_step": ks[dom]["ms_per_step"] / total,
-               "traffic": ncu_traffic(cfg.name if batch == cfg.batch else f"{cfg.name}@{batch}", dom)})
-    # whole loop against the HBM and tensor rooflines
-    t_step = res["ms_per_step"] * 1e-3 / cfg.steps
     hbm_t = step["bytes"] / (peaks["hbm_gbs"] * 1e9)
     tc_t = step["flops"] / (peaks["bf16_tflops_sustained"] * 1e12)
+    timed_classes = [c for c in per if ks.get(c, {}).get("launches_per_step", 0) > 0]
+    if not timed_classes:  # one persistent launch: the whole call is the kernel
+        timed_classes = ["persistent"]
+    if hbm_t >= tc_t:
+        dom = max(timed_classes, key=lambda c: per[c]["bytes"] * ks[c]["launches_per_step"])
+    else:
+        dom = max(timed_classes, key=lambda c: ks[c]["ms_per_step"])
+    fr = class_fractions(per[dom], ks[dom]["ms_per_launch"], peaks)
+    hbm_bound = fr["bound"] == "hbm"
+    if hbm_bound:
+        rl = {"bound": "hbm", "unit": "GB/s", "achieved": fr["achieved_gbs"], "peak": peaks["hbm_gbs"],
+              "frac": fr["frac_hbm"]}
+    else:
+        rl = {"bound": "tensor", "unit": "TFLOP/s", "achieved": fr["achieved_tflops"],
+              "peak": peaks["bf16_tflops_sustained"], "frac": fr["frac_tensor"]}
+    rl.update({"kernel": dom, "algorithmic_bytes_per_launch": per[dom]["bytes"],
+               "algorithmic_flops_per_launch": per[dom]["flops"],
+               "peak_source": f"{peak_kind} ({'hbm_gbs' if hbm_bound else 'bf16_tflops_sustained'})",
+               "ms_per_launch": ks[dom]["ms_per_launch"], "share_of_step": ks[dom]["ms_per_step"] / total,
+               "timing": "CUDA events around each launch (serialised; duration is an upper bound)",
+               "traffic": ncu_traffic(cfg.name if batch == cfg.batch else f"{cfg.name}@{batch}", dom)})
+    rl["per_class"] = {c: class_fractions(per[c], ks[c]["ms_per_launch"], peaks) for c in timed_classes}
+    # whole loop against the HBM and tensor rooflines
+    t_step = res["ms_per_step"] * 1e-3 / cfg.steps
     loop = {"euler_step_us": t_step * 1e6, "bytes_per_euler_step": step["bytes"],
             "flops_per_euler_step": step["flops"], "hbm_roofline_us": hbm_t * 1e6,
             "tensor_roofline_us": tc_t * 1e6, "frac_of_roofline": max(hbm_t, tc_t) / t_step,
+            "frac_hbm": hbm_t / t_step, "frac_tensor": tc_t / t_step,
             "achieved_gbs": step["bytes"] / t_step / 1e9, "achieved_tflops": step["flops"] / t_step / 1e12}
     shares = {c: ks[c]["ms_per_step"] / total for c in ks}
     return rl, loop, shares
@@ -454,15 +497,24 @@ def measure_ragged(args, stream, barrier, maxr, ws, gpu_index):
         flip[0] += 1
         ex.denoise(nd, od, stream)
 
+    peaks, peak_kind = load_peaks()
     with torch.cuda.stream(stream):
+        clk = ClockSampler(gpu_index).start()
         ms = maxr(timed(step, args.steps, args.warmup, stream, barrier))
         ms_loop = maxr(timed(lambda: ex.denoise(nd, od, stream), args.steps, args.warmup, stream, barrier))
-    per, st = algorithmic(cfg, cfg.batch, lens)
+        clocks = clk.stop()
+        kernels = profile_classes(ex, nd, od, stream, args)
     ex.close()
+    # rooflines of the denoise loop itself (cached rows only: the set_prefix
+    # copies are not loop work)
+    rl, loop, shares = roofline_for(cfg, cfg.batch, {"kernels": kernels, "ms_per_step": ms_loop}, peaks, peak_kind,
+                                    lens)
     return {"value": ws * cfg.batch / (ms * 1e-3), "unit": "chunks/s", "ms_per_step": ms,
-            "ms_per_step_cached_only": ms_loop, "prefix_lengths": lens,
-            "loop_roofline": {"bytes_per_euler_step": st["bytes"], "flops_per_euler_step": st["flops"]},
-            "note": "each step: 8 fresh set_prefix calls (new observations) + 8 cached rows + pae_denoise"}
+            "ms_per_step_cached_only": ms_loop, "prefix_lengths": lens, "roofline": rl, "loop_roofline": loop,
+            "kernel_shares": shares, "clocks": clocks,
+            "kernels_ms_per_launch": {c: v["ms_per_launch"] for c, v in kernels.items()},
+            "note": "each step: 8 fresh set_prefix calls (new observations) + 8 cached rows + pae_denoise; "
+                    "rooflines are for the loop alone (ms_per_step_cached_only)"}
 
 
 def measure_persistent(cfg, W, args, stream, barrier, maxr, ws):

@@ -5,7 +5,8 @@ kernels behind the C ABI.  PyTorch supplies device memory and streams.  If the
 library has not been built this module raises on first use; there is no
 fallback path.
 
-Functions keep the C names (pae_create, pae_set_prefix, pae_precompute_tables,
+Functions keep the C names (pae_create, pae_set_prefix, pae_set_prefix_hidden,
+pae_precompute_tables,
 pae_denoise, pae_denoise_host, pae_denoise_steps, pae_sync, ...).  The
 ActionExpert class wraps a context for convenience.
 """
@@ -31,7 +32,7 @@ STATUS_NAMES = {0: "PAE_OK", 1: "PAE_ERR_ARG", 2: "PAE_ERR_STATE", 3: "PAE_ERR_C
                 5: "PAE_ERR_TIMEOUT", 6: "PAE_ERR_UNSUPPORTED"}
 
 # Every symbol include/pae.h declares.
-EXPORTS = ("pae_create", "pae_set_prefix", "pae_precompute_tables", "pae_denoise", "pae_denoise_host",
+EXPORTS = ("pae_create", "pae_set_prefix", "pae_set_prefix_hidden", "pae_precompute_tables", "pae_denoise", "pae_denoise_host",
            "pae_denoise_steps", "pae_set_option", "pae_profile_read", "pae_query", "pae_plan_query", "pae_sync",
            "pae_clear_error", "pae_last_error", "pae_debug_copy", "pae_precompute_tables_static",
            "pae_destroy")
@@ -46,7 +47,9 @@ class PaeError(RuntimeError):
 class pae_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "layers", "width", "n_q_heads", "n_kv_heads", "head_dim", "mlp_dim", "action_dim", "chunk",
-        "max_batch", "max_prefix", "group_size", "dtype")] + [("rms_eps", ctypes.c_float)]
+        "max_batch", "max_prefix", "group_size", "dtype")] + [("rms_eps", ctypes.c_float),
+                                                              ("rope_base", ctypes.c_float),
+                                                              ("prefix_width", ctypes.c_int)]
 
 
 _P = ctypes.c_void_p
@@ -57,7 +60,7 @@ class pae_weights(ctypes.Structure):
     _fields_ = [(n, _P) for n in ("w_in", "b_in", "w_out", "b_out", "w_t1", "b_t1", "w_t2", "b_t2",
                                   "w_mod", "b_mod", "w_modf", "b_modf")] + \
                [(n, _PP) for n in ("w_qkv", "w_o", "w_gate", "w_up", "w_down",
-                                   "s_qkv", "s_o", "s_gate", "s_up", "s_down")]
+                                   "s_qkv", "s_o", "s_gate", "s_up", "s_down", "w_prefix_kv")]
 
 
 _lib = None
@@ -75,6 +78,7 @@ def lib() -> ctypes.CDLL:
     sig = {
         "pae_create": (i, [ctypes.POINTER(pae_config), ctypes.POINTER(pae_weights), ctypes.POINTER(v)]),
         "pae_set_prefix": (i, [v, i, vp, vp, i, st]),
+        "pae_set_prefix_hidden": (i, [v, i, vp, i, st]),
         "pae_precompute_tables": (i, [v, ctypes.POINTER(ctypes.c_double), i, st]),
         "pae_denoise": (i, [v, v, v, i, st]),
         "pae_denoise_host": (i, [v, v, v, i, st]),
@@ -128,6 +132,11 @@ def pae_set_prefix(ctx: int, row: int, k_ptrs: Sequence[int], v_ptrs: Sequence[i
     kp, _ka = _ptr_array(k_ptrs)
     vp, _va = _ptr_array(v_ptrs)
     _check(lib().pae_set_prefix(ctx, row, kp, vp, length, _stream(stream)), ctx)
+
+
+def pae_set_prefix_hidden(ctx: int, row: int, h_ptrs: Sequence[int], length: int, stream=None):
+    hp, _ha = _ptr_array(h_ptrs)
+    _check(lib().pae_set_prefix_hidden(ctx, row, hp, length, _stream(stream)), ctx)
 
 
 def pae_precompute_tables(ctx: int, t: Sequence[float], K: int, stream=None):
@@ -207,14 +216,16 @@ DTYPE_CODES = {"fp32": PAE_FP32, "bf16": PAE_BF16, "w4a16": PAE_W4A16}
 
 
 def make_config(layers, width, n_q_heads, n_kv_heads, head_dim, mlp_dim, action_dim, chunk,
-                max_batch, max_prefix, dtype, group_size=128, rms_eps=1e-6) -> pae_config:
+                max_batch, max_prefix, dtype, group_size=128, rms_eps=1e-6, rope_base=0.0,
+                prefix_width=0) -> pae_config:
     c = pae_config()
     for k, v in dict(layers=layers, width=width, n_q_heads=n_q_heads, n_kv_heads=n_kv_heads, head_dim=head_dim,
                      mlp_dim=mlp_dim, action_dim=action_dim, chunk=chunk, max_batch=max_batch,
-                     max_prefix=max_prefix, group_size=group_size).items():
+                     max_prefix=max_prefix, group_size=group_size, prefix_width=prefix_width).items():
         setattr(c, k, int(v))
     c.dtype = DTYPE_CODES[dtype] if isinstance(dtype, str) else int(dtype)
     c.rms_eps = float(rms_eps)
+    c.rope_base = float(rope_base)
     return c
 
 
@@ -253,6 +264,10 @@ class ActionExpert:
     def set_prefix(self, row: int, ks: List, vs: List, length: Optional[int] = None, stream=None):
         n = int(ks[0].shape[0]) if length is None else length
         pae_set_prefix(self.ctx, row, [t.data_ptr() for t in ks], [t.data_ptr() for t in vs], n, stream)
+
+    def set_prefix_hidden(self, row: int, hs: List, length: Optional[int] = None, stream=None):
+        n = int(hs[0].shape[0]) if length is None else length
+        pae_set_prefix_hidden(self.ctx, row, [t.data_ptr() for t in hs], n, stream)
 
     def precompute_tables(self, t: Sequence[float], stream=None):
         pae_precompute_tables(self.ctx, list(t), len(t) - 1, stream)

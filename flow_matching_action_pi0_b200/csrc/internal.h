@@ -20,6 +20,8 @@ struct Shape {
   int group;             // W4A16 group size
   float eps;
   int table_rows;        // (2L*3 + 2) D floats per step
+  int rope;              // 1: q and k heads are rotated (rows stored pair-interleaved)
+  int Dp;                // prefix hidden width (0: no prefix production)
 };
 
 // Where the modulation of one norm sits inside a step's table row.
@@ -63,8 +65,11 @@ cudaError_t launch_transition(const Shape& s, int act_bf16, const TransitionArgs
 cudaError_t launch_norm(const Shape& s, int act_bf16, const float* h, void* y, const float* scale,
                         const float* shift, int M, bool pdl, cudaStream_t st);
 
+// Prefix production: y = h / sqrt(mean(h^2) + eps) per token, [len][Dp] act dtype.
+cudaError_t launch_prefix_norm(int act_bf16, const void* h, void* y, int len, int Dp, float eps, cudaStream_t st);
+
 // --------------------------------------------------------- CUDA-core (fp32)
-enum Epi : int { EPI_QKV = 0, EPI_RESID = 1, EPI_GEGLU = 2 };
+enum Epi : int { EPI_QKV = 0, EPI_RESID = 1, EPI_GEGLU = 2, EPI_PREFIX = 3 };
 
 struct EpiArgs {
   int epi;
@@ -81,6 +86,11 @@ struct EpiArgs {
   int ss_ld;          // token stride of the sum-of-squares slots
   // EPI_GEGLU
   void* u;            // [M][F]
+  // rotary embedding (EPI_QKV, EPI_PREFIX keys): (cos, sin) [Ptot][d/2], null = off
+  const float2* rope_cs;
+  // EPI_PREFIX: token m is prefix position m of request `prefix_row`; keys and
+  // values go to kc / vc of `layer`
+  int prefix_row;
 };
 
 // out-features N (for GEGLU: F, weight rows interleaved in 128-row tiles).

@@ -59,10 +59,25 @@ __global__ void __launch_bounds__(256) k_gemm_f32(const Shape s, const float* __
     }
     __syncthreads();
   }
+  // q/k with rotation and the prefix keys/values go pair by pair: a thread's
+  // four features are two stored pairs (f0 and 4 tx are even)
+  const bool pairs = e.epi == EPI_PREFIX || (e.epi == EPI_QKV && e.rope_cs);
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     const int m = m0 + ty * 2 + i;
     if (m >= e.M) continue;
+    if (pairs) {
+#pragma unroll
+      for (int j = 0; j < 4; j += 2) {
+        const int f = f0 + tx * 4 + j;
+        if (f >= N) continue;
+        if (e.epi == EPI_PREFIX)
+          epi_prefix_pair<float>(s, e, m, f, acc[0][i][j], acc[0][i][j + 1]);
+        else
+          epi_qkv_pair<float>(s, e, m, f, acc[0][i][j], acc[0][i][j + 1]);
+      }
+      continue;
+    }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int f = f0 + tx * 4 + j;

@@ -91,11 +91,64 @@ __device__ __forceinline__ void store16_bf16(bf16* p, const float* v) {
   d[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
+__device__ __forceinline__ void store8_bf16(bf16* p, const float* v) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    w[i] = (uint32_t)__bfloat16_as_ushort(f2bf(v[2 * i])) | ((uint32_t)__bfloat16_as_ushort(f2bf(v[2 * i + 1])) << 16);
+  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Where the head `head` of the q/k block (EPI_QKV: q heads then k heads) or of
+// the prefix keys (EPI_PREFIX) of token m starts, and that token's position.
+template <int EPI>
+__device__ __forceinline__ bf16* rot_head_base(const Shape& s, const EpiArgs& e, int m, int head, int len, int& pos) {
+  if constexpr (EPI == EPI_PREFIX) {
+    pos = m;
+    return static_cast<bf16*>(e.kc) + (((size_t)(e.layer * s.Bmax + e.prefix_row) * s.Hkv + head) * s.Ptot + m) * s.d;
+  } else {
+    const int b = m / s.H, t = m - b * s.H;
+    pos = len + t;
+    if (head < s.Hq) return static_cast<bf16*>(e.q) + ((size_t)(b * s.Hq + head) * s.H + t) * s.d;
+    return static_cast<bf16*>(e.kc) +
+           (((size_t)(e.layer * s.Bmax + b) * s.Hkv + (head - s.Hq)) * s.Ptot + len + t) * s.d;
+  }
+}
+
 // Epilogue of 16 consecutive output features f..f+15 of token m (v holds the
 // accumulators; for GeGLU already gelu(gate) * up).  16 divides head_dim and
-// 128, so the run never crosses a q/k/v head.
+// 128, so the run never crosses a q/k/v head.  Rotated heads: the 16 stored
+// rows are 8 pairs, written to channels i0..i0+7 and i0+d/2..i0+d/2+7.
 template <int EPI>
 __device__ __forceinline__ void epi_vec16(const Shape& s, const EpiArgs& e, int m, int f, const float* v) {
+  if constexpr (EPI == EPI_QKV || EPI == EPI_PREFIX) {
+    const int rot_rows = (EPI == EPI_QKV ? s.Hq + s.Hkv : s.Hkv) * s.d;
+    if (e.rope_cs && f < rot_rows) {
+      const int head = f / s.d, i0 = (f - head * s.d) >> 1;
+      int pos;
+      const int len = EPI == EPI_QKV ? e.lens[m / s.H] : 0;
+      bf16* base = rot_head_base<EPI>(s, e, m, head, len, pos);
+      float lo[8], hi[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        lo[u] = v[2 * u];
+        hi[u] = v[2 * u + 1];
+        rope_turn(e.rope_cs, s.d, pos, i0 + u, lo[u], hi[u]);
+      }
+      store8_bf16(base + i0, lo);
+      store8_bf16(base + i0 + (s.d >> 1), hi);
+      return;
+    }
+  }
+  if constexpr (EPI == EPI_PREFIX) {
+    const int kvd = s.Hkv * s.d;
+    const bool is_v = f >= kvd;
+    const int fk = f - (is_v ? kvd : 0);
+    const int g = fk / s.d, j = fk - g * s.d;
+    const size_t off = (((size_t)(e.layer * s.Bmax + e.prefix_row) * s.Hkv + g) * s.Ptot + m) * s.d + j;
+    store16_bf16(static_cast<bf16*>(is_v ? e.vc : e.kc) + off, v);
+    return;
+  }
   if constexpr (EPI == EPI_RESID) {
     float* hp = e.h + (size_t)m * s.D + f;
 #pragma unroll
@@ -165,6 +218,32 @@ __device__ __forceinline__ void store4_bf16(bf16* p, float x, float y, float z, 
 template <int EPI>
 __device__ __forceinline__ void epi_vec4(const Shape& s, const EpiArgs& e, int m, int f, float4 a0, float4 a1,
                                          float4 h4, float4 g4, int len) {
+  if constexpr (EPI == EPI_QKV || EPI == EPI_PREFIX) {
+    const int rot_rows = (EPI == EPI_QKV ? s.Hq + s.Hkv : s.Hkv) * s.d;
+    if (e.rope_cs && f < rot_rows) {
+      // two stored pairs -> channels i0, i0 + 1 and i0 + d/2, i0 + d/2 + 1
+      const int head = f / s.d, i0 = (f - head * s.d) >> 1;
+      int pos;
+      bf16* base = rot_head_base<EPI>(s, e, m, head, len, pos);
+      rope_turn(e.rope_cs, s.d, pos, i0, a0.x, a0.y);
+      rope_turn(e.rope_cs, s.d, pos, i0 + 1, a0.z, a0.w);
+      const uint32_t lo = (uint32_t)__bfloat16_as_ushort(f2bf(a0.x)) | ((uint32_t)__bfloat16_as_ushort(f2bf(a0.z)) << 16);
+      const uint32_t hi = (uint32_t)__bfloat16_as_ushort(f2bf(a0.y)) | ((uint32_t)__bfloat16_as_ushort(f2bf(a0.w)) << 16);
+      *reinterpret_cast<uint32_t*>(base + i0) = lo;
+      *reinterpret_cast<uint32_t*>(base + i0 + (s.d >> 1)) = hi;
+      return;
+    }
+  }
+  if constexpr (EPI == EPI_PREFIX) {
+    const int kvd = s.Hkv * s.d;
+    const bool is_v = f >= kvd;
+    const int fk = f - (is_v ? kvd : 0);
+    const int g = fk / s.d, j = fk - g * s.d;
+    store4_bf16(static_cast<bf16*>(is_v ? e.vc : e.kc) +
+                    (((size_t)(e.layer * s.Bmax + e.prefix_row) * s.Hkv + g) * s.Ptot + m) * s.d + j,
+                a0.x, a0.y, a0.z, a0.w);
+    return;
+  }
   if constexpr (EPI == EPI_RESID) {
     h4.x = fmaf(g4.x, a0.x, h4.x);
     h4.y = fmaf(g4.y, a0.y, h4.y);
@@ -593,7 +672,7 @@ __global__ void __launch_bounds__(256, 2)
     const int col0 = threadIdx.x >> lg4;
     const int fv = ntile * 128 + (int)rank * R + 4 * g4;
     const bool fv_ok = fv < a.N;
-    const bool need_len = EPI == EPI_QKV && fv >= s.Hq * s.d;
+    const bool need_len = EPI == EPI_QKV && (fv >= s.Hq * s.d || e.rope_cs);
     float4 hv[UB];
     int lv[UB];
     float4 gv = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -744,6 +823,12 @@ cudaError_t init_all() {
   return e;
 }
 
+cudaError_t init_prefix() {
+  cudaError_t e = init_one<1, EPI_PREFIX, false, false, false>();
+  if (e == cudaSuccess) e = init_one<1, EPI_PREFIX, true, false, false>();
+  return e;
+}
+
 cudaError_t init_norm() {
   cudaError_t e = init_one<1, EPI_QKV, false, false, true>();
   if (e == cudaSuccess) e = init_one<1, EPI_QKV, true, false, true>();
@@ -768,11 +853,16 @@ cudaError_t tc_gemm_init() {
   cudaError_t e = init_all<false>();
   if (e == cudaSuccess) e = init_all<true>();
   if (e == cudaSuccess) e = init_norm();
+  if (e == cudaSuccess) e = init_prefix();
   return e;
 }
 
 cudaError_t launch_tc_gemm(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* tmX, int na, const TcPlan& p,
                            const TcGemmArgs& a, bool pdl, cudaStream_t st) {
+  if (a.e.epi == EPI_PREFIX) {  // prefix production: bf16 weights, keys/values into the slots
+    if (a.scales || a.ss_in || na != 1) return cudaErrorInvalidValue;
+    return launch_one<1, EPI_PREFIX, false, false>(s, tmW, tmX, p, a, pdl, st);
+  }
   if (a.ss_in) {  // adaRMSNorm in the kernel: bf16 weights only, QKV or gate/up
     if (a.scales) return cudaErrorInvalidValue;
     if (na == 2) return launch_one<2, EPI_GEGLU, false, true>(s, tmW, tmX, p, a, pdl, st);

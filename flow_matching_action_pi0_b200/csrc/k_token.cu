@@ -237,7 +237,37 @@ cudaError_t norm_dispatch(const Shape& s, const float* h, TA* y, const float* sc
   return launch_ex(k_norm<TA, 16>, grid, block, 0, st, 1, pdl, s, h, y, scale, shift, M);
 }
 
+// Prefix production, step 1: y = h / sqrt(mean(h^2) + eps) per prefix token
+// (a plain RMSNorm; one warp per token, the sum of squares in fp32 in a fixed
+// lane order).
+template <typename TA>
+__global__ void __launch_bounds__(256) k_prefix_norm(const TA* __restrict__ h, TA* __restrict__ y, int len, int Dp,
+                                                     float eps) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m = blockIdx.x * 8 + warp;
+  if (m >= len) return;
+  const TA* hr = h + (size_t)m * Dp;
+  float ss = 0.f;
+  for (int j = lane; j < Dp; j += 32) {
+    const float v = ld_act<TA>(hr + j);
+    ss = fmaf(v, v, ss);
+  }
+  ss = warp_sum(ss);
+  const float r = rsqrtf(ss / (float)Dp + eps);
+  TA* yr = y + (size_t)m * Dp;
+  for (int j = lane; j < Dp; j += 32) st_act<TA>(yr + j, ld_act<TA>(hr + j) * r);
+}
+
 }  // namespace
+
+cudaError_t launch_prefix_norm(int act_bf16, const void* h, void* y, int len, int Dp, float eps, cudaStream_t st) {
+  const dim3 grid((len + 7) / 8), block(256);
+  if (act_bf16)
+    k_prefix_norm<bf16><<<grid, block, 0, st>>>(static_cast<const bf16*>(h), static_cast<bf16*>(y), len, Dp, eps);
+  else
+    k_prefix_norm<float><<<grid, block, 0, st>>>(static_cast<const float*>(h), static_cast<float*>(y), len, Dp, eps);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_transition(const Shape& s, int act_bf16, const TransitionArgs& a, bool pdl, cudaStream_t st) {
   const size_t smem = (size_t)(s.D + s.A + 32) * sizeof(float);

@@ -11,6 +11,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -20,6 +21,7 @@
 
 #include "pae.h"
 #include "internal.h"
+#include "epilogue.cuh"
 
 using namespace pae;
 
@@ -77,13 +79,27 @@ __global__ void k_transpose(const T* __restrict__ src, T* __restrict__ dst, int 
   }
 }
 
+// Rotary pairing of the q/k block (rows [0, rot_rows), head_dim d): stored row
+// p of a head holds channel rope_channel(p) = p/2 + (p odd) d/2, so the two
+// channels a rotation mixes leave the GEMM side by side.  dst[r] = src[src_row(r)]
+// in units of 2 bytes, `cols` units per row; rows past rot_rows are copied as is.
+__global__ void k_permute_rows(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst, int rows, int cols,
+                               int rot_rows, int d) {
+  const size_t n = (size_t)rows * cols;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const int r = (int)(i / cols), c = (int)(i - (size_t)r * cols);
+    const int sr = r < rot_rows ? (r / d) * d + rope_channel(r % d, d) : r;
+    dst[i] = src[(size_t)sr * cols + c];
+  }
+}
+
 // Packed int4 rows [rows][kbytes] -> the kernels' layout: within every
 // 32-bit word the nibbles of k = 0..7 move to bit positions
 // 0, 16, 4, 20, 8, 24, 12, 28, so that (w >> 4i) & 0x000F000F holds the
 // pair (k = 2i, 2i + 1).  Row r goes to destination row dst_row(r):
 // mode 0 identity, 1 gate rows and 2 up rows of the 128-row interleave.
 __global__ void k_repack_int4(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, int rows, int kbytes,
-                              int mode) {
+                              int mode, int rot_rows, int d) {
   const int words = kbytes / 4;
   const size_t n = (size_t)rows * words;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
@@ -96,7 +112,13 @@ __global__ void k_repack_int4(const uint8_t* __restrict__ src, uint8_t* __restri
       const int pos = (k & 1) ? 16 + 4 * (k >> 1) : 4 * (k >> 1);
       o |= nib << pos;
     }
-    const int dr = mode == 0 ? r : ((r >> 7) * 256 + (r & 127) + (mode == 2 ? 128 : 0));
+    // mode 0 with rotation: source channel j of a q/k head goes to stored row
+    // 2j (j < d/2) or 2(j - d/2) + 1
+    int dr = mode == 0 ? r : ((r >> 7) * 256 + (r & 127) + (mode == 2 ? 128 : 0));
+    if (mode == 0 && r < rot_rows) {
+      const int j = r % d, h2 = d >> 1;
+      dr = (r / d) * d + (j < h2 ? 2 * j : 2 * (j - h2) + 1);
+    }
     reinterpret_cast<uint32_t*>(dst + (size_t)dr * kbytes)[c] = o;
   }
 }
@@ -138,6 +160,13 @@ struct pae_ctx {
   float *emb = nullptr, *zbuf = nullptr, *cbuf = nullptr, *tables = nullptr, *dt = nullptr;
   int K = 0;
   bool tables_ready = false;
+  // rotary embedding: (cos, sin) of position x channel pair, [Ptot][d/2]
+  float2* rope_cs = nullptr;
+  // prefix production: key/value rows per layer [L][2 Hkv d][Dp] (keys paired
+  // like the q/k block when rotating) and the normalised hidden states [Pmax][Dp]
+  void* w_pkv = nullptr;
+  void* ypre = nullptr;
+  CUtensorMap tmWpkv{}, tmYpre{};
   // prefix slots
   void *kc = nullptr, *vc = nullptr;
   int* lens_dev = nullptr;
@@ -390,7 +419,7 @@ AttnPlan plan_attn(const Shape& s, int B) {
 bool plan_persistent(const pae_ctx* ctx, int B, PersistArgs* pa) {
   const Shape& s = ctx->s;
   const int M = B * s.H, n = ctx->ncta;
-  if (!ctx->act_bf16 || ctx->w4 || n < 1 || M > 64 || M > n) return false;
+  if (!ctx->act_bf16 || ctx->w4 || s.rope || n < 1 || M > 64 || M > n) return false;
   if (s.d != 64 && s.d != 128 && s.d != 256) return false;
   if ((size_t)(s.D + s.A) * 4 > 128 * 1024) return false;
   *pa = PersistArgs{};
@@ -637,6 +666,7 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
       e.kc = ctx->kc;
       e.vc = ctx->vc;
       e.lens = ctx->lens_dev;
+      e.rope_cs = ctx->rope_cs;
       {
         ProfScope ps(ctx, PAE_K_QKV, st);
         NormIn nq;
@@ -847,6 +877,8 @@ Shape shape_from_config(const pae_config* cfg) {
   s.group = cfg->group_size;
   s.eps = cfg->rms_eps;
   s.table_rows = (s.L * 2 * 3 + 2) * s.D;
+  s.rope = cfg->rope_base > 0.f ? 1 : 0;
+  s.Dp = cfg->prefix_width;
   return s;
 }
 
@@ -863,6 +895,15 @@ pae_status validate_config(const pae_config* c) {
     return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: at most 16 query heads per KV head");
   if (c->width % 32 != 0 || c->width > 2048)
     return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: width must be a multiple of 32 and at most 2048");
+  if (!(c->rope_base >= 0.f) || c->rope_base > 1e30f)
+    return fail(nullptr, PAE_ERR_ARG, "config: rope_base must be 0 (off) or a finite positive base");
+  if (c->rope_base > 0.f && c->head_dim % 2 != 0)
+    return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: rotary embedding needs an even head_dim");
+  if (c->prefix_width < 0) return fail(nullptr, PAE_ERR_ARG, "config: prefix_width must be >= 0");
+  if (c->prefix_width > 0 && c->dtype != PAE_FP32 &&
+      (c->prefix_width % 64 != 0 || (2 * c->n_kv_heads * c->head_dim) % 128 != 0))
+    return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: bf16 prefix production needs prefix_width % 64 == 0 and "
+                                              "2*n_kv_heads*head_dim % 128 == 0");
   if (c->dtype == PAE_W4A16 && c->group_size != 128)
     return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: W4A16 needs group_size 128");
   if (c->dtype != PAE_FP32) {
@@ -876,6 +917,21 @@ pae_status validate_config(const pae_config* c) {
       return fail(nullptr, PAE_ERR_UNSUPPORTED, "config: chunk <= 256 and max_batch*chunk <= 4096");
   }
   return PAE_OK;
+}
+
+// Launch plan of the prefix production GEMM: 128-token tiles (the height of
+// the normalised-prefix tensor map's box) over `len` tokens, split-K so that
+// output tiles x token tiles x splits fill the SMs.
+TcPlan prefix_plan(const Shape& s, int len) {
+  TcPlan p{};
+  p.tn = 128;
+  p.tok_tiles = (len + 127) / 128;
+  const int nt = (2 * s.Hkv * s.d + 127) / 128, nkb = s.Dp / 64, base = nt * p.tok_tiles;
+  p.splits = 1;
+  for (int sp = 2; sp <= 8; sp *= 2)
+    if (nkb % sp == 0 && base * sp <= 148) p.splits = sp;
+  fit_ring(p, 1, nkb, false, false, 200u * 1024u);
+  return p;
 }
 
 }  // namespace
@@ -999,18 +1055,25 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
   CKC(cudaMemcpyAsync((char*)ctx->b_modall + mod_rows * es, w->b_modf, (size_t)2 * D * es,
                       cudaMemcpyDeviceToDevice, cs));
   for (int l = 0; l < L && ctx->w4; ++l) {
-    auto rep = [&](const void* src, void* dst, int rows, int K, int mode) {
-      k_repack_int4<<<256, 256, 0, cs>>>((const uint8_t*)src, (uint8_t*)dst, rows, K / 2, mode);
+    const int rot_rows = s.rope ? (s.Hq + s.Hkv) * s.d : 0;
+    auto rep = [&](const void* src, void* dst, int rows, int K, int mode, int rot = 0) {
+      k_repack_int4<<<256, 256, 0, cs>>>((const uint8_t*)src, (uint8_t*)dst, rows, K / 2, mode, rot, s.d);
     };
-    rep(w->w_qkv[l], (char*)ctx->q_qkv + (size_t)l * s.qkv_rows * D / 2, s.qkv_rows, D, 0);
+    rep(w->w_qkv[l], (char*)ctx->q_qkv + (size_t)l * s.qkv_rows * D / 2, s.qkv_rows, D, 0, rot_rows);
     rep(w->w_o[l], (char*)ctx->q_o + (size_t)l * D * s.attn_dim / 2, D, s.attn_dim, 0);
     rep(w->w_down[l], (char*)ctx->q_down + (size_t)l * D * F / 2, D, F, 0);
     rep(w->w_gate[l], (char*)ctx->q_gu + (size_t)l * 2 * F * D / 2, F, D, 1);
     rep(w->w_up[l], (char*)ctx->q_gu + (size_t)l * 2 * F * D / 2, F, D, 2);
     CKC(cudaGetLastError());
     const size_t g1 = D / 128, g2 = s.attn_dim / 128, g3 = F / 128;
-    CKC(cudaMemcpyAsync((char*)ctx->sc_qkv + (size_t)l * s.qkv_rows * g1 * 2, w->s_qkv[l], (size_t)s.qkv_rows * g1 * 2,
-                        cudaMemcpyDeviceToDevice, cs));
+    if (s.rope)
+      k_permute_rows<<<64, 256, 0, cs>>>((const uint16_t*)w->s_qkv[l],
+                                         (uint16_t*)((char*)ctx->sc_qkv + (size_t)l * s.qkv_rows * g1 * 2), s.qkv_rows,
+                                         (int)g1, rot_rows, s.d);
+    else
+      CKC(cudaMemcpyAsync((char*)ctx->sc_qkv + (size_t)l * s.qkv_rows * g1 * 2, w->s_qkv[l],
+                          (size_t)s.qkv_rows * g1 * 2, cudaMemcpyDeviceToDevice, cs));
+    CKC(cudaGetLastError());
     CKC(cudaMemcpyAsync((char*)ctx->sc_o + (size_t)l * D * g2 * 2, w->s_o[l], (size_t)D * g2 * 2,
                         cudaMemcpyDeviceToDevice, cs));
     CKC(cudaMemcpyAsync((char*)ctx->sc_down + (size_t)l * D * g3 * 2, w->s_down[l], (size_t)D * g3 * 2,
@@ -1021,8 +1084,14 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
     CKC(cudaMemcpy2DAsync(gu + tile, 2 * tile, w->s_up[l], tile, tile, F / 128, cudaMemcpyDeviceToDevice, cs));
   }
   for (int l = 0; l < L && !ctx->w4; ++l) {
-    CKC(cudaMemcpyAsync((char*)ctx->w_qkv + (size_t)l * s.qkv_rows * D * es, w->w_qkv[l],
-                        (size_t)s.qkv_rows * D * es, cudaMemcpyDeviceToDevice, cs));
+    if (s.rope)
+      k_permute_rows<<<256, 256, 0, cs>>>((const uint16_t*)w->w_qkv[l],
+                                          (uint16_t*)((char*)ctx->w_qkv + (size_t)l * s.qkv_rows * D * es), s.qkv_rows,
+                                          (int)(D * es / 2), (s.Hq + s.Hkv) * s.d, s.d);
+    else
+      CKC(cudaMemcpyAsync((char*)ctx->w_qkv + (size_t)l * s.qkv_rows * D * es, w->w_qkv[l],
+                          (size_t)s.qkv_rows * D * es, cudaMemcpyDeviceToDevice, cs));
+    CKC(cudaGetLastError());
     CKC(cudaMemcpyAsync((char*)ctx->w_o + (size_t)l * D * s.attn_dim * es, w->w_o[l], (size_t)D * s.attn_dim * es,
                         cudaMemcpyDeviceToDevice, cs));
     CKC(cudaMemcpyAsync((char*)ctx->w_down + (size_t)l * D * F * es, w->w_down[l], (size_t)D * F * es,
@@ -1058,6 +1127,40 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
   ALLOC(ctx->vc, slot_elems * es);
   CKC(cudaMemsetAsync(ctx->kc, 0, slot_elems * es, cs));
   CKC(cudaMemsetAsync(ctx->vc, 0, slot_elems * es, cs));
+  if (s.rope) {
+    // (cos, sin) per position and channel pair, angles in float64 from the
+    // integer positions, each rounded once to fp32
+    const int half = s.d / 2;
+    std::vector<float2> cs_host((size_t)s.Ptot * half);
+    for (int pos = 0; pos < s.Ptot; ++pos)
+      for (int i = 0; i < half; ++i) {
+        const double a = (double)pos * std::pow((double)cfg->rope_base, -2.0 * i / (double)s.d);
+        cs_host[(size_t)pos * half + i] = make_float2((float)std::cos(a), (float)std::sin(a));
+      }
+    ALLOC(ctx->rope_cs, sizeof(float2) * cs_host.size());
+    CKC(cudaMemcpyAsync(ctx->rope_cs, cs_host.data(), sizeof(float2) * cs_host.size(), cudaMemcpyHostToDevice, cs));
+    CKC(cudaStreamSynchronize(cs));  // cs_host goes out of scope
+  }
+  if (s.Dp > 0) {
+    const int kvr = 2 * s.Hkv * s.d;
+    ALLOC(ctx->w_pkv, (size_t)L * kvr * s.Dp * es);
+    ALLOC(ctx->ypre, (size_t)std::max(s.Pmax, 1) * s.Dp * es);
+    for (int l = 0; l < L; ++l) {
+      if (!w->w_prefix_kv || !w->w_prefix_kv[l]) {
+        fail(ctx, PAE_ERR_ARG, "prefix_width > 0 needs w_prefix_kv for every layer");
+        return bail(PAE_ERR_ARG);
+      }
+      k_permute_rows<<<256, 256, 0, cs>>>((const uint16_t*)w->w_prefix_kv[l],
+                                          (uint16_t*)((char*)ctx->w_pkv + (size_t)l * kvr * s.Dp * es), kvr,
+                                          (int)(s.Dp * es / 2), s.rope ? s.Hkv * s.d : 0, s.d);
+      CKC(cudaGetLastError());
+    }
+    if (ctx->act_bf16) {
+      if ((st = make_map(ctx, &ctx->tmWpkv, ctx->w_pkv, s.Dp, (uint64_t)L * kvr, 64, 128)) != PAE_OK) return bail(st);
+      if ((st = make_map(ctx, &ctx->tmYpre, ctx->ypre, s.Dp, (uint64_t)std::max(s.Pmax, 1), 64, 128)) != PAE_OK)
+        return bail(st);
+    }
+  }
   ALLOC(ctx->lens_dev, sizeof(int) * s.Bmax);
   CKC(cudaMemsetAsync(ctx->lens_dev, 0, sizeof(int) * s.Bmax, cs));
   const size_t Mmax = (size_t)s.Bmax * s.H;
@@ -1143,6 +1246,53 @@ pae_status pae_set_prefix(pae_ctx* ctx, int row, const void* const* k_per_layer,
       CK(cudaMemcpy2DAsync((char*)ctx->kc + slot, rowb, ks, s.Hkv * rowb, rowb, len, cudaMemcpyDeviceToDevice, stm));
       CK(cudaMemcpy2DAsync((char*)ctx->vc + slot, rowb, vs, s.Hkv * rowb, rowb, len, cudaMemcpyDeviceToDevice, stm));
     }
+  }
+  k_set_len<<<1, 1, 0, stm>>>(ctx->lens_dev, row, len);
+  CK(cudaGetLastError());
+  ctx->lens_host[row] = len;
+  return PAE_OK;
+}
+
+pae_status pae_set_prefix_hidden(pae_ctx* ctx, int row, const void* const* h_per_layer, int len,
+                                 pae_stream stream) {
+  if (!ctx) return fail(nullptr, PAE_ERR_ARG, "ctx is NULL");
+  pae_status st = check_err_word(ctx);
+  if (st != PAE_OK) return st;
+  const Shape& s = ctx->s;
+  if (s.Dp <= 0) return fail(ctx, PAE_ERR_STATE, "the context was created with prefix_width = 0");
+  if (row < 0 || row >= s.Bmax) return fail(ctx, PAE_ERR_ARG, "row %d out of range [0, %d)", row, s.Bmax);
+  if (len < 0 || len > s.Pmax) return fail(ctx, PAE_ERR_ARG, "len %d out of range [0, %d]", len, s.Pmax);
+  if (len > 0) {
+    if (!h_per_layer) return fail(ctx, PAE_ERR_ARG, "h_per_layer is NULL");
+    for (int l = 0; l < s.L; ++l)
+      if (!h_per_layer[l]) return fail(ctx, PAE_ERR_ARG, "layer %d hidden-state pointer is NULL", l);
+  }
+  cudaStream_t stm = reinterpret_cast<cudaStream_t>(stream);
+  const int kvr = 2 * s.Hkv * s.d;
+  const TcPlan plan = ctx->act_bf16 && len > 0 ? prefix_plan(s, len) : TcPlan{};
+  for (int l = 0; l < s.L && len > 0; ++l) {
+    CK(launch_prefix_norm(ctx->act_bf16, h_per_layer[l], ctx->ypre, len, s.Dp, s.eps, stm));
+    EpiArgs e{};
+    e.epi = EPI_PREFIX;
+    e.M = len;
+    e.kc = ctx->kc;
+    e.vc = ctx->vc;
+    e.layer = l;
+    e.prefix_row = row;
+    e.rope_cs = ctx->rope_cs;
+    if (!ctx->act_bf16) {
+      launch_gemm_simple(s, static_cast<const float*>(ctx->ypre),
+                         static_cast<const float*>(ctx->w_pkv) + (size_t)l * kvr * s.Dp, kvr, s.Dp, e, stm);
+    } else {
+      TcGemmArgs a{};
+      a.e = e;
+      a.N = kvr;
+      a.K = s.Dp;
+      a.w_row0 = l * kvr;
+      a.err = DevErr{ctx->err_dev, ctx->wait_ns};
+      CK(launch_tc_gemm(s, &ctx->tmWpkv, &ctx->tmYpre, 1, plan, a, false, stm));
+    }
+    CK(cudaGetLastError());
   }
   k_set_len<<<1, 1, 0, stm>>>(ctx->lens_dev, row, len);
   CK(cudaGetLastError());

@@ -19,6 +19,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdio>
 #include <mutex>
 
 #include "internal.h"
@@ -173,10 +174,21 @@ extern "C" pae_status pae_precompute_tables_static(int layers, int width, int dt
     if (!((t[k + 1] - t[k]) * dir > 0.0))
       return fail_static(PAE_ERR_ARG, "pae_precompute_tables_static: t must be strictly monotone");
 
+  // An error left pending by earlier, unrelated work would otherwise surface
+  // from the launch checks below as if this call had caused it.
+  cudaError_t e = cudaPeekAtLastError();
+  if (e != cudaSuccess) {
+    char msg[256];
+    snprintf(msg, sizeof msg, "pae_precompute_tables_static: a CUDA error from earlier work is pending (%s)",
+             cudaGetErrorString(e));
+    return fail_static(PAE_ERR_CUDA, msg);
+  }
   int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess)
     return fail_static(PAE_ERR_CUDA, "pae_precompute_tables_static: cudaGetDevice failed");
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail_static(PAE_ERR_UNSUPPORTED, "pae_precompute_tables_static: device ordinals of 64 and above are "
+                                            "not supported (per-device address cache)");
   float* scratch = nullptr;
   if ((e = scratch_address(dev, &scratch)) != cudaSuccess)
     return fail_static(PAE_ERR_CUDA, "pae_precompute_tables_static: cudaGetSymbolAddress failed");

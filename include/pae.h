@@ -68,12 +68,26 @@ typedef enum {
  * D <= 2048;
  * BF16/W4A16: D, Hq*d, F multiples of 128, d in {64, 128, 256}, H <= 256,
  * max_batch*H <= 4096.
+ *
+ * rope_base: 0 = no rotary position embedding (the default); > 0 = rotate
+ * every query head and every action key at its position in the request's
+ * joint [prefix | action] sequence, P_b + i for action token i of a request
+ * with a P_b-token prefix (the cached prefix keys are taken as already
+ * rotated at 0..P_b-1).  Rotate-half form: channel i < d/2 pairs with
+ * i + d/2 and turns by pos * rope_base^(-2i/d).  The angles come from a
+ * cos/sin table built once in float64 from the integer positions (the
+ * vla.cpp abstract warns that positional-index precision changes actions).
+ * prefix_width: 0 = no prefix production (the default); > 0 = the width of
+ * the hidden states pae_set_prefix_hidden projects into the K/V slots (then
+ * pae_weights.w_prefix_kv is required).
  */
 typedef struct {
   int layers, width, n_q_heads, n_kv_heads, head_dim, mlp_dim, action_dim, chunk;
   int max_batch, max_prefix, group_size;
   int dtype;        /* pae_dtype */
   float rms_eps;
+  float rope_base;  /* 0: off */
+  int prefix_width; /* 0: no pae_set_prefix_hidden */
 } pae_config;
 
 /*
@@ -93,6 +107,10 @@ typedef struct {
  * complement codes in [-8, 7], low nibble = even k) and s_qkv..s_down to bf16
  * scales [N][K/group_size]; value = code * scale.  The s_* arrays are ignored in
  * the other modes.  Attention and MLP carry no biases.
+ *   w_prefix_kv[l] [2 Hkv d][prefix_width]   prefix production (only when
+ *                                 cfg.prefix_width > 0): layer l's key rows
+ *                                 (Hkv heads) then value rows, fp32 in PAE_FP32
+ *                                 mode, bf16 otherwise (also in PAE_W4A16).
  */
 typedef struct {
   const void *w_in, *b_in, *w_out, *b_out;
@@ -100,6 +118,7 @@ typedef struct {
   const void *w_mod, *b_mod, *w_modf, *b_modf;
   const void *const *w_qkv, *const *w_o, *const *w_gate, *const *w_up, *const *w_down;
   const void *const *s_qkv, *const *s_o, *const *s_gate, *const *s_up, *const *s_down;
+  const void *const *w_prefix_kv;
 } pae_weights;
 
 /* Validate cfg, allocate the context's device buffers, copy and repack the
@@ -118,6 +137,20 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
  * 0 <= len <= max_prefix, 0 <= row < max_batch (else PAE_ERR_ARG). */
 pae_status pae_set_prefix(pae_ctx* ctx, int row, const void* const* k_per_layer,
                           const void* const* v_per_layer, int len, pae_stream stream);
+
+/* Produce and cache the prefix of request `row` from the prefix model's
+ * per-layer hidden states (report Sec. 5.1: the vision-language prefix is
+ * computed once per observation and its per-layer K/V cached): for every
+ * layer l, y = h_l / sqrt(mean(h_l^2) + rms_eps) per token (a plain RMSNorm;
+ * fold a learned gain into w_prefix_kv), [k | v] = y w_prefix_kv[l]^T, keys
+ * rotated at positions 0..len-1 when rope_base > 0, written straight into the
+ * row's K/V slot (no intermediate K/V buffer).  h_per_layer (host array of L
+ * device pointers) each point to [len][prefix_width] (fp32 in PAE_FP32 mode,
+ * bf16 otherwise).  Replaces the row's prefix like pae_set_prefix.
+ * Errors: PAE_ERR_STATE if the context was created with prefix_width == 0;
+ * PAE_ERR_ARG for a bad row, len outside [0, max_prefix] or NULL pointers. */
+pae_status pae_set_prefix_hidden(pae_ctx* ctx, int row, const void* const* h_per_layer, int len,
+                                 pae_stream stream);
 
 /* Build the timestep conditioning once for a grid t[0..K] (host, float64,
  * strictly monotone, K >= 1, K <= 64): the sinusoidal embedding, the time MLP,
@@ -260,7 +293,12 @@ pae_status pae_debug_copy(pae_ctx* ctx, const char* name, void* dst_host, size_t
  * per device that every call shares: calls whose GPU work overlaps (streams
  * with no ordering between them) race and must be serialised by the caller.
  * The first call on a device looks the array up and sets kernel attributes;
- * make that first call before any stream capture.  Asynchronous on `stream`. */
+ * make that first call before any stream capture.  That look-up is cached for
+ * the life of the process: after cudaDeviceReset on a device, restart the
+ * process before calling this entry point there again.  Devices with ordinals
+ * of 64 and above give PAE_ERR_UNSUPPORTED.  A CUDA error already pending from
+ * earlier work is reported as such (PAE_ERR_CUDA) before anything is
+ * enqueued.  Asynchronous on `stream`. */
 pae_status pae_precompute_tables_static(int layers, int width, int dtype, const pae_weights* w,
                                         const double* t, int K, float* tables, float* dt,
                                         pae_stream stream);

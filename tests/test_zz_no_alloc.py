@@ -58,6 +58,58 @@ def test_static_tables_match_context_tables(cfg):
         assert np.all(np.isfinite(got_tab)), f"call {call}: unwritten table entries"
         assert np.max(np.abs(got_tab - want_tab[:got_tab.size])) <= TOL_FP32_MAX_ABS, f"call {call}: tables differ"
         assert np.max(np.abs(got_dt - want_dt[:K])) <= TOL_FP32_MAX_ABS, f"call {call}: dt differs"
+        ref_tab, _ = _oracle_table_rows(cfg, W, grid)
+        assert np.max(np.abs(got_tab.reshape(K, rows) - ref_tab)) <= TOL_FP32_MAX_ABS, f"call {call}: vs oracle"
+
+
+def _oracle_table_rows(cfg, W, grid):
+    """The oracle's per-step tables in the library's layout: per layer l and
+    norm j the rows (scale, shift, gate), then the final (scale, shift)."""
+    import oracle
+    p = oracle.params_from_weights(cfg, W)
+    out = []
+    for tab in oracle.modulation_tables(grid, p):
+        parts = []
+        for l in range(cfg.layers):
+            for j in range(2):
+                parts += [tab.scale[l, j], tab.shift[l, j], tab.gate[l, j]]
+        parts += [tab.scale_f, tab.shift_f]
+        out.append(np.concatenate(parts))
+    return np.stack(out), np.array([t.dt for t in oracle.modulation_tables(grid, p)])
+
+
+# Sizes at the edges of the fixed scratch array and of the 16-step passes of its
+# batched GEMV: K = 17 (a second, one-step pass), K = 64 at width 2048 (the whole
+# array), and the int4 mode (its modulation weights are bf16 as in bf16 mode).
+EDGE_CASES = [
+    wl.TINY_FP32.replace(name="k17_fp32", steps=17),
+    wl.TINY_FP32.replace(name="k64_w2048_bf16", dtype=wl.BF16, layers=1, width=2048, mlp_dim=128, steps=64),
+    wl.TINY_FP32.replace(name="k64_w2048_fp32", layers=1, width=2048, mlp_dim=128, steps=64),
+    wl.TINY_FP32.replace(name="tiny_w4a16_t", dtype=wl.W4A16, steps=10),
+]
+
+
+@pytest.mark.parametrize("cfg", EDGE_CASES, ids=[c.name for c in EDGE_CASES])
+def test_static_tables_edge_sizes_match_oracle(cfg):
+    W = wl.make_weights(cfg)
+    grid = wl.uniform_grid(cfg.steps)
+    want_tab, want_dt = _oracle_table_rows(cfg, W, grid)
+    K = cfg.steps
+    rows = (6 * cfg.layers + 2) * cfg.width
+    dev_w = wd.upload_weights(cfg, W)
+    w = _weights_struct(dev_w)
+    code = fm.DTYPE_CODES[cfg.dtype]
+    for call in range(2):
+        tables = torch.full((K, rows), float("nan"), dtype=torch.float32, device="cuda")
+        dt = torch.full((K,), float("nan"), dtype=torch.float32, device="cuda")
+        fm.pae_precompute_tables_static(cfg.layers, cfg.width, code, w, list(grid), tables.data_ptr(),
+                                        dt.data_ptr())
+        torch.cuda.synchronize()
+        got = tables.cpu().numpy()
+        assert np.all(np.isfinite(got)), f"call {call}: unwritten table entries"
+        err = float(np.max(np.abs(got - want_tab)))
+        assert err <= TOL_FP32_MAX_ABS, f"{cfg.name} call {call}: tables differ from the oracle by {err:.3e}"
+        assert np.max(np.abs(dt.cpu().numpy() - want_dt)) <= 1e-6, f"{cfg.name} call {call}: dt differs"
 
 
 def test_static_tables_reject_sizes_beyond_the_scratch():

@@ -53,6 +53,8 @@ class ExpertConfig:
     rms_eps: float = 1e-6
     ragged: bool = False   # per-request prefix lengths drawn on [512, 1024]
     index: int = 0         # config index, added to every seed
+    rope_base: float = 0.0  # rotary embedding base (0: off)
+    prefix_width: int = 0   # width of the prefix model's hidden states (0: no prefix production)
 
     @property
     def qkv_dim(self) -> int:
@@ -181,6 +183,35 @@ def make_weights(cfg: ExpertConfig, seed: Optional[int] = None) -> Dict[str, obj
             else:
                 W[name].append(_normal(g, shp, std, dt))
     return W
+
+
+def make_prefix_model(cfg: ExpertConfig, prefix_len: Optional[int] = None,
+                      seed: Optional[int] = None) -> Dict[str, object]:
+    """A stand-in for the vision-language model that produces the prefix: per
+    layer a QKV projection [(Hq + 2 Hkv) d][Dp], an output projection
+    [Dp][Hq d] and a GeGLU MLP (F x Dp), all ~N(0, 0.05), and the prefix's
+    input hidden states z [P][Dp] ~N(0, 1) (Dp = cfg.prefix_width; seed
+    3 + config index).  Values are bf16-rounded in bf16 and W4A16 modes.
+    "w_prefix_kv" holds each layer's key and value rows of its QKV projection,
+    the weights the prefix production step projects with."""
+    Dp = cfg.prefix_width
+    if Dp <= 0:
+        raise ValueError("make_prefix_model needs cfg.prefix_width > 0")
+    g = rng((3 + cfg.index) if seed is None else seed)
+    dt = BF16 if cfg.dtype in (BF16, W4A16) else FP32
+    P = cfg.prefix if prefix_len is None else prefix_len
+    L, F, std = cfg.layers, cfg.mlp_dim, 0.05
+    M: Dict[str, object] = {"w_qkv": [], "w_o": [], "w_gate": [], "w_up": [], "w_down": []}
+    for _l in range(L):
+        M["w_qkv"].append(_normal(g, (cfg.qkv_dim, Dp), std, dt))
+        M["w_o"].append(_normal(g, (Dp, cfg.attn_dim), std, dt))
+        M["w_gate"].append(_normal(g, (F, Dp), std, dt))
+        M["w_up"].append(_normal(g, (F, Dp), std, dt))
+        M["w_down"].append(_normal(g, (Dp, F), std, dt))
+    M["z"] = _normal(g, (P, Dp), 1.0, dt)
+    qd = cfg.attn_dim
+    M["w_prefix_kv"] = [np.ascontiguousarray(w[qd:]) for w in M["w_qkv"]]
+    return M
 
 
 def dequantized(W: Dict[str, object], name: str, layer: int) -> np.ndarray:

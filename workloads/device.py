@@ -35,6 +35,8 @@ def upload_weights(cfg: ExpertConfig, W: Dict[str, object], device="cuda") -> Di
             out[SCALE_KEYS[name]] = [to_dev(m.scales, torch.bfloat16, device) for m in W[name]]
         else:
             out[name] = [to_dev(m, dt, device) for m in W[name]]
+    if "w_prefix_kv" in W:  # prefix production weights (activation dtype)
+        out["w_prefix_kv"] = [to_dev(m, dt, device) for m in W["w_prefix_kv"]]
     return out
 
 
@@ -50,7 +52,8 @@ def abi_config(cfg: ExpertConfig, max_batch=None, max_prefix=None) -> Dict[str, 
                 head_dim=cfg.head_dim, mlp_dim=cfg.mlp_dim, action_dim=cfg.action_dim, chunk=cfg.chunk,
                 max_batch=cfg.batch if max_batch is None else max_batch,
                 max_prefix=cfg.prefix if max_prefix is None else max_prefix,
-                dtype=cfg.dtype, group_size=cfg.group_size, rms_eps=cfg.rms_eps)
+                dtype=cfg.dtype, group_size=cfg.group_size, rms_eps=cfg.rms_eps, rope_base=cfg.rope_base,
+                prefix_width=cfg.prefix_width)
 
 
 __all__ = ["upload_weights", "upload_prefix", "abi_config", "act_dtype", "to_dev", "BF16", "FP32", "W4A16"]
