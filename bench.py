@@ -142,8 +142,9 @@ def algorithmic(cfg: wl.ExpertConfig, batch: int, lens=None):
     step_kv = L * 2 * sum(lens) * cfg.n_kv_heads * cfg.head_dim * ae
     step_flops = L * (out["qkv"]["flops"] + out["o_proj"]["flops"] + out["gate_up"]["flops"] +
                       out["down"]["flops"] + out["attention"]["flops"]) + 2 * 2 * M * A * D
-    # the persistent kernel runs a whole call (all Euler steps) in one launch
+    # the persistent kernel and the dataflow loop run a whole call (all Euler steps) in one launch
     out["persistent"] = {"bytes": cfg.steps * (step_w + step_kv), "flops": cfg.steps * step_flops}
+    out["dataflow"] = dict(out["persistent"])
     return out, {"bytes": step_w + step_kv, "flops": step_flops}
 
 
@@ -334,8 +335,10 @@ def measure(cfg, W, batch, args, stream, barrier, maxr, lens=None, with_e2e=True
         res["clocks"] = clk.stop()
         res["ms_per_step"] = maxr(ms)
         res["persistent"] = ex.query(fm.PAE_Q_PERSISTENT, batch)
-        # kernels per pae_denoise call: one persistent launch, or the captured graph's kernel nodes
-        res["graph_kernels"] = 1 if res["persistent"] else ex.query(fm.PAE_Q_GRAPH_KERNELS, batch)
+        res["dataflow"] = ex.query(fm.PAE_Q_DATAFLOW, batch)
+        # kernels per pae_denoise call: one persistent or dataflow launch, or the captured graph's kernel nodes
+        res["graph_kernels"] = 1 if (res["persistent"] or res["dataflow"]) else \
+            ex.query(fm.PAE_Q_GRAPH_KERNELS, batch)
         res["splits"] = ex.query(fm.PAE_Q_SPLITS, batch)
         res["token_tile"] = ex.query(fm.PAE_Q_TOKEN_TILE, batch)
         res["table_ms"] = table_ms
@@ -566,7 +569,9 @@ def run_ours(args, cfg):
         "kernels_ms_per_launch": {c: v["ms_per_launch"] for c, v in res["kernels"].items()},
         "gpu_launches": int(res["graph_kernels"]) * args.steps,
         "kernels_per_call": int(res["graph_kernels"]),
-        "loop": "persistent kernel" if res["persistent"] else "captured graph",
+        "loop": ("persistent kernel" if res["persistent"] else
+                 f"dataflow loop (one launch, clusters of {res['dataflow']})" if res["dataflow"] else
+                 "captured graph"),
         "splitk": {"qkv": res["splits"] & 255, "o": (res["splits"] >> 8) & 255,
                    "gate_up": (res["splits"] >> 16) & 255, "down": (res["splits"] >> 24) & 255},
         "token_tile": res["token_tile"], "table_build_ms": res["table_ms"],

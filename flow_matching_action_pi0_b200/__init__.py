@@ -24,10 +24,12 @@ PAE_FP32, PAE_BF16, PAE_W4A16 = 0, 1, 2
 PAE_OPT_USE_GRAPH, PAE_OPT_WAIT_LIMIT_US, PAE_OPT_PROFILE, PAE_OPT_PDL, PAE_OPT_MAX_SPLITK = 1, 2, 3, 4, 5
 PAE_OPT_PERSISTENT = 6
 PAE_OPT_FUSED_NORM = 7
+PAE_OPT_DATAFLOW, PAE_OPT_DATAFLOW_CLUSTER = 8, 9
 (PAE_K_TRANSITION, PAE_K_QKV, PAE_K_ATTENTION, PAE_K_OPROJ, PAE_K_NORM, PAE_K_GATEUP,
- PAE_K_DOWN, PAE_K_PERSISTENT) = range(8)
-KERNEL_CLASSES = ("transition", "qkv", "attention", "o_proj", "norm", "gate_up", "down", "persistent")
+ PAE_K_DOWN, PAE_K_PERSISTENT, PAE_K_DATAFLOW) = range(9)
+KERNEL_CLASSES = ("transition", "qkv", "attention", "o_proj", "norm", "gate_up", "down", "persistent", "dataflow")
 PAE_Q_GRAPH_KERNELS, PAE_Q_SPLITS, PAE_Q_TOKEN_TILE, PAE_Q_ATTN_SPLITS, PAE_Q_PERSISTENT, PAE_Q_FUSED_NORM = 1, 2, 3, 4, 5, 6
+PAE_Q_DATAFLOW = 7
 STATUS_NAMES = {0: "PAE_OK", 1: "PAE_ERR_ARG", 2: "PAE_ERR_STATE", 3: "PAE_ERR_CUDA", 4: "PAE_ERR_OOM",
                 5: "PAE_ERR_TIMEOUT", 6: "PAE_ERR_UNSUPPORTED"}
 

@@ -41,6 +41,12 @@ void launch_time_mlp(const Shape& s, int act_bf16, const double* t, int K, const
 void launch_mod_tables(const Shape& s, int act_bf16, const float* cbuf, int K, const void* w_all,
                        const void* b_all, float* tables, cudaStream_t st);
 
+// out[k][l][r] = W_l[r] . shift_k(l, norm) for every stored row r of the stacked
+// bf16 matrix W ([L][rows][D]); out [K][L][rows] fp32.  norm 0 = attention,
+// 1 = MLP adaRMSNorm.
+void launch_shift_bias(const Shape& s, const void* W, int rows, int norm, const float* tables, int K, float* out,
+                       cudaStream_t st);
+
 // ------------------------------------------------------------ token kernels
 // Per token: optionally (final adaRMSNorm, out_proj, Euler update of x with
 // step k_out), then optionally (in_proj of x and the first attention norm of
@@ -187,5 +193,48 @@ cudaError_t persist_init();
 // Cooperative launch of a.ncta CTAs (one per SM).
 cudaError_t launch_persistent(const Shape& s, const CUtensorMap* maps /* Wqkv, Wo, Wgu (128-row box), Wdown, Q, K, V */,
                               const PersistArgs& a, cudaStream_t st);
+
+// ------------------------------------ dataflow loop (B*H <= 64, clusters)
+// One launch of NC clusters of C CTAs runs all Euler steps of a call; stages
+// wait on per-tile counters (k_flow.cu).
+constexpr int kFlowCtrWords = 512;  // counters; the last word is the abort flag
+struct FlowArgs {
+  int M, B;                          // tokens, requests
+  int C, NC;                         // cluster size, clusters
+  int k_begin, k_end;                // Euler steps of this launch
+  int q_tiles, o_tiles, g_pairs, d_tiles;  // 128-row weight tiles (gate/up: pairs)
+  int kb_q, kb_o, kb_g, kb_d;        // 64-wide K blocks per rank
+  int a_units, a_qtiles, a_kps;      // attention clusters, query tiles per (b, kv head), keys per rank
+  float* x;
+  float* h;
+  bf16* yq;                          // bf16(h (1 + scale)) of the attention norm [64][D]
+  bf16* yg;                          // the same for the MLP norm
+  bf16* q;
+  bf16* o;
+  bf16* u;
+  bf16* kc;
+  bf16* vc;
+  const int* lens;
+  const float* tables;
+  const float* dt;
+  const float* bias_qkv;             // [K][L][qkv_rows]  W_qkv shift_attention
+  const float* bias_gu;              // [K][L][2F]        W_gate/up shift_mlp (stored row order)
+  float* ss_q;                       // [d_tiles * C][64] sums of squares for the QKV norm
+  float* ss_g;                       // [o_tiles * C][64] for the MLP norm
+  float* ss_t;                       // [64] from the transition (layer 0)
+  const bf16* w_inT;
+  const bf16* b_in;
+  const bf16* w_out;
+  const bf16* b_out;
+  const float2* rope_cs;
+  unsigned* ctr;                     // [kFlowCtrWords], zero at launch
+  DevErr err;
+};
+size_t flow_smem_bytes();
+cudaError_t flow_init();
+int flow_max_clusters(int C);        // clusters of C CTAs that fit at once (0 on error)
+// maps: W qkv, W o, W gate/up (128-row boxes), W down, y_q, o, y_g, u (64 x 64
+// boxes), q (64 x 128), k, v (64 x 64).  Cooperative cluster launch.
+cudaError_t launch_flow(const Shape& s, const CUtensorMap* maps, const FlowArgs& a, cudaStream_t st);
 
 }  // namespace pae

@@ -1,0 +1,1122 @@
+// Small-batch denoise loop as one launch of thread-block clusters (the
+// "dataflow loop", for batch * chunk <= 64 action tokens).
+//
+// At batch 1 the expert's projections are weight streams with 50 tokens each,
+// and the graph of ~126 dependent kernels per Euler step spends its time in
+// launch, set-up and drain.  Here one cooperative launch runs all Euler steps
+// of a call; inside it every stage of a layer
+//   Q  [q | k | v] = norm(h) W_qkv^T   (q, and k / v into the request's slot)
+//   A  GQA attention over [cached prefix | action keys]
+//   O  h += gate_a * (o W_o^T)
+//   G  u = gelu(norm(h) W_gate^T) * (norm(h) W_up^T)
+//   D  h += gate_m * (u W_down^T)
+// waits only for the data it reads, through per-tile counters in global
+// memory (release / acquire), never for a grid-wide barrier.
+//
+// Work split.  The grid is NC clusters of C CTAs (one CTA per SM).  A
+// projection's 128-row weight tiles go to clusters round robin; the K range of
+// a tile is split over the C ranks of its cluster, each rank multiplying its
+// K slice of the token operand by its slice of the weights (tcgen05, weights
+// as the MMA's M side, tokens as N = 64, fp32 accumulators in TMEM).  The C
+// partial tiles are summed inside the cluster: every rank parks its partial
+// in its own shared memory, a cluster barrier, then rank q adds rows
+// [q R, q R + R) of all C partials (distributed shared memory loads, in rank
+// order, so results are bitwise reproducible) and runs the epilogue for them.
+// Attention: one cluster per (request, KV head, 128 query rows), its ranks
+// taking consecutive 64-key chunks; partial outputs are merged the same way.
+//
+// adaRMSNorm.  y = h rstd (1 + scale) + shift is not formed: the producer of
+// h writes bf16(h (1 + scale)) and per-row sums of squares once, and the
+// consumer's reducer applies rstd after the contraction and adds the shift
+// term W shift from a table built with the timestep tables.  The same value
+// as W y, with no re-normalisation of fp32 h in every tile.
+//
+// Weights never depend on activations: warp 0 streams this CTA's weight
+// blocks into a ring of shared memory in schedule order and prefetches the
+// same blocks of the next layer into L2, so HBM keeps streaming while the
+// dependency chain runs.  Warp 1 issues the MMAs; warps 2-5 do the rest
+// (token operands by TMA, TMEM reads, cluster reductions, epilogues, the
+// attention softmax and the per-token transition between Euler steps).
+//
+// Every wait is bounded (%globaltimer).  A wait that runs out records
+// PAE_ERR_TIMEOUT and sets a launch-wide abort flag that every other wait
+// watches; cluster barriers are mbarrier-based and bounded too.  Before exit
+// every CTA drains its copies and MMAs and meets its cluster once more (a
+// hardware cluster barrier that all threads reach on every path), so no CTA
+// leaves while a peer may still read its shared memory.
+#include "epilogue.cuh"
+#include "launch.cuh"
+
+namespace pae {
+
+namespace {
+
+constexpr int kFThreads = 192;   // warp 0 weights, warp 1 MMA, warps 2-5 compute
+constexpr int kFCompute = 128;
+constexpr int kFRing = 5;
+constexpr uint32_t kFBlk = 16384;        // [128 rows][64] bf16 weight block
+constexpr uint32_t kFWork = 128 * 1024;  // operands, partial tiles, attention tiles
+constexpr uint32_t kFMisc = 4096;
+constexpr uint32_t kFSmem = kFRing * kFBlk + kFWork + kFMisc + 1024;
+constexpr uint32_t kFOp = 0;             // token operand [kbr][64 tokens][64] bf16
+constexpr uint32_t kFPart = 64 * 1024;   // two partial tiles [64 tokens][128 rows] fp32
+constexpr uint32_t kFTmem = 512;
+constexpr uint32_t kColS = 128;          // attention scores (P over their first 32 columns)
+constexpr uint32_t kColO = 256;          // attention output
+constexpr int CKF = 64;                  // keys per attention chunk
+constexpr long long kFDrain = 4000000000LL;
+
+enum : int { ST_Q = 0, ST_O = 1, ST_G = 2, ST_D = 3 };
+
+// ------------------------------------------------------------ small helpers
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_u32(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global_f() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+__device__ __forceinline__ void csync() {
+  __syncwarp();
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+// AND over the 128 compute threads.
+__device__ __forceinline__ bool cand(bool v) {
+  __syncwarp();
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cl(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void hw_cluster_sync() {
+  __syncwarp();
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* tm, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(tm)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
+  return (uint32_t)__bfloat16_as_ushort(f2bf(a)) | ((uint32_t)__bfloat16_as_ushort(f2bf(b)) << 16);
+}
+__device__ __forceinline__ void st_shared_f4(uint32_t addr, float4 v) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+struct FMaps {
+  const CUtensorMap* w[4];   // Q, O, G (128-row boxes), D weights
+  const CUtensorMap* x[4];   // token operands: y (QKV), o, y (gate/up), u
+  const CUtensorMap *q, *k, *v;
+};
+
+struct FC {
+  const Shape* s;
+  const FlowArgs* a;
+  FMaps mp;
+  uint8_t* ring;
+  uint8_t* work;
+  uint64_t* rfull;     // [kFRing]
+  uint64_t* rempty;    // [kFRing]
+  uint64_t* op_full;   // token operand of a projection stage landed
+  uint64_t* acc_full;  // [2] accumulator slot ready
+  uint64_t* acc_empty; // [2] accumulator slot read out
+  uint64_t* kv_full;   // attention q / K / V chunk landed
+  uint64_t* s_full;
+  uint64_t* p_full;
+  uint64_t* o_full;
+  uint64_t* cbar;      // [2] cluster barrier (count C), alternating instances
+  uint64_t* drain;
+  float* s_rstd;       // [64]
+  float* s_tmp;        // [256]
+  float* s_ml;         // [128][2] attention row max / sum
+  volatile int* s_abort;
+  volatile int* s_flag;
+  uint32_t tmem;
+  int cta, cl, rank, ct;  // ct: compute-thread index 0..127
+};
+
+__device__ __forceinline__ unsigned* abort_word(const FlowArgs& a) { return a.ctr + kFlowCtrWords - 1; }
+
+// Launch-wide abort: record the error, stop this CTA's roles, tell all CTAs.
+__device__ void raise_abort(const FC& c) {
+  *c.s_abort = 1;
+  atomicExch(reinterpret_cast<int*>(abort_word(*c.a)), 1);
+  set_error(c.a->err, DEV_TIMEOUT);
+}
+
+// Bounded mbarrier wait that also gives up once the launch is aborting.
+__device__ bool fwait(const FC& c, uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  const volatile unsigned* ab = abort_word(*c.a);
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*c.s_abort || *ab) {
+      *c.s_abort = 1;
+      return false;
+    }
+    if ((long long)(globaltimer_ns() - t0) > c.a->err.wait_ns) {
+      raise_abort(c);
+      return false;
+    }
+  }
+}
+
+// Bounded wait until a global counter reaches `target` (acquire).
+__device__ bool wait_ctr(const FC& c, const unsigned* p, unsigned target) {
+  if (ld_acquire_u32(p) >= target) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  const volatile unsigned* ab = abort_word(*c.a);
+  while (true) {
+    if (ld_acquire_u32(p) >= target) return true;
+    if (*c.s_abort || *ab) {
+      *c.s_abort = 1;
+      return false;
+    }
+    if ((long long)(globaltimer_ns() - t0) > c.a->err.wait_ns) {
+      raise_abort(c);
+      return false;
+    }
+  }
+}
+
+// Every compute thread's global writes, then one release increment of `p`.
+__device__ void publish(const FC& c, unsigned* p) {
+  __threadfence();
+  csync();
+  if (c.ct == 0) red_release_u32(p, 1u);
+}
+
+// Cluster barrier among the compute threads of the C ranks, bounded: every
+// rank's compute thread 0 arrives (release, cluster scope) on instance n's
+// mbarrier of every rank, then waits (acquire) on its own.  Instances
+// alternate between two mbarriers, so an early arrival for instance n + 1 can
+// never complete instance n.  Returns false once the launch is aborting.
+__device__ bool cl_sync(const FC& c, int& n) {
+  fence_acq_rel_cluster();
+  csync();
+  if (c.ct == 0) {
+    bool ok = !*c.s_abort;
+    if (ok) {
+      uint64_t* b = &c.cbar[n & 1];
+      const uint32_t baddr = smem_u32(b);
+      for (int r = 0; r < c.a->C; ++r) mbar_arrive_remote(map_cluster(baddr, (uint32_t)r));
+      const uint32_t par = (uint32_t)(n >> 1) & 1u;
+      ok = mbar_try_wait_cl(b, par);
+      if (!ok) {
+        const unsigned long long t0 = globaltimer_ns();
+        const volatile unsigned* ab = abort_word(*c.a);
+        while (!(ok = mbar_try_wait_cl(b, par))) {
+          if (*ab) {
+            *c.s_abort = 1;
+            break;
+          }
+          if ((long long)(globaltimer_ns() - t0) > c.a->err.wait_ns) {
+            raise_abort(c);
+            break;
+          }
+        }
+      }
+    }
+    *c.s_flag = ok ? 1 : 0;
+  }
+  csync();
+  ++n;
+  return *c.s_flag != 0;
+}
+
+// ------------------------------------------------------------ schedule
+// Projection stage geometry: output tiles (G: pairs of a gate and an up tile),
+// K blocks per rank, weight rows per layer and the first row of an item.
+struct StageG {
+  int ntiles, na, kbr, wrows;
+};
+__device__ __forceinline__ StageG stage_geo(const Shape& s, const FlowArgs& a, int st) {
+  StageG g;
+  switch (st) {
+    case ST_Q: g = StageG{a.q_tiles, 1, a.kb_q, s.qkv_rows}; break;
+    case ST_O: g = StageG{a.o_tiles, 1, a.kb_o, s.D}; break;
+    case ST_G: g = StageG{a.g_pairs, 2, a.kb_g, 2 * s.F}; break;
+    default: g = StageG{a.d_tiles, 1, a.kb_d, s.D}; break;
+  }
+  return g;
+}
+// Tiles of a stage handled by cluster cl: cl, cl + NC, ...
+__device__ __forceinline__ int cl_tiles(const FlowArgs& a, int ntiles, int cl) {
+  return cl < ntiles ? (ntiles - cl + a.NC - 1) / a.NC : 0;
+}
+// Stored weight row of item (tile t, half) in layer l.
+__device__ __forceinline__ int item_row(const StageG& g, int l, int t, int half) {
+  return l * g.wrows + (g.na == 2 ? 256 * t + 128 * half : 128 * t);
+}
+
+// Attention unit of cluster cl: (request b, KV head g, 128-row query tile
+// qt); this rank's keys [start, end) of the slot.
+struct AttU {
+  bool has;
+  int b, g, bg, qt, start, end, nch;
+};
+__device__ __forceinline__ AttU att_unit(const Shape& s, const FlowArgs& a, int cl, int rank) {
+  AttU u{};
+  u.has = cl < a.a_units;
+  if (!u.has) return u;
+  u.bg = cl / a.a_qtiles;
+  u.qt = cl - u.bg * a.a_qtiles;
+  u.b = u.bg / s.Hkv;
+  u.g = u.bg - u.b * s.Hkv;
+  const int n_valid = __ldg(a.lens + u.b) + s.H;  // set before the launch, fixed during it
+  u.start = rank * a.a_kps;
+  u.end = min(n_valid, u.start + a.a_kps);
+  u.nch = u.end > u.start ? (u.end - u.start + CKF - 1) / CKF : 0;
+  return u;
+}
+
+// Counter words.
+__device__ __forceinline__ unsigned* c_tr(const FlowArgs& a) { return a.ctr + 0; }
+__device__ __forceinline__ unsigned* c_qkv(const FlowArgs& a) { return a.ctr + 1; }
+__device__ __forceinline__ unsigned* c_att(const FlowArgs& a) { return a.ctr + 2; }
+__device__ __forceinline__ unsigned* c_y(const FlowArgs& a, int t) { return a.ctr + 3 + t; }
+__device__ __forceinline__ unsigned* c_ho(const FlowArgs& a, int t) { return a.ctr + 3 + a.d_tiles + t; }
+__device__ __forceinline__ unsigned* c_u(const FlowArgs& a, int p) { return a.ctr + 3 + a.d_tiles + a.o_tiles + p; }
+
+// ------------------------------------------------------------ weight producer
+// Warp 0, lane 0: this CTA's weight blocks in schedule order (per step, layer,
+// stage, item, K block) into the ring; each load also prefetches the same
+// block of the next layer into L2, so HBM streams one layer ahead of the
+// dependency chain.
+__device__ void producer_loop(const FC& c) {
+  const Shape& s = *c.s;
+  const FlowArgs& a = *c.a;
+  const uint64_t pol = policy_evict_first();  // a block is used once per step
+  int n = 0;
+  bool ok = true;
+  for (int k = a.k_begin; ok && k < a.k_end; ++k)
+    for (int l = 0; ok && l < s.L; ++l)
+      for (int st = 0; ok && st < 4; ++st) {
+        const StageG g = stage_geo(s, a, st);
+        const int nt = cl_tiles(a, g.ntiles, c.cl);
+        for (int j = 0; ok && j < nt; ++j) {
+          const int t = c.cl + j * a.NC;
+          for (int half = 0; ok && half < g.na; ++half) {
+            const int row0 = item_row(g, l, t, half);
+            const int nrow = l + 1 < s.L ? row0 + g.wrows : (k + 1 < a.k_end ? row0 - (s.L - 1) * g.wrows : -1);
+            for (int i = 0; i < g.kbr; ++i, ++n) {
+              const int slot = n % kFRing;
+              if (n >= kFRing && !fwait(c, &c.rempty[slot], ((n / kFRing) & 1) ^ 1)) {
+                ok = false;
+                break;
+              }
+              const int x = (c.rank * g.kbr + i) * 64;
+              mbar_arrive_expect_tx(&c.rfull[slot], kFBlk);
+              tma_load_2d_hint(c.ring + (size_t)slot * kFBlk, c.mp.w[st], x, row0, &c.rfull[slot], pol);
+              if (nrow >= 0) tma_prefetch_l2(c.mp.w[st], x, nrow);
+            }
+          }
+        }
+      }
+  // copies still in flight land before the CTA exits
+  for (int j = n > kFRing ? n - kFRing : 0; j < n; ++j)
+    if (!mbar_wait(&c.rfull[j % kFRing], (j / kFRing) & 1, kFDrain)) set_error(a.err, DEV_TIMEOUT);
+}
+
+// ------------------------------------------------------------ MMA issuer
+// Warp 1, lane 0.  Projection item: D[128 rows][64 tokens] (TMEM slot it % 2)
+// = sum over this rank's K blocks of weights [128][64] x operand [64][64]^T.
+// Attention chunk: S = Q K^T (M = 128 query rows, N = 64 keys), then
+// O += P V with P read from TMEM and V MN-major from shared memory.
+__device__ void mma_loop(const FC& c) {
+  const Shape& s = *c.s;
+  const FlowArgs& a = *c.a;
+  const int d = s.d;
+  const uint32_t idg = idesc_bf16(128, 64);
+  const uint32_t ids = idesc_bf16(128, CKF);
+  const uint32_t ido = idesc_bf16(128, d, 0, 1);
+  const uint32_t work = smem_u32(c.work), ring = smem_u32(c.ring);
+  const uint32_t qbytes = 128u * d * 2u, kvbytes = (uint32_t)CKF * d * 2u;
+  const AttU au = att_unit(s, a, c.cl, c.rank);
+  int n = 0, it = 0, sg = 0, ac = 0;
+  bool ok = true;
+  for (int k = a.k_begin; ok && k < a.k_end; ++k)
+    for (int l = 0; ok && l < s.L; ++l)
+      for (int st5 = 0; ok && st5 < 5; ++st5) {
+        if (st5 == 1) {
+          if (!au.has) continue;
+          for (int ch = 0; ch < au.nch; ++ch, ++ac) {
+            if (!fwait(c, c.kv_full, ac & 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            for (int k16 = 0; k16 < d / 16; ++k16) {
+              const uint32_t x = (uint32_t)k16 >> 2, w = ((uint32_t)k16 & 3u) * 32u;
+              umma_bf16(c.tmem + kColS, sw128_desc(work + x * 128u * 128u + w, 16, 1024),
+                        sw128_desc(work + qbytes + x * (uint32_t)CKF * 128u + w, 16, 1024), ids, k16 > 0 ? 1u : 0u);
+            }
+            umma_commit(c.s_full);
+            if (!fwait(c, c.p_full, ac & 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t vd = sw128_desc(work + qbytes + kvbytes, CKF * 128, 1024);
+            for (int k16 = 0; k16 < CKF / 16; ++k16)
+              umma_bf16_tmem_a(c.tmem + kColO, c.tmem + kColS + (uint32_t)k16 * 8u, desc_add(vd, k16 * 16u * 128u), ido,
+                               (ch > 0 || k16 > 0) ? 1u : 0u);
+            umma_commit(c.o_full);
+          }
+          continue;
+        }
+        const int st = st5 == 0 ? ST_Q : st5 - 1;
+        const StageG g = stage_geo(s, a, st);
+        const int nt = cl_tiles(a, g.ntiles, c.cl);
+        if (nt == 0) continue;
+        if (!fwait(c, c.op_full, sg & 1)) {
+          ok = false;
+          break;
+        }
+        ++sg;
+        tc_fence_after();
+        for (int j = 0; ok && j < nt; ++j)
+          for (int half = 0; ok && half < g.na; ++half, ++it) {
+            const int slot = it & 1;
+            if (it >= 2 && !fwait(c, &c.acc_empty[slot], ((it >> 1) & 1) ^ 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            for (int i = 0; i < g.kbr; ++i, ++n) {
+              const int rs = n % kFRing;
+              if (!fwait(c, &c.rfull[rs], (n / kFRing) & 1)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t sa = ring + (uint32_t)rs * kFBlk, sb = work + kFOp + (uint32_t)i * 8192u;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(c.tmem + (uint32_t)slot * 64u, sw128_desc(sa + kk * 32, 16, 1024),
+                          sw128_desc(sb + kk * 32, 16, 1024), idg, (i > 0 || kk > 0) ? 1u : 0u);
+              umma_commit(&c.rempty[rs]);
+            }
+            if (!ok) break;
+            umma_commit(&c.acc_full[slot]);
+          }
+      }
+  if (!ok && !*c.s_abort) raise_abort(c);
+  // every MMA this thread issued must finish before TMEM is freed
+  umma_commit(c.drain);
+  if (!mbar_wait(c.drain, 0, kFDrain)) set_error(a.err, DEV_TIMEOUT);
+}
+
+// ------------------------------------------------------------ compute side
+__device__ __forceinline__ float4 ldcg_f4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ float4 ldg_f4(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ void f4_to(float* v, float4 a, float4 b) {
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ uint4 pack8(const float* v) {
+  return make_uint4(pack_bf2(v[0], v[1]), pack_bf2(v[2], v[3]), pack_bf2(v[4], v[5]), pack_bf2(v[6], v[7]));
+}
+
+// Deterministic sum over the 128 compute threads (fixed tree).
+__device__ float csum(const FC& c, float v) {
+  v = warp_sum(v);
+  const int lane = c.ct & 31, w = c.ct >> 5;
+  csync();
+  if (lane == 0) c.s_tmp[w] = v;
+  csync();
+  return ((c.s_tmp[0] + c.s_tmp[1]) + c.s_tmp[2]) + c.s_tmp[3];
+}
+
+// Epilogue of the QKV projection for 8 stored rows f0.. of token m: rstd and
+// the shift term, then q (head-major) or this step's key / value into the
+// request's slot at position lens[b] + i; rotated heads store their 4 pairs
+// on channels i0.. and i0 + d/2..
+__device__ void epi_q(const FC& c, int k, int l, int m, int f0, const float* acc) {
+  const Shape& s = *c.s;
+  const FlowArgs& a = *c.a;
+  const float* bias = a.bias_qkv + ((size_t)k * s.L + l) * s.qkv_rows + f0;
+  float bv[8];
+  f4_to(bv, ldg_f4(bias), ldg_f4(bias + 4));
+  const float rs = c.s_rstd[m];
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = fmaf(rs, acc[i], bv[i]);
+  const int b = m / s.H, tt = m - b * s.H;
+  const int len = __ldg(a.lens + b);
+  const int qd = s.Hq * s.d, kvd = s.Hkv * s.d;
+  bf16* base;
+  int j;
+  if (f0 < qd) {
+    const int head = f0 / s.d;
+    j = f0 - head * s.d;
+    base = a.q + ((size_t)(b * s.Hq + head) * s.H + tt) * s.d;
+  } else {
+    const bool is_v = f0 >= qd + kvd;
+    const int fk = f0 - qd - (is_v ? kvd : 0);
+    const int g = fk / s.d;
+    j = fk - g * s.d;
+    base = (is_v ? a.vc : a.kc) + (((size_t)(l * s.Bmax + b) * s.Hkv + g) * s.Ptot + len + tt) * s.d;
+  }
+  if (a.rope_cs && f0 < qd + kvd) {
+    const int i0 = j >> 1;
+    float lo[4], hi[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      lo[u] = v[2 * u];
+      hi[u] = v[2 * u + 1];
+      rope_turn(a.rope_cs, s.d, len + tt, i0 + u, lo[u], hi[u]);
+    }
+    *reinterpret_cast<uint2*>(base + i0) = make_uint2(pack_bf2(lo[0], lo[1]), pack_bf2(lo[2], lo[3]));
+    *reinterpret_cast<uint2*>(base + i0 + (s.d >> 1)) = make_uint2(pack_bf2(hi[0], hi[1]), pack_bf2(hi[2], hi[3]));
+  } else {
+    *reinterpret_cast<uint4*>(base + j) = pack8(v);
+  }
+}
+
+// Gated residual for 8 features f0.. of token m: h += gate * acc, then (when
+// `sc` is given) the next norm's operand bf16(h (1 + scale)) and the sum of
+// the 8 squares of h.
+__device__ float epi_resid(const FC& c, int m, int f0, const float* acc, const float* gate, const float* sc,
+                           bf16* ydst) {
+  const Shape& s = *c.s;
+  float* hp = c.a->h + (size_t)m * s.D + f0;
+  float hv[8], gv[8];
+  f4_to(hv, ldcg_f4(hp), ldcg_f4(hp + 4));
+  f4_to(gv, ldg_f4(gate + f0), ldg_f4(gate + f0 + 4));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) hv[i] = fmaf(gv[i], acc[i], hv[i]);
+  reinterpret_cast<float4*>(hp)[0] = make_float4(hv[0], hv[1], hv[2], hv[3]);
+  reinterpret_cast<float4*>(hp)[1] = make_float4(hv[4], hv[5], hv[6], hv[7]);
+  float ss = 0.f;
+  if (sc) {
+    float sv[8], yv[8];
+    f4_to(sv, ldg_f4(sc + f0), ldg_f4(sc + f0 + 4));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      yv[i] = hv[i] * (1.f + sv[i]);
+      ss = fmaf(hv[i], hv[i], ss);
+    }
+    *reinterpret_cast<uint4*>(ydst + (size_t)m * s.D + f0) = pack8(yv);
+  }
+  return ss;
+}
+
+// One projection stage on this CTA.  `it` counts projection items (TMEM
+// slots, partial buffers), `sg` the operand loads compute thread 0 issued,
+// `ncl` cluster barriers.  Returns false once the launch is aborting.
+__device__ bool gemm_stage(const FC& c, int st, int k, int l, int u, int& it, int& sg, int& ncl) {
+  const Shape& s = *c.s;
+  const FlowArgs& a = *c.a;
+  const StageG g = stage_geo(s, a, st);
+  const int nt = cl_tiles(a, g.ntiles, c.cl);
+  if (nt == 0) return true;  // uniform over the cluster
+  const int C = a.C, R = 128 / C, rank = c.rank;
+  const int x0 = rank * g.kbr * 64, x1 = x0 + g.kbr * 64;
+  const unsigned uC = (unsigned)C;
+
+  // 1. the producers of this rank's K slice of the token operand, then its TMA
+  bool ok = true;
+  if (c.ct == 0) {
+    if (st == ST_Q && l == 0) {
+      ok = wait_ctr(c, c_tr(a), (unsigned)(a.M * (k - a.k_begin + 1)));
+    } else {
+      for (int t = x0 / 128; ok && t <= (x1 - 1) / 128; ++t) {
+        if (st == ST_Q) ok = wait_ctr(c, c_y(a, t), uC * (unsigned)u);
+        else if (st == ST_G) ok = wait_ctr(c, c_ho(a, t), uC * (unsigned)(u + 1));
+        else if (st == ST_D) ok = wait_ctr(c, c_u(a, t), uC * (unsigned)(u + 1));
+      }
+      if (st == ST_O) ok = wait_ctr(c, c_att(a), (unsigned)a.a_units * uC * (unsigned)(u + 1));
+    }
+    if (ok) {
+      fence_proxy_async_global_f();  // written by other CTAs' generic stores, read by TMA
+      mbar_arrive_expect_tx(c.op_full, (uint32_t)g.kbr * 8192u);
+      for (int i = 0; i < g.kbr; ++i)
+        tma_load_2d(c.work + kFOp + (size_t)i * 8192, c.mp.x[st], x0 + i * 64, 0, c.op_full);
+      ++sg;  // operand loads issued (drained before exit)
+    }
+  }
+  if (!cand(ok)) return false;
+
+  // 2. QKV and gate/up: rstd per token from the producers' sums of squares
+  //    (all of them: the norm spans every feature), while the MMAs run
+  if (st == ST_Q || st == ST_G) {
+    if (c.ct == 0) {
+      if (st == ST_Q && l > 0)
+        for (int t = 0; ok && t < a.d_tiles; ++t) ok = wait_ctr(c, c_y(a, t), uC * (unsigned)u);
+      if (st == ST_G)
+        for (int t = 0; ok && t < a.o_tiles; ++t) ok = wait_ctr(c, c_ho(a, t), uC * (unsigned)(u + 1));
+    }
+    if (!cand(ok)) return false;
+    const float* ss = st == ST_G ? a.ss_g : (l == 0 ? a.ss_t : a.ss_q);
+    const int nslots = st == ST_G ? a.o_tiles * C : (l == 0 ? 1 : a.d_tiles * C);
+    const int m = c.ct & 63, part = c.ct >> 6;
+    float acc = 0.f;
+    for (int s0 = part; s0 < nslots; s0 += 16) {
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = s0 + 2 * i < nslots ? __ldcg(ss + (size_t)(s0 + 2 * i) * 64 + m) : 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc += v[i];
+    }
+    c.s_tmp[part * 64 + m] = acc;
+    csync();
+    if (c.ct < 64) c.s_rstd[c.ct] = rsqrtf((c.s_tmp[c.ct] + c.s_tmp[64 + c.ct]) / (float)s.D + s.eps);
+    csync();
+  }
+
+  // 3. items: accumulator -> own partial tile -> cluster barrier -> reduce
+  //    this rank's rows over the C partials -> epilogue -> publish
+  const float* tab = a.tables + (size_t)k * s.table_rows;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qd = warp & 3, row = qd * 32 + lane;  // TMEM lane = weight row
+  const int per8 = R / 8, nitems = a.M * per8;
+  float keep[2][8];
+  for (int j = 0; j < nt; ++j) {
+    const int t = c.cl + j * a.NC;
+    for (int half = 0; half < g.na; ++half, ++it) {
+      const int slot = it & 1;
+      if (!cand(fwait(c, &c.acc_full[slot], (it >> 1) & 1))) return false;
+      tc_fence_after();
+      const uint32_t taddr = c.tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)slot * 64u;
+      const uint32_t pbase = smem_u32(c.work + kFPart) + (uint32_t)(it & 1) * 32768u;
+      for (int c0 = 0; c0 < a.M; c0 += 16) {
+        float v[16];
+        tmem_ld16(taddr + (uint32_t)c0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) st_shared_f32(pbase + (uint32_t)(((c0 + jj) * 128 + row) * 4), v[jj]);
+      }
+      tc_fence_before();
+      csync();
+      if (c.ct == 0) mbar_arrive(&c.acc_empty[slot]);
+      if (!cl_sync(c, ncl)) return false;
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        if (pass == 1 && nitems <= 128) break;  // uniform
+        const int idx = c.ct + pass * 128;
+        const bool valid = idx < nitems;
+        const int m = valid ? idx / per8 : 0, j8 = valid ? idx - (idx / per8) * per8 : 0;
+        const int r0 = rank * R + j8 * 8;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+        if (valid) {
+          const uint32_t la = pbase + (uint32_t)((m * 128 + r0) * 4);
+          for (int q = 0; q < C; ++q) {
+            const uint32_t ra = map_cluster(la, (uint32_t)q);
+            const float4 p0 = ld_cluster_f32x4(ra), p1 = ld_cluster_f32x4(ra + 16);
+            acc[0] += p0.x; acc[1] += p0.y; acc[2] += p0.z; acc[3] += p0.w;
+            acc[4] += p1.x; acc[5] += p1.y; acc[6] += p1.z; acc[7] += p1.w;
+          }
+        }
+        const int f0 = 128 * t + r0;
+        if (st == ST_Q) {
+          if (valid) epi_q(c, k, l, m, f0, acc);
+        } else if (st == ST_G) {
+          if (valid) {
+            const float* bias = a.bias_gu + ((size_t)k * s.L + l) * 2 * s.F + 256 * t + 128 * half + r0;
+            float bv[8];
+            f4_to(bv, ldg_f4(bias), ldg_f4(bias + 4));
+            const float rs = c.s_rstd[m];
+            if (half == 0) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) keep[pass][i] = fmaf(rs, acc[i], bv[i]);
+            } else {
+              float ov[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) ov[i] = gelu_tanh_bf16out(keep[pass][i]) * fmaf(rs, acc[i], bv[i]);
+              *reinterpret_cast<uint4*>(a.u + (size_t)m * s.F + f0) = pack8(ov);
+            }
+          }
+        } else {
+          // O: next norm = this layer's MLP norm; D: the next layer's attention norm
+          const bool has_next = st == ST_O || l + 1 < s.L;
+          const float* gate = tab + mod_offset(s, l, st == ST_O ? 0 : 1, 2);
+          const float* sc = !has_next ? nullptr
+                                      : (st == ST_O ? tab + mod_offset(s, l, 1, 0) : tab + mod_offset(s, l + 1, 0, 0));
+          float sq = 0.f;
+          if (valid) sq = epi_resid(c, m, f0, acc, gate, sc, st == ST_O ? a.yg : a.yq);
+          // the per8 threads of one token are adjacent lanes: fixed shuffle tree
+          for (int o = 1; o < per8; o <<= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+          if (valid && j8 == 0 && has_next)
+            (st == ST_O ? a.ss_g : a.ss_q)[(size_t)(t * C + rank) * 64 + m] = sq;
+        }
+      }
+      if (st == ST_Q) publish(c, c_qkv(a));
+      else if (st == ST_O) publish(c, c_ho(a, t));
+      else if (st == ST_G && half == 1) publish(c, c_u(a, t));
+      else if (st == ST_D) publish(c, c_y(a, t));
+    }
+  }
+  return true;
+}
+
+// Attention on the clusters that hold an attention unit: rank r takes keys
+// [r kps, r kps + kps) of the slot in 64-key chunks (online softmax in the
+// log2 domain, thread = query row = TMEM lane), then the C partial outputs are
+// merged in the cluster: rank weights exp2(m_r - M) / L from every rank's row
+// max and sum, each rank parks its weighted rows (fp32, 16-byte chunks
+// swizzled by row), and rank q adds rows [q R, q R + R) of all ranks in rank
+// order.  `ac` counts this CTA's chunks (barrier phases).
+__device__ bool att_stage(const FC& c, int l, int u, int& ac, int& ncl, int& kv_issued) {
+  const Shape& s = *c.s;
+  const FlowArgs& a = *c.a;
+  const AttU au = att_unit(s, a, c.cl, c.rank);
+  if (!au.has) return true;
+  const int d = s.d, nbox = d / 64, GH = s.G * s.H, C = a.C;
+  const uint32_t qbytes = 128u * d * 2u, kvbytes = (uint32_t)CKF * d * 2u;
+  // peers are done reading this CTA's partial tiles of the QKV stage
+  if (!cl_sync(c, ncl)) return false;
+  const int slot_row0 = ((l * s.Bmax + au.b) * s.Hkv + au.g) * s.Ptot;
+  bool ok = true;
+  if (c.ct == 0) {
+    ok = wait_ctr(c, c_qkv(a), (unsigned)(a.q_tiles * C * (u + 1)));
+    if (ok && au.nch > 0) {
+      fence_proxy_async_global_f();
+      mbar_arrive_expect_tx(c.kv_full, qbytes + 2u * kvbytes);
+      const int qrow0 = au.bg * GH + au.qt * 128;
+      for (int x = 0; x < nbox; ++x) tma_load_2d(c.work + (size_t)x * 128 * 128, c.mp.q, x * 64, qrow0, c.kv_full);
+      for (int x = 0; x < nbox; ++x) {
+        tma_load_2d(c.work + qbytes + (size_t)x * CKF * 128, c.mp.k, x * 64, slot_row0 + au.start, c.kv_full);
+        tma_load_2d(c.work + qbytes + kvbytes + (size_t)x * CKF * 128, c.mp.v, x * 64, slot_row0 + au.start,
+                    c.kv_full);
+      }
+      ++kv_issued;
+    }
+  }
+  if (!cand(ok)) return false;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qd = warp & 3, r = qd * 32 + lane;
+  const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+  const float scale_log2 = rsqrtf((float)d) * 1.4426950408889634f;
+  float m_run = -INFINITY, l_run = 0.f;
+  for (int ch = 0; ch < au.nch; ++ch) {
+    const int acn = ac + ch;
+    if (!cand(fwait(c, c.s_full, acn & 1))) return false;
+    tc_fence_after();
+    float sv[CKF];
+#pragma unroll
+    for (int j = 0; j < CKF; j += 16) tmem_ld16(c.tmem + lane_off + kColS + j, sv + j);
+    tmem_ld_wait();
+    const int vc = min(CKF, au.end - (au.start + ch * CKF));
+    float cmax = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < CKF; ++j) {
+      sv[j] = j < vc ? sv[j] * scale_log2 : -INFINITY;
+      cmax = fmaxf(cmax, sv[j]);
+    }
+    // lazy rescaling: the reference max moves only when the row max grows by > 8
+    const float mx = cmax > m_run + 8.f ? cmax : m_run;
+    const float alpha = exp2f(m_run - mx);
+    float psum = 0.f;
+#pragma unroll
+    for (int j = 0; j < CKF; ++j) {
+      sv[j] = exp2f(sv[j] - mx);
+      psum += sv[j];
+    }
+    l_run = l_run * alpha + psum;
+    m_run = mx;
+    // S of this chunk completing implies the previous chunk's PV completed
+    // (one MMA thread, in order): O may be rescaled and P overwritten
+    if (ch > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
+      for (int j = 0; j < d; j += 16) {
+        float ov[16];
+        tmem_ld16(c.tmem + lane_off + kColO + j, ov);
+        tmem_ld_wait();
+#pragma unroll
+        for (int t = 0; t < 16; ++t) ov[t] *= alpha;
+        tmem_st16(c.tmem + lane_off + kColO + j, ov);
+      }
+      tmem_st_wait();
+    }
+    {
+      float pk[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) pk[q] = __uint_as_float(pack_bf2(sv[2 * q], sv[2 * q + 1]));
+      tmem_st16(c.tmem + lane_off + kColS, pk);
+      tmem_st16(c.tmem + lane_off + kColS + 16, pk + 16);
+      tmem_st_wait();
+    }
+    if (vc < CKF) {
+      // masked keys have P = 0, but 0 * (NaN or Inf) in V would still poison O
+      if (!cand(fwait(c, c.kv_full, acn & 1))) return false;
+      uint8_t* vbase = c.work + qbytes + kvbytes;
+      const int rows = CKF - vc;
+      for (int i = c.ct; i < rows * nbox * 8; i += kFCompute) {
+        const int kr = vc + i / (nbox * 8), rem = i % (nbox * 8), x = rem / 8, q = rem % 8;
+        *reinterpret_cast<uint4*>(vbase + (size_t)x * CKF * 128 + kr * 128 + q * 16) = make_uint4(0, 0, 0, 0);
+      }
+      fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    csync();
+    if (c.ct == 0) mbar_arrive(c.p_full);
+    if (ch + 1 < au.nch) {
+      // the next chunk's K and V overwrite this chunk's: wait for its PV
+      if (!cand(fwait(c, c.o_full, acn & 1))) return false;
+      if (c.ct == 0) {
+        mbar_arrive_expect_tx(c.kv_full, 2u * kvbytes);
+        const int krow = slot_row0 + au.start + (ch + 1) * CKF;
+        for (int x = 0; x < nbox; ++x) {
+          tma_load_2d(c.work + qbytes + (size_t)x * CKF * 128, c.mp.k, x * 64, krow, c.kv_full);
+          tma_load_2d(c.work + qbytes + kvbytes + (size_t)x * CKF * 128, c.mp.v, x * 64, krow, c.kv_full);
+        }
+        ++kv_issued;
+      }
+    }
+  }
+  ac += au.nch;
+  if (au.nch > 0 && !cand(fwait(c, c.o_full, (ac - 1) & 1))) return false;
+  tc_fence_after();
+
+  // -------------------------------------------------- merge in the cluster
+  c.s_ml[2 * r] = au.nch > 0 ? m_run : -INFINITY;
+  c.s_ml[2 * r + 1] = au.nch > 0 ? l_run : 0.f;
+  if (!cl_sync(c, ncl)) return false;
+  float Mx = -INFINITY;
+  const uint32_t mla = smem_u32(c.s_ml + 2 * r);
+  for (int q = 0; q < C; ++q) Mx = fmaxf(Mx, ld_cluster_f32(map_cluster(mla, (uint32_t)q)));
+  float Ls = 0.f;
+  for (int q = 0; q < C; ++q) {
+    const uint32_t ra = map_cluster(mla, (uint32_t)q);
+    const float lq = ld_cluster_f32(ra + 4);
+    if (lq > 0.f) Ls = fmaf(exp2f(ld_cluster_f32(ra) - Mx), lq, Ls);
+  }
+  const float w = (au.nch > 0 && l_run > 0.f && Ls > 0.f) ? exp2f(m_run - Mx) / Ls : 0.f;
+  const uint32_t prow = smem_u32(c.work) + (uint32_t)(r * d * 4);
+  for (int j = 0; j < d; j += 16) {
+    float ov[16];
+    if (au.nch > 0) {  // uniform over the CTA
+      tmem_ld16(c.tmem + lane_off + kColO + j, ov);
+      tmem_ld_wait();
+    } else {
+#pragma unroll
+      for (int t = 0; t < 16; ++t) ov[t] = 0.f;
+    }
+#pragma unroll
+    for (int t4 = 0; t4 < 4; ++t4) {
+      const uint32_t ch4 = ((uint32_t)(j / 4 + t4)) ^ (uint32_t)(r & 7);
+      st_shared_f4(prow + ch4 * 16u, make_float4(ov[4 * t4] * w, ov[4 * t4 + 1] * w, ov[4 * t4 + 2] * w,
+                                                 ov[4 * t4 + 3] * w));
+    }
+  }
+  tc_fence_before();
+  if (!cl_sync(c, ncl)) return false;
+  const int R = 128 / C, per_row = d / 4;
+  for (int el = c.ct; el < R * per_row; el += kFCompute) {
+    const int rr = el / per_row, c4 = el - rr * per_row;
+    const int row = c.rank * R + rr, rq = au.qt * 128 + row;
+    if (rq >= GH) continue;
+    const uint32_t la = smem_u32(c.work) + (uint32_t)(row * d * 4) + (((uint32_t)c4 ^ (uint32_t)(row & 7)) * 16u);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < C; ++q) {
+      const float4 v = ld_cluster_f32x4(map_cluster(la, (uint32_t)q));
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    const int hl = rq / s.H, ti = rq - hl * s.H;
+    bf16* orow = a.o + (size_t)(au.b * s.H + ti) * s.attn_dim + (au.g * s.G + hl) * d;
+    *reinterpret_cast<uint2*>(orow + 4 * c4) = make_uint2(pack_bf2(acc.x, acc.y), pack_bf2(acc.z, acc.w));
+  }
+  publish(c, c_att(a));
+  // peers are done reading this CTA's partial before the work area is reused
+  return cl_sync(c, ncl);
+}
+
+// Token transition for token m = this CTA: (end of step k_out) final
+// adaRMSNorm, out_proj, x += dt v; (start of step k_in) h = x W_in^T + b_in,
+// its sum of squares and the first norm's operand bf16(h (1 + scale)).
+__device__ bool transition(const FC& c, int k_out, int k_in) {
+  const Shape& s = *c.s;
+  const FlowArgs& a = *c.a;
+  const int m = c.cta;
+  if (m >= a.M) return true;
+  const int D = s.D, A = s.A;
+  const int tid = c.ct, lane = tid & 31, warp = tid >> 5;
+  constexpr int nw = kFCompute / 32;
+  float* hs = reinterpret_cast<float*>(c.work);  // [D] (the operand area: this CTA's MMAs are done with it)
+  float* xs = hs + D;                            // [A]
+  float* xrow = a.x + (size_t)m * A;
+  if (k_out >= 0) {
+    bool ok = true;
+    if (tid == 0) {
+      const unsigned tgt = (unsigned)a.C * (unsigned)((k_out - a.k_begin) * s.L + s.L);
+      for (int t = 0; ok && t < a.d_tiles; ++t) ok = wait_ctr(c, c_y(a, t), tgt);
+    }
+    if (!cand(ok)) return false;
+    const float* tab = a.tables + (size_t)k_out * s.table_rows;
+    const float* sc = tab + final_offset(s, 0);
+    const float* sh = tab + final_offset(s, 1);
+    const float* hrow = a.h + (size_t)m * D;
+    float ss = 0.f;
+    for (int j = 4 * tid; j < D; j += 4 * kFCompute) {
+      const float4 v = ldcg_f4(hrow + j);
+      *reinterpret_cast<float4*>(hs + j) = v;
+      ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+    }
+    ss = csum(c, ss);
+    const float rr = rsqrtf(ss / (float)D + s.eps);
+    for (int j = 4 * tid; j < D; j += 4 * kFCompute) {
+      float4 v = *reinterpret_cast<const float4*>(hs + j);
+      const float4 cc = ldg_f4(sc + j), dd = ldg_f4(sh + j);
+      v.x = v.x * rr * (1.f + cc.x) + dd.x;
+      v.y = v.y * rr * (1.f + cc.y) + dd.y;
+      v.z = v.z * rr * (1.f + cc.z) + dd.z;
+      v.w = v.w * rr * (1.f + cc.w) + dd.w;
+      *reinterpret_cast<float4*>(hs + j) = v;
+    }
+    csync();
+    // v = y W_out^T + b_out: warp w takes outputs w, w + 4, ...; 8 inputs per lane per 256
+    const float dtk = __ldg(a.dt + k_out);
+    for (int o = warp; o < A; o += nw) {
+      float acc = 0.f;
+      const bf16* wr = a.w_out + (size_t)o * D;
+      for (int j0 = 8 * lane; j0 < D; j0 += 256) {
+        const uint4 wv = __ldg(reinterpret_cast<const uint4*>(wr + j0));
+        const uint32_t wq[4] = {wv.x, wv.y, wv.z, wv.w};
+        const float4 y0 = *reinterpret_cast<const float4*>(hs + j0);
+        const float4 y1 = *reinterpret_cast<const float4*>(hs + j0 + 4);
+        const float yv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          acc = fmaf(yv[2 * t], __uint_as_float(wq[t] << 16), acc);
+          acc = fmaf(yv[2 * t + 1], __uint_as_float(wq[t] & 0xFFFF0000u), acc);
+        }
+      }
+      const float v = warp_sum(acc);
+      if (lane == 0) {
+        const float xn = __ldcg(xrow + o) + dtk * (v + bf2f(a.b_out[o]));
+        xrow[o] = xn;
+        xs[o] = xn;
+      }
+    }
+    csync();
+  } else {
+    for (int o = tid; o < A; o += kFCompute) xs[o] = __ldcg(xrow + o);
+    csync();
+  }
+  if (k_in >= 0) {
+    const float* sc0 = a.tables + (size_t)k_in * s.table_rows + mod_offset(s, 0, 0, 0);
+    float* hrow = a.h + (size_t)m * D;
+    float ss = 0.f;
+    for (int j = 4 * tid; j < D; j += 4 * kFCompute) {
+      float acc[4];
+      {
+        const uint2 bv = __ldg(reinterpret_cast<const uint2*>(a.b_in + j));
+        acc[0] = __uint_as_float(bv.x << 16);
+        acc[1] = __uint_as_float(bv.x & 0xFFFF0000u);
+        acc[2] = __uint_as_float(bv.y << 16);
+        acc[3] = __uint_as_float(bv.y & 0xFFFF0000u);
+      }
+      for (int o = 0; o < A; ++o) {
+        const uint2 wv = __ldg(reinterpret_cast<const uint2*>(a.w_inT + (size_t)o * D + j));
+        const float xv = xs[o];
+        acc[0] = fmaf(xv, __uint_as_float(wv.x << 16), acc[0]);
+        acc[1] = fmaf(xv, __uint_as_float(wv.x & 0xFFFF0000u), acc[1]);
+        acc[2] = fmaf(xv, __uint_as_float(wv.y << 16), acc[2]);
+        acc[3] = fmaf(xv, __uint_as_float(wv.y & 0xFFFF0000u), acc[3]);
+      }
+      *reinterpret_cast<float4*>(hrow + j) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      const float4 cc = ldg_f4(sc0 + j);
+      *reinterpret_cast<uint2*>(a.yq + (size_t)m * D + j) =
+          make_uint2(pack_bf2(acc[0] * (1.f + cc.x), acc[1] * (1.f + cc.y)),
+                     pack_bf2(acc[2] * (1.f + cc.z), acc[3] * (1.f + cc.w)));
+      ss = fmaf(acc[0], acc[0], fmaf(acc[1], acc[1], fmaf(acc[2], acc[2], fmaf(acc[3], acc[3], ss))));
+    }
+    ss = csum(c, ss);
+    if (tid == 0) a.ss_t[m] = ss;
+  }
+  publish(c, c_tr(a));
+  csync();  // the work area is reused by the next stage
+  return true;
+}
+
+__device__ void compute_loop(const FC& c) {
+  const Shape& s = *c.s;
+  const FlowArgs& a = *c.a;
+  int it = 0, sg = 0, ac = 0, ncl = 0, kv_issued = 0;
+  bool ok = transition(c, -1, a.k_begin);
+  for (int k = a.k_begin; ok && k < a.k_end; ++k) {
+    for (int l = 0; ok && l < s.L; ++l) {
+      const int u = (k - a.k_begin) * s.L + l;
+      ok = gemm_stage(c, ST_Q, k, l, u, it, sg, ncl) && att_stage(c, l, u, ac, ncl, kv_issued) &&
+           gemm_stage(c, ST_O, k, l, u, it, sg, ncl) && gemm_stage(c, ST_G, k, l, u, it, sg, ncl) &&
+           gemm_stage(c, ST_D, k, l, u, it, sg, ncl);
+    }
+    if (ok) ok = transition(c, k, k + 1 < a.k_end ? k + 1 : -1);
+  }
+  // after an abort, copies this CTA issued may still be in flight: let them land
+  if (c.ct == 0) {
+    if (sg > 0 && !mbar_wait(c.op_full, (sg - 1) & 1, kFDrain)) set_error(a.err, DEV_TIMEOUT);
+    if (kv_issued > 0 && !mbar_wait(c.kv_full, (kv_issued - 1) & 1, kFDrain)) set_error(a.err, DEV_TIMEOUT);
+  }
+}
+
+__global__ void __launch_bounds__(kFThreads, 1)
+    k_flow(const __grid_constant__ CUtensorMap tmWq, const __grid_constant__ CUtensorMap tmWo,
+           const __grid_constant__ CUtensorMap tmWg, const __grid_constant__ CUtensorMap tmWd,
+           const __grid_constant__ CUtensorMap tmYq, const __grid_constant__ CUtensorMap tmO,
+           const __grid_constant__ CUtensorMap tmYg, const __grid_constant__ CUtensorMap tmU,
+           const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Shape s,
+           const __grid_constant__ FlowArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* misc = smem + kFRing * kFBlk + kFWork;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(misc);
+  FC c{};
+  c.s = &s;
+  c.a = &a;
+  c.mp.w[0] = &tmWq;
+  c.mp.w[1] = &tmWo;
+  c.mp.w[2] = &tmWg;
+  c.mp.w[3] = &tmWd;
+  c.mp.x[0] = &tmYq;
+  c.mp.x[1] = &tmO;
+  c.mp.x[2] = &tmYg;
+  c.mp.x[3] = &tmU;
+  c.mp.q = &tmQ;
+  c.mp.k = &tmK;
+  c.mp.v = &tmV;
+  c.ring = smem;
+  c.work = smem + kFRing * kFBlk;
+  c.rfull = bar;
+  c.rempty = bar + kFRing;
+  c.op_full = bar + 2 * kFRing;
+  c.acc_full = bar + 2 * kFRing + 1;   // [2]
+  c.acc_empty = bar + 2 * kFRing + 3;  // [2]
+  c.kv_full = bar + 2 * kFRing + 5;
+  c.s_full = bar + 2 * kFRing + 6;
+  c.p_full = bar + 2 * kFRing + 7;
+  c.o_full = bar + 2 * kFRing + 8;
+  c.cbar = bar + 2 * kFRing + 9;       // [2]
+  c.drain = bar + 2 * kFRing + 11;
+  constexpr int kNBar = 2 * kFRing + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 256);
+  c.s_abort = reinterpret_cast<volatile int*>(misc + 260);
+  c.s_flag = reinterpret_cast<volatile int*>(misc + 264);
+  c.s_rstd = reinterpret_cast<float*>(misc + 512);   // [64]
+  c.s_tmp = reinterpret_cast<float*>(misc + 768);    // [256]
+  c.s_ml = reinterpret_cast<float*>(misc + 1792);    // [128][2]
+  c.cta = blockIdx.x;
+  c.rank = (int)cluster_rank();
+  c.cl = blockIdx.x / a.C;
+  c.ct = (int)threadIdx.x - 64;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kNBar; ++i) mbar_init(&bar[i], (i == 2 * kFRing + 9 || i == 2 * kFRing + 10) ? a.C : 1);
+    *c.s_abort = 0;
+    *c.s_flag = 0;
+    fence_mbar_init();
+    for (int i = 0; i < 4; ++i) {
+      tma_prefetch_desc(c.mp.w[i]);
+      tma_prefetch_desc(c.mp.x[i]);
+    }
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kFTmem);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  c.tmem = *tmem_slot;
+  hw_cluster_sync();  // every rank's mbarriers exist before any remote arrive
+
+  if (warp == 0) {
+    if (lane == 0) producer_loop(c);
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) mma_loop(c);
+    __syncwarp();
+  } else {
+    compute_loop(c);
+  }
+  tc_fence_before();
+  __syncthreads();
+  hw_cluster_sync();  // no CTA leaves while a peer may still read its shared memory
+  if (warp == 0) tmem_dealloc(c.tmem, kFTmem);
+}
+
+}  // namespace
+
+size_t flow_smem_bytes() { return kFSmem; }
+
+cudaError_t flow_init() {
+  cudaError_t e = cudaFuncSetAttribute(k_flow, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFSmem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_flow, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
+}
+
+static void flow_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, int C, int NC, cudaStream_t st) {
+  cfg = cudaLaunchConfig_t{};
+  cfg.gridDim = dim3(NC * C);
+  cfg.blockDim = dim3(kFThreads);
+  cfg.dynamicSmemBytes = kFSmem;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+}
+
+int flow_max_clusters(int C) {
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[2];
+  flow_config(cfg, attr, C, 1, nullptr);
+  cfg.numAttrs = 1;  // occupancy of the cluster shape alone
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, k_flow, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+cudaError_t launch_flow(const Shape& s, const CUtensorMap* maps, const FlowArgs& a, cudaStream_t st) {
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[2];
+  flow_config(cfg, attr, a.C, a.NC, st);
+  return cudaLaunchKernelEx(&cfg, k_flow, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], maps[7],
+                            maps[8], maps[9], maps[10], s, a);
+}
+
+}  // namespace pae

@@ -10,6 +10,8 @@
 // The modulation rows are stacked [layer][norm][scale|shift|gate][D] followed by
 // the final norm's [scale|shift][D].  All weights for all steps are read once
 // (a batched GEMV with K columns); results are fp32.
+#include <algorithm>
+
 #include "internal.h"
 
 namespace pae {
@@ -91,7 +93,60 @@ void gemv(const void* W, const void* b, const float* in, int K, int R, int D, in
                                                      K, R, D, swish_out, out);
 }
 
+// The adaRMSNorm shift folded through a projection, for the small-batch
+// dataflow loop: for every step k, layer l and stored weight row r of that
+// layer, out[k][l][r] = W_l[r] . shift_k(l, norm).  (The loop applies the norm
+// as rstd * (W (h * (1 + scale))) + W shift, the same value with the shift
+// term read from here.)  One block per (layer, group of rows); the shift
+// vectors of KC steps are staged in shared memory; one warp per row.
+__global__ void k_shift_bias(const bf16* __restrict__ W, int rows, int D, int L, const float* __restrict__ tables,
+                             int table_rows, int norm, int K, float* __restrict__ out) {
+  extern __shared__ float xs[];  // [KC][D]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int bpl = (gridDim.x + L - 1) / L;  // blocks per layer
+  const int l = blockIdx.x / bpl, b = blockIdx.x - l * bpl;
+  if (l >= L) return;
+  const int shift_off = ((l * 2 + norm) * 3 + 1) * D;
+  for (int k0 = 0; k0 < K; k0 += KC) {
+    const int kc = min(KC, K - k0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kc * D; i += blockDim.x) {
+      const int j = i / D, c = i - j * D;
+      xs[i] = tables[(size_t)(k0 + j) * table_rows + shift_off + c];
+    }
+    __syncthreads();
+    for (int r = b * nw + warp; r < rows; r += bpl * nw) {
+      float acc[KC];
+#pragma unroll
+      for (int j = 0; j < KC; ++j) acc[j] = 0.f;
+      const bf16* wr = W + ((size_t)l * rows + r) * D;
+      for (int i = lane; i < D; i += 32) {
+        const float w = bf2f(wr[i]);
+#pragma unroll
+        for (int j = 0; j < KC; ++j)
+          if (j < kc) acc[j] = fmaf(w, xs[j * D + i], acc[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < KC; ++j)
+        if (j < kc) {
+          const float v = warp_sum(acc[j]);
+          if (lane == 0) out[((size_t)(k0 + j) * L + l) * rows + r] = v;
+        }
+    }
+  }
+}
+
 }  // namespace
+
+void launch_shift_bias(const Shape& s, const void* W, int rows, int norm, const float* tables, int K, float* out,
+                       cudaStream_t st) {
+  const int bpl = std::max(1, std::min(64, (rows + 63) / 64));
+  const size_t smem = (size_t)KC * s.D * sizeof(float);
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(k_shift_bias, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  k_shift_bias<<<bpl * s.L, 256, smem, st>>>(static_cast<const bf16*>(W), rows, s.D, s.L, tables, s.table_rows, norm,
+                                             K, out);
+}
 
 void launch_time_mlp(const Shape& s, int act_bf16, const double* t, int K, const void* w_t1, const void* b_t1,
                      const void* w_t2, const void* b_t2, float* emb, float* zbuf, float* cbuf, float* dt,

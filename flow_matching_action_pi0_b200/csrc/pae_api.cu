@@ -57,6 +57,8 @@ struct Plan {
   AttnPlan attn{};
   bool persist = false;  // eligible for the persistent kernel
   PersistArgs pa{};
+  bool flow = false;       // eligible for the dataflow loop (clusters, per-tile counters)
+  FlowArgs fa{};
   bool fuse_norm = false;  // QKV / gate-up normalise their fp32 operand in-kernel
   // token-operand maps; a map's box height is the token tile of the projection
   // that reads it (QKV and gate/up may tile the same y differently)
@@ -146,6 +148,17 @@ struct pae_ctx {
   float* pw_part = nullptr;
   float* pw_ss = nullptr;
   unsigned* pw_ctr = nullptr;
+  // dataflow loop (batch * chunk <= 64): the MLP norm's operand, sums of
+  // squares, the projected adaRMSNorm shifts per step, counters, 64-row maps
+  bool flow_capable = false;
+  bool use_flow = true;
+  int flow_cluster = 0;          // 0: automatic
+  int flow_max_cl[17] = {};      // clusters of C CTAs that fit at once
+  void* yg = nullptr;
+  float *f_ssq = nullptr, *f_ssg = nullptr, *f_sst = nullptr;
+  float *bias_qkv = nullptr, *bias_gu = nullptr;
+  unsigned* f_ctr = nullptr;
+  CUtensorMap tmYq64{}, tmYg64{}, tmO64{}, tmU64{};
   // in-kernel adaRMSNorm: per-token sum-of-squares slots [kSsSlots][ss_ld]
   bool use_fused_norm = false;  // opt-in: measured slower than the norm kernels under PDL
   float* ss_buf = nullptr;
@@ -474,6 +487,78 @@ bool plan_persistent(const pae_ctx* ctx, int B, PersistArgs* pa) {
   return true;
 }
 
+// Dataflow-loop plan for M = B*H <= 64 tokens (bf16 weights): the cluster
+// size C must split every projection's K range into whole 64-wide blocks per
+// rank with the token operand slice within 64 KB; the grid is as many
+// clusters of C as fit at once (one CTA per SM), which must cover the
+// attention units (request, KV head, 128 query rows) and the M token CTAs of
+// the transition.  Among the sizes that fit, the one with the most CTAs (ties:
+// the larger C).  Returns false when the batch or shape is not eligible.
+bool plan_flow(const pae_ctx* ctx, int B, FlowArgs* fa) {
+  const Shape& s = ctx->s;
+  const int M = B * s.H;
+  if (!ctx->flow_capable || M < 1 || M > 64) return false;
+  const int nkD = s.D / 64, nkA = s.attn_dim / 64, nkF = s.F / 64;
+  const int qtiles = (s.G * s.H + 127) / 128;
+  const int units = B * s.Hkv * qtiles;
+  if (3 + 2 * (s.D / 128) + s.F / 128 + 1 > kFlowCtrWords) return false;
+  if (s.d > 256 || 128 * s.d * 2 + 2 * 64 * s.d * 2 > 128 * 1024) return false;
+  int bestC = 0, bestNC = 0;
+  for (int C : {16, 8, 4, 2}) {
+    if (ctx->flow_cluster && C != ctx->flow_cluster) continue;
+    if (nkD % C || nkA % C || nkF % C) continue;
+    if ((nkF / C) * 8192 > 64 * 1024 || (nkA / C) * 8192 > 64 * 1024 || (nkD / C) * 8192 > 64 * 1024) continue;
+    const int NC = std::min(ctx->flow_max_cl[C], 148 / C);
+    if (NC < units || NC * C < M) continue;
+    if (NC * C > bestNC * bestC) {
+      bestC = C;
+      bestNC = NC;
+    }
+  }
+  if (!bestC) return false;
+  *fa = FlowArgs{};
+  fa->M = M;
+  fa->B = B;
+  fa->C = bestC;
+  fa->NC = bestNC;
+  fa->q_tiles = s.qkv_rows / 128;
+  fa->o_tiles = s.D / 128;
+  fa->g_pairs = s.F / 128;
+  fa->d_tiles = s.D / 128;
+  fa->kb_q = nkD / bestC;
+  fa->kb_o = nkA / bestC;
+  fa->kb_g = nkD / bestC;
+  fa->kb_d = nkF / bestC;
+  fa->a_units = units;
+  fa->a_qtiles = qtiles;
+  const int chunks = (s.Ptot + 63) / 64;
+  fa->a_kps = 64 * ((chunks + bestC - 1) / bestC);
+  fa->x = ctx->x;
+  fa->h = ctx->h;
+  fa->yq = static_cast<bf16*>(ctx->y);
+  fa->yg = static_cast<bf16*>(ctx->yg);
+  fa->q = static_cast<bf16*>(ctx->q);
+  fa->o = static_cast<bf16*>(ctx->o);
+  fa->u = static_cast<bf16*>(ctx->u);
+  fa->kc = static_cast<bf16*>(ctx->kc);
+  fa->vc = static_cast<bf16*>(ctx->vc);
+  fa->lens = ctx->lens_dev;
+  fa->tables = ctx->tables;
+  fa->dt = ctx->dt;
+  fa->bias_qkv = ctx->bias_qkv;
+  fa->bias_gu = ctx->bias_gu;
+  fa->ss_q = ctx->f_ssq;
+  fa->ss_g = ctx->f_ssg;
+  fa->ss_t = ctx->f_sst;
+  fa->w_inT = static_cast<const bf16*>(ctx->w_inT);
+  fa->b_in = static_cast<const bf16*>(ctx->b_in);
+  fa->w_out = static_cast<const bf16*>(ctx->w_out);
+  fa->b_out = static_cast<const bf16*>(ctx->b_out);
+  fa->rope_cs = ctx->rope_cs;
+  fa->ctr = ctx->f_ctr;
+  return true;
+}
+
 // The launch shapes of one batch size (tensor-core modes): host arithmetic
 // only, shared by the context and pae_plan_query.
 struct LaunchPlans {
@@ -506,6 +591,7 @@ pae_status build_plan(pae_ctx* ctx, int B, Plan* P) {
   P->M = B * s.H;
   if (!ctx->act_bf16) return PAE_OK;
   P->persist = plan_persistent(ctx, B, &P->pa);
+  P->flow = plan_flow(ctx, B, &P->fa);
   const LaunchPlans LP = plan_launches(s, B, ctx->w4 != 0, ctx->max_splitk, ctx->use_fused_norm);
   P->qkv = LP.qkv;
   P->o = LP.o;
@@ -771,6 +857,29 @@ pae_status check_rows(pae_ctx* ctx, int batch) {
 }
 
 bool use_persist(const pae_ctx* ctx, const Plan* P) { return ctx->use_persistent && P->persist; }
+bool use_flow(const pae_ctx* ctx, const Plan* P) { return ctx->use_flow && P->flow && !use_persist(ctx, P); }
+
+// Steps k_begin..k_end-1 (and the final Euler update) as one dataflow launch.
+pae_status enqueue_flow(pae_ctx* ctx, Plan* P, int k_begin, int k_end, cudaStream_t st) {
+  FlowArgs fa = P->fa;
+  fa.k_begin = k_begin;
+  fa.k_end = k_end;
+  fa.err = DevErr{ctx->err_dev, ctx->wait_ns};
+  const CUtensorMap maps[11] = {ctx->tmWqkv, ctx->tmWo,   ctx->tmWgu1, ctx->tmWdown, ctx->tmYq64, ctx->tmO64,
+                                ctx->tmYg64, ctx->tmU64,  ctx->tmQ,    ctx->tmK,     ctx->tmV};
+  P->recs.clear();
+  ctx->rec_sink = &P->recs;
+  ctx->ev_next = 0;
+  CK(cudaMemsetAsync(ctx->f_ctr, 0, sizeof(unsigned) * kFlowCtrWords, st));
+  cudaError_t e;
+  {
+    ProfScope ps(ctx, PAE_K_DATAFLOW, st);
+    e = launch_flow(ctx->s, maps, fa, st);
+  }
+  ctx->rec_sink = nullptr;
+  if (e != cudaSuccess) return fail(ctx, PAE_ERR_CUDA, "dataflow launch: %s", cudaGetErrorString(e));
+  return PAE_OK;
+}
 
 // Steps k_begin..k_end-1 (and the final Euler update) as one persistent launch.
 pae_status enqueue_persistent(pae_ctx* ctx, Plan* P, int k_begin, int k_end, cudaStream_t st) {
@@ -798,6 +907,7 @@ pae_status run_loop(pae_ctx* ctx, Plan* P, cudaStream_t stream) {
   if (pst != PAE_OK) return pst;
   ctx->last_plan = P;
   if (use_persist(ctx, P)) return enqueue_persistent(ctx, P, 0, ctx->K, stream);
+  if (use_flow(ctx, P)) return enqueue_flow(ctx, P, 0, ctx->K, stream);
   if (!ctx->use_graph) {
     P->recs.clear();
     ctx->rec_sink = &P->recs;
@@ -1207,6 +1317,24 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
     ALLOC(ctx->pw_ss, sizeof(float) * kPersistGroups * 64);
     ALLOC(ctx->pw_ctr, sizeof(unsigned) * kPersistCtrWords);
   }
+  if (ctx->act_bf16 && !ctx->w4) {
+    // dataflow loop: buffers, 64-row operand maps, occupancy of each cluster size
+    ctx->flow_capable = true;
+    CKC(flow_init());
+    for (int C : {2, 4, 8, 16}) ctx->flow_max_cl[C] = flow_max_clusters(C);
+    ALLOC(ctx->yg, Mpad * D * es);
+    CKC(cudaMemsetAsync(ctx->yg, 0, Mpad * D * es, cs));
+    ALLOC(ctx->f_ssq, sizeof(float) * (size_t)(D / 128) * 16 * 64);
+    ALLOC(ctx->f_ssg, sizeof(float) * (size_t)(D / 128) * 16 * 64);
+    ALLOC(ctx->f_sst, sizeof(float) * 64);
+    ALLOC(ctx->bias_qkv, sizeof(float) * (size_t)kMaxSteps * L * s.qkv_rows);
+    ALLOC(ctx->bias_gu, sizeof(float) * (size_t)kMaxSteps * L * 2 * F);
+    ALLOC(ctx->f_ctr, sizeof(unsigned) * kFlowCtrWords);
+    if ((st = make_map(ctx, &ctx->tmYq64, ctx->y, D, Mmax, 64, 64)) != PAE_OK) return bail(st);
+    if ((st = make_map(ctx, &ctx->tmYg64, ctx->yg, D, Mmax, 64, 64)) != PAE_OK) return bail(st);
+    if ((st = make_map(ctx, &ctx->tmO64, ctx->o, s.attn_dim, Mmax, 64, 64)) != PAE_OK) return bail(st);
+    if ((st = make_map(ctx, &ctx->tmU64, ctx->u, F, Mmax, 64, 64)) != PAE_OK) return bail(st);
+  }
   if (ctx->act_bf16) {
     CKC(attn_tc_init());
     const uint64_t kv_rows = (uint64_t)L * s.Bmax * s.Hkv * s.Ptot;
@@ -1316,6 +1444,11 @@ pae_status pae_precompute_tables(pae_ctx* ctx, const double* t, int K, pae_strea
   launch_time_mlp(ctx->s, ctx->act_bf16, ctx->t_dev, K, ctx->w_t1, ctx->b_t1, ctx->w_t2, ctx->b_t2, ctx->emb,
                   ctx->zbuf, ctx->cbuf, ctx->dt, stm);
   launch_mod_tables(ctx->s, ctx->act_bf16, ctx->cbuf, K, ctx->w_modall, ctx->b_modall, ctx->tables, stm);
+  if (ctx->flow_capable) {
+    // the adaRMSNorm shifts projected through W_qkv and W_gate/up, per step and layer
+    launch_shift_bias(ctx->s, ctx->w_qkv, ctx->s.qkv_rows, 0, ctx->tables, K, ctx->bias_qkv, stm);
+    launch_shift_bias(ctx->s, ctx->w_gu, 2 * ctx->s.F, 1, ctx->tables, K, ctx->bias_gu, stm);
+  }
   CK(cudaGetLastError());
   if (K != ctx->K) drop_graphs(ctx);
   ctx->K = K;
@@ -1372,6 +1505,8 @@ pae_status pae_denoise_steps(pae_ctx* ctx, const float* x_in, float* x_out, int 
   ctx->last_plan = P;
   if (use_persist(ctx, P)) {
     if ((st = enqueue_persistent(ctx, P, k_begin, k_end, stm)) != PAE_OK) return st;
+  } else if (use_flow(ctx, P)) {
+    if ((st = enqueue_flow(ctx, P, k_begin, k_end, stm)) != PAE_OK) return st;
   } else {
     P->recs.clear();
     ctx->rec_sink = &P->recs;
@@ -1406,6 +1541,17 @@ pae_status pae_set_option(pae_ctx* ctx, int option, long long value) {
       ctx->use_pdl = value != 0;
       return PAE_OK;
     case PAE_OPT_PERSISTENT: ctx->use_persistent = value != 0; return PAE_OK;
+    case PAE_OPT_DATAFLOW: ctx->use_flow = value != 0; return PAE_OK;
+    case PAE_OPT_DATAFLOW_CLUSTER:
+      if (value != 0 && value != 2 && value != 4 && value != 8 && value != 16)
+        return fail(ctx, PAE_ERR_ARG, "dataflow cluster size must be 0 (automatic), 2, 4, 8 or 16");
+      if ((int)value != ctx->flow_cluster) {
+        drop_graphs(ctx);
+        ctx->plans.clear();
+        ctx->last_plan = nullptr;
+      }
+      ctx->flow_cluster = (int)value;
+      return PAE_OK;
     case PAE_OPT_FUSED_NORM:
       if ((value != 0) != ctx->use_fused_norm) {
         drop_graphs(ctx);
@@ -1455,6 +1601,7 @@ pae_status pae_query(pae_ctx* ctx, int what, int batch, long long* value) {
     case PAE_Q_ATTN_SPLITS: *value = P->attn.splits; return PAE_OK;
     case PAE_Q_PERSISTENT: *value = use_persist(ctx, P) ? 1 : 0; return PAE_OK;
     case PAE_Q_FUSED_NORM: *value = P->fuse_norm ? 1 : 0; return PAE_OK;
+    case PAE_Q_DATAFLOW: *value = use_flow(ctx, P) ? P->fa.C : 0; return PAE_OK;
     default: return fail(ctx, PAE_ERR_ARG, "unknown query %d", what);
   }
 }

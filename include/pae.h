@@ -201,14 +201,26 @@ pae_status pae_denoise_steps(pae_ctx* ctx, const float* x_in, float* x_out, int 
  * projections apply the adaRMSNorm to their fp32 input inside the kernel
  * (statistics from the residual projections' epilogues) instead of separate
  * norm kernels, for batches of at most one 64-token tile.  Both round within
- * the parity tolerance; each is bitwise reproducible. */
+ * the parity tolerance; each is bitwise reproducible.
+ * PAE_OPT_DATAFLOW (default 1, bf16 weights): batches with batch * chunk <= 64
+ * run all K steps as one launch of thread-block clusters whose stages wait on
+ * per-tile counters instead of kernel boundaries (no CUDA graph for these
+ * batches; pae_denoise_steps takes the same path).  0 uses the captured graph
+ * of per-stage kernels.  The two paths round differently (the dataflow loop
+ * applies each adaRMSNorm's 1/rms after the projection and its shift as a
+ * precomputed projected term); both stay within the parity tolerance and each
+ * is bitwise reproducible.  PAE_OPT_DATAFLOW_CLUSTER (default 0 = automatic):
+ * force the cluster size (2, 4, 8 or 16) of the dataflow loop; a batch it
+ * does not fit runs the graph. */
 enum {
   PAE_OPT_USE_GRAPH = 1,
   PAE_OPT_WAIT_LIMIT_US = 2,
   PAE_OPT_PDL = 4,
   PAE_OPT_MAX_SPLITK = 5,
   PAE_OPT_PERSISTENT = 6,
-  PAE_OPT_FUSED_NORM = 7
+  PAE_OPT_FUSED_NORM = 7,
+  PAE_OPT_DATAFLOW = 8,
+  PAE_OPT_DATAFLOW_CLUSTER = 9
 };
 pae_status pae_set_option(pae_ctx* ctx, int option, long long value);
 
@@ -222,7 +234,8 @@ enum {
   PAE_K_GATEUP = 5,     /* GeGLU gate/up projection                                   */
   PAE_K_DOWN = 6,       /* down projection, gated residual                            */
   PAE_K_PERSISTENT = 7, /* the whole loop as one persistent kernel (small batches)    */
-  PAE_K_COUNT = 8
+  PAE_K_DATAFLOW = 8,   /* the whole loop as one launch of clusters (small batches)   */
+  PAE_K_COUNT = 9
 };
 /* PAE_OPT_PROFILE (default 0): bit mask of PAE_K_* classes.  Launches of those
  * classes are bracketed by CUDA events on their stream (inside the captured
@@ -239,14 +252,17 @@ pae_status pae_profile_read(pae_ctx* ctx, int kernel_class, double* total_ms, in
  * of the attention for `batch`.  PAE_Q_PERSISTENT: 1 if pae_denoise runs the
  * persistent kernel for `batch` (option on and the batch eligible), else 0.
  * PAE_Q_FUSED_NORM: 1 if the graph for `batch` normalises inside the
- * projections (no separate norm kernels), else 0. */
+ * projections (no separate norm kernels), else 0.  PAE_Q_DATAFLOW: the
+ * cluster size of the dataflow loop pae_denoise runs for `batch` (0: it runs
+ * the graph or the persistent kernel). */
 enum {
   PAE_Q_GRAPH_KERNELS = 1,
   PAE_Q_SPLITS = 2,
   PAE_Q_TOKEN_TILE = 3,
   PAE_Q_ATTN_SPLITS = 4,
   PAE_Q_PERSISTENT = 5,
-  PAE_Q_FUSED_NORM = 6
+  PAE_Q_FUSED_NORM = 6,
+  PAE_Q_DATAFLOW = 7
 };
 pae_status pae_query(pae_ctx* ctx, int what, int batch, long long* value);
 
