@@ -17,16 +17,19 @@ namespace pae {
 typedef __nv_bfloat16 bf16;
 
 // Error word values written by kernels (host maps them to pae_status).
-enum : int { DEV_OK = 0, DEV_TIMEOUT = 5, DEV_BAD_SHAPE = 6 };
+// DEV_DRAIN: a wait for copies or MMAs already issued (the bounded drain
+// before a CTA exits) ran out; the context cannot be trusted afterwards.
+enum : int { DEV_OK = 0, DEV_TIMEOUT = 5, DEV_BAD_SHAPE = 6, DEV_DRAIN = 7 };
 
 struct DevErr {
   int* word;          // host-mapped pinned int; 0 = no error
   long long wait_ns;  // bound of every device-side wait
 };
 
+// The most severe code wins (DEV_DRAIN over DEV_TIMEOUT).
 __device__ __forceinline__ void set_error(const DevErr& e, int code) {
   if (e.word) {
-    atomicCAS(e.word, 0, code);
+    atomicMax(e.word, code);
     __threadfence_system();
   }
 }

@@ -195,9 +195,9 @@ __global__ void __launch_bounds__(384, 1)
       for (int x = 0; x < nbox; ++x) tma_load_2d(smem + L.k_off(st) + x * CK * 128, &tmK, x * 64, krow, &k_full[st]);
       issued = c + 1;
     }
-    if (!mbar_wait(q_full, 0, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
+    if (!mbar_wait(q_full, 0, kDrainNs)) set_error(a.err, DEV_DRAIN);
     for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c)
-      if (!mbar_wait(&k_full[c & 1], (c >> 1) & 1, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
+      if (!mbar_wait(&k_full[c & 1], (c >> 1) & 1, kDrainNs)) set_error(a.err, DEV_DRAIN);
   }
   if (warp == 6 && lane == 0 && nch > 0) {
     const uint32_t kvbytes = CK * d * 2;
@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(384, 1)
       issued = c + 1;
     }
     for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c)
-      if (!mbar_wait(&v_full[c & 1], (c >> 1) & 1, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
+      if (!mbar_wait(&v_full[c & 1], (c >> 1) & 1, kDrainNs)) set_error(a.err, DEV_DRAIN);
   }
 
   // ------------------------------------------------------------ MMA (warp 5)
@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     // every MMA this thread issued must finish before TMEM is freed
     umma_commit(drain);
-    if (!mbar_wait(drain, 0, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
+    if (!mbar_wait(drain, 0, kDrainNs)) set_error(a.err, DEV_DRAIN);
   }
   __syncwarp();
 

@@ -155,7 +155,7 @@ struct FC {
   uint64_t* cbar;      // [2] cluster barrier (count C), alternating instances
   uint64_t* drain;
   float* s_rstd;       // [64]
-  float* s_tmp;        // [256]
+  float* s_tmp;        // [512]
   float* s_ml;         // [128][2] attention row max / sum
   volatile int* s_abort;
   volatile int* s_flag;
@@ -344,7 +344,7 @@ __device__ void producer_loop(const FC& c) {
       }
   // copies still in flight land before the CTA exits
   for (int j = n > kFRing ? n - kFRing : 0; j < n; ++j)
-    if (!mbar_wait(&c.rfull[j % kFRing], (j / kFRing) & 1, kFDrain)) set_error(a.err, DEV_TIMEOUT);
+    if (!mbar_wait(&c.rfull[j % kFRing], (j / kFRing) & 1, kFDrain)) set_error(a.err, DEV_DRAIN);
 }
 
 // ------------------------------------------------------------ MMA issuer
@@ -433,7 +433,7 @@ __device__ void mma_loop(const FC& c) {
   if (!ok && !*c.s_abort) raise_abort(c);
   // every MMA this thread issued must finish before TMEM is freed
   umma_commit(c.drain);
-  if (!mbar_wait(c.drain, 0, kFDrain)) set_error(a.err, DEV_TIMEOUT);
+  if (!mbar_wait(c.drain, 0, kFDrain)) set_error(a.err, DEV_DRAIN);
 }
 
 // ------------------------------------------------------------ compute side
@@ -461,12 +461,9 @@ __device__ float csum(const FC& c, float v) {
 // the shift term, then q (head-major) or this step's key / value into the
 // request's slot at position lens[b] + i; rotated heads store their 4 pairs
 // on channels i0.. and i0 + d/2..
-__device__ void epi_q(const FC& c, int k, int l, int m, int f0, const float* acc) {
+__device__ void epi_q(const FC& c, int k, int l, int m, int f0, const float* acc, const float* bv) {
   const Shape& s = *c.s;
   const FlowArgs& a = *c.a;
-  const float* bias = a.bias_qkv + ((size_t)k * s.L + l) * s.qkv_rows + f0;
-  float bv[8];
-  f4_to(bv, ldg_f4(bias), ldg_f4(bias + 4));
   const float rs = c.s_rstd[m];
   float v[8];
 #pragma unroll
@@ -503,27 +500,34 @@ __device__ void epi_q(const FC& c, int k, int l, int m, int f0, const float* acc
   }
 }
 
+// Epilogue inputs of one reducer thread (token m, 8 rows from f0), read before
+// the cluster barrier so that their latency overlaps the wait for the peers:
+// the shift term (QKV, gate/up) or the residual stream, gate and next norm
+// scale (O, down).
+struct EpiIn {
+  float b[8];  // bias (QKV, gate/up) or gate (O, down)
+  float h[8];  // residual stream (O, down)
+  float sc[8]; // next norm's scale (O, down; unused without a next norm)
+};
+
 // Gated residual for 8 features f0.. of token m: h += gate * acc, then (when
-// `sc` is given) the next norm's operand bf16(h (1 + scale)) and the sum of
-// the 8 squares of h.
-__device__ float epi_resid(const FC& c, int m, int f0, const float* acc, const float* gate, const float* sc,
+// `has_next`) the next norm's operand bf16(h (1 + scale)) and the sum of the 8
+// squares of h.
+__device__ float epi_resid(const FC& c, int m, int f0, const float* acc, const EpiIn& in, bool has_next,
                            bf16* ydst) {
   const Shape& s = *c.s;
   float* hp = c.a->h + (size_t)m * s.D + f0;
-  float hv[8], gv[8];
-  f4_to(hv, ldcg_f4(hp), ldcg_f4(hp + 4));
-  f4_to(gv, ldg_f4(gate + f0), ldg_f4(gate + f0 + 4));
+  float hv[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) hv[i] = fmaf(gv[i], acc[i], hv[i]);
+  for (int i = 0; i < 8; ++i) hv[i] = fmaf(in.b[i], acc[i], in.h[i]);
   reinterpret_cast<float4*>(hp)[0] = make_float4(hv[0], hv[1], hv[2], hv[3]);
   reinterpret_cast<float4*>(hp)[1] = make_float4(hv[4], hv[5], hv[6], hv[7]);
   float ss = 0.f;
-  if (sc) {
-    float sv[8], yv[8];
-    f4_to(sv, ldg_f4(sc + f0), ldg_f4(sc + f0 + 4));
+  if (has_next) {
+    float yv[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      yv[i] = hv[i] * (1.f + sv[i]);
+      yv[i] = hv[i] * (1.f + in.sc[i]);
       ss = fmaf(hv[i], hv[i], ss);
     }
     *reinterpret_cast<uint4*>(ydst + (size_t)m * s.D + f0) = pack8(yv);
@@ -531,9 +535,44 @@ __device__ float epi_resid(const FC& c, int m, int f0, const float* acc, const f
   return ss;
 }
 
+// rstd per token for the QKV / gate-up norm from the producers' sums of
+// squares ss[slot][64]: thread (4 tokens, slot group) sums every 8th slot with
+// all its loads in flight, then the 8 group sums per token are added in a
+// fixed order.
+__device__ void compute_rstd(const FC& c, const float* ss, int nslots) {
+  const Shape& s = *c.s;
+  const int m4 = c.ct & 15, grp = c.ct >> 4;  // 16 x 4 tokens, 8 slot groups
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = grp; s0 < nslots; s0 += 8 * 16) {
+    float4 v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      v[i] = s0 + 8 * i < nslots ? ldcg_f4(ss + (size_t)(s0 + 8 * i) * 64 + 4 * m4) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      acc.x += v[i].x;
+      acc.y += v[i].y;
+      acc.z += v[i].z;
+      acc.w += v[i].w;
+    }
+  }
+  *reinterpret_cast<float4*>(c.s_tmp + grp * 64 + 4 * m4) = acc;
+  csync();
+  if (c.ct < 64) {
+    float t = 0.f;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) t += c.s_tmp[g * 64 + c.ct];
+    c.s_rstd[c.ct] = rsqrtf(t / (float)s.D + s.eps);
+  }
+  csync();
+}
+
 // One projection stage on this CTA.  `it` counts projection items (TMEM
 // slots, partial buffers), `sg` the operand loads compute thread 0 issued,
-// `ncl` cluster barriers.  Returns false once the launch is aborting.
+// `ncl` cluster barriers.  The outputs of all items are published together at
+// the end of the stage (one fence): a consumer's own reduction needs every
+// rank of its cluster, and so in effect the last item of each producer stage.
+// Returns false once the launch is aborting.
 __device__ bool gemm_stage(const FC& c, int st, int k, int l, int u, int& it, int& sg, int& ncl) {
   const Shape& s = *c.s;
   const FlowArgs& a = *c.a;
@@ -577,29 +616,21 @@ __device__ bool gemm_stage(const FC& c, int st, int k, int l, int u, int& it, in
         for (int t = 0; ok && t < a.o_tiles; ++t) ok = wait_ctr(c, c_ho(a, t), uC * (unsigned)(u + 1));
     }
     if (!cand(ok)) return false;
-    const float* ss = st == ST_G ? a.ss_g : (l == 0 ? a.ss_t : a.ss_q);
-    const int nslots = st == ST_G ? a.o_tiles * C : (l == 0 ? 1 : a.d_tiles * C);
-    const int m = c.ct & 63, part = c.ct >> 6;
-    float acc = 0.f;
-    for (int s0 = part; s0 < nslots; s0 += 16) {
-      float v[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = s0 + 2 * i < nslots ? __ldcg(ss + (size_t)(s0 + 2 * i) * 64 + m) : 0.f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc += v[i];
-    }
-    c.s_tmp[part * 64 + m] = acc;
-    csync();
-    if (c.ct < 64) c.s_rstd[c.ct] = rsqrtf((c.s_tmp[c.ct] + c.s_tmp[64 + c.ct]) / (float)s.D + s.eps);
-    csync();
+    if (st == ST_G) compute_rstd(c, a.ss_g, a.o_tiles * C);
+    else if (l > 0) compute_rstd(c, a.ss_q, a.d_tiles * C);
+    else compute_rstd(c, a.ss_t, 1);
   }
 
   // 3. items: accumulator -> own partial tile -> cluster barrier -> reduce
-  //    this rank's rows over the C partials -> epilogue -> publish
+  //    this rank's rows over the C partials -> epilogue
   const float* tab = a.tables + (size_t)k * s.table_rows;
+  const bool has_next = st == ST_O || (st == ST_D && l + 1 < s.L);
+  const float* gate = tab + mod_offset(s, l, st == ST_O ? 0 : 1, 2);
+  const float* scn = !has_next ? nullptr : (st == ST_O ? tab + mod_offset(s, l, 1, 0) : tab + mod_offset(s, l + 1, 0, 0));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qd = warp & 3, row = qd * 32 + lane;  // TMEM lane = weight row
   const int per8 = R / 8, nitems = a.M * per8;
+  const int npass = nitems > 128 ? 2 : 1;
   float keep[2][8];
   for (int j = 0; j < nt; ++j) {
     const int t = c.cl + j * a.NC;
@@ -619,10 +650,31 @@ __device__ bool gemm_stage(const FC& c, int st, int k, int l, int u, int& it, in
       tc_fence_before();
       csync();
       if (c.ct == 0) mbar_arrive(&c.acc_empty[slot]);
+      // epilogue inputs of this thread's (token, 8 rows) item: the first pass's
+      // are read before the barrier, the second's (small batches with 32 rows
+      // per rank) at the start of that pass
+      EpiIn in;
+      auto load_in = [&](int pass) {
+        const int idx = c.ct + pass * 128;
+        if (idx >= nitems) return;
+        const int m = idx / per8, r0 = rank * R + (idx - m * per8) * 8;
+        const int f0 = 128 * t + r0;
+        if (st == ST_Q || st == ST_G) {
+          const float* bias = st == ST_Q ? a.bias_qkv + ((size_t)k * s.L + l) * s.qkv_rows + f0
+                                         : a.bias_gu + ((size_t)k * s.L + l) * 2 * s.F + 256 * t + 128 * half + r0;
+          f4_to(in.b, ldg_f4(bias), ldg_f4(bias + 4));
+        } else {
+          const float* hp = a.h + (size_t)m * s.D + f0;
+          f4_to(in.h, ldcg_f4(hp), ldcg_f4(hp + 4));
+          f4_to(in.b, ldg_f4(gate + f0), ldg_f4(gate + f0 + 4));
+          if (has_next) f4_to(in.sc, ldg_f4(scn + f0), ldg_f4(scn + f0 + 4));
+        }
+      };
+      load_in(0);
       if (!cl_sync(c, ncl)) return false;
-#pragma unroll
-      for (int pass = 0; pass < 2; ++pass) {
-        if (pass == 1 && nitems <= 128) break;  // uniform
+#pragma unroll 1
+      for (int pass = 0; pass < npass; ++pass) {  // uniform
+        if (pass == 1) load_in(1);
         const int idx = c.ct + pass * 128;
         const bool valid = idx < nitems;
         const int m = valid ? idx / per8 : 0, j8 = valid ? idx - (idx / per8) * per8 : 0;
@@ -641,41 +693,37 @@ __device__ bool gemm_stage(const FC& c, int st, int k, int l, int u, int& it, in
         }
         const int f0 = 128 * t + r0;
         if (st == ST_Q) {
-          if (valid) epi_q(c, k, l, m, f0, acc);
+          if (valid) epi_q(c, k, l, m, f0, acc, in.b);
         } else if (st == ST_G) {
           if (valid) {
-            const float* bias = a.bias_gu + ((size_t)k * s.L + l) * 2 * s.F + 256 * t + 128 * half + r0;
-            float bv[8];
-            f4_to(bv, ldg_f4(bias), ldg_f4(bias + 4));
             const float rs = c.s_rstd[m];
             if (half == 0) {
 #pragma unroll
-              for (int i = 0; i < 8; ++i) keep[pass][i] = fmaf(rs, acc[i], bv[i]);
+              for (int i = 0; i < 8; ++i) keep[pass][i] = fmaf(rs, acc[i], in.b[i]);
             } else {
               float ov[8];
 #pragma unroll
-              for (int i = 0; i < 8; ++i) ov[i] = gelu_tanh_bf16out(keep[pass][i]) * fmaf(rs, acc[i], bv[i]);
+              for (int i = 0; i < 8; ++i) ov[i] = gelu_tanh_bf16out(keep[pass][i]) * fmaf(rs, acc[i], in.b[i]);
               *reinterpret_cast<uint4*>(a.u + (size_t)m * s.F + f0) = pack8(ov);
             }
           }
         } else {
-          // O: next norm = this layer's MLP norm; D: the next layer's attention norm
-          const bool has_next = st == ST_O || l + 1 < s.L;
-          const float* gate = tab + mod_offset(s, l, st == ST_O ? 0 : 1, 2);
-          const float* sc = !has_next ? nullptr
-                                      : (st == ST_O ? tab + mod_offset(s, l, 1, 0) : tab + mod_offset(s, l + 1, 0, 0));
           float sq = 0.f;
-          if (valid) sq = epi_resid(c, m, f0, acc, gate, sc, st == ST_O ? a.yg : a.yq);
+          if (valid) sq = epi_resid(c, m, f0, acc, in, has_next, st == ST_O ? a.yg : a.yq);
           // the per8 threads of one token are adjacent lanes: fixed shuffle tree
           for (int o = 1; o < per8; o <<= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-          if (valid && j8 == 0 && has_next)
-            (st == ST_O ? a.ss_g : a.ss_q)[(size_t)(t * C + rank) * 64 + m] = sq;
+          if (valid && j8 == 0 && has_next) (st == ST_O ? a.ss_g : a.ss_q)[(size_t)(t * C + rank) * 64 + m] = sq;
         }
       }
-      if (st == ST_Q) publish(c, c_qkv(a));
-      else if (st == ST_O) publish(c, c_ho(a, t));
-      else if (st == ST_G && half == 1) publish(c, c_u(a, t));
-      else if (st == ST_D) publish(c, c_y(a, t));
+    }
+  }
+  // 4. publish every item of the stage (one fence)
+  __threadfence();
+  csync();
+  if (c.ct == 0) {
+    for (int j = 0; j < nt; ++j) {
+      const int t = c.cl + j * a.NC;
+      red_release_u32(st == ST_Q ? c_qkv(a) : st == ST_O ? c_ho(a, t) : st == ST_G ? c_u(a, t) : c_y(a, t), 1u);
     }
   }
   return true;
@@ -977,8 +1025,8 @@ __device__ void compute_loop(const FC& c) {
   }
   // after an abort, copies this CTA issued may still be in flight: let them land
   if (c.ct == 0) {
-    if (sg > 0 && !mbar_wait(c.op_full, (sg - 1) & 1, kFDrain)) set_error(a.err, DEV_TIMEOUT);
-    if (kv_issued > 0 && !mbar_wait(c.kv_full, (kv_issued - 1) & 1, kFDrain)) set_error(a.err, DEV_TIMEOUT);
+    if (sg > 0 && !mbar_wait(c.op_full, (sg - 1) & 1, kFDrain)) set_error(a.err, DEV_DRAIN);
+    if (kv_issued > 0 && !mbar_wait(c.kv_full, (kv_issued - 1) & 1, kFDrain)) set_error(a.err, DEV_DRAIN);
   }
 }
 
@@ -1026,8 +1074,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
   c.s_abort = reinterpret_cast<volatile int*>(misc + 260);
   c.s_flag = reinterpret_cast<volatile int*>(misc + 264);
   c.s_rstd = reinterpret_cast<float*>(misc + 512);   // [64]
-  c.s_tmp = reinterpret_cast<float*>(misc + 768);    // [256]
-  c.s_ml = reinterpret_cast<float*>(misc + 1792);    // [128][2]
+  c.s_tmp = reinterpret_cast<float*>(misc + 768);    // [512]
+  c.s_ml = reinterpret_cast<float*>(misc + 2816);    // [128][2]
   c.cta = blockIdx.x;
   c.rank = (int)cluster_rank();
   c.cl = blockIdx.x / a.C;
@@ -1111,12 +1159,26 @@ int flow_max_clusters(int C) {
   return n;
 }
 
+// A cooperative launch guarantees that all clusters are resident together.
+// Where the runtime does not take the cooperative attribute together with a
+// cluster shape, the plain cluster launch of the same grid (no more clusters
+// than fit at once) is used; every wait is bounded either way.
 cudaError_t launch_flow(const Shape& s, const CUtensorMap* maps, const FlowArgs& a, cudaStream_t st) {
+  static bool cooperative_ok = true;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[2];
   flow_config(cfg, attr, a.C, a.NC, st);
-  return cudaLaunchKernelEx(&cfg, k_flow, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], maps[7],
-                            maps[8], maps[9], maps[10], s, a);
+  if (!cooperative_ok) cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k_flow, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6],
+                                     maps[7], maps[8], maps[9], maps[10], s, a);
+  if ((e == cudaErrorInvalidValue || e == cudaErrorNotSupported) && cooperative_ok) {
+    cudaGetLastError();
+    cooperative_ok = false;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k_flow, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], maps[7],
+                           maps[8], maps[9], maps[10], s, a);
+  }
+  return e;
 }
 
 }  // namespace pae

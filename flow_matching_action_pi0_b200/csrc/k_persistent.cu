@@ -865,7 +865,7 @@ __device__ void compute_loop(const Ctx& c) {
   if (ok) transition(c, a.k_end - 1, -1);
   // after an abort, attention copies may still be in flight: let the last land
   if (c.tid == 0 && *c.s_loads > 0 && !mbar_wait(c.bars.kv_full, (*c.s_loads - 1) & 1, kDrainNs))
-    set_error(a.err, DEV_TIMEOUT);
+    set_error(a.err, DEV_DRAIN);
 }
 
 // ------------------------------------------------------------ weight producer
@@ -895,7 +895,7 @@ __device__ void producer_loop(const Ctx& c) {
       }
   // copies still in flight must land before the CTA exits
   for (int j = n > kRing ? n - kRing : 0; j < n; ++j)
-    if (!mbar_wait(&c.bars.full[j % kRing], (j / kRing) & 1, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
+    if (!mbar_wait(&c.bars.full[j % kRing], (j / kRing) & 1, kDrainNs)) set_error(a.err, DEV_DRAIN);
 }
 
 // ------------------------------------------------------------ MMA issuer
@@ -978,7 +978,7 @@ __device__ void mma_loop(const Ctx& c) {
   if (!ok && !*c.s_abort) raise_abort(c);
   // every MMA this thread issued must finish before TMEM is freed
   umma_commit(c.bars.drain);
-  if (!mbar_wait(c.bars.drain, 0, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
+  if (!mbar_wait(c.bars.drain, 0, kDrainNs)) set_error(a.err, DEV_DRAIN);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)

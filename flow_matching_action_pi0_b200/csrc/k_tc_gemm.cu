@@ -365,7 +365,7 @@ __global__ void __launch_bounds__(256, 2)
     }
     // Loads still in flight must land before this CTA may exit.
     for (int kb = issued > p.stages ? issued - p.stages : 0; kb < issued; ++kb)
-      if (!mbar_wait(&full[kb % p.stages], (kb / p.stages) & 1, kDrainNs)) set_error(a.err, DEV_TIMEOUT);
+      if (!mbar_wait(&full[kb % p.stages], (kb / p.stages) & 1, kDrainNs)) set_error(a.err, DEV_DRAIN);
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------------- MMA
     const uint32_t idesc = idesc_bf16(128, p.tn);
@@ -546,7 +546,7 @@ __global__ void __launch_bounds__(256, 2)
 
   // ------------------------------------------------------------------ epilogue
   const bool acc_ok = mbar_wait(accf, 0, kDrainNs);
-  if (!acc_ok) set_error(a.err, DEV_TIMEOUT);
+  if (!acc_ok) set_error(a.err, DEV_DRAIN);
   tc_fence_after();
   // CTA-uniform decision: the TMEM loads below are warp-collective.
   const bool ok = __syncthreads_and(acc_ok ? 1 : 0) != 0 && s_flag[0] == 0;

@@ -241,6 +241,9 @@ pae_status dev_alloc(pae_ctx* ctx, void** p, size_t bytes) {
 pae_status check_err_word(pae_ctx* ctx) {
   if (ctx->err_host && *(volatile int*)ctx->err_host != 0) {
     const int code = *(volatile int*)ctx->err_host;
+    if (code == DEV_DRAIN)
+      return fail(ctx, PAE_ERR_TIMEOUT, "device error word set (%d): a drain of copies or MMAs already issued ran "
+                                        "out; destroy this context", code);
     return fail(ctx, PAE_ERR_TIMEOUT, "device error word set (%d): a bounded device wait ran out", code);
   }
   return PAE_OK;
@@ -1639,7 +1642,8 @@ pae_status pae_sync(pae_ctx* ctx, pae_stream stream) {
 void pae_clear_error(pae_ctx* ctx) {
   if (!ctx) return;
   cudaDeviceSynchronize();
-  if (ctx->err_host) *(volatile int*)ctx->err_host = 0;
+  // a failed drain stays: the context's memory may still be written by copies
+  if (ctx->err_host && *(volatile int*)ctx->err_host != DEV_DRAIN) *(volatile int*)ctx->err_host = 0;
   ctx->last_error.clear();
 }
 

@@ -276,7 +276,11 @@ pae_status pae_query(pae_ctx* ctx, int what, int batch, long long* value);
 pae_status pae_plan_query(const pae_config* cfg, int what, int batch, long long* value);
 
 /* Synchronise `stream` and report the device error word (PAE_ERR_TIMEOUT if a
- * bounded wait ran out since the last pae_clear_error). */
+ * bounded wait ran out since the last pae_clear_error).  pae_clear_error
+ * resets it so the context can be used again, except after a failed drain
+ * (the last bounded wait for copies or MMAs a kernel had already issued, whose
+ * message says so): then copies may still be landing in the context's memory
+ * and the error stays until the context is destroyed. */
 pae_status pae_sync(pae_ctx* ctx, pae_stream stream);
 void pae_clear_error(pae_ctx* ctx);
 
