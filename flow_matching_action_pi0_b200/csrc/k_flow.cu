@@ -68,6 +68,23 @@ constexpr long long kFDrain = 4000000000LL;
 
 enum : int { ST_Q = 0, ST_O = 1, ST_G = 2, ST_D = 3 };
 
+// Stage timestamps for performance analysis, compiled in only with
+// -DPAE_FLOW_TRACE: compute thread 0 of every CTA records %globaltimer at
+// fixed points of one layer (layer 1 of the first step of a launch) into
+// g_flow_trace[cta][event]; pae_flow_trace_read copies them out.
+#ifdef PAE_FLOW_TRACE
+constexpr int kTraceEv = 48;
+__device__ unsigned long long g_flow_trace[256 * kTraceEv];
+#define FTRACE(c, on, ev)                                                                  \
+  do {                                                                                     \
+    if ((on) && (c).ct == 0) g_flow_trace[(c).cta * kTraceEv + (ev)] = globaltimer_ns(); \
+  } while (0)
+#else
+#define FTRACE(c, on, ev) \
+  do {                    \
+  } while (0)
+#endif
+
 // ------------------------------------------------------------ small helpers
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
   unsigned v;
@@ -582,6 +599,11 @@ __device__ bool gemm_stage(const FC& c, int st, int k, int l, int u, int& it, in
   const int C = a.C, R = 128 / C, rank = c.rank;
   const int x0 = rank * g.kbr * 64, x1 = x0 + g.kbr * 64;
   const unsigned uC = (unsigned)C;
+  const bool tr = k == a.k_begin && l == 1;
+  const int tb = st * 10;
+  (void)tr;
+  (void)tb;
+  FTRACE(c, tr, tb + 0);
 
   // 1. the producers of this rank's K slice of the token operand, then its TMA
   bool ok = true;
@@ -604,6 +626,7 @@ __device__ bool gemm_stage(const FC& c, int st, int k, int l, int u, int& it, in
       ++sg;  // operand loads issued (drained before exit)
     }
   }
+  FTRACE(c, tr, tb + 1);
   if (!cand(ok)) return false;
 
   // 2. QKV and gate/up: rstd per token from the producers' sums of squares
@@ -637,6 +660,7 @@ __device__ bool gemm_stage(const FC& c, int st, int k, int l, int u, int& it, in
     for (int half = 0; half < g.na; ++half, ++it) {
       const int slot = it & 1;
       if (!cand(fwait(c, &c.acc_full[slot], (it >> 1) & 1))) return false;
+      if (j == 0 && half == 0) FTRACE(c, tr, tb + 2);
       tc_fence_after();
       const uint32_t taddr = c.tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)slot * 64u;
       const uint32_t pbase = smem_u32(c.work + kFPart) + (uint32_t)(it & 1) * 32768u;
@@ -671,7 +695,9 @@ __device__ bool gemm_stage(const FC& c, int st, int k, int l, int u, int& it, in
         }
       };
       load_in(0);
+      if (j == 0 && half == 0) FTRACE(c, tr, tb + 3);
       if (!cl_sync(c, ncl)) return false;
+      if (j == 0 && half == 0) FTRACE(c, tr, tb + 4);
 #pragma unroll 1
       for (int pass = 0; pass < npass; ++pass) {  // uniform
         if (pass == 1) load_in(1);
@@ -718,8 +744,10 @@ __device__ bool gemm_stage(const FC& c, int st, int k, int l, int u, int& it, in
     }
   }
   // 4. publish every item of the stage (one fence)
+  FTRACE(c, tr, tb + 5);
   __threadfence();
   csync();
+  FTRACE(c, tr, tb + 6);
   if (c.ct == 0) {
     for (int j = 0; j < nt; ++j) {
       const int t = c.cl + j * a.NC;
@@ -743,6 +771,9 @@ __device__ bool att_stage(const FC& c, int l, int u, int& ac, int& ncl, int& kv_
   if (!au.has) return true;
   const int d = s.d, nbox = d / 64, GH = s.G * s.H, C = a.C;
   const uint32_t qbytes = 128u * d * 2u, kvbytes = (uint32_t)CKF * d * 2u;
+  const bool tr = u == 1;
+  (void)tr;
+  FTRACE(c, tr, 40);
   // peers are done reading this CTA's partial tiles of the QKV stage
   if (!cl_sync(c, ncl)) return false;
   const int slot_row0 = ((l * s.Bmax + au.b) * s.Hkv + au.g) * s.Ptot;
@@ -762,6 +793,7 @@ __device__ bool att_stage(const FC& c, int l, int u, int& ac, int& ncl, int& kv_
       ++kv_issued;
     }
   }
+  FTRACE(c, tr, 41);
   if (!cand(ok)) return false;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -772,6 +804,7 @@ __device__ bool att_stage(const FC& c, int l, int u, int& ac, int& ncl, int& kv_
   for (int ch = 0; ch < au.nch; ++ch) {
     const int acn = ac + ch;
     if (!cand(fwait(c, c.s_full, acn & 1))) return false;
+    if (ch == 0) FTRACE(c, tr, 42);
     tc_fence_after();
     float sv[CKF];
 #pragma unroll
@@ -846,6 +879,7 @@ __device__ bool att_stage(const FC& c, int l, int u, int& ac, int& ncl, int& kv_
   }
   ac += au.nch;
   if (au.nch > 0 && !cand(fwait(c, c.o_full, (ac - 1) & 1))) return false;
+  FTRACE(c, tr, 43);
   tc_fence_after();
 
   // -------------------------------------------------- merge in the cluster
@@ -880,7 +914,9 @@ __device__ bool att_stage(const FC& c, int l, int u, int& ac, int& ncl, int& kv_
     }
   }
   tc_fence_before();
+  FTRACE(c, tr, 44);
   if (!cl_sync(c, ncl)) return false;
+  FTRACE(c, tr, 45);
   const int R = 128 / C, per_row = d / 4;
   for (int el = c.ct; el < R * per_row; el += kFCompute) {
     const int rr = el / per_row, c4 = el - rr * per_row;
@@ -896,7 +932,9 @@ __device__ bool att_stage(const FC& c, int l, int u, int& ac, int& ncl, int& kv_
     bf16* orow = a.o + (size_t)(au.b * s.H + ti) * s.attn_dim + (au.g * s.G + hl) * d;
     *reinterpret_cast<uint2*>(orow + 4 * c4) = make_uint2(pack_bf2(acc.x, acc.y), pack_bf2(acc.z, acc.w));
   }
+  FTRACE(c, tr, 46);
   publish(c, c_att(a));
+  FTRACE(c, tr, 47);
   // peers are done reading this CTA's partial before the work area is reused
   return cl_sync(c, ncl);
 }
@@ -1121,6 +1159,12 @@ __global__ void __launch_bounds__(kFThreads, 1)
 }
 
 }  // namespace
+
+#ifdef PAE_FLOW_TRACE
+extern "C" int pae_flow_trace_read(void* dst, size_t bytes) {
+  return (int)cudaMemcpyFromSymbol(dst, g_flow_trace, bytes < sizeof(g_flow_trace) ? bytes : sizeof(g_flow_trace));
+}
+#endif
 
 size_t flow_smem_bytes() { return kFSmem; }
 
