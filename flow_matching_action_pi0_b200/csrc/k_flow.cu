@@ -240,12 +240,12 @@ __device__ void publish(const FC& c, unsigned* p) {
 __device__ bool cl_sync(const FC& c, int& n) {
   fence_acq_rel_cluster();
   csync();
+  uint64_t* b = &c.cbar[n & 1];
+  // compute thread r arrives on rank r's instance (one remote arrive each)
+  if (c.ct < c.a->C && !*c.s_abort) mbar_arrive_remote(map_cluster(smem_u32(b), (uint32_t)c.ct));
   if (c.ct == 0) {
     bool ok = !*c.s_abort;
     if (ok) {
-      uint64_t* b = &c.cbar[n & 1];
-      const uint32_t baddr = smem_u32(b);
-      for (int r = 0; r < c.a->C; ++r) mbar_arrive_remote(map_cluster(baddr, (uint32_t)r));
       const uint32_t par = (uint32_t)(n >> 1) & 1u;
       ok = mbar_try_wait_cl(b, par);
       if (!ok) {
