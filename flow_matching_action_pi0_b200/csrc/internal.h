@@ -46,6 +46,10 @@ void launch_mod_tables(const Shape& s, int act_bf16, const float* cbuf, int K, c
 // 1 = MLP adaRMSNorm.
 void launch_shift_bias(const Shape& s, const void* W, int rows, int norm, const float* tables, int K, float* out,
                        cudaStream_t st);
+// The same from packed int4 weights [L][rows][D/2] (create-time nibble order)
+// and their group scales [L][rows][D/128].
+void launch_shift_bias_w4(const Shape& s, const void* Wq, const void* scales, int rows, int norm,
+                          const float* tables, int K, float* out, cudaStream_t st);
 
 // ------------------------------------------------------------ token kernels
 // Per token: optionally (final adaRMSNorm, out_proj, Euler update of x with
@@ -227,13 +231,16 @@ struct FlowArgs {
   const bf16* w_out;
   const bf16* b_out;
   const float2* rope_cs;
+  int w4;                            // int4 weights (packed maps; wsc = group scales)
+  const bf16* wsc[4];                // W4A16: [rows][K/128] scales of QKV, O, gate/up (stored order), down
   unsigned* ctr;                     // [kFlowCtrWords], zero at launch
   DevErr err;
 };
 size_t flow_smem_bytes();
 cudaError_t flow_init();
 int flow_max_clusters(int C);        // clusters of C CTAs that fit at once (0 on error)
-// maps: W qkv, W o, W gate/up (128-row boxes), W down, y_q, o, y_g, u (64 x 64
+// maps: W qkv, W o, W gate/up (128-row boxes), W down (bf16 [128][64] boxes, or
+// with w4 the packed [128 rows][32 bytes] boxes), y_q, o, y_g, u (64 x 64
 // boxes), q (64 x 128), k, v (64 x 64).  Cooperative cluster launch.
 cudaError_t launch_flow(const Shape& s, const CUtensorMap* maps, const FlowArgs& a, cudaStream_t st);
 

@@ -53,7 +53,9 @@ namespace {
 
 constexpr int kFThreads = 192;   // warp 0 weights, warp 1 MMA, warps 2-5 compute
 constexpr int kFCompute = 128;
-constexpr int kFRing = 5;
+constexpr int kFRing = 5;                // bf16 weight ring depth (W4A16: 4 slots + the packed ring)
+constexpr int kFRawRing = 4;             // packed int4 blocks [128 rows][32 bytes] in flight (W4A16)
+constexpr uint32_t kFRawBlk = 4096;
 constexpr uint32_t kFBlk = 16384;        // [128 rows][64] bf16 weight block
 constexpr uint32_t kFWork = 128 * 1024;  // operands, partial tiles, attention tiles
 constexpr uint32_t kFMisc = 4096;
@@ -160,8 +162,11 @@ struct FC {
   FMaps mp;
   uint8_t* ring;
   uint8_t* work;
-  uint64_t* rfull;     // [kFRing]
+  uint64_t* rfull;     // [kFRing] bf16 weight block in slot ready for the MMAs
   uint64_t* rempty;    // [kFRing]
+  uint64_t* raw_full;  // [kFRawRing] packed int4 block landed (W4A16)
+  uint8_t* raw;        // packed int4 ring (W4A16)
+  int nring;           // ring depth in use (kFRing, or kFRing - 1 with the int4 ring)
   uint64_t* op_full;   // token operand of a projection stage landed
   uint64_t* acc_full;  // [2] accumulator slot ready
   uint64_t* acc_empty; // [2] accumulator slot read out
@@ -325,43 +330,152 @@ __device__ __forceinline__ unsigned* c_ho(const FlowArgs& a, int t) { return a.c
 __device__ __forceinline__ unsigned* c_u(const FlowArgs& a, int p) { return a.ctr + 3 + a.d_tiles + a.o_tiles + p; }
 
 // ------------------------------------------------------------ weight producer
-// Warp 0, lane 0: this CTA's weight blocks in schedule order (per step, layer,
-// stage, item, K block) into the ring; each load also prefetches the same
-// block of the next layer into L2, so HBM streams one layer ahead of the
-// dependency chain.
-__device__ void producer_loop(const FC& c) {
+// Weight block n of this CTA's schedule (per step, layer, stage, item, K block):
+// which matrix, its K offset (elements), its first weight row, and the same
+// block's row in the next layer (or layer 0 of the next step; -1: none).
+struct Blk {
+  int st, x, row0, nrow, kofs;
+};
+__device__ __forceinline__ int blocks_per_layer(const FC& c) {
+  int n = 0;
+  for (int st = 0; st < 4; ++st) {
+    const StageG g = stage_geo(*c.s, *c.a, st);
+    n += cl_tiles(*c.a, g.ntiles, c.cl) * g.na * g.kbr;
+  }
+  return n;
+}
+__device__ bool block_at(const FC& c, int nbl, int n, Blk& b) {
   const Shape& s = *c.s;
   const FlowArgs& a = *c.a;
+  if (nbl == 0) return false;
+  const int kl = n / nbl;
+  if (kl >= (a.k_end - a.k_begin) * s.L) return false;
+  int r = n - kl * nbl;
+  const int l = kl % s.L;
+  const bool last = kl + 1 >= (a.k_end - a.k_begin) * s.L;
+  for (int st = 0; st < 4; ++st) {
+    const StageG g = stage_geo(s, a, st);
+    const int cnt = cl_tiles(a, g.ntiles, c.cl) * g.na * g.kbr;
+    if (r < cnt) {
+      const int item = r / g.kbr, i = r - item * g.kbr;
+      const int j = item / g.na, half = item - j * g.na;
+      b.st = st;
+      b.kofs = (c.rank * g.kbr + i) * 64;
+      b.x = b.kofs;
+      b.row0 = item_row(g, l, c.cl + j * a.NC, half);
+      b.nrow = last ? -1 : (l + 1 < s.L ? b.row0 + g.wrows : b.row0 - (s.L - 1) * g.wrows);
+      return true;
+    }
+    r -= cnt;
+  }
+  return false;
+}
+
+// Packed int4 weights -> bf16 code * group scale, rounded once (to nearest
+// even): two codes per call from one 32-bit word whose nibbles were permuted
+// at create time so that (w >> 4i) & 0x000F000F holds the pair (2i, 2i + 1).
+// (n ^ 8) | 0x4300 is the bf16 of 128 + (code + 8); subtracting 136 is exact.
+__device__ __forceinline__ uint32_t dq_pair(uint32_t w, int i, __nv_bfloat162 sc) {
+  const uint32_t t = (((w >> (4 * i)) & 0x000F000Fu) ^ 0x00080008u) | 0x43004300u;
+  __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&t);
+  const __nv_bfloat162 off = __floats2bfloat162_rn(136.f, 136.f);
+  v = __hmul2(__hsub2(v, off), sc);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Warp 0.  bf16 weights: lane 0 streams this CTA's weight blocks (16 KB) into
+// the ring in schedule order.  int4 weights: lane 0 keeps kFRawRing packed
+// blocks (4 KB) in flight; all 32 lanes turn each landed block into a bf16
+// block of the ring (4 rows per lane, 128-byte swizzled like a TMA tile).
+// Either way each load also prefetches the same block of the next layer into
+// L2, so HBM streams one layer ahead of the dependency chain.
+__device__ void producer_warp(const FC& c) {
+  const FlowArgs& a = *c.a;
+  const int lane = threadIdx.x & 31;
   const uint64_t pol = policy_evict_first();  // a block is used once per step
+  const int nbl = blocks_per_layer(c);
+  const int R = c.nring;
   int n = 0;
   bool ok = true;
-  for (int k = a.k_begin; ok && k < a.k_end; ++k)
-    for (int l = 0; ok && l < s.L; ++l)
-      for (int st = 0; ok && st < 4; ++st) {
-        const StageG g = stage_geo(s, a, st);
-        const int nt = cl_tiles(a, g.ntiles, c.cl);
-        for (int j = 0; ok && j < nt; ++j) {
-          const int t = c.cl + j * a.NC;
-          for (int half = 0; ok && half < g.na; ++half) {
-            const int row0 = item_row(g, l, t, half);
-            const int nrow = l + 1 < s.L ? row0 + g.wrows : (k + 1 < a.k_end ? row0 - (s.L - 1) * g.wrows : -1);
-            for (int i = 0; i < g.kbr; ++i, ++n) {
-              const int slot = n % kFRing;
-              if (n >= kFRing && !fwait(c, &c.rempty[slot], ((n / kFRing) & 1) ^ 1)) {
-                ok = false;
-                break;
-              }
-              const int x = (c.rank * g.kbr + i) * 64;
-              mbar_arrive_expect_tx(&c.rfull[slot], kFBlk);
-              tma_load_2d_hint(c.ring + (size_t)slot * kFBlk, c.mp.w[st], x, row0, &c.rfull[slot], pol);
-              if (nrow >= 0) tma_prefetch_l2(c.mp.w[st], x, nrow);
-            }
-          }
+  if (!a.w4) {
+    if (lane == 0) {
+      Blk b;
+      for (; block_at(c, nbl, n, b); ++n) {
+        const int slot = n % R;
+        if (n >= R && !fwait(c, &c.rempty[slot], ((n / R) & 1) ^ 1)) {
+          ok = false;
+          break;
         }
+        mbar_arrive_expect_tx(&c.rfull[slot], kFBlk);
+        tma_load_2d_hint(c.ring + (size_t)slot * kFBlk, c.mp.w[b.st], b.x, b.row0, &c.rfull[slot], pol);
+        if (b.nrow >= 0) tma_prefetch_l2(c.mp.w[b.st], b.x, b.nrow);
       }
-  // copies still in flight land before the CTA exits
-  for (int j = n > kFRing ? n - kFRing : 0; j < n; ++j)
-    if (!mbar_wait(&c.rfull[j % kFRing], (j / kFRing) & 1, kFDrain)) set_error(a.err, DEV_DRAIN);
+      // copies still in flight land before the CTA exits
+      for (int j = n > R ? n - R : 0; j < n; ++j)
+        if (!mbar_wait(&c.rfull[j % R], (j / R) & 1, kFDrain)) set_error(a.err, DEV_DRAIN);
+    }
+    __syncwarp();
+    return;
+  }
+  // ---- int4: packed blocks in flight, dequantised by the whole warp
+  int issued = 0;
+  auto issue = [&](int m) -> bool {
+    Blk b;
+    if (!block_at(c, nbl, m, b)) return false;
+    const int rs = m % kFRawRing;
+    mbar_arrive_expect_tx(&c.raw_full[rs], kFRawBlk);
+    tma_load_2d_hint(c.raw + (size_t)rs * kFRawBlk, c.mp.w[b.st], b.x / 2, b.row0, &c.raw_full[rs], pol);
+    if (b.nrow >= 0) tma_prefetch_l2(c.mp.w[b.st], b.x / 2, b.nrow);
+    return true;
+  };
+  if (lane == 0)
+    while (issued < kFRawRing && issue(issued)) ++issued;
+  issued = __shfl_sync(0xffffffffu, issued, 0);
+  Blk b;
+  for (; ok && block_at(c, nbl, n, b); ++n) {
+    const int rs = n % kFRawRing, slot = n % R;
+    bool w = fwait(c, &c.raw_full[rs], (n / kFRawRing) & 1);
+    if (w && n >= R) w = fwait(c, &c.rempty[slot], ((n / R) & 1) ^ 1);
+    if (!__all_sync(0xffffffffu, w)) {
+      ok = false;
+      break;
+    }
+    // rows lane, lane + 32, lane + 64, lane + 96 of the block
+    const StageG g = stage_geo(*c.s, a, b.st);
+    const int K = g.kbr * 64 * a.C;  // the matrix's K
+    const int gpr = K / 128, grp = b.kofs / 128;
+    const uint8_t* rb = c.raw + (size_t)rs * kFRawBlk;
+    const uint32_t ab = smem_u32(c.ring + (size_t)slot * kFBlk);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int r = lane + 32 * q;
+      const bf16 sv = a.wsc[b.st][(size_t)(b.row0 + r) * gpr + grp];
+      const __nv_bfloat162 sc = __halves2bfloat162(sv, sv);
+      const uint4 w0 = *reinterpret_cast<const uint4*>(rb + r * 32);
+      const uint4 w1 = *reinterpret_cast<const uint4*>(rb + r * 32 + 16);
+      const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        const uint32_t addr = ab + (uint32_t)r * 128u + (((uint32_t)cc ^ (uint32_t)(r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dq_pair(words[cc], 0, sc)),
+                     "r"(dq_pair(words[cc], 1, sc)), "r"(dq_pair(words[cc], 2, sc)), "r"(dq_pair(words[cc], 3, sc))
+                     : "memory");
+      }
+    }
+    fence_proxy_async_smem();  // the tensor cores read what the warp just wrote
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&c.rfull[slot]);
+      if (issue(issued)) ++issued;  // the raw slot of block n is free now
+    }
+    issued = __shfl_sync(0xffffffffu, issued, 0);
+  }
+  if (!ok && !*c.s_abort) raise_abort(c);
+  // packed copies still in flight land before the CTA exits
+  if (lane == 0)
+    for (int j = issued > kFRawRing ? issued - kFRawRing : 0; j < issued; ++j)
+      if (!mbar_wait(&c.raw_full[j % kFRawRing], (j / kFRawRing) & 1, kFDrain)) set_error(a.err, DEV_DRAIN);
+  __syncwarp();
 }
 
 // ------------------------------------------------------------ MMA issuer
@@ -430,8 +544,8 @@ __device__ void mma_loop(const FC& c) {
             }
             tc_fence_after();
             for (int i = 0; i < g.kbr; ++i, ++n) {
-              const int rs = n % kFRing;
-              if (!fwait(c, &c.rfull[rs], (n / kFRing) & 1)) {
+              const int rs = n % c.nring;
+              if (!fwait(c, &c.rfull[rs], (n / c.nring) & 1)) {
                 ok = false;
                 break;
               }
@@ -1107,7 +1221,10 @@ __global__ void __launch_bounds__(kFThreads, 1)
   c.o_full = bar + 2 * kFRing + 8;
   c.cbar = bar + 2 * kFRing + 9;       // [2]
   c.drain = bar + 2 * kFRing + 11;
-  constexpr int kNBar = 2 * kFRing + 12;
+  c.raw_full = bar + 2 * kFRing + 12;  // [kFRawRing]
+  constexpr int kNBar = 2 * kFRing + 12 + kFRawRing;
+  c.nring = a.w4 ? kFRing - 1 : kFRing;
+  c.raw = smem + (kFRing - 1) * kFBlk;  // int4 mode: the fifth bf16 slot holds the packed ring
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 256);
   c.s_abort = reinterpret_cast<volatile int*>(misc + 260);
   c.s_flag = reinterpret_cast<volatile int*>(misc + 264);
@@ -1144,7 +1261,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
   hw_cluster_sync();  // every rank's mbarriers exist before any remote arrive
 
   if (warp == 0) {
-    if (lane == 0) producer_loop(c);
+    producer_warp(c);
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) mma_loop(c);

@@ -136,7 +136,68 @@ __global__ void k_shift_bias(const bf16* __restrict__ W, int rows, int D, int L,
   }
 }
 
+// The same for int4 weights: W[r][k] = code * scale[r][k / 128], codes packed
+// two per byte with the nibbles of every 32-bit word permuted at create time
+// (nibble of k = 8c + e at bit 4 (e / 2) + 16 (e % 2) of word c).
+__global__ void k_shift_bias_w4(const uint8_t* __restrict__ Wq, const bf16* __restrict__ sc, int rows, int D, int L,
+                                const float* __restrict__ tables, int table_rows, int norm, int K,
+                                float* __restrict__ out) {
+  extern __shared__ float xs[];  // [KC][D]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int bpl = (gridDim.x + L - 1) / L;
+  const int l = blockIdx.x / bpl, b = blockIdx.x - l * bpl;
+  if (l >= L) return;
+  const int shift_off = ((l * 2 + norm) * 3 + 1) * D;
+  const int words = D / 8, gpr = D / 128;
+  for (int k0 = 0; k0 < K; k0 += KC) {
+    const int kc = min(KC, K - k0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kc * D; i += blockDim.x) {
+      const int j = i / D, c = i - j * D;
+      xs[i] = tables[(size_t)(k0 + j) * table_rows + shift_off + c];
+    }
+    __syncthreads();
+    for (int r = b * nw + warp; r < rows; r += bpl * nw) {
+      float acc[KC];
+#pragma unroll
+      for (int j = 0; j < KC; ++j) acc[j] = 0.f;
+      const size_t row = (size_t)l * rows + r;
+      const uint32_t* wr = reinterpret_cast<const uint32_t*>(Wq + row * (D / 2));
+      for (int c = lane; c < words; c += 32) {
+        const uint32_t w = wr[c];
+        const float sv = bf2f(sc[row * gpr + (8 * c) / 128]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int sh = 4 * (e >> 1) + 16 * (e & 1);
+          const int code = (int)((w >> sh) & 0xFu);
+          const float wv = (float)(code >= 8 ? code - 16 : code) * sv;
+          const int kk = 8 * c + e;
+#pragma unroll
+          for (int j = 0; j < KC; ++j)
+            if (j < kc) acc[j] = fmaf(wv, xs[j * D + kk], acc[j]);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < KC; ++j)
+        if (j < kc) {
+          const float v = warp_sum(acc[j]);
+          if (lane == 0) out[((size_t)(k0 + j) * L + l) * rows + r] = v;
+        }
+    }
+  }
+}
+
 }  // namespace
+
+void launch_shift_bias_w4(const Shape& s, const void* Wq, const void* scales, int rows, int norm,
+                          const float* tables, int K, float* out, cudaStream_t st) {
+  const int bpl = std::max(1, std::min(64, (rows + 63) / 64));
+  const size_t smem = (size_t)KC * s.D * sizeof(float);
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(k_shift_bias_w4, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  k_shift_bias_w4<<<bpl * s.L, 256, smem, st>>>(static_cast<const uint8_t*>(Wq), static_cast<const bf16*>(scales),
+                                                rows, s.D, s.L, tables, s.table_rows, norm, K, out);
+}
 
 void launch_shift_bias(const Shape& s, const void* W, int rows, int norm, const float* tables, int K, float* out,
                        cudaStream_t st) {

@@ -168,6 +168,7 @@ struct pae_ctx {
   void *q_qkv = nullptr, *q_o = nullptr, *q_gu = nullptr, *q_down = nullptr;
   void *sc_qkv = nullptr, *sc_o = nullptr, *sc_gu = nullptr, *sc_down = nullptr;
   CUtensorMap tmQqkv{}, tmQo{}, tmQgu{}, tmQdown{};
+  CUtensorMap tmQgu1{};  // packed gate/up with 128-row boxes (dataflow loop)
   // tables
   double* t_dev = nullptr;
   float *emb = nullptr, *zbuf = nullptr, *cbuf = nullptr, *tables = nullptr, *dt = nullptr;
@@ -558,6 +559,11 @@ bool plan_flow(const pae_ctx* ctx, int B, FlowArgs* fa) {
   fa->w_out = static_cast<const bf16*>(ctx->w_out);
   fa->b_out = static_cast<const bf16*>(ctx->b_out);
   fa->rope_cs = ctx->rope_cs;
+  fa->w4 = ctx->w4;
+  fa->wsc[0] = static_cast<const bf16*>(ctx->sc_qkv);
+  fa->wsc[1] = static_cast<const bf16*>(ctx->sc_o);
+  fa->wsc[2] = static_cast<const bf16*>(ctx->sc_gu);
+  fa->wsc[3] = static_cast<const bf16*>(ctx->sc_down);
   fa->ctr = ctx->f_ctr;
   return true;
 }
@@ -868,8 +874,10 @@ pae_status enqueue_flow(pae_ctx* ctx, Plan* P, int k_begin, int k_end, cudaStrea
   fa.k_begin = k_begin;
   fa.k_end = k_end;
   fa.err = DevErr{ctx->err_dev, ctx->wait_ns};
-  const CUtensorMap maps[11] = {ctx->tmWqkv, ctx->tmWo,   ctx->tmWgu1, ctx->tmWdown, ctx->tmYq64, ctx->tmO64,
-                                ctx->tmYg64, ctx->tmU64,  ctx->tmQ,    ctx->tmK,     ctx->tmV};
+  const bool w4 = ctx->w4 != 0;
+  const CUtensorMap maps[11] = {w4 ? ctx->tmQqkv : ctx->tmWqkv, w4 ? ctx->tmQo : ctx->tmWo,
+                                w4 ? ctx->tmQgu1 : ctx->tmWgu1, w4 ? ctx->tmQdown : ctx->tmWdown,
+                                ctx->tmYq64, ctx->tmO64, ctx->tmYg64, ctx->tmU64, ctx->tmQ, ctx->tmK, ctx->tmV};
   P->recs.clear();
   ctx->rec_sink = &P->recs;
   ctx->ev_next = 0;
@@ -1305,6 +1313,8 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
       return bail(st);
     if ((st = make_map_u8(ctx, &ctx->tmQdown, ctx->q_down, F / 2, (uint64_t)L * D, 32, 128)) != PAE_OK)
       return bail(st);
+    if ((st = make_map_u8(ctx, &ctx->tmQgu1, ctx->q_gu, D / 2, (uint64_t)L * 2 * F, 32, 128)) != PAE_OK)
+      return bail(st);
   }
   if (ctx->act_bf16 && !ctx->w4) {
     // persistent kernel: 128-row gate/up boxes, workspace, one CTA per SM
@@ -1320,7 +1330,7 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
     ALLOC(ctx->pw_ss, sizeof(float) * kPersistGroups * 64);
     ALLOC(ctx->pw_ctr, sizeof(unsigned) * kPersistCtrWords);
   }
-  if (ctx->act_bf16 && !ctx->w4) {
+  if (ctx->act_bf16) {
     // dataflow loop: buffers, 64-row operand maps, occupancy of each cluster size
     ctx->flow_capable = true;
     CKC(flow_init());
@@ -1449,8 +1459,13 @@ pae_status pae_precompute_tables(pae_ctx* ctx, const double* t, int K, pae_strea
   launch_mod_tables(ctx->s, ctx->act_bf16, ctx->cbuf, K, ctx->w_modall, ctx->b_modall, ctx->tables, stm);
   if (ctx->flow_capable) {
     // the adaRMSNorm shifts projected through W_qkv and W_gate/up, per step and layer
-    launch_shift_bias(ctx->s, ctx->w_qkv, ctx->s.qkv_rows, 0, ctx->tables, K, ctx->bias_qkv, stm);
-    launch_shift_bias(ctx->s, ctx->w_gu, 2 * ctx->s.F, 1, ctx->tables, K, ctx->bias_gu, stm);
+    if (ctx->w4) {
+      launch_shift_bias_w4(ctx->s, ctx->q_qkv, ctx->sc_qkv, ctx->s.qkv_rows, 0, ctx->tables, K, ctx->bias_qkv, stm);
+      launch_shift_bias_w4(ctx->s, ctx->q_gu, ctx->sc_gu, 2 * ctx->s.F, 1, ctx->tables, K, ctx->bias_gu, stm);
+    } else {
+      launch_shift_bias(ctx->s, ctx->w_qkv, ctx->s.qkv_rows, 0, ctx->tables, K, ctx->bias_qkv, stm);
+      launch_shift_bias(ctx->s, ctx->w_gu, 2 * ctx->s.F, 1, ctx->tables, K, ctx->bias_gu, stm);
+    }
   }
   CK(cudaGetLastError());
   if (K != ctx->K) drop_graphs(ctx);

@@ -61,6 +61,12 @@ def test_tiny_bf16_head_dim_256_cluster_sizes():
     assert max_abs(a, b) < 2e-2
 
 
+def test_tiny_w4a16_batch3_rope():
+    # int4 weights: packed blocks dequantised by the weight producer warp
+    cfg = wl.TINY_FP32.replace(name="tiny_w4a16_df", dtype=wl.W4A16, batch=3, rope_base=10000.0)
+    _case(cfg, lengths=[64, 9, 0])
+
+
 def test_step_split_bitwise_and_host_buffers():
     cfg = wl.TINY_FP32.replace(name="tiny_bf16_df_split", dtype=wl.BF16, batch=2)
     ex, W = build_expert(cfg)
@@ -122,6 +128,11 @@ def test_dataflow_wait_timeout_reports_status():
 @pytest.mark.parametrize("cluster", [16, 8])
 def test_pi05_bf16_bs1_dataflow(cluster):
     _case(wl.PI05_BF16_BS1.replace(name=f"pi05_bf16_bs1_df{cluster}"), cluster=cluster, graph_too=cluster == 16)
+
+
+@pytest.mark.slow
+def test_pi05_w4a16_bs1_dataflow():
+    _case(wl.PI05_W4A16_BS1.replace(name="pi05_w4a16_bs1_df"), graph_too=False)
 
 
 @pytest.mark.slow
