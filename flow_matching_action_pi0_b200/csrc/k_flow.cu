@@ -534,6 +534,10 @@ __device__ void mma_loop(const FC& c) {
           break;
         }
         ++sg;
+#ifdef PAE_FLOW_TRACE
+        const bool trm = k == a.k_begin && l == 1;
+        if (trm) g_flow_trace[c.cta * kTraceEv + st * 10 + 7] = globaltimer_ns();
+#endif
         tc_fence_after();
         for (int j = 0; ok && j < nt; ++j)
           for (int half = 0; ok && half < g.na; ++half, ++it) {
@@ -549,6 +553,9 @@ __device__ void mma_loop(const FC& c) {
                 ok = false;
                 break;
               }
+#ifdef PAE_FLOW_TRACE
+              if (trm && j == 0 && half == 0 && i == 0) g_flow_trace[c.cta * kTraceEv + st * 10 + 8] = globaltimer_ns();
+#endif
               tc_fence_after();
               const uint32_t sa = ring + (uint32_t)rs * kFBlk, sb = work + kFOp + (uint32_t)i * 8192u;
 #pragma unroll
@@ -559,6 +566,9 @@ __device__ void mma_loop(const FC& c) {
             }
             if (!ok) break;
             umma_commit(&c.acc_full[slot]);
+#ifdef PAE_FLOW_TRACE
+            if (trm && j == nt - 1 && half == g.na - 1) g_flow_trace[c.cta * kTraceEv + st * 10 + 9] = globaltimer_ns();
+#endif
           }
       }
   if (!ok && !*c.s_abort) raise_abort(c);
@@ -767,8 +777,8 @@ __device__ bool gemm_stage(const FC& c, int st, int k, int l, int u, int& it, in
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qd = warp & 3, row = qd * 32 + lane;  // TMEM lane = weight row
   const int per8 = R / 8, nitems = a.M * per8;
-  const int npass = nitems > 128 ? 2 : 1;
-  float keep[2][8];
+  const int npass = (nitems + 127) / 128;  // at most 4 (64 tokens x 8 row groups with C = 2)
+  float keep[4][8];
   for (int j = 0; j < nt; ++j) {
     const int t = c.cl + j * a.NC;
     for (int half = 0; half < g.na; ++half, ++it) {
@@ -814,7 +824,7 @@ __device__ bool gemm_stage(const FC& c, int st, int k, int l, int u, int& it, in
       if (j == 0 && half == 0) FTRACE(c, tr, tb + 4);
 #pragma unroll 1
       for (int pass = 0; pass < npass; ++pass) {  // uniform
-        if (pass == 1) load_in(1);
+        if (pass > 0) load_in(pass);
         const int idx = c.ct + pass * 128;
         const bool valid = idx < nitems;
         const int m = valid ? idx / per8 : 0, j8 = valid ? idx - (idx / per8) * per8 : 0;
@@ -823,12 +833,24 @@ __device__ bool gemm_stage(const FC& c, int st, int k, int l, int u, int& it, in
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = 0.f;
         if (valid) {
+          // up to 8 ranks' loads in flight at once (distributed shared memory
+          // has a long latency), then added in rank order
           const uint32_t la = pbase + (uint32_t)((m * 128 + r0) * 4);
-          for (int q = 0; q < C; ++q) {
-            const uint32_t ra = map_cluster(la, (uint32_t)q);
-            const float4 p0 = ld_cluster_f32x4(ra), p1 = ld_cluster_f32x4(ra + 16);
-            acc[0] += p0.x; acc[1] += p0.y; acc[2] += p0.z; acc[3] += p0.w;
-            acc[4] += p1.x; acc[5] += p1.y; acc[6] += p1.z; acc[7] += p1.w;
+          for (int q0 = 0; q0 < C; q0 += 8) {
+            float4 p[8][2];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              if (q0 + q < C) {
+                const uint32_t ra = map_cluster(la, (uint32_t)(q0 + q));
+                p[q][0] = ld_cluster_f32x4(ra);
+                p[q][1] = ld_cluster_f32x4(ra + 16);
+              }
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              if (q0 + q < C) {
+                acc[0] += p[q][0].x; acc[1] += p[q][0].y; acc[2] += p[q][0].z; acc[3] += p[q][0].w;
+                acc[4] += p[q][1].x; acc[5] += p[q][1].y; acc[6] += p[q][1].z; acc[7] += p[q][1].w;
+              }
           }
         }
         const int f0 = 128 * t + r0;
@@ -1000,15 +1022,24 @@ __device__ bool att_stage(const FC& c, int l, int u, int& ac, int& ncl, int& kv_
   c.s_ml[2 * r] = au.nch > 0 ? m_run : -INFINITY;
   c.s_ml[2 * r + 1] = au.nch > 0 ? l_run : 0.f;
   if (!cl_sync(c, ncl)) return false;
-  float Mx = -INFINITY;
+  // every rank's (max, sum) of this row, all loads in flight at once
+  float mq[16], lq[16];
   const uint32_t mla = smem_u32(c.s_ml + 2 * r);
-  for (int q = 0; q < C; ++q) Mx = fmaxf(Mx, ld_cluster_f32(map_cluster(mla, (uint32_t)q)));
+#pragma unroll
+  for (int q = 0; q < 16; ++q)
+    if (q < C) {
+      const uint32_t ra = map_cluster(mla, (uint32_t)q);
+      mq[q] = ld_cluster_f32(ra);
+      lq[q] = ld_cluster_f32(ra + 4);
+    }
+  float Mx = -INFINITY;
+#pragma unroll
+  for (int q = 0; q < 16; ++q)
+    if (q < C) Mx = fmaxf(Mx, mq[q]);
   float Ls = 0.f;
-  for (int q = 0; q < C; ++q) {
-    const uint32_t ra = map_cluster(mla, (uint32_t)q);
-    const float lq = ld_cluster_f32(ra + 4);
-    if (lq > 0.f) Ls = fmaf(exp2f(ld_cluster_f32(ra) - Mx), lq, Ls);
-  }
+#pragma unroll
+  for (int q = 0; q < 16; ++q)
+    if (q < C && lq[q] > 0.f) Ls = fmaf(exp2f(mq[q] - Mx), lq[q], Ls);
   const float w = (au.nch > 0 && l_run > 0.f && Ls > 0.f) ? exp2f(m_run - Mx) / Ls : 0.f;
   const uint32_t prow = smem_u32(c.work) + (uint32_t)(r * d * 4);
   for (int j = 0; j < d; j += 16) {
@@ -1038,9 +1069,16 @@ __device__ bool att_stage(const FC& c, int l, int u, int& ac, int& ncl, int& kv_
     if (rq >= GH) continue;
     const uint32_t la = smem_u32(c.work) + (uint32_t)(row * d * 4) + (((uint32_t)c4 ^ (uint32_t)(row & 7)) * 16u);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int q = 0; q < C; ++q) {
-      const float4 v = ld_cluster_f32x4(map_cluster(la, (uint32_t)q));
-      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    for (int q0 = 0; q0 < C; q0 += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (q0 + q < C) v[q] = ld_cluster_f32x4(map_cluster(la, (uint32_t)(q0 + q)));
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (q0 + q < C) {
+          acc.x += v[q].x; acc.y += v[q].y; acc.z += v[q].z; acc.w += v[q].w;
+        }
     }
     const int hl = rq / s.H, ti = rq - hl * s.H;
     bf16* orow = a.o + (size_t)(au.b * s.H + ti) * s.attn_dim + (au.g * s.G + hl) * d;

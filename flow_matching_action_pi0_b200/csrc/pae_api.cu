@@ -151,7 +151,7 @@ struct pae_ctx {
   // dataflow loop (batch * chunk <= 64): the MLP norm's operand, sums of
   // squares, the projected adaRMSNorm shifts per step, counters, 64-row maps
   bool flow_capable = false;
-  bool use_flow = true;
+  bool use_flow = false;  // opt-in until it beats the captured graph at batch 1
   int flow_cluster = 0;          // 0: automatic
   int flow_max_cl[17] = {};      // clusters of C CTAs that fit at once
   void* yg = nullptr;

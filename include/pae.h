@@ -202,11 +202,11 @@ pae_status pae_denoise_steps(pae_ctx* ctx, const float* x_in, float* x_out, int 
  * (statistics from the residual projections' epilogues) instead of separate
  * norm kernels, for batches of at most one 64-token tile.  Both round within
  * the parity tolerance; each is bitwise reproducible.
- * PAE_OPT_DATAFLOW (default 1, bf16 weights): batches with batch * chunk <= 64
+ * PAE_OPT_DATAFLOW (default 0, bf16 / int4 weights): batches with batch * chunk <= 64
  * run all K steps as one launch of thread-block clusters whose stages wait on
  * per-tile counters instead of kernel boundaries (no CUDA graph for these
  * batches; pae_denoise_steps takes the same path).  0 uses the captured graph
- * of per-stage kernels.  The two paths round differently (the dataflow loop
+ * of per-stage kernels (the faster one at the pi0.5 shape so far).  The two paths round differently (the dataflow loop
  * applies each adaRMSNorm's 1/rms after the projection and its shift as a
  * precomputed projected term); both stay within the parity tolerance and each
  * is bitwise reproducible.  PAE_OPT_DATAFLOW_CLUSTER (default 0 = automatic):

@@ -16,6 +16,7 @@ pytestmark = pytest.mark.gpu
 def _case(cfg, lengths=None, cluster=0, graph_too=True):
     ex, W = build_expert(cfg)
     try:
+        ex.set_option(fm.PAE_OPT_DATAFLOW, 1)
         if cluster:
             ex.set_option(fm.PAE_OPT_DATAFLOW_CLUSTER, cluster)
         ks, vs = wl.make_prefix(cfg, lengths=lengths)
@@ -71,6 +72,7 @@ def test_step_split_bitwise_and_host_buffers():
     cfg = wl.TINY_FP32.replace(name="tiny_bf16_df_split", dtype=wl.BF16, batch=2)
     ex, W = build_expert(cfg)
     try:
+        ex.set_option(fm.PAE_OPT_DATAFLOW, 1)
         ks, vs = wl.make_prefix(cfg, lengths=[64, 33])
         set_prefixes(ex, cfg, ks, vs)
         ex.precompute_tables(wl.uniform_grid(cfg.steps))
@@ -100,6 +102,7 @@ def test_dataflow_wait_timeout_reports_status():
     cfg = wl.TINY_FP32.replace(name="tiny_bf16_df_to", dtype=wl.BF16)
     ex, W = build_expert(cfg)
     try:
+        ex.set_option(fm.PAE_OPT_DATAFLOW, 1)
         ks, vs = wl.make_prefix(cfg)
         set_prefixes(ex, cfg, ks, vs)
         ex.precompute_tables(wl.uniform_grid(cfg.steps))
