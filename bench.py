@@ -111,6 +111,7 @@ class ClockSampler:
 
 
 FUSED_NORM = [0]  # PAE_OPT_FUSED_NORM for every context the benchmark creates
+DATAFLOW = [-1]   # PAE_OPT_DATAFLOW for every context (-1: the library default)
 
 
 def algorithmic(cfg: wl.ExpertConfig, batch: int, lens=None):
@@ -266,6 +267,8 @@ def setup_context(cfg, W, batch: int, lens=None):
     ex = fm.ActionExpert(fm.make_config(**wd.abi_config(cfg, max_batch=batch)), dev_w)
     del dev_w
     ex.set_option(fm.PAE_OPT_FUSED_NORM, FUSED_NORM[0])
+    if DATAFLOW[0] >= 0:
+        ex.set_option(fm.PAE_OPT_DATAFLOW, DATAFLOW[0])
     if lens is None:
         lens = [cfg.prefix] * batch
     ks, vs = wl.make_prefix(cfg, lengths=lens)
@@ -446,8 +449,9 @@ def run_minimal(args, cfg):
     with torch.cuda.stream(stream):
         ms = timed(lambda: ex.denoise(nd, od, stream), args.steps, args.warmup, stream, lambda: None)
     persist = ex.query(fm.PAE_Q_PERSISTENT, cfg.batch)
-    k = 1 if persist else ex.query(fm.PAE_Q_GRAPH_KERNELS, cfg.batch)
-    print(json.dumps({"workload": cfg.name, "pdl": args.pdl, "persistent": persist,
+    flow = ex.query(fm.PAE_Q_DATAFLOW, cfg.batch)
+    k = 1 if (persist or flow) else ex.query(fm.PAE_Q_GRAPH_KERNELS, cfg.batch)
+    print(json.dumps({"workload": cfg.name, "pdl": args.pdl, "persistent": persist, "dataflow": flow,
                       "max_splitk": args.max_splitk, "ms_per_step": ms,
                       "splits": ex.query(fm.PAE_Q_SPLITS, cfg.batch), "graph_kernels": k,
                       "launches_before_timed": 1 + cfg.batch + 4 + args.warmup * k}), flush=True)
@@ -686,6 +690,8 @@ def main():
     ap.add_argument("--max-splitk", type=int, default=0, help="cap on the projection split-K (0: library default)")
     ap.add_argument("--fused-norm", type=int, default=0,
                     help="adaRMSNorm inside the projections for batches of <= 64 tokens (1/0; 0 keeps norm kernels)")
+    ap.add_argument("--dataflow", type=int, default=-1,
+                    help="dataflow loop for batches of <= 64 tokens (1/0; -1 keeps the library default)")
     ap.add_argument("--persistent", type=int, default=0,
                     help="persistent kernel for batches of <= 64 tokens (1/0; 0 runs the captured graph)")
     args = ap.parse_args()
@@ -693,6 +699,7 @@ def main():
         args.warmup = 3
     cfg = wl.CONFIGS[args.config]
     FUSED_NORM[0] = args.fused_norm
+    DATAFLOW[0] = args.dataflow
     if args.impl == "reference":
         return run_reference(args, cfg)
     if args.minimal:

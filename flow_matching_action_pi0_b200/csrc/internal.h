@@ -206,8 +206,9 @@ struct FlowArgs {
   int M, B;                          // tokens, requests
   int C, NC;                         // cluster size, clusters
   int k_begin, k_end;                // Euler steps of this launch
-  int q_tiles, o_tiles, g_pairs, d_tiles;  // 128-row weight tiles (gate/up: pairs)
-  int kb_q, kb_o, kb_g, kb_d;        // 64-wide K blocks per rank
+  int q_units, o_tiles, g_units, d_tiles;  // QKV / gate-up whole-K units, O / down split-K tiles (128 rows)
+  int q_base, o_base, g_base, d_base, a_base;  // first CTA (units) or cluster (tiles, attention)
+  int kb_q, kb_o, kb_g, kb_d;        // 64-wide K blocks per unit (QKV, gate/up) or per rank (O, down)
   int a_units, a_qtiles, a_kps;      // attention clusters, query tiles per (b, kv head), keys per rank
   float* x;
   float* h;
@@ -239,9 +240,10 @@ struct FlowArgs {
 size_t flow_smem_bytes();
 cudaError_t flow_init();
 int flow_max_clusters(int C);        // clusters of C CTAs that fit at once (0 on error)
-// maps: W qkv, W o, W gate/up (128-row boxes), W down (bf16 [128][64] boxes, or
-// with w4 the packed [128 rows][32 bytes] boxes), y_q, o, y_g, u (64 x 64
-// boxes), q (64 x 128), k, v (64 x 64).  Cooperative cluster launch.
+// maps: W qkv, W o, W gate/up (64-row boxes), W down (bf16 [128][64] boxes,
+// gate/up [64][64]; with w4 the packed [128 rows][32 bytes] boxes, gate/up
+// [64][32 bytes]), y_q, o, y_g, u (64 x 64 boxes), q (64 x 128), k, v
+// (64 x 64).  Cooperative cluster launch.
 cudaError_t launch_flow(const Shape& s, const CUtensorMap* maps, const FlowArgs& a, cudaStream_t st);
 
 }  // namespace pae

@@ -10,40 +10,50 @@
 //   O  h += gate_a * (o W_o^T)
 //   G  u = gelu(norm(h) W_gate^T) * (norm(h) W_up^T)
 //   D  h += gate_m * (u W_down^T)
-// waits only for the data it reads, through per-tile counters in global
+// waits only for the data it reads, through per-unit counters in global
 // memory (release / acquire), never for a grid-wide barrier.
 //
-// Work split.  The grid is NC clusters of C CTAs (one CTA per SM).  A
-// projection's 128-row weight tiles go to clusters round robin; the K range of
-// a tile is split over the C ranks of its cluster, each rank multiplying its
-// K slice of the token operand by its slice of the weights (tcgen05, weights
-// as the MMA's M side, tokens as N = 64, fp32 accumulators in TMEM).  The C
-// partial tiles are summed inside the cluster: every rank parks its partial
-// in its own shared memory, a cluster barrier, then rank q adds rows
-// [q R, q R + R) of all C partials (distributed shared memory loads, in rank
-// order, so results are bitwise reproducible) and runs the epilogue for them.
-// Attention: one cluster per (request, KV head, 128 query rows), its ranks
-// taking consecutive 64-key chunks; partial outputs are merged the same way.
+// Work split.  The grid is NC clusters of C CTAs (one CTA per SM).
+//  * QKV and gate/up (K = width) are cut into 128-row units, and one CTA
+//    multiplies a unit over the whole K range (tcgen05, weights as the MMA's
+//    M side, tokens as N = 64, fp32 accumulators in TMEM): no partial sum
+//    leaves the CTA.  A gate/up unit holds 64 gate rows and the 64 up rows of
+//    the same features (two 64-row weight boxes per K block), so the unit's
+//    own epilogue forms the GeGLU product.
+//  * O and down (K = heads x head_dim, and the MLP width) split K over the C
+//    ranks of a cluster, one 128-row tile per cluster.  The C partial tiles
+//    are summed by a reduce-scatter inside the cluster: rank p stores rows
+//    [q R, q R + R) of its partial, straight from registers, into rank q's
+//    shared memory (st.async, counted in bytes by q's mbarrier), and rank q
+//    adds the C slices in rank order (bitwise reproducible) and runs the
+//    epilogue for its R = 128 / C rows.
+//  * Attention: one cluster per (request, KV head, 128 query rows), its ranks
+//    taking consecutive 64-key chunks (online softmax); rank p stores its
+//    unnormalised output rows with their running max and sum into the rows'
+//    owner, which merges the C partial softmaxes.
+// A receiver tells its peers that its receive area is free (one remote
+// mbarrier arrival each) as soon as it is, long before the data is ready, so
+// an exchange costs no cluster barrier.
 //
 // adaRMSNorm.  y = h rstd (1 + scale) + shift is not formed: the producer of
 // h writes bf16(h (1 + scale)) and per-row sums of squares once, and the
-// consumer's reducer applies rstd after the contraction and adds the shift
+// consumer's epilogue applies rstd after the contraction and adds the shift
 // term W shift from a table built with the timestep tables.  The same value
-// as W y, with no re-normalisation of fp32 h in every tile.
+// as W y, with no re-normalisation of fp32 h in every unit.
 //
 // Weights never depend on activations: warp 0 streams this CTA's weight
 // blocks into a ring of shared memory in schedule order and prefetches the
 // same blocks of the next layer into L2, so HBM keeps streaming while the
 // dependency chain runs.  Warp 1 issues the MMAs; warps 2-5 do the rest
-// (token operands by TMA, TMEM reads, cluster reductions, epilogues, the
-// attention softmax and the per-token transition between Euler steps).
+// (token operands by TMA, TMEM reads, exchanges, epilogues, the attention
+// softmax and the per-token transition between Euler steps).
 //
 // Every wait is bounded (%globaltimer).  A wait that runs out records
 // PAE_ERR_TIMEOUT and sets a launch-wide abort flag that every other wait
-// watches; cluster barriers are mbarrier-based and bounded too.  Before exit
-// every CTA drains its copies and MMAs and meets its cluster once more (a
-// hardware cluster barrier that all threads reach on every path), so no CTA
-// leaves while a peer may still read its shared memory.
+// watches.  Before exit every CTA drains its copies, MMAs and any exchange
+// still open, and meets its cluster once more (a hardware cluster barrier
+// that all threads reach on every path), so no CTA leaves while a peer may
+// still write its shared memory.
 #include "epilogue.cuh"
 #include "launch.cuh"
 
@@ -57,23 +67,25 @@ constexpr int kFRing = 5;                // bf16 weight ring depth (W4A16: 4 slo
 constexpr int kFRawRing = 4;             // packed int4 blocks [128 rows][32 bytes] in flight (W4A16)
 constexpr uint32_t kFRawBlk = 4096;
 constexpr uint32_t kFBlk = 16384;        // [128 rows][64] bf16 weight block
-constexpr uint32_t kFWork = 128 * 1024;  // operands, partial tiles, attention tiles
+constexpr uint32_t kFWork = 128 * 1024;  // operands, epilogue tiles, attention tiles, receive areas
 constexpr uint32_t kFMisc = 4096;
 constexpr uint32_t kFSmem = kFRing * kFBlk + kFWork + kFMisc + 1024;
-constexpr uint32_t kFOp = 0;             // token operand [kbr][64 tokens][64] bf16
-constexpr uint32_t kFPart = 64 * 1024;   // two partial tiles [64 tokens][128 rows] fp32
+constexpr uint32_t kFOp = 0;             // token operand [kb][64 tokens][64] bf16
+constexpr uint32_t kFRx = 64 * 1024;     // split-K receive area [C][R rows][Mp tokens] fp32 (<= 32 KB)
 constexpr uint32_t kFTmem = 512;
 constexpr uint32_t kColS = 128;          // attention scores (P over their first 32 columns)
 constexpr uint32_t kColO = 256;          // attention output
 constexpr int CKF = 64;                  // keys per attention chunk
 constexpr long long kFDrain = 4000000000LL;
+constexpr long long kFExitWait = 2000000LL;  // an exchange left open by an abort, at exit
 
 enum : int { ST_Q = 0, ST_O = 1, ST_G = 2, ST_D = 3 };
 
 // Stage timestamps for performance analysis, compiled in only with
-// -DPAE_FLOW_TRACE: compute thread 0 of every CTA records %globaltimer at
-// fixed points of one layer (layer 1 of the first step of a launch) into
-// g_flow_trace[cta][event]; pae_flow_trace_read copies them out.
+// -DPAE_FLOW_TRACE: compute thread 0 (events 0-6 of a stage, 40-47 of
+// attention) and the MMA thread (events 7-9 of a stage) of every CTA record
+// %globaltimer at fixed points of one layer (layer 1 of the first step of a
+// launch) into g_flow_trace[cta][event]; pae_flow_trace_read copies them out.
 #ifdef PAE_FLOW_TRACE
 constexpr int kTraceEv = 48;
 __device__ unsigned long long g_flow_trace[256 * kTraceEv];
@@ -97,7 +109,6 @@ __device__ __forceinline__ void red_release_u32(unsigned* p, unsigned v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async_global_f() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
-__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
 __device__ __forceinline__ void csync() {
   __syncwarp();
   asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -150,8 +161,26 @@ __device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
   asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
+// Stores into another CTA's shared memory whose completion is counted (in
+// bytes) by an mbarrier of that CTA.
+__device__ __forceinline__ void st_async_f4(uint32_t addr, float4 v, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+               "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(rbar)
+               : "memory");
+}
+__device__ __forceinline__ void st_async_f2(uint32_t addr, float a, float b, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(addr), "f"(a),
+               "f"(b), "r"(rbar)
+               : "memory");
+}
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
+
 struct FMaps {
-  const CUtensorMap* w[4];   // Q, O, G (128-row boxes), D weights
+  const CUtensorMap* w[4];   // weights: Q, O, D with 128-row boxes; G with 64-row boxes
   const CUtensorMap* x[4];   // token operands: y (QKV), o, y (gate/up), u
   const CUtensorMap *q, *k, *v;
 };
@@ -167,22 +196,24 @@ struct FC {
   uint64_t* raw_full;  // [kFRawRing] packed int4 block landed (W4A16)
   uint8_t* raw;        // packed int4 ring (W4A16)
   int nring;           // ring depth in use (kFRing, or kFRing - 1 with the int4 ring)
-  uint64_t* op_full;   // token operand of a projection stage landed
-  uint64_t* acc_full;  // [2] accumulator slot ready
-  uint64_t* acc_empty; // [2] accumulator slot read out
+  uint64_t* op_full;   // [4] token operand groups of a projection stage landed
+  uint64_t* acc_full;  // [2] split-K accumulator slot ready
+  uint64_t* acc_empty; // [2] split-K accumulator slot read out
+  uint64_t* acc_all;   // every whole-K unit of a stage accumulated
   uint64_t* kv_full;   // attention q / K / V chunk landed
   uint64_t* s_full;
   uint64_t* p_full;
   uint64_t* o_full;
-  uint64_t* cbar;      // [2] cluster barrier (count C), alternating instances
+  uint64_t* rx;        // exchange: this CTA's receive area filled (1 arrival + bytes)
+  uint64_t* rdy;       // exchange: every peer's receive area free (C - 1 arrivals)
   uint64_t* drain;
   float* s_rstd;       // [64]
   float* s_tmp;        // [512]
-  float* s_ml;         // [128][2] attention row max / sum
+  float* s_st;         // [C][R][2] attention (max, sum) received for this rank's rows
   volatile int* s_abort;
   volatile int* s_flag;
   uint32_t tmem;
-  int cta, cl, rank, ct;  // ct: compute-thread index 0..127
+  int cta, ncta, cl, rank, ct;  // ct: compute-thread index 0..127
 };
 
 __device__ __forceinline__ unsigned* abort_word(const FlowArgs& a) { return a.ctr + kFlowCtrWords - 1; }
@@ -194,13 +225,15 @@ __device__ void raise_abort(const FC& c) {
   set_error(c.a->err, DEV_TIMEOUT);
 }
 
-// Bounded mbarrier wait that also gives up once the launch is aborting.
+// Bounded mbarrier wait (acquire at cluster scope, which also covers data
+// that other CTAs of the cluster stored) that gives up once the launch is
+// aborting.
 __device__ bool fwait(const FC& c, uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_cl(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   const volatile unsigned* ab = abort_word(*c.a);
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_cl(bar, parity)) return true;
     if (*c.s_abort || *ab) {
       *c.s_abort = 1;
       return false;
@@ -237,67 +270,80 @@ __device__ void publish(const FC& c, unsigned* p) {
   if (c.ct == 0) red_release_u32(p, 1u);
 }
 
-// Cluster barrier among the compute threads of the C ranks, bounded: every
-// rank's compute thread 0 arrives (release, cluster scope) on instance n's
-// mbarrier of every rank, then waits (acquire) on its own.  Instances
-// alternate between two mbarriers, so an early arrival for instance n + 1 can
-// never complete instance n.  Returns false once the launch is aborting.
-__device__ bool cl_sync(const FC& c, int& n) {
-  fence_acq_rel_cluster();
-  csync();
-  uint64_t* b = &c.cbar[n & 1];
-  // compute thread r arrives on rank r's instance (one remote arrive each)
-  if (c.ct < c.a->C && !*c.s_abort) mbar_arrive_remote(map_cluster(smem_u32(b), (uint32_t)c.ct));
-  if (c.ct == 0) {
-    bool ok = !*c.s_abort;
-    if (ok) {
-      const uint32_t par = (uint32_t)(n >> 1) & 1u;
-      ok = mbar_try_wait_cl(b, par);
-      if (!ok) {
-        const unsigned long long t0 = globaltimer_ns();
-        const volatile unsigned* ab = abort_word(*c.a);
-        while (!(ok = mbar_try_wait_cl(b, par))) {
-          if (*ab) {
-            *c.s_abort = 1;
-            break;
-          }
-          if ((long long)(globaltimer_ns() - t0) > c.a->err.wait_ns) {
-            raise_abort(c);
-            break;
-          }
-        }
-      }
-    }
-    *c.s_flag = ok ? 1 : 0;
+// ------------------------------------------------------------ exchanges
+// An exchange moves data between the C ranks of a cluster into each rank's
+// receive area.  `xn` counts this CTA's exchanges; every rank of a cluster
+// takes part in the same exchanges in the same order, so the mbarrier phases
+// agree.
+//  open:  the receive area is free: arm rx for `bytes` from the peers, then
+//         one remote arrival on every peer's rdy (release: everything this
+//         CTA did with the area before is ordered before the peers' stores).
+//  ready: every peer's area is free (rdy complete), so stores may start.
+//  wait:  every peer's bytes landed (rx complete) and this CTA's own slice,
+//         written with plain stores, is visible to all compute threads.
+__device__ void xchg_open(const FC& c, uint32_t bytes) {
+  const int C = c.a->C;
+  if (C == 1 || c.ct != 0 || *c.s_abort) return;
+  mbar_arrive_expect_tx(c.rx, bytes);
+  for (int q = 1; q < C; ++q) {
+    const uint32_t peer = (uint32_t)((c.rank + q) % C);
+    mbar_arrive_remote(map_cluster(smem_u32(c.rdy), peer));
   }
-  csync();
-  ++n;
-  return *c.s_flag != 0;
+}
+__device__ bool xchg_ready(const FC& c, int xn) {
+  if (c.a->C == 1) return true;
+  bool ok = true;
+  if (c.ct == 0) ok = !*c.s_abort && fwait(c, c.rdy, (uint32_t)xn & 1u);
+  if (!cand(ok)) return false;
+  return mbar_try_wait_cl(c.rdy, (uint32_t)xn & 1u);  // each thread's own acquire (complete by now)
+}
+__device__ bool xchg_wait(const FC& c, int xn) {
+  csync();  // own slice stored
+  if (c.a->C == 1) return true;
+  bool ok = true;
+  if (c.ct == 0) ok = !*c.s_abort && fwait(c, c.rx, (uint32_t)xn & 1u);
+  if (!cand(ok)) return false;
+  return mbar_try_wait_cl(c.rx, (uint32_t)xn & 1u);
 }
 
 // ------------------------------------------------------------ schedule
-// Projection stage geometry: output tiles (G: pairs of a gate and an up tile),
-// K blocks per rank, weight rows per layer and the first row of an item.
+// Projection stage geometry: units (Q, G: 128-row whole-K units; O, D:
+// 128-row tiles split over the cluster), K blocks per unit or per rank, and
+// weight rows per layer.
 struct StageG {
-  int ntiles, na, kbr, wrows;
+  int units, kb, wrows;
+  bool whole;
 };
 __device__ __forceinline__ StageG stage_geo(const Shape& s, const FlowArgs& a, int st) {
-  StageG g;
   switch (st) {
-    case ST_Q: g = StageG{a.q_tiles, 1, a.kb_q, s.qkv_rows}; break;
-    case ST_O: g = StageG{a.o_tiles, 1, a.kb_o, s.D}; break;
-    case ST_G: g = StageG{a.g_pairs, 2, a.kb_g, 2 * s.F}; break;
-    default: g = StageG{a.d_tiles, 1, a.kb_d, s.D}; break;
+    case ST_Q: return StageG{a.q_units, a.kb_q, s.qkv_rows, true};
+    case ST_O: return StageG{a.o_tiles, a.kb_o, s.D, false};
+    case ST_G: return StageG{a.g_units, a.kb_g, 2 * s.F, true};
+    default: return StageG{a.d_tiles, a.kb_d, s.D, false};
   }
-  return g;
 }
-// Tiles of a stage handled by cluster cl: cl, cl + NC, ...
-__device__ __forceinline__ int cl_tiles(const FlowArgs& a, int ntiles, int cl) {
-  return cl < ntiles ? (ntiles - cl + a.NC - 1) / a.NC : 0;
+// Units owned by this CTA (whole-K: unit i runs on CTA (base + i) mod ncta)
+// or by its cluster (tiles: tile t runs on cluster (base + t) mod NC): the
+// count, and the first one in `first`; the others follow every n.
+__device__ __forceinline__ int owned(const FC& c, int st, const StageG& g, int& first) {
+  const FlowArgs& a = *c.a;
+  const bool w = g.whole;
+  const int n = w ? c.ncta : a.NC, me = w ? c.cta : c.cl;
+  const int base = st == ST_Q ? a.q_base : st == ST_O ? a.o_base : st == ST_G ? a.g_base : a.d_base;
+  first = ((me - base) % n + n) % n;
+  return first < g.units ? (g.units - first + n - 1) / n : 0;
 }
-// Stored weight row of item (tile t, half) in layer l.
-__device__ __forceinline__ int item_row(const StageG& g, int l, int t, int half) {
-  return l * g.wrows + (g.na == 2 ? 256 * t + 128 * half : 128 * t);
+__device__ __forceinline__ int unit_step(const FC& c, const StageG& g) { return g.whole ? c.ncta : c.a->NC; }
+// Stored weight rows of unit / tile t in layer l: the first box's first row,
+// and the second 64-row half's (gate/up: the up rows of the same features).
+__device__ __forceinline__ void unit_rows(const Shape& s, int st, const StageG& g, int l, int t, int& r0, int& r1) {
+  if (st == ST_G) {
+    r0 = l * g.wrows + 256 * (t >> 1) + 64 * (t & 1);
+    r1 = r0 + 128;
+  } else {
+    r0 = l * g.wrows + 128 * t;
+    r1 = r0 + 64;
+  }
 }
 
 // Attention unit of cluster cl: (request b, KV head g, 128-row query tile
@@ -308,10 +354,11 @@ struct AttU {
 };
 __device__ __forceinline__ AttU att_unit(const Shape& s, const FlowArgs& a, int cl, int rank) {
   AttU u{};
-  u.has = cl < a.a_units;
+  const int unit = ((cl - a.a_base) % a.NC + a.NC) % a.NC;
+  u.has = unit < a.a_units;
   if (!u.has) return u;
-  u.bg = cl / a.a_qtiles;
-  u.qt = cl - u.bg * a.a_qtiles;
+  u.bg = unit / a.a_qtiles;
+  u.qt = unit - u.bg * a.a_qtiles;
   u.b = u.bg / s.Hkv;
   u.g = u.bg - u.b * s.Hkv;
   const int n_valid = __ldg(a.lens + u.b) + s.H;  // set before the launch, fixed during it
@@ -327,20 +374,28 @@ __device__ __forceinline__ unsigned* c_qkv(const FlowArgs& a) { return a.ctr + 1
 __device__ __forceinline__ unsigned* c_att(const FlowArgs& a) { return a.ctr + 2; }
 __device__ __forceinline__ unsigned* c_y(const FlowArgs& a, int t) { return a.ctr + 3 + t; }
 __device__ __forceinline__ unsigned* c_ho(const FlowArgs& a, int t) { return a.ctr + 3 + a.d_tiles + t; }
-__device__ __forceinline__ unsigned* c_u(const FlowArgs& a, int p) { return a.ctr + 3 + a.d_tiles + a.o_tiles + p; }
+__device__ __forceinline__ unsigned* c_u(const FlowArgs& a, int j) { return a.ctr + 3 + a.d_tiles + a.o_tiles + j; }
+
+// Operand groups: the K blocks of a stage's token operand arrive in up to 4
+// groups, each on its own mbarrier, so the first MMAs start before the last
+// blocks land.  Group gi holds blocks [gi gsz, min(kb, (gi + 1) gsz)).
+__device__ __forceinline__ int op_gsz(int kb) { return (kb + 3) / 4; }
 
 // ------------------------------------------------------------ weight producer
-// Weight block n of this CTA's schedule (per step, layer, stage, item, K block):
-// which matrix, its K offset (elements), its first weight row, and the same
-// block's row in the next layer (or layer 0 of the next step; -1: none).
+// Weight block n of this CTA's schedule (per step, layer, stage, unit, K
+// block): which matrix, its K offset (elements), the rows of its two 64-row
+// halves, and the row offset of the same block in the next layer (or layer 0
+// of the next step; `last`: none).
 struct Blk {
-  int st, x, row0, nrow, kofs;
+  int st, kofs, row0, row1, dnext;
+  bool last;
 };
 __device__ __forceinline__ int blocks_per_layer(const FC& c) {
   int n = 0;
   for (int st = 0; st < 4; ++st) {
     const StageG g = stage_geo(*c.s, *c.a, st);
-    n += cl_tiles(*c.a, g.ntiles, c.cl) * g.na * g.kbr;
+    int first;
+    n += owned(c, st, g, first) * g.kb;
   }
   return n;
 }
@@ -352,18 +407,17 @@ __device__ bool block_at(const FC& c, int nbl, int n, Blk& b) {
   if (kl >= (a.k_end - a.k_begin) * s.L) return false;
   int r = n - kl * nbl;
   const int l = kl % s.L;
-  const bool last = kl + 1 >= (a.k_end - a.k_begin) * s.L;
   for (int st = 0; st < 4; ++st) {
     const StageG g = stage_geo(s, a, st);
-    const int cnt = cl_tiles(a, g.ntiles, c.cl) * g.na * g.kbr;
+    int first;
+    const int cnt = owned(c, st, g, first) * g.kb;
     if (r < cnt) {
-      const int item = r / g.kbr, i = r - item * g.kbr;
-      const int j = item / g.na, half = item - j * g.na;
+      const int item = r / g.kb, i = r - item * g.kb;
       b.st = st;
-      b.kofs = (c.rank * g.kbr + i) * 64;
-      b.x = b.kofs;
-      b.row0 = item_row(g, l, c.cl + j * a.NC, half);
-      b.nrow = last ? -1 : (l + 1 < s.L ? b.row0 + g.wrows : b.row0 - (s.L - 1) * g.wrows);
+      b.kofs = (g.whole ? i : c.rank * g.kb + i) * 64;
+      unit_rows(s, st, g, l, first + item * unit_step(c, g), b.row0, b.row1);
+      b.last = kl + 1 >= (a.k_end - a.k_begin) * s.L;
+      b.dnext = l + 1 < s.L ? g.wrows : -(s.L - 1) * g.wrows;
       return true;
     }
     r -= cnt;
@@ -383,12 +437,13 @@ __device__ __forceinline__ uint32_t dq_pair(uint32_t w, int i, __nv_bfloat162 sc
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// Warp 0.  bf16 weights: lane 0 streams this CTA's weight blocks (16 KB) into
-// the ring in schedule order.  int4 weights: lane 0 keeps kFRawRing packed
-// blocks (4 KB) in flight; all 32 lanes turn each landed block into a bf16
-// block of the ring (4 rows per lane, 128-byte swizzled like a TMA tile).
-// Either way each load also prefetches the same block of the next layer into
-// L2, so HBM streams one layer ahead of the dependency chain.
+// Warp 0.  bf16 weights: lane 0 streams this CTA's weight blocks (16 KB: one
+// 128-row box, or for gate/up two 64-row boxes) into the ring in schedule
+// order.  int4 weights: lane 0 keeps kFRawRing packed blocks (4 KB) in
+// flight; all 32 lanes turn each landed block into a bf16 block of the ring
+// (4 rows per lane, 128-byte swizzled like a TMA tile).  Either way each load
+// also prefetches the same block of the next layer into L2, so HBM streams
+// one layer ahead of the dependency chain.
 __device__ void producer_warp(const FC& c) {
   const FlowArgs& a = *c.a;
   const int lane = threadIdx.x & 31;
@@ -406,9 +461,20 @@ __device__ void producer_warp(const FC& c) {
           ok = false;
           break;
         }
+        uint8_t* dst = c.ring + (size_t)slot * kFBlk;
+        const CUtensorMap* tm = c.mp.w[b.st];
         mbar_arrive_expect_tx(&c.rfull[slot], kFBlk);
-        tma_load_2d_hint(c.ring + (size_t)slot * kFBlk, c.mp.w[b.st], b.x, b.row0, &c.rfull[slot], pol);
-        if (b.nrow >= 0) tma_prefetch_l2(c.mp.w[b.st], b.x, b.nrow);
+        if (b.st == ST_G) {
+          tma_load_2d_hint(dst, tm, b.kofs, b.row0, &c.rfull[slot], pol);
+          tma_load_2d_hint(dst + kFBlk / 2, tm, b.kofs, b.row1, &c.rfull[slot], pol);
+          if (!b.last) {
+            tma_prefetch_l2(tm, b.kofs, b.row0 + b.dnext);
+            tma_prefetch_l2(tm, b.kofs, b.row1 + b.dnext);
+          }
+        } else {
+          tma_load_2d_hint(dst, tm, b.kofs, b.row0, &c.rfull[slot], pol);
+          if (!b.last) tma_prefetch_l2(tm, b.kofs, b.row0 + b.dnext);
+        }
       }
       // copies still in flight land before the CTA exits
       for (int j = n > R ? n - R : 0; j < n; ++j)
@@ -423,9 +489,20 @@ __device__ void producer_warp(const FC& c) {
     Blk b;
     if (!block_at(c, nbl, m, b)) return false;
     const int rs = m % kFRawRing;
+    uint8_t* dst = c.raw + (size_t)rs * kFRawBlk;
+    const CUtensorMap* tm = c.mp.w[b.st];
     mbar_arrive_expect_tx(&c.raw_full[rs], kFRawBlk);
-    tma_load_2d_hint(c.raw + (size_t)rs * kFRawBlk, c.mp.w[b.st], b.x / 2, b.row0, &c.raw_full[rs], pol);
-    if (b.nrow >= 0) tma_prefetch_l2(c.mp.w[b.st], b.x / 2, b.nrow);
+    if (b.st == ST_G) {
+      tma_load_2d_hint(dst, tm, b.kofs / 2, b.row0, &c.raw_full[rs], pol);
+      tma_load_2d_hint(dst + kFRawBlk / 2, tm, b.kofs / 2, b.row1, &c.raw_full[rs], pol);
+      if (!b.last) {
+        tma_prefetch_l2(tm, b.kofs / 2, b.row0 + b.dnext);
+        tma_prefetch_l2(tm, b.kofs / 2, b.row1 + b.dnext);
+      }
+    } else {
+      tma_load_2d_hint(dst, tm, b.kofs / 2, b.row0, &c.raw_full[rs], pol);
+      if (!b.last) tma_prefetch_l2(tm, b.kofs / 2, b.row0 + b.dnext);
+    }
     return true;
   };
   if (lane == 0)
@@ -440,16 +517,18 @@ __device__ void producer_warp(const FC& c) {
       ok = false;
       break;
     }
-    // rows lane, lane + 32, lane + 64, lane + 96 of the block
+    // rows lane, lane + 32, lane + 64, lane + 96 of the block; rows 64.. are
+    // the second box (gate/up: the up rows)
     const StageG g = stage_geo(*c.s, a, b.st);
-    const int K = g.kbr * 64 * a.C;  // the matrix's K
+    const int K = g.whole ? g.kb * 64 : g.kb * 64 * a.C;  // the matrix's K
     const int gpr = K / 128, grp = b.kofs / 128;
     const uint8_t* rb = c.raw + (size_t)rs * kFRawBlk;
     const uint32_t ab = smem_u32(c.ring + (size_t)slot * kFBlk);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int r = lane + 32 * q;
-      const bf16 sv = a.wsc[b.st][(size_t)(b.row0 + r) * gpr + grp];
+      const int srow = r < 64 ? b.row0 + r : b.row1 + (r - 64);
+      const bf16 sv = a.wsc[b.st][(size_t)srow * gpr + grp];
       const __nv_bfloat162 sc = __halves2bfloat162(sv, sv);
       const uint4 w0 = *reinterpret_cast<const uint4*>(rb + r * 32);
       const uint4 w1 = *reinterpret_cast<const uint4*>(rb + r * 32 + 16);
@@ -479,10 +558,12 @@ __device__ void producer_warp(const FC& c) {
 }
 
 // ------------------------------------------------------------ MMA issuer
-// Warp 1, lane 0.  Projection item: D[128 rows][64 tokens] (TMEM slot it % 2)
-// = sum over this rank's K blocks of weights [128][64] x operand [64][64]^T.
-// Attention chunk: S = Q K^T (M = 128 query rows, N = 64 keys), then
-// O += P V with P read from TMEM and V MN-major from shared memory.
+// Warp 1, lane 0.  Whole-K stage: unit j of this CTA accumulates
+// D[128 rows][64 tokens] in TMEM columns 64 j over all K blocks, one commit
+// for the stage.  Split-K stage: tile item it accumulates this rank's K
+// blocks in slot it % 2 (columns 0 / 64), one commit per item.  Attention
+// chunk: S = Q K^T (M = 128 query rows, N = 64 keys), then O += P V with P
+// read from TMEM and V MN-major from shared memory.
 __device__ void mma_loop(const FC& c) {
   const Shape& s = *c.s;
   const FlowArgs& a = *c.a;
@@ -493,7 +574,8 @@ __device__ void mma_loop(const FC& c) {
   const uint32_t work = smem_u32(c.work), ring = smem_u32(c.ring);
   const uint32_t qbytes = 128u * d * 2u, kvbytes = (uint32_t)CKF * d * 2u;
   const AttU au = att_unit(s, a, c.cl, c.rank);
-  int n = 0, it = 0, sg = 0, ac = 0;
+  int n = 0, it = 0, ac = 0;
+  int opn[4] = {0, 0, 0, 0};
   bool ok = true;
   for (int k = a.k_begin; ok && k < a.k_end; ++k)
     for (int l = 0; ok && l < s.L; ++l)
@@ -527,49 +609,65 @@ __device__ void mma_loop(const FC& c) {
         }
         const int st = st5 == 0 ? ST_Q : st5 - 1;
         const StageG g = stage_geo(s, a, st);
-        const int nt = cl_tiles(a, g.ntiles, c.cl);
-        if (nt == 0) continue;
-        if (!fwait(c, c.op_full, sg & 1)) {
-          ok = false;
-          break;
-        }
-        ++sg;
+        int first;
+        const int nu = owned(c, st, g, first);
+        if (nu == 0) continue;
+        const int gsz = op_gsz(g.kb);
 #ifdef PAE_FLOW_TRACE
         const bool trm = k == a.k_begin && l == 1;
-        if (trm) g_flow_trace[c.cta * kTraceEv + st * 10 + 7] = globaltimer_ns();
 #endif
-        tc_fence_after();
-        for (int j = 0; ok && j < nt; ++j)
-          for (int half = 0; ok && half < g.na; ++half, ++it) {
+        for (int j = 0; ok && j < nu; ++j) {
+          uint32_t col;
+          if (g.whole) {
+            col = 64u * (uint32_t)j;
+          } else {
             const int slot = it & 1;
             if (it >= 2 && !fwait(c, &c.acc_empty[slot], ((it >> 1) & 1) ^ 1)) {
               ok = false;
               break;
             }
-            tc_fence_after();
-            for (int i = 0; i < g.kbr; ++i, ++n) {
-              const int rs = n % c.nring;
-              if (!fwait(c, &c.rfull[rs], (n / c.nring) & 1)) {
+            col = 64u * (uint32_t)slot;
+          }
+          tc_fence_after();
+          for (int i = 0; i < g.kb; ++i, ++n) {
+            if (j == 0 && i % gsz == 0) {
+              const int gi = i / gsz;
+              if (!fwait(c, &c.op_full[gi], (uint32_t)opn[gi] & 1u)) {
                 ok = false;
                 break;
               }
+              ++opn[gi];
 #ifdef PAE_FLOW_TRACE
-              if (trm && j == 0 && half == 0 && i == 0) g_flow_trace[c.cta * kTraceEv + st * 10 + 8] = globaltimer_ns();
+              if (trm && gi == 0) g_flow_trace[c.cta * kTraceEv + st * 10 + 7] = globaltimer_ns();
 #endif
-              tc_fence_after();
-              const uint32_t sa = ring + (uint32_t)rs * kFBlk, sb = work + kFOp + (uint32_t)i * 8192u;
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                umma_bf16(c.tmem + (uint32_t)slot * 64u, sw128_desc(sa + kk * 32, 16, 1024),
-                          sw128_desc(sb + kk * 32, 16, 1024), idg, (i > 0 || kk > 0) ? 1u : 0u);
-              umma_commit(&c.rempty[rs]);
             }
-            if (!ok) break;
-            umma_commit(&c.acc_full[slot]);
+            const int rs = n % c.nring;
+            if (!fwait(c, &c.rfull[rs], (n / c.nring) & 1)) {
+              ok = false;
+              break;
+            }
 #ifdef PAE_FLOW_TRACE
-            if (trm && j == nt - 1 && half == g.na - 1) g_flow_trace[c.cta * kTraceEv + st * 10 + 9] = globaltimer_ns();
+            if (trm && j == 0 && i == 0) g_flow_trace[c.cta * kTraceEv + st * 10 + 8] = globaltimer_ns();
 #endif
+            tc_fence_after();
+            const uint32_t sa = ring + (uint32_t)rs * kFBlk, sb = work + kFOp + (uint32_t)i * 8192u;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16(c.tmem + col, sw128_desc(sa + kk * 32, 16, 1024), sw128_desc(sb + kk * 32, 16, 1024), idg,
+                        (i > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(&c.rempty[rs]);
           }
+          if (!ok) break;
+          if (!g.whole) {
+            umma_commit(&c.acc_full[it & 1]);
+            ++it;
+          }
+        }
+        if (!ok) break;
+        if (g.whole) umma_commit(c.acc_all);
+#ifdef PAE_FLOW_TRACE
+        if (trm) g_flow_trace[c.cta * kTraceEv + st * 10 + 9] = globaltimer_ns();
+#endif
       }
   if (!ok && !*c.s_abort) raise_abort(c);
   // every MMA this thread issued must finish before TMEM is freed
@@ -641,14 +739,13 @@ __device__ void epi_q(const FC& c, int k, int l, int m, int f0, const float* acc
   }
 }
 
-// Epilogue inputs of one reducer thread (token m, 8 rows from f0), read before
-// the cluster barrier so that their latency overlaps the wait for the peers:
-// the shift term (QKV, gate/up) or the residual stream, gate and next norm
+// Epilogue inputs of one reducing thread (token m, 8 rows from f0), read
+// while the exchange is in flight: the residual stream, gate and next norm
 // scale (O, down).
 struct EpiIn {
-  float b[8];  // bias (QKV, gate/up) or gate (O, down)
-  float h[8];  // residual stream (O, down)
-  float sc[8]; // next norm's scale (O, down; unused without a next norm)
+  float b[8];  // gate
+  float h[8];  // residual stream
+  float sc[8]; // next norm's scale (unused without a next norm)
 };
 
 // Gated residual for 8 features f0.. of token m: h += gate * acc, then (when
@@ -708,199 +805,280 @@ __device__ void compute_rstd(const FC& c, const float* ss, int nslots) {
   csync();
 }
 
-// One projection stage on this CTA.  `it` counts projection items (TMEM
-// slots, partial buffers), `sg` the operand loads compute thread 0 issued,
-// `ncl` cluster barriers.  The outputs of all items are published together at
-// the end of the stage (one fence): a consumer's own reduction needs every
-// rank of its cluster, and so in effect the last item of each producer stage.
-// Returns false once the launch is aborting.
-__device__ bool gemm_stage(const FC& c, int st, int k, int l, int u, int& it, int& sg, int& ncl) {
+// Compute thread 0: the token operand [64 tokens][kb * 64] from column x0,
+// in up to 4 groups (8 KB per block).  `opn` counts each group's uses.
+__device__ void issue_operand(const FC& c, int st, int x0, int kb, int* opn) {
+  fence_proxy_async_global_f();  // written by other CTAs' generic stores, read by TMA
+  fence_proxy_async_smem();      // this CTA's generic stores to the area come first
+  const int gsz = op_gsz(kb);
+  for (int gi = 0; gi * gsz < kb; ++gi) {
+    const int b0 = gi * gsz, b1 = min(kb, b0 + gsz);
+    mbar_arrive_expect_tx(&c.op_full[gi], (uint32_t)(b1 - b0) * 8192u);
+    for (int i = b0; i < b1; ++i)
+      tma_load_2d(c.work + kFOp + (size_t)i * 8192, c.mp.x[st], x0 + i * 64, 0, &c.op_full[gi]);
+    ++opn[gi];
+  }
+}
+
+// QKV or gate/up on this CTA: its whole-K units.  The operand is the full
+// width, so every producer of it must be done; rstd comes from all their
+// sums of squares.  Each unit's accumulator goes through shared memory
+// ([64 tokens][128 rows] fp32, in the operand area once the MMAs are done)
+// so that a thread's epilogue covers 8 consecutive features of one token.
+// `sw` counts this CTA's whole-K stages (the acc_all phase).
+__device__ bool whole_stage(const FC& c, int st, int k, int l, int u, int& sw, int* opn) {
   const Shape& s = *c.s;
   const FlowArgs& a = *c.a;
   const StageG g = stage_geo(s, a, st);
-  const int nt = cl_tiles(a, g.ntiles, c.cl);
-  if (nt == 0) return true;  // uniform over the cluster
-  const int C = a.C, R = 128 / C, rank = c.rank;
-  const int x0 = rank * g.kbr * 64, x1 = x0 + g.kbr * 64;
-  const unsigned uC = (unsigned)C;
+  int first;
+  const int nu = owned(c, st, g, first);
+  if (nu == 0) return true;
+  const unsigned uC = (unsigned)a.C;
   const bool tr = k == a.k_begin && l == 1;
   const int tb = st * 10;
   (void)tr;
   (void)tb;
   FTRACE(c, tr, tb + 0);
 
-  // 1. the producers of this rank's K slice of the token operand, then its TMA
+  // 1. every producer of the operand, then its TMA
   bool ok = true;
   if (c.ct == 0) {
     if (st == ST_Q && l == 0) {
       ok = wait_ctr(c, c_tr(a), (unsigned)(a.M * (k - a.k_begin + 1)));
+    } else if (st == ST_Q) {
+      for (int t = 0; ok && t < a.d_tiles; ++t) ok = wait_ctr(c, c_y(a, t), uC * (unsigned)u);
     } else {
-      for (int t = x0 / 128; ok && t <= (x1 - 1) / 128; ++t) {
-        if (st == ST_Q) ok = wait_ctr(c, c_y(a, t), uC * (unsigned)u);
-        else if (st == ST_G) ok = wait_ctr(c, c_ho(a, t), uC * (unsigned)(u + 1));
-        else if (st == ST_D) ok = wait_ctr(c, c_u(a, t), uC * (unsigned)(u + 1));
-      }
-      if (st == ST_O) ok = wait_ctr(c, c_att(a), (unsigned)a.a_units * uC * (unsigned)(u + 1));
+      for (int t = 0; ok && t < a.o_tiles; ++t) ok = wait_ctr(c, c_ho(a, t), uC * (unsigned)(u + 1));
     }
-    if (ok) {
-      fence_proxy_async_global_f();  // written by other CTAs' generic stores, read by TMA
-      mbar_arrive_expect_tx(c.op_full, (uint32_t)g.kbr * 8192u);
-      for (int i = 0; i < g.kbr; ++i)
-        tma_load_2d(c.work + kFOp + (size_t)i * 8192, c.mp.x[st], x0 + i * 64, 0, c.op_full);
-      ++sg;  // operand loads issued (drained before exit)
-    }
+    if (ok) issue_operand(c, st, 0, g.kb, opn);
   }
   FTRACE(c, tr, tb + 1);
   if (!cand(ok)) return false;
 
-  // 2. QKV and gate/up: rstd per token from the producers' sums of squares
-  //    (all of them: the norm spans every feature), while the MMAs run
-  if (st == ST_Q || st == ST_G) {
-    if (c.ct == 0) {
-      if (st == ST_Q && l > 0)
-        for (int t = 0; ok && t < a.d_tiles; ++t) ok = wait_ctr(c, c_y(a, t), uC * (unsigned)u);
-      if (st == ST_G)
-        for (int t = 0; ok && t < a.o_tiles; ++t) ok = wait_ctr(c, c_ho(a, t), uC * (unsigned)(u + 1));
-    }
-    if (!cand(ok)) return false;
-    if (st == ST_G) compute_rstd(c, a.ss_g, a.o_tiles * C);
-    else if (l > 0) compute_rstd(c, a.ss_q, a.d_tiles * C);
-    else compute_rstd(c, a.ss_t, 1);
-  }
+  // 2. rstd per token from the producers' sums of squares, while the MMAs run
+  if (st == ST_G) compute_rstd(c, a.ss_g, a.o_tiles * a.C);
+  else if (l > 0) compute_rstd(c, a.ss_q, a.d_tiles * a.C);
+  else compute_rstd(c, a.ss_t, 1);
+  FTRACE(c, tr, tb + 2);
 
-  // 3. items: accumulator -> own partial tile -> cluster barrier -> reduce
-  //    this rank's rows over the C partials -> epilogue
+  // 3. every unit accumulated: the operand area is free from here on
+  if (!cand(fwait(c, c.acc_all, (uint32_t)sw & 1u))) return false;
+  ++sw;
+  tc_fence_after();
+  FTRACE(c, tr, tb + 3);
+
+  // 4. per unit: accumulator -> tile -> epilogue
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qd = warp & 3, row = qd * 32 + lane;  // TMEM lane = weight row
+  const uint32_t tile = smem_u32(c.work);
+  const int Mc = (a.M + 15) & ~15;  // accumulator columns read, 16 at a time
+  const float* tb_row = st == ST_Q ? a.bias_qkv + ((size_t)k * s.L + l) * s.qkv_rows
+                                   : a.bias_gu + ((size_t)k * s.L + l) * 2 * s.F;
+  for (int j = 0; j < nu; ++j) {
+    const int t = first + j * c.ncta;
+    if (j > 0) csync();  // the previous unit's epilogue has read the tile
+    const uint32_t taddr = c.tmem + ((uint32_t)(qd * 32) << 16) + 64u * (uint32_t)j;
+    for (int c0 = 0; c0 < Mc; c0 += 16) {
+      float v[16];
+      tmem_ld16(taddr + (uint32_t)c0, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) st_shared_f32(tile + (uint32_t)(((c0 + jj) * 128 + row) * 4), v[jj]);
+    }
+    tc_fence_before();
+    csync();
+    if (st == ST_Q) {
+      for (int idx = c.ct; idx < a.M * 16; idx += kFCompute) {
+        const int m = idx >> 4, r0 = (idx & 15) * 8;
+        float acc[8], bv[8];
+        const uint32_t ta = tile + (uint32_t)((m * 128 + r0) * 4);
+        f4_to(acc, ld_shared_f4(ta), ld_shared_f4(ta + 16));
+        const int f0 = 128 * t + r0;
+        f4_to(bv, ldg_f4(tb_row + f0), ldg_f4(tb_row + f0 + 4));
+        epi_q(c, k, l, m, f0, acc, bv);
+      }
+    } else {
+      int g0, g1;
+      unit_rows(s, ST_G, g, 0, t, g0, g1);  // gate and up rows within a layer
+      for (int idx = c.ct; idx < a.M * 8; idx += kFCompute) {
+        const int m = idx >> 3, r0 = (idx & 7) * 8;
+        float gv[8], uv[8], bg[8], bu[8], ov[8];
+        const uint32_t ta = tile + (uint32_t)((m * 128 + r0) * 4);
+        f4_to(gv, ld_shared_f4(ta), ld_shared_f4(ta + 16));
+        f4_to(uv, ld_shared_f4(ta + 256), ld_shared_f4(ta + 272));
+        f4_to(bg, ldg_f4(tb_row + g0 + r0), ldg_f4(tb_row + g0 + r0 + 4));
+        f4_to(bu, ldg_f4(tb_row + g1 + r0), ldg_f4(tb_row + g1 + r0 + 4));
+        const float rs = c.s_rstd[m];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ov[i] = gelu_tanh_bf16out(fmaf(rs, gv[i], bg[i])) * fmaf(rs, uv[i], bu[i]);
+        *reinterpret_cast<uint4*>(a.u + (size_t)m * s.F + 64 * t + r0) = pack8(ov);
+      }
+    }
+  }
+  FTRACE(c, tr, tb + 4);
+
+  // 5. publish every unit (one fence)
+  __threadfence();
+  csync();
+  if (c.ct == 0) {
+    if (st == ST_Q) {
+      red_release_u32(c_qkv(a), (unsigned)nu);
+    } else {
+      for (int j = 0; j < nu; ++j) red_release_u32(c_u(a, first + j * c.ncta), 1u);
+    }
+  }
+  FTRACE(c, tr, tb + 5);
+  return true;
+}
+
+// O or down on this CTA's cluster: its tiles, K split over the ranks.  Per
+// tile, rank p's partial row r goes to rank r / R (R = 128 / C rows each),
+// which adds the C slices in rank order and applies the gated residual, the
+// next norm's operand and its sums of squares.  `it` counts split-K items
+// (TMEM slot), `xn` exchanges; `xopen` marks an exchange armed and not yet
+// complete (drained at exit after an abort).
+__device__ bool split_stage(const FC& c, int st, int k, int l, int u, int& it, int& xn, bool& xopen, int* opn) {
+  const Shape& s = *c.s;
+  const FlowArgs& a = *c.a;
+  const StageG g = stage_geo(s, a, st);
+  int first;
+  const int nt = owned(c, st, g, first);
+  if (nt == 0) return true;  // uniform over the cluster
+  const int C = a.C, R = 128 / C, rank = c.rank;
+  const int x0 = rank * g.kb * 64, x1 = x0 + g.kb * 64;
+  const bool tr = k == a.k_begin && l == 1;
+  const int tb = st * 10;
+  (void)tr;
+  (void)tb;
+  FTRACE(c, tr, tb + 0);
+
+  // 1. the producers of this rank's K slice of the operand, then its TMA
+  bool ok = true;
+  if (c.ct == 0) {
+    if (st == ST_O) {
+      ok = wait_ctr(c, c_att(a), (unsigned)a.a_units * (unsigned)C * (unsigned)(u + 1));
+    } else {
+      for (int j = x0 / 64; ok && j <= (x1 - 1) / 64; ++j) ok = wait_ctr(c, c_u(a, j), (unsigned)(u + 1));
+    }
+    if (ok) issue_operand(c, st, x0, g.kb, opn);
+  }
+  FTRACE(c, tr, tb + 1);
+  if (!cand(ok)) return false;
+
   const float* tab = a.tables + (size_t)k * s.table_rows;
   const bool has_next = st == ST_O || (st == ST_D && l + 1 < s.L);
   const float* gate = tab + mod_offset(s, l, st == ST_O ? 0 : 1, 2);
   const float* scn = !has_next ? nullptr : (st == ST_O ? tab + mod_offset(s, l, 1, 0) : tab + mod_offset(s, l + 1, 0, 0));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qd = warp & 3, row = qd * 32 + lane;  // TMEM lane = weight row
+  const int Mp = (a.M + 3) & ~3;                   // tokens exchanged per row
+  const uint32_t rx = smem_u32(c.work) + kFRx;     // [C][R][Mp] fp32
+  const float* rxf = reinterpret_cast<const float*>(c.work + kFRx);
+  const uint32_t xbytes = (uint32_t)((C - 1) * R * Mp * 4);
   const int per8 = R / 8, nitems = a.M * per8;
-  const int npass = (nitems + 127) / 128;  // at most 4 (64 tokens x 8 row groups with C = 2)
-  float keep[4][8];
+  const int npass = (nitems + kFCompute - 1) / kFCompute;
+  // this thread's partial row goes to its owner's slice of rank `rank`
+  const int owner = row / R, orow = row - owner * R;
+  const bool local = owner == rank;
+  const uint32_t dl = rx + (uint32_t)((rank * R + orow) * Mp * 4);
+  const uint32_t dst = local ? dl : map_cluster(dl, (uint32_t)owner);
+  const uint32_t dbar = map_cluster(smem_u32(c.rx), (uint32_t)owner);
   for (int j = 0; j < nt; ++j) {
-    const int t = c.cl + j * a.NC;
-    for (int half = 0; half < g.na; ++half, ++it) {
-      const int slot = it & 1;
-      if (!cand(fwait(c, &c.acc_full[slot], (it >> 1) & 1))) return false;
-      if (j == 0 && half == 0) FTRACE(c, tr, tb + 2);
-      tc_fence_after();
-      const uint32_t taddr = c.tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)slot * 64u;
-      const uint32_t pbase = smem_u32(c.work + kFPart) + (uint32_t)(it & 1) * 32768u;
-      for (int c0 = 0; c0 < a.M; c0 += 16) {
-        float v[16];
-        tmem_ld16(taddr + (uint32_t)c0, v);
-        tmem_ld_wait();
+    const int t = first + j * a.NC;
+    // a. the receive area is free: previous exchange reduced, operand below it
+    xchg_open(c, xbytes);
+    xopen = true;
+    const int slot = it & 1;
+    if (!cand(fwait(c, &c.acc_full[slot], (uint32_t)(it >> 1) & 1u))) return false;
+    ++it;
+    tc_fence_after();
+    if (j == 0) FTRACE(c, tr, tb + 2);
+    // b. epilogue inputs of the first pass, in flight during the exchange
+    EpiIn in;
+    auto load_in = [&](int pass) {
+      const int idx = c.ct + pass * kFCompute;
+      if (idx >= nitems) return;
+      const int m = idx / per8, f0 = 128 * t + rank * R + (idx - m * per8) * 8;
+      const float* hp = a.h + (size_t)m * s.D + f0;
+      f4_to(in.h, ldcg_f4(hp), ldcg_f4(hp + 4));
+      f4_to(in.b, ldg_f4(gate + f0), ldg_f4(gate + f0 + 4));
+      if (has_next) f4_to(in.sc, ldg_f4(scn + f0), ldg_f4(scn + f0 + 4));
+    };
+    load_in(0);
+    // c. every peer's receive area is free: partial rows to their owners
+    if (!xchg_ready(c, xn)) return false;
+    if (j == 0) FTRACE(c, tr, tb + 3);
+    const uint32_t taddr = c.tmem + ((uint32_t)(qd * 32) << 16) + 64u * (uint32_t)slot;
+    for (int c0 = 0; c0 < Mp; c0 += 16) {
+      float v[16];
+      tmem_ld16(taddr + (uint32_t)c0, v);
+      tmem_ld_wait();
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) st_shared_f32(pbase + (uint32_t)(((c0 + jj) * 128 + row) * 4), v[jj]);
-      }
-      tc_fence_before();
-      csync();
-      if (c.ct == 0) mbar_arrive(&c.acc_empty[slot]);
-      // epilogue inputs of this thread's (token, 8 rows) item: the first pass's
-      // are read before the barrier, the second's (small batches with 32 rows
-      // per rank) at the start of that pass
-      EpiIn in;
-      auto load_in = [&](int pass) {
-        const int idx = c.ct + pass * 128;
-        if (idx >= nitems) return;
-        const int m = idx / per8, r0 = rank * R + (idx - m * per8) * 8;
-        const int f0 = 128 * t + r0;
-        if (st == ST_Q || st == ST_G) {
-          const float* bias = st == ST_Q ? a.bias_qkv + ((size_t)k * s.L + l) * s.qkv_rows + f0
-                                         : a.bias_gu + ((size_t)k * s.L + l) * 2 * s.F + 256 * t + 128 * half + r0;
-          f4_to(in.b, ldg_f4(bias), ldg_f4(bias + 4));
-        } else {
-          const float* hp = a.h + (size_t)m * s.D + f0;
-          f4_to(in.h, ldcg_f4(hp), ldcg_f4(hp + 4));
-          f4_to(in.b, ldg_f4(gate + f0), ldg_f4(gate + f0 + 4));
-          if (has_next) f4_to(in.sc, ldg_f4(scn + f0), ldg_f4(scn + f0 + 4));
-        }
-      };
-      load_in(0);
-      if (j == 0 && half == 0) FTRACE(c, tr, tb + 3);
-      if (!cl_sync(c, ncl)) return false;
-      if (j == 0 && half == 0) FTRACE(c, tr, tb + 4);
-#pragma unroll 1
-      for (int pass = 0; pass < npass; ++pass) {  // uniform
-        if (pass > 0) load_in(pass);
-        const int idx = c.ct + pass * 128;
-        const bool valid = idx < nitems;
-        const int m = valid ? idx / per8 : 0, j8 = valid ? idx - (idx / per8) * per8 : 0;
-        const int r0 = rank * R + j8 * 8;
-        float acc[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-        if (valid) {
-          // up to 8 ranks' loads in flight at once (distributed shared memory
-          // has a long latency), then added in rank order
-          const uint32_t la = pbase + (uint32_t)((m * 128 + r0) * 4);
-          for (int q0 = 0; q0 < C; q0 += 8) {
-            float4 p[8][2];
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              if (q0 + q < C) {
-                const uint32_t ra = map_cluster(la, (uint32_t)(q0 + q));
-                p[q][0] = ld_cluster_f32x4(ra);
-                p[q][1] = ld_cluster_f32x4(ra + 16);
-              }
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              if (q0 + q < C) {
-                acc[0] += p[q][0].x; acc[1] += p[q][0].y; acc[2] += p[q][0].z; acc[3] += p[q][0].w;
-                acc[4] += p[q][1].x; acc[5] += p[q][1].y; acc[6] += p[q][1].z; acc[7] += p[q][1].w;
-              }
-          }
-        }
-        const int f0 = 128 * t + r0;
-        if (st == ST_Q) {
-          if (valid) epi_q(c, k, l, m, f0, acc, in.b);
-        } else if (st == ST_G) {
-          if (valid) {
-            const float rs = c.s_rstd[m];
-            if (half == 0) {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) keep[pass][i] = fmaf(rs, acc[i], in.b[i]);
-            } else {
-              float ov[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) ov[i] = gelu_tanh_bf16out(keep[pass][i]) * fmaf(rs, acc[i], in.b[i]);
-              *reinterpret_cast<uint4*>(a.u + (size_t)m * s.F + f0) = pack8(ov);
-            }
-          }
-        } else {
-          float sq = 0.f;
-          if (valid) sq = epi_resid(c, m, f0, acc, in, has_next, st == ST_O ? a.yg : a.yq);
-          // the per8 threads of one token are adjacent lanes: fixed shuffle tree
-          for (int o = 1; o < per8; o <<= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-          if (valid && j8 == 0 && has_next) (st == ST_O ? a.ss_g : a.ss_q)[(size_t)(t * C + rank) * 64 + m] = sq;
+      for (int e = 0; e < 4; ++e) {
+        const int col = c0 + 4 * e;
+        if (col < Mp) {
+          const float4 f = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+          if (local) st_shared_f4(dst + (uint32_t)col * 4u, f);
+          else st_async_f4(dst + (uint32_t)col * 4u, f, dbar);
         }
       }
     }
+    tc_fence_before();
+    csync();
+    if (c.ct == 0) mbar_arrive(&c.acc_empty[slot]);
+    if (j == 0) FTRACE(c, tr, tb + 4);
+    // d. every peer's slice landed
+    if (!xchg_wait(c, xn)) return false;
+    ++xn;
+    xopen = false;
+    if (j == 0) FTRACE(c, tr, tb + 5);
+    // e. sum the C slices in rank order, then the epilogue of 8 rows
+#pragma unroll 1
+    for (int pass = 0; pass < npass; ++pass) {  // uniform
+      if (pass > 0) load_in(pass);
+      const int idx = c.ct + pass * kFCompute;
+      const bool valid = idx < nitems;
+      const int m = valid ? idx / per8 : 0, j8 = valid ? idx - (idx / per8) * per8 : 0;
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      if (valid) {
+        const float* p = rxf + (size_t)(j8 * 8) * Mp + m;
+        for (int q = 0; q < C; ++q) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] += p[(size_t)(q * R + i) * Mp];
+        }
+      }
+      const int f0 = 128 * t + rank * R + j8 * 8;
+      float sq = 0.f;
+      if (valid) sq = epi_resid(c, m, f0, acc, in, has_next, st == ST_O ? a.yg : a.yq);
+      // the per8 threads of one token are adjacent lanes: fixed shuffle tree
+      for (int o = 1; o < per8; o <<= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      if (valid && j8 == 0 && has_next) (st == ST_O ? a.ss_g : a.ss_q)[(size_t)(t * C + rank) * 64 + m] = sq;
+    }
+    csync();  // the receive area has been read
   }
-  // 4. publish every item of the stage (one fence)
-  FTRACE(c, tr, tb + 5);
+  // publish every tile of the stage (one fence)
   __threadfence();
   csync();
-  FTRACE(c, tr, tb + 6);
   if (c.ct == 0) {
     for (int j = 0; j < nt; ++j) {
-      const int t = c.cl + j * a.NC;
-      red_release_u32(st == ST_Q ? c_qkv(a) : st == ST_O ? c_ho(a, t) : st == ST_G ? c_u(a, t) : c_y(a, t), 1u);
+      const int t = first + j * a.NC;
+      red_release_u32(st == ST_O ? c_ho(a, t) : c_y(a, t), 1u);
     }
   }
+  FTRACE(c, tr, tb + 6);
   return true;
 }
 
 // Attention on the clusters that hold an attention unit: rank r takes keys
 // [r kps, r kps + kps) of the slot in 64-key chunks (online softmax in the
-// log2 domain, thread = query row = TMEM lane), then the C partial outputs are
-// merged in the cluster: rank weights exp2(m_r - M) / L from every rank's row
-// max and sum, each rank parks its weighted rows (fp32, 16-byte chunks
-// swizzled by row), and rank q adds rows [q R, q R + R) of all ranks in rank
-// order.  `ac` counts this CTA's chunks (barrier phases).
-__device__ bool att_stage(const FC& c, int l, int u, int& ac, int& ncl, int& kv_issued) {
+// log2 domain, thread = query row = TMEM lane).  Then every rank stores its
+// unnormalised output rows with their running (max, sum) into the rows'
+// owner (rank row / R), which weights rank p's rows by exp2(m_p - M) / L
+// (M, L over all ranks) and adds them in rank order.  `ac` counts this CTA's
+// chunks (barrier phases).
+__device__ bool att_stage(const FC& c, int l, int u, int& ac, int& xn, bool& xopen, int& kv_issued) {
   const Shape& s = *c.s;
   const FlowArgs& a = *c.a;
   const AttU au = att_unit(s, a, c.cl, c.rank);
@@ -910,14 +1088,13 @@ __device__ bool att_stage(const FC& c, int l, int u, int& ac, int& ncl, int& kv_
   const bool tr = u == 1;
   (void)tr;
   FTRACE(c, tr, 40);
-  // peers are done reading this CTA's partial tiles of the QKV stage
-  if (!cl_sync(c, ncl)) return false;
   const int slot_row0 = ((l * s.Bmax + au.b) * s.Hkv + au.g) * s.Ptot;
   bool ok = true;
   if (c.ct == 0) {
-    ok = wait_ctr(c, c_qkv(a), (unsigned)(a.q_tiles * C * (u + 1)));
+    ok = wait_ctr(c, c_qkv(a), (unsigned)(a.q_units * (u + 1)));
     if (ok && au.nch > 0) {
       fence_proxy_async_global_f();
+      fence_proxy_async_smem();
       mbar_arrive_expect_tx(c.kv_full, qbytes + 2u * kvbytes);
       const int qrow0 = au.bg * GH + au.qt * 128;
       for (int x = 0; x < nbox; ++x) tma_load_2d(c.work + (size_t)x * 128 * 128, c.mp.q, x * 64, qrow0, c.kv_full);
@@ -1015,80 +1192,96 @@ __device__ bool att_stage(const FC& c, int l, int u, int& ac, int& ncl, int& kv_
   }
   ac += au.nch;
   if (au.nch > 0 && !cand(fwait(c, c.o_full, (ac - 1) & 1))) return false;
-  FTRACE(c, tr, 43);
   tc_fence_after();
+  FTRACE(c, tr, 43);
 
   // -------------------------------------------------- merge in the cluster
-  c.s_ml[2 * r] = au.nch > 0 ? m_run : -INFINITY;
-  c.s_ml[2 * r + 1] = au.nch > 0 ? l_run : 0.f;
-  if (!cl_sync(c, ncl)) return false;
-  // every rank's (max, sum) of this row, all loads in flight at once
-  float mq[16], lq[16];
-  const uint32_t mla = smem_u32(c.s_ml + 2 * r);
-#pragma unroll
-  for (int q = 0; q < 16; ++q)
-    if (q < C) {
-      const uint32_t ra = map_cluster(mla, (uint32_t)q);
-      mq[q] = ld_cluster_f32(ra);
-      lq[q] = ld_cluster_f32(ra + 4);
-    }
-  float Mx = -INFINITY;
-#pragma unroll
-  for (int q = 0; q < 16; ++q)
-    if (q < C) Mx = fmaxf(Mx, mq[q]);
-  float Ls = 0.f;
-#pragma unroll
-  for (int q = 0; q < 16; ++q)
-    if (q < C && lq[q] > 0.f) Ls = fmaf(exp2f(mq[q] - Mx), lq[q], Ls);
-  const float w = (au.nch > 0 && l_run > 0.f && Ls > 0.f) ? exp2f(m_run - Mx) / Ls : 0.f;
-  const uint32_t prow = smem_u32(c.work) + (uint32_t)(r * d * 4);
-  for (int j = 0; j < d; j += 16) {
-    float ov[16];
-    if (au.nch > 0) {  // uniform over the CTA
-      tmem_ld16(c.tmem + lane_off + kColO + j, ov);
-      tmem_ld_wait();
+  // the work area (q, K, V) is free once every thread is past its last use
+  csync();
+  const int R = 128 / C, owner = r / R, orow = r - owner * R;
+  xchg_open(c, (uint32_t)((C - 1) * R * (d * 4 + 8)));
+  xopen = true;
+  if (!xchg_ready(c, xn)) return false;
+  FTRACE(c, tr, 44);
+  {
+    const bool local = owner == c.rank;
+    const uint32_t ra = smem_u32(c.work) + (uint32_t)((c.rank * R + orow) * d * 4);
+    const uint32_t sa = smem_u32(c.s_st) + (uint32_t)((c.rank * R + orow) * 8);
+    const uint32_t dbar = map_cluster(smem_u32(c.rx), (uint32_t)owner);
+    const uint32_t dr = local ? ra : map_cluster(ra, (uint32_t)owner);
+    const uint32_t ds = local ? sa : map_cluster(sa, (uint32_t)owner);
+    const float mv = au.nch > 0 ? m_run : -INFINITY, lv = au.nch > 0 ? l_run : 0.f;
+    if (local) {
+      st_shared_f32(ds, mv);
+      st_shared_f32(ds + 4, lv);
     } else {
-#pragma unroll
-      for (int t = 0; t < 16; ++t) ov[t] = 0.f;
+      st_async_f2(ds, mv, lv, dbar);
     }
+    for (int j = 0; j < d; j += 16) {
+      float ov[16];
+      if (au.nch > 0) {  // uniform over the CTA
+        tmem_ld16(c.tmem + lane_off + kColO + j, ov);
+        tmem_ld_wait();
+      } else {
 #pragma unroll
-    for (int t4 = 0; t4 < 4; ++t4) {
-      const uint32_t ch4 = ((uint32_t)(j / 4 + t4)) ^ (uint32_t)(r & 7);
-      st_shared_f4(prow + ch4 * 16u, make_float4(ov[4 * t4] * w, ov[4 * t4 + 1] * w, ov[4 * t4 + 2] * w,
-                                                 ov[4 * t4 + 3] * w));
+        for (int t = 0; t < 16; ++t) ov[t] = 0.f;
+      }
+#pragma unroll
+      for (int t4 = 0; t4 < 4; ++t4) {
+        const float4 f = make_float4(ov[4 * t4], ov[4 * t4 + 1], ov[4 * t4 + 2], ov[4 * t4 + 3]);
+        const uint32_t o = (uint32_t)((j + 4 * t4) * 4);
+        if (local) st_shared_f4(dr + o, f);
+        else st_async_f4(dr + o, f, dbar);
+      }
     }
   }
   tc_fence_before();
-  FTRACE(c, tr, 44);
-  if (!cl_sync(c, ncl)) return false;
+  if (!xchg_wait(c, xn)) return false;
+  ++xn;
+  xopen = false;
   FTRACE(c, tr, 45);
-  const int R = 128 / C, per_row = d / 4;
+  // weight of rank q's slice of row rr: exp2(m_q - M) / L, in s_tmp[rr][q] (R C = 128 floats)
+  if (c.ct < R) {
+    float mq[16], lq[16];
+    float Mx = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+      if (q < C) {
+        mq[q] = c.s_st[(q * R + c.ct) * 2];
+        lq[q] = c.s_st[(q * R + c.ct) * 2 + 1];
+        Mx = fmaxf(Mx, mq[q]);
+      }
+    float Ls = 0.f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+      if (q < C && lq[q] > 0.f) Ls = fmaf(exp2f(mq[q] - Mx), lq[q], Ls);
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+      if (q < C) c.s_tmp[c.ct * C + q] = (lq[q] > 0.f && Ls > 0.f) ? exp2f(mq[q] - Mx) / Ls : 0.f;
+  }
+  csync();
+  const int per_row = d / 4;
   for (int el = c.ct; el < R * per_row; el += kFCompute) {
     const int rr = el / per_row, c4 = el - rr * per_row;
-    const int row = c.rank * R + rr, rq = au.qt * 128 + row;
+    const int rq = au.qt * 128 + c.rank * R + rr;
     if (rq >= GH) continue;
-    const uint32_t la = smem_u32(c.work) + (uint32_t)(row * d * 4) + (((uint32_t)c4 ^ (uint32_t)(row & 7)) * 16u);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int q0 = 0; q0 < C; q0 += 8) {
-      float4 v[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        if (q0 + q < C) v[q] = ld_cluster_f32x4(map_cluster(la, (uint32_t)(q0 + q)));
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        if (q0 + q < C) {
-          acc.x += v[q].x; acc.y += v[q].y; acc.z += v[q].z; acc.w += v[q].w;
-        }
+    for (int q = 0; q < C; ++q) {
+      const float w = c.s_tmp[rr * C + q];
+      const float4 v = ld_shared_f4(smem_u32(c.work) + (uint32_t)(((q * R + rr) * d + 4 * c4) * 4));
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
     }
     const int hl = rq / s.H, ti = rq - hl * s.H;
     bf16* orow = a.o + (size_t)(au.b * s.H + ti) * s.attn_dim + (au.g * s.G + hl) * d;
     *reinterpret_cast<uint2*>(orow + 4 * c4) = make_uint2(pack_bf2(acc.x, acc.y), pack_bf2(acc.z, acc.w));
   }
   FTRACE(c, tr, 46);
-  publish(c, c_att(a));
+  publish(c, c_att(a));  // its barrier also ends every thread's reads of the area
   FTRACE(c, tr, 47);
-  // peers are done reading this CTA's partial before the work area is reused
-  return cl_sync(c, ncl);
+  return true;
 }
 
 // Token transition for token m = this CTA: (end of step k_out) final
@@ -1202,21 +1395,26 @@ __device__ bool transition(const FC& c, int k_out, int k_in) {
 __device__ void compute_loop(const FC& c) {
   const Shape& s = *c.s;
   const FlowArgs& a = *c.a;
-  int it = 0, sg = 0, ac = 0, ncl = 0, kv_issued = 0;
+  int it = 0, sw = 0, ac = 0, xn = 0, kv_issued = 0;
+  int opn[4] = {0, 0, 0, 0};
+  bool xopen = false;
   bool ok = transition(c, -1, a.k_begin);
   for (int k = a.k_begin; ok && k < a.k_end; ++k) {
     for (int l = 0; ok && l < s.L; ++l) {
       const int u = (k - a.k_begin) * s.L + l;
-      ok = gemm_stage(c, ST_Q, k, l, u, it, sg, ncl) && att_stage(c, l, u, ac, ncl, kv_issued) &&
-           gemm_stage(c, ST_O, k, l, u, it, sg, ncl) && gemm_stage(c, ST_G, k, l, u, it, sg, ncl) &&
-           gemm_stage(c, ST_D, k, l, u, it, sg, ncl);
+      ok = whole_stage(c, ST_Q, k, l, u, sw, opn) && att_stage(c, l, u, ac, xn, xopen, kv_issued) &&
+           split_stage(c, ST_O, k, l, u, it, xn, xopen, opn) && whole_stage(c, ST_G, k, l, u, sw, opn) &&
+           split_stage(c, ST_D, k, l, u, it, xn, xopen, opn);
     }
     if (ok) ok = transition(c, k, k + 1 < a.k_end ? k + 1 : -1);
   }
-  // after an abort, copies this CTA issued may still be in flight: let them land
+  // after an abort, copies this CTA issued may still be in flight, and peers
+  // may still be storing into an exchange it had opened: let them land
   if (c.ct == 0) {
-    if (sg > 0 && !mbar_wait(c.op_full, (sg - 1) & 1, kFDrain)) set_error(a.err, DEV_DRAIN);
+    for (int gi = 0; gi < 4; ++gi)
+      if (opn[gi] > 0 && !mbar_wait(&c.op_full[gi], (opn[gi] - 1) & 1, kFDrain)) set_error(a.err, DEV_DRAIN);
     if (kv_issued > 0 && !mbar_wait(c.kv_full, (kv_issued - 1) & 1, kFDrain)) set_error(a.err, DEV_DRAIN);
+    if (xopen && a.C > 1) (void)mbar_wait(c.rx, (uint32_t)xn & 1u, kFExitWait);
   }
 }
 
@@ -1248,19 +1446,22 @@ __global__ void __launch_bounds__(kFThreads, 1)
   c.mp.v = &tmV;
   c.ring = smem;
   c.work = smem + kFRing * kFBlk;
-  c.rfull = bar;
-  c.rempty = bar + kFRing;
-  c.op_full = bar + 2 * kFRing;
-  c.acc_full = bar + 2 * kFRing + 1;   // [2]
-  c.acc_empty = bar + 2 * kFRing + 3;  // [2]
-  c.kv_full = bar + 2 * kFRing + 5;
-  c.s_full = bar + 2 * kFRing + 6;
-  c.p_full = bar + 2 * kFRing + 7;
-  c.o_full = bar + 2 * kFRing + 8;
-  c.cbar = bar + 2 * kFRing + 9;       // [2]
-  c.drain = bar + 2 * kFRing + 11;
-  c.raw_full = bar + 2 * kFRing + 12;  // [kFRawRing]
-  constexpr int kNBar = 2 * kFRing + 12 + kFRawRing;
+  // mbarriers
+  c.rfull = bar;                   // [kFRing]
+  c.rempty = bar + kFRing;         // [kFRing]
+  c.op_full = bar + 2 * kFRing;    // [4]
+  c.acc_full = c.op_full + 4;      // [2]
+  c.acc_empty = c.acc_full + 2;    // [2]
+  c.acc_all = c.acc_empty + 2;
+  c.kv_full = c.acc_all + 1;
+  c.s_full = c.kv_full + 1;
+  c.p_full = c.s_full + 1;
+  c.o_full = c.p_full + 1;
+  c.rx = c.o_full + 1;
+  c.rdy = c.rx + 1;
+  c.drain = c.rdy + 1;
+  c.raw_full = c.drain + 1;        // [kFRawRing]
+  const int nbar = (int)(c.raw_full + kFRawRing - bar);
   c.nring = a.w4 ? kFRing - 1 : kFRing;
   c.raw = smem + (kFRing - 1) * kFBlk;  // int4 mode: the fifth bf16 slot holds the packed ring
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 256);
@@ -1268,15 +1469,16 @@ __global__ void __launch_bounds__(kFThreads, 1)
   c.s_flag = reinterpret_cast<volatile int*>(misc + 264);
   c.s_rstd = reinterpret_cast<float*>(misc + 512);   // [64]
   c.s_tmp = reinterpret_cast<float*>(misc + 768);    // [512]
-  c.s_ml = reinterpret_cast<float*>(misc + 2816);    // [128][2]
+  c.s_st = reinterpret_cast<float*>(misc + 2816);    // [C][R][2] = 1 KB
   c.cta = blockIdx.x;
+  c.ncta = gridDim.x;
   c.rank = (int)cluster_rank();
   c.cl = blockIdx.x / a.C;
   c.ct = (int)threadIdx.x - 64;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNBar; ++i) mbar_init(&bar[i], (i == 2 * kFRing + 9 || i == 2 * kFRing + 10) ? a.C : 1);
+    for (int i = 0; i < nbar; ++i) mbar_init(&bar[i], (&bar[i] == c.rdy && a.C > 1) ? (uint32_t)(a.C - 1) : 1u);
     *c.s_abort = 0;
     *c.s_flag = 0;
     fence_mbar_init();
@@ -1296,7 +1498,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
   __syncthreads();
   tc_fence_after();
   c.tmem = *tmem_slot;
-  hw_cluster_sync();  // every rank's mbarriers exist before any remote arrive
+  hw_cluster_sync();  // every rank's mbarriers exist before any remote arrival or store
 
   if (warp == 0) {
     producer_warp(c);
@@ -1309,7 +1511,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  hw_cluster_sync();  // no CTA leaves while a peer may still read its shared memory
+  hw_cluster_sync();  // no CTA leaves while a peer may still write its shared memory
   if (warp == 0) tmem_dealloc(c.tmem, kFTmem);
 }
 

@@ -159,6 +159,7 @@ struct pae_ctx {
   float *bias_qkv = nullptr, *bias_gu = nullptr;
   unsigned* f_ctr = nullptr;
   CUtensorMap tmYq64{}, tmYg64{}, tmO64{}, tmU64{};
+  CUtensorMap tmWg64{};  // gate/up with 64-row boxes (dataflow loop)
   // in-kernel adaRMSNorm: per-token sum-of-squares slots [kSsSlots][ss_ld]
   bool use_fused_norm = false;  // opt-in: measured slower than the norm kernels under PDL
   float* ss_buf = nullptr;
@@ -168,7 +169,7 @@ struct pae_ctx {
   void *q_qkv = nullptr, *q_o = nullptr, *q_gu = nullptr, *q_down = nullptr;
   void *sc_qkv = nullptr, *sc_o = nullptr, *sc_gu = nullptr, *sc_down = nullptr;
   CUtensorMap tmQqkv{}, tmQo{}, tmQgu{}, tmQdown{};
-  CUtensorMap tmQgu1{};  // packed gate/up with 128-row boxes (dataflow loop)
+  CUtensorMap tmQg64{};  // packed gate/up with 64-row boxes (dataflow loop)
   // tables
   double* t_dev = nullptr;
   float *emb = nullptr, *zbuf = nullptr, *cbuf = nullptr, *tables = nullptr, *dt = nullptr;
@@ -491,32 +492,41 @@ bool plan_persistent(const pae_ctx* ctx, int B, PersistArgs* pa) {
   return true;
 }
 
-// Dataflow-loop plan for M = B*H <= 64 tokens (bf16 weights): the cluster
-// size C must split every projection's K range into whole 64-wide blocks per
-// rank with the token operand slice within 64 KB; the grid is as many
-// clusters of C as fit at once (one CTA per SM), which must cover the
-// attention units (request, KV head, 128 query rows) and the M token CTAs of
-// the transition.  Among the sizes that fit, the one with the most CTAs (ties:
-// the larger C).  Returns false when the batch or shape is not eligible.
+// Dataflow-loop plan for M = B*H <= 64 tokens.  QKV and gate/up run as
+// 128-row whole-K units, one CTA each (the token operand, 64 x width bf16,
+// within the 128 KB work area: width <= 1024); at most 8 units per CTA (TMEM
+// columns).  O and down split K over the C ranks of a cluster with a
+// 64-wide block count per rank and the operand slice within 64 KB.  The grid
+// is as many clusters of C as fit at once (one CTA per SM), which must cover
+// the attention units (request, KV head, 128 query rows) and the M token CTAs
+// of the transition.  Preferred: every O and down tile on a cluster of its
+// own, then the larger C (fewer K blocks per rank).  Returns false when the
+// batch or shape is not eligible.
 bool plan_flow(const pae_ctx* ctx, int B, FlowArgs* fa) {
   const Shape& s = ctx->s;
   const int M = B * s.H;
   if (!ctx->flow_capable || M < 1 || M > 64) return false;
+  if (s.D % 128 || s.D > 1024 || s.qkv_rows % 128 || s.F % 128 || s.attn_dim % 64) return false;
   const int nkD = s.D / 64, nkA = s.attn_dim / 64, nkF = s.F / 64;
   const int qtiles = (s.G * s.H + 127) / 128;
   const int units = B * s.Hkv * qtiles;
-  if (3 + 2 * (s.D / 128) + s.F / 128 + 1 > kFlowCtrWords) return false;
+  const int q_units = s.qkv_rows / 128, g_units = s.F / 64, tiles = s.D / 128;
+  if (3 + 2 * tiles + g_units + 1 > kFlowCtrWords) return false;
   if (s.d > 256 || 128 * s.d * 2 + 2 * 64 * s.d * 2 > 128 * 1024) return false;
   int bestC = 0, bestNC = 0;
+  bool bestFit = false;
   for (int C : {16, 8, 4, 2}) {
     if (ctx->flow_cluster && C != ctx->flow_cluster) continue;
-    if (nkD % C || nkA % C || nkF % C) continue;
-    if ((nkF / C) * 8192 > 64 * 1024 || (nkA / C) * 8192 > 64 * 1024 || (nkD / C) * 8192 > 64 * 1024) continue;
-    const int NC = std::min(ctx->flow_max_cl[C], 148 / C);
-    if (NC < units || NC * C < M) continue;
-    if (NC * C > bestNC * bestC) {
+    if (nkA % C || nkF % C) continue;
+    if ((nkF / C) * 8192 > 64 * 1024 || (nkA / C) * 8192 > 64 * 1024) continue;
+    const int NC = std::min(ctx->flow_max_cl[C], 148 / C), ncta = NC * C;
+    if (NC < 1 || NC < units || ncta < M) continue;
+    if ((q_units + ncta - 1) / ncta > 8 || (g_units + ncta - 1) / ncta > 8) continue;
+    const bool fit = tiles <= NC;
+    if (!bestC || (fit && !bestFit)) {
       bestC = C;
       bestNC = NC;
+      bestFit = fit;
     }
   }
   if (!bestC) return false;
@@ -525,13 +535,20 @@ bool plan_flow(const pae_ctx* ctx, int B, FlowArgs* fa) {
   fa->B = B;
   fa->C = bestC;
   fa->NC = bestNC;
-  fa->q_tiles = s.qkv_rows / 128;
-  fa->o_tiles = s.D / 128;
-  fa->g_pairs = s.F / 128;
-  fa->d_tiles = s.D / 128;
-  fa->kb_q = nkD / bestC;
+  fa->q_units = q_units;
+  fa->o_tiles = tiles;
+  fa->g_units = g_units;
+  fa->d_tiles = tiles;
+  // O tiles from cluster 0, down tiles on the last clusters, attention after
+  // the O tiles; QKV units from CTA 0, gate/up units after them
+  fa->o_base = 0;
+  fa->d_base = std::max(0, bestNC - tiles);
+  fa->a_base = tiles < bestNC ? tiles : 0;
+  fa->q_base = 0;
+  fa->g_base = q_units % (bestNC * bestC);
+  fa->kb_q = nkD;
   fa->kb_o = nkA / bestC;
-  fa->kb_g = nkD / bestC;
+  fa->kb_g = nkD;
   fa->kb_d = nkF / bestC;
   fa->a_units = units;
   fa->a_qtiles = qtiles;
@@ -876,7 +893,7 @@ pae_status enqueue_flow(pae_ctx* ctx, Plan* P, int k_begin, int k_end, cudaStrea
   fa.err = DevErr{ctx->err_dev, ctx->wait_ns};
   const bool w4 = ctx->w4 != 0;
   const CUtensorMap maps[11] = {w4 ? ctx->tmQqkv : ctx->tmWqkv, w4 ? ctx->tmQo : ctx->tmWo,
-                                w4 ? ctx->tmQgu1 : ctx->tmWgu1, w4 ? ctx->tmQdown : ctx->tmWdown,
+                                w4 ? ctx->tmQg64 : ctx->tmWg64, w4 ? ctx->tmQdown : ctx->tmWdown,
                                 ctx->tmYq64, ctx->tmO64, ctx->tmYg64, ctx->tmU64, ctx->tmQ, ctx->tmK, ctx->tmV};
   P->recs.clear();
   ctx->rec_sink = &P->recs;
@@ -1313,7 +1330,7 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
       return bail(st);
     if ((st = make_map_u8(ctx, &ctx->tmQdown, ctx->q_down, F / 2, (uint64_t)L * D, 32, 128)) != PAE_OK)
       return bail(st);
-    if ((st = make_map_u8(ctx, &ctx->tmQgu1, ctx->q_gu, D / 2, (uint64_t)L * 2 * F, 32, 128)) != PAE_OK)
+    if ((st = make_map_u8(ctx, &ctx->tmQg64, ctx->q_gu, D / 2, (uint64_t)L * 2 * F, 32, 64)) != PAE_OK)
       return bail(st);
   }
   if (ctx->act_bf16 && !ctx->w4) {
@@ -1343,6 +1360,8 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
     ALLOC(ctx->bias_qkv, sizeof(float) * (size_t)kMaxSteps * L * s.qkv_rows);
     ALLOC(ctx->bias_gu, sizeof(float) * (size_t)kMaxSteps * L * 2 * F);
     ALLOC(ctx->f_ctr, sizeof(unsigned) * kFlowCtrWords);
+    if (!ctx->w4 && (st = make_map(ctx, &ctx->tmWg64, ctx->w_gu, D, (uint64_t)L * 2 * F, 64, 64)) != PAE_OK)
+      return bail(st);
     if ((st = make_map(ctx, &ctx->tmYq64, ctx->y, D, Mmax, 64, 64)) != PAE_OK) return bail(st);
     if ((st = make_map(ctx, &ctx->tmYg64, ctx->yg, D, Mmax, 64, 64)) != PAE_OK) return bail(st);
     if ((st = make_map(ctx, &ctx->tmO64, ctx->o, s.attn_dim, Mmax, 64, 64)) != PAE_OK) return bail(st);

@@ -16,7 +16,9 @@ TOL_BF16_REL_RMS = 1e-2
 
 
 def max_abs(a, b) -> float:
-    return float(np.max(np.abs(np.asarray(a, np.float64) - np.asarray(b, np.float64))))
+    """Largest absolute difference (0 for empty arrays, e.g. a zero-length prefix)."""
+    d = np.abs(np.asarray(a, np.float64) - np.asarray(b, np.float64))
+    return float(d.max()) if d.size else 0.0
 
 
 def rel_rms(a, b) -> float:
