@@ -433,7 +433,8 @@ def roofline_for(cfg, batch, res, peaks, peak_kind, lens):
 def run_minimal(args, cfg):
     """Warm-up and timed pae_denoise calls only (for ncu launch ranges): the
     launches before the timed region are 1 (weight transpose) + batch
-    (prefix lengths) + 4 (tables) + warmup x graph kernels."""
+    (prefix lengths) + 6 (tables: time MLP, modulation rows, two projected
+    shift tables) + warmup x graph kernels."""
     import torch
     import flow_matching_action_pi0_b200 as fm
     torch.cuda.set_device(0)
@@ -454,7 +455,7 @@ def run_minimal(args, cfg):
     print(json.dumps({"workload": cfg.name, "pdl": args.pdl, "persistent": persist, "dataflow": flow,
                       "max_splitk": args.max_splitk, "ms_per_step": ms,
                       "splits": ex.query(fm.PAE_Q_SPLITS, cfg.batch), "graph_kernels": k,
-                      "launches_before_timed": 1 + cfg.batch + 4 + args.warmup * k}), flush=True)
+                      "launches_before_timed": 1 + cfg.batch + 6 + args.warmup * k}), flush=True)
     ex.close()
     return 0
 

@@ -25,6 +25,7 @@ PAE_OPT_USE_GRAPH, PAE_OPT_WAIT_LIMIT_US, PAE_OPT_PROFILE, PAE_OPT_PDL, PAE_OPT_
 PAE_OPT_PERSISTENT = 6
 PAE_OPT_FUSED_NORM = 7
 PAE_OPT_DATAFLOW, PAE_OPT_DATAFLOW_CLUSTER = 8, 9
+PAE_OPT_FACTORED_NORM = 10
 (PAE_K_TRANSITION, PAE_K_QKV, PAE_K_ATTENTION, PAE_K_OPROJ, PAE_K_NORM, PAE_K_GATEUP,
  PAE_K_DOWN, PAE_K_PERSISTENT, PAE_K_DATAFLOW) = range(9)
 KERNEL_CLASSES = ("transition", "qkv", "attention", "o_proj", "norm", "gate_up", "down", "persistent", "dataflow")

@@ -68,6 +68,7 @@ struct TransitionArgs {
   float* x_dst;           // write x here after the out step (may equal x)
   int M;
   float* ss_out;          // non-null: the first norm's sum of squares per token -> ss_out[m] (slot 0)
+  int y_factored;         // 1: y = bf16(h (1 + scale)) without rstd and shift (factored adaRMSNorm)
 };
 cudaError_t launch_transition(const Shape& s, int act_bf16, const TransitionArgs& a, bool pdl, cudaStream_t st);
 
@@ -101,6 +102,17 @@ struct EpiArgs {
   // EPI_PREFIX: token m is prefix position m of request `prefix_row`; keys and
   // values go to kc / vc of `layer`
   int prefix_row;
+  // Factored adaRMSNorm.  A consumer (EPI_QKV, EPI_GEGLU with f_ss set) reads
+  // the operand bf16(h (1 + scale)) and applies out = rstd[m] acc + f_bias[row]
+  // (f_bias: W shift of this step and layer, stored row order), rstd[m] =
+  // rsqrt(sum of f_nslots slots (stride ss_ld) / D + eps).  The producer
+  // (EPI_RESID with y_out set, split-K only) also writes y_out[m][f] =
+  // bf16(h (1 + y_scale[f])) and the slots (ss_out).
+  const float* f_bias;
+  const float* f_ss;
+  int f_nslots;
+  void* y_out;
+  const float* y_scale;
 };
 
 // out-features N (for GEGLU: F, weight rows interleaved in 128-row tiles).

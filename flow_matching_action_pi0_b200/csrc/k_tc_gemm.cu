@@ -49,7 +49,7 @@ __host__ __device__ inline uint32_t tmem_cols_for(int n) {
 }
 
 struct TcSmemLayout {
-  uint32_t a_bytes, b_bytes, raw_bytes, h_bytes, stage_bytes, recv_off, recv_bytes, bar_off, norm_off, total;
+  uint32_t a_bytes, b_bytes, raw_bytes, h_bytes, stage_bytes, recv_off, recv_bytes, bar_off, norm_off, rs_off, total;
 };
 
 // Per stage: the bf16 weight tile A ([128*na][64], 128-byte swizzled), the
@@ -73,7 +73,8 @@ __host__ __device__ inline TcSmemLayout tc_layout(int na, const TcPlan& p, bool 
   const uint32_t used = p.recv_alias ? (ring > L.recv_bytes ? ring : L.recv_bytes) : ring + L.recv_bytes;
   L.bar_off = (used + 15u) & ~15u;
   L.norm_off = L.bar_off + 256;  // rstd [64] + partial sums [2][64]
-  L.total = L.norm_off + (norm ? 768u : 0u) + 1024;  // + slack for 1024-byte alignment
+  L.rs_off = L.norm_off + (norm ? 768u : 0u);  // factored adaRMSNorm: rstd of the tile's tokens [256]
+  L.total = L.rs_off + 1024u + 1024u;  // + slack for 1024-byte alignment
   return L;
 }
 
@@ -545,6 +546,28 @@ __global__ void __launch_bounds__(256, 2)
   pdl_wait();  // the epilogue reads the residual stream / slot lengths
 
   // ------------------------------------------------------------------ epilogue
+  // Factored adaRMSNorm: rstd of the tile's tokens from the producers' sums of
+  // squares (slots added in a fixed order), while the MMAs finish.
+  const float* s_rs = reinterpret_cast<const float*>(smem + L.rs_off);
+  constexpr bool kFactor = EPI == EPI_QKV || EPI == EPI_GEGLU;
+  if (kFactor && a.e.f_ss) {
+    const int col = threadIdx.x, m = ttile * p.tn + col;
+    if (col < p.tn) {
+      float acc = 0.f;
+      if (m < a.e.M) {
+        const float* sp = a.e.f_ss + m;
+        constexpr int NB = 8;
+        for (int s0 = 0; s0 < a.e.f_nslots; s0 += NB) {
+          float v[NB];
+#pragma unroll
+          for (int i = 0; i < NB; ++i) v[i] = s0 + i < a.e.f_nslots ? __ldcg(sp + (size_t)(s0 + i) * a.e.ss_ld) : 0.f;
+#pragma unroll
+          for (int i = 0; i < NB; ++i) acc += v[i];
+        }
+      }
+      const_cast<float*>(s_rs)[col] = rsqrtf(acc / (float)s.D + s.eps);
+    }
+  }
   const bool acc_ok = mbar_wait(accf, 0, kDrainNs);
   if (!acc_ok) set_error(a.err, DEV_DRAIN);
   tc_fence_after();
@@ -581,9 +604,27 @@ __global__ void __launch_bounds__(256, 2)
       reg_fence16(x0);
       if (NA == 2) reg_fence16(x1);
     };
+    // factored adaRMSNorm: this thread's row bias (gate/up: the gate row and
+    // the up row 128 below it)
+    const bool fac = kFactor && e.f_ss != nullptr;
+    float fb0 = 0.f, fb1 = 0.f;
+    if (fac && ntile * 128 + row < a.N) {
+      const int srow = NA == 2 ? ntile * 256 + row : ntile * 128 + row;
+      fb0 = e.f_bias[srow];
+      if (NA == 2) fb1 = e.f_bias[srow + 128];
+    }
     auto emit = [&](int c, const float* x0, const float* x1) {
+      if (fac) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) tb[j * TLD + lane] = NA == 2 ? gelu_tanh_bf16out(x0[j]) * x1[j] : x0[j];
+        for (int j = 0; j < 16; ++j) {
+          const float rs = s_rs[c * 16 + j];
+          const float g = fmaf(rs, x0[j], fb0);
+          tb[j * TLD + lane] = NA == 2 ? gelu_tanh_bf16out(g) * fmaf(rs, x1[j], fb1) : g;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) tb[j * TLD + lane] = NA == 2 ? gelu_tanh_bf16out(x0[j]) * x1[j] : x0[j];
+      }
       __syncwarp();
       const int m = mbase + c * 16 + jt;
       if (m < e.M && f < a.N) {
@@ -677,6 +718,14 @@ __global__ void __launch_bounds__(256, 2)
     int lv[UB];
     float4 gv = make_float4(0.f, 0.f, 0.f, 0.f);
     if (EPI == EPI_RESID && ok && vec && fv_ok) gv = *reinterpret_cast<const float4*>(e.gate + fv);
+    // factored adaRMSNorm: the 4 rows' bias (gate/up: gate rows, up rows 128 below)
+    const bool fac = kFactor && e.f_ss != nullptr;
+    float4 fbv0 = make_float4(0.f, 0.f, 0.f, 0.f), fbv1 = fbv0;
+    if (fac && ok && fv_ok) {
+      const int srow = NA == 2 ? ntile * 256 + (fv - ntile * 128) : fv;
+      fbv0 = *reinterpret_cast<const float4*>(e.f_bias + srow);
+      if (NA == 2) fbv1 = *reinterpret_cast<const float4*>(e.f_bias + srow + 128);
+    }
     auto prefetch = [&](int cb) {
 #pragma unroll
       for (int k = 0; k < UB; ++k) {
@@ -717,7 +766,17 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
         for (int k = 0; k < UB; ++k) {
           const int col = cb + k * cstep4, m = mbase + col;
-          if (col < p.tn && m < e.M && fv_ok) epi_vec4<EPI>(s, e, m, fv, s0[k], s1[k], hv[k], gv, lv[k]);
+          if (col < p.tn && m < e.M && fv_ok) {
+            if (fac) {
+              const float rs = s_rs[col];
+              s0[k] = make_float4(fmaf(rs, s0[k].x, fbv0.x), fmaf(rs, s0[k].y, fbv0.y), fmaf(rs, s0[k].z, fbv0.z),
+                                  fmaf(rs, s0[k].w, fbv0.w));
+              if (NA == 2)
+                s1[k] = make_float4(fmaf(rs, s1[k].x, fbv1.x), fmaf(rs, s1[k].y, fbv1.y), fmaf(rs, s1[k].z, fbv1.z),
+                                    fmaf(rs, s1[k].w, fbv1.w));
+            }
+            epi_vec4<EPI>(s, e, m, fv, s0[k], s1[k], hv[k], gv, lv[k]);
+          }
         }
       }
     } else if (ok) {
@@ -753,6 +812,7 @@ __global__ void __launch_bounds__(256, 2)
         // adjacent lanes (R is a power of two <= 32), reduced by a fixed
         // shuffle tree into slot (tile * S + rank).
         const float g = e.gate[f];
+        const float ysc = e.y_out ? 1.f + e.y_scale[f] : 0.f;
         float hv1[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
@@ -766,6 +826,7 @@ __global__ void __launch_bounds__(256, 2)
           if (i < n) {
             hv1[i] = fmaf(g, s0[i], hv1[i]);
             e.h[(size_t)ms[i] * s.D + f] = hv1[i];
+            if (e.y_out) static_cast<bf16*>(e.y_out)[(size_t)ms[i] * s.D + f] = f2bf(hv1[i] * ysc);
             v[i] = hv1[i] * hv1[i];
           }
         }
@@ -777,10 +838,13 @@ __global__ void __launch_bounds__(256, 2)
             for (int i = 0; i < 8; ++i) v[i] += __shfl_xor_sync(gmask, v[i], o);
           }
         }
-        if (rr == 0) {
+        // one slot per 32 rows: (tile * S + rank) * NW + rr / 32, NW = max(1, R / 32)
+        if ((rr & 31) == 0) {
+          const int NW = R > 32 ? R / 32 : 1;
+          const size_t slot = (size_t)(ntile * S + (int)rank) * NW + rr / 32;
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            if (i < n) e.ss_out[(size_t)(ntile * S + (int)rank) * e.ss_ld + ms[i]] = v[i];
+            if (i < n) e.ss_out[slot * e.ss_ld + ms[i]] = v[i];
         }
       }
     }

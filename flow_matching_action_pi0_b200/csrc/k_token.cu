@@ -163,14 +163,15 @@ __global__ void __launch_bounds__(256) k_transition(const Shape s, const Transit
     }
     ss = block_sum(ss, red);
     if (a.ss_out && tid == 0) a.ss_out[m] = ss;  // slot 0 for a projection that normalises in-kernel
-    const float r = rsqrtf(ss / (float)D + s.eps);
+    // factored: the projection applies rstd and the shift term itself
+    const float r = a.y_factored ? 1.f : rsqrtf(ss / (float)D + s.eps);
     const float* sc = a.tab_in + mod_offset(s, 0, 0, 0);
     const float* sh = a.tab_in + mod_offset(s, 0, 0, 1);
     TA* yrow = static_cast<TA*>(a.y) + (size_t)m * D;
     for (int j = 4 * tid; j < D; j += 4 * blockDim.x) {
       const float4 v = *reinterpret_cast<const float4*>(hs + j);
       const float4 c = *reinterpret_cast<const float4*>(sc + j);
-      const float4 d = *reinterpret_cast<const float4*>(sh + j);
+      const float4 d = a.y_factored ? make_float4(0.f, 0.f, 0.f, 0.f) : *reinterpret_cast<const float4*>(sh + j);
       const float o[4] = {v.x * r * (1.f + c.x) + d.x, v.y * r * (1.f + c.y) + d.y, v.z * r * (1.f + c.z) + d.z,
                           v.w * r * (1.f + c.w) + d.w};
       store4(yrow + j, o);

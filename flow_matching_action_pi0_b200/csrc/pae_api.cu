@@ -60,6 +60,7 @@ struct Plan {
   bool flow = false;       // eligible for the dataflow loop (clusters, per-tile counters)
   FlowArgs fa{};
   bool fuse_norm = false;  // QKV / gate-up normalise their fp32 operand in-kernel
+  bool factored = false;   // adaRMSNorm factored into the projections' epilogues (no norm kernels)
   // token-operand maps; a map's box height is the token tile of the projection
   // that reads it (QKV and gate/up may tile the same y differently)
   CUtensorMap tmY{}, tmYg{}, tmO{}, tmU{}, tmH{}, tmHg{};
@@ -162,6 +163,7 @@ struct pae_ctx {
   CUtensorMap tmWg64{};  // gate/up with 64-row boxes (dataflow loop)
   // in-kernel adaRMSNorm: per-token sum-of-squares slots [kSsSlots][ss_ld]
   bool use_fused_norm = false;  // opt-in: measured slower than the norm kernels under PDL
+  bool use_factored = true;     // adaRMSNorm factored into the projections' epilogues
   float* ss_buf = nullptr;
   int ss_ld = 0;
   // int4 weights (W4A16): packed codes [L*rows][K/2] and group scales [L*rows][K/128]
@@ -591,8 +593,10 @@ struct LaunchPlans {
   TcPlan qkv, o, gu, down;
   AttnPlan attn;
   bool fuse_norm;
+  bool factored;
 };
-LaunchPlans plan_launches(const Shape& s, int B, bool w4, int max_splitk, bool use_fused_norm) {
+LaunchPlans plan_launches(const Shape& s, int B, bool w4, int max_splitk, bool use_fused_norm,
+                          bool use_factored = true) {
   LaunchPlans L{};
   const int M = B * s.H;
   L.o = plan_gemm(M, s.D, s.attn_dim, 1, max_splitk, w4);
@@ -608,6 +612,13 @@ LaunchPlans plan_launches(const Shape& s, int B, bool w4, int max_splitk, bool u
   L.qkv = plan_gemm(M, s.qkv_rows, s.D, 1, max_splitk, w4, L.fuse_norm, whole_sm);
   L.gu = plan_gemm(M, s.F, s.D, 2, max_splitk, w4, L.fuse_norm, whole_sm);
   L.attn = plan_attn(s, B);
+  // Factored adaRMSNorm: the residual projections' split-K epilogue (one row
+  // per thread, R = 128 / S <= 64 rows per rank) writes the next operand
+  // bf16(h (1 + scale)) and per-token sums of squares (one slot per 32 rows),
+  // and QKV / gate-up apply rstd and the projected shift in their epilogues.
+  const auto nslots = [](const TcPlan& p) { return p.splits * std::max(1, 128 / p.splits / 32); };
+  L.factored = use_factored && !L.fuse_norm && L.o.splits >= 2 && L.down.splits >= 2 &&
+               (s.D / 128) * std::max(nslots(L.o), nslots(L.down)) <= kSsSlots;
   return L;
 }
 
@@ -618,13 +629,14 @@ pae_status build_plan(pae_ctx* ctx, int B, Plan* P) {
   if (!ctx->act_bf16) return PAE_OK;
   P->persist = plan_persistent(ctx, B, &P->pa);
   P->flow = plan_flow(ctx, B, &P->fa);
-  const LaunchPlans LP = plan_launches(s, B, ctx->w4 != 0, ctx->max_splitk, ctx->use_fused_norm);
+  const LaunchPlans LP = plan_launches(s, B, ctx->w4 != 0, ctx->max_splitk, ctx->use_fused_norm, ctx->use_factored);
   P->qkv = LP.qkv;
   P->o = LP.o;
   P->gu = LP.gu;
   P->down = LP.down;
   P->attn = LP.attn;
   P->fuse_norm = LP.fuse_norm;
+  P->factored = LP.factored;
   const uint64_t Mmax = (uint64_t)s.Bmax * s.H;
   pae_status st;
   if ((st = make_map(ctx, &P->tmY, ctx->y, s.D, Mmax, 64, P->qkv.tn)) != PAE_OK) return st;
@@ -757,9 +769,13 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
   ta.b_out = ctx->b_out;
   ta.dt = ctx->dt;
   ta.M = M;
-  ta.ss_out = P.fuse_norm ? ctx->ss_buf : nullptr;
+  ta.ss_out = (P.fuse_norm || P.factored) ? ctx->ss_buf : nullptr;
+  ta.y_factored = P.factored ? 1 : 0;
   ctx->ev_next = 0;
   const int slots_o = (s.D / 128) * P.o.splits, slots_down = (s.D / 128) * P.down.splits;
+  // factored adaRMSNorm: one slot per (tile, rank, 32 rows)
+  const int fslots_o = slots_o * std::max(1, 128 / P.o.splits / 32);
+  const int fslots_down = slots_down * std::max(1, 128 / P.down.splits / 32);
   for (int k = k_begin; k < k_end; ++k) {
     const float* tk = tab(ctx, k);
     ta.tab_out = (k == k_begin) ? nullptr : tab(ctx, k - 1);
@@ -779,6 +795,12 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
       e.vc = ctx->vc;
       e.lens = ctx->lens_dev;
       e.rope_cs = ctx->rope_cs;
+      if (P.factored) {
+        e.f_bias = ctx->bias_qkv + ((size_t)k * s.L + l) * s.qkv_rows;
+        e.f_ss = ctx->ss_buf;
+        e.ss_ld = ctx->ss_ld;
+        e.f_nslots = l == 0 ? 1 : fslots_down;
+      }
       {
         ProfScope ps(ctx, PAE_K_QKV, st);
         NormIn nq;
@@ -804,15 +826,19 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
       e.epi = EPI_RESID;
       e.h = ctx->h;
       e.gate = tk + mod_offset(s, l, 0, 2);
-      if (P.fuse_norm) {
+      if (P.fuse_norm || P.factored) {
         e.ss_out = ctx->ss_buf;
         e.ss_ld = ctx->ss_ld;
+      }
+      if (P.factored) {
+        e.y_out = ctx->y;
+        e.y_scale = tk + mod_offset(s, l, 1, 0);
       }
       {
         ProfScope ps(ctx, PAE_K_OPROJ, st);
         run_gemm(ctx, P, 1, l, e, st);
       }
-      if (!P.fuse_norm) {
+      if (!P.fuse_norm && !P.factored) {
         ProfScope ps(ctx, PAE_K_NORM, st);
         launch_norm(s, ctx->act_bf16, ctx->h, ctx->y, tk + mod_offset(s, l, 1, 0), tk + mod_offset(s, l, 1, 1), M,
                     pdl_on(ctx), st);
@@ -821,6 +847,12 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
       e.M = M;
       e.epi = EPI_GEGLU;
       e.u = ctx->u;
+      if (P.factored) {
+        e.f_bias = ctx->bias_gu + ((size_t)k * s.L + l) * 2 * s.F;
+        e.f_ss = ctx->ss_buf;
+        e.ss_ld = ctx->ss_ld;
+        e.f_nslots = fslots_o;
+      }
       {
         ProfScope ps(ctx, PAE_K_GATEUP, st);
         NormIn ng;
@@ -832,15 +864,19 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
       e.epi = EPI_RESID;
       e.h = ctx->h;
       e.gate = tk + mod_offset(s, l, 1, 2);
-      if (P.fuse_norm) {
+      if (P.fuse_norm || (P.factored && l + 1 < s.L)) {
         e.ss_out = ctx->ss_buf;
         e.ss_ld = ctx->ss_ld;
+      }
+      if (P.factored && l + 1 < s.L) {
+        e.y_out = ctx->y;
+        e.y_scale = tk + mod_offset(s, l + 1, 0, 0);
       }
       {
         ProfScope ps(ctx, PAE_K_DOWN, st);
         run_gemm(ctx, P, 3, l, e, st);
       }
-      if (l + 1 < s.L && !P.fuse_norm) {
+      if (l + 1 < s.L && !P.fuse_norm && !P.factored) {
         ProfScope ps(ctx, PAE_K_NORM, st);
         launch_norm(s, ctx->act_bf16, ctx->h, ctx->y, tk + mod_offset(s, l + 1, 0, 0), tk + mod_offset(s, l + 1, 0, 1),
                     M, pdl_on(ctx), st);
@@ -1597,6 +1633,14 @@ pae_status pae_set_option(pae_ctx* ctx, int option, long long value) {
       }
       ctx->use_fused_norm = value != 0;
       return PAE_OK;
+    case PAE_OPT_FACTORED_NORM:
+      if ((value != 0) != ctx->use_factored) {
+        drop_graphs(ctx);
+        ctx->plans.clear();
+        ctx->last_plan = nullptr;
+      }
+      ctx->use_factored = value != 0;
+      return PAE_OK;
     case PAE_OPT_PROFILE:
       if (value < 0 || value >= (1LL << PAE_K_COUNT)) return fail(ctx, PAE_ERR_ARG, "bad profile mask");
       if ((unsigned)value != ctx->profile_mask) drop_graphs(ctx);
@@ -1637,7 +1681,7 @@ pae_status pae_query(pae_ctx* ctx, int what, int batch, long long* value) {
     case PAE_Q_TOKEN_TILE: *value = P->qkv.tn; return PAE_OK;
     case PAE_Q_ATTN_SPLITS: *value = P->attn.splits; return PAE_OK;
     case PAE_Q_PERSISTENT: *value = use_persist(ctx, P) ? 1 : 0; return PAE_OK;
-    case PAE_Q_FUSED_NORM: *value = P->fuse_norm ? 1 : 0; return PAE_OK;
+    case PAE_Q_FUSED_NORM: *value = P->fuse_norm ? 1 : P->factored ? 2 : 0; return PAE_OK;
     case PAE_Q_DATAFLOW: *value = use_flow(ctx, P) ? P->fa.C : 0; return PAE_OK;
     default: return fail(ctx, PAE_ERR_ARG, "unknown query %d", what);
   }
@@ -1661,7 +1705,7 @@ pae_status pae_plan_query(const pae_config* cfg, int what, int batch, long long*
       break;
     case PAE_Q_TOKEN_TILE: *value = L.qkv.tn; break;
     case PAE_Q_ATTN_SPLITS: *value = L.attn.splits; break;
-    default: *value = L.fuse_norm ? 1 : 0; break;
+    default: *value = L.fuse_norm ? 1 : L.factored ? 2 : 0; break;
   }
   return PAE_OK;
 }

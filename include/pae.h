@@ -202,6 +202,14 @@ pae_status pae_denoise_steps(pae_ctx* ctx, const float* x_in, float* x_out, int 
  * (statistics from the residual projections' epilogues) instead of separate
  * norm kernels, for batches of at most one 64-token tile.  Both round within
  * the parity tolerance; each is bitwise reproducible.
+ * PAE_OPT_FACTORED_NORM (default 1, bf16 / int4 weights; PAE_OPT_FUSED_NORM
+ * takes precedence): no separate norm kernels.  The O and down projections'
+ * split-K epilogues write the next norm's operand bf16(h (1 + scale)) and
+ * per-token sums of squares of h; QKV and gate/up multiply their accumulators
+ * by 1/rms and add the shift projected through their weights (tables built by
+ * pae_precompute_tables): the same value as projecting adaRMSNorm(h), rounded
+ * differently (within the parity tolerance, bitwise reproducible).  Batches
+ * whose O or down plan has no split-K keep the norm kernels.  0: norm kernels.
  * PAE_OPT_DATAFLOW (default 0, bf16 / int4 weights): batches with batch * chunk <= 64
  * run all K steps as one launch of thread-block clusters whose stages wait on
  * per-tile counters instead of kernel boundaries (no CUDA graph for these
@@ -220,7 +228,8 @@ enum {
   PAE_OPT_PERSISTENT = 6,
   PAE_OPT_FUSED_NORM = 7,
   PAE_OPT_DATAFLOW = 8,
-  PAE_OPT_DATAFLOW_CLUSTER = 9
+  PAE_OPT_DATAFLOW_CLUSTER = 9,
+  PAE_OPT_FACTORED_NORM = 10
 };
 pae_status pae_set_option(pae_ctx* ctx, int option, long long value);
 
@@ -251,8 +260,9 @@ pae_status pae_profile_read(pae_ctx* ctx, int kernel_class, double* total_ms, in
  * PAE_Q_TOKEN_TILE: MMA token tile for `batch`.  PAE_Q_ATTN_SPLITS: key splits
  * of the attention for `batch`.  PAE_Q_PERSISTENT: 1 if pae_denoise runs the
  * persistent kernel for `batch` (option on and the batch eligible), else 0.
- * PAE_Q_FUSED_NORM: 1 if the graph for `batch` normalises inside the
- * projections (no separate norm kernels), else 0.  PAE_Q_DATAFLOW: the
+ * PAE_Q_FUSED_NORM: how the graph for `batch` applies adaRMSNorm: 0 separate
+ * norm kernels, 1 inside the projections from fp32 h (PAE_OPT_FUSED_NORM), 2
+ * factored into the projections' epilogues (PAE_OPT_FACTORED_NORM).  PAE_Q_DATAFLOW: the
  * cluster size of the dataflow loop pae_denoise runs for `batch` (0: it runs
  * the graph or the persistent kernel). */
 enum {

@@ -121,6 +121,9 @@ def test_ragged_bf16_bs16_all_rows_then_fresh_prefixes():
 
 
 def _fused_vs_separate(cfg, lengths=None):
+    """The three ways the graph applies adaRMSNorm (factored into the
+    projections' epilogues by default, in-kernel from fp32 h, separate norm
+    kernels) each match the oracle and are bitwise reproducible."""
     ex, W = build_expert(cfg)
     try:
         ks, vs = wl.make_prefix(cfg, lengths=lengths)
@@ -128,24 +131,36 @@ def _fused_vs_separate(cfg, lengths=None):
         grid = wl.uniform_grid(cfg.steps)
         ex.precompute_tables(grid)
         noise = wl.make_noise(cfg)
-        assert ex.query(fm.PAE_Q_FUSED_NORM, cfg.batch) == 0  # off by default
-        ex.set_option(fm.PAE_OPT_FUSED_NORM, 1)
-        assert ex.query(fm.PAE_Q_FUSED_NORM, cfg.batch) == 1
-        fused = run_gpu(ex, noise)
-        np.testing.assert_array_equal(run_gpu(ex, noise), fused)  # bitwise reproducible
-        ex.set_option(fm.PAE_OPT_FUSED_NORM, 0)
+        ref = oracle_rows(cfg, W, ks, vs, noise, grid)
+        assert ex.query(fm.PAE_Q_FUSED_NORM, cfg.batch) == 2  # factored by default
+        factored = run_gpu(ex, noise)
+        np.testing.assert_array_equal(run_gpu(ex, noise), factored)  # bitwise reproducible
+        assert_parity(factored, ref, cfg.dtype, cfg.name + " factored norm")
+        if cfg.dtype != wl.W4A16:
+            ex.set_option(fm.PAE_OPT_FUSED_NORM, 1)
+            assert ex.query(fm.PAE_Q_FUSED_NORM, cfg.batch) == 1
+            fused = run_gpu(ex, noise)
+            np.testing.assert_array_equal(run_gpu(ex, noise), fused)
+            assert_parity(fused, ref, cfg.dtype, cfg.name + " in-kernel norm")
+            ex.set_option(fm.PAE_OPT_FUSED_NORM, 0)
+        ex.set_option(fm.PAE_OPT_FACTORED_NORM, 0)
         assert ex.query(fm.PAE_Q_FUSED_NORM, cfg.batch) == 0
         sep = run_gpu(ex, noise)
-        ref = oracle_rows(cfg, W, ks, vs, noise, grid)
-        assert_parity(fused, ref, cfg.dtype, cfg.name + " in-kernel norm")
         assert_parity(sep, ref, cfg.dtype, cfg.name + " norm kernels")
+        assert max_abs(sep, factored) < 2e-2
     finally:
         ex.close()
 
 
 def test_fused_norm_tiny_batch3_ragged():
-    # adaRMSNorm inside the QKV / gate-up projections vs the separate norm kernels
+    # factored / in-kernel adaRMSNorm vs the separate norm kernels
     _fused_vs_separate(wl.TINY_FP32.replace(name="tiny_bf16_fn", dtype=wl.BF16, batch=3), lengths=[64, 5, 0])
+
+
+def test_factored_norm_tiny_w4a16_rope():
+    # int4 weights: the projected shifts come from the packed weights
+    cfg = wl.TINY_FP32.replace(name="tiny_w4a16_fn", dtype=wl.W4A16, batch=2, rope_base=10000.0)
+    _fused_vs_separate(cfg, lengths=[64, 17])
 
 
 @pytest.mark.slow

@@ -25,8 +25,9 @@ def test_pi05_plans_match_the_gpu_contexts():
     assert _splits(cfg, 1) == (4, 8, 4, 8)
     assert fm.pae_plan_query(cfg, fm.PAE_Q_TOKEN_TILE, 1) == 64
     assert fm.pae_plan_query(cfg, fm.PAE_Q_ATTN_SPLITS, 1) == 8
-    assert fm.pae_plan_query(cfg, fm.PAE_Q_FUSED_NORM, 1) == 0
+    assert fm.pae_plan_query(cfg, fm.PAE_Q_FUSED_NORM, 1) == 2  # norm factored into the epilogues
     assert _splits(cfg, 32) == (1, 2, 1, 2)
+    assert fm.pae_plan_query(cfg, fm.PAE_Q_FUSED_NORM, 32) == 2
     assert fm.pae_plan_query(cfg, fm.PAE_Q_TOKEN_TILE, 32) == 240
     assert fm.pae_plan_query(cfg, fm.PAE_Q_ATTN_SPLITS, 32) == 1
     w4 = _cfg(wl.PI05_W4A16_BS1)
