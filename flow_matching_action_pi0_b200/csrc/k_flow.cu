@@ -22,18 +22,20 @@
 //    own epilogue forms the GeGLU product.
 //  * O and down (K = heads x head_dim, and the MLP width) split K over the C
 //    ranks of a cluster, one 128-row tile per cluster.  The C partial tiles
-//    are summed by a reduce-scatter inside the cluster: rank p stores rows
-//    [q R, q R + R) of its partial, straight from registers, into rank q's
-//    shared memory (st.async, counted in bytes by q's mbarrier), and rank q
+//    are summed by a reduce-scatter inside the cluster: rank p stages rows
+//    [q R, q R + R) of its partial for rank q and sends them with one bulk
+//    copy into q's shared memory (counted in bytes by q's mbarrier); rank q
 //    adds the C slices in rank order (bitwise reproducible) and runs the
 //    epilogue for its R = 128 / C rows.
 //  * Attention: one cluster per (request, KV head, 128 query rows), its ranks
-//    taking consecutive 64-key chunks (online softmax); rank p stores its
-//    unnormalised output rows with their running max and sum into the rows'
-//    owner, which merges the C partial softmaxes.
+//    taking consecutive 64-key chunks (online softmax); rank p sends its
+//    unnormalised output rows (bf16) and their running max and sum (fp32) to
+//    the rows' owner, which merges the C partial softmaxes in fp32.
 // A receiver tells its peers that its receive area is free (one remote
 // mbarrier arrival each) as soon as it is, long before the data is ready, so
-// an exchange costs no cluster barrier.
+// an exchange costs no cluster barrier.  A peer's arrival for the next
+// exchange also tells the sender that its previous copies have landed, so
+// the staging area is reused only then.
 //
 // adaRMSNorm.  y = h rstd (1 + scale) + shift is not formed: the producer of
 // h writes bf16(h (1 + scale)) and per-row sums of squares once, and the
@@ -72,6 +74,8 @@ constexpr uint32_t kFMisc = 4096;
 constexpr uint32_t kFSmem = kFRing * kFBlk + kFWork + kFMisc + 1024;
 constexpr uint32_t kFOp = 0;             // token operand [kb][64 tokens][64] bf16
 constexpr uint32_t kFRx = 64 * 1024;     // split-K receive area [C][R rows][Mp tokens] fp32 (<= 32 KB)
+constexpr uint32_t kFStg = 96 * 1024;    // split-K rows staged by owner [C][R][Mp] fp32 (<= 32 KB)
+constexpr uint32_t kFAStg = 64 * 1024;   // attention rows staged by owner [C][R][d] bf16 (<= 64 KB)
 constexpr uint32_t kFTmem = 512;
 constexpr uint32_t kColS = 128;          // attention scores (P over their first 32 columns)
 constexpr uint32_t kColO = 256;          // attention output
@@ -163,14 +167,16 @@ __device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
 
 // Stores into another CTA's shared memory whose completion is counted (in
 // bytes) by an mbarrier of that CTA.
-__device__ __forceinline__ void st_async_f4(uint32_t addr, float4 v, uint32_t rbar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
-               "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(rbar)
-               : "memory");
-}
 __device__ __forceinline__ void st_async_f2(uint32_t addr, float a, float b, uint32_t rbar) {
   asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(addr), "f"(a),
                "f"(b), "r"(rbar)
+               : "memory");
+}
+// Bulk copy of `bytes` from this CTA's shared memory into another CTA's,
+// counted (in bytes) by that CTA's mbarrier (both cluster addresses).
+__device__ __forceinline__ void bulk_push(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t rbar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "r"(src), "r"(bytes), "r"(rbar)
                : "memory");
 }
 __device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
@@ -210,6 +216,7 @@ struct FC {
   float* s_rstd;       // [64]
   float* s_tmp;        // [512]
   float* s_st;         // [C][R][2] attention (max, sum) received for this rank's rows
+  int* s_len;          // [64] prefix length of every request (fixed during a launch)
   volatile int* s_abort;
   volatile int* s_flag;
   uint32_t tmem;
@@ -261,6 +268,39 @@ __device__ bool wait_ctr(const FC& c, const unsigned* p, unsigned target) {
       return false;
     }
   }
+}
+
+// Bounded wait by one whole warp until the counters p[0..n) all reach
+// `target`: lane i polls p[i], p[i + 32], ..., so every load is in flight at
+// once (one round trip instead of n).  Warp-uniform result; the closing
+// __syncwarp orders every lane's acquire before what lane 0 does next.
+__device__ bool wait_ctrs(const FC& c, const unsigned* p, int n, unsigned target) {
+  const int lane = threadIdx.x & 31;
+  auto done = [&]() {
+    bool d = true;
+    for (int i = lane; i < n; i += 32) d = ld_acquire_u32(p + i) >= target && d;
+    return __all_sync(0xffffffffu, d);
+  };
+  const unsigned long long t0 = globaltimer_ns();
+  const volatile unsigned* ab = abort_word(*c.a);
+  while (!done()) {
+    int stop = 0;  // 1: the launch is aborting, 2: this wait ran out
+    if (lane == 0) {
+      if (*c.s_abort || *ab) stop = 1;
+      else if ((long long)(globaltimer_ns() - t0) > c.a->err.wait_ns) stop = 2;
+    }
+    stop = __shfl_sync(0xffffffffu, stop, 0);
+    if (stop) {
+      if (lane == 0) {
+        if (stop == 2) raise_abort(c);
+        else *c.s_abort = 1;
+      }
+      __syncwarp();
+      return false;
+    }
+  }
+  __syncwarp();
+  return true;
 }
 
 // Every compute thread's global writes, then one release increment of `p`.
@@ -698,9 +738,10 @@ __device__ float csum(const FC& c, float v) {
 
 // Epilogue of the QKV projection for 8 stored rows f0.. of token m: rstd and
 // the shift term, then q (head-major) or this step's key / value into the
-// request's slot at position lens[b] + i; rotated heads store their 4 pairs
-// on channels i0.. and i0 + d/2..
-__device__ void epi_q(const FC& c, int k, int l, int m, int f0, const float* acc, const float* bv) {
+// request's slot at position len + i; rotated heads store their 4 pairs on
+// channels i0.. and i0 + d/2.., turned by the (cos, sin) values cs[0..4).
+__device__ void epi_q(const FC& c, int l, int m, int len, int f0, const float* acc, const float* bv,
+                      const float2* cs) {
   const Shape& s = *c.s;
   const FlowArgs& a = *c.a;
   const float rs = c.s_rstd[m];
@@ -708,7 +749,6 @@ __device__ void epi_q(const FC& c, int k, int l, int m, int f0, const float* acc
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] = fmaf(rs, acc[i], bv[i]);
   const int b = m / s.H, tt = m - b * s.H;
-  const int len = __ldg(a.lens + b);
   const int qd = s.Hq * s.d, kvd = s.Hkv * s.d;
   bf16* base;
   int j;
@@ -723,14 +763,15 @@ __device__ void epi_q(const FC& c, int k, int l, int m, int f0, const float* acc
     j = fk - g * s.d;
     base = (is_v ? a.vc : a.kc) + (((size_t)(l * s.Bmax + b) * s.Hkv + g) * s.Ptot + len + tt) * s.d;
   }
-  if (a.rope_cs && f0 < qd + kvd) {
+  if (cs) {
     const int i0 = j >> 1;
     float lo[4], hi[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      lo[u] = v[2 * u];
-      hi[u] = v[2 * u + 1];
-      rope_turn(a.rope_cs, s.d, len + tt, i0 + u, lo[u], hi[u]);
+      const float2 t = cs[u];
+      const float x = v[2 * u], y = v[2 * u + 1];
+      lo[u] = x * t.x - y * t.y;
+      hi[u] = y * t.x + x * t.y;
     }
     *reinterpret_cast<uint2*>(base + i0) = make_uint2(pack_bf2(lo[0], lo[1]), pack_bf2(lo[2], lo[3]));
     *reinterpret_cast<uint2*>(base + i0 + (s.d >> 1)) = make_uint2(pack_bf2(hi[0], hi[1]), pack_bf2(hi[2], hi[3]));
@@ -842,15 +883,11 @@ __device__ bool whole_stage(const FC& c, int st, int k, int l, int u, int& sw, i
 
   // 1. every producer of the operand, then its TMA
   bool ok = true;
-  if (c.ct == 0) {
-    if (st == ST_Q && l == 0) {
-      ok = wait_ctr(c, c_tr(a), (unsigned)(a.M * (k - a.k_begin + 1)));
-    } else if (st == ST_Q) {
-      for (int t = 0; ok && t < a.d_tiles; ++t) ok = wait_ctr(c, c_y(a, t), uC * (unsigned)u);
-    } else {
-      for (int t = 0; ok && t < a.o_tiles; ++t) ok = wait_ctr(c, c_ho(a, t), uC * (unsigned)(u + 1));
-    }
-    if (ok) issue_operand(c, st, 0, g.kb, opn);
+  if (c.ct < 32) {
+    if (st == ST_Q && l == 0) ok = wait_ctrs(c, c_tr(a), 1, (unsigned)(a.M * (k - a.k_begin + 1)));
+    else if (st == ST_Q) ok = wait_ctrs(c, c_y(a, 0), a.d_tiles, uC * (unsigned)u);
+    else ok = wait_ctrs(c, c_ho(a, 0), a.o_tiles, uC * (unsigned)(u + 1));
+    if (ok && c.ct == 0) issue_operand(c, st, 0, g.kb, opn);
   }
   FTRACE(c, tr, tb + 1);
   if (!cand(ok)) return false;
@@ -867,16 +904,33 @@ __device__ bool whole_stage(const FC& c, int st, int k, int l, int u, int& sw, i
   tc_fence_after();
   FTRACE(c, tr, tb + 3);
 
-  // 4. per unit: accumulator -> tile -> epilogue
+  // 4. per unit: epilogue inputs staged (bias row in s_tmp; for rotated QKV
+  //    rows the (cos, sin) of the unit's 64 pairs at every token's position,
+  //    [M][64] float2 after the tile), accumulator -> tile, epilogue
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qd = warp & 3, row = qd * 32 + lane;  // TMEM lane = weight row
   const uint32_t tile = smem_u32(c.work);
+  const float2* cstage = reinterpret_cast<const float2*>(c.work + 32768);
   const int Mc = (a.M + 15) & ~15;  // accumulator columns read, 16 at a time
   const float* tb_row = st == ST_Q ? a.bias_qkv + ((size_t)k * s.L + l) * s.qkv_rows
                                    : a.bias_gu + ((size_t)k * s.L + l) * 2 * s.F;
+  const int rot_rows = (s.Hq + s.Hkv) * s.d;
   for (int j = 0; j < nu; ++j) {
     const int t = first + j * c.ncta;
-    if (j > 0) csync();  // the previous unit's epilogue has read the tile
+    if (j > 0) csync();  // the previous unit's epilogue has read the tile and the staged inputs
+    int g0 = 0, g1 = 0;
+    if (st == ST_G) unit_rows(s, ST_G, g, 0, t, g0, g1);  // gate and up rows within a layer
+    c.s_tmp[c.ct] = st == ST_Q ? tb_row[128 * t + c.ct] : tb_row[c.ct < 64 ? g0 + c.ct : g1 + c.ct - 64];
+    const bool rot = st == ST_Q && a.rope_cs != nullptr && 128 * t < rot_rows;
+    if (rot) {
+      float2* cw = reinterpret_cast<float2*>(c.work + 32768);
+      for (int idx = c.ct; idx < a.M * 64; idx += kFCompute) {
+        const int m = idx >> 6, jj = idx & 63;
+        const int b = m / s.H, pos = c.s_len[b] + (m - b * s.H);
+        const int i = ((128 * t + 2 * jj) % s.d) >> 1;
+        cw[idx] = a.rope_cs[(size_t)pos * (s.d >> 1) + i];
+      }
+    }
     const uint32_t taddr = c.tmem + ((uint32_t)(qd * 32) << 16) + 64u * (uint32_t)j;
     for (int c0 = 0; c0 < Mc; c0 += 16) {
       float v[16];
@@ -893,24 +947,22 @@ __device__ bool whole_stage(const FC& c, int st, int k, int l, int u, int& sw, i
         float acc[8], bv[8];
         const uint32_t ta = tile + (uint32_t)((m * 128 + r0) * 4);
         f4_to(acc, ld_shared_f4(ta), ld_shared_f4(ta + 16));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) bv[i] = c.s_tmp[r0 + i];
         const int f0 = 128 * t + r0;
-        f4_to(bv, ldg_f4(tb_row + f0), ldg_f4(tb_row + f0 + 4));
-        epi_q(c, k, l, m, f0, acc, bv);
+        epi_q(c, l, m, c.s_len[m / s.H], f0, acc, bv, rot && f0 < rot_rows ? cstage + m * 64 + r0 / 2 : nullptr);
       }
     } else {
-      int g0, g1;
-      unit_rows(s, ST_G, g, 0, t, g0, g1);  // gate and up rows within a layer
       for (int idx = c.ct; idx < a.M * 8; idx += kFCompute) {
         const int m = idx >> 3, r0 = (idx & 7) * 8;
-        float gv[8], uv[8], bg[8], bu[8], ov[8];
+        float gv[8], uv[8], ov[8];
         const uint32_t ta = tile + (uint32_t)((m * 128 + r0) * 4);
         f4_to(gv, ld_shared_f4(ta), ld_shared_f4(ta + 16));
         f4_to(uv, ld_shared_f4(ta + 256), ld_shared_f4(ta + 272));
-        f4_to(bg, ldg_f4(tb_row + g0 + r0), ldg_f4(tb_row + g0 + r0 + 4));
-        f4_to(bu, ldg_f4(tb_row + g1 + r0), ldg_f4(tb_row + g1 + r0 + 4));
         const float rs = c.s_rstd[m];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) ov[i] = gelu_tanh_bf16out(fmaf(rs, gv[i], bg[i])) * fmaf(rs, uv[i], bu[i]);
+        for (int i = 0; i < 8; ++i)
+          ov[i] = gelu_tanh_bf16out(fmaf(rs, gv[i], c.s_tmp[r0 + i])) * fmaf(rs, uv[i], c.s_tmp[64 + r0 + i]);
         *reinterpret_cast<uint4*>(a.u + (size_t)m * s.F + 64 * t + r0) = pack8(ov);
       }
     }
@@ -954,13 +1006,10 @@ __device__ bool split_stage(const FC& c, int st, int k, int l, int u, int& it, i
 
   // 1. the producers of this rank's K slice of the operand, then its TMA
   bool ok = true;
-  if (c.ct == 0) {
-    if (st == ST_O) {
-      ok = wait_ctr(c, c_att(a), (unsigned)a.a_units * (unsigned)C * (unsigned)(u + 1));
-    } else {
-      for (int j = x0 / 64; ok && j <= (x1 - 1) / 64; ++j) ok = wait_ctr(c, c_u(a, j), (unsigned)(u + 1));
-    }
-    if (ok) issue_operand(c, st, x0, g.kb, opn);
+  if (c.ct < 32) {
+    if (st == ST_O) ok = wait_ctrs(c, c_att(a), 1, (unsigned)a.a_units * (unsigned)C * (unsigned)(u + 1));
+    else ok = wait_ctrs(c, c_u(a, x0 / 64), (x1 - 1) / 64 - x0 / 64 + 1, (unsigned)(u + 1));
+    if (ok && c.ct == 0) issue_operand(c, st, x0, g.kb, opn);
   }
   FTRACE(c, tr, tb + 1);
   if (!cand(ok)) return false;
@@ -977,12 +1026,13 @@ __device__ bool split_stage(const FC& c, int st, int k, int l, int u, int& it, i
   const uint32_t xbytes = (uint32_t)((C - 1) * R * Mp * 4);
   const int per8 = R / 8, nitems = a.M * per8;
   const int npass = (nitems + kFCompute - 1) / kFCompute;
-  // this thread's partial row goes to its owner's slice of rank `rank`
+  // this thread's partial row: own rows straight into this rank's slice of
+  // the receive area, the others staged by owner for one bulk copy per peer
   const int owner = row / R, orow = row - owner * R;
-  const bool local = owner == rank;
-  const uint32_t dl = rx + (uint32_t)((rank * R + orow) * Mp * 4);
-  const uint32_t dst = local ? dl : map_cluster(dl, (uint32_t)owner);
-  const uint32_t dbar = map_cluster(smem_u32(c.rx), (uint32_t)owner);
+  const uint32_t stg = smem_u32(c.work) + kFStg;  // [C][R][Mp] fp32
+  const uint32_t slice = (uint32_t)(R * Mp * 4);
+  const uint32_t dst = owner == rank ? rx + (uint32_t)rank * slice + (uint32_t)(orow * Mp * 4)
+                                     : stg + (uint32_t)owner * slice + (uint32_t)(orow * Mp * 4);
   for (int j = 0; j < nt; ++j) {
     const int t = first + j * a.NC;
     // a. the receive area is free: previous exchange reduced, operand below it
@@ -1005,7 +1055,8 @@ __device__ bool split_stage(const FC& c, int st, int k, int l, int u, int& it, i
       if (has_next) f4_to(in.sc, ldg_f4(scn + f0), ldg_f4(scn + f0 + 4));
     };
     load_in(0);
-    // c. every peer's receive area is free: partial rows to their owners
+    // c. every peer's receive area is free (and so every copy this CTA sent
+    //    in the previous exchange has landed: the staging area is free too)
     if (!xchg_ready(c, xn)) return false;
     if (j == 0) FTRACE(c, tr, tb + 3);
     const uint32_t taddr = c.tmem + ((uint32_t)(qd * 32) << 16) + 64u * (uint32_t)slot;
@@ -1016,16 +1067,16 @@ __device__ bool split_stage(const FC& c, int st, int k, int l, int u, int& it, i
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int col = c0 + 4 * e;
-        if (col < Mp) {
-          const float4 f = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-          if (local) st_shared_f4(dst + (uint32_t)col * 4u, f);
-          else st_async_f4(dst + (uint32_t)col * 4u, f, dbar);
-        }
+        if (col < Mp) st_shared_f4(dst + (uint32_t)col * 4u, make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]));
       }
     }
+    fence_proxy_async_smem();  // the bulk copies read what the threads stored
     tc_fence_before();
     csync();
     if (c.ct == 0) mbar_arrive(&c.acc_empty[slot]);
+    if (c.ct < C && c.ct != rank)  // thread q sends the rows rank q owns
+      bulk_push(map_cluster(rx + (uint32_t)rank * slice, (uint32_t)c.ct), stg + (uint32_t)c.ct * slice, slice,
+                map_cluster(smem_u32(c.rx), (uint32_t)c.ct));
     if (j == 0) FTRACE(c, tr, tb + 4);
     // d. every peer's slice landed
     if (!xchg_wait(c, xn)) return false;
@@ -1196,26 +1247,29 @@ __device__ bool att_stage(const FC& c, int l, int u, int& ac, int& xn, bool& xop
   FTRACE(c, tr, 43);
 
   // -------------------------------------------------- merge in the cluster
-  // the work area (q, K, V) is free once every thread is past its last use
+  // Rows travel as bf16 (unnormalised partial outputs; the weights are
+  // applied in fp32 by the owner): receive area [C][R][d] at the start of
+  // the work area, rows staged by owner [C][R][d] at kFAStg, one bulk copy
+  // per peer; (max, sum) per row as fp32 stores into the owner's s_st.
+  // The work area (q, K, V) is free once every thread is past its last use.
   csync();
   const int R = 128 / C, owner = r / R, orow = r - owner * R;
-  xchg_open(c, (uint32_t)((C - 1) * R * (d * 4 + 8)));
+  const uint32_t slice = (uint32_t)(R * d * 2);
+  xchg_open(c, (uint32_t)(C - 1) * (slice + (uint32_t)(R * 8)));
   xopen = true;
   if (!xchg_ready(c, xn)) return false;
   FTRACE(c, tr, 44);
   {
     const bool local = owner == c.rank;
-    const uint32_t ra = smem_u32(c.work) + (uint32_t)((c.rank * R + orow) * d * 4);
+    const uint32_t rx = smem_u32(c.work), stg = smem_u32(c.work) + kFAStg;
+    const uint32_t dr = (local ? rx + (uint32_t)c.rank * slice : stg + (uint32_t)owner * slice) + (uint32_t)(orow * d * 2);
     const uint32_t sa = smem_u32(c.s_st) + (uint32_t)((c.rank * R + orow) * 8);
-    const uint32_t dbar = map_cluster(smem_u32(c.rx), (uint32_t)owner);
-    const uint32_t dr = local ? ra : map_cluster(ra, (uint32_t)owner);
-    const uint32_t ds = local ? sa : map_cluster(sa, (uint32_t)owner);
     const float mv = au.nch > 0 ? m_run : -INFINITY, lv = au.nch > 0 ? l_run : 0.f;
     if (local) {
-      st_shared_f32(ds, mv);
-      st_shared_f32(ds + 4, lv);
+      st_shared_f32(sa, mv);
+      st_shared_f32(sa + 4, lv);
     } else {
-      st_async_f2(ds, mv, lv, dbar);
+      st_async_f2(map_cluster(sa, (uint32_t)owner), mv, lv, map_cluster(smem_u32(c.rx), (uint32_t)owner));
     }
     for (int j = 0; j < d; j += 16) {
       float ov[16];
@@ -1226,16 +1280,21 @@ __device__ bool att_stage(const FC& c, int l, int u, int& ac, int& xn, bool& xop
 #pragma unroll
         for (int t = 0; t < 16; ++t) ov[t] = 0.f;
       }
-#pragma unroll
-      for (int t4 = 0; t4 < 4; ++t4) {
-        const float4 f = make_float4(ov[4 * t4], ov[4 * t4 + 1], ov[4 * t4 + 2], ov[4 * t4 + 3]);
-        const uint32_t o = (uint32_t)((j + 4 * t4) * 4);
-        if (local) st_shared_f4(dr + o, f);
-        else st_async_f4(dr + o, f, dbar);
-      }
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dr + (uint32_t)j * 2u), "r"(pack_bf2(ov[0], ov[1])),
+                   "r"(pack_bf2(ov[2], ov[3])), "r"(pack_bf2(ov[4], ov[5])), "r"(pack_bf2(ov[6], ov[7]))
+                   : "memory");
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dr + (uint32_t)j * 2u + 16u),
+                   "r"(pack_bf2(ov[8], ov[9])), "r"(pack_bf2(ov[10], ov[11])), "r"(pack_bf2(ov[12], ov[13])),
+                   "r"(pack_bf2(ov[14], ov[15]))
+                   : "memory");
     }
+    fence_proxy_async_smem();  // the bulk copies read what the threads stored
+    tc_fence_before();
+    csync();
+    if (c.ct < C && c.ct != c.rank)  // thread q sends the rows rank q owns
+      bulk_push(map_cluster(rx + (uint32_t)c.rank * slice, (uint32_t)c.ct), stg + (uint32_t)c.ct * slice, slice,
+                map_cluster(smem_u32(c.rx), (uint32_t)c.ct));
   }
-  tc_fence_before();
   if (!xchg_wait(c, xn)) return false;
   ++xn;
   xopen = false;
@@ -1268,11 +1327,11 @@ __device__ bool att_stage(const FC& c, int l, int u, int& ac, int& xn, bool& xop
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int q = 0; q < C; ++q) {
       const float w = c.s_tmp[rr * C + q];
-      const float4 v = ld_shared_f4(smem_u32(c.work) + (uint32_t)(((q * R + rr) * d + 4 * c4) * 4));
-      acc.x = fmaf(w, v.x, acc.x);
-      acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z);
-      acc.w = fmaf(w, v.w, acc.w);
+      const uint2 p = *reinterpret_cast<const uint2*>(c.work + ((size_t)(q * R + rr) * d + 4 * c4) * 2);
+      acc.x = fmaf(w, __uint_as_float(p.x << 16), acc.x);
+      acc.y = fmaf(w, __uint_as_float(p.x & 0xFFFF0000u), acc.y);
+      acc.z = fmaf(w, __uint_as_float(p.y << 16), acc.z);
+      acc.w = fmaf(w, __uint_as_float(p.y & 0xFFFF0000u), acc.w);
     }
     const int hl = rq / s.H, ti = rq - hl * s.H;
     bf16* orow = a.o + (size_t)(au.b * s.H + ti) * s.attn_dim + (au.g * s.G + hl) * d;
@@ -1300,10 +1359,7 @@ __device__ bool transition(const FC& c, int k_out, int k_in) {
   float* xrow = a.x + (size_t)m * A;
   if (k_out >= 0) {
     bool ok = true;
-    if (tid == 0) {
-      const unsigned tgt = (unsigned)a.C * (unsigned)((k_out - a.k_begin) * s.L + s.L);
-      for (int t = 0; ok && t < a.d_tiles; ++t) ok = wait_ctr(c, c_y(a, t), tgt);
-    }
+    if (tid < 32) ok = wait_ctrs(c, c_y(a, 0), a.d_tiles, (unsigned)a.C * (unsigned)((k_out - a.k_begin) * s.L + s.L));
     if (!cand(ok)) return false;
     const float* tab = a.tables + (size_t)k_out * s.table_rows;
     const float* sc = tab + final_offset(s, 0);
@@ -1398,6 +1454,8 @@ __device__ void compute_loop(const FC& c) {
   int it = 0, sw = 0, ac = 0, xn = 0, kv_issued = 0;
   int opn[4] = {0, 0, 0, 0};
   bool xopen = false;
+  if (c.ct < a.B) c.s_len[c.ct] = __ldg(a.lens + c.ct);  // set before the launch, fixed during it
+  csync();
   bool ok = transition(c, -1, a.k_begin);
   for (int k = a.k_begin; ok && k < a.k_end; ++k) {
     for (int l = 0; ok && l < s.L; ++l) {
@@ -1415,6 +1473,14 @@ __device__ void compute_loop(const FC& c) {
       if (opn[gi] > 0 && !mbar_wait(&c.op_full[gi], (opn[gi] - 1) & 1, kFDrain)) set_error(a.err, DEV_DRAIN);
     if (kv_issued > 0 && !mbar_wait(c.kv_full, (kv_issued - 1) & 1, kFDrain)) set_error(a.err, DEV_DRAIN);
     if (xopen && a.C > 1) (void)mbar_wait(c.rx, (uint32_t)xn & 1u, kFExitWait);
+    // after an abort, bulk copies this CTA sent may not have been awaited by
+    // their receivers: give them time to read this CTA's staging area (they
+    // take microseconds) before the exit barrier
+    if (*c.s_abort && (xn > 0 || xopen)) {
+      const unsigned long long t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 200000ull) {
+      }
+    }
   }
 }
 
@@ -1470,6 +1536,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
   c.s_rstd = reinterpret_cast<float*>(misc + 512);   // [64]
   c.s_tmp = reinterpret_cast<float*>(misc + 768);    // [512]
   c.s_st = reinterpret_cast<float*>(misc + 2816);    // [C][R][2] = 1 KB
+  c.s_len = reinterpret_cast<int*>(misc + 3840);     // [64]
   c.cta = blockIdx.x;
   c.ncta = gridDim.x;
   c.rank = (int)cluster_rank();

@@ -774,8 +774,8 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
   ctx->ev_next = 0;
   const int slots_o = (s.D / 128) * P.o.splits, slots_down = (s.D / 128) * P.down.splits;
   // factored adaRMSNorm: one slot per (tile, rank, 32 rows)
-  const int fslots_o = slots_o * std::max(1, 128 / P.o.splits / 32);
-  const int fslots_down = slots_down * std::max(1, 128 / P.down.splits / 32);
+  const int fslots_o = P.factored ? slots_o * std::max(1, 128 / P.o.splits / 32) : 0;
+  const int fslots_down = P.factored ? slots_down * std::max(1, 128 / P.down.splits / 32) : 0;
   for (int k = k_begin; k < k_end; ++k) {
     const float* tk = tab(ctx, k);
     ta.tab_out = (k == k_begin) ? nullptr : tab(ctx, k - 1);
