@@ -112,6 +112,7 @@ class ClockSampler:
 
 FUSED_NORM = [0]  # PAE_OPT_FUSED_NORM for every context the benchmark creates
 DATAFLOW = [-1]   # PAE_OPT_DATAFLOW for every context (-1: the library default)
+FACTORED = [-1]   # PAE_OPT_FACTORED_NORM for every context (-1: the library default)
 
 
 def algorithmic(cfg: wl.ExpertConfig, batch: int, lens=None):
@@ -151,9 +152,17 @@ def algorithmic(cfg: wl.ExpertConfig, batch: int, lens=None):
 
 # The files each kernel class is compiled from (its own file and the headers
 # it includes); a traffic figure stays valid while these are unchanged.
+_GEMM_SOURCES = ["k_tc_gemm.cu", "epilogue.cuh", "internal.h", "common.cuh", "launch.cuh"]
 KERNEL_SOURCES = {
     "attention": ["k_attn_tc.cu", "internal.h", "common.cuh", "launch.cuh"],
-    "gemm": ["k_tc_gemm.cu", "epilogue.cuh", "internal.h", "common.cuh", "launch.cuh"],
+    "gemm": _GEMM_SOURCES,
+    "qkv": _GEMM_SOURCES,
+    "o_proj": _GEMM_SOURCES,
+    "gate_up": _GEMM_SOURCES,
+    "down": _GEMM_SOURCES,
+    "transition": ["k_token.cu", "internal.h", "common.cuh", "launch.cuh"],
+    "norm": ["k_token.cu", "internal.h", "common.cuh", "launch.cuh"],
+    "dataflow": ["k_flow.cu", "epilogue.cuh", "internal.h", "common.cuh", "launch.cuh"],
 }
 
 
@@ -269,6 +278,8 @@ def setup_context(cfg, W, batch: int, lens=None):
     ex.set_option(fm.PAE_OPT_FUSED_NORM, FUSED_NORM[0])
     if DATAFLOW[0] >= 0:
         ex.set_option(fm.PAE_OPT_DATAFLOW, DATAFLOW[0])
+    if FACTORED[0] >= 0:
+        ex.set_option(fm.PAE_OPT_FACTORED_NORM, FACTORED[0])
     if lens is None:
         lens = [cfg.prefix] * batch
     ks, vs = wl.make_prefix(cfg, lengths=lens)
@@ -419,6 +430,9 @@ def roofline_for(cfg, batch, res, peaks, peak_kind, lens):
                "timing": "CUDA events around each launch (serialised; duration is an upper bound)",
                "traffic": ncu_traffic(cfg.name if batch == cfg.batch else f"{cfg.name}@{batch}", dom)})
     rl["per_class"] = {c: class_fractions(per[c], ks[c]["ms_per_launch"], peaks) for c in timed_classes}
+    wname = cfg.name if batch == cfg.batch else f"{cfg.name}@{batch}"
+    for c in timed_classes:
+        rl["per_class"][c]["traffic"] = ncu_traffic(wname, c)
     # whole loop against the HBM and tensor rooflines
     t_step = res["ms_per_step"] * 1e-3 / cfg.steps
     loop = {"euler_step_us": t_step * 1e6, "bytes_per_euler_step": step["bytes"],
@@ -693,6 +707,8 @@ def main():
                     help="adaRMSNorm inside the projections for batches of <= 64 tokens (1/0; 0 keeps norm kernels)")
     ap.add_argument("--dataflow", type=int, default=-1,
                     help="dataflow loop for batches of <= 64 tokens (1/0; -1 keeps the library default)")
+    ap.add_argument("--factored-norm", dest="factored_norm", type=int, default=-1,
+                    help="adaRMSNorm factored into the projections' epilogues (1/0; -1 keeps the library default)")
     ap.add_argument("--persistent", type=int, default=0,
                     help="persistent kernel for batches of <= 64 tokens (1/0; 0 runs the captured graph)")
     args = ap.parse_args()
@@ -701,6 +717,7 @@ def main():
     cfg = wl.CONFIGS[args.config]
     FUSED_NORM[0] = args.fused_norm
     DATAFLOW[0] = args.dataflow
+    FACTORED[0] = args.factored_norm
     if args.impl == "reference":
         return run_reference(args, cfg)
     if args.minimal:

@@ -414,12 +414,16 @@ __global__ void __launch_bounds__(384, 1)
 
   if (gridDim.y > 1) {
     // Split-KV merge inside the cluster of key splits.  Every CTA parks its
-    // unnormalised O rows (stride d+4 floats, bank-conflict free) and its row
-    // max / sum in shared memory (the Q and K/V buffers are idle now); CTA
-    // rank r then merges rows [r*R, r*R+R) over all ranks in rank order.
+    // unnormalised O rows as bf16 (row stride d + 8, bank-conflict free; the
+    // Q and K/V buffers are idle now) and its row max / sum in shared memory;
+    // CTA rank r then merges rows [r*R, r*R+R) over all ranks in rank order.
+    // Distributed shared memory moves a few tens of GB/s per SM, so the rows
+    // travel in bf16 (the weights and the sum stay fp32) and each (row, rank)
+    // weight exp2(m_q - M) / L is formed once, not per column.
     __syncthreads();  // all MMAs and TMEM reads of this CTA are done
-    const int ld = d + 4;
-    float* red = reinterpret_cast<float*>(smem);
+    const int ldb = d + 8;
+    bf16* red = reinterpret_cast<bf16*>(smem);
+    float* tbl = reinterpret_cast<float*>(smem + (size_t)QROWS * ldb * 2);  // [R][S] (m, l), then weights
     if (smx) {
       const int h = warp >= 8 ? 1 : 0;
       const int r = (warp & 3) * 32 + lane;
@@ -431,10 +435,12 @@ __global__ void __launch_bounds__(384, 1)
           tmem_ld16(t_o + lane_off + j, ov);
           tmem_ld_wait();
         }
+        uint32_t pk[8];
 #pragma unroll
-        for (int t = 0; t < 16; t += 4)
-          *reinterpret_cast<float4*>(red + r * ld + j + t) =
-              has ? make_float4(ov[t], ov[t + 1], ov[t + 2], ov[t + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int t = 0; t < 8; ++t) pk[t] = has ? pack_bf16x2(ov[2 * t], ov[2 * t + 1]) : 0u;
+        uint4* dst = reinterpret_cast<uint4*>(red + r * ldb + j);
+        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       }
       if (!has && h == 0) {
         s_ml[2 * r] = -INFINITY;
@@ -446,43 +452,54 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t rank = cluster_rank();
     const int R = QROWS / S;
     const uint32_t red_base = smem_u32(red), ml_base = smem_u32(s_ml);
-    const int per_row = d / 4;  // float4 columns
+    // (max, sum) of every (row, rank) once, then the row's weights
+    if ((int)threadIdx.x < R * S) {
+      const int rr = threadIdx.x / S, q = threadIdx.x - rr * S;
+      const uint32_t ra = map_cluster(ml_base + (uint32_t)(((int)rank * R + rr) * 8), (uint32_t)q);
+      tbl[2 * threadIdx.x] = ld_cluster_f32(ra);
+      tbl[2 * threadIdx.x + 1] = ld_cluster_f32(ra + 4);
+    }
+    __syncthreads();
+    float* wt = tbl + 2 * R * S;  // [R][S]
+    if ((int)threadIdx.x < R) {
+      const float* e = tbl + 2 * threadIdx.x * S;
+      float M = -INFINITY;
+      for (int q = 0; q < S; ++q) M = fmaxf(M, e[2 * q]);
+      float wsum = 0.f;
+      for (int q = 0; q < S; ++q)
+        if (e[2 * q + 1] > 0.f) wsum = fmaf(exp2f(e[2 * q] - M), e[2 * q + 1], wsum);
+      const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+      for (int q = 0; q < S; ++q)
+        wt[threadIdx.x * S + q] = e[2 * q + 1] > 0.f ? exp2f(e[2 * q] - M) * inv : 0.f;
+    }
+    __syncthreads();
+    const int per_row = d / 8;  // 16-byte column groups
     for (int el = threadIdx.x; el < R * per_row; el += blockDim.x) {
-      const int rr = el / per_row, c4 = el - rr * per_row;
+      const int rr = el / per_row, c8 = el - rr * per_row;
       const int row = (int)rank * R + rr;
       const int rq = qt * QROWS + row;
       if (rq >= GH) continue;
-      // issue every rank's loads first (they pipeline), then merge in rank order
-      float ms[8], ls[8];
-      float4 vs[8];
+      // every rank's loads first (they pipeline), then the merge in rank order
+      uint4 vs[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q)
-        if (q < S) {
-          ms[q] = ld_cluster_f32(map_cluster(ml_base + row * 8, (uint32_t)q));
-          ls[q] = ld_cluster_f32(map_cluster(ml_base + row * 8 + 4, (uint32_t)q));
-          vs[q] = ld_cluster_f32x4(map_cluster(red_base + (uint32_t)((row * ld + c4 * 4) * 4), (uint32_t)q));
-        }
-      float M = -INFINITY;
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        if (q < S) M = fmaxf(M, ms[q]);
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      float wsum = 0.f;
+        if (q < S) vs[q] = ld_cluster_u32x4(map_cluster(red_base + (uint32_t)((row * ldb + c8 * 8) * 2), (uint32_t)q));
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        if (q >= S || !(ls[q] > 0.f)) continue;
-        const float w = exp2f(ms[q] - M);
-        wsum = fmaf(w, ls[q], wsum);
-        acc[0] = fmaf(w, vs[q].x, acc[0]);
-        acc[1] = fmaf(w, vs[q].y, acc[1]);
-        acc[2] = fmaf(w, vs[q].z, acc[2]);
-        acc[3] = fmaf(w, vs[q].w, acc[3]);
+        if (q >= S) continue;
+        const float w = wt[rr * S + q];
+        const uint32_t u[4] = {vs[q].x, vs[q].y, vs[q].z, vs[q].w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          acc[2 * t] = fmaf(w, __uint_as_float(u[t] << 16), acc[2 * t]);
+          acc[2 * t + 1] = fmaf(w, __uint_as_float(u[t] & 0xFFFF0000u), acc[2 * t + 1]);
+        }
       }
-      const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
       const int hl = rq / s.H, ti = rq - hl * s.H;
       bf16* orow = reinterpret_cast<bf16*>(a.o) + (size_t)(b * s.H + ti) * s.attn_dim + (g * s.G + hl) * d;
-      *reinterpret_cast<uint2*>(orow + c4 * 4) =
-          make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+      *reinterpret_cast<uint4*>(orow + c8 * 8) = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                                            pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
     }
     cluster_sync();  // peers may still be reading this CTA's partial
   }

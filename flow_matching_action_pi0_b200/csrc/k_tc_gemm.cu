@@ -547,25 +547,36 @@ __global__ void __launch_bounds__(256, 2)
 
   // ------------------------------------------------------------------ epilogue
   // Factored adaRMSNorm: rstd of the tile's tokens from the producers' sums of
-  // squares (slots added in a fixed order), while the MMAs finish.
-  const float* s_rs = reinterpret_cast<const float*>(smem + L.rs_off);
+  // squares, while the MMAs finish.  Thread = (token, part): the P parts of a
+  // token take every P-th slot with all loads in flight, and the token's
+  // thread adds the P partial sums in a fixed order.
+  float* s_rs = reinterpret_cast<float*>(smem + L.rs_off);
   constexpr bool kFactor = EPI == EPI_QKV || EPI == EPI_GEGLU;
   if (kFactor && a.e.f_ss) {
-    const int col = threadIdx.x, m = ttile * p.tn + col;
+    const int P = p.tn <= 64 ? 4 : p.tn <= 128 ? 2 : 1;
+    const int col = threadIdx.x % (256 / P), part = threadIdx.x / (256 / P);
+    const int m = ttile * p.tn + col;
     if (col < p.tn) {
       float acc = 0.f;
       if (m < a.e.M) {
         const float* sp = a.e.f_ss + m;
-        constexpr int NB = 8;
-        for (int s0 = 0; s0 < a.e.f_nslots; s0 += NB) {
+        constexpr int NB = 16;
+        for (int s0 = part; s0 < a.e.f_nslots; s0 += NB * P) {
           float v[NB];
 #pragma unroll
-          for (int i = 0; i < NB; ++i) v[i] = s0 + i < a.e.f_nslots ? __ldcg(sp + (size_t)(s0 + i) * a.e.ss_ld) : 0.f;
+          for (int i = 0; i < NB; ++i)
+            v[i] = s0 + i * P < a.e.f_nslots ? __ldcg(sp + (size_t)(s0 + i * P) * a.e.ss_ld) : 0.f;
 #pragma unroll
           for (int i = 0; i < NB; ++i) acc += v[i];
         }
       }
-      const_cast<float*>(s_rs)[col] = rsqrtf(acc / (float)s.D + s.eps);
+      s_rs[part * p.tn + col] = acc;
+    }
+    __syncthreads();
+    if (threadIdx.x < p.tn) {
+      float t = 0.f;
+      for (int q = 0; q < P; ++q) t += s_rs[q * p.tn + threadIdx.x];
+      s_rs[threadIdx.x] = rsqrtf(t / (float)s.D + s.eps);
     }
   }
   const bool acc_ok = mbar_wait(accf, 0, kDrainNs);
@@ -702,11 +713,11 @@ __global__ void __launch_bounds__(256, 2)
     // 4*(t % (R/4)).. and tokens t / (R/4) + k * 256 / (R/4), one float4 per
     // source in rank order.  The loads the epilogue needs (residual stream,
     // gate, slot lengths) are issued before the cluster barrier, so they
-    // overlap the wait for the slowest rank.  (The residual epilogue that
-    // also writes the per-token sums of squares keeps one row per thread: its
-    // shuffle tree runs over the R threads of a token.)
+    // overlap the wait for the slowest rank.  The residual epilogue that also
+    // feeds the next norm (ss_out) adds the squares of a token's R rows over
+    // its R/4 adjacent lanes into slot (tile * S + rank).
     constexpr int UB = 8;  // tokens per batch
-    const bool vec = !(EPI == EPI_RESID && e.ss_out);
+    constexpr bool vec = true;
     const int G4 = R / 4, lg4 = __ffs(G4) - 1;
     const int g4 = threadIdx.x & (G4 - 1);
     const int cstep4 = 256 >> lg4;
@@ -716,8 +727,11 @@ __global__ void __launch_bounds__(256, 2)
     const bool need_len = EPI == EPI_QKV && (fv >= s.Hq * s.d || e.rope_cs);
     float4 hv[UB];
     int lv[UB];
-    float4 gv = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (EPI == EPI_RESID && ok && vec && fv_ok) gv = *reinterpret_cast<const float4*>(e.gate + fv);
+    float4 gv = make_float4(0.f, 0.f, 0.f, 0.f), ysv = gv;
+    if (EPI == EPI_RESID && ok && vec && fv_ok) {
+      gv = *reinterpret_cast<const float4*>(e.gate + fv);
+      if (e.y_out) ysv = *reinterpret_cast<const float4*>(e.y_scale + fv);
+    }
     // factored adaRMSNorm: the 4 rows' bias (gate/up: gate rows, up rows 128 below)
     const bool fac = kFactor && e.f_ss != nullptr;
     float4 fbv0 = make_float4(0.f, 0.f, 0.f, 0.f), fbv1 = fbv0;
@@ -778,73 +792,29 @@ __global__ void __launch_bounds__(256, 2)
             epi_vec4<EPI>(s, e, m, fv, s0[k], s1[k], hv[k], gv, lv[k]);
           }
         }
-      }
-    } else if (ok) {
-      // Thread t keeps one row (t % R) and walks the tokens t / R, t / R + 256 / R, ...
-      const int rr = threadIdx.x % R;
-      const int f = ntile * 128 + (int)rank * R + rr;
-      const int cstep = 256 / R;
-      const uint32_t rbase = smem_u32(recv) + (uint32_t)rr * 4u;
-      const uint32_t src_stride = (uint32_t)p.tn * R * 4u;
-#pragma unroll 1
-      for (int c0 = threadIdx.x / R; c0 < p.tn; c0 += 8 * cstep) {
-        float s0[8];
-        int ms[8];
-        int n = 0;
+        if constexpr (EPI == EPI_RESID) {
+          if (e.ss_out) {
+            // the next norm: operand bf16(h (1 + scale)) of the 4 rows, and the
+            // sum of squares of h over this rank's R rows per token (the R/4
+            // threads of a token are adjacent lanes: fixed shuffle tree)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int col = c0 + i * cstep;
-          s0[i] = 0.f;
-          ms[i] = mbase + col;
-          if (col < p.tn && mbase + col < e.M) n = i + 1;
-        }
-        if (n == 0 || f >= a.N) break;
-#pragma unroll 1
-        for (int src = 0; src < S; ++src) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint32_t addr = rbase + (uint32_t)(c0 + i * cstep) * R * 4u + src * src_stride;
-            if (i < n) s0[i] += ld_shared_f32(addr);
+            for (int k = 0; k < UB; ++k) {
+              const int col = cb + k * cstep4, m = mbase + col;
+              const bool valid = col < p.tn && m < e.M && fv_ok;
+              float sq = 0.f;
+              if (valid) {
+                const float4 h4 = make_float4(fmaf(gv.x, s0[k].x, hv[k].x), fmaf(gv.y, s0[k].y, hv[k].y),
+                                              fmaf(gv.z, s0[k].z, hv[k].z), fmaf(gv.w, s0[k].w, hv[k].w));
+                sq = fmaf(h4.x, h4.x, fmaf(h4.y, h4.y, fmaf(h4.z, h4.z, h4.w * h4.w)));
+                if (e.y_out)
+                  store4_bf16(static_cast<bf16*>(e.y_out) + (size_t)m * s.D + fv, h4.x * (1.f + ysv.x),
+                              h4.y * (1.f + ysv.y), h4.z * (1.f + ysv.z), h4.w * (1.f + ysv.w));
+              }
+              const unsigned gm = G4 >= 32 ? 0xffffffffu : (((1u << G4) - 1u) << (lane & ~(G4 - 1)));
+              for (int o = 1; o < G4; o <<= 1) sq += __shfl_xor_sync(gm, sq, o);
+              if (valid && g4 == 0) e.ss_out[(size_t)(ntile * S + (int)rank) * e.ss_ld + m] = sq;
+            }
           }
-        }
-        // Gated residual, then the sum of squares of the updated h over this
-        // rank's R rows per token: the R threads of a token group are
-        // adjacent lanes (R is a power of two <= 32), reduced by a fixed
-        // shuffle tree into slot (tile * S + rank).
-        const float g = e.gate[f];
-        const float ysc = e.y_out ? 1.f + e.y_scale[f] : 0.f;
-        float hv1[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (i < n) hv1[i] = e.h[(size_t)ms[i] * s.D + f];
-        const int lane_g = (threadIdx.x & 31) & ~(R - 1);
-        const unsigned gmask = R >= 32 ? 0xffffffffu : (((1u << R) - 1u) << lane_g);
-        float v[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          v[i] = 0.f;
-          if (i < n) {
-            hv1[i] = fmaf(g, s0[i], hv1[i]);
-            e.h[(size_t)ms[i] * s.D + f] = hv1[i];
-            if (e.y_out) static_cast<bf16*>(e.y_out)[(size_t)ms[i] * s.D + f] = f2bf(hv1[i] * ysc);
-            v[i] = hv1[i] * hv1[i];
-          }
-        }
-#pragma unroll
-        for (int lvl = 4; lvl >= 0; --lvl) {  // offsets R/2 .. 1, all eight tokens per level
-          const int o = 1 << lvl;
-          if (o < R) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] += __shfl_xor_sync(gmask, v[i], o);
-          }
-        }
-        // one slot per 32 rows: (tile * S + rank) * NW + rr / 32, NW = max(1, R / 32)
-        if ((rr & 31) == 0) {
-          const int NW = R > 32 ? R / 32 : 1;
-          const size_t slot = (size_t)(ntile * S + (int)rank) * NW + rr / 32;
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            if (i < n) e.ss_out[slot * e.ss_ld + ms[i]] = v[i];
         }
       }
     }

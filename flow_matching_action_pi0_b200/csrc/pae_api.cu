@@ -163,7 +163,7 @@ struct pae_ctx {
   CUtensorMap tmWg64{};  // gate/up with 64-row boxes (dataflow loop)
   // in-kernel adaRMSNorm: per-token sum-of-squares slots [kSsSlots][ss_ld]
   bool use_fused_norm = false;  // opt-in: measured slower than the norm kernels under PDL
-  bool use_factored = true;     // adaRMSNorm factored into the projections' epilogues
+  bool use_factored = false;    // opt-in: measured slower than the norm kernels under PDL
   float* ss_buf = nullptr;
   int ss_ld = 0;
   // int4 weights (W4A16): packed codes [L*rows][K/2] and group scales [L*rows][K/128]
@@ -596,7 +596,7 @@ struct LaunchPlans {
   bool factored;
 };
 LaunchPlans plan_launches(const Shape& s, int B, bool w4, int max_splitk, bool use_fused_norm,
-                          bool use_factored = true) {
+                          bool use_factored) {
   LaunchPlans L{};
   const int M = B * s.H;
   L.o = plan_gemm(M, s.D, s.attn_dim, 1, max_splitk, w4);
@@ -608,17 +608,19 @@ LaunchPlans plan_launches(const Shape& s, int B, bool w4, int max_splitk, bool u
   L.fuse_norm = use_fused_norm && !w4 && M <= 64 && tn_small <= 64 && L.o.splits >= 4 && L.down.splits >= 4 &&
                 L.o.tok_tiles == 1 && L.down.tok_tiles == 1 &&
                 (s.D / 128) * std::max(L.o.splits, L.down.splits) <= kSsSlots;
-  const bool whole_sm = !L.fuse_norm;  // they follow the norm kernel
+  // Factored adaRMSNorm: the residual projections' split-K epilogue writes
+  // the next operand bf16(h (1 + scale)) and per-token sums of squares (one
+  // slot per tile and rank), and QKV / gate-up apply rstd and the projected
+  // shift in their epilogues: no norm kernels.
+  L.factored = use_factored && !L.fuse_norm && L.o.splits >= 2 && L.down.splits >= 2 &&
+               (s.D / 128) * std::max(L.o.splits, L.down.splits) <= kSsSlots;
+  // QKV and gate/up take a whole SM only after a norm kernel, which holds no
+  // shared memory; after a projection they keep the two-CTA footprint so
+  // that they can start beside its last CTAs.
+  const bool whole_sm = !L.fuse_norm && !L.factored;
   L.qkv = plan_gemm(M, s.qkv_rows, s.D, 1, max_splitk, w4, L.fuse_norm, whole_sm);
   L.gu = plan_gemm(M, s.F, s.D, 2, max_splitk, w4, L.fuse_norm, whole_sm);
   L.attn = plan_attn(s, B);
-  // Factored adaRMSNorm: the residual projections' split-K epilogue (one row
-  // per thread, R = 128 / S <= 64 rows per rank) writes the next operand
-  // bf16(h (1 + scale)) and per-token sums of squares (one slot per 32 rows),
-  // and QKV / gate-up apply rstd and the projected shift in their epilogues.
-  const auto nslots = [](const TcPlan& p) { return p.splits * std::max(1, 128 / p.splits / 32); };
-  L.factored = use_factored && !L.fuse_norm && L.o.splits >= 2 && L.down.splits >= 2 &&
-               (s.D / 128) * std::max(nslots(L.o), nslots(L.down)) <= kSsSlots;
   return L;
 }
 
@@ -774,8 +776,7 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
   ctx->ev_next = 0;
   const int slots_o = (s.D / 128) * P.o.splits, slots_down = (s.D / 128) * P.down.splits;
   // factored adaRMSNorm: one slot per (tile, rank, 32 rows)
-  const int fslots_o = P.factored ? slots_o * std::max(1, 128 / P.o.splits / 32) : 0;
-  const int fslots_down = P.factored ? slots_down * std::max(1, 128 / P.down.splits / 32) : 0;
+  const int fslots_o = slots_o, fslots_down = slots_down;  // one slot per (tile, rank)
   for (int k = k_begin; k < k_end; ++k) {
     const float* tk = tab(ctx, k);
     ta.tab_out = (k == k_begin) ? nullptr : tab(ctx, k - 1);
@@ -1697,7 +1698,7 @@ pae_status pae_plan_query(const pae_config* cfg, int what, int batch, long long*
   *value = 0;
   if (cfg->dtype == PAE_FP32) return PAE_OK;  // CUDA-core kernels: no tensor-core launch plan
   const Shape s = shape_from_config(cfg);
-  const LaunchPlans L = plan_launches(s, batch, cfg->dtype == PAE_W4A16, kDefaultMaxSplitK, false);
+  const LaunchPlans L = plan_launches(s, batch, cfg->dtype == PAE_W4A16, kDefaultMaxSplitK, false, false);
   switch (what) {
     case PAE_Q_SPLITS:
       *value = (long long)L.qkv.splits | ((long long)L.o.splits << 8) | ((long long)L.gu.splits << 16) |

@@ -202,14 +202,16 @@ pae_status pae_denoise_steps(pae_ctx* ctx, const float* x_in, float* x_out, int 
  * (statistics from the residual projections' epilogues) instead of separate
  * norm kernels, for batches of at most one 64-token tile.  Both round within
  * the parity tolerance; each is bitwise reproducible.
- * PAE_OPT_FACTORED_NORM (default 1, bf16 / int4 weights; PAE_OPT_FUSED_NORM
- * takes precedence): no separate norm kernels.  The O and down projections'
+ * PAE_OPT_FACTORED_NORM (default 0, bf16 / int4 weights; PAE_OPT_FUSED_NORM
+ * takes precedence): 1 removes the separate norm kernels.  The O and down projections'
  * split-K epilogues write the next norm's operand bf16(h (1 + scale)) and
  * per-token sums of squares of h; QKV and gate/up multiply their accumulators
  * by 1/rms and add the shift projected through their weights (tables built by
  * pae_precompute_tables): the same value as projecting adaRMSNorm(h), rounded
  * differently (within the parity tolerance, bitwise reproducible).  Batches
- * whose O or down plan has no split-K keep the norm kernels.  0: norm kernels.
+ * whose O or down plan has no split-K keep the norm kernels.  Off by default:
+ * at the pi0.5 shape the graph with the (cheap, shared-memory-free) norm
+ * kernels overlaps better under programmatic dependent launch.
  * PAE_OPT_DATAFLOW (default 0, bf16 / int4 weights): batches with batch * chunk <= 64
  * run all K steps as one launch of thread-block clusters whose stages wait on
  * per-tile counters instead of kernel boundaries (no CUDA graph for these

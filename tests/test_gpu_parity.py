@@ -121,9 +121,9 @@ def test_ragged_bf16_bs16_all_rows_then_fresh_prefixes():
 
 
 def _fused_vs_separate(cfg, lengths=None):
-    """The three ways the graph applies adaRMSNorm (factored into the
-    projections' epilogues by default, in-kernel from fp32 h, separate norm
-    kernels) each match the oracle and are bitwise reproducible."""
+    """The three ways the graph applies adaRMSNorm (separate norm kernels by
+    default, factored into the projections' epilogues, in-kernel from fp32 h)
+    each match the oracle and are bitwise reproducible."""
     ex, W = build_expert(cfg)
     try:
         ks, vs = wl.make_prefix(cfg, lengths=lengths)
@@ -132,22 +132,22 @@ def _fused_vs_separate(cfg, lengths=None):
         ex.precompute_tables(grid)
         noise = wl.make_noise(cfg)
         ref = oracle_rows(cfg, W, ks, vs, noise, grid)
-        assert ex.query(fm.PAE_Q_FUSED_NORM, cfg.batch) == 2  # factored by default
+        assert ex.query(fm.PAE_Q_FUSED_NORM, cfg.batch) == 0  # norm kernels by default
+        sep = run_gpu(ex, noise)
+        assert_parity(sep, ref, cfg.dtype, cfg.name + " norm kernels")
+        ex.set_option(fm.PAE_OPT_FACTORED_NORM, 1)
+        assert ex.query(fm.PAE_Q_FUSED_NORM, cfg.batch) == 2
         factored = run_gpu(ex, noise)
         np.testing.assert_array_equal(run_gpu(ex, noise), factored)  # bitwise reproducible
         assert_parity(factored, ref, cfg.dtype, cfg.name + " factored norm")
+        assert max_abs(sep, factored) < 2e-2
+        ex.set_option(fm.PAE_OPT_FACTORED_NORM, 0)
         if cfg.dtype != wl.W4A16:
             ex.set_option(fm.PAE_OPT_FUSED_NORM, 1)
             assert ex.query(fm.PAE_Q_FUSED_NORM, cfg.batch) == 1
             fused = run_gpu(ex, noise)
             np.testing.assert_array_equal(run_gpu(ex, noise), fused)
             assert_parity(fused, ref, cfg.dtype, cfg.name + " in-kernel norm")
-            ex.set_option(fm.PAE_OPT_FUSED_NORM, 0)
-        ex.set_option(fm.PAE_OPT_FACTORED_NORM, 0)
-        assert ex.query(fm.PAE_Q_FUSED_NORM, cfg.batch) == 0
-        sep = run_gpu(ex, noise)
-        assert_parity(sep, ref, cfg.dtype, cfg.name + " norm kernels")
-        assert max_abs(sep, factored) < 2e-2
     finally:
         ex.close()
 

@@ -25,9 +25,9 @@ def test_pi05_plans_match_the_gpu_contexts():
     assert _splits(cfg, 1) == (4, 8, 4, 8)
     assert fm.pae_plan_query(cfg, fm.PAE_Q_TOKEN_TILE, 1) == 64
     assert fm.pae_plan_query(cfg, fm.PAE_Q_ATTN_SPLITS, 1) == 8
-    assert fm.pae_plan_query(cfg, fm.PAE_Q_FUSED_NORM, 1) == 2  # norm factored into the epilogues
+    assert fm.pae_plan_query(cfg, fm.PAE_Q_FUSED_NORM, 1) == 0  # norm kernels by default
     assert _splits(cfg, 32) == (1, 2, 1, 2)
-    assert fm.pae_plan_query(cfg, fm.PAE_Q_FUSED_NORM, 32) == 2
+    assert fm.pae_plan_query(cfg, fm.PAE_Q_FUSED_NORM, 32) == 0
     assert fm.pae_plan_query(cfg, fm.PAE_Q_TOKEN_TILE, 32) == 240
     assert fm.pae_plan_query(cfg, fm.PAE_Q_ATTN_SPLITS, 32) == 1
     w4 = _cfg(wl.PI05_W4A16_BS1)
@@ -44,9 +44,10 @@ def test_fp32_mode_has_no_tensor_core_plan():
 def test_plan_rules_at_every_batch(base):
     """Split-K factors are powers of two that divide the K blocks; a batch of
     one token tile takes the padded token count; larger batches take tiles of
-    128..256 tokens; at <= 64 tokens QKV and gate/up stay within one CTA per SM
-    and O / down within two; split-KV is a power of two <= 8 that only
-    multiplies a launch still under one wave."""
+    128..256 tokens; at <= 64 tokens every projection stays within two CTAs
+    per SM, and QKV / gate-up within one when they follow a norm kernel (norm
+    not factored into the epilogues); split-KV is a power of two <= 8 that
+    only multiplies a launch still under one wave."""
     c = base.replace(batch=min(40, 4096 // base.chunk))
     cfg = _cfg(c)
     D, F, qd = c.width, c.mlp_dim, c.n_q_heads * c.head_dim
@@ -66,7 +67,8 @@ def test_plan_rules_at_every_batch(base):
             assert 128 <= tn <= 256, (B, tn)
         if tn <= 64:
             ntok = -(-M // tn)
-            assert tiles[0] * ntok * sp[0] <= SMS and tiles[2] * ntok * sp[2] <= SMS, (B, sp)
+            per_sm = 2 if fm.pae_plan_query(cfg, fm.PAE_Q_FUSED_NORM, B) == 2 else 1
+            assert tiles[0] * ntok * sp[0] <= per_sm * SMS and tiles[2] * ntok * sp[2] <= per_sm * SMS, (B, sp)
             assert tiles[1] * ntok * sp[1] <= 2 * SMS and tiles[3] * ntok * sp[3] <= 2 * SMS, (B, sp)
         a = fm.pae_plan_query(cfg, fm.PAE_Q_ATTN_SPLITS, B)
         assert a >= 1 and a & (a - 1) == 0 and a <= 8
