@@ -13,11 +13,13 @@
 //   8 warps    online softmax on S_c (two threads per row, log2 domain),
 //              rescale O in TMEM when the row max grows by more than 2^8
 //              (otherwise keep the old reference), write P_c as bf16
-//              pairs back into TMEM over the first 32 columns of S_c
+//              pairs into a TMEM buffer of its own (32 columns)
 //   MMA warp   O += P_c V_c   (M=128, N=head_dim, K=64; A = P_c read from
 //              TMEM, V read MN-major from shared memory)
 // Warps 0-3 and 8-11 run the softmax and the output (two threads per query
-// row: one per 32-key half of the chunk; row = TMEM lane);
+// row: one per 32-key half of the chunk; row = TMEM lane).  Both threads of a
+// row read the whole row of S for its maximum (the same value in both, no
+// exchange), so the softmax threads share no barrier inside the chunk loop;
 // warp 4 streams Q and the K chunks, warp 6 the V chunks (2-slot rings each,
 // a K slot refilled as soon as S of its chunk is done); warp 5 issues the MMAs;
 // all twelve warps take part in the split-KV merge.
@@ -84,9 +86,10 @@ __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+// TMEM columns: S double-buffered (2 x CK), O (d), P double-buffered (2 x CK/2).
 __host__ __device__ inline uint32_t attn_tmem_cols(int d) {
   uint32_t c = 32;
-  while ((int)c < 2 * CK + d) c <<= 1;
+  while ((int)c < 3 * CK + d) c <<= 1;
   return c;
 }
 
@@ -150,6 +153,7 @@ __global__ void __launch_bounds__(384, 1)
   const int n_prefix = a.lens[b];
   const uint32_t t_s[2] = {tmem, tmem + CK};
   const uint32_t t_o = tmem + 2 * CK;
+  const uint32_t t_p[2] = {t_o + (uint32_t)d, t_o + (uint32_t)d + CK / 2};
 
   // ------------------------------------------------------------ producers
   // Warp 4 streams Q once and the K chunks, warp 6 the V chunks: a K slot is
@@ -255,7 +259,7 @@ __global__ void __launch_bounds__(384, 1)
       // A = P in TMEM: 16 keys per MMA = 8 columns of bf16 pairs
 #pragma unroll
       for (int k16 = 0; k16 < CK / 16; ++k16)
-        umma_bf16_tmem_a(t_o, t_s[st] + k16 * 8u, desc_add(v_desc, k16 * 16u * 128u), idesc_o,
+        umma_bf16_tmem_a(t_o, t_p[st] + k16 * 8u, desc_add(v_desc, k16 * 16u * 128u), idesc_o,
                          (c > 0 || k16 > 0) ? 1u : 0u);
       umma_commit(&o_done[st]);
       umma_commit(&v_empty[st]);
@@ -289,15 +293,21 @@ __global__ void __launch_bounds__(384, 1)
   bool ok = true;
   for (int c = 0; c < nch; ++c) {
     const int st = c & 1;
-    const bool w1 = mbar_wait(&s_full[st], (c >> 1) & 1, a.err.wait_ns);
-    if (!named_and(1, 256, w1 && s_flag[0] == 0)) {  // uniform: named barriers follow
+    // warp-uniform: the warp's collectives below need every lane
+    const bool w1 = __all_sync(0xffffffffu, mbar_wait(&s_full[st], (c >> 1) & 1, a.err.wait_ns));
+    if (!w1 || s_flag[0] != 0) {
       ok = false;
+      s_flag[0] = 1;  // every thread stops at its next check
       break;
     }
     tc_fence_after();
-    float sv[CK / 2];
+    // this half's 32 scores, and the other half's for the row maximum (the
+    // maximum is exact in any order, so both threads of the row agree)
+    float sv[CK / 2], so[CK / 2];
     tmem_ld16(t_s[st] + lane_off + h * 32, sv);
     tmem_ld16(t_s[st] + lane_off + h * 32 + 16, sv + 16);
+    tmem_ld16(t_s[st] + lane_off + (1 - h) * 32, so);
+    tmem_ld16(t_s[st] + lane_off + (1 - h) * 32 + 16, so + 16);
     tmem_ld_wait();
     const int vc = min(CK, end - (start + c * CK));
     float cmax = -INFINITY;
@@ -305,11 +315,8 @@ __global__ void __launch_bounds__(384, 1)
     for (int j = 0; j < CK / 2; ++j) {
       sv[j] = j + h * 32 < vc ? sv[j] * scale_log2 : -INFINITY;
       cmax = fmaxf(cmax, sv[j]);
+      cmax = fmaxf(cmax, j + (1 - h) * 32 < vc ? so[j] * scale_log2 : -INFINITY);
     }
-    s_ml[h * QROWS + r] = cmax;
-    named_sync(1, 256);
-    cmax = fmaxf(s_ml[r], s_ml[QROWS + r]);  // same operands, same order, in both halves
-    named_sync(1, 256);                      // both read before the next chunk writes
     // Lazy rescaling: the reference maximum moves only when the row maximum
     // grows by more than 8 (a factor 256), so O is rescaled in TMEM rarely.
     // Probabilities then lie in [0, 256]; the final O / l is the same.
@@ -323,9 +330,9 @@ __global__ void __launch_bounds__(384, 1)
     }
     l_run = l_run * alpha + psum;
     m_run = mx;
-    // P goes into the S columns of this buffer (both halves read them before
-    // the exchange barriers); PV of chunk c - 2, which read the previous P
-    // there, finished before S of chunk c did (commits complete in issue order).
+    // P goes into its own buffer; PV of chunk c - 2, which read the previous
+    // P there, finished before S of chunk c did (commits complete in issue
+    // order).
     bool good = true;
     if (good && c > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
       // O may be rescaled only once PV of the previous chunk has landed in it.
@@ -349,7 +356,7 @@ __global__ void __launch_bounds__(384, 1)
       float pk[16];
 #pragma unroll
       for (int q = 0; q < 16; ++q) pk[q] = __uint_as_float(pack_bf16x2(sv[2 * q], sv[2 * q + 1]));
-      tmem_st16(t_s[st] + lane_off + h * 16, pk);
+      tmem_st16(t_p[st] + lane_off + h * 16, pk);
       tmem_st_wait();
     }
     if (vc < CK) {
