@@ -310,24 +310,36 @@ __global__ void __launch_bounds__(384, 1)
     tmem_ld16(t_s[st] + lane_off + (1 - h) * 32 + 16, so + 16);
     tmem_ld_wait();
     const int vc = min(CK, end - (start + c * CK));
-    float cmax = -INFINITY;
+    // row maximum as a tree (a chain of 64 dependent max operations would be
+    // the longest latency of the chunk at two warps per scheduler)
 #pragma unroll
     for (int j = 0; j < CK / 2; ++j) {
       sv[j] = j + h * 32 < vc ? sv[j] * scale_log2 : -INFINITY;
-      cmax = fmaxf(cmax, sv[j]);
-      cmax = fmaxf(cmax, j + (1 - h) * 32 < vc ? so[j] * scale_log2 : -INFINITY);
+      so[j] = j + (1 - h) * 32 < vc ? so[j] * scale_log2 : -INFINITY;
     }
+    float mt[CK / 2];
+#pragma unroll
+    for (int j = 0; j < CK / 2; ++j) mt[j] = fmaxf(sv[j], so[j]);
+#pragma unroll
+    for (int w = CK / 4; w >= 1; w >>= 1)
+#pragma unroll
+      for (int j = 0; j < w; ++j) mt[j] = fmaxf(mt[j], mt[j + w]);
+    const float cmax = mt[0];
     // Lazy rescaling: the reference maximum moves only when the row maximum
     // grows by more than 8 (a factor 256), so O is rescaled in TMEM rarely.
     // Probabilities then lie in [0, 256]; the final O / l is the same.
     const float mx = cmax > m_run + 8.f ? cmax : m_run;
     const float alpha = exp2f(m_run - mx);  // 1 when unchanged; 0 on the first chunk
-    float psum = 0.f;
 #pragma unroll
-    for (int j = 0; j < CK / 2; ++j) {
-      sv[j] = exp2f(sv[j] - mx);
-      psum += sv[j];
-    }
+    for (int j = 0; j < CK / 2; ++j) sv[j] = exp2f(sv[j] - mx);
+    // row sum as a fixed tree (bitwise reproducible)
+#pragma unroll
+    for (int j = 0; j < CK / 2; ++j) mt[j] = sv[j];
+#pragma unroll
+    for (int w = CK / 4; w >= 1; w >>= 1)
+#pragma unroll
+      for (int j = 0; j < w; ++j) mt[j] += mt[j + w];
+    const float psum = mt[0];
     l_run = l_run * alpha + psum;
     m_run = mx;
     // P goes into its own buffer; PV of chunk c - 2, which read the previous
