@@ -23,7 +23,8 @@
 // warp 4 streams Q and the K chunks, warp 6 the V chunks (2-slot rings each,
 // a K slot refilled as soon as S of its chunk is done); warp 5 issues the MMAs;
 // all twelve warps take part in the split-KV merge.
-// Key splits (split-KV, for small batches) form a thread-block cluster; their
+// Key splits (split-KV, for small batches; up to 16, a non-portable cluster
+// size) form a thread-block cluster; their
 // unnormalised partial O rows, row maxima and sums are merged through
 // distributed shared memory in rank order, so the result is bitwise
 // reproducible and no partial touches global memory.
@@ -499,13 +500,13 @@ __global__ void __launch_bounds__(384, 1)
       const int rq = qt * QROWS + row;
       if (rq >= GH) continue;
       // every rank's loads first (they pipeline), then the merge in rank order
-      uint4 vs[8];
+      uint4 vs[16];
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
+      for (int q = 0; q < 16; ++q)
         if (q < S) vs[q] = ld_cluster_u32x4(map_cluster(red_base + (uint32_t)((row * ldb + c8 * 8) * 2), (uint32_t)q));
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
+      for (int q = 0; q < 16; ++q) {
         if (q >= S) continue;
         const float w = wt[rr * S + q];
         const uint32_t u[4] = {vs[q].x, vs[q].y, vs[q].z, vs[q].w};
@@ -533,7 +534,9 @@ __global__ void __launch_bounds__(384, 1)
 size_t attn_tc_smem_bytes(int d) { return attn_layout(d).total; }
 
 cudaError_t attn_tc_init() {
-  return cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  cudaError_t e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
 }
 
 cudaError_t launch_attn_tc(const Shape& s, const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,

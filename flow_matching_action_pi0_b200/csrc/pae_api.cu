@@ -426,7 +426,7 @@ AttnPlan plan_attn(const Shape& s, int B) {
   const int base = B * s.Hkv * p.qtiles;
   const int max_splits = (s.Ptot + 63) / 64;
   int splits = 1;
-  while (splits < 8 && base * splits * 2 <= 148 && splits * 2 <= max_splits) splits *= 2;
+  while (splits < 16 && base * splits * 2 <= 148 && splits * 2 <= max_splits) splits *= 2;
   p.keys_per_split = ((s.Ptot + splits - 1) / splits + 63) / 64 * 64;
   p.splits = splits;
   return p;

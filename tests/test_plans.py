@@ -24,7 +24,7 @@ def test_pi05_plans_match_the_gpu_contexts():
     cfg = _cfg(wl.PI05_BF16_BS32)
     assert _splits(cfg, 1) == (4, 8, 4, 8)
     assert fm.pae_plan_query(cfg, fm.PAE_Q_TOKEN_TILE, 1) == 64
-    assert fm.pae_plan_query(cfg, fm.PAE_Q_ATTN_SPLITS, 1) == 8
+    assert fm.pae_plan_query(cfg, fm.PAE_Q_ATTN_SPLITS, 1) == 16
     assert fm.pae_plan_query(cfg, fm.PAE_Q_FUSED_NORM, 1) == 0  # norm kernels by default
     assert _splits(cfg, 32) == (1, 2, 1, 2)
     assert fm.pae_plan_query(cfg, fm.PAE_Q_FUSED_NORM, 32) == 0
@@ -46,7 +46,7 @@ def test_plan_rules_at_every_batch(base):
     one token tile takes the padded token count; larger batches take tiles of
     128..256 tokens; at <= 64 tokens every projection stays within two CTAs
     per SM, and QKV / gate-up within one when they follow a norm kernel (norm
-    not factored into the epilogues); split-KV is a power of two <= 8 that
+    not factored into the epilogues); split-KV is a power of two <= 16 that
     only multiplies a launch still under one wave."""
     c = base.replace(batch=min(40, 4096 // base.chunk))
     cfg = _cfg(c)
@@ -71,7 +71,7 @@ def test_plan_rules_at_every_batch(base):
             assert tiles[0] * ntok * sp[0] <= per_sm * SMS and tiles[2] * ntok * sp[2] <= per_sm * SMS, (B, sp)
             assert tiles[1] * ntok * sp[1] <= 2 * SMS and tiles[3] * ntok * sp[3] <= 2 * SMS, (B, sp)
         a = fm.pae_plan_query(cfg, fm.PAE_Q_ATTN_SPLITS, B)
-        assert a >= 1 and a & (a - 1) == 0 and a <= 8
+        assert a >= 1 and a & (a - 1) == 0 and a <= 16
         qtiles = -(-(c.n_q_heads // c.n_kv_heads) * c.chunk // 128)
         if a > 1:
             assert B * c.n_kv_heads * qtiles * a <= SMS
