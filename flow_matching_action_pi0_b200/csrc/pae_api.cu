@@ -426,7 +426,9 @@ AttnPlan plan_attn(const Shape& s, int B) {
   const int base = B * s.Hkv * p.qtiles;
   const int max_splits = (s.Ptot + 63) / 64;
   int splits = 1;
-  while (splits < 16 && base * splits * 2 <= 148 && splits * 2 <= max_splits) splits *= 2;
+  // at most 8: 16 splits (one 64-key chunk per CTA at batch 1) measured
+  // slower, 21.2 against 19.7 us per launch (the merge grows with the ranks)
+  while (splits < 8 && base * splits * 2 <= 148 && splits * 2 <= max_splits) splits *= 2;
   p.keys_per_split = ((s.Ptot + splits - 1) / splits + 63) / 64 * 64;
   p.splits = splits;
   return p;

@@ -215,7 +215,7 @@ def test_launch_plans_pi05_shape():
     """The planner's choices at the pi0.5 expert shape (host logic behind the
     numbers in the benchmark): at batch 1 QKV and gate/up split K four ways with
     one CTA per SM, O-proj and down eight ways, 64-token tiles, attention split
-    over 16 key ranges; at batch 32 token tiles of 240 (QKV), split-K 2 for O-proj
+    over 8 key ranges; at batch 32 token tiles of 240 (QKV), split-K 2 for O-proj
     and down only, and no split-KV."""
     cfg = wl.PI05_BF16_BS32
     ex, _ = build_expert(cfg)
@@ -226,7 +226,7 @@ def test_launch_plans_pi05_shape():
 
         assert splits(1) == (4, 8, 4, 8)
         assert ex.query(fm.PAE_Q_TOKEN_TILE, 1) == 64
-        assert ex.query(fm.PAE_Q_ATTN_SPLITS, 1) == 16
+        assert ex.query(fm.PAE_Q_ATTN_SPLITS, 1) == 8
         assert splits(32) == (1, 2, 1, 2)
         assert ex.query(fm.PAE_Q_TOKEN_TILE, 32) == 240
         assert ex.query(fm.PAE_Q_ATTN_SPLITS, 32) == 1

@@ -24,7 +24,7 @@ def test_pi05_plans_match_the_gpu_contexts():
     cfg = _cfg(wl.PI05_BF16_BS32)
     assert _splits(cfg, 1) == (4, 8, 4, 8)
     assert fm.pae_plan_query(cfg, fm.PAE_Q_TOKEN_TILE, 1) == 64
-    assert fm.pae_plan_query(cfg, fm.PAE_Q_ATTN_SPLITS, 1) == 16
+    assert fm.pae_plan_query(cfg, fm.PAE_Q_ATTN_SPLITS, 1) == 8
     assert fm.pae_plan_query(cfg, fm.PAE_Q_FUSED_NORM, 1) == 0  # norm kernels by default
     assert _splits(cfg, 32) == (1, 2, 1, 2)
     assert fm.pae_plan_query(cfg, fm.PAE_Q_FUSED_NORM, 32) == 0
