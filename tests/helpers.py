@@ -22,15 +22,15 @@ def max_abs(a, b) -> float:
 
 
 def assert_bf16_slot_close(got, ref, what: str) -> None:
-    """K/V slot contents stored in bf16: a value of magnitude m carries up to
-    m * 2^-8 of storage rounding on top of the bf16 operand rounding of the
-    projection, so the bound per element is 5e-3 + m / 128 (the task's own
-    tolerances apply to the final actions, checked separately)."""
+    """K/V slot contents stored in bf16: the bf16-mode absolute bound 2e-2
+    (the task's figure for final actions) plus the storage rounding a value of
+    magnitude m carries, up to m * 2^-8, taken as m / 128 per element (the
+    final actions are checked separately at the task's own tolerances)."""
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     if got.size == 0:
         return
-    excess = np.abs(got - ref) - (5e-3 + np.abs(ref) / 128.0)
+    excess = np.abs(got - ref) - (2e-2 + np.abs(ref) / 128.0)
     assert excess.max() <= 0.0, f"{what}: max excess over the bf16 bound {excess.max():.3e}"
 
 
