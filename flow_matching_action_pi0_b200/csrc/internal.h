@@ -144,10 +144,6 @@ struct TcGemmArgs {
   int N;           // output features (GEGLU: F)
   int K;
   int w_row0;      // first row of this layer's matrix inside the stacked weight map
-  // weights of the next projections in the loop, requested into L2 by the
-  // producer before it waits for the previous kernel (null / 0: none)
-  const void* pf_base[2];
-  size_t pf_bytes[2];
   DevErr err;
 };
 cudaError_t launch_tc_gemm(const Shape& s, const CUtensorMap* tmW, const CUtensorMap* tmX, int na,

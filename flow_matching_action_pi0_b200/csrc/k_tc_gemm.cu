@@ -347,22 +347,6 @@ __global__ void __launch_bounds__(256, 2)
       mbar_arrive_expect_tx(&full[kb], tx);
       tma_load_2d_hint(smem + (size_t)kb * L.stage_bytes + wdst, &tmW, wx + kb * wstep, wrow, &full[kb], pol_w);
     }
-    // The next projections' weights into L2, this CTA's share of each: the
-    // loop's weight stream runs ahead of its dependency chain.
-    {
-      const size_t nct = (size_t)gridDim.x * gridDim.y * gridDim.z;
-      const size_t cid = blockIdx.x + (size_t)gridDim.x * (blockIdx.y + (size_t)gridDim.y * blockIdx.z);
-      for (int m = 0; m < 2; ++m) {
-        if (!a.pf_bytes[m]) continue;
-        const size_t per = ((a.pf_bytes[m] + nct - 1) / nct + 15) & ~size_t(15);
-        const size_t beg = cid * per, end = beg + per < a.pf_bytes[m] ? beg + per : a.pf_bytes[m];
-        const char* base = static_cast<const char*>(a.pf_base[m]);
-        for (size_t off = beg; off < end; off += 65536) {
-          const uint32_t n = (uint32_t)((end - off < 65536 ? end - off : 65536) & ~size_t(15));
-          if (n) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + off), "r"(n) : "memory");
-        }
-      }
-    }
     pdl_wait();
     for (int kb = 0; kb < npre; ++kb)
       tma_load_2d(smem + (size_t)kb * L.stage_bytes + xdst, &tmX, k0 + kb * 64, ttile * p.tn, &full[kb]);

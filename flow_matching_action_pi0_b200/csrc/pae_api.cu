@@ -745,22 +745,6 @@ void run_gemm(pae_ctx* ctx, const Plan& P, int which, int layer, const EpiArgs& 
              a.w_row0 = layer * s.D; a.scales = (const bf16*)ctx->sc_down; break;
   }
   if (!w4) a.scales = nullptr;
-  // L2 prefetch of the next two projections' weights (QKV -> O, gate/up;
-  // O -> gate/up, down; gate/up -> down, next layer's QKV; down -> next
-  // layer's QKV and O; after the last layer, the next Euler step's first)
-  {
-    const size_t eb = w4 ? 1 : 2;  // int4 packed: half a byte per weight (K/2 bytes per row)
-    const size_t kdiv = w4 ? 2 : 1;
-    const void* base[4] = {w4 ? ctx->q_qkv : ctx->w_qkv, w4 ? ctx->q_o : ctx->w_o, w4 ? ctx->q_gu : ctx->w_gu,
-                           w4 ? ctx->q_down : ctx->w_down};
-    const size_t bytes[4] = {(size_t)s.qkv_rows * s.D * eb / kdiv, (size_t)s.D * s.attn_dim * eb / kdiv,
-                             (size_t)2 * s.F * s.D * eb / kdiv, (size_t)s.D * s.F * eb / kdiv};
-    for (int m = 0; m < 2; ++m) {
-      const int nxt = which + 1 + m, w = nxt % 4, l = (layer + nxt / 4) % s.L;  // last layer: the next step's
-      a.pf_base[m] = static_cast<const char*>(base[w]) + (size_t)l * bytes[w];
-      a.pf_bytes[m] = bytes[w];
-    }
-  }
   if (norm.scale) {
     tx = which == 2 ? &P.tmHg : &P.tmH;
     a.ss_in = ctx->ss_buf;
