@@ -252,6 +252,16 @@ __device__ bool fwait(const FC& c, uint64_t* bar, uint32_t parity) {
   }
 }
 
+// One compute thread waits on the mbarrier, the others on the CTA barrier
+// that follows (it orders their later reads after that thread's acquire):
+// 128 threads polling one mbarrier would take shared-memory bandwidth from
+// the copies landing in this CTA.  Returns false once the launch is aborting.
+__device__ bool cwait(const FC& c, uint64_t* bar, uint32_t parity) {
+  bool ok = true;
+  if (c.ct == 0) ok = fwait(c, bar, parity);
+  return cand(ok);
+}
+
 // Bounded wait until a global counter reaches `target` (acquire).
 __device__ bool wait_ctr(const FC& c, const unsigned* p, unsigned target) {
   if (ld_acquire_u32(p) >= target) return true;
@@ -899,7 +909,7 @@ __device__ bool whole_stage(const FC& c, int st, int k, int l, int u, int& sw, i
   FTRACE(c, tr, tb + 2);
 
   // 3. every unit accumulated: the operand area is free from here on
-  if (!cand(fwait(c, c.acc_all, (uint32_t)sw & 1u))) return false;
+  if (!cwait(c, c.acc_all, (uint32_t)sw & 1u)) return false;
   ++sw;
   tc_fence_after();
   FTRACE(c, tr, tb + 3);
@@ -1039,7 +1049,7 @@ __device__ bool split_stage(const FC& c, int st, int k, int l, int u, int& it, i
     xchg_open(c, xbytes);
     xopen = true;
     const int slot = it & 1;
-    if (!cand(fwait(c, &c.acc_full[slot], (uint32_t)(it >> 1) & 1u))) return false;
+    if (!cwait(c, &c.acc_full[slot], (uint32_t)(it >> 1) & 1u)) return false;
     ++it;
     tc_fence_after();
     if (j == 0) FTRACE(c, tr, tb + 2);
@@ -1167,7 +1177,7 @@ __device__ bool att_stage(const FC& c, int l, int u, int& ac, int& xn, bool& xop
   float m_run = -INFINITY, l_run = 0.f;
   for (int ch = 0; ch < au.nch; ++ch) {
     const int acn = ac + ch;
-    if (!cand(fwait(c, c.s_full, acn & 1))) return false;
+    if (!cwait(c, c.s_full, acn & 1)) return false;
     if (ch == 0) FTRACE(c, tr, 42);
     tc_fence_after();
     float sv[CKF];
@@ -1215,7 +1225,7 @@ __device__ bool att_stage(const FC& c, int l, int u, int& ac, int& xn, bool& xop
     }
     if (vc < CKF) {
       // masked keys have P = 0, but 0 * (NaN or Inf) in V would still poison O
-      if (!cand(fwait(c, c.kv_full, acn & 1))) return false;
+      if (!cwait(c, c.kv_full, acn & 1)) return false;
       uint8_t* vbase = c.work + qbytes + kvbytes;
       const int rows = CKF - vc;
       for (int i = c.ct; i < rows * nbox * 8; i += kFCompute) {
@@ -1229,7 +1239,7 @@ __device__ bool att_stage(const FC& c, int l, int u, int& ac, int& xn, bool& xop
     if (c.ct == 0) mbar_arrive(c.p_full);
     if (ch + 1 < au.nch) {
       // the next chunk's K and V overwrite this chunk's: wait for its PV
-      if (!cand(fwait(c, c.o_full, acn & 1))) return false;
+      if (!cwait(c, c.o_full, acn & 1)) return false;
       if (c.ct == 0) {
         mbar_arrive_expect_tx(c.kv_full, 2u * kvbytes);
         const int krow = slot_row0 + au.start + (ch + 1) * CKF;
@@ -1242,7 +1252,7 @@ __device__ bool att_stage(const FC& c, int l, int u, int& ac, int& xn, bool& xop
     }
   }
   ac += au.nch;
-  if (au.nch > 0 && !cand(fwait(c, c.o_full, (ac - 1) & 1))) return false;
+  if (au.nch > 0 && !cwait(c, c.o_full, (ac - 1) & 1)) return false;
   tc_fence_after();
   FTRACE(c, tr, 43);
 
