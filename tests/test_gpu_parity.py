@@ -166,3 +166,29 @@ def test_factored_norm_tiny_w4a16_rope():
 @pytest.mark.slow
 def test_fused_norm_pi05_bs1():
     _fused_vs_separate(wl.PI05_BF16_BS1)
+
+
+@pytest.mark.slow
+def test_factored_norm_pi05_bs32_sampled_rows():
+    """Batch 32 with the adaRMSNorm factored into the projections: O and down
+    run split-K 2, so each rank's residual epilogue sums the squares of 64
+    features per token over 16 lanes (8 at most at batch 1), across several
+    token tiles; rows that straddle tile edges match the oracle, and the run
+    is bitwise reproducible."""
+    cfg = wl.PI05_BF16_BS32
+    rows = [0, 3, 4, 14, 31]
+    ex, W = build_expert(cfg)
+    try:
+        ks, vs = wl.make_prefix(cfg)
+        set_prefixes(ex, cfg, ks, vs)
+        grid = wl.uniform_grid(cfg.steps)
+        ex.precompute_tables(grid)
+        noise = wl.make_noise(cfg)
+        ex.set_option(fm.PAE_OPT_FACTORED_NORM, 1)
+        assert ex.query(fm.PAE_Q_FUSED_NORM, cfg.batch) == 2
+        out = run_gpu(ex, noise)
+        np.testing.assert_array_equal(run_gpu(ex, noise), out)
+        ref = oracle_rows(cfg, W, ks, vs, noise, grid, rows=rows)
+        assert_parity(out[rows], ref, cfg.dtype, cfg.name + " factored norm")
+    finally:
+        ex.close()
