@@ -157,11 +157,17 @@ struct AttnPlan {
   int splits;          // key splits (split-KV)
   int keys_per_split;  // multiple of 64
 };
+// Split-KV scratch: one slot per CTA of a split launch (the planner keeps
+// those launches within one wave of 148 SMs), 128 rows each.
+constexpr int kAttnMaxSplits = 8;
+constexpr int kAttnPartSlots = 148;
 struct AttnArgs {
   const int* lens;
   int layer;
   int keys_per_split;
   void* o;             // [M][Hq d] bf16, token-major
+  __nv_bfloat16* part_o;  // [kAttnPartSlots][128][d] unnormalised partial rows (split-KV)
+  float2* part_ml;        // [kAttnPartSlots][128] (row max, row sum) in the log2 domain
   DevErr err;
 };
 size_t attn_tc_smem_bytes(int d);

@@ -10,24 +10,25 @@
 //
 // One CTA = (b, g, 128-row query tile, key split).  Per 64-key chunk c:
 //   MMA warp   S_c = Q K_c^T  (M=128, N=64, K=head_dim; TMEM, double buffered)
-//   8 warps    online softmax on S_c (two threads per row, log2 domain),
+//   16 warps   online softmax on S_c (four threads per row, log2 domain),
 //              rescale O in TMEM when the row max grows by more than 2^8
 //              (otherwise keep the old reference), write P_c as bf16
 //              pairs into a TMEM buffer of its own (32 columns)
 //   MMA warp   O += P_c V_c   (M=128, N=head_dim, K=64; A = P_c read from
 //              TMEM, V read MN-major from shared memory)
-// Warps 0-3 and 8-11 run the softmax and the output (two threads per query
-// row: one per 32-key half of the chunk; row = TMEM lane).  Both threads of a
-// row read the whole row of S for its maximum (the same value in both, no
-// exchange), so the softmax threads share no barrier inside the chunk loop;
-// warp 4 streams Q and the K chunks, warp 6 the V chunks (2-slot rings each,
-// a K slot refilled as soon as S of its chunk is done); warp 5 issues the MMAs;
-// all twelve warps take part in the split-KV merge.
-// Key splits (split-KV, for small batches; up to 16, a non-portable cluster
-// size) form a thread-block cluster; their
-// unnormalised partial O rows, row maxima and sums are merged through
-// distributed shared memory in rank order, so the result is bitwise
-// reproducible and no partial touches global memory.
+// Warps 0-3 and 8-19 run the softmax and the output (four threads per query
+// row, one per 16-key quarter of the chunk; row = TMEM lane): the softmax is
+// a latency chain per chunk (TMEM load, maximum, exp2, TMEM store), and four
+// warps per scheduler hide more of it than two.  The four parts of a row meet
+// once per chunk at a shared-memory exchange of their maxima.  Warp 4 streams
+// Q and the K chunks, warp 6 the V chunks (2-slot rings each, a K slot
+// refilled as soon as S of its chunk is done); warp 5 issues the MMAs; all
+// twenty warps take part in the split-KV merge.
+// Key splits (split-KV, for small batches; up to 8) form a thread-block
+// cluster: each writes its unnormalised partial O rows, row maxima and sums
+// to a scratch slot in global memory (L2), and after one cluster barrier the
+// ranks merge disjoint row ranges in rank order, so the result is bitwise
+// reproducible.
 #include "internal.h"
 #include "launch.cuh"
 
@@ -38,6 +39,7 @@ namespace {
 constexpr int CK = 64;          // keys per chunk
 constexpr int QROWS = 128;      // query rows per CTA
 constexpr long long kDrainNs = 4000000000LL;
+constexpr int kMaxSplits = kAttnMaxSplits;  // key splits per cluster
 
 struct AttnSmem {
   uint32_t q_off, k0_off, v0_off, slot, bar_off, ml_off, total;
@@ -56,7 +58,7 @@ __host__ __device__ inline AttnSmem attn_layout(int d) {
   L.slot = 2 * kvbytes;                    // [K0 | V0 | K1 | V1]
   L.bar_off = qbytes + 4 * kvbytes;        // (P lives in TMEM, over its S columns)
   L.ml_off = L.bar_off + 256;
-  L.total = L.ml_off + QROWS * 12 + 1024;
+  L.total = L.ml_off + QROWS * 48 + 1024;
   return L;
 }
 
@@ -64,6 +66,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   const uint32_t lo = __bfloat16_as_ushort(f2bf(a));
   const uint32_t hi = __bfloat16_as_ushort(f2bf(b));
   return lo | (hi << 16);
+}
+
+// 2^x by the hardware approximation (relative error about 2^-22; results
+// below 2^-126 flush to zero, far under the bf16 rounding of P).
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 32 lanes x 32 bit, 8 consecutive columns per thread.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
 }
 
 // AND-reduction over the threads of named barrier `id` (`n` of them).  Lanes
@@ -94,9 +111,10 @@ __host__ __device__ inline uint32_t attn_tmem_cols(int d) {
   return c;
 }
 
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(640, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const Shape s, const AttnArgs a) {
+  GTRACE_BEGIN_SHARED();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int d = s.d;
@@ -114,8 +132,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* v_empty = bars + 14;  // [2] V slot free once PV of its chunk is done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);  // [0] abort
-  float* s_ml = reinterpret_cast<float*>(smem + L.ml_off);                // [128][2] row max, row sum
-  int* s_ok = reinterpret_cast<int*>(smem + L.ml_off + QROWS * 8);        // [128]
+  float* s_l = reinterpret_cast<float*>(smem + L.ml_off);   // [4][128] partial row sums
+  float* s_pm = s_l + 4 * QROWS;                            // [2][4][128] partial maxima
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x, split = blockIdx.y, bg = blockIdx.z;
@@ -130,8 +148,9 @@ __global__ void __launch_bounds__(384, 1)
   const float scale_log2 = rsqrtf((float)d) * 1.4426950408889634f;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 16; ++i) mbar_init(&bars[i], (i == 9 || i == 10) ? 256 : 1);
+    for (int i = 0; i < 16; ++i) mbar_init(&bars[i], (i == 9 || i == 10) ? 512 : 1);
     s_flag[0] = 0;
+    s_flag[1] = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
@@ -151,10 +170,11 @@ __global__ void __launch_bounds__(384, 1)
   // written by pae_set_prefix before the loop, so the producers fetch the
   // chunks that lie wholly inside the prefix before waiting (below).
   if (warp != 4 && warp != 6) pdl_wait();
+  GTRACE_WAITED();
   const int n_prefix = a.lens[b];
-  const uint32_t t_s[2] = {tmem, tmem + CK};
+  const uint32_t t_s0 = tmem;                  // S of chunk parity st at t_s0 + st * CK
   const uint32_t t_o = tmem + 2 * CK;
-  const uint32_t t_p[2] = {t_o + (uint32_t)d, t_o + (uint32_t)d + CK / 2};
+  const uint32_t t_p0 = t_o + (uint32_t)d;     // P of chunk parity st at t_p0 + st * CK / 2
 
   // ------------------------------------------------------------ producers
   // Warp 4 streams Q once and the K chunks, warp 6 the V chunks: a K slot is
@@ -239,7 +259,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll 4
       for (int k16 = 0; k16 < d / 16; ++k16) {
         const uint32_t x = (uint32_t)k16 >> 2, w = ((uint32_t)k16 & 3u) * 32u;
-        umma_bf16(t_s[st], desc_add(q_desc, x * QROWS * 128u + w), desc_add(k_desc, x * CK * 128u + w), idesc_s,
+        umma_bf16(t_s0 + (uint32_t)(st * CK), desc_add(q_desc, x * QROWS * 128u + w), desc_add(k_desc, x * CK * 128u + w), idesc_s,
                   k16 > 0 ? 1u : 0u);
       }
       umma_commit(&s_full[st]);
@@ -260,7 +280,7 @@ __global__ void __launch_bounds__(384, 1)
       // A = P in TMEM: 16 keys per MMA = 8 columns of bf16 pairs
 #pragma unroll
       for (int k16 = 0; k16 < CK / 16; ++k16)
-        umma_bf16_tmem_a(t_o, t_p[st] + k16 * 8u, desc_add(v_desc, k16 * 16u * 128u), idesc_o,
+        umma_bf16_tmem_a(t_o, t_p0 + (uint32_t)(st * (CK / 2)) + k16 * 8u, desc_add(v_desc, k16 * 16u * 128u), idesc_o,
                          (c > 0 || k16 > 0) ? 1u : 0u);
       umma_commit(&o_done[st]);
       umma_commit(&v_empty[st]);
@@ -277,99 +297,99 @@ __global__ void __launch_bounds__(384, 1)
   __syncwarp();
 
   // ------------------------------------------------------------ softmax
-  // Warps 0-3 and 8-11: thread = (query row r = TMEM lane, column half h);
-  // half h owns key columns [32h, 32h + 32) of each chunk and output columns
-  // [h d/2, (h+1) d/2).  The two halves of a row agree on the running
-  // reference maximum through shared memory (s_ml as [2][128] exchange
-  // slots, two barriers per chunk); each keeps its own partial row sum, added
-  // in a fixed order at the end.  Decisions that guard a named barrier are
-  // taken CTA-uniformly over the 256 softmax threads (bar.red.and).
+  // Sixteen warps (0-3 and 8-19): thread = (query row r = TMEM lane, part p
+  // of 4); part p owns key columns [16p, 16p + 16) of each chunk, the P
+  // columns [8p, 8p + 8) (its keys as bf16 pairs: the A operand slice of the
+  // chunk's p-th PV MMA) and output columns [p d/4, (p+1) d/4).  The four
+  // parts of a row agree on the chunk maximum through shared memory
+  // (s_pm[chunk parity][part][row]; the maximum is exact in any order), with
+  // one barrier over the 512 softmax threads per chunk that also takes the
+  // CTA-uniform go / stop decision (bar.red.and); each part keeps its own
+  // partial row sum, added in part order at the end.
   const bool smx = warp < 4 || warp >= 8;
   if (smx) {
-  const int h = warp >= 8 ? 1 : 0;
+  const int part = warp < 4 ? 0 : (warp - 4) >> 2;
   const int r = (warp & 3) * 32 + lane;  // query row within the tile (TMEM lane)
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-  const int oc0 = h * (d / 2), oc1 = oc0 + d / 2;  // this half's output columns
+  const int oc0 = part * (d / 4), oc1 = oc0 + d / 4;  // this part's output columns
   float m_run = -INFINITY, l_run = 0.f;
   bool ok = true;
   for (int c = 0; c < nch; ++c) {
     const int st = c & 1;
-    // warp-uniform: the warp's collectives below need every lane
-    const bool w1 = __all_sync(0xffffffffu, mbar_wait(&s_full[st], (c >> 1) & 1, a.err.wait_ns));
-    if (!w1 || s_flag[0] != 0) {
-      ok = false;
-      s_flag[0] = 1;  // every thread stops at its next check
-      break;
-    }
+    const bool got = mbar_wait(&s_full[st], (c >> 1) & 1, a.err.wait_ns);
+    __syncwarp();
     tc_fence_after();
-    // this half's 32 scores, and the other half's for the row maximum (the
-    // maximum is exact in any order, so both threads of the row agree)
-    float sv[CK / 2], so[CK / 2];
-    tmem_ld16(t_s[st] + lane_off + h * 32, sv);
-    tmem_ld16(t_s[st] + lane_off + h * 32 + 16, sv + 16);
-    tmem_ld16(t_s[st] + lane_off + (1 - h) * 32, so);
-    tmem_ld16(t_s[st] + lane_off + (1 - h) * 32 + 16, so + 16);
+    float sv[16];
+    tmem_ld16(t_s0 + (uint32_t)(st * CK) + lane_off + part * 16, sv);
     tmem_ld_wait();
+    reg_fence16(sv);
     const int vc = min(CK, end - (start + c * CK));
-    // row maximum as a tree (a chain of 64 dependent max operations would be
-    // the longest latency of the chunk at two warps per scheduler)
+    // Masking (the last chunk only) and the maximum work on the raw scores:
+    // the scale is positive, so max(scale x) = scale max(x), and the scale
+    // then rides in the FMA that feeds exp2.
+    if (vc < CK) {
 #pragma unroll
-    for (int j = 0; j < CK / 2; ++j) {
-      sv[j] = j + h * 32 < vc ? sv[j] * scale_log2 : -INFINITY;
-      so[j] = j + (1 - h) * 32 < vc ? so[j] * scale_log2 : -INFINITY;
+      for (int j = 0; j < 16; ++j) sv[j] = j + part * 16 < vc ? sv[j] : -INFINITY;
     }
-    float mt[CK / 2];
+    float mt[8];
 #pragma unroll
-    for (int j = 0; j < CK / 2; ++j) mt[j] = fmaxf(sv[j], so[j]);
+    for (int j = 0; j < 8; ++j) mt[j] = fmaxf(sv[j], sv[j + 8]);
 #pragma unroll
-    for (int w = CK / 4; w >= 1; w >>= 1)
+    for (int w = 4; w >= 1; w >>= 1)
 #pragma unroll
       for (int j = 0; j < w; ++j) mt[j] = fmaxf(mt[j], mt[j + w]);
-    const float cmax = mt[0];
+    s_pm[(st * 4 + part) * QROWS + r] = mt[0];
+    // every part's maximum is in place, and all 512 threads go on or all stop
+    if (!named_and(1, 512, got && s_flag[0] == 0)) {
+      ok = false;
+      break;
+    }
+    const float* pm = s_pm + st * 4 * QROWS + r;
+    const float cmax = fmaxf(fmaxf(pm[0], pm[QROWS]), fmaxf(pm[2 * QROWS], pm[3 * QROWS])) * scale_log2;
     // Lazy rescaling: the reference maximum moves only when the row maximum
     // grows by more than 8 (a factor 256), so O is rescaled in TMEM rarely.
     // Probabilities then lie in [0, 256]; the final O / l is the same.
     const float mx = cmax > m_run + 8.f ? cmax : m_run;
-    const float alpha = exp2f(m_run - mx);  // 1 when unchanged; 0 on the first chunk
+    const float alpha = ex2_ftz(m_run - mx);  // 1 when unchanged; 0 on the first chunk
+    const float nmx = -mx;
 #pragma unroll
-    for (int j = 0; j < CK / 2; ++j) sv[j] = exp2f(sv[j] - mx);
+    for (int j = 0; j < 16; ++j) sv[j] = ex2_ftz(fmaf(sv[j], scale_log2, nmx));
     // row sum as a fixed tree (bitwise reproducible)
 #pragma unroll
-    for (int j = 0; j < CK / 2; ++j) mt[j] = sv[j];
+    for (int j = 0; j < 8; ++j) mt[j] = sv[j] + sv[j + 8];
 #pragma unroll
-    for (int w = CK / 4; w >= 1; w >>= 1)
+    for (int w = 4; w >= 1; w >>= 1)
 #pragma unroll
       for (int j = 0; j < w; ++j) mt[j] += mt[j + w];
-    const float psum = mt[0];
-    l_run = l_run * alpha + psum;
+    l_run = l_run * alpha + mt[0];
     m_run = mx;
     // P goes into its own buffer; PV of chunk c - 2, which read the previous
     // P there, finished before S of chunk c did (commits complete in issue
     // order).
-    bool good = true;
-    if (good && c > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
+    if (c > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
       // O may be rescaled only once PV of the previous chunk has landed in it.
-      good = __all_sync(0xffffffffu, mbar_wait(&o_done[st ^ 1], ((c - 1) >> 1) & 1, a.err.wait_ns));
+      const bool good = __all_sync(0xffffffffu, mbar_wait(&o_done[st ^ 1], ((c - 1) >> 1) & 1, a.err.wait_ns));
       if (good) {
         tc_fence_after();
         for (int jj = oc0; jj < oc1; jj += 16) {
           float ov[16];
           tmem_ld16(t_o + lane_off + jj, ov);
           tmem_ld_wait();
+          reg_fence16(ov);
 #pragma unroll
           for (int t = 0; t < 16; ++t) ov[t] *= alpha;
           tmem_st16(t_o + lane_off + jj, ov);
         }
         tmem_st_wait();
+      } else {
+        s_flag[0] = 1;  // every softmax thread stops at the next chunk's barrier
       }
     }
-    if (!good) s_flag[0] = 1;  // every thread stops at the next uniform check
-    // P row in TMEM: keys 32h .. 32h + 31 as bf16 pairs in columns 16h .. 16h + 15
     {
-      float pk[16];
+      uint32_t pk[8];
 #pragma unroll
-      for (int q = 0; q < 16; ++q) pk[q] = __uint_as_float(pack_bf16x2(sv[2 * q], sv[2 * q + 1]));
-      tmem_st16(t_p[st] + lane_off + h * 16, pk);
+      for (int q = 0; q < 8; ++q) pk[q] = pack_bf16x2(sv[2 * q], sv[2 * q + 1]);
+      tmem_st8(t_p0 + (uint32_t)(st * (CK / 2)) + lane_off + part * 8, pk);
       tmem_st_wait();
     }
     if (vc < CK) {
@@ -379,7 +399,7 @@ __global__ void __launch_bounds__(384, 1)
       if (w3) {
         uint8_t* vbase = smem + L.v_off(st);
         const int rows = CK - vc;
-        for (int i = h * QROWS + r; i < rows * nbox * 8; i += 2 * QROWS) {
+        for (int i = part * QROWS + r; i < rows * nbox * 8; i += 4 * QROWS) {
           const int rr = vc + i / (nbox * 8), rem = i % (nbox * 8), x = rem / 8, ch = rem % 8;
           *reinterpret_cast<uint4*>(vbase + x * CK * 128 + rr * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
         }
@@ -391,16 +411,16 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_before();
     mbar_arrive(&p_full[st]);
   }
-  if (!ok || s_flag[0]) set_error(a.err, DEV_TIMEOUT);
+  if (!ok) set_error(a.err, DEV_TIMEOUT);
   // PVs complete in issue order: the last chunk's commit covers them all
   if (nch > 0 && ok) ok = mbar_wait(&o_done[(nch - 1) & 1], ((nch - 1) >> 1) & 1, kDrainNs);
-  ok = named_and(1, 256, ok) && s_flag[0] == 0;  // CTA-uniform among the 256 softmax threads
+  ok = named_and(1, 512, ok && s_flag[0] == 0);  // CTA-uniform among the 512 softmax threads
+  if (threadIdx.x == 0) s_flag[1] = ok ? 1 : 0;  // for the split-KV merge (read after a CTA barrier)
   tc_fence_after();
-  // row sum = half 0 + half 1 (the exchange slots are free: both passed the barrier)
-  s_ml[h * QROWS + r] = l_run;
-  named_sync(1, 256);
-  const float l_tot = s_ml[r] + s_ml[QROWS + r];
-  named_sync(1, 256);
+  // row sum = the four parts' sums in part order
+  s_l[part * QROWS + r] = l_run;
+  named_sync(1, 512);
+  const float l_tot = ((s_l[r] + s_l[QROWS + r]) + s_l[2 * QROWS + r]) + s_l[3 * QROWS + r];
 
   // ------------------------------------------------------------ output (single split)
   const int nsplit = gridDim.y;
@@ -411,49 +431,67 @@ __global__ void __launch_bounds__(384, 1)
     bf16* orow = reinterpret_cast<bf16*>(a.o) + (size_t)(b * s.H + ti) * s.attn_dim + (g * s.G + hl) * d;
     const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
     if (ok) {
-      for (int jj = oc0; jj < oc1; jj += 16) {
-        float ov[16];
+      // 32 columns per TMEM round trip (16 when a part has only 16: d = 64)
+      for (int jj = oc0; jj < oc1; jj += 32) {
+        const bool two = jj + 16 < oc1;  // uniform
+        float ov[32];
         tmem_ld16(t_o + lane_off + jj, ov);
+        if (two) tmem_ld16(t_o + lane_off + jj + 16, ov + 16);
         tmem_ld_wait();
+        reg_fence16(ov);
+        reg_fence16(ov + 16);
         if (row_valid && nch > 0) {
-          uint32_t pk[8];
+          uint32_t pk[16];
 #pragma unroll
-          for (int t = 0; t < 8; ++t) pk[t] = pack_bf16x2(ov[2 * t] * inv, ov[2 * t + 1] * inv);
+          for (int t = 0; t < 16; ++t) pk[t] = pack_bf16x2(ov[2 * t] * inv, ov[2 * t + 1] * inv);
           uint4* dst = reinterpret_cast<uint4*>(orow + jj);
           dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          if (two) {
+            dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+            dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+          }
         }
       }
     }
-  } else if (h == 0) {
-    s_ok[r] = ok ? 1 : 0;
-    s_ml[2 * r] = m_run;
-    s_ml[2 * r + 1] = l_tot;
+  } else {
+    // Split-KV: the row (max, sum) goes to this CTA's scratch slot now; the
+    // unnormalised O rows are parked in shared memory below and written out
+    // row-contiguously.  Rows without keys (or after a stop) have (-inf, 0).
+    const int slot = (blockIdx.z * gridDim.x + qt) * nsplit + split;
+    if (part == 0)
+      a.part_ml[(size_t)slot * QROWS + r] = (ok && nch > 0) ? make_float2(m_run, l_tot) : make_float2(-INFINITY, 0.f);
   }
   }  // softmax warps
 
   if (gridDim.y > 1) {
-    // Split-KV merge inside the cluster of key splits.  Every CTA parks its
-    // unnormalised O rows as bf16 (row stride d + 8, bank-conflict free; the
-    // Q and K/V buffers are idle now) and its row max / sum in shared memory;
-    // CTA rank r then merges rows [r*R, r*R+R) over all ranks in rank order.
-    // Distributed shared memory moves a few tens of GB/s per SM, so the rows
-    // travel in bf16 (the weights and the sum stay fp32) and each (row, rank)
-    // weight exp2(m_q - M) / L is formed once, not per column.
-    __syncthreads();  // all MMAs and TMEM reads of this CTA are done
+    // Split-KV merge inside the cluster of key splits, through L2.  Every CTA
+    // parks its unnormalised O rows as bf16 in shared memory (row stride
+    // d + 8, bank-conflict free; Q and the K/V ring are idle now: every MMA
+    // and every load has completed) and copies them to its scratch slot with
+    // row-contiguous 16-byte stores (coalesced; zeros for a CTA without keys,
+    // so the merge reads only defined values).  After one cluster barrier
+    // (its release / acquire at cluster scope orders these writes before the
+    // peers' reads), CTA rank r merges rows [r*R, r*R+R) over all ranks in
+    // rank order, so the result is bitwise reproducible.  An SM moves about
+    // 60 GB/s into L2 and 90-170 GB/s out of it, against a few tens of GB/s
+    // over distributed shared memory.
+    const int S = gridDim.y;
+    const int slot = (blockIdx.z * gridDim.x + qt) * S + split;
     const int ldb = d + 8;
     bf16* red = reinterpret_cast<bf16*>(smem);
-    float* tbl = reinterpret_cast<float*>(smem + (size_t)QROWS * ldb * 2);  // [R][S] (m, l), then weights
+    __syncthreads();  // every MMA and TMEM read of this CTA is done; s_ok is final
+    const bool has = s_flag[1] != 0 && nch > 0;  // CTA-uniform
     if (smx) {
-      const int h = warp >= 8 ? 1 : 0;
+      const int part = warp < 4 ? 0 : (warp - 4) >> 2;
       const int r = (warp & 3) * 32 + lane;
       const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-      const bool has = s_ok[r] && nch > 0;
-      for (int j = h * (d / 2); j < (h + 1) * (d / 2); j += 16) {
+      for (int j = part * (d / 4); j < (part + 1) * (d / 4); j += 16) {
         float ov[16];
-        if (__all_sync(0xffffffffu, s_ok[(warp & 3) * 32] != 0) && nch > 0) {
+        if (has) {
           tmem_ld16(t_o + lane_off + j, ov);
           tmem_ld_wait();
+          reg_fence16(ov);
         }
         uint32_t pk[8];
 #pragma unroll
@@ -462,53 +500,52 @@ __global__ void __launch_bounds__(384, 1)
         dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       }
-      if (!has && h == 0) {
-        s_ml[2 * r] = -INFINITY;
-        s_ml[2 * r + 1] = 0.f;
+    }
+    __syncthreads();
+    {
+      const int per_row = d / 8;  // 16-byte column groups
+      bf16* prow = a.part_o + (size_t)slot * QROWS * d;
+      for (int el = threadIdx.x; el < QROWS * per_row; el += blockDim.x) {
+        const int row = el / per_row, c8 = el - row * per_row;
+        *reinterpret_cast<uint4*>(prow + (size_t)row * d + c8 * 8) =
+            *reinterpret_cast<const uint4*>(red + row * ldb + c8 * 8);
       }
     }
     cluster_sync();
-    const int S = gridDim.y;
-    const uint32_t rank = cluster_rank();
+    GTRACE_MARK(1);  // every rank's partial is in L2
     const int R = QROWS / S;
-    const uint32_t red_base = smem_u32(red), ml_base = smem_u32(s_ml);
-    // (max, sum) of every (row, rank) once, then the row's weights
-    if ((int)threadIdx.x < R * S) {
-      const int rr = threadIdx.x / S, q = threadIdx.x - rr * S;
-      const uint32_t ra = map_cluster(ml_base + (uint32_t)(((int)rank * R + rr) * 8), (uint32_t)q);
-      tbl[2 * threadIdx.x] = ld_cluster_f32(ra);
-      tbl[2 * threadIdx.x + 1] = ld_cluster_f32(ra + 4);
-    }
-    __syncthreads();
-    float* wt = tbl + 2 * R * S;  // [R][S]
-    if ((int)threadIdx.x < R) {
-      const float* e = tbl + 2 * threadIdx.x * S;
-      float M = -INFINITY;
-      for (int q = 0; q < S; ++q) M = fmaxf(M, e[2 * q]);
-      float wsum = 0.f;
-      for (int q = 0; q < S; ++q)
-        if (e[2 * q + 1] > 0.f) wsum = fmaf(exp2f(e[2 * q] - M), e[2 * q + 1], wsum);
-      const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-      for (int q = 0; q < S; ++q)
-        wt[threadIdx.x * S + q] = e[2 * q + 1] > 0.f ? exp2f(e[2 * q] - M) * inv : 0.f;
-    }
-    __syncthreads();
-    const int per_row = d / 8;  // 16-byte column groups
+    const int row0 = (int)cluster_rank() * R;
+    const int slot0 = slot - split;
+    const int per_row = d / 8;
     for (int el = threadIdx.x; el < R * per_row; el += blockDim.x) {
       const int rr = el / per_row, c8 = el - rr * per_row;
-      const int row = (int)rank * R + rr;
+      const int row = row0 + rr;
       const int rq = qt * QROWS + row;
       if (rq >= GH) continue;
-      // every rank's loads first (they pipeline), then the merge in rank order
-      uint4 vs[16];
+      // every rank's rows and statistics are requested first (one L2 round
+      // trip), then the weights exp2(m_q - M) / L and the merge in rank order
+      uint4 vs[kMaxSplits];
+      float2 ml[kMaxSplits];
 #pragma unroll
-      for (int q = 0; q < 16; ++q)
-        if (q < S) vs[q] = ld_cluster_u32x4(map_cluster(red_base + (uint32_t)((row * ldb + c8 * 8) * 2), (uint32_t)q));
+      for (int q = 0; q < kMaxSplits; ++q)
+        if (q < S) {
+          vs[q] = __ldcg(reinterpret_cast<const uint4*>(a.part_o + ((size_t)(slot0 + q) * QROWS + row) * d + c8 * 8));
+          ml[q] = __ldcg(a.part_ml + (size_t)(slot0 + q) * QROWS + row);
+        }
+      float M = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < kMaxSplits; ++q)
+        if (q < S) M = fmaxf(M, ml[q].x);
+      float wsum = 0.f;
+#pragma unroll
+      for (int q = 0; q < kMaxSplits; ++q)
+        if (q < S && ml[q].y > 0.f) wsum = fmaf(exp2f(ml[q].x - M), ml[q].y, wsum);
+      const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        if (q >= S) continue;
-        const float w = wt[rr * S + q];
+      for (int q = 0; q < kMaxSplits; ++q) {
+        if (q >= S || !(ml[q].y > 0.f)) continue;
+        const float w = exp2f(ml[q].x - M) * inv;
         const uint32_t u[4] = {vs[q].x, vs[q].y, vs[q].z, vs[q].w};
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
@@ -521,12 +558,13 @@ __global__ void __launch_bounds__(384, 1)
       *reinterpret_cast<uint4*>(orow + c8 * 8) = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
                                                             pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
     }
-    cluster_sync();  // peers may still be reading this CTA's partial
+    GTRACE_MARK(2);  // merged rows written
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, ncols);
+  GTRACE_END(4);
 }
 
 }  // namespace
@@ -534,7 +572,8 @@ __global__ void __launch_bounds__(384, 1)
 size_t attn_tc_smem_bytes(int d) { return attn_layout(d).total; }
 
 cudaError_t attn_tc_init() {
-  cudaError_t e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  // 1 KB under the 227 KB limit leaves room for a little static shared memory
+  cudaError_t e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   return e;
 }
@@ -542,8 +581,15 @@ cudaError_t attn_tc_init() {
 cudaError_t launch_attn_tc(const Shape& s, const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                            const AttnPlan& p, const AttnArgs& a, int B, bool pdl, cudaStream_t st) {
   dim3 grid(p.qtiles, p.splits, B * s.Hkv);
-  return launch_ex(k_attn_tc, grid, dim3(384), attn_tc_smem_bytes(s.d), st, p.splits, pdl, *tmQ, *tmK, *tmV, s,
+  return launch_ex(k_attn_tc, grid, dim3(640), attn_tc_smem_bytes(s.d), st, p.splits, pdl, *tmQ, *tmK, *tmV, s,
                    a);
 }
 
 }  // namespace pae
+
+#ifdef PAE_GRAPH_TRACE
+// Trace builds only: hand this file's kernels the launch-trace buffer.
+extern "C" int pae_graph_trace_bind_attn(void* buf, void* ctr, unsigned cap) {
+  return (int)pae::gtrace_bind_tu(buf, ctr, cap);
+}
+#endif

@@ -288,6 +288,7 @@ template <int NA, int EPI, bool SPLIT, bool W4, bool NORM>
 __global__ void __launch_bounds__(256, 2)
     k_tc_gemm(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, const Shape s,
               const TcPlan p, const TcGemmArgs a) {
+  GTRACE_BEGIN();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const TcSmemLayout L = tc_layout(NA, p, W4, NORM);
@@ -348,6 +349,7 @@ __global__ void __launch_bounds__(256, 2)
       tma_load_2d_hint(smem + (size_t)kb * L.stage_bytes + wdst, &tmW, wx + kb * wstep, wrow, &full[kb], pol_w);
     }
     pdl_wait();
+    GTRACE_WAITED();
     for (int kb = 0; kb < npre; ++kb)
       tma_load_2d(smem + (size_t)kb * L.stage_bytes + xdst, &tmX, k0 + kb * 64, ttile * p.tn, &full[kb]);
     int issued = npre;
@@ -367,6 +369,7 @@ __global__ void __launch_bounds__(256, 2)
     // Loads still in flight must land before this CTA may exit.
     for (int kb = issued > p.stages ? issued - p.stages : 0; kb < issued; ++kb)
       if (!mbar_wait(&full[kb % p.stages], (kb / p.stages) & 1, kDrainNs)) set_error(a.err, DEV_DRAIN);
+    GTRACE_MARK(5);  // every load of this CTA has landed
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------------- MMA
     const uint32_t idesc = idesc_bf16(128, p.tn);
@@ -581,6 +584,7 @@ __global__ void __launch_bounds__(256, 2)
   }
   const bool acc_ok = mbar_wait(accf, 0, kDrainNs);
   if (!acc_ok) set_error(a.err, DEV_DRAIN);
+  GTRACE_MARK(1);  // accumulator complete
   tc_fence_after();
   // CTA-uniform decision: the TMEM loads below are warp-collective.
   const bool ok = __syncthreads_and(acc_ok ? 1 : 0) != 0 && s_flag[0] == 0;
@@ -750,8 +754,10 @@ __global__ void __launch_bounds__(256, 2)
         }
       }
     };
+    GTRACE_MARK(2);  // partials pushed
     if (ok && vec) prefetch(col0);
     cluster_sync();
+    GTRACE_MARK(3);  // every rank's partials arrived
     if (ok && vec) {
       const uint32_t rb = smem_u32(recv) + (uint32_t)(16 * g4);
       const uint32_t src_stride = (uint32_t)p.tn * R * 4u;
@@ -820,9 +826,11 @@ __global__ void __launch_bounds__(256, 2)
     }
   }
 
+  GTRACE_MARK(4);  // epilogue written
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, ncols);
+  GTRACE_END(1 + EPI);
 }
 
 size_t smem_bytes_impl(int na, const TcPlan& p, bool w4, bool norm) { return tc_layout(na, p, w4, norm).total; }
@@ -908,3 +916,10 @@ cudaError_t launch_tc_gemm(const Shape& s, const CUtensorMap* tmW, const CUtenso
 }
 
 }  // namespace pae
+
+#ifdef PAE_GRAPH_TRACE
+// Trace builds only: hand this file's kernels the launch-trace buffer.
+extern "C" int pae_graph_trace_bind_gemm(void* buf, void* ctr, unsigned cap) {
+  return (int)pae::gtrace_bind_tu(buf, ctr, cap);
+}
+#endif

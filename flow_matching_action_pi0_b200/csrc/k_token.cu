@@ -58,6 +58,7 @@ __device__ __forceinline__ void store4(float* p, const float* v) {
 // Requires D % 8 == 0 (16-byte weight loads).
 template <typename TW, typename TA>
 __global__ void __launch_bounds__(256) k_transition(const Shape s, const TransitionArgs a) {
+  GTRACE_BEGIN();
   extern __shared__ float sm[];
   float* hs = sm;             // [D]
   float* xs = hs + s.D;       // [A]
@@ -68,6 +69,7 @@ __global__ void __launch_bounds__(256) k_transition(const Shape s, const Transit
   const float* xsrc = a.x_src + (size_t)m * A;
   float* xdst = a.x_dst + (size_t)m * A;
   pdl_wait();
+  GTRACE_WAITED();
   pdl_launch_dependents();
 
   if (a.tab_out) {
@@ -177,6 +179,7 @@ __global__ void __launch_bounds__(256) k_transition(const Shape s, const Transit
       store4(yrow + j, o);
     }
   }
+  GTRACE_END(6);
 }
 
 // One warp per token; the row stays in registers (NV float4 per lane).
@@ -184,6 +187,7 @@ template <typename TA, int NV>
 __global__ void __launch_bounds__(256) k_norm(const Shape s, const float* __restrict__ h, TA* __restrict__ y,
                                               const float* __restrict__ scale, const float* __restrict__ shift,
                                               int M) {
+  GTRACE_BEGIN();
   const int lane = threadIdx.x & 31;
   const int m = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int D = s.D;
@@ -199,6 +203,7 @@ __global__ void __launch_bounds__(256) k_norm(const Shape s, const float* __rest
     }
   }
   pdl_wait();
+  GTRACE_WAITED();
   pdl_launch_dependents();
   if (m >= M) return;
   const float* hr = h + (size_t)m * D;
@@ -225,6 +230,7 @@ __global__ void __launch_bounds__(256) k_norm(const Shape s, const float* __rest
       store4(yr + j, o);
     }
   }
+  GTRACE_END(5);
 }
 
 template <typename TA>
@@ -283,3 +289,10 @@ cudaError_t launch_norm(const Shape& s, int act_bf16, const float* h, void* y, c
 }
 
 }  // namespace pae
+
+#ifdef PAE_GRAPH_TRACE
+// Trace builds only: hand this file's kernels the launch-trace buffer.
+extern "C" int pae_graph_trace_bind_token(void* buf, void* ctr, unsigned cap) {
+  return (int)pae::gtrace_bind_tu(buf, ctr, cap);
+}
+#endif

@@ -166,6 +166,8 @@ struct pae_ctx {
   bool use_factored = false;    // opt-in: measured slower than the norm kernels under PDL
   float* ss_buf = nullptr;
   int ss_ld = 0;
+  // split-KV merge scratch: partial rows [kAttnPartSlots][128][d] bf16, then (max, sum) [kAttnPartSlots][128]
+  void* attn_part = nullptr;
   // int4 weights (W4A16): packed codes [L*rows][K/2] and group scales [L*rows][K/128]
   int w4 = 0;
   void *q_qkv = nullptr, *q_o = nullptr, *q_gu = nullptr, *q_down = nullptr;
@@ -639,6 +641,9 @@ pae_status build_plan(pae_ctx* ctx, int B, Plan* P) {
   P->gu = LP.gu;
   P->down = LP.down;
   P->attn = LP.attn;
+  if (P->attn.splits > 1 &&
+      (P->attn.splits > kAttnMaxSplits || B * s.Hkv * P->attn.qtiles * P->attn.splits > kAttnPartSlots))
+    return fail(ctx, PAE_ERR_UNSUPPORTED, "split-KV plan exceeds the merge scratch (%d splits)", P->attn.splits);
   P->fuse_norm = LP.fuse_norm;
   P->factored = LP.factored;
   const uint64_t Mmax = (uint64_t)s.Bmax * s.H;
@@ -818,6 +823,9 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
           aa.layer = l;
           aa.keys_per_split = P.attn.keys_per_split;
           aa.o = ctx->o;
+          aa.part_o = static_cast<bf16*>(ctx->attn_part);
+          aa.part_ml = reinterpret_cast<float2*>(static_cast<char*>(ctx->attn_part) +
+                                                 (size_t)kAttnPartSlots * 128 * s.d * 2);
           aa.err = DevErr{ctx->err_dev, ctx->wait_ns};
           launch_attn_tc(s, &ctx->tmQ, &ctx->tmK, &ctx->tmV, P.attn, aa, P.B, pdl_on(ctx), st);
         } else {
@@ -1354,6 +1362,11 @@ pae_status pae_create(const pae_config* cfg, const pae_weights* w, pae_ctx** out
   ctx->ss_ld = (int)Mpad;
   ALLOC(ctx->ss_buf, sizeof(float) * kSsSlots * Mpad);
   CKC(cudaMemsetAsync(ctx->ss_buf, 0, sizeof(float) * kSsSlots * Mpad, cs));
+  if (ctx->act_bf16) {
+    const size_t part_bytes = (size_t)kAttnPartSlots * 128 * (s.d * 2 + 8);
+    ALLOC(ctx->attn_part, part_bytes);
+    CKC(cudaMemsetAsync(ctx->attn_part, 0, part_bytes, cs));
+  }
   if (ctx->act_bf16 && !ctx->w4) {
     if ((st = make_map(ctx, &ctx->tmWqkv, ctx->w_qkv, D, (uint64_t)L * s.qkv_rows, 64, 128)) != PAE_OK) return bail(st);
     if ((st = make_map(ctx, &ctx->tmWo, ctx->w_o, s.attn_dim, (uint64_t)L * D, 64, 128)) != PAE_OK) return bail(st);
