@@ -68,9 +68,11 @@ __global__ void __launch_bounds__(256) k_transition(const Shape s, const Transit
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
   const float* xsrc = a.x_src + (size_t)m * A;
   float* xdst = a.x_dst + (size_t)m * A;
+  // This kernel holds no TMEM, so its successor (a projection, which only
+  // streams weights before its own wait) may be scheduled at once.
+  pdl_launch_dependents();
   pdl_wait();
   GTRACE_WAITED();
-  pdl_launch_dependents();
 
   if (a.tab_out) {
     const float* hrow = a.h + (size_t)m * D;
@@ -202,9 +204,12 @@ __global__ void __launch_bounds__(256) k_norm(const Shape s, const float* __rest
       ds[i] = __ldg(reinterpret_cast<const float4*>(shift + j));
     }
   }
+  // No TMEM or other resource is taken after this point, so the successor (a
+  // projection) is let in before the wait: its CTAs become resident while the
+  // projection before this kernel still runs and stream their weights early.
+  pdl_launch_dependents();
   pdl_wait();
   GTRACE_WAITED();
-  pdl_launch_dependents();
   if (m >= M) return;
   const float* hr = h + (size_t)m * D;
   float4 v[NV];
