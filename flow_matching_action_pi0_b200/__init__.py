@@ -31,6 +31,7 @@ PAE_OPT_FACTORED_NORM = 10
 KERNEL_CLASSES = ("transition", "qkv", "attention", "o_proj", "norm", "gate_up", "down", "persistent", "dataflow")
 PAE_Q_GRAPH_KERNELS, PAE_Q_SPLITS, PAE_Q_TOKEN_TILE, PAE_Q_ATTN_SPLITS, PAE_Q_PERSISTENT, PAE_Q_FUSED_NORM = 1, 2, 3, 4, 5, 6
 PAE_Q_DATAFLOW = 7
+PAE_Q_ATTN_CHUNK = 8
 STATUS_NAMES = {0: "PAE_OK", 1: "PAE_ERR_ARG", 2: "PAE_ERR_STATE", 3: "PAE_ERR_CUDA", 4: "PAE_ERR_OOM",
                 5: "PAE_ERR_TIMEOUT", 6: "PAE_ERR_UNSUPPORTED"}
 

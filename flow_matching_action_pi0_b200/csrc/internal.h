@@ -155,7 +155,8 @@ cudaError_t tc_gemm_init();  // once per process: opt in to large dynamic shared
 struct AttnPlan {
   int qtiles;          // ceil(G*H / 128) query tiles per (request, KV head)
   int splits;          // key splits (split-KV)
-  int keys_per_split;  // multiple of 64
+  int keys_per_split;  // multiple of 64 (and of chunk)
+  int chunk;           // keys per attention chunk: 64 or 128
 };
 // Split-KV scratch: one slot per CTA of a split launch (the planner keeps
 // those launches within one wave of 148 SMs), 128 rows each.

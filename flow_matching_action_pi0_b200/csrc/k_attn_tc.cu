@@ -8,22 +8,28 @@
 // reading: every action token sees all valid prefix keys and all H action
 // keys; keys past lens[b] + H are masked.
 //
-// One CTA = (b, g, 128-row query tile, key split).  Per 64-key chunk c:
-//   MMA warp   S_c = Q K_c^T  (M=128, N=64, K=head_dim; TMEM, double buffered)
+// One CTA = (b, g, 128-row query tile, key split).  Per chunk c of CK keys
+// (CK = 64 or 128, a template parameter):
+//   MMA warp   S_c = Q K_c^T  (M=128, N=CK, K=head_dim; TMEM, double
+//              buffered: chunk c in S buffer c % 2)
 //   16 warps   online softmax on S_c (four threads per row, log2 domain),
 //              rescale O in TMEM when the row max grows by more than 2^8
-//              (otherwise keep the old reference), write P_c as bf16
-//              pairs into a TMEM buffer of its own (32 columns)
-//   MMA warp   O += P_c V_c   (M=128, N=head_dim, K=64; A = P_c read from
+//              (otherwise keep the old reference), write P_c as bf16 pairs
+//              over the first CK/2 columns of S_c's own buffer
+//   MMA warp   O += P_c V_c   (M=128, N=head_dim, K=CK; A = P_c read from
 //              TMEM, V read MN-major from shared memory)
 // Warps 0-3 and 8-19 run the softmax and the output (four threads per query
-// row, one per 16-key quarter of the chunk; row = TMEM lane): the softmax is
-// a latency chain per chunk (TMEM load, maximum, exp2, TMEM store), and four
-// warps per scheduler hide more of it than two.  The four parts of a row meet
-// once per chunk at a shared-memory exchange of their maxima.  Warp 4 streams
-// Q and the K chunks, warp 6 the V chunks (2-slot rings each, a K slot
-// refilled as soon as S of its chunk is done); warp 5 issues the MMAs; all
-// twenty warps take part in the split-KV merge.
+// row, one per CK/4-key quarter of the chunk; row = TMEM lane); four warps
+// per scheduler hide more of the softmax's latency chain (TMEM load, maximum
+// exchange, exp2, TMEM store) than two.  The four parts of a row meet once
+// per chunk at a shared-memory exchange of their maxima.  Warp 4 streams Q
+// and the K chunks, warp 6 the V chunks, through rings of 128/CK slots of CK
+// keys (the same shared memory either way): K of chunk c is loaded once S of
+// the chunk that last used its slot is done, V once that chunk's PV is done.
+// Long key ranges take CK = 128 (half the chunks, each S with N = 128);
+// a split of only 128 keys takes two 64-key chunks, whose softmax and PV
+// overlap.  Warp 5 issues the MMAs; all twenty warps take part in the
+// split-KV merge.
 // Key splits (split-KV, for small batches; up to 8) form a thread-block
 // cluster: each writes its unnormalised partial O rows, row maxima and sums
 // to a scratch slot in global memory (L2), and after one cluster barrier the
@@ -36,27 +42,25 @@ namespace pae {
 
 namespace {
 
-constexpr int CK = 64;          // keys per chunk
 constexpr int QROWS = 128;      // query rows per CTA
+constexpr int RING_KEYS = 128;  // keys of K (and of V) held in shared memory
 constexpr long long kDrainNs = 4000000000LL;
 constexpr int kMaxSplits = kAttnMaxSplits;  // key splits per cluster
 
 struct AttnSmem {
-  uint32_t q_off, k0_off, v0_off, slot, bar_off, ml_off, total;
-  // ring slot st of K / V (arithmetic, so no local-memory array is indexed)
-  __host__ __device__ uint32_t k_off(int st) const { return k0_off + (uint32_t)st * slot; }
-  __host__ __device__ uint32_t v_off(int st) const { return v0_off + (uint32_t)st * slot; }
+  uint32_t q_off, k_off, v_off, bar_off, ml_off, total;
 };
 
+// K ring, V ring: RING_KEYS keys each, as 128/CK slots of d/64 boxes [CK][64]
+// (slot j at j * CK * d * 2 bytes from the ring's start).
 __host__ __device__ inline AttnSmem attn_layout(int d) {
   AttnSmem L;
-  const uint32_t qbytes = QROWS * d * 2;   // d/64 boxes of [128][64]
-  const uint32_t kvbytes = CK * d * 2;     // d/64 boxes of [64][64]
+  const uint32_t qbytes = QROWS * d * 2;       // d/64 boxes of [128][64]
+  const uint32_t ringbytes = RING_KEYS * d * 2;
   L.q_off = 0;
-  L.k0_off = qbytes;
-  L.v0_off = qbytes + kvbytes;
-  L.slot = 2 * kvbytes;                    // [K0 | V0 | K1 | V1]
-  L.bar_off = qbytes + 4 * kvbytes;        // (P lives in TMEM, over its S columns)
+  L.k_off = qbytes;
+  L.v_off = qbytes + ringbytes;
+  L.bar_off = qbytes + 2 * ringbytes;          // (P lives in TMEM, over its S columns)
   L.ml_off = L.bar_off + 256;
   L.total = L.ml_off + QROWS * 48 + 1024;
   return L;
@@ -74,13 +78,6 @@ __device__ __forceinline__ float ex2_ftz(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 32 lanes x 32 bit, 8 consecutive columns per thread.
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* v) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
-               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-               : "memory");
 }
 
 // AND-reduction over the threads of named barrier `id` (`n` of them).  Lanes
@@ -104,32 +101,57 @@ __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-// TMEM columns: S double-buffered (2 x CK), O (d), P double-buffered (2 x CK/2).
+// TMEM columns: S double-buffered (2 x CK, P written over the first half of
+// its chunk's buffer), O (d).
+template <int CK>
 __host__ __device__ inline uint32_t attn_tmem_cols(int d) {
   uint32_t c = 32;
-  while ((int)c < 3 * CK + d) c <<= 1;
+  while ((int)c < 2 * CK + d) c <<= 1;
   return c;
 }
 
+// 32 lanes x 32 bit, 8 / 16 consecutive columns per thread.
+__device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t* v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+template <int CK>
 __global__ void __launch_bounds__(640, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const Shape s, const AttnArgs a) {
+  constexpr int NSLOT = RING_KEYS / CK;  // ring slots: chunk c in slot c % NSLOT
+  constexpr int HALVES = CK / 64;        // 64-key boxes per chunk
+  constexpr int KP = CK / 4;             // keys per softmax part
   GTRACE_BEGIN_SHARED();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int d = s.d;
   const int nbox = d / 64;
   const AttnSmem L = attn_layout(d);
+  // Barrier phases count uses: the K / V slot barriers complete once per use
+  // of their slot (chunk c: slot c % NSLOT, parity (c / NSLOT) & 1), the
+  // per-buffer ones (S, P, PV) once per use of their buffer (chunk c: buffer
+  // c & 1, parity (c >> 1) & 1).
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;   // [2]
-  uint64_t* v_full = bars + 3;   // [2]
-  uint64_t* k_empty = bars + 5;  // [2] K slot free once S of its chunk is done
-  uint64_t* s_full = bars + 7;   // [2]
-  uint64_t* p_full = bars + 9;    // [2] P buffer j written (chunks j, j + 2, ...)
-  uint64_t* o_done = bars + 11;   // [2] PV of the chunks in P buffer j done
+  uint64_t* k_full = bars + 1;    // [NSLOT] K chunk landed
+  uint64_t* v_full = bars + 3;    // [NSLOT] V chunk landed
+  uint64_t* k_empty = bars + 5;   // [NSLOT] K slot free once S of its chunk is done
+  uint64_t* s_full = bars + 7;    // [2] S buffer j computed
+  uint64_t* p_full = bars + 9;    // [2] P written over S buffer j (chunks j, j + 2, ...)
+  uint64_t* o_done = bars + 11;   // [2] PV of the chunk in buffer j done
   uint64_t* drain = bars + 13;
-  uint64_t* v_empty = bars + 14;  // [2] V slot free once PV of its chunk is done
+  uint64_t* v_empty = bars + 14;  // [NSLOT] V slot free once PV of its chunk is done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);  // [0] abort
   float* s_l = reinterpret_cast<float*>(smem + L.ml_off);   // [4][128] partial row sums
@@ -156,7 +178,7 @@ __global__ void __launch_bounds__(640, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
-  const uint32_t ncols = attn_tmem_cols(d);
+  const uint32_t ncols = attn_tmem_cols<CK>(d);
   if (warp == 0) {
     tmem_alloc(tmem_slot, ncols);
     tmem_relinquish();
@@ -172,75 +194,68 @@ __global__ void __launch_bounds__(640, 1)
   if (warp != 4 && warp != 6) pdl_wait();
   GTRACE_WAITED();
   const int n_prefix = a.lens[b];
-  const uint32_t t_s0 = tmem;                  // S of chunk parity st at t_s0 + st * CK
+  const uint32_t t_s0 = tmem;                  // S (then P) of chunk parity st at t_s0 + st * CK
   const uint32_t t_o = tmem + 2 * CK;
-  const uint32_t t_p0 = t_o + (uint32_t)d;     // P of chunk parity st at t_p0 + st * CK / 2
 
   // ------------------------------------------------------------ producers
-  // Warp 4 streams Q once and the K chunks, warp 6 the V chunks: a K slot is
-  // refilled as soon as S of its chunk is done, ahead of the PV that frees V.
-  // chunks 0 and 1 (the two ring slots) if they end inside the prefix
-  const int npre = nch < 2 ? (start + CK <= n_prefix ? nch : 0)
-                            : (start + 2 * CK <= n_prefix ? 2 : (start + CK <= n_prefix ? 1 : 0));
-  if (warp == 4) {
-    if (lane == 0)
-      for (int c = 0; c < npre; ++c) {
-        mbar_arrive_expect_tx(&k_full[c], CK * d * 2);
-        for (int x = 0; x < nbox; ++x)
-          tma_load_2d(smem + L.k_off(c) + x * CK * 128, &tmK, x * 64, slot_row0 + start + c * CK, &k_full[c]);
+  // Warp 4 streams Q once and the K chunks, warp 6 the V chunks.  A chunk
+  // arrives as CK/64 boxes of 64 keys (64-row boxes; a second one lands 8 KB
+  // into each 16 KB box region, a whole number of 1024-byte swizzle atoms).
+  // The first RING_KEYS keys' boxes that lie wholly inside the prefix (written
+  // before the loop) are fetched before waiting for the previous kernel, the
+  // rest after it; a chunk's barrier expects all of its bytes once.
+  const uint32_t kvbytes = CK * d * 2;  // one chunk of K (or V)
+  auto load_piece = [&](uint32_t ring, const CUtensorMap* tm, uint64_t* bar, int c, int h) {
+    const uint32_t off = ring + (uint32_t)(c % NSLOT) * kvbytes + (uint32_t)h * 64u * 128u;
+    for (int x = 0; x < nbox; ++x)
+      tma_load_2d(smem + off + x * CK * 128, tm, x * 64, slot_row0 + start + c * CK + h * 64, bar + (c % NSLOT));
+  };
+  // 64-key pieces fetched early (pieces 0, 1 = keys [start, start + 128)),
+  // only those of chunks that exist
+  const int npre_p = min(min(nch * HALVES, 2), start + 128 <= n_prefix ? 2 : start + 64 <= n_prefix ? 1 : 0);
+  if (warp == 4 || warp == 6) {
+    if (lane == 0) {
+      const bool is_k = warp == 4;
+      for (int i = 0; i < npre_p; ++i) {
+        const int c = i / HALVES, h = i % HALVES;
+        if (h == 0) mbar_arrive_expect_tx((is_k ? k_full : v_full) + c, kvbytes);
+        load_piece(is_k ? L.k_off : L.v_off, is_k ? &tmK : &tmV, is_k ? k_full : v_full, c, h);
       }
+    }
     __syncwarp();
     pdl_wait();
   }
-  if (warp == 6) {
-    if (lane == 0)
-      for (int c = 0; c < npre; ++c) {
-        mbar_arrive_expect_tx(&v_full[c], CK * d * 2);
-        for (int x = 0; x < nbox; ++x)
-          tma_load_2d(smem + L.v_off(c) + x * CK * 128, &tmV, x * 64, slot_row0 + start + c * CK, &v_full[c]);
-      }
-    __syncwarp();
-    pdl_wait();
-  }
-  if (warp == 4 && lane == 0 && nch > 0) {
-    const uint32_t kvbytes = CK * d * 2;
-    mbar_arrive_expect_tx(q_full, QROWS * d * 2);
-    const int qrow0 = bg * GH + qt * QROWS;
-    for (int x = 0; x < nbox; ++x) tma_load_2d(smem + L.q_off + x * QROWS * 128, &tmQ, x * 64, qrow0, q_full);
-    int issued = npre;
-    for (int c = npre; c < nch; ++c) {
-      const int st = c & 1;
-      if (c >= 2 && !mbar_wait(&k_empty[st], ((c >> 1) & 1) ^ 1, a.err.wait_ns)) {
+  if ((warp == 4 || warp == 6) && lane == 0 && nch > 0) {
+    const bool is_k = warp == 4;
+    uint64_t* full = is_k ? k_full : v_full;
+    uint64_t* empty = is_k ? k_empty : v_empty;  // S (K) or PV (V) of the slot's previous chunk done
+    const CUtensorMap* tm = is_k ? &tmK : &tmV;
+    const uint32_t ring = is_k ? L.k_off : L.v_off;
+    if (is_k) {
+      mbar_arrive_expect_tx(q_full, QROWS * d * 2);
+      const int qrow0 = bg * GH + qt * QROWS;
+      for (int x = 0; x < nbox; ++x) tma_load_2d(smem + L.q_off + x * QROWS * 128, &tmQ, x * 64, qrow0, q_full);
+    }
+    int issued = 0;
+    for (int c = 0; c < nch; ++c) {
+      const int slot = c % NSLOT, use = c / NSLOT;
+      if (use > 0 && !mbar_wait(empty + slot, (use & 1) ^ 1, a.err.wait_ns)) {
         s_flag[0] = 1;
         set_error(a.err, DEV_TIMEOUT);
         break;
       }
-      const int krow = slot_row0 + start + c * CK;
-      mbar_arrive_expect_tx(&k_full[st], kvbytes);
-      for (int x = 0; x < nbox; ++x) tma_load_2d(smem + L.k_off(st) + x * CK * 128, &tmK, x * 64, krow, &k_full[st]);
+      const int p0 = c * HALVES;  // this chunk's first piece
+      if (p0 >= npre_p) mbar_arrive_expect_tx(full + slot, kvbytes);
+      for (int h = 0; h < HALVES; ++h)
+        if (p0 + h >= npre_p) load_piece(ring, tm, full, c, h);
       issued = c + 1;
     }
-    if (!mbar_wait(q_full, 0, kDrainNs)) set_error(a.err, DEV_DRAIN);
-    for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c)
-      if (!mbar_wait(&k_full[c & 1], (c >> 1) & 1, kDrainNs)) set_error(a.err, DEV_DRAIN);
-  }
-  if (warp == 6 && lane == 0 && nch > 0) {
-    const uint32_t kvbytes = CK * d * 2;
-    int issued = npre;
-    for (int c = npre; c < nch; ++c) {
-      const int st = c & 1;
-      if (c >= 2 && !mbar_wait(&v_empty[st], ((c >> 1) & 1) ^ 1, a.err.wait_ns)) {
-        s_flag[0] = 1;
-        set_error(a.err, DEV_TIMEOUT);
-        break;
-      }
-      const int krow = slot_row0 + start + c * CK;
-      mbar_arrive_expect_tx(&v_full[st], kvbytes);
-      for (int x = 0; x < nbox; ++x) tma_load_2d(smem + L.v_off(st) + x * CK * 128, &tmV, x * 64, krow, &v_full[st]);
-      issued = c + 1;
-    }
-    for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c)
-      if (!mbar_wait(&v_full[c & 1], (c >> 1) & 1, kDrainNs)) set_error(a.err, DEV_DRAIN);
+    // Loads still in flight must land before this CTA may exit: only the last
+    // NSLOT chunks' can be (every earlier one was consumed by an MMA that
+    // completed).
+    if (is_k && !mbar_wait(q_full, 0, kDrainNs)) set_error(a.err, DEV_DRAIN);
+    for (int c = issued > NSLOT ? issued - NSLOT : 0; c < issued; ++c)
+      if (!mbar_wait(full + c % NSLOT, (c / NSLOT) & 1, kDrainNs)) set_error(a.err, DEV_DRAIN);
   }
 
   // ------------------------------------------------------------ MMA (warp 5)
@@ -251,40 +266,46 @@ __global__ void __launch_bounds__(640, 1)
     bool good = mbar_wait(q_full, 0, a.err.wait_ns);
     // descriptors are built once per operand and stepped in 16-byte units
     const uint64_t q_desc = sw128_desc(q_base, 16, 1024);
+    const uint64_t k_desc = sw128_desc(smem_u32(smem + L.k_off), 16, 1024);
+    const uint64_t v_desc = sw128_desc(smem_u32(smem + L.v_off), CK * 128, 1024);
+    const uint32_t slot_bytes = (uint32_t)CK * (uint32_t)d * 2u;
+    // S of chunk c into buffer c & 1.  That buffer last held P of chunk c - 2:
+    // its PV must be complete first (waited on explicitly, not left to the
+    // issue order).
     auto issue_s = [&](int c) -> bool {
-      const int st = c & 1;
-      if (!mbar_wait(&k_full[st], (c >> 1) & 1, a.err.wait_ns)) return false;
+      const int st = c & 1, slot = c % NSLOT;
+      if (!mbar_wait(k_full + slot, (c / NSLOT) & 1, a.err.wait_ns)) return false;
+      if (c >= 2 && !mbar_wait(&o_done[st], ((c >> 1) & 1) ^ 1, a.err.wait_ns)) return false;
       tc_fence_after();
-      const uint64_t k_desc = sw128_desc(smem_u32(smem + L.k_off(st)), 16, 1024);
 #pragma unroll 4
       for (int k16 = 0; k16 < d / 16; ++k16) {
         const uint32_t x = (uint32_t)k16 >> 2, w = ((uint32_t)k16 & 3u) * 32u;
-        umma_bf16(t_s0 + (uint32_t)(st * CK), desc_add(q_desc, x * QROWS * 128u + w), desc_add(k_desc, x * CK * 128u + w), idesc_s,
-                  k16 > 0 ? 1u : 0u);
+        umma_bf16(t_s0 + (uint32_t)(st * CK), desc_add(q_desc, x * QROWS * 128u + w),
+                  desc_add(k_desc, slot * slot_bytes + x * CK * 128u + w), idesc_s, k16 > 0 ? 1u : 0u);
       }
       umma_commit(&s_full[st]);
-      umma_commit(&k_empty[st]);
+      umma_commit(k_empty + slot);
       return true;
     };
+    // Order: S of the next chunk first (the softmax needs it as soon as the
+    // current chunk's is done), then PV of the current chunk once its P is in.
     if (good) good = issue_s(0);
-    if (good && nch > 1) good = issue_s(1);
     for (int c = 0; good && c < nch; ++c) {
-      const int st = c & 1;
+      const int st = c & 1, slot = c % NSLOT;
+      if (c + 1 < nch && !(good = issue_s(c + 1))) break;
       if (!mbar_wait(&p_full[st], (c >> 1) & 1, a.err.wait_ns) ||
-          !mbar_wait(&v_full[st], (c >> 1) & 1, a.err.wait_ns)) {
+          !mbar_wait(v_full + slot, (c / NSLOT) & 1, a.err.wait_ns)) {
         good = false;
         break;
       }
       tc_fence_after();
-      const uint64_t v_desc = sw128_desc(smem_u32(smem + L.v_off(st)), CK * 128, 1024);
-      // A = P in TMEM: 16 keys per MMA = 8 columns of bf16 pairs
+      // A = P in TMEM (over S buffer st): 16 keys per MMA = 8 columns of bf16 pairs
 #pragma unroll
       for (int k16 = 0; k16 < CK / 16; ++k16)
-        umma_bf16_tmem_a(t_o, t_p0 + (uint32_t)(st * (CK / 2)) + k16 * 8u, desc_add(v_desc, k16 * 16u * 128u), idesc_o,
-                         (c > 0 || k16 > 0) ? 1u : 0u);
+        umma_bf16_tmem_a(t_o, t_s0 + (uint32_t)(st * CK) + k16 * 8u,
+                         desc_add(v_desc, slot * slot_bytes + k16 * 16u * 128u), idesc_o, (c > 0 || k16 > 0) ? 1u : 0u);
       umma_commit(&o_done[st]);
-      umma_commit(&v_empty[st]);
-      if (c + 2 < nch) good = issue_s(c + 2);
+      umma_commit(v_empty + slot);
     }
     if (!good) {
       s_flag[0] = 1;
@@ -298,10 +319,13 @@ __global__ void __launch_bounds__(640, 1)
 
   // ------------------------------------------------------------ softmax
   // Sixteen warps (0-3 and 8-19): thread = (query row r = TMEM lane, part p
-  // of 4); part p owns key columns [16p, 16p + 16) of each chunk, the P
-  // columns [8p, 8p + 8) (its keys as bf16 pairs: the A operand slice of the
-  // chunk's p-th PV MMA) and output columns [p d/4, (p+1) d/4).  The four
-  // parts of a row agree on the chunk maximum through shared memory
+  // of 4); part p owns key columns [KP p, KP p + KP) of each chunk, the P
+  // columns [KP p / 2, KP (p + 1) / 2) (its keys as bf16 pairs: the A operand
+  // of the chunk's PV MMAs for those keys) and output columns
+  // [p d/4, (p+1) d/4).  P
+  // overwrites S columns that other parts of the row read: every part has its
+  // S in registers before the barrier below, and P is written after it.  The
+  // four parts of a row agree on the chunk maximum through shared memory
   // (s_pm[chunk parity][part][row]; the maximum is exact in any order), with
   // one barrier over the 512 softmax threads per chunk that also takes the
   // CTA-uniform go / stop decision (bar.red.and); each part keeps its own
@@ -319,23 +343,25 @@ __global__ void __launch_bounds__(640, 1)
     const bool got = mbar_wait(&s_full[st], (c >> 1) & 1, a.err.wait_ns);
     __syncwarp();
     tc_fence_after();
-    float sv[16];
-    tmem_ld16(t_s0 + (uint32_t)(st * CK) + lane_off + part * 16, sv);
+    float sv[KP];
+#pragma unroll
+    for (int j = 0; j < KP; j += 16) tmem_ld16(t_s0 + (uint32_t)(st * CK) + lane_off + part * KP + j, sv + j);
     tmem_ld_wait();
-    reg_fence16(sv);
+#pragma unroll
+    for (int j = 0; j < KP; j += 16) reg_fence16(sv + j);
     const int vc = min(CK, end - (start + c * CK));
     // Masking (the last chunk only) and the maximum work on the raw scores:
     // the scale is positive, so max(scale x) = scale max(x), and the scale
     // then rides in the FMA that feeds exp2.
     if (vc < CK) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) sv[j] = j + part * 16 < vc ? sv[j] : -INFINITY;
+      for (int j = 0; j < KP; ++j) sv[j] = j + part * KP < vc ? sv[j] : -INFINITY;
     }
-    float mt[8];
+    float mt[KP / 2];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) mt[j] = fmaxf(sv[j], sv[j + 8]);
+    for (int j = 0; j < KP / 2; ++j) mt[j] = fmaxf(sv[j], sv[j + KP / 2]);
 #pragma unroll
-    for (int w = 4; w >= 1; w >>= 1)
+    for (int w = KP / 4; w >= 1; w >>= 1)
 #pragma unroll
       for (int j = 0; j < w; ++j) mt[j] = fmaxf(mt[j], mt[j + w]);
     s_pm[(st * 4 + part) * QROWS + r] = mt[0];
@@ -353,19 +379,18 @@ __global__ void __launch_bounds__(640, 1)
     const float alpha = ex2_ftz(m_run - mx);  // 1 when unchanged; 0 on the first chunk
     const float nmx = -mx;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) sv[j] = ex2_ftz(fmaf(sv[j], scale_log2, nmx));
+    for (int j = 0; j < KP; ++j) sv[j] = ex2_ftz(fmaf(sv[j], scale_log2, nmx));
     // row sum as a fixed tree (bitwise reproducible)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) mt[j] = sv[j] + sv[j + 8];
+    for (int j = 0; j < KP / 2; ++j) mt[j] = sv[j] + sv[j + KP / 2];
 #pragma unroll
-    for (int w = 4; w >= 1; w >>= 1)
+    for (int w = KP / 4; w >= 1; w >>= 1)
 #pragma unroll
       for (int j = 0; j < w; ++j) mt[j] += mt[j + w];
     l_run = l_run * alpha + mt[0];
     m_run = mx;
-    // P goes into its own buffer; PV of chunk c - 2, which read the previous
-    // P there, finished before S of chunk c did (commits complete in issue
-    // order).
+    // P goes over S of this chunk; PV of chunk c - 2, which read the previous
+    // P there, completed before S of chunk c was issued.
     if (c > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
       // O may be rescaled only once PV of the previous chunk has landed in it.
       const bool good = __all_sync(0xffffffffu, mbar_wait(&o_done[st ^ 1], ((c - 1) >> 1) & 1, a.err.wait_ns));
@@ -386,18 +411,21 @@ __global__ void __launch_bounds__(640, 1)
       }
     }
     {
-      uint32_t pk[8];
+      uint32_t pk[KP / 2];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) pk[q] = pack_bf16x2(sv[2 * q], sv[2 * q + 1]);
-      tmem_st8(t_p0 + (uint32_t)(st * (CK / 2)) + lane_off + part * 8, pk);
+      for (int q = 0; q < KP / 2; ++q) pk[q] = pack_bf16x2(sv[2 * q], sv[2 * q + 1]);
+      if constexpr (KP == 32)
+        tmem_st16u(t_s0 + (uint32_t)(st * CK) + lane_off + part * 16, pk);
+      else
+        tmem_st8u(t_s0 + (uint32_t)(st * CK) + lane_off + part * 8, pk);
       tmem_st_wait();
     }
     if (vc < CK) {
       // Masked keys have P = 0, but 0 * (NaN or Inf) in V would still poison O:
       // zero the V rows past the valid keys once their load has landed.
-      const bool w3 = mbar_wait(&v_full[st], (c >> 1) & 1, kDrainNs);
+      const bool w3 = mbar_wait(v_full + c % NSLOT, (c / NSLOT) & 1, kDrainNs);
       if (w3) {
-        uint8_t* vbase = smem + L.v_off(st);
+        uint8_t* vbase = smem + L.v_off + (c % NSLOT) * kvbytes;
         const int rows = CK - vc;
         for (int i = part * QROWS + r; i < rows * nbox * 8; i += 4 * QROWS) {
           const int rr = vc + i / (nbox * 8), rem = i % (nbox * 8), x = rem / 8, ch = rem % 8;
@@ -571,17 +599,29 @@ __global__ void __launch_bounds__(640, 1)
 
 size_t attn_tc_smem_bytes(int d) { return attn_layout(d).total; }
 
-cudaError_t attn_tc_init() {
+template <int CK>
+cudaError_t attn_init_one() {
   // 1 KB under the 227 KB limit leaves room for a little static shared memory
-  cudaError_t e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaError_t e = cudaFuncSetAttribute(k_attn_tc<CK>, cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_attn_tc<CK>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
+}
+
+cudaError_t attn_tc_init() {
+  cudaError_t e = attn_init_one<64>();
+  if (e == cudaSuccess) e = attn_init_one<128>();
   return e;
 }
 
 cudaError_t launch_attn_tc(const Shape& s, const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                            const AttnPlan& p, const AttnArgs& a, int B, bool pdl, cudaStream_t st) {
   dim3 grid(p.qtiles, p.splits, B * s.Hkv);
-  return launch_ex(k_attn_tc, grid, dim3(640), attn_tc_smem_bytes(s.d), st, p.splits, pdl, *tmQ, *tmK, *tmV, s,
+  if (p.chunk != 64 && p.chunk != 128) return cudaErrorInvalidValue;
+  if (a.keys_per_split % p.chunk != 0) return cudaErrorInvalidValue;
+  if (p.chunk == 128)
+    return launch_ex(k_attn_tc<128>, grid, dim3(640), attn_tc_smem_bytes(s.d), st, p.splits, pdl, *tmQ, *tmK, *tmV,
+                     s, a);
+  return launch_ex(k_attn_tc<64>, grid, dim3(640), attn_tc_smem_bytes(s.d), st, p.splits, pdl, *tmQ, *tmK, *tmV, s,
                    a);
 }
 

@@ -266,7 +266,8 @@ pae_status pae_profile_read(pae_ctx* ctx, int kernel_class, double* total_ms, in
  * norm kernels, 1 inside the projections from fp32 h (PAE_OPT_FUSED_NORM), 2
  * factored into the projections' epilogues (PAE_OPT_FACTORED_NORM).  PAE_Q_DATAFLOW: the
  * cluster size of the dataflow loop pae_denoise runs for `batch` (0: it runs
- * the graph or the persistent kernel). */
+ * the graph or the persistent kernel).  PAE_Q_ATTN_CHUNK: keys per chunk of
+ * the graph's attention kernel for `batch` (64 or 128). */
 enum {
   PAE_Q_GRAPH_KERNELS = 1,
   PAE_Q_SPLITS = 2,
@@ -274,14 +275,16 @@ enum {
   PAE_Q_ATTN_SPLITS = 4,
   PAE_Q_PERSISTENT = 5,
   PAE_Q_FUSED_NORM = 6,
-  PAE_Q_DATAFLOW = 7
+  PAE_Q_DATAFLOW = 7,
+  PAE_Q_ATTN_CHUNK = 8
 };
 pae_status pae_query(pae_ctx* ctx, int what, int batch, long long* value);
 
 /* The same launch-plan queries without a context or a device: what a context
  * created from `cfg`, with its options at their defaults, would use for
- * `batch` (PAE_Q_SPLITS, PAE_Q_TOKEN_TILE, PAE_Q_ATTN_SPLITS or
- * PAE_Q_FUSED_NORM; 0 in PAE_FP32 mode, which has no tensor-core plan).
+ * `batch` (PAE_Q_SPLITS, PAE_Q_TOKEN_TILE, PAE_Q_ATTN_SPLITS,
+ * PAE_Q_ATTN_CHUNK or PAE_Q_FUSED_NORM; 0 in PAE_FP32 mode, which has no
+ * tensor-core plan).
  * Host arithmetic only.  Errors: PAE_ERR_ARG for a NULL argument, a batch
  * outside [1, max_batch] or another query; the config is checked as by
  * pae_create (PAE_ERR_ARG / PAE_ERR_UNSUPPORTED). */

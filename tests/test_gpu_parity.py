@@ -1,15 +1,15 @@
 """GPU-vs-oracle parity on the same seeded inputs, through the C ABI.
 
-Small configs are compared element by element on every output; the full-size
-pi0.5-shaped configs on every output (batch 1) or on sampled rows that the
-oracle computes one by one (batch 32, ragged batch 16), in the same launch
-configuration the benchmark times (captured graph, same batch size).
+Small configs and the full-size pi0.5-shaped configs (batch 1, batch 32,
+ragged batch 16) are compared element by element on every output, in the same
+launch configuration the benchmark times (captured graph, same batch size).
 """
 import numpy as np
 import pytest
 
 import flow_matching_action_pi0_b200 as fm
 import workloads as wl
+from workloads.device import abi_config
 from tests.helpers import assert_parity, build_expert, max_abs, oracle_rows, run_gpu, set_prefixes
 
 pytestmark = pytest.mark.gpu
@@ -54,6 +54,20 @@ def test_tiny_bf16_gqa2_many_tokens():
     # Hkv = 2, 300 tokens (two token tiles with a ragged tail)
     cfg = wl.TINY_FP32.replace(name="tiny_bf16_gqa2", dtype=wl.BF16, n_kv_heads=2, batch=20, chunk=15)
     _run_case(cfg, lengths=[(7 * b) % 65 for b in range(20)])
+
+
+def test_tiny_bf16_long_prefixes_128key_chunks():
+    # Splits of >= 256 keys run in 128-key chunks through a one-slot K / V ring:
+    # ragged prefixes of 0..600 keys at batch 40 give two key splits of 384 keys
+    # (three chunks each, the slot reloaded twice, a masked last chunk, empty
+    # splits for short rows) merged through the split-KV scratch.
+    cfg = wl.TINY_FP32.replace(name="tiny_bf16_long", dtype=wl.BF16, batch=40, prefix=600)
+    lens = [(37 * b + 5) % 601 for b in range(40)]
+    lens[:4] = [0, 1, 600, 64]
+    c = fm.make_config(**abi_config(cfg))
+    assert fm.pae_plan_query(c, fm.PAE_Q_ATTN_CHUNK, 40) == 128
+    assert fm.pae_plan_query(c, fm.PAE_Q_ATTN_SPLITS, 40) == 2
+    _run_case(cfg, lengths=lens)
 
 
 def test_tiny_w4a16():

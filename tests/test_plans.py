@@ -30,13 +30,18 @@ def test_pi05_plans_match_the_gpu_contexts():
     assert fm.pae_plan_query(cfg, fm.PAE_Q_FUSED_NORM, 32) == 0
     assert fm.pae_plan_query(cfg, fm.PAE_Q_TOKEN_TILE, 32) == 240
     assert fm.pae_plan_query(cfg, fm.PAE_Q_ATTN_SPLITS, 32) == 1
+    # 128 keys per split at batch 1 run as two 64-key chunks, the whole slot
+    # at batch 32 as 128-key chunks
+    assert fm.pae_plan_query(cfg, fm.PAE_Q_ATTN_CHUNK, 1) == 64
+    assert fm.pae_plan_query(cfg, fm.PAE_Q_ATTN_CHUNK, 32) == 128
+    assert fm.pae_plan_query(_cfg(wl.RAGGED_BF16_BS16), fm.PAE_Q_ATTN_CHUNK, 16) == 128
     w4 = _cfg(wl.PI05_W4A16_BS1)
     assert _splits(w4, 1) == (4, 8, 4, 8)
 
 
 def test_fp32_mode_has_no_tensor_core_plan():
     cfg = _cfg(wl.TINY_FP32)
-    for q in (fm.PAE_Q_SPLITS, fm.PAE_Q_TOKEN_TILE, fm.PAE_Q_ATTN_SPLITS, fm.PAE_Q_FUSED_NORM):
+    for q in (fm.PAE_Q_SPLITS, fm.PAE_Q_TOKEN_TILE, fm.PAE_Q_ATTN_SPLITS, fm.PAE_Q_ATTN_CHUNK, fm.PAE_Q_FUSED_NORM):
         assert fm.pae_plan_query(cfg, q, 1) == 0
 
 
@@ -72,6 +77,7 @@ def test_plan_rules_at_every_batch(base):
             assert tiles[1] * ntok * sp[1] <= 2 * SMS and tiles[3] * ntok * sp[3] <= 2 * SMS, (B, sp)
         a = fm.pae_plan_query(cfg, fm.PAE_Q_ATTN_SPLITS, B)
         assert a >= 1 and a & (a - 1) == 0 and a <= 16
+        assert fm.pae_plan_query(cfg, fm.PAE_Q_ATTN_CHUNK, B) in (64, 128)
         qtiles = -(-(c.n_q_heads // c.n_kv_heads) * c.chunk // 128)
         if a > 1:
             assert B * c.n_kv_heads * qtiles * a <= SMS
