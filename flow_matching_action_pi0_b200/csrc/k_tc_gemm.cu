@@ -72,7 +72,7 @@ __host__ __device__ inline TcSmemLayout tc_layout(int na, const TcPlan& p, bool 
   L.recv_off = p.recv_alias ? 0u : ring;
   const uint32_t used = p.recv_alias ? (ring > L.recv_bytes ? ring : L.recv_bytes) : ring + L.recv_bytes;
   L.bar_off = (used + 15u) & ~15u;
-  L.norm_off = L.bar_off + 256;  // rstd [64] + partial sums [2][64]
+  L.norm_off = L.bar_off + 512;  // (barriers) then rstd [64] + partial sums [2][64]
   L.rs_off = L.norm_off + (norm ? 768u : 0u);  // factored adaRMSNorm: rstd of the tile's tokens [256]
   L.total = L.rs_off + 1024u + 1024u;  // + slack for 1024-byte alignment
   return L;
@@ -296,7 +296,8 @@ __global__ void __launch_bounds__(256, 2)
   uint64_t* empty = full + p.stages;
   uint64_t* a_ready = empty + p.stages;  // int4 weights: A tile dequantised / norm: B tile built
   uint64_t* accf = a_ready + p.stages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  uint64_t* wfull = accf + 1;  // int4 weights: the packed tile landed (the token tile completes on full)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wfull + p.stages);
   volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);  // [0] abort
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -311,6 +312,7 @@ __global__ void __launch_bounds__(256, 2)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
       mbar_init(&a_ready[i], 128);
+      mbar_init(&wfull[i], 1);
     }
     mbar_init(accf, 1);
     s_flag[0] = 0;
@@ -342,11 +344,16 @@ __global__ void __launch_bounds__(256, 2)
     const uint32_t wdst = W4 ? L.a_bytes + L.b_bytes : 0u;         // raw tile or A tile
     const int wx = W4 ? (k0 + 0) / 2 : k0;                            // packed: two codes per byte
     const int wstep = W4 ? 32 : 64;
-    const uint32_t tx = W4 ? L.raw_bytes + L.b_bytes : NORM ? L.a_bytes + L.b_bytes + L.h_bytes : L.a_bytes + L.b_bytes;
+    // int4 weights: the packed tile completes on its own barrier (wfull), so
+    // the dequantising warps turn the first ring into bf16 before the wait;
+    // full then counts only the token tile.
+    const uint32_t tx = W4 ? L.b_bytes : NORM ? L.a_bytes + L.b_bytes + L.h_bytes : L.a_bytes + L.b_bytes;
     const uint32_t xdst = L.a_bytes;  // the B tile, or (norm) the fp32 staging that the B tile overlays
     for (int kb = 0; kb < npre; ++kb) {
+      uint64_t* wbar = W4 ? &wfull[kb] : &full[kb];
+      if (W4) mbar_arrive_expect_tx(wbar, L.raw_bytes);
       mbar_arrive_expect_tx(&full[kb], tx);
-      tma_load_2d_hint(smem + (size_t)kb * L.stage_bytes + wdst, &tmW, wx + kb * wstep, wrow, &full[kb], pol_w);
+      tma_load_2d_hint(smem + (size_t)kb * L.stage_bytes + wdst, &tmW, wx + kb * wstep, wrow, wbar, pol_w);
     }
     pdl_wait();
     GTRACE_WAITED();
@@ -361,14 +368,18 @@ __global__ void __launch_bounds__(256, 2)
         break;
       }
       uint8_t* sa = smem + (size_t)st * L.stage_bytes;
+      uint64_t* wbar = W4 ? &wfull[st] : &full[st];
+      if (W4) mbar_arrive_expect_tx(wbar, L.raw_bytes);
       mbar_arrive_expect_tx(&full[st], tx);
-      tma_load_2d_hint(sa + wdst, &tmW, wx + kb * wstep, wrow, &full[st], pol_w);
+      tma_load_2d_hint(sa + wdst, &tmW, wx + kb * wstep, wrow, wbar, pol_w);
       tma_load_2d(sa + xdst, &tmX, k0 + kb * 64, ttile * p.tn, &full[st]);
       issued = kb + 1;
     }
     // Loads still in flight must land before this CTA may exit.
-    for (int kb = issued > p.stages ? issued - p.stages : 0; kb < issued; ++kb)
+    for (int kb = issued > p.stages ? issued - p.stages : 0; kb < issued; ++kb) {
       if (!mbar_wait(&full[kb % p.stages], (kb / p.stages) & 1, kDrainNs)) set_error(a.err, DEV_DRAIN);
+      if (W4 && !mbar_wait(&wfull[kb % p.stages], (kb / p.stages) & 1, kDrainNs)) set_error(a.err, DEV_DRAIN);
+    }
     GTRACE_MARK(5);  // every load of this CTA has landed
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------------- MMA
@@ -516,7 +527,7 @@ __global__ void __launch_bounds__(256, 2)
     const bf16* srow0 = a.scales + (size_t)(a.w_row0 + ntile * 128 * NA + dr) * gpr;
     for (int kb = 0; kb < nkb; ++kb) {
       const int st = kb % p.stages;
-      if (!mbar_wait(&full[st], (kb / p.stages) & 1, a.err.wait_ns)) {
+      if (!mbar_wait(&wfull[st], (kb / p.stages) & 1, a.err.wait_ns)) {
         s_flag[0] = 1;
         set_error(a.err, DEV_TIMEOUT);
         break;
