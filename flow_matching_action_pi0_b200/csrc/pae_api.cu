@@ -206,6 +206,10 @@ struct pae_ctx {
   std::vector<cudaEvent_t> ev_pool;
   int ev_next = 0;
   std::vector<ProfRec>* rec_sink = nullptr;
+  // First error a launch helper returned while enqueue_steps ran: one that
+  // rejects its arguments returns before launching, so the runtime's last
+  // error would not show it.
+  cudaError_t enq_err = cudaSuccess;
   cudaStream_t cap_stream = nullptr;
   EncodeTiledFn encode = nullptr;
   std::string last_error;
@@ -725,6 +729,18 @@ struct NormIn {
   int nslots = 0;
 };
 
+// Keep the first launch-helper error of the current enqueue_steps call.
+void note_launch(pae_ctx* ctx, cudaError_t e) {
+  if (e != cudaSuccess && ctx->enq_err == cudaSuccess) ctx->enq_err = e;
+}
+
+// The launch errors of the last enqueue_steps call: a helper's own refusal
+// first, else the runtime's last error.
+cudaError_t enqueue_error(pae_ctx* ctx) {
+  const cudaError_t e = cudaGetLastError();
+  return ctx->enq_err != cudaSuccess ? ctx->enq_err : e;
+}
+
 void run_gemm(pae_ctx* ctx, const Plan& P, int which, int layer, const EpiArgs& e, cudaStream_t st,
               const NormIn& norm = NormIn{}) {
   const Shape& s = ctx->s;
@@ -768,7 +784,7 @@ void run_gemm(pae_ctx* ctx, const Plan& P, int which, int layer, const EpiArgs& 
     a.nscale = norm.scale;
     a.nshift = norm.shift;
   }
-  launch_tc_gemm(s, tw, tx, na, *p, a, pdl_on(ctx), st);
+  note_launch(ctx, launch_tc_gemm(s, tw, tx, na, *p, a, pdl_on(ctx), st));
 }
 
 // Enqueue Euler steps k_begin..k_end-1 for the plan's batch on `st`, with the
@@ -776,6 +792,7 @@ void run_gemm(pae_ctx* ctx, const Plan& P, int which, int layer, const EpiArgs& 
 void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStream_t st) {
   const Shape& s = ctx->s;
   const int M = P.M;
+  ctx->enq_err = cudaSuccess;
   TransitionArgs ta{};
   ta.x = ctx->x;
   ta.x_src = ctx->x;
@@ -801,7 +818,7 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
     ta.tab_in = tk;
     {
       ProfScope ps(ctx, PAE_K_TRANSITION, st);
-      launch_transition(s, ctx->act_bf16, ta, pdl_on(ctx), st);
+      note_launch(ctx, launch_transition(s, ctx->act_bf16, ta, pdl_on(ctx), st));
     }
     for (int l = 0; l < s.L; ++l) {
       EpiArgs e{};
@@ -837,7 +854,7 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
           aa.part_ml = reinterpret_cast<float2*>(static_cast<char*>(ctx->attn_part) +
                                                  (size_t)kAttnPartSlots * 128 * s.d * 2);
           aa.err = DevErr{ctx->err_dev, ctx->wait_ns};
-          launch_attn_tc(s, &ctx->tmQ, &ctx->tmK, &ctx->tmV, P.attn, aa, P.B, pdl_on(ctx), st);
+          note_launch(ctx, launch_attn_tc(s, &ctx->tmQ, &ctx->tmK, &ctx->tmV, P.attn, aa, P.B, pdl_on(ctx), st));
         } else {
           launch_attention_simple(s, ctx->act_bf16, ctx->q, ctx->kc, ctx->vc, ctx->lens_dev, l, ctx->o, P.B, st);
         }
@@ -861,8 +878,8 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
       }
       if (!P.fuse_norm && !P.factored) {
         ProfScope ps(ctx, PAE_K_NORM, st);
-        launch_norm(s, ctx->act_bf16, ctx->h, ctx->y, tk + mod_offset(s, l, 1, 0), tk + mod_offset(s, l, 1, 1), M,
-                    pdl_on(ctx), st);
+        note_launch(ctx, launch_norm(s, ctx->act_bf16, ctx->h, ctx->y, tk + mod_offset(s, l, 1, 0),
+                                     tk + mod_offset(s, l, 1, 1), M, pdl_on(ctx), st));
       }
       e = EpiArgs{};
       e.M = M;
@@ -899,8 +916,8 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
       }
       if (l + 1 < s.L && !P.fuse_norm && !P.factored) {
         ProfScope ps(ctx, PAE_K_NORM, st);
-        launch_norm(s, ctx->act_bf16, ctx->h, ctx->y, tk + mod_offset(s, l + 1, 0, 0), tk + mod_offset(s, l + 1, 0, 1),
-                    M, pdl_on(ctx), st);
+        note_launch(ctx, launch_norm(s, ctx->act_bf16, ctx->h, ctx->y, tk + mod_offset(s, l + 1, 0, 0),
+                                     tk + mod_offset(s, l + 1, 0, 1), M, pdl_on(ctx), st));
       }
     }
   }
@@ -909,7 +926,7 @@ void enqueue_steps(pae_ctx* ctx, const Plan& P, int k_begin, int k_end, cudaStre
   ta.tab_in = nullptr;
   {
     ProfScope ps(ctx, PAE_K_TRANSITION, st);
-    launch_transition(s, ctx->act_bf16, ta, pdl_on(ctx), st);
+    note_launch(ctx, launch_transition(s, ctx->act_bf16, ta, pdl_on(ctx), st));
   }
 }
 
@@ -998,7 +1015,7 @@ pae_status run_loop(pae_ctx* ctx, Plan* P, cudaStream_t stream) {
     ctx->rec_sink = &P->recs;
     enqueue_steps(ctx, *P, 0, ctx->K, stream);
     ctx->rec_sink = nullptr;
-    CK(cudaGetLastError());
+    CK(enqueue_error(ctx));
     return PAE_OK;
   }
   if (!P->graph || P->graph_K != ctx->K) {
@@ -1010,7 +1027,7 @@ pae_status run_loop(pae_ctx* ctx, Plan* P, cudaStream_t stream) {
     CK(cudaStreamBeginCapture(ctx->cap_stream, cudaStreamCaptureModeThreadLocal));
     enqueue_steps(ctx, *P, 0, ctx->K, ctx->cap_stream);
     ctx->rec_sink = nullptr;
-    cudaError_t e1 = cudaGetLastError();
+    cudaError_t e1 = enqueue_error(ctx);
     cudaError_t e2 = cudaStreamEndCapture(ctx->cap_stream, &g);
     if (e1 != cudaSuccess || e2 != cudaSuccess) {
       if (g) cudaGraphDestroy(g);
@@ -1611,6 +1628,7 @@ pae_status pae_denoise_steps(pae_ctx* ctx, const float* x_in, float* x_out, int 
     ctx->rec_sink = &P->recs;
     enqueue_steps(ctx, *P, k_begin, k_end, stm);
     ctx->rec_sink = nullptr;
+    CK(enqueue_error(ctx));
   }
   CK(cudaGetLastError());
   CK(cudaMemcpyAsync(x_out, ctx->x, bytes, cudaMemcpyDeviceToDevice, stm));
